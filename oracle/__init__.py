@@ -1,0 +1,181 @@
+"""CPU oracle of the reduced cross-entropy (RECE / SCE) loss -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this package.  It shares no code with the CUDA library and never calls it.
+
+Every function takes fp32 numpy arrays (bf16 inputs are passed as their exact fp32
+upcast) and follows the definitions cited in ``rece_oracle.c``:
+
+* ``bucketize``     -- RECE paper, section 3, Algorithm 1 (argmax over random vectors)
+* ``stable_argsort``-- Algorithm 1's argsort, read as a stable sort
+* ``chunk_start``   -- Algorithm 1's chunk sets, start of chunk c = ceil(c*M/n_c)
+* ``select``        -- candidates of the chunk windows over all rounds, positive removed,
+                       de-duplicated, the k best by (score desc, item asc) (SCE abstract)
+* ``rece_loss`` / ``rece_grad``       -- Algorithm 1's loss, equation (4) on the subset
+* ``full_ce_loss`` / ``full_ce_grad`` -- equations (3) and (4) over the whole catalogue
+* ``rece_forward``  -- the whole forward path, steps 1 to 5, given the random vectors B
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+        i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+        i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        lib.oracle_bucketize.argtypes = [f32p, i64, i32, f32p, i32, i32p]
+        lib.oracle_bucketize.restype = None
+        lib.oracle_stable_argsort.argtypes = [i32p, i64, i32p]
+        lib.oracle_stable_argsort.restype = None
+        lib.oracle_chunk_start.argtypes = [i64, i64, i64]
+        lib.oracle_chunk_start.restype = i64
+        lib.oracle_select.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32, i32,
+                                      i32p, i32p, i32p, f32p, i64p]
+        lib.oracle_select.restype = None
+        lib.oracle_rece_loss.argtypes = [f32p, f32p, i32p, i64, i32, i32, i32p, f64p, f64p,
+                                         f64p]
+        lib.oracle_rece_loss.restype = None
+        lib.oracle_rece_grad.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32p, f64p,
+                                         ctypes.c_double, f64p, f64p]
+        lib.oracle_rece_grad.restype = None
+        lib.oracle_full_ce_loss.argtypes = [f32p, f32p, i32p, i64, i64, i32, f64p, f64p, f64p]
+        lib.oracle_full_ce_loss.restype = None
+        lib.oracle_full_ce_grad.argtypes = [f32p, f32p, i32p, i64, i64, i32, f64p,
+                                            ctypes.c_double, f64p, f64p]
+        lib.oracle_full_ce_grad.restype = None
+        lib.oracle_dot_f32.argtypes = [f32p, f32p, i32]
+        lib.oracle_dot_f32.restype = ctypes.c_float
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _i32(a):
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def dot_f32(a, b) -> np.float32:
+    """fp32 fmaf-chain inner product, the score every integer decision is taken on."""
+    a, b = _f32(a), _f32(b)
+    return np.float32(_load().oracle_dot_f32(a, b, a.shape[0]))
+
+
+def bucketize(V, B) -> np.ndarray:
+    """Bucket id of every row of V: argmax_b <B[b], v> (ties to the lowest b)."""
+    V, B = _f32(V), _f32(B)
+    out = np.empty(V.shape[0], np.int32)
+    _load().oracle_bucketize(V, V.shape[0], V.shape[1], B, B.shape[0], out)
+    return out
+
+
+def stable_argsort(keys) -> np.ndarray:
+    keys = _i32(keys)
+    out = np.empty(keys.shape[0], np.int32)
+    _load().oracle_stable_argsort(keys, keys.shape[0], out)
+    return out
+
+
+def chunk_start(c: int, M: int, n_c: int) -> int:
+    return int(_load().oracle_chunk_start(c, M, n_c))
+
+
+def select(X, Y, target, permX, permY, n_c, n_ec, k):
+    """Top-k negatives of every row over all rounds' chunk windows.
+
+    permX: [n_r, N], permY: [n_r, C].  Returns (selected [N,k] int32 -1 padded,
+    sel_score [N,k] fp32, n_cand [N] int64)."""
+    X, Y, target = _f32(X), _f32(Y), _i32(target)
+    permX, permY = _i32(permX), _i32(permY)
+    N, d = X.shape
+    C = Y.shape[0]
+    n_r = permX.shape[0]
+    sel = np.empty((N, k), np.int32)
+    score = np.empty((N, k), np.float32)
+    n_cand = np.empty(N, np.int64)
+    _load().oracle_select(X, Y, target, N, C, d, n_c, n_ec, n_r, k, permX, permY, sel, score,
+                          n_cand)
+    return sel, score, n_cand
+
+
+def rece_loss(X, Y, target, selected):
+    """(loss, row_loss [N] fp64, lse [N] fp64) of the reduced CE for a given selection."""
+    X, Y, target, selected = _f32(X), _f32(Y), _i32(target), _i32(selected)
+    N, d = X.shape
+    k = selected.shape[1] if selected.ndim == 2 else 0
+    row = np.empty(N, np.float64)
+    lse = np.empty(N, np.float64)
+    loss = np.zeros(1, np.float64)
+    _load().oracle_rece_loss(X, Y, target, N, d, k, selected.reshape(N, k), row, lse, loss)
+    return float(loss[0]), row, lse
+
+
+def rece_grad(X, Y, target, selected, lse, dloss=1.0):
+    """(dX [N,d], dY [C,d]) in fp64 of the reduced CE, selection held constant."""
+    X, Y, target, selected = _f32(X), _f32(Y), _i32(target), _i32(selected)
+    N, d = X.shape
+    C = Y.shape[0]
+    k = selected.shape[1]
+    dX = np.empty((N, d), np.float64)
+    dY = np.empty((C, d), np.float64)
+    _load().oracle_rece_grad(X, Y, target, N, C, d, k, selected,
+                             np.ascontiguousarray(lse, np.float64), float(dloss), dX, dY)
+    return dX, dY
+
+
+def full_ce_loss(X, Y, target):
+    X, Y, target = _f32(X), _f32(Y), _i32(target)
+    N, d = X.shape
+    row = np.empty(N, np.float64)
+    lse = np.empty(N, np.float64)
+    loss = np.zeros(1, np.float64)
+    _load().oracle_full_ce_loss(X, Y, target, N, Y.shape[0], d, row, lse, loss)
+    return float(loss[0]), row, lse
+
+
+def full_ce_grad(X, Y, target, lse, dloss=1.0):
+    X, Y, target = _f32(X), _f32(Y), _i32(target)
+    N, d = X.shape
+    C = Y.shape[0]
+    dX = np.empty((N, d), np.float64)
+    dY = np.empty((C, d), np.float64)
+    _load().oracle_full_ce_grad(X, Y, target, N, C, d, np.ascontiguousarray(lse, np.float64),
+                                float(dloss), dX, dY)
+    return dX, dY
+
+
+def rece_forward(X, Y, target, B, n_c, n_ec, k):
+    """Steps 1-5 of the path given the random vectors B [n_r, n_b, d].
+
+    Returns a dict with per-round bucket ids (bx [n_r,N], by [n_r,C]), stable orders
+    (permX, permY), the selection, candidate counts, and the loss values."""
+    X, Y, B = _f32(X), _f32(Y), _f32(B)
+    n_r = B.shape[0]
+    bx = np.stack([bucketize(X, B[r]) for r in range(n_r)]) if n_r else np.zeros((0, len(X)))
+    by = np.stack([bucketize(Y, B[r]) for r in range(n_r)])
+    permX = np.stack([stable_argsort(bx[r]) for r in range(n_r)])
+    permY = np.stack([stable_argsort(by[r]) for r in range(n_r)])
+    sel, score, n_cand = select(X, Y, target, permX, permY, n_c, n_ec, k)
+    loss, row, lse = rece_loss(X, Y, target, sel)
+    return dict(bx=bx, by=by, permX=permX, permY=permY, selected=sel, sel_score=score,
+                n_cand=n_cand, loss=loss, row_loss=row, lse=lse)

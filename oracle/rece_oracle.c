@@ -1,0 +1,306 @@
+/*
+ * rece_oracle.c -- plain, slow, CPU reference of the reduced cross-entropy loss.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the oracle that the CUDA path is checked
+ * against.  Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+ * load it.  It shares no code, header, table or constant with the CUDA library, and
+ * the CUDA library never calls it.
+ *
+ * Sources (cited by page title and section):
+ *   [RECE]  "RECE: Reduced Cross-Entropy Loss for Large-Catalogue Sequential
+ *           Recommenders", section 3 (Reduced Cross-Entropy): equations (3) and (4),
+ *           Algorithm 1, and the paragraph before Algorithm 1 (rounds, duplicate pairs,
+ *           neighbouring chunks).
+ *   [SCE]   "Scalable Cross-Entropy Loss for Sequential Recommendations with Large
+ *           Item Catalogs", abstract (softmax approximated over a subset found by
+ *           maximum inner product search, i.e. the top-k negatives per row).
+ *
+ * Precision.  Every decision that yields an integer (bucket argmax, candidate order)
+ * is taken on fp32 scores, each formed by one fixed-order fused multiply-add chain
+ *     s = 0; for t = 0..d-1: s = fmaf(a[t], b[t], s)
+ * (both sides use this order so the indices they produce can be compared bit for
+ * bit).  Loss values and gradients are computed in fp64 from the fp32 inputs.
+ * Build with -ffp-contract=off and without fast-math.
+ *
+ * Readings of the pages (where they are silent or ambiguous):
+ *   - chunk c of an M-element sorted array starts at ceil(c*M/n_c);
+ *   - the window of chunk c is the union of chunks max(0,c-n_ec)..min(n_c-1,c+n_ec)
+ *     of the sorted catalogue (edge chunks see fewer items);
+ *   - the row's own positive item is never a negative;
+ *   - candidates from all rounds are united and de-duplicated by item id (subtracting
+ *     ln(count) from a logit seen count times, as the pages do, is the same thing);
+ *   - the negatives kept are the k best candidates by (score descending, item id
+ *     ascending); with fewer than k candidates all are kept;
+ *   - selection and buckets are constants for the gradient;
+ *   - the loss is the mean over rows; an empty batch has loss 0.
+ *
+ * Parity of every function here is pinned by tests that do not call this file's
+ * arithmetic (brute force on exactly representable inputs, library sorts and argmax,
+ * the full-CE identity, finite differences, invariants).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* One fp32 score: the fixed-order fmaf chain over the d coordinates. */
+static float dot_f32(const float* a, const float* b, int32_t d) {
+  float s = 0.0f;
+  for (int32_t t = 0; t < d; ++t) s = fmaf(a[t], b[t], s);
+  return s;
+}
+
+/* The same inner product in fp64 (for loss values and gradients). */
+static double dot_f64(const float* a, const float* b, int32_t d) {
+  double s = 0.0;
+  for (int32_t t = 0; t < d; ++t) s += (double)a[t] * (double)b[t];
+  return s;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* [RECE] Algorithm 1, the two argmax steps: bucket of row v = index of the random
+ * vector b_k with the largest inner product <b_k, v>.  Ties go to the lowest k. */
+void oracle_bucketize(const float* V, int64_t M, int32_t d, const float* B, int32_t n_b,
+                      int32_t* bucket) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i) {
+    const float* v = V + i * (int64_t)d;
+    int32_t best = 0;
+    float best_s = dot_f32(B, v, d);
+    for (int32_t b = 1; b < n_b; ++b) {
+      float s = dot_f32(B + (int64_t)b * d, v, d);
+      if (s > best_s) {
+        best_s = s;
+        best = b;
+      }
+    }
+    bucket[i] = best;
+  }
+}
+
+typedef struct {
+  int32_t key;
+  int32_t idx;
+} key_idx_t;
+
+static int cmp_key_idx(const void* pa, const void* pb) {
+  const key_idx_t* a = (const key_idx_t*)pa;
+  const key_idx_t* b = (const key_idx_t*)pb;
+  if (a->key != b->key) return a->key < b->key ? -1 : 1;
+  return a->idx < b->idx ? -1 : (a->idx > b->idx ? 1 : 0);
+}
+
+/* [RECE] Algorithm 1, the two argsort steps, read as a stable sort: perm lists the
+ * element indices in order of (key ascending, original index ascending). */
+void oracle_stable_argsort(const int32_t* keys, int64_t M, int32_t* perm) {
+  key_idx_t* a = (key_idx_t*)malloc(sizeof(key_idx_t) * (size_t)(M > 0 ? M : 1));
+  for (int64_t i = 0; i < M; ++i) {
+    a[i].key = keys[i];
+    a[i].idx = (int32_t)i;
+  }
+  qsort(a, (size_t)M, sizeof(key_idx_t), cmp_key_idx);
+  for (int64_t i = 0; i < M; ++i) perm[i] = a[i].idx;
+  free(a);
+}
+
+/* [RECE] Algorithm 1, chunk sets: element i of an M-long sorted array is in chunk c
+ * when c*M/n_c <= i < (c+1)*M/n_c, so chunk c starts at ceil(c*M/n_c). */
+int64_t oracle_chunk_start(int64_t c, int64_t M, int64_t n_c) {
+  return (c * M + n_c - 1) / n_c;
+}
+
+typedef struct {
+  float score;
+  int32_t item;
+} cand_t;
+
+/* Candidate order of [SCE]: higher score first; equal scores by lower item id. */
+static int cmp_cand(const void* pa, const void* pb) {
+  const cand_t* a = (const cand_t*)pa;
+  const cand_t* b = (const cand_t*)pb;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
+  return a->item < b->item ? -1 : (a->item > b->item ? 1 : 0);
+}
+
+/* Chunk index that holds sorted position pos (a plain search over the chunk starts). */
+static int64_t chunk_of(int64_t pos, int64_t M, int64_t n_c) {
+  int64_t c = 0;
+  while (c + 1 < n_c && oracle_chunk_start(c + 1, M, n_c) <= pos) ++c;
+  return c;
+}
+
+/* Steps 3-4: for every row, the candidate negatives from all rounds (window items of
+ * the row's chunk, positive removed, de-duplicated) and the k best of them.
+ *   permX [n_r*N], permY [n_r*C]  : per-round stable bucket orders (from above)
+ *   selected [N*k]               : item ids, best first, -1 padded
+ *   sel_score [N*k]              : their fp32 scores (-inf for padding)
+ *   n_cand [N]                   : number of distinct candidates of each row */
+void oracle_select(const float* X, const float* Y, const int32_t* target, int64_t N, int64_t C,
+                   int32_t d, int32_t n_c, int32_t n_ec, int32_t n_r, int32_t k,
+                   const int32_t* permX, const int32_t* permY, int32_t* selected,
+                   float* sel_score, int64_t* n_cand) {
+  /* position of each row in each round's sorted order */
+  int64_t* posX = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N * n_r > 0 ? N * n_r : 1));
+  for (int32_t r = 0; r < n_r; ++r)
+    for (int64_t p = 0; p < N; ++p) posX[(int64_t)r * N + permX[(int64_t)r * N + p]] = p;
+
+#pragma omp parallel
+  {
+    unsigned char* seen = (unsigned char*)calloc((size_t)C, 1);
+    cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)C);
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t i = 0; i < N; ++i) {
+      int64_t n = 0;
+      for (int32_t r = 0; r < n_r; ++r) {
+        int64_t c = chunk_of(posX[(int64_t)r * N + i], N, n_c);
+        int64_t c_lo = c - n_ec < 0 ? 0 : c - n_ec;
+        int64_t c_hi = c + n_ec + 1 > n_c ? n_c : c + n_ec + 1;
+        int64_t q_lo = oracle_chunk_start(c_lo, C, n_c);
+        int64_t q_hi = oracle_chunk_start(c_hi, C, n_c);
+        for (int64_t q = q_lo; q < q_hi; ++q) {
+          int32_t j = permY[(int64_t)r * C + q];
+          if (j == target[i] || seen[j]) continue;
+          seen[j] = 1;
+          cand[n].item = j;
+          ++n;
+        }
+      }
+      for (int64_t a = 0; a < n; ++a) {
+        cand[a].score = dot_f32(X + i * (int64_t)d, Y + (int64_t)cand[a].item * d, d);
+        seen[cand[a].item] = 0;
+      }
+      qsort(cand, (size_t)n, sizeof(cand_t), cmp_cand);
+      for (int32_t a = 0; a < k; ++a) {
+        if (a < n) {
+          selected[i * (int64_t)k + a] = cand[a].item;
+          sel_score[i * (int64_t)k + a] = cand[a].score;
+        } else {
+          selected[i * (int64_t)k + a] = -1;
+          sel_score[i * (int64_t)k + a] = -INFINITY;
+        }
+      }
+      n_cand[i] = n;
+    }
+    free(cand);
+    free(seen);
+  }
+  free(posX);
+}
+
+/* Step 5, [RECE] Algorithm 1 loss lines with [SCE]'s subset: per row
+ *   l+   = <x_i, y_{z_i}>,  l_ij = <x_i, y_j> for j in S_i
+ *   lse  = log(exp(l+) + sum_j exp(l_ij)),  loss_i = lse - l+,  L = mean_i loss_i
+ * in fp64.  selected entries < 0 are padding. */
+void oracle_rece_loss(const float* X, const float* Y, const int32_t* target, int64_t N,
+                      int32_t d, int32_t k, const int32_t* selected, double* row_loss,
+                      double* lse, double* loss) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    double lp = dot_f64(x, Y + (int64_t)target[i] * d, d);
+    double m = lp;
+    for (int32_t a = 0; a < k; ++a) {
+      int32_t j = selected[i * (int64_t)k + a];
+      if (j < 0) continue;
+      double l = dot_f64(x, Y + (int64_t)j * d, d);
+      if (l > m) m = l;
+    }
+    double s = exp(lp - m);
+    for (int32_t a = 0; a < k; ++a) {
+      int32_t j = selected[i * (int64_t)k + a];
+      if (j < 0) continue;
+      s += exp(dot_f64(x, Y + (int64_t)j * d, d) - m);
+    }
+    lse[i] = m + log(s);
+    row_loss[i] = lse[i] - lp;
+  }
+  double total = 0.0;
+  for (int64_t i = 0; i < N; ++i) total += row_loss[i];
+  *loss = N > 0 ? total / (double)N : 0.0;
+}
+
+/* Step 6, [RECE] equation (4) restricted to the row's positive and its selected
+ * negatives (selection held constant):
+ *   p_ij = exp(l_ij - lse_i),  g_ij = (p_ij - [j == z_i]) * dloss / N
+ *   dX_i = sum_j g_ij y_j,     dY_j = sum_i g_ij x_i            (fp64) */
+void oracle_rece_grad(const float* X, const float* Y, const int32_t* target, int64_t N, int64_t C,
+                      int32_t d, int32_t k, const int32_t* selected, const double* lse,
+                      double dloss, double* dX, double* dY) {
+  double scale = N > 0 ? dloss / (double)N : 0.0;
+  memset(dY, 0, sizeof(double) * (size_t)C * (size_t)d);
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    double* dx = dX + i * (int64_t)d;
+    for (int32_t t = 0; t < d; ++t) dx[t] = 0.0;
+    for (int32_t a = -1; a < k; ++a) {
+      int32_t j = a < 0 ? target[i] : selected[i * (int64_t)k + a];
+      if (j < 0) continue;
+      const float* y = Y + (int64_t)j * d;
+      double p = exp(dot_f64(x, y, d) - lse[i]);
+      double g = (a < 0 ? p - 1.0 : p) * scale;
+      double* dy = dY + (int64_t)j * d;
+      for (int32_t t = 0; t < d; ++t) {
+        dx[t] += g * (double)y[t];
+        dy[t] += g * (double)x[t];
+      }
+    }
+  }
+}
+
+/* [RECE] equation (3): full cross-entropy over the whole catalogue, in fp64. */
+void oracle_full_ce_loss(const float* X, const float* Y, const int32_t* target, int64_t N,
+                         int64_t C, int32_t d, double* row_loss, double* lse, double* loss) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < C; ++j) {
+      double l = dot_f64(x, Y + j * d, d);
+      if (l > m) m = l;
+    }
+    double s = 0.0;
+    for (int64_t j = 0; j < C; ++j) s += exp(dot_f64(x, Y + j * d, d) - m);
+    lse[i] = m + log(s);
+    row_loss[i] = lse[i] - dot_f64(x, Y + (int64_t)target[i] * d, d);
+  }
+  double total = 0.0;
+  for (int64_t i = 0; i < N; ++i) total += row_loss[i];
+  *loss = N > 0 ? total / (double)N : 0.0;
+}
+
+/* [RECE] equation (4) over the whole catalogue: g_ij = (softmax_ij - [j == z_i]) dloss/N. */
+void oracle_full_ce_grad(const float* X, const float* Y, const int32_t* target, int64_t N,
+                         int64_t C, int32_t d, const double* lse, double dloss, double* dX,
+                         double* dY) {
+  double scale = N > 0 ? dloss / (double)N : 0.0;
+  memset(dY, 0, sizeof(double) * (size_t)C * (size_t)d);
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    double* dx = dX + i * (int64_t)d;
+    for (int32_t t = 0; t < d; ++t) dx[t] = 0.0;
+    for (int64_t j = 0; j < C; ++j) {
+      const float* y = Y + j * d;
+      double g = (exp(dot_f64(x, y, d) - lse[i]) - (j == target[i] ? 1.0 : 0.0)) * scale;
+      double* dy = dY + j * d;
+      for (int32_t t = 0; t < d; ++t) {
+        dx[t] += g * (double)y[t];
+        dy[t] += g * (double)x[t];
+      }
+    }
+  }
+}
+
+/* Exposed for the tests: the fp32 fmaf-chain score of one pair. */
+float oracle_dot_f32(const float* a, const float* b, int32_t d) { return dot_f32(a, b, d); }
