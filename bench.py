@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the reduced cross-entropy loss, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sasrec]
+
+One step = the whole path on one batch: bucketing + sort (rece_bucketize_sort), chunk
+scores + top-k + loss (rece_loss_fwd) and gradients (rece_loss_bwd), with fresh random
+vectors B every step.  Inputs are synthetic (seeded, shaped like the RECE paper's
+SASRec workloads) and resident in HBM; L2 is flushed (a 256 MiB write) between timed
+steps because the inputs fit in L2.  Multi-GPU: every rank runs the whole path on its own
+batch against its own copy of the catalogue (weak scaling, no collective on the data
+path); the time is the max over ranks.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle instead (a
+deliberately slow baseline, rank 0 only).
+"""
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "rows/sec RECE loss fwd+bwd (1×B200), % roofline, peak HBM vs full CE"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="sasrec")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-memory", action="store_true")
+    ap.add_argument("--flags", type=int, default=0, help="rece_config_t.flags")
+    return ap.parse_args()
+
+
+def workload_desc(w):
+    return (f"{w.name}: N={w.N} (rows), d={w.d}, C={w.C}, {w.dtype}, n_b={w.n_b}, n_c={w.n_c}, "
+            f"n_ec={w.n_ec}, n_r={w.n_r}, k={w.k}, targets "
+            + (f"Zipf({w.target_alpha})" if w.target_alpha else "uniform"))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"),
+                    sm_max_mhz=d.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+# ------------------------------------------------------------------ algorithmic work
+def chunk_start(c, M, n_c):
+    return (c * M + n_c - 1) // n_c
+
+
+def pairs_per_round(w):
+    """Sum over chunks of (rows in chunk) x (items in its window)."""
+    tot = 0
+    for c in range(w.n_c):
+        rows = chunk_start(c + 1, w.N, w.n_c) - chunk_start(c, w.N, w.n_c)
+        lo, hi = max(0, c - w.n_ec), min(w.n_c, c + w.n_ec + 1)
+        tot += rows * (chunk_start(hi, w.C, w.n_c) - chunk_start(lo, w.C, w.n_c))
+    return tot
+
+
+def stage_work(w):
+    """Algorithmic (flops, bytes) of every stage, per step (one launch sequence)."""
+    e = 2 if w.dtype == "bf16" else 4
+    N, C, d, nb, nr, k = w.N, w.C, w.d, w.n_b, w.n_r, w.k
+    return {
+        "bucketize": (2 * (N + C) * nb * d * nr, nr * (N + C) * (d * e + 4)),
+        "sort": (0, nr * (N + C) * 16),
+        "select": (2 * d * pairs_per_round(w) * nr, nr * (N + C) * d * e + nr * N * k * 8),
+        "merge_loss": (0, nr * N * k * 8 + N * k * 4 + 8 * N + N * d * e),
+        "mean": (0, 4 * N),
+        "bwd_rows": (4 * N * (k + 1) * d, N * d * e + N * (k + 1) * d * e + 4 * N * k
+                     + N * d * 4 + 8 * N * (k + 1)),
+        "bwd_sort": (0, 3 * N * (k + 1) * 16),
+        "bwd_items": (2 * N * (k + 1) * d, N * (k + 1) * 8 + N * (k + 1) * d * e + C * d * 4),
+    }
+
+
+def stage_bound(stage, flags, dtype):
+    if stage in ("bucketize", "select"):
+        if dtype == "bf16" and not (flags & 1) and TENSOR_STAGES.get(stage, False):
+            return "tensor"
+        return "alu"
+    return "hbm"
+
+
+# stages that run on tcgen05 in bf16 mode (without RECE_FLAG_FMA_SCORES)
+TENSOR_STAGES = {}
+
+
+KERNEL_SOURCES = {
+    "bucketize": ["bucketize.cu"], "sort": ["sort.cu"], "select": ["select.cu"],
+    "merge_loss": ["loss.cu"], "mean": ["loss.cu"], "bwd_rows": ["backward.cu"],
+    "bwd_sort": ["sort.cu"], "bwd_items": ["backward.cu"],
+}
+
+
+def source_hash(stage):
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[stage]:
+        h.update(open(os.path.join(ROOT, "reduced_cross_entropy_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(stage, workload):
+    """DRAM bytes per launch of this stage from a committed ncu capture, if the kernel
+    source is unchanged since (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{stage}@{workload}")
+    if not d or d.get("source_sha") != source_hash(stage):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_step_seconds(w, X, Y, t, B, rows=256, bucket_frac=16):
+    """Estimated seconds of one whole step of the CPU oracle, from a bounded sample:
+    bucketing of every bucket_frac-th row of X and Y (scaled up), the full stable sorts,
+    and selection + loss + gradient of `rows` rows (scaled by N / rows)."""
+    import oracle
+    n_r = w.n_r
+    t0 = time.perf_counter()
+    for r in range(n_r):
+        oracle.bucketize(X[::bucket_frac], B[r])
+        oracle.bucketize(Y[::bucket_frac], B[r])
+    t_bucket = (time.perf_counter() - t0) * bucket_frac
+    # valid orders for the sampled rows come from a full (untimed) bucketing, once
+    if not hasattr(oracle_step_seconds, "_perm"):
+        bx = np.stack([oracle.bucketize(X, B[r]) for r in range(n_r)])
+        by = np.stack([oracle.bucketize(Y, B[r]) for r in range(n_r)])
+        oracle_step_seconds._perm = (bx, by)
+    bx, by = oracle_step_seconds._perm
+    t0 = time.perf_counter()
+    px = np.stack([oracle.stable_argsort(bx[r]) for r in range(n_r)])
+    py = np.stack([oracle.stable_argsort(by[r]) for r in range(n_r)])
+    t_sort = time.perf_counter() - t0
+    sample = np.linspace(0, w.N - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    sel, _, _ = oracle.select(X, Y, t, px, py, w.n_c, w.n_ec, w.k, rows=sample)
+    _, _, lse = oracle.rece_loss(X[sample], Y, t[sample], sel)
+    oracle.rece_grad(X[sample], Y, t[sample], sel, lse, 1.0)
+    t_rows = (time.perf_counter() - t0) * w.N / rows
+    return t_bucket + t_sort + t_rows
+
+
+def oracle_sample_desc(rows, bucket_frac):
+    return (f"bucketing of every {bucket_frac}th row of X and Y (x{bucket_frac}), full stable "
+            f"sorts, selection+loss+gradient of {rows} evenly spaced rows (x N/{rows})")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from reduced_cross_entropy_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    X, Y, t = synth.make_inputs(w, seed=0)
+    B = synth.projections(0, 0, w.n_r, w.n_b, w.d, w.dtype)
+    rows, frac = 128, 32
+    for _ in range(args.warmup):
+        oracle_step_seconds(w, X, Y, t, B, rows, frac)
+    secs = [oracle_step_seconds(w, X, Y, t, B, rows, frac) for _ in range(args.steps)]
+    total = sum(secs)
+    value = w.N * args.steps / total
+    cores = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_desc(w)},
+            "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
+                             "sample": oracle_sample_desc(rows, frac)},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from reduced_cross_entropy_b200 import _lib, ops, synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    L = _lib.lib()
+    w = synth.WORKLOADS[args.workload]
+    X, Y, t = synth.make_inputs(w, seed=rank)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype,
+                    flags=args.flags)
+    Xd = torch.from_numpy(X).to(dev).to(tdt)
+    Yd = torch.from_numpy(Y).to(dev).to(tdt)
+    td = torch.from_numpy(t).to(dev)
+    n_steps = args.warmup + args.steps
+    Bs = [torch.from_numpy(synth.projections(0, s, w.n_r, w.n_b, w.d, w.dtype)).to(dev).to(tdt)
+          for s in range(n_steps)]
+    ws = plan.workspace(dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    sel = torch.empty(w.N, w.k, dtype=torch.int32, device=dev)
+    lse = torch.empty(w.N, dtype=torch.float32, device=dev)
+    dloss = torch.ones(1, dtype=torch.float32, device=dev)
+    dX = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+    dY = torch.empty(w.C, w.d, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = lambda x: ctypes.c_void_p(x.data_ptr())  # noqa: E731
+    nbytes = ctypes.c_size_t(ws.numel())
+
+    def step(Bt):
+        _lib.check(L.rece_bucketize_sort(plan._h, vp(Bt), vp(Xd), vp(Yd), vp(ws), nbytes, sp),
+                   "bucketize_sort")
+        _lib.check(L.rece_loss_fwd(plan._h, vp(Xd), vp(Yd), vp(td), vp(ws), nbytes, vp(loss),
+                                   None, vp(sel), vp(lse), sp), "loss_fwd")
+        _lib.check(L.rece_loss_bwd(plan._h, vp(Xd), vp(Yd), vp(td), vp(sel), vp(lse),
+                                   vp(dloss), vp(ws), nbytes, vp(dX), vp(dY), sp), "loss_bwd")
+
+    for s in range(args.warmup):
+        flush.zero_()
+        step(Bs[s])
+    torch.cuda.synchronize(dev)
+    assert ops.device_status(ws) == 0
+
+    # timed region: K steps, each bracketed by events; per-stage events recorded by the
+    # library on the same stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    n_st = len(_lib.STAGES)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_st)]
+           for _ in range(args.steps)]
+    for row in sev:  # torch creates the CUDA event at its first record
+        for e in row:
+            e.record(stream)
+    sev_h = [(ctypes.c_void_p * (2 * n_st))(*[ctypes.c_void_p(e.cuda_event) for e in row])
+             for row in sev]
+    launches0 = L.rece_kernel_launch_count()
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            _lib.check(L.rece_plan_set_stage_events(plan._h, sev_h[s]), "stage events")
+            ev[s][0].record(stream)
+            step(Bs[args.warmup + s])
+            ev[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    launches = L.rece_kernel_launch_count() - launches0
+    L.rece_plan_set_stage_events(plan._h, None)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    stage_ms = {name: statistics.mean(sev[s][2 * i].elapsed_time(sev[s][2 * i + 1])
+                                      for s in range(args.steps))
+                for i, name in enumerate(_lib.STAGES)}
+    value = world * w.N * args.steps / (total_ms / 1000.0)
+
+    # roofline of the dominant stage
+    peaks = load_peaks()
+    work = stage_work(w)
+    dom = max(stage_ms, key=stage_ms.get)
+    bound = stage_bound(dom, args.flags, w.dtype)
+    flops, bytes_ = work[dom]
+    sec = stage_ms[dom] / 1000.0
+    if bound == "hbm":
+        achieved, peak, unit = bytes_ / sec / 1e9, peaks["hbm_gbs"], "GB/s"
+    elif bound == "tensor":
+        achieved, peak, unit = flops / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:  # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+        achieved, peak, unit = flops / sec / 1e12, 148 * 128 * 2 * peaks["sm_max_mhz"] / 1e6, \
+            "TFLOP/s"
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak,
+                "peak_source": peaks["source"] if bound != "alu" else
+                "derived: 148 SM x 128 FP32 lanes x 2 x sm_max_mhz",
+                "traffic": recorded_traffic(dom, w.name),
+                "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
+
+    # end to end: host (pinned) inputs copied in, loss copied out, every step
+    Xh = torch.from_numpy(X).to(tdt).pin_memory()
+    Yh = torch.from_numpy(Y).to(tdt).pin_memory()
+    th = torch.from_numpy(t).pin_memory()
+    Bh = [b.cpu().pin_memory() for b in Bs]
+    loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+    h2d = Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size() + th.numel() * 4 \
+        + Bh[0].numel() * Bh[0].element_size()
+    Bd = torch.empty_like(Bs[0])
+    e2e_ms = []
+    for s in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Xd.copy_(Xh, non_blocking=True)
+        Yd.copy_(Yh, non_blocking=True)
+        td.copy_(th, non_blocking=True)
+        Bd.copy_(Bh[s], non_blocking=True)
+        step(Bd)
+        loss_h.copy_(loss, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if s >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        tt = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_total = float(tt.item())
+    e2e = {"value": world * w.N * args.steps / (e2e_total / 1000.0), "unit": "rows/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4}
+
+    line = {"metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": workload_desc(w),
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "scores": "fmaf CUDA cores" if (args.flags & 1 or
+                                                       not TENSOR_STAGES) else "tcgen05"},
+            "roofline": roofline, "stages_ms": stage_ms, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clk.summary()}
+
+    if rank == 0 and world == 1 and not args.no_memory:
+        line["peak_hbm"] = measure_memory(torch, ops, plan, w, Xd, Yd, td, Bs[0], dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        rows, frac = 256, 16
+        secs = oracle_step_seconds(w, X, Y, t, synth.projections(0, 0, w.n_r, w.n_b, w.d,
+                                                                   w.dtype), rows, frac)
+        line["cpu_baseline"] = {"value": w.N / secs, "unit": "rows/s",
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": oracle_sample_desc(rows, frac)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
+    """Peak HBM of one RECE fwd+bwd vs the fused exact full CE and the materialised
+    full CE (logits + their gradient in fp32), all from the same resident inputs."""
+    out = {}
+    base = torch.cuda.memory_allocated(dev)
+
+    def peak(fn):
+        torch.cuda.synchronize(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        fn()
+        torch.cuda.synchronize(dev)
+        return torch.cuda.max_memory_allocated(dev) - base
+
+    def rece():
+        ws = plan.workspace(dev)
+        ops.bucketize_sort(plan, B, Xd, Yd, ws)
+        _, _, s, l = ops.loss_fwd(plan, Xd, Yd, td, ws, want_row_loss=False)
+        ops.loss_bwd(plan, Xd, Yd, td, s, l, torch.ones(1, device=dev), ws)
+
+    def fused():
+        _, _, l, ws = ops.full_ce_fwd(Xd, Yd, td)
+        ops.full_ce_bwd(Xd, Yd, td, l, torch.ones(1, device=dev), ws)
+
+    out["rece_bytes"] = peak(rece)
+    out["full_ce_fused_bytes"] = peak(fused)
+    mat = 8 * w.N * w.C
+    out["full_ce_materialised_bytes_computed"] = mat
+    free = torch.cuda.mem_get_info(dev)[0]
+    if 3 * mat < free:
+        def materialised():
+            Xr = Xd.float().requires_grad_()
+            Yr = Yd.float().requires_grad_()
+            torch.nn.functional.cross_entropy(Xr @ Yr.T, td.long()).backward()
+        out["full_ce_materialised_bytes_measured"] = peak(materialised)
+    ref = out.get("full_ce_materialised_bytes_measured", mat)
+    out["ratio_vs_materialised"] = ref / max(out["rece_bytes"], 1)
+    out["ratio_vs_fused"] = out["full_ce_fused_bytes"] / max(out["rece_bytes"], 1)
+    out["note"] = "bytes above the resident inputs; torch.cuda.max_memory_allocated"
+    return out
+
+
+if __name__ == "__main__":
+    main()

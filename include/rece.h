@@ -1,0 +1,207 @@
+/*
+ * rece.h -- C ABI of the B200 (sm_100a) reduced cross-entropy library.
+ *
+ * The loss is RECE ("RECE: Reduced Cross-Entropy Loss for Large-Catalogue Sequential
+ * Recommenders", section 3, Algorithm 1) with the top-k subset of SCE ("Scalable
+ * Cross-Entropy Loss for Sequential Recommendations with Large Item Catalogs",
+ * abstract):
+ *
+ *   1. project the model outputs X [N x d] and the catalogue Y [C x d] onto n_b random
+ *      vectors and give every row the bucket with the largest inner product;
+ *   2. sort the rows of X and of Y by bucket (stable);
+ *   3. split both sorted arrays into n_c equal chunks and score every row of chunk c
+ *      against the items of chunks c-n_ec .. c+n_ec, over n_r independent rounds;
+ *   4. keep, per row, the k highest-scoring negatives (the positive excluded, rounds
+ *      united and de-duplicated, ties to the lower item id);
+ *   5. softmax cross-entropy over the positive plus those negatives, mean over rows;
+ *   6. gradients dX and dY of that loss (selection held constant).
+ * The N x C logit matrix is never formed.  An exact fused full cross-entropy
+ * (equations 3 and 4 of the RECE paper) is provided for comparison.
+ *
+ * Conventions shared by every call
+ *   - Pointers marked "device" point to GPU memory the caller owns; the library never
+ *     allocates device memory.  Matrices are row-major and contiguous.
+ *   - Element type of X, Y, B: fp32 in RECE_MODE_FP32_EXACT, bf16 in RECE_MODE_BF16.
+ *     Losses, log-sum-exps and gradients are always fp32.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
+ *     only enqueue work; nothing synchronises except rece_get_device_status.
+ *   - Host-side argument errors are returned at once and enqueue nothing.  Bad device
+ *     data (a target outside [0, C)) cannot be seen on the host: the kernels record it
+ *     in the workspace's status word, the affected rows get a NaN loss, and
+ *     rece_get_device_status reports it.
+ *   - No global state: plans are independent host objects; one plan may be used from
+ *     one thread at a time.
+ */
+#ifndef RECE_H_
+#define RECE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RECE_API __attribute__((visibility("default")))
+#else
+#define RECE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RECE_OK = 0,
+  RECE_ERR_INVALID_ARG = 1,  /* a size, pointer or config field is out of range */
+  RECE_ERR_UNSUPPORTED = 2,  /* valid, but not implemented for this mode/shape */
+  RECE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+  RECE_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, ...) */
+  RECE_ERR_DEVICE_INPUT = 5, /* device-side input error recorded (see status word) */
+  RECE_ERR_TIMEOUT = 6,      /* a bounded device wait gave up */
+  RECE_ERR_NO_DEVICE = 7     /* no usable sm_100 device for this call */
+} rece_status_t;
+
+typedef enum {
+  /* fp32 inputs; every score that decides an index (bucket, selection) is the fixed-
+   * order chain s = fmaf(a[t], b[t], s), t = 0..d-1 from s = 0, so indices are
+   * reproducible bit for bit by any implementation of the same chain. */
+  RECE_MODE_FP32_EXACT = 0,
+  /* bf16 inputs; scores come from the tcgen05 tensor cores (fp32 accumulation). */
+  RECE_MODE_BF16 = 1
+} rece_mode_t;
+
+/* rece_config_t.flags */
+#define RECE_FLAG_FMA_SCORES 0x1u /* bf16 mode: use the fmaf-chain CUDA-core kernels for
+                                     the scores as well (bit-exact on bf16 inputs) */
+
+/* Bits of the device status word (rece_get_device_status). */
+#define RECE_DEVICE_BAD_TARGET 0x1u /* some target outside [0, C) */
+#define RECE_DEVICE_TIMEOUT 0x2u    /* a bounded wait inside a kernel gave up */
+
+typedef struct {
+  int64_t N;     /* rows (batch x sequence), >= 0 */
+  int64_t C;     /* catalogue size, >= 1 */
+  int32_t d;     /* embedding width, >= 1 (bf16 mode: multiple of 16 for tcgen05) */
+  int32_t n_b;   /* random vectors per round, 1 .. 4096 */
+  int32_t n_c;   /* chunks, 1 .. min(N, C) (any n_c <= C when N = 0) */
+  int32_t n_ec;  /* neighbouring chunks on each side, >= 0 */
+  int32_t n_r;   /* rounds, 1 .. 8 */
+  int32_t k;     /* negatives kept per row, 1 .. 4096 */
+  int32_t mode;  /* rece_mode_t */
+  uint32_t flags;
+} rece_config_t;
+
+typedef struct rece_plan_s* rece_plan_t;
+
+/* Byte offsets of the intermediate arrays inside the workspace (valid between
+ * rece_bucketize_sort and the next rece_loss_bwd on that workspace).  The status word
+ * is always at offset 0. */
+typedef struct {
+  size_t status;   /* uint32 device status word */
+  size_t bucket_x; /* int32 [n_r][N]: bucket id of every row of X, per round */
+  size_t bucket_y; /* int32 [n_r][C] */
+  size_t perm_x;   /* int32 [n_r][N]: row ids in stable bucket order, per round */
+  size_t perm_y;   /* int32 [n_r][C] */
+  size_t bucket_start_y; /* int32 [n_r][bucket_start_stride]: first sorted position of
+                            each bucket id b (entries b >= n_b hold C) */
+  size_t bucket_start_stride; /* elements per round: 2^ceil(log2 n_b) + 1 */
+} rece_workspace_layout_t;
+
+/* Validate cfg and build a host-side plan (no CUDA call, no device memory).
+ * cfg, plan: host pointers.  On success *plan owns a host object freed by
+ * rece_plan_destroy.  RECE_ERR_INVALID_ARG / RECE_ERR_UNSUPPORTED on a bad config. */
+RECE_API rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* plan);
+RECE_API void rece_plan_destroy(rece_plan_t plan);
+
+/* Device workspace bytes the plan needs (one buffer, caller-allocated, 256-byte
+ * aligned).  The same buffer serves rece_bucketize_sort, rece_loss_fwd and
+ * rece_loss_bwd; rece_loss_bwd reuses the space the forward intermediates held. */
+RECE_API rece_status_t rece_plan_workspace_size(rece_plan_t plan, size_t* bytes);
+RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspace_layout_t* layout);
+
+/* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].
+ *   B  device, [n_r][n_b][d] random vectors (one set per round; the caller draws them,
+ *      N(0,1), afresh for every call as the paper does)
+ *   X  device, [N][d];  Y device, [C][d]
+ * Writes bucket ids and stable per-round orders into the workspace, and clears the
+ * status word.  Must precede rece_loss_fwd on the same workspace and stream. */
+RECE_API rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X,
+                                  const void* Y, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Steps 3-5 [RECE Algorithm 1: chunks, windows, logits, loss; SCE abstract: top-k].
+ *   targets  device int32 [N], positive item of every row, in [0, C)
+ *   loss     device fp32 [1]: mean over rows of the per-row loss (0 when N = 0)
+ *   row_loss device fp32 [N] or NULL
+ *   selected device int32 [N][k]: the kept negatives, best first (score descending,
+ *            item id ascending), -1 where a row has fewer than k candidates
+ *   lse      device fp32 [N]: log(exp(l+) + sum over selected exp(l)) per row
+ * selected and lse are what rece_loss_bwd needs. */
+RECE_API rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
+                            const int32_t* targets, void* workspace, size_t workspace_bytes,
+                            float* loss, float* row_loss, int32_t* selected, float* lse,
+                            void* stream);
+
+/* Step 6 [RECE equation (4) on the positive and the kept negatives]:
+ *   g_ij = (exp(l_ij - lse_i) - [j == z_i]) * dloss / N
+ *   dX_i = sum_j g_ij y_j,   dY_j = sum_i g_ij x_i
+ *   dloss  device fp32 [1]: gradient of the caller's objective w.r.t. the mean loss
+ *   dX     device fp32 [N][d], dY device fp32 [C][d]: overwritten (items no row touched
+ *          get exactly 0).  Deterministic: no floating-point atomics. */
+RECE_API rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
+                            const int32_t* targets, const int32_t* selected,
+                            const float* lse, const float* dloss, void* workspace,
+                            size_t workspace_bytes, float* dX, float* dY, void* stream);
+
+/* Exact full cross-entropy [RECE equations (3) and (4)], fused: the logits are formed
+ * tile by tile on chip and never stored.  Arguments as above; mode picks the input
+ * element type.  The workspace (rece_full_ce_workspace_size bytes) holds the status
+ * word. */
+RECE_API rece_status_t rece_full_ce_workspace_size(int64_t N, int64_t C, int32_t d, int32_t mode,
+                                          size_t* bytes);
+RECE_API rece_status_t rece_full_ce_fwd(int64_t N, int64_t C, int32_t d, int32_t mode, const void* X,
+                               const void* Y, const int32_t* targets, void* workspace,
+                               size_t workspace_bytes, float* loss, float* row_loss,
+                               float* lse, void* stream);
+RECE_API rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t mode, const void* X,
+                               const void* Y, const int32_t* targets, const float* lse,
+                               const float* dloss, void* workspace, size_t workspace_bytes,
+                               float* dX, float* dY, void* stream);
+
+/* Synchronises `stream`, then copies the workspace's status word to *device_flags
+ * (RECE_DEVICE_* bits).  Returns RECE_ERR_DEVICE_INPUT / RECE_ERR_TIMEOUT when a bit is
+ * set, RECE_ERR_CUDA when the stream reports an error. */
+RECE_API rece_status_t rece_get_device_status(const void* workspace, uint32_t* device_flags,
+                                     void* stream);
+
+/* Stages of the path that rece_plan_set_stage_events can time. */
+#define RECE_STAGE_BUCKETIZE 0  /* step 1: projection + argmax, X and Y, all rounds */
+#define RECE_STAGE_SORT 1       /* step 2: stable bucket sorts, all rounds */
+#define RECE_STAGE_SELECT 2     /* steps 3-4: chunk scores + per-round top-k */
+#define RECE_STAGE_MERGE_LOSS 3 /* steps 4-5: round merge, de-duplication, row losses */
+#define RECE_STAGE_MEAN 4       /* step 5: mean over rows */
+#define RECE_STAGE_BWD_ROWS 5   /* step 6: coefficients and dX, one row at a time */
+#define RECE_STAGE_BWD_SORT 6   /* step 6: (item, row) pairs put in item order */
+#define RECE_STAGE_BWD_ITEMS 7  /* step 6: dY, one item at a time */
+#define RECE_NUM_STAGES 8
+
+/* Optional timing hook: events points to 2 * RECE_NUM_STAGES cudaEvent_t handles (as
+ * void*) owned by the caller; each later call records events[2s] on its stream just
+ * before stage s and events[2s+1] just after it.  NULL switches the hook off.  The
+ * handles must outlive their use; the plan does not own them. */
+RECE_API rece_status_t rece_plan_set_stage_events(rece_plan_t plan, void* const* events);
+
+/* Number of CUDA kernels this library has launched in the process so far (all plans,
+ * all threads); lets a caller count the kernels in a timed region. */
+RECE_API uint64_t rece_kernel_launch_count(void);
+
+/* Static, human-readable name of a status code. */
+RECE_API const char* rece_status_string(rece_status_t status);
+
+/* Detail of the last error returned on the calling thread (a CUDA error name and the
+ * failing step, or the argument that was rejected).  Thread-local, never NULL. */
+RECE_API const char* rece_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RECE_H_ */

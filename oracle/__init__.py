@@ -41,8 +41,9 @@ def _load():
         lib.oracle_stable_argsort.restype = None
         lib.oracle_chunk_start.argtypes = [i64, i64, i64]
         lib.oracle_chunk_start.restype = i64
+        i64p_or_null = ctypes.c_void_p
         lib.oracle_select.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32, i32,
-                                      i32p, i32p, i32p, f32p, i64p]
+                                      i32p, i32p, i64p_or_null, i64, i32p, f32p, i64p]
         lib.oracle_select.restype = None
         lib.oracle_rece_loss.argtypes = [f32p, f32p, i32p, i64, i32, i32, i32p, f64p, f64p,
                                          f64p]
@@ -100,21 +101,26 @@ def chunk_start(c: int, M: int, n_c: int) -> int:
     return int(_load().oracle_chunk_start(c, M, n_c))
 
 
-def select(X, Y, target, permX, permY, n_c, n_ec, k):
-    """Top-k negatives of every row over all rounds' chunk windows.
+def select(X, Y, target, permX, permY, n_c, n_ec, k, rows=None):
+    """Top-k negatives of every row (or of `rows` only) over all rounds' chunk windows.
 
-    permX: [n_r, N], permY: [n_r, C].  Returns (selected [N,k] int32 -1 padded,
-    sel_score [N,k] fp32, n_cand [N] int64)."""
+    permX: [n_r, N], permY: [n_r, C].  Returns (selected [R,k] int32 -1 padded,
+    sel_score [R,k] fp32, n_cand [R] int64) for the R requested rows."""
     X, Y, target = _f32(X), _f32(Y), _i32(target)
     permX, permY = _i32(permX), _i32(permY)
     N, d = X.shape
     C = Y.shape[0]
     n_r = permX.shape[0]
-    sel = np.empty((N, k), np.int32)
-    score = np.empty((N, k), np.float32)
-    n_cand = np.empty(N, np.int64)
-    _load().oracle_select(X, Y, target, N, C, d, n_c, n_ec, n_r, k, permX, permY, sel, score,
-                          n_cand)
+    if rows is None:
+        R, rows_p = N, None
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        R, rows_p = rows.shape[0], rows.ctypes.data_as(ctypes.c_void_p)
+    sel = np.empty((R, k), np.int32)
+    score = np.empty((R, k), np.float32)
+    n_cand = np.empty(R, np.int64)
+    _load().oracle_select(X, Y, target, N, C, d, n_c, n_ec, n_r, k, permX, permY, rows_p, R,
+                          sel, score, n_cand)
     return sel, score, n_cand
 
 

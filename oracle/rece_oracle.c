@@ -144,13 +144,14 @@ static int64_t chunk_of(int64_t pos, int64_t M, int64_t n_c) {
 /* Steps 3-4: for every row, the candidate negatives from all rounds (window items of
  * the row's chunk, positive removed, de-duplicated) and the k best of them.
  *   permX [n_r*N], permY [n_r*C]  : per-round stable bucket orders (from above)
- *   selected [N*k]               : item ids, best first, -1 padded
- *   sel_score [N*k]              : their fp32 scores (-inf for padding)
- *   n_cand [N]                   : number of distinct candidates of each row */
+ *   rows [n_rows]                : the rows to compute (NULL: all N rows, n_rows = N)
+ *   selected [n_rows*k]          : item ids, best first, -1 padded
+ *   sel_score [n_rows*k]         : their fp32 scores (-inf for padding)
+ *   n_cand [n_rows]              : number of distinct candidates of each row */
 void oracle_select(const float* X, const float* Y, const int32_t* target, int64_t N, int64_t C,
                    int32_t d, int32_t n_c, int32_t n_ec, int32_t n_r, int32_t k,
-                   const int32_t* permX, const int32_t* permY, int32_t* selected,
-                   float* sel_score, int64_t* n_cand) {
+                   const int32_t* permX, const int32_t* permY, const int64_t* rows,
+                   int64_t n_rows, int32_t* selected, float* sel_score, int64_t* n_cand) {
   /* position of each row in each round's sorted order */
   int64_t* posX = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N * n_r > 0 ? N * n_r : 1));
   for (int32_t r = 0; r < n_r; ++r)
@@ -161,7 +162,8 @@ void oracle_select(const float* X, const float* Y, const int32_t* target, int64_
     unsigned char* seen = (unsigned char*)calloc((size_t)C, 1);
     cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)C);
 #pragma omp for schedule(dynamic, 16)
-    for (int64_t i = 0; i < N; ++i) {
+    for (int64_t o = 0; o < n_rows; ++o) {
+      const int64_t i = rows ? rows[o] : o;
       int64_t n = 0;
       for (int32_t r = 0; r < n_r; ++r) {
         int64_t c = chunk_of(posX[(int64_t)r * N + i], N, n_c);
@@ -184,14 +186,14 @@ void oracle_select(const float* X, const float* Y, const int32_t* target, int64_
       qsort(cand, (size_t)n, sizeof(cand_t), cmp_cand);
       for (int32_t a = 0; a < k; ++a) {
         if (a < n) {
-          selected[i * (int64_t)k + a] = cand[a].item;
-          sel_score[i * (int64_t)k + a] = cand[a].score;
+          selected[o * (int64_t)k + a] = cand[a].item;
+          sel_score[o * (int64_t)k + a] = cand[a].score;
         } else {
-          selected[i * (int64_t)k + a] = -1;
-          sel_score[i * (int64_t)k + a] = -INFINITY;
+          selected[o * (int64_t)k + a] = -1;
+          sel_score[o * (int64_t)k + a] = -INFINITY;
         }
       }
-      n_cand[i] = n;
+      n_cand[o] = n;
     }
     free(cand);
     free(seen);

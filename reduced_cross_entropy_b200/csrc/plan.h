@@ -1,0 +1,122 @@
+// plan.h -- host-side plan of the RECE library and the internal kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "rece.h"
+
+namespace rece {
+
+// Counting-sort geometry: one CTA sorts a tile of kSortTile elements (8 warps x 512).
+constexpr int kSortTile = 4096;
+constexpr int kSortThreads = 256;
+constexpr int kMaxDigitBits = 12;  // up to 4096 buckets in one pass
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int bits_for(int64_t n_values) {  // digit bits so that values 0..n_values-1 fit
+  int b = 0;
+  while ((int64_t(1) << b) < n_values) ++b;
+  return b;
+}
+
+// Scratch of one counting sort pass over M elements with `bits`-bit digits.
+inline size_t sort_scratch_bytes(int64_t M, int bits) {
+  int64_t tiles = ceil_div(M > 0 ? M : 1, kSortTile);
+  int64_t digits = int64_t(1) << bits;
+  return align256(sizeof(int32_t) * size_t(digits * tiles)) +
+         align256(sizeof(int32_t) * size_t(digits + 1));
+}
+
+struct Layout {
+  size_t status = 0;
+  // forward region (from rece_bucketize_sort to the end of rece_loss_fwd)
+  size_t bx = 0, by = 0, px = 0, py = 0, bstart_y = 0, bstart_x = 0;
+  size_t sort_scratch = 0;
+  size_t list_score = 0, list_item = 0, row_loss_tmp = 0;
+  size_t fwd_end = 0;
+  // backward region (rece_loss_bwd), overlaps the forward region
+  size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_scratch = 0;
+  size_t bwd_end = 0;
+  size_t total = 0;
+};
+
+}  // namespace rece
+
+struct rece_plan_s {
+  rece_config_t cfg;
+  int64_t x_chunk_max;  // ceil(N / n_c)
+  int64_t y_chunk_max;  // ceil(C / n_c)
+  int64_t w_max;        // longest window (items)
+  int32_t sel_rows;     // rows per CTA of the exact selection kernel
+  int32_t bucket_bits;  // digit bits of the bucket sort
+  int32_t item_bits;    // key bits of the backward item sort (values 0..C)
+  int64_t entries;      // N * (k + 1): (row, item) pairs of the backward
+  rece::Layout lay;
+  void* stage_events[2 * RECE_NUM_STAGES];  // optional timing hook (cudaEvent_t)
+  bool timed;
+};
+
+namespace rece {
+
+// Process-wide count of kernel launches (statistics only).
+void count_launches(int n);
+
+// Records the stage's start (end = 0) or end (end = 1) event when timing is on.
+inline void stage_mark(const rece_plan_s& p, int stage, int end, cudaStream_t st) {
+  if (p.timed) cudaEventRecord(static_cast<cudaEvent_t>(p.stage_events[2 * stage + end]), st);
+}
+
+// ---------------------------------------------------------------- launchers
+// All launchers enqueue on `st` and return the launch error (cudaSuccess if none).
+
+// K1: bucket[r][i] = argmax_b <B[r][b], V[i]> (fmaf chain, ties to lowest b).
+template <typename T>
+cudaError_t launch_bucketize_fma(const T* V, int64_t M, int d, const T* B, int n_b, int n_r,
+                                 int32_t* bucket, cudaStream_t st);
+
+// K2: one stable counting-sort pass over M elements.  Element p carries id
+// (in_ids ? in_ids[p] : p) and key keys[id]; it is ordered by digit (key >> shift) &
+// ((1 << bits) - 1).  Writes out_ids (the new order of ids), optionally the sorted
+// digit-keys (out_keys[p] = keys[out_ids[p]]) and digit_start[0..2^bits] (first output
+// position of every digit; digit_start[2^bits] = M).
+cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,
+                             int bits, void* scratch, int32_t* out_ids, int32_t* out_keys,
+                             int32_t* digit_start, cudaStream_t st);
+
+// K3 (fmaf-chain CUDA-core version): per-round top-k lists of every row.
+template <typename T>
+cudaError_t launch_select_fma(const rece_plan_s& p, const T* X, const T* Y,
+                              const int32_t* targets, const int32_t* px, const int32_t* py,
+                              float* list_score, int32_t* list_item, cudaStream_t st);
+
+// K4: merge the rounds' lists, de-duplicate, keep k, loss per row.
+template <typename T>
+cudaError_t launch_merge_loss(const rece_plan_s& p, const T* X, const T* Y,
+                              const int32_t* targets, const float* list_score,
+                              const int32_t* list_item, int32_t* selected, float* lse,
+                              float* row_loss, uint32_t* status, cudaStream_t st);
+
+// K7: loss[0] = sum(row_loss) / N in a fixed order.
+cudaError_t launch_mean(const float* row_loss, int64_t N, float* loss, cudaStream_t st);
+
+// K5: backward.
+template <typename T>
+cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
+                            const int32_t* targets, const int32_t* selected, const float* lse,
+                            const float* dloss, char* ws, float* dX, float* dY,
+                            uint32_t* status, cudaStream_t st);
+
+// K6: exact full cross-entropy.
+template <typename T>
+cudaError_t launch_full_ce_fwd(int64_t N, int64_t C, int d, const T* X, const T* Y,
+                               const int32_t* targets, float* row_loss, float* lse,
+                               uint32_t* status, cudaStream_t st);
+template <typename T>
+cudaError_t launch_full_ce_bwd(int64_t N, int64_t C, int d, const T* X, const T* Y,
+                               const int32_t* targets, const float* lse, const float* dloss,
+                               float* dX, float* dY, cudaStream_t st);
+
+}  // namespace rece

@@ -1,0 +1,391 @@
+// rece_abi.cu -- the C ABI declared in include/rece.h: plan validation, workspace
+// layout and the launch sequence of every entry point.  No device memory is allocated
+// here: every device buffer, the workspace included, belongs to the caller.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace rece {
+size_t select_fma_smem_bytes(int G, int d, int64_t w_max);
+int merge_pow2(int n_r, int k);
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+}  // namespace rece
+
+using namespace rece;
+
+namespace {
+
+constexpr size_t kMaxSmem = 227 * 1024;
+constexpr int64_t kInt32Max = 2147483647;
+
+thread_local char g_last_error[256] = "";
+
+rece_status_t fail(rece_status_t s, const char* msg) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+  return s;
+}
+
+rece_status_t cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return RECE_ERR_CUDA;
+}
+
+#define RECE_CUDA(call, where)                   \
+  do {                                           \
+    cudaError_t e_ = (call);                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+int64_t window_len(int64_t c, int64_t C, int64_t n_c, int64_t n_ec) {
+  const int64_t lo = c - n_ec < 0 ? 0 : c - n_ec;
+  const int64_t hi = c + n_ec + 1 > n_c ? n_c : c + n_ec + 1;
+  return chunk_start(hi, C, n_c) - chunk_start(lo, C, n_c);
+}
+
+void build_layout(rece_plan_s& p) {
+  const auto& c = p.cfg;
+  Layout& L = p.lay;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.status = take(sizeof(uint32_t));
+  const size_t region = off;
+  const size_t nb_stride = (size_t(1) << p.bucket_bits) + 1;
+  L.bx = take(sizeof(int32_t) * c.n_r * c.N);
+  L.by = take(sizeof(int32_t) * c.n_r * c.C);
+  L.px = take(sizeof(int32_t) * c.n_r * c.N);
+  L.py = take(sizeof(int32_t) * c.n_r * c.C);
+  L.bstart_x = take(sizeof(int32_t) * c.n_r * nb_stride);
+  L.bstart_y = take(sizeof(int32_t) * c.n_r * nb_stride);
+  L.sort_scratch = take(sort_scratch_bytes(c.N > c.C ? c.N : c.C, p.bucket_bits));
+  L.list_score = take(sizeof(float) * size_t(c.n_r) * c.N * c.k);
+  L.list_item = take(sizeof(int32_t) * size_t(c.n_r) * c.N * c.k);
+  L.row_loss_tmp = take(sizeof(float) * c.N);
+  L.fwd_end = off;
+  off = region;
+  const size_t E = size_t(p.entries);
+  L.e_key = take(sizeof(int32_t) * E);
+  L.e_g = take(sizeof(float) * E);
+  L.e_perm_a = take(sizeof(int32_t) * E);
+  L.e_perm_b = take(sizeof(int32_t) * E);
+  L.e_sorted_key = take(sizeof(int32_t) * E);
+  L.e_scratch = take(sort_scratch_bytes(p.entries, 8));
+  L.bwd_end = off;
+  L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
+}
+
+rece_status_t check_plan_ws(rece_plan_t plan, const void* ws, size_t ws_bytes) {
+  if (!plan) return fail(RECE_ERR_INVALID_ARG, "plan is NULL");
+  if (!ws) return fail(RECE_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(RECE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (ws_bytes < plan->lay.total) return fail(RECE_ERR_WORKSPACE, "workspace too small");
+  return RECE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rece_status_string(rece_status_t s) {
+  switch (s) {
+    case RECE_OK: return "RECE_OK";
+    case RECE_ERR_INVALID_ARG: return "RECE_ERR_INVALID_ARG";
+    case RECE_ERR_UNSUPPORTED: return "RECE_ERR_UNSUPPORTED";
+    case RECE_ERR_WORKSPACE: return "RECE_ERR_WORKSPACE";
+    case RECE_ERR_CUDA: return "RECE_ERR_CUDA";
+    case RECE_ERR_DEVICE_INPUT: return "RECE_ERR_DEVICE_INPUT";
+    case RECE_ERR_TIMEOUT: return "RECE_ERR_TIMEOUT";
+    case RECE_ERR_NO_DEVICE: return "RECE_ERR_NO_DEVICE";
+  }
+  return "RECE_ERR_UNKNOWN";
+}
+
+const char* rece_last_error_string(void) { return g_last_error; }
+
+rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
+  if (!cfg || !out) return fail(RECE_ERR_INVALID_ARG, "cfg or plan pointer is NULL");
+  *out = nullptr;
+  const rece_config_t& c = *cfg;
+  if (c.N < 0 || c.C < 1 || c.C >= kInt32Max) return fail(RECE_ERR_INVALID_ARG, "N or C out of range");
+  if (c.d < 1) return fail(RECE_ERR_INVALID_ARG, "d must be >= 1");
+  if (c.n_b < 1 || c.n_b > (1 << kMaxDigitBits))
+    return fail(RECE_ERR_INVALID_ARG, "n_b must be in [1, 4096]");
+  if (c.n_r < 1 || c.n_r > 8) return fail(RECE_ERR_INVALID_ARG, "n_r must be in [1, 8]");
+  if (c.k < 1 || c.k > 4096) return fail(RECE_ERR_INVALID_ARG, "k must be in [1, 4096]");
+  if (c.n_ec < 0) return fail(RECE_ERR_INVALID_ARG, "n_ec must be >= 0");
+  if (c.n_c < 1 || c.n_c > c.C || (c.N > 0 && c.n_c > c.N))
+    return fail(RECE_ERR_INVALID_ARG, "n_c must be in [1, min(N, C)]");
+  if (c.mode != RECE_MODE_FP32_EXACT && c.mode != RECE_MODE_BF16)
+    return fail(RECE_ERR_INVALID_ARG, "unknown mode");
+  if ((c.flags & ~RECE_FLAG_FMA_SCORES) != 0) return fail(RECE_ERR_INVALID_ARG, "unknown flag");
+  if (c.N * (int64_t(c.k) + 1) >= kInt32Max || c.N * c.n_r >= kInt32Max ||
+      c.C * c.n_r >= kInt32Max || c.N * c.d >= (int64_t(1) << 40))
+    return fail(RECE_ERR_UNSUPPORTED, "sizes exceed 32-bit pair indexing");
+  if (int64_t(c.n_r) * c.k > 8192) return fail(RECE_ERR_UNSUPPORTED, "n_r * k must be <= 8192");
+
+  rece_plan_s* p = new (std::nothrow) rece_plan_s();
+  if (!p) return fail(RECE_ERR_INVALID_ARG, "out of host memory");
+  p->cfg = c;
+  p->x_chunk_max = c.N > 0 ? ceil_div(c.N, c.n_c) : 0;
+  p->y_chunk_max = ceil_div(c.C, c.n_c);
+  p->w_max = 0;
+  for (int64_t ch = 0; ch < c.n_c; ++ch) {
+    const int64_t w = window_len(ch, c.C, c.n_c, c.n_ec);
+    if (w > p->w_max) p->w_max = w;
+  }
+  p->sel_rows = 0;
+  for (int G = 8; G >= 1; G >>= 1) {
+    if (select_fma_smem_bytes(G, c.d, p->w_max) <= kMaxSmem) {
+      p->sel_rows = G;
+      break;
+    }
+  }
+  if (p->sel_rows == 0) {
+    delete p;
+    return fail(RECE_ERR_UNSUPPORTED, "chunk window too long for the selection kernel");
+  }
+  p->bucket_bits = bits_for(c.n_b);
+  p->item_bits = bits_for(c.C + 1);
+  p->entries = c.N * (int64_t(c.k) + 1);
+  p->timed = false;
+  for (void*& e : p->stage_events) e = nullptr;
+  build_layout(*p);
+  *out = p;
+  return RECE_OK;
+}
+
+void rece_plan_destroy(rece_plan_t plan) { delete plan; }
+
+rece_status_t rece_plan_set_stage_events(rece_plan_t plan, void* const* events) {
+  if (!plan) return fail(RECE_ERR_INVALID_ARG, "plan is NULL");
+  plan->timed = events != nullptr;
+  for (int i = 0; i < 2 * RECE_NUM_STAGES; ++i) {
+    plan->stage_events[i] = events ? events[i] : nullptr;
+    if (events && !events[i]) {
+      plan->timed = false;
+      return fail(RECE_ERR_INVALID_ARG, "NULL event handle");
+    }
+  }
+  return RECE_OK;
+}
+
+uint64_t rece_kernel_launch_count(void) { return g_launches.load(); }
+
+rece_status_t rece_plan_workspace_size(rece_plan_t plan, size_t* bytes) {
+  if (!plan || !bytes) return fail(RECE_ERR_INVALID_ARG, "NULL argument");
+  *bytes = plan->lay.total;
+  return RECE_OK;
+}
+
+rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspace_layout_t* l) {
+  if (!plan || !l) return fail(RECE_ERR_INVALID_ARG, "NULL argument");
+  l->status = plan->lay.status;
+  l->bucket_x = plan->lay.bx;
+  l->bucket_y = plan->lay.by;
+  l->perm_x = plan->lay.px;
+  l->perm_y = plan->lay.py;
+  l->bucket_start_y = plan->lay.bstart_y;
+  l->bucket_start_stride = (size_t(1) << plan->bucket_bits) + 1;
+  return RECE_OK;
+}
+
+rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X, const void* Y,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
+  if (s != RECE_OK) return s;
+  const auto& c = plan->cfg;
+  if (!B || !Y || (c.N > 0 && !X)) return fail(RECE_ERR_INVALID_ARG, "NULL input");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const Layout& L = plan->lay;
+  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, sizeof(uint32_t), st), "status reset");
+  int32_t* bx = reinterpret_cast<int32_t*>(ws + L.bx);
+  int32_t* by = reinterpret_cast<int32_t*>(ws + L.by);
+  stage_mark(*plan, RECE_STAGE_BUCKETIZE, 0, st);
+  if (c.mode == RECE_MODE_FP32_EXACT) {
+    RECE_CUDA(launch_bucketize_fma(static_cast<const float*>(X), c.N, c.d,
+                                   static_cast<const float*>(B), c.n_b, c.n_r, bx, st),
+              "bucketize X");
+    RECE_CUDA(launch_bucketize_fma(static_cast<const float*>(Y), c.C, c.d,
+                                   static_cast<const float*>(B), c.n_b, c.n_r, by, st),
+              "bucketize Y");
+  } else {
+    RECE_CUDA(launch_bucketize_fma(static_cast<const __nv_bfloat16*>(X), c.N, c.d,
+                                   static_cast<const __nv_bfloat16*>(B), c.n_b, c.n_r, bx, st),
+              "bucketize X");
+    RECE_CUDA(launch_bucketize_fma(static_cast<const __nv_bfloat16*>(Y), c.C, c.d,
+                                   static_cast<const __nv_bfloat16*>(B), c.n_b, c.n_r, by, st),
+              "bucketize Y");
+  }
+  stage_mark(*plan, RECE_STAGE_BUCKETIZE, 1, st);
+  stage_mark(*plan, RECE_STAGE_SORT, 0, st);
+  const size_t stride = (size_t(1) << plan->bucket_bits) + 1;
+  for (int r = 0; r < c.n_r; ++r) {
+    RECE_CUDA(launch_sort_pass(bx + int64_t(r) * c.N, nullptr, c.N, 0, plan->bucket_bits,
+                               ws + L.sort_scratch,
+                               reinterpret_cast<int32_t*>(ws + L.px) + int64_t(r) * c.N, nullptr,
+                               reinterpret_cast<int32_t*>(ws + L.bstart_x) + r * stride, st),
+              "sort X");
+    RECE_CUDA(launch_sort_pass(by + int64_t(r) * c.C, nullptr, c.C, 0, plan->bucket_bits,
+                               ws + L.sort_scratch,
+                               reinterpret_cast<int32_t*>(ws + L.py) + int64_t(r) * c.C, nullptr,
+                               reinterpret_cast<int32_t*>(ws + L.bstart_y) + r * stride, st),
+              "sort Y");
+  }
+  stage_mark(*plan, RECE_STAGE_SORT, 1, st);
+  return RECE_OK;
+}
+
+rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
+                            const int32_t* targets, void* workspace, size_t workspace_bytes,
+                            float* loss, float* row_loss, int32_t* selected, float* lse,
+                            void* stream) {
+  rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
+  if (s != RECE_OK) return s;
+  const auto& c = plan->cfg;
+  if (!loss || !Y || (c.N > 0 && (!X || !targets || !selected || !lse)))
+    return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const Layout& L = plan->lay;
+  const int32_t* px = reinterpret_cast<const int32_t*>(ws + L.px);
+  const int32_t* py = reinterpret_cast<const int32_t*>(ws + L.py);
+  float* ls = reinterpret_cast<float*>(ws + L.list_score);
+  int32_t* li = reinterpret_cast<int32_t*>(ws + L.list_item);
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + L.row_loss_tmp);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  if (c.mode == RECE_MODE_FP32_EXACT) {
+    const float* Xf = static_cast<const float*>(X);
+    const float* Yf = static_cast<const float*>(Y);
+    stage_mark(*plan, RECE_STAGE_SELECT, 0, st);
+    RECE_CUDA(launch_select_fma(*plan, Xf, Yf, targets, px, py, ls, li, st), "select");
+    stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
+    stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
+    RECE_CUDA(launch_merge_loss(*plan, Xf, Yf, targets, ls, li, selected, lse, rl, status, st),
+              "merge/loss");
+  } else {
+    const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+    const __nv_bfloat16* Yb = static_cast<const __nv_bfloat16*>(Y);
+    stage_mark(*plan, RECE_STAGE_SELECT, 0, st);
+    RECE_CUDA(launch_select_fma(*plan, Xb, Yb, targets, px, py, ls, li, st), "select");
+    stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
+    stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
+    RECE_CUDA(launch_merge_loss(*plan, Xb, Yb, targets, ls, li, selected, lse, rl, status, st),
+              "merge/loss");
+  }
+  stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 1, st);
+  stage_mark(*plan, RECE_STAGE_MEAN, 0, st);
+  RECE_CUDA(launch_mean(rl, c.N, loss, st), "mean");
+  stage_mark(*plan, RECE_STAGE_MEAN, 1, st);
+  return RECE_OK;
+}
+
+rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
+                            const int32_t* targets, const int32_t* selected, const float* lse,
+                            const float* dloss, void* workspace, size_t workspace_bytes,
+                            float* dX, float* dY, void* stream) {
+  rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
+  if (s != RECE_OK) return s;
+  const auto& c = plan->cfg;
+  if (!Y || !dY || (c.N > 0 && (!X || !targets || !selected || !lse || !dloss || !dX)))
+    return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan->lay.status);
+  if (c.mode == RECE_MODE_FP32_EXACT)
+    RECE_CUDA(launch_backward(*plan, static_cast<const float*>(X), static_cast<const float*>(Y),
+                              targets, selected, lse, dloss, ws, dX, dY, status, st),
+              "backward");
+  else
+    RECE_CUDA(launch_backward(*plan, static_cast<const __nv_bfloat16*>(X),
+                              static_cast<const __nv_bfloat16*>(Y), targets, selected, lse,
+                              dloss, ws, dX, dY, status, st),
+              "backward");
+  return RECE_OK;
+}
+
+rece_status_t rece_full_ce_workspace_size(int64_t N, int64_t C, int32_t d, int32_t mode,
+                                          size_t* bytes) {
+  if (!bytes || N < 0 || C < 1 || d < 1 || (mode != RECE_MODE_FP32_EXACT && mode != RECE_MODE_BF16))
+    return fail(RECE_ERR_INVALID_ARG, "bad full-CE arguments");
+  *bytes = align256(sizeof(uint32_t)) + align256(sizeof(float) * size_t(N));
+  return RECE_OK;
+}
+
+rece_status_t rece_full_ce_fwd(int64_t N, int64_t C, int32_t d, int32_t mode, const void* X,
+                               const void* Y, const int32_t* targets, void* workspace,
+                               size_t workspace_bytes, float* loss, float* row_loss, float* lse,
+                               void* stream) {
+  size_t need = 0;
+  rece_status_t s = rece_full_ce_workspace_size(N, C, d, mode, &need);
+  if (s != RECE_OK) return s;
+  if (!workspace || workspace_bytes < need) return fail(RECE_ERR_WORKSPACE, "workspace too small");
+  if (!loss || !Y || (N > 0 && (!X || !targets || !lse)))
+    return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + align256(sizeof(uint32_t)));
+  RECE_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), st), "status reset");
+  if (mode == RECE_MODE_FP32_EXACT)
+    RECE_CUDA(launch_full_ce_fwd(N, C, d, static_cast<const float*>(X),
+                                 static_cast<const float*>(Y), targets, rl, lse, status, st),
+              "full CE forward");
+  else
+    RECE_CUDA(launch_full_ce_fwd(N, C, d, static_cast<const __nv_bfloat16*>(X),
+                                 static_cast<const __nv_bfloat16*>(Y), targets, rl, lse, status,
+                                 st),
+              "full CE forward");
+  RECE_CUDA(launch_mean(rl, N, loss, st), "mean");
+  return RECE_OK;
+}
+
+rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t mode, const void* X,
+                               const void* Y, const int32_t* targets, const float* lse,
+                               const float* dloss, void* workspace, size_t workspace_bytes,
+                               float* dX, float* dY, void* stream) {
+  size_t need = 0;
+  rece_status_t s = rece_full_ce_workspace_size(N, C, d, mode, &need);
+  if (s != RECE_OK) return s;
+  if (!workspace || workspace_bytes < need) return fail(RECE_ERR_WORKSPACE, "workspace too small");
+  if (!Y || !dY || (N > 0 && (!X || !targets || !lse || !dloss || !dX)))
+    return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mode == RECE_MODE_FP32_EXACT)
+    RECE_CUDA(launch_full_ce_bwd(N, C, d, static_cast<const float*>(X),
+                                 static_cast<const float*>(Y), targets, lse, dloss, dX, dY, st),
+              "full CE backward");
+  else
+    RECE_CUDA(launch_full_ce_bwd(N, C, d, static_cast<const __nv_bfloat16*>(X),
+                                 static_cast<const __nv_bfloat16*>(Y), targets, lse, dloss, dX,
+                                 dY, st),
+              "full CE backward");
+  return RECE_OK;
+}
+
+rece_status_t rece_get_device_status(const void* workspace, uint32_t* device_flags,
+                                     void* stream) {
+  if (!workspace || !device_flags) return fail(RECE_ERR_INVALID_ARG, "NULL argument");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RECE_CUDA(cudaStreamSynchronize(st), "stream synchronize");
+  RECE_CUDA(cudaMemcpy(device_flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost),
+            "status read");
+  if (*device_flags & RECE_DEVICE_TIMEOUT) return fail(RECE_ERR_TIMEOUT, "device wait timed out");
+  if (*device_flags) return fail(RECE_ERR_DEVICE_INPUT, "device input error");
+  return RECE_OK;
+}
+
+}  // extern "C"

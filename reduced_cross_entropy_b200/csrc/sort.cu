@@ -1,0 +1,207 @@
+// sort.cu -- step 2 of the path: stable counting sort by bucket id (RECE, section 3,
+// Algorithm 1: the argsort steps, read as stable), reused with 8-bit digits as the
+// passes of an LSD radix sort of the backward's (item, row) pairs.
+//
+// One pass over M elements with b-bit digits:
+//   hist     per tile of 4096 elements, the count of every digit (digit-major matrix)
+//   scan     exclusive prefix over tiles for every digit, then over digits
+//   scatter  every warp walks its 512 elements in order; __match_any_sync groups the
+//            lanes holding the same digit, so an element's rank is the number of
+//            earlier elements with its digit: in earlier tiles, earlier warps of its
+//            tile, earlier steps of its warp, lower lanes of its step.  Stable.
+#include "common.cuh"
+#include "plan.h"
+
+namespace rece {
+namespace {
+
+constexpr int kWarps = kSortThreads / 32;      // 8
+constexpr int kPerWarp = kSortTile / kWarps;   // 512
+constexpr int kSteps = kPerWarp / 32;          // 16
+
+__device__ __forceinline__ int32_t elem_id(const int32_t* in_ids, int64_t p) {
+  return in_ids ? in_ids[p] : int32_t(p);
+}
+
+__global__ void __launch_bounds__(kSortThreads) k_sort_hist(const int32_t* __restrict__ keys,
+                                                            const int32_t* __restrict__ in_ids,
+                                                            int64_t M, int shift, int bits,
+                                                            int32_t* __restrict__ hist,
+                                                            int64_t tiles) {
+  extern __shared__ int32_t sh_cnt[];
+  const int digits = 1 << bits, mask = digits - 1;
+  for (int i = threadIdx.x; i < digits; i += blockDim.x) sh_cnt[i] = 0;
+  __syncthreads();
+  const int64_t base = int64_t(blockIdx.x) * kSortTile;
+  for (int e = threadIdx.x; e < kSortTile; e += blockDim.x) {
+    const int64_t p = base + e;
+    if (p < M) atomicAdd(&sh_cnt[(keys[elem_id(in_ids, p)] >> shift) & mask], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < digits; i += blockDim.x)
+    hist[int64_t(i) * tiles + blockIdx.x] = sh_cnt[i];
+}
+
+// Exclusive block scan of one value per thread; returns the exclusive prefix and
+// writes the block total to *total (all threads see it after the call).
+__device__ int32_t block_exclusive_scan(int32_t v, int32_t* sh_warp, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sh_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = lane < nw ? sh_warp[lane] : 0;
+    int32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    if (lane < nw) sh_warp[lane] = wi - w;
+    if (lane == nw - 1) *total = wi;
+  }
+  __syncthreads();
+  const int32_t r = sh_warp[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// grid = digits; row d of hist becomes its exclusive prefix over tiles; total -> out[d].
+__global__ void __launch_bounds__(256) k_sort_scan_tiles(int32_t* __restrict__ hist,
+                                                         int64_t tiles,
+                                                         int32_t* __restrict__ out) {
+  __shared__ int32_t sh_warp[32];
+  __shared__ int32_t sh_total;
+  int32_t* row = hist + int64_t(blockIdx.x) * tiles;
+  int32_t carry = 0;
+  for (int64_t c0 = 0; c0 < tiles; c0 += blockDim.x) {
+    const int64_t i = c0 + threadIdx.x;
+    const int32_t v = i < tiles ? row[i] : 0;
+    const int32_t ex = block_exclusive_scan(v, sh_warp, &sh_total);
+    if (i < tiles) row[i] = carry + ex;
+    carry += sh_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[blockIdx.x] = carry;
+}
+
+// One block: start[0..digits) = exclusive prefix of the totals held there; start[digits] = M.
+__global__ void __launch_bounds__(1024) k_sort_scan_digits(int32_t* __restrict__ start,
+                                                           int digits) {
+  __shared__ int32_t sh_warp[32];
+  __shared__ int32_t sh_total;
+  int32_t carry = 0;
+  for (int c0 = 0; c0 < digits; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    const int32_t v = i < digits ? start[i] : 0;
+    const int32_t ex = block_exclusive_scan(v, sh_warp, &sh_total);
+    if (i < digits) start[i] = carry + ex;
+    carry += sh_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) start[digits] = carry;
+}
+
+__global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
+    const int32_t* __restrict__ keys, const int32_t* __restrict__ in_ids, int64_t M, int shift,
+    int bits, const int32_t* __restrict__ hist, int64_t tiles,
+    const int32_t* __restrict__ digit_start, int32_t* __restrict__ out_ids,
+    int32_t* __restrict__ out_keys) {
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  const int digits = 1 << bits, mask = digits - 1;
+  uint16_t* cnt = reinterpret_cast<uint16_t*>(sh_raw);  // [kWarps][digits]
+  int32_t* tile_base =
+      reinterpret_cast<int32_t*>(sh_raw + ((kWarps * digits * sizeof(uint16_t) + 15) & ~15));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t tile = blockIdx.x;
+
+  for (int i = tid; i < kWarps * digits; i += blockDim.x) cnt[i] = 0;
+  for (int i = tid; i < digits; i += blockDim.x)
+    tile_base[i] = digit_start[i] + hist[int64_t(i) * tiles + tile];
+  __syncthreads();
+
+  const int64_t wbase = tile * kSortTile + int64_t(warp) * kPerWarp;
+  uint16_t* wcnt = cnt + warp * digits;
+  // pass 1: this warp's count of every digit
+  for (int s = 0; s < kSteps; ++s) {
+    const int64_t p = wbase + s * 32 + lane;
+    const bool ok = p < M;
+    const int dg = ok ? ((keys[elem_id(in_ids, p)] >> shift) & mask) : (0x40000000 | lane);
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
+    if (ok && lane == __ffs(peers) - 1) wcnt[dg] += uint16_t(__popc(peers));
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive prefix over the warps of the tile, per digit
+  for (int dg = tid; dg < digits; dg += blockDim.x) {
+    uint16_t run = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const uint16_t c = cnt[w * digits + dg];
+      cnt[w * digits + dg] = run;
+      run = uint16_t(run + c);
+    }
+  }
+  __syncthreads();
+  // pass 2: scatter in order
+  for (int s = 0; s < kSteps; ++s) {
+    const int64_t p = wbase + s * 32 + lane;
+    const bool ok = p < M;
+    int32_t id = 0, key = 0;
+    if (ok) {
+      id = elem_id(in_ids, p);
+      key = keys[id];
+    }
+    const int dg = ok ? ((key >> shift) & mask) : (0x40000000 | lane);
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
+    const int base = ok ? int(wcnt[dg]) : 0;
+    __syncwarp();
+    if (ok) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int64_t pos = int64_t(tile_base[dg]) + base + rank;
+      out_ids[pos] = id;
+      if (out_keys) out_keys[pos] = key;
+      if (lane == __ffs(peers) - 1) wcnt[dg] = uint16_t(base + __popc(peers));
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,
+                             int bits, void* scratch, int32_t* out_ids, int32_t* out_keys,
+                             int32_t* digit_start, cudaStream_t st) {
+  const int digits = 1 << bits;
+  const int64_t tiles = ceil_div(M > 0 ? M : 1, kSortTile);
+  int32_t* hist = static_cast<int32_t*>(scratch);
+  int32_t* start = digit_start
+                       ? digit_start
+                       : reinterpret_cast<int32_t*>(static_cast<char*>(scratch) +
+                                                    align256(sizeof(int32_t) * size_t(digits * tiles)));
+  if (M == 0) {
+    if (digit_start) return cudaMemsetAsync(digit_start, 0, sizeof(int32_t) * (digits + 1), st);
+    return cudaSuccess;
+  }
+  k_sort_hist<<<unsigned(tiles), kSortThreads, sizeof(int32_t) * digits, st>>>(
+      keys, in_ids, M, shift, bits, hist, tiles);
+  k_sort_scan_tiles<<<digits, 256, 0, st>>>(hist, tiles, start);
+  k_sort_scan_digits<<<1, 1024, 0, st>>>(start, digits);
+  const size_t smem = ((kWarps * digits * sizeof(uint16_t) + 15) & ~size_t(15)) +
+                      sizeof(int32_t) * digits;
+  // Opt in to the largest dynamic shared memory the scatter can use (per device; cheap).
+  cudaError_t e = cudaFuncSetAttribute(
+      k_sort_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      int(sizeof(uint16_t) * kWarps * (1 << kMaxDigitBits) + sizeof(int32_t) * (1 << kMaxDigitBits) + 16));
+  if (e != cudaSuccess) return e;
+  k_sort_scatter<<<unsigned(tiles), kSortThreads, smem, st>>>(
+      keys, in_ids, M, shift, bits, hist, tiles, start, out_ids, out_keys);
+  count_launches(4);
+  return cudaGetLastError();
+}
+
+}  // namespace rece

@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/rece.h declares, validates configs and sizes its workspace."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from reduced_cross_entropy_b200 import _lib, build
+from reduced_cross_entropy_b200.ops import Plan
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    build.build()
+    return _lib.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "rece.h")).read()
+    return sorted(set(re.findall(r"RECE_API[^;(]*?\b(rece_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 13
+    assert sorted(_lib.EXPORTS) == names
+    L = _lib.lib()
+    for n in names:
+        assert getattr(L, n) is not None
+
+
+def test_status_strings():
+    L = _lib.lib()
+    for code, name in _lib.STATUS_NAMES.items():
+        assert L.rece_status_string(code).decode() == name
+
+
+def cfg(**kw):
+    base = dict(N=256, C=4096, d=64, n_b=16, n_c=8, n_ec=1, n_r=1, k=32, mode=0, flags=0)
+    base.update(kw)
+    return _lib.Config(**base)
+
+
+def create(c):
+    h = ctypes.c_void_p()
+    s = _lib.lib().rece_plan_create(ctypes.byref(c), ctypes.byref(h))
+    if s == 0:
+        _lib.lib().rece_plan_destroy(h)
+    return s
+
+
+@pytest.mark.parametrize("bad", [
+    dict(N=-1), dict(C=0), dict(d=0), dict(n_b=0), dict(n_b=4097), dict(n_r=0), dict(n_r=9),
+    dict(k=0), dict(k=4097), dict(n_ec=-1), dict(n_c=0), dict(n_c=257), dict(C=100, n_c=101),
+    dict(mode=2), dict(flags=0x80),
+])
+def test_invalid_configs_rejected(bad):
+    assert create(cfg(**bad)) == 1
+    assert _lib.lib().rece_last_error_string().decode() != ""
+
+
+def test_unsupported_sizes():
+    assert create(cfg(n_r=4, k=4096)) == 2           # merge buffer bound n_r * k <= 8192
+    assert create(cfg(N=1 << 21, k=1024, n_c=8)) == 2  # 32-bit pair indexing
+
+
+def test_valid_edge_configs():
+    assert create(cfg()) == 0
+    assert create(cfg(N=0, n_c=8)) == 0                 # empty batch
+    assert create(cfg(C=1, N=5, n_c=1, k=1)) == 0       # single item
+    assert create(cfg(n_b=1, n_c=1, k=4095)) == 0       # full-CE reduction
+    assert create(cfg(n_b=4096)) == 0
+
+
+def test_null_arguments():
+    L = _lib.lib()
+    assert L.rece_plan_create(None, None) == 1
+    assert L.rece_plan_workspace_size(None, None) == 1
+    assert L.rece_bucketize_sort(None, None, None, None, None, 0, None) == 1
+
+
+def test_workspace_size_and_layout():
+    for w in [dict(), dict(N=25600, C=100000, n_b=256, n_c=64, n_r=2, k=256, mode=1),
+              dict(N=0, n_c=8)]:
+        p = Plan(**{k: v for k, v in {**dict(N=256, C=4096, d=64, n_b=16, n_c=8, n_ec=1, n_r=1,
+                                             k=32), **w}.items() if k != "mode"},
+                 mode=w.get("mode", 0))
+        c = p.cfg
+        lay = p.layout
+        assert lay.status == 0
+        offs = [lay.bucket_x, lay.bucket_y, lay.perm_x, lay.perm_y, lay.bucket_start_y]
+        assert all(o % 256 == 0 for o in offs)
+        assert lay.bucket_y >= lay.bucket_x + 4 * c.n_r * c.N
+        assert lay.perm_x >= lay.bucket_y + 4 * c.n_r * c.C
+        lists = 8 * c.n_r * c.N * c.k
+        pairs = 5 * 4 * c.N * (c.k + 1)
+        assert p.workspace_bytes >= max(lists, pairs)
+        assert lay.bucket_start_stride == (1 << (c.n_b - 1).bit_length()) + 1
+
+
+def test_full_ce_workspace_size():
+    size = ctypes.c_size_t()
+    assert _lib.lib().rece_full_ce_workspace_size(100, 10, 8, 0, ctypes.byref(size)) == 0
+    assert size.value >= 4 + 400
+    assert _lib.lib().rece_full_ce_workspace_size(100, 0, 8, 0, ctypes.byref(size)) == 1
+
+
+def test_calls_reject_small_workspace_without_gpu():
+    p = Plan(N=256, C=4096, d=64, n_b=16, n_c=8, n_r=1, k=32, mode="fp32")
+    L = _lib.lib()
+    ws = ctypes.c_void_p(256)  # never dereferenced: rejected on the host first
+    s = L.rece_bucketize_sort(p._h, ctypes.c_void_p(512), ctypes.c_void_p(512),
+                              ctypes.c_void_p(512), ws, 16, None)
+    assert s == 3

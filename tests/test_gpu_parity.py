@@ -1,0 +1,169 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, element by element.
+
+Bar: bucket ids, sort orders and selected index sets bit-exact (fmaf-chain scoring:
+fp32 mode, and bf16 mode with RECE_FLAG_FMA_SCORES); loss, per-row loss, lse, dX and
+dY within 1e-4 relative (max-norm), the oracle computing them in fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from reduced_cross_entropy_b200 import ops, synth
+from tests.gpu_common import max_rel, run_gpu, run_oracle, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-4
+W = synth.WORKLOADS
+
+CASES = {
+    "tiny": W["tiny"],
+    "tiny_bf16_rounds2": W["tiny"].scaled(256, 4096, dtype="bf16", n_r=2, k=40),
+    "ragged": synth.Workload("ragged", N=1000, C=5003, d=48, dtype="fp32", n_b=37, n_c=13,
+                             n_ec=2, n_r=3, k=50),
+    "k_over_window": synth.Workload("kw", N=300, C=700, d=16, dtype="fp32", n_b=5, n_c=10,
+                                    n_ec=0, n_r=2, k=200),
+    "d_not_mult8": synth.Workload("d7", N=200, C=999, d=7, dtype="fp32", n_b=3, n_c=4, n_ec=1,
+                                  n_r=1, k=20),
+    "sasrec_scaled": W["sasrec"].scaled(3200, 12500, n_c=8),
+    "lm_scaled": W["lm"].scaled(512, 4000, n_c=4, n_b=64, k=128, d=256),
+    "large_norms_scaled": W["large"].scaled(2000, 20000, n_c=10, n_b=128, k=128),
+}
+
+
+def compare(w, g, o, exact_indices=True):
+    if exact_indices:
+        np.testing.assert_array_equal(g["bx"], o["bx"])
+        np.testing.assert_array_equal(g["by"], o["by"])
+        np.testing.assert_array_equal(g["permX"], o["permX"])
+        np.testing.assert_array_equal(g["permY"], o["permY"])
+        np.testing.assert_array_equal(g["selected"], o["selected"])
+    assert abs(g["loss"] - o["loss"]) <= TOL * abs(o["loss"])
+    assert max_rel(g["row_loss"], o["row_loss"]) <= TOL
+    assert max_rel(g["lse"], o["lse"]) <= TOL
+    assert max_rel(g["dX"], o["dX"]) <= TOL
+    assert max_rel(g["dY"], o["dY"]) <= TOL
+    assert g["status"] == 0
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_parity_fma_path(name):
+    w = CASES[name]
+    X, Y, t = synth.make_inputs(w, seed=0)
+    B = synth.projections(0, 0, w.n_r, w.n_b, w.d, w.dtype)
+    flags = 1 if w.dtype == "bf16" else 0
+    compare(w, run_gpu(w, X, Y, t, B, flags=flags, dloss=0.75),
+            run_oracle(w, X, Y, t, B, dloss=0.75))
+
+
+def test_parity_ties_on_exact_inputs():
+    """Integer-valued inputs: every score is exact and ties are everywhere, so the
+    lowest-index tie rules of argmax, sort and selection are all exercised."""
+    w = synth.Workload("ties", N=640, C=3000, d=12, dtype="fp32", n_b=6, n_c=16, n_ec=1,
+                       n_r=2, k=37)
+    X, Y, t = synth.integer_inputs(w.N, w.C, w.d, seed=3)
+    B = synth.integer_inputs(w.n_r * w.n_b, 1, w.d, seed=4)[0].reshape(w.n_r, w.n_b, w.d)
+    compare(w, run_gpu(w, X, Y, t, B), run_oracle(w, X, Y, t, B))
+
+
+def test_full_ce_identity_one_bucket_one_chunk():
+    """n_b = 1, n_c = 1, k = C - 1: the reduced loss is the full cross-entropy, and the
+    fused full-CE op agrees with both."""
+    w = synth.Workload("full", N=300, C=500, d=32, dtype="fp32", n_b=1, n_c=1, n_ec=0, n_r=1,
+                       k=499)
+    X, Y, t = synth.make_inputs(w, seed=7)
+    B = synth.projections(7, 0, 1, 1, w.d)
+    g = run_gpu(w, X, Y, t, B)
+    o_loss, o_row, o_lse = oracle.full_ce_loss(X, Y, t)
+    assert abs(g["loss"] - o_loss) <= TOL * o_loss
+    assert max_rel(g["row_loss"], o_row) <= TOL
+    Xd, Yd, td = to_dev(X, "fp32"), to_dev(Y, "fp32"), torch.from_numpy(t).cuda()
+    loss, row, lse, ws = ops.full_ce_fwd(Xd, Yd, td)
+    assert abs(loss.item() - o_loss) <= TOL * o_loss
+    assert max_rel(row.cpu().numpy(), o_row) <= TOL
+    dX, dY = ops.full_ce_bwd(Xd, Yd, td, lse, torch.ones(1, device="cuda"), ws)
+    fX, fY = oracle.full_ce_grad(X, Y, t, o_lse)
+    assert max_rel(dX.cpu().numpy(), fX) <= TOL
+    assert max_rel(dY.cpu().numpy(), fY) <= TOL
+    assert max_rel(g["dX"], fX) <= TOL and max_rel(g["dY"], fY) <= TOL
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_full_ce_op_parity(dtype):
+    w = synth.Workload("fce", N=333, C=2049, d=40, dtype=dtype, n_b=1, n_c=1, n_ec=0, n_r=1,
+                       k=1, target_alpha=1.0)
+    X, Y, t = synth.make_inputs(w, seed=11)
+    Xd, Yd, td = to_dev(X, dtype), to_dev(Y, dtype), torch.from_numpy(t).cuda()
+    loss, row, lse, ws = ops.full_ce_fwd(Xd, Yd, td)
+    o_loss, o_row, o_lse = oracle.full_ce_loss(X, Y, t)
+    assert abs(loss.item() - o_loss) <= TOL * o_loss
+    assert max_rel(row.cpu().numpy(), o_row) <= TOL
+    assert max_rel(lse.cpu().numpy(), o_lse) <= TOL
+    dX, dY = ops.full_ce_bwd(Xd, Yd, td, lse, torch.full((1,), 2.0, device="cuda"), ws)
+    fX, fY = oracle.full_ce_grad(X, Y, t, o_lse, 2.0)
+    assert max_rel(dX.cpu().numpy(), fX) <= TOL
+    assert max_rel(dY.cpu().numpy(), fY) <= TOL
+
+
+def test_empty_batch():
+    w = synth.Workload("empty", N=0, C=100, d=8, dtype="fp32", n_b=4, n_c=5, n_ec=1, n_r=1, k=3)
+    X = np.zeros((0, 8), np.float32)
+    Y = synth.make_inputs(w.scaled(5, 100), 0)[1]
+    g = run_gpu(w, X, Y, np.zeros(0, np.int32), synth.projections(0, 0, 1, 4, 8))
+    assert g["loss"] == 0.0
+    assert g["dY"].shape == (100, 8) and np.all(g["dY"] == 0)
+
+
+def test_single_item_catalogue():
+    w = synth.Workload("one", N=50, C=1, d=8, dtype="fp32", n_b=2, n_c=1, n_ec=1, n_r=1, k=4)
+    X, Y, _ = synth.make_inputs(w, 1)
+    t = np.zeros(50, np.int32)
+    g = run_gpu(w, X, Y, t, synth.projections(1, 0, 1, 2, 8))
+    assert np.all(g["selected"] == -1)
+    assert g["loss"] == 0.0 and np.all(g["row_loss"] == 0.0)
+    assert np.all(g["dX"] == 0.0) and np.all(g["dY"] == 0.0)
+
+
+def test_bad_target_sets_device_flag():
+    w = W["tiny"].scaled(64, 512, n_c=4)
+    X, Y, t = synth.make_inputs(w, 2)
+    t[5] = w.C          # out of range
+    t[9] = -3
+    g = run_gpu(w, X, Y, t, synth.projections(2, 0, 1, w.n_b, w.d))
+    assert g["status"] & 1
+    assert np.isnan(g["row_loss"][5]) and np.isnan(g["row_loss"][9])
+    ok = np.ones(64, bool)
+    ok[[5, 9]] = False
+    assert np.all(np.isfinite(g["row_loss"][ok]))
+
+
+def test_backward_is_deterministic():
+    w = CASES["sasrec_scaled"]
+    X, Y, t = synth.make_inputs(w, seed=5)
+    B = synth.projections(5, 0, w.n_r, w.n_b, w.d, w.dtype)
+    a = run_gpu(w, X, Y, t, B, flags=1)
+    b = run_gpu(w, X, Y, t, B, flags=1)
+    for key in ("selected", "row_loss", "lse", "dX", "dY"):
+        np.testing.assert_array_equal(a[key], b[key])
+    assert a["loss"] == b["loss"]
+
+
+def test_sort_many_buckets_and_one_bucket():
+    for n_b in (4096, 1):
+        w = synth.Workload("sort", N=20000, C=30011, d=16, dtype="fp32", n_b=n_b, n_c=16,
+                           n_ec=1, n_r=1, k=8)
+        X, Y, t = synth.make_inputs(w, 9)
+        B = synth.projections(9, 0, 1, n_b, 16)
+        plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode="fp32")
+        ws = plan.workspace()
+        ops.bucketize_sort(plan, to_dev(B, "fp32"), to_dev(X, "fp32"), to_dev(Y, "fp32"), ws)
+        bx, by = (a.cpu().numpy()[0] for a in plan.bucket_ids(ws))
+        px, py = (a.cpu().numpy()[0] for a in plan.permutations(ws))
+        np.testing.assert_array_equal(bx, oracle.bucketize(X, B[0]))
+        np.testing.assert_array_equal(by, oracle.bucketize(Y, B[0]))
+        np.testing.assert_array_equal(px, np.argsort(bx, kind="stable"))
+        np.testing.assert_array_equal(py, np.argsort(by, kind="stable"))
+        starts = plan.bucket_starts_y(ws).cpu().numpy()[0]
+        np.testing.assert_array_equal(starts[:n_b + 1],
+                                      np.searchsorted(np.sort(by), np.arange(n_b + 1)))
