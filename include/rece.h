@@ -166,6 +166,28 @@ RECE_API rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t
                                const float* dloss, void* workspace, size_t workspace_bytes,
                                float* dX, float* dY, void* stream);
 
+/* Stable bucket sort that allocates nothing (the pages have no counterpart: this is an
+ * interface for callers, not a step of the method).  It is step 2's sort on its own, for
+ * callers that cannot give the library device memory: code running inside another
+ * application's fixed device-memory arena (a plugin or custom operator that is not
+ * allowed to allocate), or a loop that cannot take an allocation's latency and implicit
+ * synchronisation.  Its scratch (per-tile histograms) is a 4 MiB array of device memory
+ * inside the library image; every GPU the library is used on holds it until the process
+ * exits.
+ *   bucket_ids   device int32 [M], values in [0, n_b) (others sort by their low bits)
+ *   order        device int32 [M]: element indices by (bucket asc, index asc)
+ *   bucket_start device int32 [2^ceil(log2 n_b) + 1] or NULL: first position of every
+ *                bucket id (entries from n_b on hold M)
+ * Returns RECE_ERR_UNSUPPORTED, having launched nothing, when the histograms of M
+ * elements by 2^ceil(log2 n_b) buckets do not fit the 4 MiB (about M * n_b <= 2^30 /
+ * 4096 * 4096: e.g. M <= 1,040,000 at n_b = 4096, M <= 16.7M at n_b = 256).
+ * The first call on a device looks up the array's device address (make that first call
+ * before any stream capture).  All calls share the array: calls whose GPU work can
+ * overlap (unordered streams or threads) race; order them. */
+RECE_API rece_status_t rece_bucket_sort_static(const int32_t* bucket_ids, int64_t M,
+                                               int32_t n_b, int32_t* order,
+                                               int32_t* bucket_start, void* stream);
+
 /* Synchronises `stream`, then copies the workspace's status word to *device_flags
  * (RECE_DEVICE_* bits).  Returns RECE_ERR_DEVICE_INPUT / RECE_ERR_TIMEOUT when a bit is
  * set, RECE_ERR_CUDA when the stream reports an error. */

@@ -25,7 +25,7 @@ EXPORTS = (
     "rece_plan_workspace_layout", "rece_bucketize_sort", "rece_loss_fwd", "rece_loss_bwd",
     "rece_full_ce_workspace_size", "rece_full_ce_fwd", "rece_full_ce_bwd",
     "rece_get_device_status", "rece_status_string", "rece_last_error_string",
-    "rece_plan_set_stage_events", "rece_kernel_launch_count",
+    "rece_plan_set_stage_events", "rece_kernel_launch_count", "rece_bucket_sort_static",
 )
 STAGES = ("bucketize", "sort", "select", "merge_loss", "mean", "bwd_rows", "bwd_sort",
           "bwd_items")
@@ -82,6 +82,7 @@ def lib():
         "rece_last_error_string": ([], ctypes.c_char_p),
         "rece_plan_set_stage_events": ([vp, ctypes.POINTER(vp)], st),
         "rece_kernel_launch_count": ([], ctypes.c_uint64),
+        "rece_bucket_sort_static": ([vp, i64, i32, vp, vp, vp], st),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)

@@ -17,6 +17,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 }
 void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+void set_last_error(const char* msg);
 }  // namespace rece
 
 using namespace rece;
@@ -96,6 +97,8 @@ rece_status_t check_plan_ws(rece_plan_t plan, const void* ws, size_t ws_bytes) {
 }
 
 }  // namespace
+
+void rece::set_last_error(const char* msg) { fail(RECE_OK, msg); }
 
 extern "C" {
 
