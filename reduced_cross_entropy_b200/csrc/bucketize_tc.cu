@@ -1,0 +1,238 @@
+// bucketize_tc.cu -- step 1 on the tcgen05 tensor cores (bf16 mode): for every row v of
+// X and of Y and every round r, bucket = argmax_b <B[r][b], v> (RECE, section 3,
+// Algorithm 1, the argmax steps); ties go to the lowest b.
+//
+// A persistent, warp-specialised GEMM with the argmax fused into its epilogue:
+//   warp 0      TMA producer: per stage one 128-row x 64 slice of V and one up-to-256-row
+//               x 64 slice of B_r (128-byte swizzle), 4 stages in flight;
+//   warp 1      MMA issuer: M=128 x N=bn x K=16 tcgen05.mma per 32-byte step, fp32
+//               accumulators in TMEM, two 256-column buffers so the epilogue of one tile
+//               overlaps the MMAs of the next;
+//   warps 2-5   epilogue: thread = row; reads its row of the accumulator with
+//               tcgen05.ld and keeps the running (max, argmax).
+// The (rows x n_b) projection matrix never leaves the chip.  Work item = (round, 128-row
+// tile of X or Y); the CTA loops over items with a grid stride.
+#include <climits>
+
+#include "common.cuh"
+#include "plan.h"
+#include "sm100.cuh"
+#include "tc.h"
+
+namespace rece {
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 4;
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr uint32_t kStageABytes = kBM * kBK * 2;  // 16 KB
+constexpr uint32_t kStageBBytes = kBN * kBK * 2;  // 32 KB
+constexpr uint64_t kTimeoutNs = 1000000000ull;    // 1 s per wait
+constexpr int kThreads = 192;
+
+struct __align__(1024) Smem {
+  uint8_t a[kStages][kStageABytes];
+  uint8_t b[kStages][kStageBBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void on_timeout(Smem& s, uint32_t* status) {
+  *reinterpret_cast<volatile int*>(&s.abort) = 1;
+  raise_flag(status, RECE_DEVICE_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_bucketize_tc(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+    const __grid_constant__ CUtensorMap tmB, int64_t N, int64_t C, int d, int n_b, int n_r,
+    int bn, int32_t* __restrict__ bx, int32_t* __restrict__ by, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                     ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tX = (N + kBM - 1) / kBM, tY = (C + kBM - 1) / kBM;
+  const int64_t per_round = tX + tY, items = per_round * n_r;
+  const int n_nt = (n_b + kBN - 1) / kBN;
+  const int nk = d / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abortp = &s.abort;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    uint32_t it = 0;
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmY);
+      prefetch_tmap(&tmB);
+      for (int64_t item = blockIdx.x; item < items && !*abortp; item += gridDim.x) {
+        const int r = int(item / per_round);
+        const int64_t t = item % per_round;
+        const bool isY = t >= tX;
+        const int64_t row0 = (isY ? t - tX : t) * kBM;
+        for (int nt = 0; nt < n_nt && !*abortp; ++nt) {
+          for (int ks = 0; ks < nk; ++ks, ++it) {
+            const int st = it % kStages;
+            const uint32_t n = it / kStages;
+            if (!mbar_wait(&s.empty[st], (n & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+              on_timeout(s, status);
+              break;
+            }
+            mbar_arrive_expect_tx(&s.full[st], kStageABytes + uint32_t(bn) * kBK * 2);
+            tma_load_2d(s.a[st], isY ? &tmY : &tmX, &s.full[st], ks * kBK, int32_t(row0));
+            tma_load_2d(s.b[st], &tmB, &s.full[st], ks * kBK, r * n_b + nt * kBN);
+          }
+        }
+      }
+      // teardown: the last load of every stage has landed (or we give up after the limit)
+      for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+        mbar_wait_limit(&s.full[j % kStages], (j / kStages) & 1u, kTimeoutNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, bn);
+      uint32_t it = 0, acc_it = 0;
+      for (int64_t item = blockIdx.x; item < items && !*abortp; item += gridDim.x) {
+        for (int nt = 0; nt < n_nt && !*abortp; ++nt, ++acc_it) {
+          const int a = acc_it & 1;
+          const uint32_t m = acc_it >> 1;
+          if (!mbar_wait(&s.acc_empty[a], (m & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+            on_timeout(s, status);
+            break;
+          }
+          tc_fence_after();
+          bool ok = true;
+          for (int ks = 0; ks < nk; ++ks, ++it) {
+            const int st = it % kStages;
+            if (!mbar_wait(&s.full[st], (it / kStages) & 1u, &s.abort, kTimeoutNs)) {
+              on_timeout(s, status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t da = desc_k_sw128(smem_u32(s.a[st]));
+            const uint64_t db = desc_k_sw128(smem_u32(s.b[st]));
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              mma_bf16(tmem + a * kBN, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+            mma_commit(&s.empty[st]);
+          }
+          if (!ok) break;
+          mma_commit(&s.acc_full[a]);
+        }
+      }
+      // teardown: every MMA issued so far has completed
+      mma_commit(&s.drain);
+      mbar_wait_limit(&s.drain, 0, kTimeoutNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_local = q * 32 + lane;
+    uint32_t acc_it = 0;
+    for (int64_t item = blockIdx.x; item < items && !*abortp; item += gridDim.x) {
+      const int r = int(item / per_round);
+      const int64_t t = item % per_round;
+      const bool isY = t >= tX;
+      const int64_t row0 = (isY ? t - tX : t) * kBM;
+      float best = -INFINITY;
+      int best_b = INT_MAX;
+      bool ok = true;
+      for (int nt = 0; nt < n_nt; ++nt, ++acc_it) {
+        const int a = acc_it & 1;
+        if (!mbar_wait(&s.acc_full[a], (acc_it >> 1) & 1u, &s.abort, kTimeoutNs)) {
+          on_timeout(s, status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kBN);
+        for (int c0 = 0; c0 < bn; c0 += 32) {
+          float v[32];
+          tmem_load32(taddr + c0, v);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int b = nt * kBN + c0 + u;
+            if (b < n_b && v[u] > best) {
+              best = v[u];
+              best_b = b;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.acc_empty[a]);
+      }
+      if (!ok) break;
+      const int64_t row = row0 + row_local;
+      const int64_t M = isY ? C : N;
+      if (row < M) (isY ? by : bx)[int64_t(r) * M + row] = best_b;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void* Y,
+                                const void* B, int32_t* bx, int32_t* by, uint32_t* status,
+                                cudaStream_t st) {
+  const auto& c = p.cfg;
+  const int bn = c.n_b >= kBN ? kBN : ((c.n_b + 15) / 16) * 16;
+  CUtensorMap tmX, tmY, tmB;
+  cudaError_t e;
+  // an empty X still needs a valid descriptor: point it at Y (no X tile is ever loaded)
+  e = make_tmap_bf16(&tmX, c.N > 0 ? X : Y, c.N > 0 ? c.N : c.C, c.d, kBM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&tmY, Y, c.C, c.d, kBM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&tmB, B, uint64_t(c.n_r) * c.n_b, c.d, bn);
+  if (e != cudaSuccess) return e;
+  const int64_t items = (ceil_div(c.N, kBM) + ceil_div(c.C, kBM)) * c.n_r;
+  const int grid = int(items < sm_count() ? items : sm_count());
+  const size_t smem = sizeof(Smem) + 1024;
+  e = cudaFuncSetAttribute(k_bucketize_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(smem));
+  if (e != cudaSuccess) return e;
+  k_bucketize_tc<<<grid, kThreads, smem, st>>>(tmX, tmY, tmB, c.N, c.C, c.d, c.n_b, c.n_r, bn,
+                                               bx, by, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace rece

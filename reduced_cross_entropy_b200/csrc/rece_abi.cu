@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "plan.h"
+#include "tc.h"
 
 namespace rece {
 size_t select_fma_smem_bytes(int G, int d, int64_t w_max);
@@ -225,6 +226,10 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
     RECE_CUDA(launch_bucketize_fma(static_cast<const float*>(Y), c.C, c.d,
                                    static_cast<const float*>(B), c.n_b, c.n_r, by, st),
               "bucketize Y");
+  } else if (tc_supported(*plan)) {
+    RECE_CUDA(launch_bucketize_tc(*plan, X, Y, B, bx, by,
+                                  reinterpret_cast<uint32_t*>(ws + L.status), st),
+              "bucketize (tcgen05)");
   } else {
     RECE_CUDA(launch_bucketize_fma(static_cast<const __nv_bfloat16*>(X), c.N, c.d,
                                    static_cast<const __nv_bfloat16*>(B), c.n_b, c.n_r, bx, st),
