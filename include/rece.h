@@ -75,6 +75,10 @@ typedef enum {
 /* Bits of the device status word (rece_get_device_status). */
 #define RECE_DEVICE_BAD_TARGET 0x1u /* some target outside [0, C) */
 #define RECE_DEVICE_TIMEOUT 0x2u    /* a bounded wait inside a kernel gave up */
+#define RECE_DEVICE_INEXACT 0x4u    /* bf16 tensor-core mode: some rows' top-k could not be
+                                       certified exact (a candidate list overflowed or a
+                                       threshold was above the k-th kept score); the 32-bit
+                                       word after the status word counts those rows */
 
 typedef struct {
   int64_t N;     /* rows (batch x sequence), >= 0 */
@@ -189,8 +193,9 @@ RECE_API rece_status_t rece_bucket_sort_static(const int32_t* bucket_ids, int64_
                                                int32_t* bucket_start, void* stream);
 
 /* Synchronises `stream`, then copies the workspace's status word to *device_flags
- * (RECE_DEVICE_* bits).  Returns RECE_ERR_DEVICE_INPUT / RECE_ERR_TIMEOUT when a bit is
- * set, RECE_ERR_CUDA when the stream reports an error. */
+ * (RECE_DEVICE_* bits).  Returns RECE_ERR_TIMEOUT / RECE_ERR_DEVICE_INPUT when the
+ * timeout / bad-target bit is set (RECE_DEVICE_INEXACT alone is informational and returns
+ * RECE_OK), RECE_ERR_CUDA when the stream reports an error. */
 RECE_API rece_status_t rece_get_device_status(const void* workspace, uint32_t* device_flags,
                                      void* stream);
 

@@ -1,0 +1,278 @@
+// merge_tc.cu -- steps 4-5 for the tensor-core selection: one warp per row.
+//
+// The row's candidates are the (score, sorted position) pairs its rounds emitted.  A pair
+// of round r is translated to its item j and dropped when j is the row's positive or when
+// j also lies in the row's window of an earlier round r' < r (that round saw the same
+// pair, so the union of the rounds stays de-duplicated -- the RECE paper's ln(count)
+// correction for repeated pairs amounts to counting each pair once).  The k best of the
+// rest by (score descending, item ascending) are found with a warp radix select (4 passes
+// of 8 bits on the score key, then the item ids if the k-th place is tied), ordered best
+// first with a bitonic sort, and give the row's loss (RECE, Algorithm 1's loss lines):
+//   lse_i = log(exp(l+) + sum_j exp(l_j)),  loss_i = lse_i - l+.
+// Exactness check: each round recorded the largest score it did not emit; if no list
+// overflowed and every such score is below the k-th kept score, nothing left out could
+// have been selected.  Rows failing the check are counted in the status area (second word) and
+// flagged RECE_DEVICE_INEXACT.
+#include "common.cuh"
+#include "plan.h"
+#include "tc.h"
+
+namespace rece {
+namespace {
+
+constexpr int kThreads = 256;
+
+struct WarpSel {
+  uint32_t T;
+  int need;
+  int eq;
+};
+
+// Among n elements of the warp (get(q, key) -> in play, its key), the want-th largest key.
+template <typename Get>
+__device__ WarpSel warp_radix_select(int n, int want, Get get, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, pmask = 0;
+  int eq = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int q = lane; q < n; q += 32) {
+      uint32_t key;
+      if (get(q, key) && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    int c[8], s = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {  // lane 0 holds the highest 8 bins, highest first
+      c[u] = int(hist[255 - 8 * lane - u]);
+      s += c[u];
+    }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - s;
+    const bool mine = excl < want && want <= incl;
+    int digit = 0, above = 0, cnt = 0;
+    if (mine) {
+      int run = excl;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (run + c[u] >= want) {
+          digit = 255 - 8 * lane - u;
+          above = run;
+          cnt = c[u];
+          break;
+        }
+        run += c[u];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
+    digit = __shfl_sync(0xFFFFFFFFu, digit, src);
+    above = __shfl_sync(0xFFFFFFFFu, above, src);
+    cnt = __shfl_sync(0xFFFFFFFFu, cnt, src);
+    want -= above;
+    eq = cnt;
+    prefix |= uint32_t(digit) << shift;
+    pmask |= 0xFFu << shift;
+    __syncwarp();
+  }
+  return WarpSel{prefix, want, eq};
+}
+
+__device__ void warp_bitonic_sort_asc(uint64_t* a, int P) {
+  const int lane = threadIdx.x & 31;
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int e = lane; e < (P >> 1); e += 32) {
+        const int lo = 2 * stride * (e / stride) + (e % stride), hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint64_t x = a[lo], y = a[hi];
+        if ((x > y) == up) {
+          a[lo] = y;
+          a[hi] = x;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_merge_tc(
+    const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
+    const int32_t* __restrict__ py, const int32_t* __restrict__ invX,
+    const int32_t* __restrict__ chunkY, const int2* __restrict__ list,
+    const int32_t* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
+    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Q, int cap, int P,
+    int32_t* __restrict__ selected, float* __restrict__ lse_out, float* __restrict__ row_loss,
+    uint32_t* status) {
+  extern __shared__ __align__(16) uint8_t sh_raw[];
+  const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t per_warp = size_t(P) * 8 + size_t(cap) * 8 + 1024;
+  uint8_t* base = sh_raw + per_warp * wid;
+  uint64_t* sel = reinterpret_cast<uint64_t*>(base);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(base + size_t(P) * 8);
+  int32_t* items = reinterpret_cast<int32_t*>(keys + cap);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(items + cap);
+
+  const int64_t i = int64_t(blockIdx.x) * warps + wid;
+  if (i >= N) return;  // whole warp leaves together; no block-wide barriers below
+  const int32_t z = targets[i];
+  const bool z_ok = z >= 0 && z < C;
+
+  // gather the candidates of all rounds
+  int cx[8];
+  for (int r = 0; r < n_r; ++r) cx[r] = int((int64_t(invX[int64_t(r) * N + i]) * n_c) / N);
+  int n = 0;
+  bool overflow = false;
+  float theta_max = -INFINITY;
+  for (int r = 0; r < n_r; ++r) {
+    const int64_t p = invX[int64_t(r) * N + i];
+    const int cnt = list_count[int64_t(r) * N + p];
+    overflow |= cnt > Q;
+    theta_max = fmaxf(theta_max, list_theta[int64_t(r) * N + p]);
+    const int m = cnt < Q ? cnt : Q;
+    const int2* L = list + (int64_t(r) * N + p) * Q;
+    for (int a0 = 0; a0 < m; a0 += 32) {
+      const int a = a0 + lane;
+      bool keep = false;
+      uint32_t key = 0;
+      int32_t j = -1;
+      if (a < m) {
+        const int2 e = L[a];
+        j = py[int64_t(r) * C + e.y];
+        keep = j != z;
+        for (int rp = 0; rp < r && keep; ++rp) {
+          const int dc = chunkY[int64_t(rp) * C + j] - cx[rp];
+          if (dc >= -n_ec && dc <= n_ec) keep = false;
+        }
+        key = score_key(__int_as_float(e.x));
+      }
+      const unsigned b = __ballot_sync(0xFFFFFFFFu, keep);
+      if (keep) {
+        const int pos = n + __popc(b & ((1u << lane) - 1u));
+        keys[pos] = key;
+        items[pos] = j;
+      }
+      n += __popc(b);
+    }
+  }
+  __syncwarp();
+
+  // the k best
+  const int kk = k < n ? k : n;
+  const bool all = kk >= n;
+  WarpSel s1{0, 0, 0}, s2{0, 0, 0};
+  bool tie = false;
+  if (!all) {
+    s1 = warp_radix_select(
+        n, kk, [&](int q, uint32_t& key) { key = keys[q]; return true; }, hist);
+    if (s1.need != s1.eq) {
+      tie = true;
+      const uint32_t Tk = s1.T;
+      s2 = warp_radix_select(
+          n, s1.need,
+          [&](int q, uint32_t& key) {
+            key = ~uint32_t(items[q]);
+            return keys[q] == Tk;
+          },
+          hist);
+    }
+  }
+  int ns = 0;
+  for (int a0 = 0; a0 < n; a0 += 32) {
+    const int a = a0 + lane;
+    bool take = false;
+    if (a < n) {
+      const uint32_t key = keys[a];
+      take = all || key > s1.T ||
+             (key == s1.T && (!tie || ~uint32_t(items[a]) >= s2.T));
+    }
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, take);
+    if (take) sel[ns + __popc(b & ((1u << lane) - 1u))] = ~cand_key(keys[a], items[a]);
+    ns += __popc(b);
+  }
+  for (int a = ns + lane; a < P; a += 32) sel[a] = ~0ull;
+  __syncwarp();
+  warp_bitonic_sort_asc(sel, P);
+  for (int a = lane; a < k; a += 32) selected[i * k + a] = a < ns ? cand_item(~sel[a]) : -1;
+
+  // theta_max: the largest score some round did not emit (-inf if every round emitted all)
+  const float s_k = ns == k ? key_score(uint32_t((~sel[k - 1]) >> 32)) : -INFINITY;
+  if (lane == 0 && (overflow || (theta_max > -INFINITY && theta_max >= s_k))) {
+    atomicAdd(status + 1, 1u);
+    raise_flag(status, RECE_DEVICE_INEXACT);
+  }
+
+  // loss of the row
+  float part = 0.0f;
+  if (z_ok) {
+    const T* x = X + i * d;
+    const T* y = Y + int64_t(z) * d;
+    for (int t = lane; t < d; t += 32) part = fmaf(to_f32(x[t]), to_f32(y[t]), part);
+  }
+  const float lp = warp_sum(part);
+  const float best = ns > 0 ? key_score(uint32_t((~sel[0]) >> 32)) : -INFINITY;
+  const float m = fmaxf(lp, best);
+  float acc = 0.0f;
+  for (int a = lane; a < ns; a += 32) acc += expf(key_score(uint32_t((~sel[a]) >> 32)) - m);
+  const float tot = warp_sum(acc) + expf(lp - m);
+  if (lane == 0) {
+    if (!z_ok) {
+      raise_flag(status, RECE_DEVICE_BAD_TARGET);
+      lse_out[i] = NAN;
+      if (row_loss) row_loss[i] = NAN;
+    } else {
+      const float lse = m + logf(tot);
+      lse_out[i] = lse;
+      if (row_loss) row_loss[i] = lse - lp;
+    }
+  }
+}
+
+}  // namespace
+
+int tc_list_capacity(int k);
+
+size_t merge_tc_warp_bytes(int n_r, int k) {
+  int P = 2;
+  while (P < k) P <<= 1;
+  const size_t cap = size_t(n_r) * tc_list_capacity(k);
+  return size_t(P) * 8 + cap * 8 + 1024;
+}
+
+template <typename T>
+cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
+                            const int32_t* py, const int32_t* invX, const int32_t* chunkY,
+                            const int2* list, const int32_t* list_count,
+                            const float* list_theta, int32_t* selected, float* lse,
+                            float* row_loss, uint32_t* status, cudaStream_t st) {
+  const auto& c = p.cfg;
+  if (c.N == 0) return cudaSuccess;
+  int P = 2;
+  while (P < c.k) P <<= 1;
+  const int Q = tc_list_capacity(c.k);
+  const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
+  int warps = int((200 * 1024) / per_warp);
+  warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
+  const size_t smem = per_warp * warps;
+  cudaError_t e = cudaFuncSetAttribute(k_merge_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  k_merge_tc<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
+      X, Y, targets, py, invX, chunkY, list, list_count, list_theta, c.N, c.C, c.d, c.k, c.n_r,
+      c.n_c, c.n_ec, Q, c.n_r * Q, P, selected, lse, row_loss, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_merge_tc<__nv_bfloat16>(
+    const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
+    const int32_t*, const int32_t*, const int32_t*, const int2*, const int32_t*, const float*,
+    int32_t*, float*, float*, uint32_t*, cudaStream_t);
+
+}  // namespace rece

@@ -36,6 +36,8 @@ struct Layout {
   size_t bx = 0, by = 0, px = 0, py = 0, bstart_y = 0, bstart_x = 0;
   size_t sort_scratch = 0;
   size_t list_score = 0, list_item = 0, row_loss_tmp = 0;
+  // tensor-core path (bf16 mode): sorted row copies, inverse orders, candidate lists
+  size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0;
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_scratch = 0;
@@ -54,6 +56,7 @@ struct rece_plan_s {
   int32_t bucket_bits;  // digit bits of the bucket sort
   int32_t item_bits;    // key bits of the backward item sort (values 0..C)
   int64_t entries;      // N * (k + 1): (row, item) pairs of the backward
+  bool use_tc;          // bf16 mode on the tcgen05 kernels
   rece::Layout lay;
   void* stage_events[2 * RECE_NUM_STAGES];  // optional timing hook (cudaEvent_t)
   bool timed;

@@ -62,7 +62,7 @@ void build_layout(rece_plan_s& p) {
     off += align256(bytes);
     return o;
   };
-  L.status = take(sizeof(uint32_t));
+  L.status = take(2 * sizeof(uint32_t));  // flags, count of inexact rows
   const size_t region = off;
   const size_t nb_stride = (size_t(1) << p.bucket_bits) + 1;
   L.bx = take(sizeof(int32_t) * c.n_r * c.N);
@@ -72,8 +72,19 @@ void build_layout(rece_plan_s& p) {
   L.bstart_x = take(sizeof(int32_t) * c.n_r * nb_stride);
   L.bstart_y = take(sizeof(int32_t) * c.n_r * nb_stride);
   L.sort_scratch = take(sort_scratch_bytes(c.N > c.C ? c.N : c.C, p.bucket_bits));
-  L.list_score = take(sizeof(float) * size_t(c.n_r) * c.N * c.k);
-  L.list_item = take(sizeof(int32_t) * size_t(c.n_r) * c.N * c.k);
+  if (p.use_tc) {
+    const size_t Q = size_t(tc_list_capacity(c.k));
+    L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
+    L.ys = take(sizeof(uint16_t) * size_t(c.n_r) * c.C * c.d);
+    L.inv_x = take(sizeof(int32_t) * c.n_r * c.N);
+    L.chunk_y = take(sizeof(int32_t) * c.n_r * c.C);
+    L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
+    L.tc_count = take(sizeof(int32_t) * c.n_r * c.N);
+    L.tc_theta = take(sizeof(float) * c.n_r * c.N);
+  } else {
+    L.list_score = take(sizeof(float) * size_t(c.n_r) * c.N * c.k);
+    L.list_item = take(sizeof(int32_t) * size_t(c.n_r) * c.N * c.k);
+  }
   L.row_loss_tmp = take(sizeof(float) * c.N);
   L.fwd_end = off;
   off = region;
@@ -166,6 +177,11 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   p->entries = c.N * (int64_t(c.k) + 1);
   p->timed = false;
   for (void*& e : p->stage_events) e = nullptr;
+  p->use_tc = tc_supported(*p);
+  if (p->use_tc && merge_tc_warp_bytes(c.n_r, c.k) > 200 * 1024) {
+    delete p;
+    return fail(RECE_ERR_UNSUPPORTED, "n_r * k too large for the tensor-core merge");
+  }
   build_layout(*p);
   *out = p;
   return RECE_OK;
@@ -215,7 +231,7 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const Layout& L = plan->lay;
-  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, sizeof(uint32_t), st), "status reset");
+  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, 2 * sizeof(uint32_t), st), "status reset");
   int32_t* bx = reinterpret_cast<int32_t*>(ws + L.bx);
   int32_t* by = reinterpret_cast<int32_t*>(ws + L.by);
   stage_mark(*plan, RECE_STAGE_BUCKETIZE, 0, st);
@@ -226,7 +242,7 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
     RECE_CUDA(launch_bucketize_fma(static_cast<const float*>(Y), c.C, c.d,
                                    static_cast<const float*>(B), c.n_b, c.n_r, by, st),
               "bucketize Y");
-  } else if (tc_supported(*plan)) {
+  } else if (plan->use_tc) {
     RECE_CUDA(launch_bucketize_tc(*plan, X, Y, B, bx, by,
                                   reinterpret_cast<uint32_t*>(ws + L.status), st),
               "bucketize (tcgen05)");
@@ -252,6 +268,16 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
                                reinterpret_cast<int32_t*>(ws + L.py) + int64_t(r) * c.C, nullptr,
                                reinterpret_cast<int32_t*>(ws + L.bstart_y) + r * stride, st),
               "sort Y");
+  }
+  if (plan->use_tc) {
+    RECE_CUDA(launch_permute_rows(X, c.N, c.d, reinterpret_cast<const int32_t*>(ws + L.px),
+                                  c.n_r, c.n_c, ws + L.xs,
+                                  reinterpret_cast<int32_t*>(ws + L.inv_x), nullptr, st),
+              "permute X");
+    RECE_CUDA(launch_permute_rows(Y, c.C, c.d, reinterpret_cast<const int32_t*>(ws + L.py),
+                                  c.n_r, c.n_c, ws + L.ys, nullptr,
+                                  reinterpret_cast<int32_t*>(ws + L.chunk_y), st),
+              "permute Y");
   }
   stage_mark(*plan, RECE_STAGE_SORT, 1, st);
   return RECE_OK;
@@ -284,6 +310,22 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
     RECE_CUDA(launch_merge_loss(*plan, Xf, Yf, targets, ls, li, selected, lse, rl, status, st),
               "merge/loss");
+  } else if (plan->use_tc) {
+    const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+    const __nv_bfloat16* Yb = static_cast<const __nv_bfloat16*>(Y);
+    int2* list = reinterpret_cast<int2*>(ws + L.tc_list);
+    int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.tc_count);
+    float* theta = reinterpret_cast<float*>(ws + L.tc_theta);
+    stage_mark(*plan, RECE_STAGE_SELECT, 0, st);
+    RECE_CUDA(launch_select_tc(*plan, ws + L.xs, ws + L.ys, list, cnt, theta, status, st),
+              "select (tcgen05)");
+    stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
+    stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
+    RECE_CUDA(launch_merge_tc(*plan, Xb, Yb, targets, py,
+                              reinterpret_cast<const int32_t*>(ws + L.inv_x),
+                              reinterpret_cast<const int32_t*>(ws + L.chunk_y), list, cnt, theta,
+                              selected, lse, rl, status, st),
+              "merge/loss (tcgen05 lists)");
   } else {
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
     const __nv_bfloat16* Yb = static_cast<const __nv_bfloat16*>(Y);
@@ -329,7 +371,7 @@ rece_status_t rece_full_ce_workspace_size(int64_t N, int64_t C, int32_t d, int32
                                           size_t* bytes) {
   if (!bytes || N < 0 || C < 1 || d < 1 || (mode != RECE_MODE_FP32_EXACT && mode != RECE_MODE_BF16))
     return fail(RECE_ERR_INVALID_ARG, "bad full-CE arguments");
-  *bytes = align256(sizeof(uint32_t)) + align256(sizeof(float) * size_t(N));
+  *bytes = align256(2 * sizeof(uint32_t)) + align256(sizeof(float) * size_t(N));
   return RECE_OK;
 }
 
@@ -346,8 +388,8 @@ rece_status_t rece_full_ce_fwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + align256(sizeof(uint32_t)));
-  RECE_CUDA(cudaMemsetAsync(status, 0, sizeof(uint32_t), st), "status reset");
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + align256(2 * sizeof(uint32_t)));
+  RECE_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), st), "status reset");
   if (mode == RECE_MODE_FP32_EXACT)
     RECE_CUDA(launch_full_ce_fwd(N, C, d, static_cast<const float*>(X),
                                  static_cast<const float*>(Y), targets, rl, lse, status, st),
@@ -392,7 +434,7 @@ rece_status_t rece_get_device_status(const void* workspace, uint32_t* device_fla
   RECE_CUDA(cudaMemcpy(device_flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost),
             "status read");
   if (*device_flags & RECE_DEVICE_TIMEOUT) return fail(RECE_ERR_TIMEOUT, "device wait timed out");
-  if (*device_flags) return fail(RECE_ERR_DEVICE_INPUT, "device input error");
+  if (*device_flags & RECE_DEVICE_BAD_TARGET) return fail(RECE_ERR_DEVICE_INPUT, "device input error");
   return RECE_OK;
 }
 

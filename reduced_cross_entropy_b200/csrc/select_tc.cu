@@ -1,0 +1,340 @@
+// select_tc.cu -- steps 3-4 on the tcgen05 tensor cores (bf16 mode): chunk-window scores
+// (RECE, section 3, Algorithm 1: chunk sets, neighbour window, chunk logits; the rounds
+// paragraph) and the candidates for each row's top-k negatives (SCE abstract).
+//
+// Work item = (round r, 128 consecutive sorted rows).  Their chunks' windows are a
+// contiguous range of sorted catalogue rows (the union of the windows), streamed by TMA in
+// 256-row tiles; tcgen05.mma forms the 128 x 256 score tile in TMEM.  Each row's thread
+// reads its row of the tile and looks only at columns inside its own window.  The window
+// is streamed three times, the threshold found without any assumption on the scores'
+// distribution:
+//   pass 1  per row: count and max m of its window's scores;
+//   pass 2  per row: exact histogram, in shared memory, of key(m) - key(s) >> 20 where key
+//           is the order-preserving integer image of an fp32 score -- 8 bins per binade
+//           of |s| below m (128 bins, the last one open), so the bins follow the scores'
+//           own scale whatever their distribution;
+//   pass 3  the smallest bin b* whose cumulative count reaches E = 1.25 k + 8 sets the
+//           cut: every score in a bin <= b* is emitted as (score, sorted position) to the
+//           row's list (equal scores share a bin, so a tie is never split); the largest
+//           score NOT emitted is recorded.
+// The list keeps up to Q entries (Q = 2k + 64) and the count of all that passed.  The
+// merge kernel keeps the k best; the selection is exact whenever no list overflowed and
+// every round's largest non-emitted score is below the k-th kept score, which the merge
+// kernel checks row by row.  Score tiles never reach HBM.
+#include "common.cuh"
+#include "plan.h"
+#include "sm100.cuh"
+#include "tc.h"
+
+namespace rece {
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 3;
+constexpr int kPasses = 3;
+constexpr int kBins = 128;
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr uint32_t kStageABytes = kBM * kBK * 2;
+constexpr uint32_t kStageBBytes = kBN * kBK * 2;
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+constexpr int kThreads = 192;
+
+struct __align__(1024) Smem {
+  uint8_t a[kStages][kStageABytes];
+  uint8_t b[kStages][kStageBBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  uint32_t hist[kBins][kBM];  // per row (column) gap histogram of pass 2
+};
+
+__device__ __forceinline__ void on_timeout(Smem& s, uint32_t* status) {
+  *reinterpret_cast<volatile int*>(&s.abort) = 1;
+  raise_flag(status, RECE_DEVICE_TIMEOUT);
+}
+
+struct ItemGeom {
+  int r;
+  int64_t p0;   // first sorted row of the tile
+  int64_t U0;   // union window [U0, U1) in sorted catalogue positions
+  int nt;       // 256-wide tiles covering it
+};
+
+// Order-preserving integer image of an fp32 score (a < b  <=>  key(a) < key(b)).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return u ^ (uint32_t(int32_t(u) >> 31) | 0x80000000u);
+}
+
+__device__ __forceinline__ int64_t chunk_of(int64_t p, int64_t M, int n_c) {
+  return (p * n_c) / M;
+}
+
+__device__ __forceinline__ ItemGeom item_geom(int64_t item, int64_t tiles_per_round, int64_t N,
+                                              int64_t C, int n_c, int n_ec) {
+  ItemGeom g;
+  g.r = int(item / tiles_per_round);
+  g.p0 = (item % tiles_per_round) * kBM;
+  const int64_t last = (g.p0 + kBM - 1 < N - 1) ? g.p0 + kBM - 1 : N - 1;
+  const int64_t cf = chunk_of(g.p0, N, n_c), cl = chunk_of(last, N, n_c);
+  g.U0 = chunk_start(cf - n_ec < 0 ? 0 : cf - n_ec, C, n_c);
+  const int64_t U1 = chunk_start(cl + n_ec + 1 > n_c ? n_c : cl + n_ec + 1, C, n_c);
+  g.nt = int((U1 - g.U0 + kBN - 1) / kBN);
+  return g;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_select_tc(
+    const __grid_constant__ CUtensorMap tmXs, const __grid_constant__ CUtensorMap tmYs,
+    int64_t N, int64_t C, int d, int n_c, int n_ec, int n_r, int Q, int E,
+    int2* __restrict__ list, int32_t* __restrict__ list_count, float* __restrict__ list_theta,
+    uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                     ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tiles_per_round = (N + kBM - 1) / kBM;
+  const int64_t items = tiles_per_round * n_r;
+  const int nk = d / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abortp = &s.abort;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmXs);
+      prefetch_tmap(&tmYs);
+      uint32_t it = 0;
+      for (int64_t item = blockIdx.x; item < items && !*abortp; item += gridDim.x) {
+        const ItemGeom g = item_geom(item, tiles_per_round, N, C, n_c, n_ec);
+        const int32_t arow = int32_t(int64_t(g.r) * N + g.p0);
+        for (int pass = 0; pass < kPasses && !*abortp; ++pass) {
+          for (int t = 0; t < g.nt && !*abortp; ++t) {
+            const int32_t brow = int32_t(int64_t(g.r) * C + g.U0 + int64_t(t) * kBN);
+            for (int ks = 0; ks < nk; ++ks, ++it) {
+              const int st = it % kStages;
+              if (!mbar_wait(&s.empty[st], ((it / kStages) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+                on_timeout(s, status);
+                break;
+              }
+              mbar_arrive_expect_tx(&s.full[st], kStageABytes + kStageBBytes);
+              tma_load_2d(s.a[st], &tmXs, &s.full[st], ks * kBK, arow);
+              tma_load_2d(s.b[st], &tmYs, &s.full[st], ks * kBK, brow);
+            }
+          }
+        }
+      }
+      for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+        mbar_wait_limit(&s.full[j % kStages], (j / kStages) & 1u, kTimeoutNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+      uint32_t it = 0, acc_it = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < items && ok && !*abortp; item += gridDim.x) {
+        const ItemGeom g = item_geom(item, tiles_per_round, N, C, n_c, n_ec);
+        for (int tt = 0; tt < kPasses * g.nt && ok; ++tt, ++acc_it) {
+          const int a = acc_it & 1;
+          if (!mbar_wait(&s.acc_empty[a], ((acc_it >> 1) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+            on_timeout(s, status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int ks = 0; ks < nk; ++ks, ++it) {
+            const int st = it % kStages;
+            if (!mbar_wait(&s.full[st], (it / kStages) & 1u, &s.abort, kTimeoutNs)) {
+              on_timeout(s, status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t da = desc_k_sw128(smem_u32(s.a[st]));
+            const uint64_t db = desc_k_sw128(smem_u32(s.b[st]));
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              mma_bf16(tmem + a * kBN, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+            mma_commit(&s.empty[st]);
+          }
+          if (!ok) break;
+          mma_commit(&s.acc_full[a]);
+        }
+      }
+      mma_commit(&s.drain);
+      mbar_wait_limit(&s.drain, 0, kTimeoutNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;
+    const int row_local = q4 * 32 + lane;
+    uint32_t acc_it = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < items && ok && !*abortp; item += gridDim.x) {
+      const ItemGeom g = item_geom(item, tiles_per_round, N, C, n_c, n_ec);
+      const int64_t p = g.p0 + row_local;
+      const bool valid = p < N;
+      int64_t w0 = 0, w1 = 0;  // this row's window, in sorted catalogue positions
+      if (valid) {
+        const int64_t c = chunk_of(p, N, n_c);
+        w0 = chunk_start(c - n_ec < 0 ? 0 : c - n_ec, C, n_c);
+        w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
+      }
+      int cnt = 0;
+      float mx = -INFINITY, not_emitted = -INFINITY;
+      uint32_t kmx = 0;    // key of the row's max
+      bool emit_all = false;
+      uint32_t limit = 0;  // pass 3 emits a score iff key(m) - key(s) < limit
+      int emitted = 0;
+      uint32_t* hcol = &s.hist[0][row_local];
+      int2* out = list + (int64_t(g.r) * N + (valid ? p : 0)) * Q;
+      for (int pass = 0; pass < kPasses && ok; ++pass) {
+        if (pass == 1) {
+          emit_all = !valid || cnt <= E;
+          kmx = order_key(mx);
+          for (int b = 0; b < kBins; ++b) hcol[b * kBM] = 0;
+        } else if (pass == 2 && !emit_all) {
+          uint32_t cum = 0;
+          int bstar = kBins - 1;
+          for (int b = 0; b < kBins; ++b) {
+            cum += hcol[b * kBM];
+            if (cum >= uint32_t(E)) {
+              bstar = b;
+              break;
+            }
+          }
+          if (bstar >= kBins - 1) emit_all = true;
+          else limit = uint32_t(bstar + 1) << 20;
+        }
+        for (int t = 0; t < g.nt; ++t, ++acc_it) {
+          const int a = acc_it & 1;
+          if (!mbar_wait(&s.acc_full[a], (acc_it >> 1) & 1u, &s.abort, kTimeoutNs)) {
+            on_timeout(s, status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int64_t q0 = g.U0 + int64_t(t) * kBN;
+          const uint32_t taddr = tmem + (uint32_t(q4 * 32) << 16) + uint32_t(a * kBN);
+#pragma unroll 1
+          for (int c0 = 0; c0 < kBN; c0 += 32) {
+            const int64_t qa = q0 + c0;
+            const bool need = valid && qa < w1 && qa + 32 > w0 && !(pass == 1 && emit_all);
+            if (!__any_sync(0xFFFFFFFFu, need)) continue;
+            float v[32];
+            tmem_load32(taddr + c0, v);
+            if (!need) continue;
+            const bool inside = qa >= w0 && qa + 32 <= w1;
+            if (pass == 0) {
+              if (inside) {
+                cnt += 32;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) mx = fmaxf(mx, v[u]);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  if (qa + u >= w0 && qa + u < w1) {
+                    ++cnt;
+                    mx = fmaxf(mx, v[u]);
+                  }
+                }
+              }
+            } else if (pass == 1) {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                if (inside || (qa + u >= w0 && qa + u < w1)) {
+                  const uint32_t raw = (kmx - order_key(v[u])) >> 20;
+                  hcol[(raw < kBins - 1 ? raw : kBins - 1) * kBM] += 1u;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                if (inside || (qa + u >= w0 && qa + u < w1)) {
+                  if (emit_all || kmx - order_key(v[u]) < limit) {
+                    if (emitted < Q)
+                      out[emitted] = make_int2(__float_as_int(v[u]), int32_t(qa + u));
+                    ++emitted;
+                  } else {
+                    not_emitted = fmaxf(not_emitted, v[u]);
+                  }
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.acc_empty[a]);
+        }
+      }
+      if (ok && valid) {
+        list_count[int64_t(g.r) * N + p] = emitted;
+        list_theta[int64_t(g.r) * N + p] = not_emitted;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+int tc_list_capacity(int k) { return 2 * k + 64; }
+int tc_emit_target(int k) { return k + k / 4 + 8; }
+
+cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys, int2* list,
+                             int32_t* list_count, float* list_theta, uint32_t* status,
+                             cudaStream_t st) {
+  const auto& c = p.cfg;
+  if (c.N == 0) return cudaSuccess;
+  CUtensorMap tmXs, tmYs;
+  cudaError_t e = make_tmap_bf16(&tmXs, Xs, uint64_t(c.n_r) * c.N, c.d, kBM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&tmYs, Ys, uint64_t(c.n_r) * c.C, c.d, kBN);
+  if (e != cudaSuccess) return e;
+  const int64_t items = ceil_div(c.N, kBM) * c.n_r;
+  const int grid = int(items < sm_count() ? items : sm_count());
+  const size_t smem = sizeof(Smem) + 1024;
+  e = cudaFuncSetAttribute(k_select_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  k_select_tc<<<grid, kThreads, smem, st>>>(tmXs, tmYs, c.N, c.C, c.d, c.n_c, c.n_ec, c.n_r,
+                                            tc_list_capacity(c.k), tc_emit_target(c.k), list,
+                                            list_count, list_theta, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace rece

@@ -23,4 +23,25 @@ cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void*
                                 const void* B, int32_t* bx, int32_t* by, uint32_t* status,
                                 cudaStream_t st);
 
+// Sorted row copies (bf16) and inverse orders / per-round chunk of every row.
+cudaError_t launch_permute_rows(const void* V, int64_t M, int d, const int32_t* perm, int n_r,
+                                int n_c, void* Vs, int32_t* inv, int32_t* chunk,
+                                cudaStream_t st);
+
+// K3 on tensor cores: per (round, sorted row) the candidate list (score bits, sorted
+// catalogue position), its count and threshold.
+int tc_list_capacity(int k);
+cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys, int2* list,
+                             int32_t* list_count, float* list_theta, uint32_t* status,
+                             cudaStream_t st);
+
+// K4 for the tensor-core lists: merge, select, order, loss, exactness check.
+size_t merge_tc_warp_bytes(int n_r, int k);
+template <typename T>
+cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
+                            const int32_t* py, const int32_t* invX, const int32_t* chunkY,
+                            const int2* list, const int32_t* list_count,
+                            const float* list_theta, int32_t* selected, float* lse,
+                            float* row_loss, uint32_t* status, cudaStream_t st);
+
 }  // namespace rece

@@ -57,3 +57,47 @@ def test_bucketize_tc_random_inputs_near_ties_only():
             for row, i in enumerate(diff):
                 a, b = P[row, got[i]], P[row, want[i]]
                 assert abs(a - b) <= 1e-5 * np.abs(P[row]).max()
+
+
+# ---------------------------------------------------------------- whole path, tcgen05
+TC_CASES = {
+    "tiny_bf16_rounds2": synth.WORKLOADS["tiny"].scaled(256, 4096, dtype="bf16", n_r=2, k=40),
+    "sasrec_scaled": synth.WORKLOADS["sasrec"].scaled(3200, 12500, n_c=8),
+    "sasrec_scaled_2": synth.WORKLOADS["sasrec"].scaled(6400, 25000, n_c=16),
+    "large_norms_scaled": synth.WORKLOADS["large"].scaled(2000, 20000, n_c=10, n_b=128, k=128),
+    "lm_scaled": synth.WORKLOADS["lm"].scaled(512, 4000, n_c=4, n_b=64, k=128, d=256),
+    "very_large_scaled": synth.WORKLOADS["very_large"].scaled(4096, 40000, n_c=64, n_b=256,
+                                                              k=256),
+}
+
+
+def recall(sel_gpu, sel_orc):
+    hit = tot = 0
+    for a, b in zip(sel_gpu, sel_orc):
+        sb = set(b[b >= 0].tolist())
+        hit += len(sb & set(a[a >= 0].tolist()))
+        tot += len(sb)
+    return hit / max(tot, 1)
+
+
+@pytest.mark.parametrize("name", sorted(TC_CASES))
+def test_tc_path_recall_and_loss(name):
+    w = TC_CASES[name]
+    X, Y, t = synth.make_inputs(w, seed=3)
+    B = synth.projections(3, 0, w.n_r, w.n_b, w.d, "bf16")
+    g = run_gpu(w, X, Y, t, B, flags=0, dloss=1.0)
+    o = run_oracle(w, X, Y, t, B, dloss=1.0)
+    rc = recall(g["selected"], o["selected"])
+    assert rc >= 0.99, rc
+    assert abs(g["loss"] - o["loss"]) <= 1e-2 * abs(o["loss"])
+    assert g["status"] & ~0x4 == 0
+    # every row's kept negatives are distinct, never the positive, and inside its windows
+    for i in range(0, w.N, max(1, w.N // 64)):
+        s = g["selected"][i]
+        s = s[s >= 0]
+        assert len(set(s.tolist())) == len(s) and t[i] not in set(s.tolist())
+    # gradients of the selection the GPU made, against the oracle's fp64 formula
+    _, _, lse = oracle.rece_loss(X, Y, t, g["selected"])
+    oX, oY = oracle.rece_grad(X, Y, t, g["selected"], lse, 1.0)
+    assert max_rel(g["dX"], oX) <= 1e-3
+    assert max_rel(g["dY"], oY) <= 1e-3
