@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
     const int32_t* __restrict__ py, const int32_t* __restrict__ invX,
     const int32_t* __restrict__ chunkY, const int2* __restrict__ list,
-    const int32_t* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
-    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Q, int cap, int P,
+    const int4* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
+    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap, int P,
     int32_t* __restrict__ selected, float* __restrict__ lse_out, float* __restrict__ row_loss,
     uint32_t* status) {
   extern __shared__ __align__(16) uint8_t sh_raw[];
@@ -132,34 +132,45 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
   float theta_max = -INFINITY;
   for (int r = 0; r < n_r; ++r) {
     const int64_t p = invX[int64_t(r) * N + i];
-    const int cnt = list_count[int64_t(r) * N + p];
-    overflow |= cnt > Q;
+    // four sub-lists (one per epilogue warpgroup of the selection kernel)
+    const int4 c4 = list_count[int64_t(r) * N + p];
     theta_max = fmaxf(theta_max, list_theta[int64_t(r) * N + p]);
-    const int m = cnt < Q ? cnt : Q;
-    const int2* L = list + (int64_t(r) * N + p) * Q;
-    for (int a0 = 0; a0 < m; a0 += 32) {
-      const int a = a0 + lane;
-      bool keep = false;
-      uint32_t key = 0;
-      int32_t j = -1;
-      if (a < m) {
-        const int2 e = L[a];
-        j = py[int64_t(r) * C + e.y];
-        keep = j != z;
-        for (int rp = 0; rp < r && keep; ++rp) {
-          const int dc = chunkY[int64_t(rp) * C + j] - cx[rp];
-          if (dc >= -n_ec && dc <= n_ec) keep = false;
+    const int cs[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      overflow |= cs[w] > Qw;
+      const int m = cs[w] < Qw ? cs[w] : Qw;
+      const int2* L = list + ((int64_t(r) * N + p) * 4 + w) * Qw;
+      for (int a0 = 0; a0 < m; a0 += 32) {
+        const int a = a0 + lane;
+        bool keep = false;
+        uint32_t key = 0;
+        int32_t j = -1;
+        if (a < m) {
+          const int2 e = L[a];
+          j = py[int64_t(r) * C + e.y];
+          keep = j != z;
+          for (int rp = 0; rp < r && keep; ++rp) {
+            const int dc = chunkY[int64_t(rp) * C + j] - cx[rp];
+            if (dc >= -n_ec && dc <= n_ec) keep = false;
+          }
+          key = score_key(__int_as_float(e.x));
         }
-        key = score_key(__int_as_float(e.x));
+        const unsigned b = __ballot_sync(0xFFFFFFFFu, keep);
+        if (keep) {
+          const int pos = n + __popc(b & ((1u << lane) - 1u));
+          if (pos < cap) {
+            keys[pos] = key;
+            items[pos] = j;
+          }
+        }
+        n += __popc(b);
       }
-      const unsigned b = __ballot_sync(0xFFFFFFFFu, keep);
-      if (keep) {
-        const int pos = n + __popc(b & ((1u << lane) - 1u));
-        keys[pos] = key;
-        items[pos] = j;
-      }
-      n += __popc(b);
     }
+  }
+  if (n > cap) {  // more candidates than the buffer holds: keep the first cap, flag the row
+    overflow = true;
+    n = cap;
   }
   __syncwarp();
 
@@ -238,24 +249,27 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
 
 int tc_list_capacity(int k);
 
+// Candidates buffered per row: the selection emits about 1.25k + (one histogram bin) per
+// round, so 2k + 64 per round leaves ample room; a row with more is flagged inexact.
+int merge_tc_cap(int n_r, int k) { return n_r * (2 * k + 64); }
+
 size_t merge_tc_warp_bytes(int n_r, int k) {
   int P = 2;
   while (P < k) P <<= 1;
-  const size_t cap = size_t(n_r) * tc_list_capacity(k);
-  return size_t(P) * 8 + cap * 8 + 1024;
+  return size_t(P) * 8 + size_t(merge_tc_cap(n_r, k)) * 8 + 1024;
 }
 
 template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
-                            const int2* list, const int32_t* list_count,
+                            const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, float* lse,
                             float* row_loss, uint32_t* status, cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
   int P = 2;
   while (P < c.k) P <<= 1;
-  const int Q = tc_list_capacity(c.k);
+  const int Qw = tc_sublist_capacity(c.k);
   const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
   int warps = int((200 * 1024) / per_warp);
   warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
@@ -265,14 +279,14 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   if (e != cudaSuccess) return e;
   k_merge_tc<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
       X, Y, targets, py, invX, chunkY, list, list_count, list_theta, c.N, c.C, c.d, c.k, c.n_r,
-      c.n_c, c.n_ec, Q, c.n_r * Q, P, selected, lse, row_loss, status);
+      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), P, selected, lse, row_loss, status);
   count_launches(1);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_merge_tc<__nv_bfloat16>(
     const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
-    const int32_t*, const int32_t*, const int32_t*, const int2*, const int32_t*, const float*,
+    const int32_t*, const int32_t*, const int32_t*, const int2*, const int4*, const float*,
     int32_t*, float*, float*, uint32_t*, cudaStream_t);
 
 }  // namespace rece

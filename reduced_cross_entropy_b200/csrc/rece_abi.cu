@@ -79,7 +79,7 @@ void build_layout(rece_plan_s& p) {
     L.inv_x = take(sizeof(int32_t) * c.n_r * c.N);
     L.chunk_y = take(sizeof(int32_t) * c.n_r * c.C);
     L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
-    L.tc_count = take(sizeof(int32_t) * c.n_r * c.N);
+    L.tc_count = take(sizeof(int4) * c.n_r * c.N);
     L.tc_theta = take(sizeof(float) * c.n_r * c.N);
   } else {
     L.list_score = take(sizeof(float) * size_t(c.n_r) * c.N * c.k);
@@ -314,7 +314,7 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
     const __nv_bfloat16* Yb = static_cast<const __nv_bfloat16*>(Y);
     int2* list = reinterpret_cast<int2*>(ws + L.tc_list);
-    int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.tc_count);
+    int4* cnt = reinterpret_cast<int4*>(ws + L.tc_count);
     float* theta = reinterpret_cast<float*>(ws + L.tc_theta);
     stage_mark(*plan, RECE_STAGE_SELECT, 0, st);
     RECE_CUDA(launch_select_tc(*plan, ws + L.xs, ws + L.ys, list, cnt, theta, status, st),

@@ -17,7 +17,9 @@
 //           cut: every score in a bin <= b* is emitted as (score, sorted position) to the
 //           row's list (equal scores share a bin, so a tie is never split); the largest
 //           score NOT emitted is recorded.
-// The list keeps up to Q entries (Q = 2k + 64) and the count of all that passed.  The
+// Each of the four epilogue warpgroups (one per 128-column TMEM accumulator, every fourth
+// tile) writes its own sub-list of the row, up to k + 32 entries, and its count of all that
+// passed.  The
 // merge kernel keeps the k best; the selection is exact whenever no list overflowed and
 // every round's largest non-emitted score is below the k-th kept score, which the merge
 // kernel checks row by row.  Score tiles never reach HBM.
@@ -31,28 +33,35 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kPasses = 3;
 constexpr int kBins = 128;
 constexpr int kBM = 128;
-constexpr int kBN = 256;
+constexpr int kBN = 128;
 constexpr int kBK = 64;
 constexpr uint32_t kStageABytes = kBM * kBK * 2;
 constexpr uint32_t kStageBBytes = kBN * kBK * 2;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
-constexpr int kThreads = 192;
+constexpr int kAcc = 4;       // TMEM accumulators of kBN columns, one per epilogue warpgroup
+constexpr int kEpiWarps = 4 * kAcc;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;
 
 struct __align__(1024) Smem {
   uint8_t a[kStages][kStageABytes];
   uint8_t b[kStages][kStageBBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full[kAcc];
+  uint64_t acc_empty[kAcc];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  uint32_t hist[kBins][kBM];  // per row (column) gap histogram of pass 2
+  uint32_t hist[kBins][kBM];  // per row (column) histogram of pass 2
+  float part_mx[kAcc][kBM];   // pass 1 partial results of the warpgroups
+  int part_cnt[kAcc][kBM];
+  int emit_cnt[kAcc][kBM];    // pass 3 entries each warpgroup emitted, per row
+  uint32_t ne_key[kBM];       // pass 3 key of the largest score not emitted, per row
 };
 
 __device__ __forceinline__ void on_timeout(Smem& s, uint32_t* status) {
@@ -71,6 +80,10 @@ struct ItemGeom {
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return u ^ (uint32_t(int32_t(u) >> 31) | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
 __device__ __forceinline__ int64_t chunk_of(int64_t p, int64_t M, int n_c) {
@@ -92,8 +105,8 @@ __device__ __forceinline__ ItemGeom item_geom(int64_t item, int64_t tiles_per_ro
 
 __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
     const __grid_constant__ CUtensorMap tmXs, const __grid_constant__ CUtensorMap tmYs,
-    int64_t N, int64_t C, int d, int n_c, int n_ec, int n_r, int Q, int E,
-    int2* __restrict__ list, int32_t* __restrict__ list_count, float* __restrict__ list_theta,
+    int64_t N, int64_t C, int d, int n_c, int n_ec, int n_r, int Qw, int E,
+    int2* __restrict__ list, int4* __restrict__ list_count, float* __restrict__ list_theta,
     uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -108,9 +121,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAcc; ++i) {
       mbar_init(&s.acc_full[i], 1);
-      mbar_init(&s.acc_empty[i], 4);
+      mbar_init(&s.acc_empty[i], 4);  // the 4 warps of the warpgroup that owns it
     }
     mbar_init(&s.drain, 1);
     s.abort = 0;
@@ -163,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
       for (int64_t item = blockIdx.x; item < items && ok && !*abortp; item += gridDim.x) {
         const ItemGeom g = item_geom(item, tiles_per_round, N, C, n_c, n_ec);
         for (int tt = 0; tt < kPasses * g.nt && ok; ++tt, ++acc_it) {
-          const int a = acc_it & 1;
-          if (!mbar_wait(&s.acc_empty[a], ((acc_it >> 1) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+          const int a = acc_it % kAcc;
+          if (!mbar_wait(&s.acc_empty[a], ((acc_it / kAcc) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
             on_timeout(s, status);
             ok = false;
             break;
@@ -194,11 +207,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q4 = warp & 3;
+    // Warpgroup wg owns TMEM accumulator wg, i.e. every kAcc-th tile; each row has one
+    // thread in each warpgroup, combined through shared memory at pass boundaries, and
+    // each warpgroup fills its own sub-list of the row (no shared counter).
+    const int wg = (warp - 2) >> 2;
+    const int q4 = warp & 3;  // TMEM lane quarter this warp may access
     const int row_local = q4 * 32 + lane;
     uint32_t acc_it = 0;
     bool ok = true;
-    for (int64_t item = blockIdx.x; item < items && ok && !*abortp; item += gridDim.x) {
+    for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
       const ItemGeom g = item_geom(item, tiles_per_round, N, C, n_c, n_ec);
       const int64_t p = g.p0 + row_local;
       const bool valid = p < N;
@@ -210,36 +227,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
       }
       int cnt = 0;
       float mx = -INFINITY, not_emitted = -INFINITY;
-      uint32_t kmx = 0;    // key of the row's max
-      bool emit_all = false;
-      uint32_t limit = 0;  // pass 3 emits a score iff key(m) - key(s) < limit
-      int emitted = 0;
+      uint32_t kmx = 0;     // key of the row's max
+      uint32_t limit = 0;   // pass 3 emits a score iff key(m) - key(s) < limit
+      bool histo = false;   // pass 2 needed (else every window score is emitted)
       uint32_t* hcol = &s.hist[0][row_local];
-      int2* out = list + (int64_t(g.r) * N + (valid ? p : 0)) * Q;
-      for (int pass = 0; pass < kPasses && ok; ++pass) {
+      int2* out = list + ((int64_t(g.r) * N + (valid ? p : 0)) * kAcc + wg) * Qw;
+      int emitted = 0;
+      for (int pass = 0; pass < kPasses; ++pass) {
         if (pass == 1) {
-          emit_all = !valid || cnt <= E;
+          // combine the warpgroups' max / count; reset this item's shared state
+          named_barrier(1, kEpiThreads);
+          s.part_mx[wg][row_local] = mx;
+          s.part_cnt[wg][row_local] = cnt;
+          for (int b = wg * (kBins / kAcc); b < (wg + 1) * (kBins / kAcc); ++b) hcol[b * kBM] = 0;
+          if (wg == 0) s.ne_key[row_local] = 0;
+          named_barrier(1, kEpiThreads);
+          mx = s.part_mx[0][row_local];
+          cnt = s.part_cnt[0][row_local];
+#pragma unroll
+          for (int w = 1; w < kAcc; ++w) {
+            mx = fmaxf(mx, s.part_mx[w][row_local]);
+            cnt += s.part_cnt[w][row_local];
+          }
+          histo = valid && cnt > E;
           kmx = order_key(mx);
-          for (int b = 0; b < kBins; ++b) hcol[b * kBM] = 0;
-        } else if (pass == 2 && !emit_all) {
-          uint32_t cum = 0;
-          int bstar = kBins - 1;
-          for (int b = 0; b < kBins; ++b) {
-            cum += hcol[b * kBM];
-            if (cum >= uint32_t(E)) {
-              bstar = b;
-              break;
+          limit = 0xFFFFFFFFu;  // emit everything unless pass 2 finds a cut
+        } else if (pass == 2) {
+          named_barrier(1, kEpiThreads);  // every histogram increment has landed
+          if (histo) {
+            uint32_t cum = 0;
+            for (int b = 0; b < kBins - 1; ++b) {
+              cum += hcol[b * kBM];
+              if (cum >= uint32_t(E)) {
+                limit = uint32_t(b + 1) << 20;
+                break;
+              }
             }
           }
-          if (bstar >= kBins - 1) emit_all = true;
-          else limit = uint32_t(bstar + 1) << 20;
         }
         for (int t = 0; t < g.nt; ++t, ++acc_it) {
-          const int a = acc_it & 1;
-          if (!mbar_wait(&s.acc_full[a], (acc_it >> 1) & 1u, &s.abort, kTimeoutNs)) {
-            on_timeout(s, status);
+          const int a = acc_it % kAcc;
+          if (a != wg) continue;  // another warpgroup's tile
+          if (!ok || !mbar_wait(&s.acc_full[a], (acc_it / kAcc) & 1u, &s.abort, kTimeoutNs)) {
+            if (ok) on_timeout(s, status);
             ok = false;
-            break;
+            continue;  // keep the loop structure so every barrier is still met
           }
           tc_fence_after();
           const int64_t q0 = g.U0 + int64_t(t) * kBN;
@@ -247,45 +279,50 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 32) {
             const int64_t qa = q0 + c0;
-            const bool need = valid && qa < w1 && qa + 32 > w0 && !(pass == 1 && emit_all);
+            const bool need = valid && qa < w1 && qa + 32 > w0 && (pass != 1 || histo);
             if (!__any_sync(0xFFFFFFFFu, need)) continue;
             float v[32];
             tmem_load32(taddr + c0, v);
             if (!need) continue;
-            const bool inside = qa >= w0 && qa + 32 <= w1;
-            if (pass == 0) {
-              if (inside) {
+            if (qa >= w0 && qa + 32 <= w1) {
+              // chunk entirely inside the row's window: no per-column test
+              if (pass == 0) {
                 cnt += 32;
+                float m4[4] = {mx, v[0], v[1], v[2]};
 #pragma unroll
-                for (int u = 0; u < 32; ++u) mx = fmaxf(mx, v[u]);
+                for (int u = 3; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+              } else if (pass == 1) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  const uint32_t raw = (kmx - order_key(v[u])) >> 20;
+                  atomicAdd(&hcol[min(raw, uint32_t(kBins - 1)) * kBM], 1u);
+                }
               } else {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                  if (qa + u >= w0 && qa + u < w1) {
-                    ++cnt;
-                    mx = fmaxf(mx, v[u]);
-                  }
-                }
-              }
-            } else if (pass == 1) {
-#pragma unroll
-              for (int u = 0; u < 32; ++u) {
-                if (inside || (qa + u >= w0 && qa + u < w1)) {
-                  const uint32_t raw = (kmx - order_key(v[u])) >> 20;
-                  hcol[(raw < kBins - 1 ? raw : kBins - 1) * kBM] += 1u;
+                  const bool e = kmx - order_key(v[u]) < limit;
+                  if (e && emitted < Qw) out[emitted] = make_int2(__float_as_int(v[u]), int32_t(qa + u));
+                  emitted += e ? 1 : 0;
+                  not_emitted = e ? not_emitted : fmaxf(not_emitted, v[u]);
                 }
               }
             } else {
+              const int lo = int(w0 > qa ? w0 - qa : 0), hi = int(w1 < qa + 32 ? w1 - qa : 32);
 #pragma unroll
               for (int u = 0; u < 32; ++u) {
-                if (inside || (qa + u >= w0 && qa + u < w1)) {
-                  if (emit_all || kmx - order_key(v[u]) < limit) {
-                    if (emitted < Q)
-                      out[emitted] = make_int2(__float_as_int(v[u]), int32_t(qa + u));
-                    ++emitted;
-                  } else {
-                    not_emitted = fmaxf(not_emitted, v[u]);
-                  }
+                if (u < lo || u >= hi) continue;
+                if (pass == 0) {
+                  ++cnt;
+                  mx = fmaxf(mx, v[u]);
+                } else if (pass == 1) {
+                  const uint32_t raw = (kmx - order_key(v[u])) >> 20;
+                  atomicAdd(&hcol[min(raw, uint32_t(kBins - 1)) * kBM], 1u);
+                } else {
+                  const bool e = kmx - order_key(v[u]) < limit;
+                  if (e && emitted < Qw) out[emitted] = make_int2(__float_as_int(v[u]), int32_t(qa + u));
+                  emitted += e ? 1 : 0;
+                  not_emitted = e ? not_emitted : fmaxf(not_emitted, v[u]);
                 }
               }
             }
@@ -295,9 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           if (lane == 0) mbar_arrive(&s.acc_empty[a]);
         }
       }
-      if (ok && valid) {
-        list_count[int64_t(g.r) * N + p] = emitted;
-        list_theta[int64_t(g.r) * N + p] = not_emitted;
+      if (not_emitted > -INFINITY) atomicMax(&s.ne_key[row_local], order_key(not_emitted));
+      s.emit_cnt[wg][row_local] = emitted;
+      named_barrier(1, kEpiThreads);
+      if (wg == 0 && ok && valid) {
+        const uint32_t nk2 = s.ne_key[row_local];
+        list_count[int64_t(g.r) * N + p] = make_int4(s.emit_cnt[0][row_local], s.emit_cnt[1][row_local],
+                                                     s.emit_cnt[2][row_local], s.emit_cnt[3][row_local]);
+        list_theta[int64_t(g.r) * N + p] = nk2 == 0 ? -INFINITY : key_to_float(nk2);
       }
     }
   }
@@ -312,11 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
 
 }  // namespace
 
-int tc_list_capacity(int k) { return 2 * k + 64; }
+// Capacity of each warpgroup's sub-list of a (round, row): a warpgroup sees a quarter of
+// the window, so k + 32 leaves wide room above its share of the ~1.25k emitted scores.
+int tc_sublist_capacity(int k) { return k + 32; }
+int tc_list_capacity(int k) { return kAcc * tc_sublist_capacity(k); }
 int tc_emit_target(int k) { return k + k / 4 + 8; }
 
 cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys, int2* list,
-                             int32_t* list_count, float* list_theta, uint32_t* status,
+                             int4* list_count, float* list_theta, uint32_t* status,
                              cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
@@ -331,7 +376,7 @@ cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Y
   e = cudaFuncSetAttribute(k_select_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   k_select_tc<<<grid, kThreads, smem, st>>>(tmXs, tmYs, c.N, c.C, c.d, c.n_c, c.n_ec, c.n_r,
-                                            tc_list_capacity(c.k), tc_emit_target(c.k), list,
+                                            tc_sublist_capacity(c.k), tc_emit_target(c.k), list,
                                             list_count, list_theta, status);
   count_launches(1);
   return cudaGetLastError();

@@ -30,9 +30,10 @@ cudaError_t launch_permute_rows(const void* V, int64_t M, int d, const int32_t* 
 
 // K3 on tensor cores: per (round, sorted row) the candidate list (score bits, sorted
 // catalogue position), its count and threshold.
-int tc_list_capacity(int k);
+int tc_list_capacity(int k);      // entries per (round, row): 4 sub-lists
+int tc_sublist_capacity(int k);   // entries per sub-list
 cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys, int2* list,
-                             int32_t* list_count, float* list_theta, uint32_t* status,
+                             int4* list_count, float* list_theta, uint32_t* status,
                              cudaStream_t st);
 
 // K4 for the tensor-core lists: merge, select, order, loss, exactness check.
@@ -40,7 +41,7 @@ size_t merge_tc_warp_bytes(int n_r, int k);
 template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
-                            const int2* list, const int32_t* list_count,
+                            const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, float* lse,
                             float* row_loss, uint32_t* status, cudaStream_t st);
 
