@@ -2,12 +2,16 @@
 // restricted to the positive and the kept negatives; selection held constant).
 //
 //   g_ij = (exp(l_ij - lse_i) - [j == z_i]) * dloss / N
-//   dX_i = sum_j g_ij y_j          (one warp per row, slots in order: deterministic)
+//   dX_i = sum_j g_ij y_j          (one warp per row: every lane computes whole dot
+//                                   products for its own slots, then the lanes sweep the
+//                                   dimensions adding the slots in order)
 //   dY_j = sum_i g_ij x_i          (no float atomics: the (item, row) pairs are put in
-//                                   item order by a stable LSD radix sort, then every
-//                                   item sums its pairs in row order)
+//                                   item order by a stable LSD radix sort that carries g
+//                                   along, then one warp per item sums its pairs in row
+//                                   order)
 // Pair e = i*(k+1) + s holds slot s of row i (s = 0: the positive, s >= 1: selected
-// negative s-1); an empty slot carries the key C, which sorts after every item.
+// negative s-1); an empty slot carries the key C, which sorts after every item.  Every
+// sum has a fixed order: the gradients are deterministic.
 #include "common.cuh"
 #include "plan.h"
 
@@ -16,15 +20,32 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <typename T>
-__device__ __forceinline__ float warp_dot(const T* __restrict__ a, const T* __restrict__ b,
-                                          int d, int lane) {
-  float s = 0.0f;
-  for (int t = lane; t < d; t += 32) s = fmaf(to_f32(a[t]), to_f32(b[t]), s);
-  return warp_sum(s);
+__device__ __forceinline__ float2 load_pair(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+__device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// One warp per row: coefficients g of every slot, the pair keys, and dX_i.
+// <x, y> with x in shared memory (fp32) and y a catalogue row, t ascending.
+template <typename T>
+__device__ __forceinline__ float dot_row(const float* xs, const T* __restrict__ y, int d) {
+  float s = 0.0f;
+  if ((d & 7) == 0) {
+    for (int t = 0; t < d; t += 8) {
+      float v[8];
+      load8(y + t, v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s = fmaf(xs[t + u], v[u], s);
+    }
+  } else {
+    for (int t = 0; t < d; ++t) s = fmaf(xs[t], to_f32(y[t]), s);
+  }
+  return s;
+}
+
+// One warp per row; shared memory per warp: x (d floats), g and item of every slot.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_rows(
     const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
@@ -32,95 +53,118 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
     const float* __restrict__ dloss, int64_t N, int64_t C, int d, int k,
     int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
     uint32_t* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t i = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
-  if (i >= N) return;
+  extern __shared__ __align__(16) float sh_f[];
+  const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slots = k + 1;
+  const int per_warp = d + 2 * slots;
+  float* xs = sh_f + size_t(per_warp) * wid;
+  float* gs = xs + d;
+  int32_t* js = reinterpret_cast<int32_t*>(gs + slots);
+  const int64_t i = int64_t(blockIdx.x) * warps + wid;
+  if (i >= N) return;  // the warp leaves together; no block-wide barrier follows
   const float scale = dloss[0] / float(N);
   const float li = lse[i];
-  const T* x = X + i * d;
-  const int slots = k + 1;
-  int32_t* keys = e_key + i * slots;
-  float* gs = e_g + i * slots;
-  for (int s = 0; s < slots; ++s) {
+  for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
+  __syncwarp();
+
+  // coefficients: one slot per lane at a time
+  for (int s = lane; s < slots; s += 32) {
     int32_t j = s == 0 ? targets[i] : selected[i * k + (s - 1)];
     float g = 0.0f;
     if (j >= 0 && j < C) {
-      const float l = warp_dot(x, Y + int64_t(j) * d, d, lane);
-      const float p = expf(l - li);
+      const float p = expf(dot_row(xs, Y + int64_t(j) * d, d) - li);
       g = (s == 0 ? p - 1.0f : p) * scale;
     } else {
-      if (s == 0 && lane == 0) raise_flag(status, RECE_DEVICE_BAD_TARGET);
-      j = int32_t(C);
+      if (s == 0) raise_flag(status, RECE_DEVICE_BAD_TARGET);
+      j = -1;
     }
-    if (lane == 0) {
-      keys[s] = j;
-      gs[s] = g;
-    }
+    gs[s] = g;
+    js[s] = j;
+    e_key[i * slots + s] = j < 0 ? int32_t(C) : j;
+    e_g[i * slots + s] = g;
   }
   __syncwarp();
-  for (int t0 = 0; t0 < d; t0 += 32 * 4) {
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int s = 0; s < slots; ++s) {
-      const int32_t j = keys[s];
-      if (j >= C) continue;
-      const float g = gs[s];
-      const T* y = Y + int64_t(j) * d;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = t0 + u * 32 + lane;
-        if (t < d) acc[u] = fmaf(g, to_f32(y[t]), acc[u]);
+
+  // dX_i: lanes over dimensions (two each), slots in order
+  if ((d & 1) == 0) {
+    for (int t0 = 0; t0 < d; t0 += 64) {
+      const int t = t0 + 2 * lane;
+      float a0 = 0.0f, a1 = 0.0f;
+      if (t < d) {
+#pragma unroll 4
+        for (int s = 0; s < slots; ++s) {
+          const int32_t j = js[s];
+          if (j < 0) continue;
+          const float g = gs[s];
+          const float2 y = load_pair(Y + int64_t(j) * d + t);
+          a0 = fmaf(g, y.x, a0);
+          a1 = fmaf(g, y.y, a1);
+        }
+        *reinterpret_cast<float2*>(dX + i * d + t) = make_float2(a0, a1);
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int t = t0 + u * 32 + lane;
-      if (t < d) dX[i * d + t] = acc[u];
+  } else {
+    for (int t = lane; t < d; t += 32) {
+      float a = 0.0f;
+      for (int s = 0; s < slots; ++s) {
+        const int32_t j = js[s];
+        if (j >= 0) a = fmaf(gs[s], to_f32(Y[int64_t(j) * d + t]), a);
+      }
+      dX[i * d + t] = a;
     }
   }
 }
 
-__device__ __forceinline__ int64_t lower_bound(const int32_t* a, int64_t n, int32_t v) {
-  int64_t lo = 0, hi = n;
-  while (lo < hi) {
-    const int64_t mid = (lo + hi) >> 1;
-    if (a[mid] < v) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
-
-// One warp per item: dY_j = sum over its pairs (row order) of g * x_row.
+// One warp per item: dY_j = sum over its pairs (row order) of g * x_row.  The pairs are
+// read 32 at a time (entry id and g, contiguous), then broadcast one by one.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_items(
-    const T* __restrict__ X, int64_t C, int d, int k, int64_t E,
-    const int32_t* __restrict__ sorted_key, const int32_t* __restrict__ order,
-    const float* __restrict__ e_g, float* __restrict__ dY) {
+    const T* __restrict__ X, int64_t C, int d, int k, const int32_t* __restrict__ item_start,
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ sorted_g,
+    float* __restrict__ dY) {
   const int lane = threadIdx.x & 31;
   const int64_t j = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
   if (j >= C) return;
-  const int64_t lo = lower_bound(sorted_key, E, int32_t(j));
-  const int64_t hi = lower_bound(sorted_key, E, int32_t(j + 1));
+  const int64_t lo = item_start[j], hi = item_start[j + 1];
   const int slots = k + 1;
-  for (int t0 = 0; t0 < d; t0 += 32 * 4) {
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int64_t p = lo; p < hi; ++p) {
-      const int32_t e = order[p];
-      const float g = e_g[e];
-      const T* x = X + int64_t(e / slots) * d;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = t0 + u * 32 + lane;
-        if (t < d) acc[u] = fmaf(g, to_f32(x[t]), acc[u]);
+  const bool pairs = (d & 1) == 0;
+  const int step = pairs ? 64 : 32;
+  for (int t0 = 0; t0 < d; t0 += step) {
+    const int t = pairs ? t0 + 2 * lane : t0 + lane;
+    float a0 = 0.0f, a1 = 0.0f;
+    for (int64_t b = lo; b < hi; b += 32) {
+      const int n = int(hi - b < 32 ? hi - b : 32);
+      int32_t row = 0;
+      float g = 0.0f;
+      if (lane < n) {
+        row = sorted_id[b + lane] / slots;
+        g = sorted_g[b + lane];
+      }
+#pragma unroll 4
+      for (int q = 0; q < n; ++q) {
+        const int32_t r = __shfl_sync(0xFFFFFFFFu, row, q);
+        const float gq = __shfl_sync(0xFFFFFFFFu, g, q);
+        if (t < d) {
+          if (pairs) {
+            const float2 x = load_pair(X + int64_t(r) * d + t);
+            a0 = fmaf(gq, x.x, a0);
+            a1 = fmaf(gq, x.y, a1);
+          } else {
+            a0 = fmaf(gq, to_f32(X[int64_t(r) * d + t]), a0);
+          }
+        }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int t = t0 + u * 32 + lane;
-      if (t < d) dY[j * d + t] = acc[u];
+    if (t < d) {
+      if (pairs) *reinterpret_cast<float2*>(dY + j * d + t) = make_float2(a0, a1);
+      else dY[j * d + t] = a0;
     }
   }
 }
 
 }  // namespace
+
+size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 * (k + 1)); }
 
 template <typename T>
 cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
@@ -135,34 +179,57 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   int32_t* perm_a = reinterpret_cast<int32_t*>(ws + L.e_perm_a);
   int32_t* perm_b = reinterpret_cast<int32_t*>(ws + L.e_perm_b);
   int32_t* sorted_key = reinterpret_cast<int32_t*>(ws + L.e_sorted_key);
+  float* sorted_g = reinterpret_cast<float*>(ws + L.e_sorted_g);
   void* scratch = ws + L.e_scratch;
-  const int warps = kThreads / 32;
   stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
   if (c.N > 0) {
-    k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), kThreads, 0, st>>>(
+    const size_t per_warp = bwd_rows_warp_bytes(c.d, c.k);
+    int warps = int((200 * 1024) / per_warp);
+    warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
+    const size_t smem = per_warp * warps;
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_rows<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
         X, Y, targets, selected, lse, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX, status);
     count_launches(1);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
-  // LSD radix sort of the pairs by item key (values 0..C), 8 bits per pass
+  // LSD radix sort of the pairs by item key (values 0..C), as few passes as the
+  // counting sort's 12-bit digit limit allows.  Every pass writes keys and g in its output
+  // order, so the next pass reads them contiguously; the ids say where each pair came from.
+  int32_t* key_buf[2] = {reinterpret_cast<int32_t*>(ws + L.e_key_b), sorted_key};
+  float* g_buf[2] = {reinterpret_cast<float*>(ws + L.e_g_b), sorted_g};
+  const int passes = p.item_passes;
   const int32_t* in = nullptr;
+  const int32_t* kin = e_key;
+  const float* gin = e_g;
   int32_t* out = perm_a;
-  for (int shift = 0; shift < p.item_bits; shift += 8) {
-    const int bits = min(8, p.item_bits - shift);
-    const bool last = shift + 8 >= p.item_bits;
-    cudaError_t e = launch_sort_pass(e_key, in, E, shift, bits, scratch, out,
-                                     last ? sorted_key : nullptr, nullptr, st);
+  int shift = 0;
+  for (int ps = 0; ps < passes; ++ps) {
+    const int bits = (ps + 1 < passes) ? p.item_pass_bits : p.item_bits - shift;
+    // the last pass lands in sorted_key / sorted_g
+    const int slot = (passes - 1 - ps) % 2 == 0 ? 1 : 0;
+    cudaError_t e = launch_sort_pass(kin, in, E, shift, bits, scratch, out, key_buf[slot],
+                                     nullptr, st, gin, g_buf[slot], ps > 0);
     if (e != cudaSuccess) return e;
+    shift += bits;
     in = out;
+    kin = key_buf[slot];
+    gin = g_buf[slot];
     out = (out == perm_a) ? perm_b : perm_a;
   }
+  int32_t* item_start = reinterpret_cast<int32_t*>(ws + L.e_item_start);
+  cudaError_t e2 = launch_segment_starts(sorted_key, E, int32_t(c.C), item_start, st);
+  if (e2 != cudaSuccess) return e2;
   stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
-  k_bwd_items<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(X, c.C, c.d, c.k, E,
-                                                                      sorted_key, in, e_g, dY);
+  const int warps = kThreads / 32;
+  k_bwd_items<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
+      X, c.C, c.d, c.k, item_start, in, sorted_g, dY);
   count_launches(1);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
   return cudaGetLastError();

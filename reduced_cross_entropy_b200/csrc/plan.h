@@ -40,7 +40,8 @@ struct Layout {
   size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0;
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
-  size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_scratch = 0;
+  size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_sorted_g = 0,
+         e_key_b = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0;
   size_t bwd_end = 0;
   size_t total = 0;
 };
@@ -55,6 +56,8 @@ struct rece_plan_s {
   int32_t sel_rows;     // rows per CTA of the exact selection kernel
   int32_t bucket_bits;  // digit bits of the bucket sort
   int32_t item_bits;    // key bits of the backward item sort (values 0..C)
+  int32_t item_passes;  // LSD passes of that sort (digits of at most 12 bits)
+  int32_t item_pass_bits;  // digit bits of every pass but the last
   int64_t entries;      // N * (k + 1): (row, item) pairs of the backward
   bool use_tc;          // bf16 mode on the tcgen05 kernels
   rece::Layout lay;
@@ -82,12 +85,22 @@ cudaError_t launch_bucketize_fma(const T* V, int64_t M, int d, const T* B, int n
 
 // K2: one stable counting-sort pass over M elements.  Element p carries id
 // (in_ids ? in_ids[p] : p) and key keys[id]; it is ordered by digit (key >> shift) &
-// ((1 << bits) - 1).  Writes out_ids (the new order of ids), optionally the sorted
-// digit-keys (out_keys[p] = keys[out_ids[p]]) and digit_start[0..2^bits] (first output
-// position of every digit; digit_start[2^bits] = M).
+// ((1 << bits) - 1).  Writes out_ids (the new order of ids), optionally the sorted keys
+// (out_keys[p] = keys[out_ids[p]]), a carried payload (out_payload[p] =
+// payload[out_ids[p]]) and digit_start[0..2^bits] (first output position of every digit;
+// digit_start[2^bits] = M).
+// With in_order, element p's key and payload are keys[p] and payload[p] (a previous pass
+// wrote them in the order of its output) instead of being looked up by id.
 cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,
                              int bits, void* scratch, int32_t* out_ids, int32_t* out_keys,
-                             int32_t* digit_start, cudaStream_t st);
+                             int32_t* digit_start, cudaStream_t st,
+                             const float* payload = nullptr, float* out_payload = nullptr,
+                             bool in_order = false);
+
+// start[j] = first position of a key >= j in the sorted keys, for j = 0..n_vals (so the
+// keys equal to j occupy [start[j], start[j+1])).
+cudaError_t launch_segment_starts(const int32_t* sorted, int64_t M, int32_t n_vals,
+                                  int32_t* start, cudaStream_t st);
 
 // K3 (fmaf-chain CUDA-core version): per-round top-k lists of every row.
 template <typename T>

@@ -94,7 +94,11 @@ void build_layout(rece_plan_s& p) {
   L.e_perm_a = take(sizeof(int32_t) * E);
   L.e_perm_b = take(sizeof(int32_t) * E);
   L.e_sorted_key = take(sizeof(int32_t) * E);
-  L.e_scratch = take(sort_scratch_bytes(p.entries, 8));
+  L.e_sorted_g = take(sizeof(float) * E);
+  L.e_key_b = take(sizeof(int32_t) * E);
+  L.e_g_b = take(sizeof(float) * E);
+  L.e_item_start = take(sizeof(int32_t) * (size_t(c.C) + 1));
+  L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
@@ -174,6 +178,9 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   }
   p->bucket_bits = bits_for(c.n_b);
   p->item_bits = bits_for(c.C + 1);
+  p->item_passes = int32_t((p->item_bits + kMaxDigitBits - 1) / kMaxDigitBits);
+  if (p->item_passes < 1) p->item_passes = 1;
+  p->item_pass_bits = (p->item_bits + p->item_passes - 1) / p->item_passes;
   p->entries = c.N * (int64_t(c.k) + 1);
   p->timed = false;
   for (void*& e : p->stage_events) e = nullptr;

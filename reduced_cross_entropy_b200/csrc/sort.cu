@@ -22,12 +22,18 @@ constexpr int kSteps = kPerWarp / 32;          // 16
 __device__ __forceinline__ int32_t elem_id(const int32_t* in_ids, int64_t p) {
   return in_ids ? in_ids[p] : int32_t(p);
 }
+// Key (and payload) of the element at position p: stored by id, or already in the order
+// of the positions (in_order: a previous pass wrote them permuted).
+__device__ __forceinline__ int32_t elem_key(const int32_t* keys, const int32_t* in_ids,
+                                            int64_t p, bool in_order) {
+  return in_order ? keys[p] : keys[elem_id(in_ids, p)];
+}
 
 __global__ void __launch_bounds__(kSortThreads) k_sort_hist(const int32_t* __restrict__ keys,
                                                             const int32_t* __restrict__ in_ids,
                                                             int64_t M, int shift, int bits,
                                                             int32_t* __restrict__ hist,
-                                                            int64_t tiles) {
+                                                            int64_t tiles, bool in_order) {
   extern __shared__ int32_t sh_cnt[];
   const int digits = 1 << bits, mask = digits - 1;
   for (int i = threadIdx.x; i < digits; i += blockDim.x) sh_cnt[i] = 0;
@@ -35,7 +41,7 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_hist(const int32_t* __res
   const int64_t base = int64_t(blockIdx.x) * kSortTile;
   for (int e = threadIdx.x; e < kSortTile; e += blockDim.x) {
     const int64_t p = base + e;
-    if (p < M) atomicAdd(&sh_cnt[(keys[elem_id(in_ids, p)] >> shift) & mask], 1);
+    if (p < M) atomicAdd(&sh_cnt[(elem_key(keys, in_ids, p, in_order) >> shift) & mask], 1);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < digits; i += blockDim.x)
@@ -111,7 +117,8 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
     const int32_t* __restrict__ keys, const int32_t* __restrict__ in_ids, int64_t M, int shift,
     int bits, const int32_t* __restrict__ hist, int64_t tiles,
     const int32_t* __restrict__ digit_start, int32_t* __restrict__ out_ids,
-    int32_t* __restrict__ out_keys) {
+    int32_t* __restrict__ out_keys, const float* __restrict__ payload,
+    float* __restrict__ out_payload, bool in_order) {
   extern __shared__ __align__(16) unsigned char sh_raw[];
   const int digits = 1 << bits, mask = digits - 1;
   uint16_t* cnt = reinterpret_cast<uint16_t*>(sh_raw);  // [kWarps][digits]
@@ -131,7 +138,8 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
   for (int s = 0; s < kSteps; ++s) {
     const int64_t p = wbase + s * 32 + lane;
     const bool ok = p < M;
-    const int dg = ok ? ((keys[elem_id(in_ids, p)] >> shift) & mask) : (0x40000000 | lane);
+    const int dg = ok ? ((elem_key(keys, in_ids, p, in_order) >> shift) & mask)
+                      : (0x40000000 | lane);
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
     if (ok && lane == __ffs(peers) - 1) wcnt[dg] += uint16_t(__popc(peers));
     __syncwarp();
@@ -154,7 +162,7 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
     int32_t id = 0, key = 0;
     if (ok) {
       id = elem_id(in_ids, p);
-      key = keys[id];
+      key = in_order ? keys[p] : keys[id];
     }
     const int dg = ok ? ((key >> shift) & mask) : (0x40000000 | lane);
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
@@ -165,17 +173,39 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
       const int64_t pos = int64_t(tile_base[dg]) + base + rank;
       out_ids[pos] = id;
       if (out_keys) out_keys[pos] = key;
+      if (out_payload) out_payload[pos] = in_order ? payload[p] : payload[id];
       if (lane == __ffs(peers) - 1) wcnt[dg] = uint16_t(base + __popc(peers));
     }
     __syncwarp();
   }
 }
 
+// start[j] = first position p of sorted (non-decreasing) keys with key >= j, j in [0, n_vals]:
+// thread p fills the starts of the values between key[p-1] and key[p].
+__global__ void __launch_bounds__(256) k_segment_starts(const int32_t* __restrict__ sorted,
+                                                        int64_t M, int32_t n_vals,
+                                                        int32_t* __restrict__ start) {
+  const int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (p > M) return;
+  const int32_t prev = p > 0 ? sorted[p - 1] : -1;
+  int32_t cur = p < M ? sorted[p] : n_vals;
+  if (cur > n_vals) cur = n_vals;
+  for (int32_t j = prev + 1; j <= cur; ++j) start[j] = int32_t(p);
+}
+
 }  // namespace
+
+cudaError_t launch_segment_starts(const int32_t* sorted, int64_t M, int32_t n_vals,
+                                  int32_t* start, cudaStream_t st) {
+  k_segment_starts<<<unsigned(ceil_div(M + 1, 256)), 256, 0, st>>>(sorted, M, n_vals, start);
+  count_launches(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,
                              int bits, void* scratch, int32_t* out_ids, int32_t* out_keys,
-                             int32_t* digit_start, cudaStream_t st) {
+                             int32_t* digit_start, cudaStream_t st, const float* payload,
+                             float* out_payload, bool in_order) {
   const int digits = 1 << bits;
   const int64_t tiles = ceil_div(M > 0 ? M : 1, kSortTile);
   int32_t* hist = static_cast<int32_t*>(scratch);
@@ -188,7 +218,7 @@ cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t
     return cudaSuccess;
   }
   k_sort_hist<<<unsigned(tiles), kSortThreads, sizeof(int32_t) * digits, st>>>(
-      keys, in_ids, M, shift, bits, hist, tiles);
+      keys, in_ids, M, shift, bits, hist, tiles, in_order);
   k_sort_scan_tiles<<<digits, 256, 0, st>>>(hist, tiles, start);
   k_sort_scan_digits<<<1, 1024, 0, st>>>(start, digits);
   const size_t smem = ((kWarps * digits * sizeof(uint16_t) + 15) & ~size_t(15)) +
@@ -199,7 +229,8 @@ cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t
       int(sizeof(uint16_t) * kWarps * (1 << kMaxDigitBits) + sizeof(int32_t) * (1 << kMaxDigitBits) + 16));
   if (e != cudaSuccess) return e;
   k_sort_scatter<<<unsigned(tiles), kSortThreads, smem, st>>>(
-      keys, in_ids, M, shift, bits, hist, tiles, start, out_ids, out_keys);
+      keys, in_ids, M, shift, bits, hist, tiles, start, out_ids, out_keys, payload, out_payload,
+      in_order);
   count_launches(4);
   return cudaGetLastError();
 }
