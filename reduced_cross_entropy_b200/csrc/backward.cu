@@ -162,6 +162,149 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items(
   }
 }
 
+// ---------------------------------------------------------------- d % 8 == 0 kernels
+// Eight lanes (a "quarter" of the warp) share one catalogue / input row: lane `sub` of
+// quarter q covers dims 8*sub + 64*m, one 16-byte vector (bf16) or two (fp32) each, so a
+// warp-wide load touches four whole rows.  The quarters take every fourth slot / pair and
+// are added at the end in a fixed order (q0+q1)+(q2+q3): still deterministic.
+
+template <typename T>
+__device__ __forceinline__ void load8v(const T* p, float (&v)[8]) { load8(p, v); }
+
+// One warp per row.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
+    const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
+    const int32_t* __restrict__ selected, const float* __restrict__ lse,
+    const float* __restrict__ dloss, int64_t N, int64_t C, int d, int k,
+    int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
+    uint32_t* status) {
+  extern __shared__ __align__(16) float sh_f[];
+  const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = lane >> 3, sub = lane & 7;
+  const int slots = k + 1;
+  const int per_warp = d + 2 * slots;
+  float* xs = sh_f + size_t(per_warp) * wid;
+  float* gs = xs + d;
+  int32_t* js = reinterpret_cast<int32_t*>(gs + slots);
+  const int64_t i = int64_t(blockIdx.x) * warps + wid;
+  if (i >= N) return;  // the warp leaves together; no block-wide barrier follows
+  const float scale = dloss[0] / float(N);
+  const float li = lse[i];
+  for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
+  __syncwarp();
+
+  // coefficients: four slots per step, one per quarter
+  for (int s0 = 0; s0 < slots; s0 += 4) {
+    const int s = s0 + q;
+    int32_t j = -1;
+    if (s < slots) j = s == 0 ? targets[i] : selected[i * k + (s - 1)];
+    const bool ok = j >= 0 && j < C;
+    float part = 0.0f;
+    if (ok) {
+      const T* y = Y + int64_t(j) * d;
+      for (int t = 8 * sub; t < d; t += 64) {
+        float v[8];
+        load8v(y + t, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part = fmaf(xs[t + u], v[u], part);
+      }
+    }
+    part += __shfl_xor_sync(0xFFFFFFFFu, part, 4);
+    part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
+    part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
+    if (sub == 0 && s < slots) {
+      float g = 0.0f;
+      if (ok) {
+        const float p = expf(part - li);
+        g = (s == 0 ? p - 1.0f : p) * scale;
+      } else if (s == 0) {
+        raise_flag(status, RECE_DEVICE_BAD_TARGET);
+      }
+      gs[s] = g;
+      js[s] = ok ? j : -1;
+      e_key[i * slots + s] = ok ? j : int32_t(C);
+      e_g[i * slots + s] = g;
+    }
+  }
+  __syncwarp();
+
+  // dX_i: quarter q adds the slots s = q (mod 4) in order over its lane's 8 dims
+  for (int t0 = 0; t0 < d; t0 += 64) {
+    const int t = t0 + 8 * sub;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (t < d) {
+#pragma unroll 2
+      for (int s = q; s < slots; s += 4) {
+        const int32_t j = js[s];
+        if (j < 0) continue;
+        const float g = gs[s];
+        float v[8];
+        load8v(Y + int64_t(j) * d + t, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = fmaf(g, v[u], acc[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], 8);
+      acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], 16);
+    }
+    if (q == 0 && t < d) {
+      float4* o = reinterpret_cast<float4*>(dX + i * d + t);
+      o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+}
+
+// One warp per item; quarter q adds the pairs b = lo + q (mod 4) in row order.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
+    const T* __restrict__ X, int64_t C, int d, int k, const int32_t* __restrict__ item_start,
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ sorted_g,
+    float* __restrict__ dY) {
+  const int lane = threadIdx.x & 31, q = lane >> 3, sub = lane & 7;
+  const int64_t j = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  if (j >= C) return;
+  const int64_t lo = item_start[j], hi = item_start[j + 1];
+  const int slots = k + 1;
+  for (int t0 = 0; t0 < d; t0 += 64) {
+    const int t = t0 + 8 * sub;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int64_t b = lo; b < hi; b += 32) {
+      const int n = int(hi - b < 32 ? hi - b : 32);
+      int32_t row = 0;
+      float g = 0.0f;
+      if (lane < n) {
+        row = sorted_id[b + lane] / slots;
+        g = sorted_g[b + lane];
+      }
+      for (int e0 = 0; e0 < n; e0 += 4) {
+        const int e = e0 + q;
+        const int32_t r = __shfl_sync(0xFFFFFFFFu, row, e & 31);
+        const float ge = __shfl_sync(0xFFFFFFFFu, g, e & 31);
+        if (e < n && t < d) {
+          float v[8];
+          load8v(X + int64_t(r) * d + t, v);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[u] = fmaf(ge, v[u], acc[u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], 8);
+      acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], 16);
+    }
+    if (q == 0 && t < d) {
+      float4* o = reinterpret_cast<float4*>(dY + j * d + t);
+      o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+}
+
 }  // namespace
 
 size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 * (k + 1)); }
@@ -187,11 +330,16 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
     int warps = int((200 * 1024) / per_warp);
     warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
     const size_t smem = per_warp * warps;
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_rows<T>,
+    const bool v8 = (c.d % 8) == 0;
+    cudaError_t e = cudaFuncSetAttribute(v8 ? k_bwd_rows_v8<T> : k_bwd_rows<T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
-        X, Y, targets, selected, lse, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX, status);
+    if (v8)
+      k_bwd_rows_v8<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
+          X, Y, targets, selected, lse, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX, status);
+    else
+      k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
+          X, Y, targets, selected, lse, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX, status);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -228,8 +376,12 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
   const int warps = kThreads / 32;
-  k_bwd_items<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
-      X, c.C, c.d, c.k, item_start, in, sorted_g, dY);
+  if (c.d % 8 == 0)
+    k_bwd_items_v8<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
+        X, c.C, c.d, c.k, item_start, in, sorted_g, dY);
+  else
+    k_bwd_items<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
+        X, c.C, c.d, c.k, item_start, in, sorted_g, dY);
   count_launches(1);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
   return cudaGetLastError();
