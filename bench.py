@@ -97,16 +97,15 @@ def stage_work(w):
     }
 
 
-def stage_bound(stage, flags, dtype):
+def uses_tensor_cores(w, flags):
+    """bf16 mode without RECE_FLAG_FMA_SCORES and d a multiple of 64: tcgen05 kernels."""
+    return w.dtype == "bf16" and not (flags & 1) and w.d % 64 == 0
+
+
+def stage_bound(stage, w, flags):
     if stage in ("bucketize", "select"):
-        if dtype == "bf16" and not (flags & 1) and TENSOR_STAGES.get(stage, False):
-            return "tensor"
-        return "alu"
+        return "tensor" if uses_tensor_cores(w, flags) else "alu"
     return "hbm"
-
-
-# stages that run on tcgen05 in bf16 mode (without RECE_FLAG_FMA_SCORES)
-TENSOR_STAGES = {}
 
 
 KERNEL_SOURCES = {
@@ -360,7 +359,7 @@ def main():
     peaks = load_peaks()
     work = stage_work(w)
     dom = max(stage_ms, key=stage_ms.get)
-    bound = stage_bound(dom, args.flags, w.dtype)
+    bound = stage_bound(dom, w, args.flags)
     flops, bytes_ = work[dom]
     sec = stage_ms[dom] / 1000.0
     if bound == "hbm":
@@ -415,8 +414,8 @@ def main():
             "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": workload_desc(w),
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "scores": "fmaf CUDA cores" if (args.flags & 1 or
-                                                       not TENSOR_STAGES) else "tcgen05"},
+                       "scores": "tcgen05" if uses_tensor_cores(w, args.flags)
+                       else "fmaf CUDA cores"},
             "roofline": roofline, "stages_ms": stage_ms, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk.summary()}
 

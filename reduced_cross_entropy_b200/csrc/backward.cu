@@ -194,37 +194,54 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
   for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
   __syncwarp();
 
-  // coefficients: four slots per step, one per quarter
-  for (int s0 = 0; s0 < slots; s0 += 4) {
-    const int s = s0 + q;
-    int32_t j = -1;
-    if (s < slots) j = s == 0 ? targets[i] : selected[i * k + (s - 1)];
-    const bool ok = j >= 0 && j < C;
-    float part = 0.0f;
-    if (ok) {
-      const T* y = Y + int64_t(j) * d;
-      for (int t = 8 * sub; t < d; t += 64) {
-        float v[8];
-        load8v(y + t, v);
+  // coefficients: sixteen slots per step, four per quarter, their rows loaded together
+  for (int s0 = 0; s0 < slots; s0 += 16) {
+    int32_t j[4];
+    bool ok[4];
+    float part[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) part = fmaf(xs[t + u], v[u], part);
-      }
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0 + 4 * u + q;
+      j[u] = -1;
+      if (s < slots) j[u] = s == 0 ? targets[i] : selected[i * k + (s - 1)];
+      ok[u] = j[u] >= 0 && j[u] < C;
+      part[u] = 0.0f;
     }
-    part += __shfl_xor_sync(0xFFFFFFFFu, part, 4);
-    part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
-    part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
-    if (sub == 0 && s < slots) {
-      float g = 0.0f;
-      if (ok) {
-        const float p = expf(part - li);
-        g = (s == 0 ? p - 1.0f : p) * scale;
-      } else if (s == 0) {
-        raise_flag(status, RECE_DEVICE_BAD_TARGET);
+    for (int t = 8 * sub; t < d; t += 64) {
+      float v[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (ok[u]) load8v(Y + int64_t(j[u]) * d + t, v[u]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (ok[u]) {
+#pragma unroll
+          for (int uu = 0; uu < 8; ++uu) part[u] = fmaf(xs[t + uu], v[u][uu], part[u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      part[u] += __shfl_xor_sync(0xFFFFFFFFu, part[u], 4);
+      part[u] += __shfl_xor_sync(0xFFFFFFFFu, part[u], 2);
+      part[u] += __shfl_xor_sync(0xFFFFFFFFu, part[u], 1);
+    }
+    if (sub == 0) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = s0 + 4 * u + q;
+        if (s >= slots) continue;
+        float g = 0.0f;
+        if (ok[u]) {
+          const float p = expf(part[u] - li);
+          g = (s == 0 ? p - 1.0f : p) * scale;
+        } else if (s == 0) {
+          raise_flag(status, RECE_DEVICE_BAD_TARGET);
+        }
+        gs[s] = g;
+        js[s] = ok[u] ? j[u] : -1;
+        e_key[i * slots + s] = ok[u] ? j[u] : int32_t(C);
+        e_g[i * slots + s] = g;
       }
-      gs[s] = g;
-      js[s] = ok ? j : -1;
-      e_key[i * slots + s] = ok ? j : int32_t(C);
-      e_g[i * slots + s] = g;
     }
   }
   __syncwarp();
@@ -234,15 +251,24 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
     const int t = t0 + 8 * sub;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (t < d) {
-#pragma unroll 2
-      for (int s = q; s < slots; s += 4) {
-        const int32_t j = js[s];
-        if (j < 0) continue;
-        const float g = gs[s];
-        float v[8];
-        load8v(Y + int64_t(j) * d + t, v);
+      for (int s = q; s < slots; s += 16) {
+        float v[4][8];
+        float g[4];
+        bool has[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = fmaf(g, v[u], acc[u]);
+        for (int u = 0; u < 4; ++u) {
+          const int su = s + 4 * u;
+          const int32_t j = su < slots ? js[su] : -1;
+          has[u] = j >= 0;
+          g[u] = has[u] ? gs[su] : 0.0f;
+          if (has[u]) load8v(Y + int64_t(j) * d + t, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (has[u]) {
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu) acc[uu] = fmaf(g[u], v[u][uu], acc[uu]);
+          }
       }
     }
 #pragma unroll

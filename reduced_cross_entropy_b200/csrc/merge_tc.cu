@@ -132,36 +132,49 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
   float theta_max = -INFINITY;
   for (int r = 0; r < n_r; ++r) {
     const int64_t p = invX[int64_t(r) * N + i];
-    // four sub-lists (one per epilogue warpgroup of the selection kernel)
+    // four sub-lists (one per epilogue warpgroup of the selection kernel), read as one
+    // concatenated list, four independent entries per lane in flight at a time
     const int4 c4 = list_count[int64_t(r) * N + p];
     theta_max = fmaxf(theta_max, list_theta[int64_t(r) * N + p]);
-    const int cs[4] = {c4.x, c4.y, c4.z, c4.w};
+    const int cs[4] = {c4.x < Qw ? c4.x : Qw, c4.y < Qw ? c4.y : Qw, c4.z < Qw ? c4.z : Qw,
+                       c4.w < Qw ? c4.w : Qw};
+    overflow |= c4.x > Qw || c4.y > Qw || c4.z > Qw || c4.w > Qw;
+    const int total = cs[0] + cs[1] + cs[2] + cs[3];
+    const int2* L = list + (int64_t(r) * N + p) * 4 * Qw;
+    for (int a0 = 0; a0 < total; a0 += 128) {
+      int2 e[4];
+      int32_t jj[4];
+      bool in[4];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      overflow |= cs[w] > Qw;
-      const int m = cs[w] < Qw ? cs[w] : Qw;
-      const int2* L = list + ((int64_t(r) * N + p) * 4 + w) * Qw;
-      for (int a0 = 0; a0 < m; a0 += 32) {
-        const int a = a0 + lane;
-        bool keep = false;
-        uint32_t key = 0;
-        int32_t j = -1;
-        if (a < m) {
-          const int2 e = L[a];
-          j = py[int64_t(r) * C + e.y];
-          keep = j != z;
-          for (int rp = 0; rp < r && keep; ++rp) {
-            const int dc = chunkY[int64_t(rp) * C + j] - cx[rp];
-            if (dc >= -n_ec && dc <= n_ec) keep = false;
-          }
-          key = score_key(__int_as_float(e.x));
+      for (int u = 0; u < 4; ++u) {
+        int a = a0 + 32 * u + lane;
+        in[u] = a < total;
+        int w = 0;
+        while (w < 3 && a >= cs[w]) {
+          a -= cs[w];
+          ++w;
         }
-        const unsigned b = __ballot_sync(0xFFFFFFFFu, keep);
-        if (keep) {
+        e[u] = in[u] ? L[w * Qw + a] : make_int2(0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) jj[u] = in[u] ? py[int64_t(r) * C + e[u].y] : -1;
+      bool keep[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        keep[u] = in[u] && jj[u] != z;
+        for (int rp = 0; rp < r && keep[u]; ++rp) {
+          const int dc = chunkY[int64_t(rp) * C + jj[u]] - cx[rp];
+          if (dc >= -n_ec && dc <= n_ec) keep[u] = false;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const unsigned b = __ballot_sync(0xFFFFFFFFu, keep[u]);
+        if (keep[u]) {
           const int pos = n + __popc(b & ((1u << lane) - 1u));
           if (pos < cap) {
-            keys[pos] = key;
-            items[pos] = j;
+            keys[pos] = score_key(__int_as_float(e[u].x));
+            items[pos] = jj[u];
           }
         }
         n += __popc(b);

@@ -39,10 +39,15 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_hist(const int32_t* __res
   for (int i = threadIdx.x; i < digits; i += blockDim.x) sh_cnt[i] = 0;
   __syncthreads();
   const int64_t base = int64_t(blockIdx.x) * kSortTile;
-  for (int e = threadIdx.x; e < kSortTile; e += blockDim.x) {
-    const int64_t p = base + e;
-    if (p < M) atomicAdd(&sh_cnt[(elem_key(keys, in_ids, p, in_order) >> shift) & mask], 1);
+  int32_t kv[kSortTile / kSortThreads];
+#pragma unroll
+  for (int u = 0; u < kSortTile / kSortThreads; ++u) {
+    const int64_t p = base + u * kSortThreads + threadIdx.x;
+    kv[u] = p < M ? elem_key(keys, in_ids, p, in_order) : -1;
   }
+#pragma unroll
+  for (int u = 0; u < kSortTile / kSortThreads; ++u)
+    if (kv[u] >= 0) atomicAdd(&sh_cnt[(kv[u] >> shift) & mask], 1);
   __syncthreads();
   for (int i = threadIdx.x; i < digits; i += blockDim.x)
     hist[int64_t(i) * tiles + blockIdx.x] = sh_cnt[i];
@@ -113,6 +118,14 @@ __global__ void __launch_bounds__(1024) k_sort_scan_digits(int32_t* __restrict__
   if (threadIdx.x == 0) start[digits] = carry;
 }
 
+// Shared memory of the scatter: per-warp digit counts, per-digit offsets, and the tile
+// staged in digit order (id, key, payload) so that the global writes are contiguous runs.
+__host__ __device__ constexpr size_t scatter_smem_bytes(int bits) {
+  return ((size_t(kWarps) * (size_t(1) << bits) * 2 + 15) & ~size_t(15))  // cnt (uint16)
+         + size_t(3) * 4 * (size_t(1) << bits)                            // offsets
+         + size_t(kSortTile) * 12;                                        // staged tile
+}
+
 __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
     const int32_t* __restrict__ keys, const int32_t* __restrict__ in_ids, int64_t M, int shift,
     int bits, const int32_t* __restrict__ hist, int64_t tiles,
@@ -122,30 +135,52 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
   extern __shared__ __align__(16) unsigned char sh_raw[];
   const int digits = 1 << bits, mask = digits - 1;
   uint16_t* cnt = reinterpret_cast<uint16_t*>(sh_raw);  // [kWarps][digits]
-  int32_t* tile_base =
-      reinterpret_cast<int32_t*>(sh_raw + ((kWarps * digits * sizeof(uint16_t) + 15) & ~15));
+  int32_t* gbase = reinterpret_cast<int32_t*>(sh_raw + ((kWarps * digits * 2 + 15) & ~15));
+  int32_t* lbase = gbase + digits;   // first staged position of each digit in this tile
+  int32_t* total = lbase + digits;   // this tile's count of each digit
+  int32_t* s_id = total + digits;
+  int32_t* s_key = s_id + kSortTile;
+  float* s_pay = reinterpret_cast<float*>(s_key + kSortTile);
+  __shared__ int32_t sh_warp[32];
+  __shared__ int32_t sh_total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t tile = blockIdx.x;
+  const int64_t tile0 = tile * kSortTile;
+  const int n_tile = int(M - tile0 < kSortTile ? M - tile0 : kSortTile);
 
   for (int i = tid; i < kWarps * digits; i += blockDim.x) cnt[i] = 0;
   for (int i = tid; i < digits; i += blockDim.x)
-    tile_base[i] = digit_start[i] + hist[int64_t(i) * tiles + tile];
+    gbase[i] = digit_start[i] + hist[int64_t(i) * tiles + tile];
   __syncthreads();
 
-  const int64_t wbase = tile * kSortTile + int64_t(warp) * kPerWarp;
+  const int64_t wbase = tile0 + int64_t(warp) * kPerWarp;
   uint16_t* wcnt = cnt + warp * digits;
-  // pass 1: this warp's count of every digit
+  // every lane's 16 elements (one per warp step), loaded up front, all in flight together
+  int32_t r_id[kSteps], r_key[kSteps];
+  float r_pay[kSteps];
+#pragma unroll
   for (int s = 0; s < kSteps; ++s) {
     const int64_t p = wbase + s * 32 + lane;
-    const bool ok = p < M;
-    const int dg = ok ? ((elem_key(keys, in_ids, p, in_order) >> shift) & mask)
-                      : (0x40000000 | lane);
+    r_id[s] = 0;
+    r_key[s] = 0;
+    r_pay[s] = 0.0f;
+    if (p < M) {
+      r_id[s] = elem_id(in_ids, p);
+      r_key[s] = in_order ? keys[p] : keys[r_id[s]];
+      if (payload) r_pay[s] = in_order ? payload[p] : payload[r_id[s]];
+    }
+  }
+  // pass 1: this warp's count of every digit
+#pragma unroll
+  for (int s = 0; s < kSteps; ++s) {
+    const bool ok = wbase + s * 32 + lane < M;
+    const int dg = ok ? ((r_key[s] >> shift) & mask) : (0x40000000 | lane);
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
     if (ok && lane == __ffs(peers) - 1) wcnt[dg] += uint16_t(__popc(peers));
     __syncwarp();
   }
   __syncthreads();
-  // exclusive prefix over the warps of the tile, per digit
+  // per digit: exclusive prefix over the warps; the tile's total
   for (int dg = tid; dg < digits; dg += blockDim.x) {
     uint16_t run = 0;
     for (int w = 0; w < kWarps; ++w) {
@@ -153,30 +188,47 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
       cnt[w * digits + dg] = run;
       run = uint16_t(run + c);
     }
+    total[dg] = run;
   }
   __syncthreads();
-  // pass 2: scatter in order
+  // staged position of each digit's first element: exclusive scan of the totals
+  int32_t carry = 0;
+  for (int c0 = 0; c0 < digits; c0 += blockDim.x) {
+    const int dg = c0 + tid;
+    const int32_t v = dg < digits ? total[dg] : 0;
+    const int32_t ex = block_exclusive_scan(v, sh_warp, &sh_total);
+    if (dg < digits) lbase[dg] = carry + ex;
+    carry += sh_total;
+    __syncthreads();
+  }
+  // pass 2: stage every element at its rank, in order
+#pragma unroll
   for (int s = 0; s < kSteps; ++s) {
-    const int64_t p = wbase + s * 32 + lane;
-    const bool ok = p < M;
-    int32_t id = 0, key = 0;
-    if (ok) {
-      id = elem_id(in_ids, p);
-      key = in_order ? keys[p] : keys[id];
-    }
+    const bool ok = wbase + s * 32 + lane < M;
+    const int32_t key = r_key[s];
     const int dg = ok ? ((key >> shift) & mask) : (0x40000000 | lane);
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
     const int base = ok ? int(wcnt[dg]) : 0;
     __syncwarp();
     if (ok) {
       const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int64_t pos = int64_t(tile_base[dg]) + base + rank;
-      out_ids[pos] = id;
-      if (out_keys) out_keys[pos] = key;
-      if (out_payload) out_payload[pos] = in_order ? payload[p] : payload[id];
+      const int lp = lbase[dg] + base + rank;
+      s_id[lp] = r_id[s];
+      s_key[lp] = key;
+      s_pay[lp] = r_pay[s];
       if (lane == __ffs(peers) - 1) wcnt[dg] = uint16_t(base + __popc(peers));
     }
     __syncwarp();
+  }
+  __syncthreads();
+  // write out: consecutive staged positions of a digit go to consecutive global positions
+  for (int lp = tid; lp < n_tile; lp += blockDim.x) {
+    const int32_t key = s_key[lp];
+    const int dg = (key >> shift) & mask;
+    const int64_t pos = int64_t(gbase[dg]) + (lp - lbase[dg]);
+    out_ids[pos] = s_id[lp];
+    if (out_keys) out_keys[pos] = key;
+    if (out_payload) out_payload[pos] = s_pay[lp];
   }
 }
 
@@ -221,12 +273,10 @@ cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t
       keys, in_ids, M, shift, bits, hist, tiles, in_order);
   k_sort_scan_tiles<<<digits, 256, 0, st>>>(hist, tiles, start);
   k_sort_scan_digits<<<1, 1024, 0, st>>>(start, digits);
-  const size_t smem = ((kWarps * digits * sizeof(uint16_t) + 15) & ~size_t(15)) +
-                      sizeof(int32_t) * digits;
   // Opt in to the largest dynamic shared memory the scatter can use (per device; cheap).
-  cudaError_t e = cudaFuncSetAttribute(
-      k_sort_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      int(sizeof(uint16_t) * kWarps * (1 << kMaxDigitBits) + sizeof(int32_t) * (1 << kMaxDigitBits) + 16));
+  const size_t smem = scatter_smem_bytes(bits);
+  cudaError_t e = cudaFuncSetAttribute(k_sort_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(scatter_smem_bytes(kMaxDigitBits)));
   if (e != cudaSuccess) return e;
   k_sort_scatter<<<unsigned(tiles), kSortThreads, smem, st>>>(
       keys, in_ids, M, shift, bits, hist, tiles, start, out_ids, out_keys, payload, out_payload,
