@@ -295,6 +295,7 @@ def main():
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     sel = torch.empty(w.N, w.k, dtype=torch.int32, device=dev)
     lse = torch.empty(w.N, dtype=torch.float32, device=dev)
+    logits = torch.empty(w.N, w.k + 1, dtype=torch.float32, device=dev)
     dloss = torch.ones(1, dtype=torch.float32, device=dev)
     dX = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
     dY = torch.empty(w.C, w.d, dtype=torch.float32, device=dev)
@@ -308,9 +309,10 @@ def main():
         _lib.check(L.rece_bucketize_sort(plan._h, vp(Bt), vp(Xd), vp(Yd), vp(ws), nbytes, sp),
                    "bucketize_sort")
         _lib.check(L.rece_loss_fwd(plan._h, vp(Xd), vp(Yd), vp(td), vp(ws), nbytes, vp(loss),
-                                   None, vp(sel), vp(lse), sp), "loss_fwd")
+                                   None, vp(sel), vp(lse), vp(logits), sp), "loss_fwd")
         _lib.check(L.rece_loss_bwd(plan._h, vp(Xd), vp(Yd), vp(td), vp(sel), vp(lse),
-                                   vp(dloss), vp(ws), nbytes, vp(dX), vp(dY), sp), "loss_bwd")
+                                   vp(logits), vp(dloss), vp(ws), nbytes, vp(dX), vp(dY), sp),
+                   "loss_bwd")
 
     for s in range(args.warmup):
         flush.zero_()
@@ -451,8 +453,8 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
     def rece():
         ws = plan.workspace(dev)
         ops.bucketize_sort(plan, B, Xd, Yd, ws)
-        _, _, s, l = ops.loss_fwd(plan, Xd, Yd, td, ws, want_row_loss=False)
-        ops.loss_bwd(plan, Xd, Yd, td, s, l, torch.ones(1, device=dev), ws)
+        _, _, s, l, lg = ops.loss_fwd(plan, Xd, Yd, td, ws, want_row_loss=False)
+        ops.loss_bwd(plan, Xd, Yd, td, s, l, torch.ones(1, device=dev), ws, logits=lg)
 
     def fused():
         _, _, l, ws = ops.full_ce_fwd(Xd, Yd, td)

@@ -138,22 +138,27 @@ RECE_API rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, cons
  *   selected device int32 [N][k]: the kept negatives, best first (score descending,
  *            item id ascending), -1 where a row has fewer than k candidates
  *   lse      device fp32 [N]: log(exp(l+) + sum over selected exp(l)) per row
- * selected and lse are what rece_loss_bwd needs. */
+ *   logits   device fp32 [N][k+1] or NULL: the logits the loss used, the positive's
+ *            first, then those of `selected` (-inf where selected is -1)
+ * selected and lse (and logits, which spare the backward recomputing them) are what
+ * rece_loss_bwd needs. */
 RECE_API rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
                             const int32_t* targets, void* workspace, size_t workspace_bytes,
                             float* loss, float* row_loss, int32_t* selected, float* lse,
-                            void* stream);
+                            float* logits, void* stream);
 
 /* Step 6 [RECE equation (4) on the positive and the kept negatives]:
  *   g_ij = (exp(l_ij - lse_i) - [j == z_i]) * dloss / N
+ *   logits device fp32 [N][k+1] from rece_loss_fwd, or NULL to recompute the l_ij
  *   dX_i = sum_j g_ij y_j,   dY_j = sum_i g_ij x_i
  *   dloss  device fp32 [1]: gradient of the caller's objective w.r.t. the mean loss
  *   dX     device fp32 [N][d], dY device fp32 [C][d]: overwritten (items no row touched
  *          get exactly 0).  Deterministic: no floating-point atomics. */
 RECE_API rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
                             const int32_t* targets, const int32_t* selected,
-                            const float* lse, const float* dloss, void* workspace,
-                            size_t workspace_bytes, float* dX, float* dY, void* stream);
+                            const float* lse, const float* logits, const float* dloss,
+                            void* workspace, size_t workspace_bytes, float* dX, float* dY,
+                            void* stream);
 
 /* Exact full cross-entropy [RECE equations (3) and (4)], fused: the logits are formed
  * tile by tile on chip and never stored.  Arguments as above; mode picks the input

@@ -72,8 +72,8 @@ def lib():
         "rece_plan_workspace_size": ([vp, ctypes.POINTER(sz)], st),
         "rece_plan_workspace_layout": ([vp, ctypes.POINTER(WorkspaceLayout)], st),
         "rece_bucketize_sort": ([vp, vp, vp, vp, vp, sz, vp], st),
-        "rece_loss_fwd": ([vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp], st),
-        "rece_loss_bwd": ([vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp], st),
+        "rece_loss_fwd": ([vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp, vp], st),
+        "rece_loss_bwd": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp], st),
         "rece_full_ce_workspace_size": ([i64, i64, i32, i32, ctypes.POINTER(sz)], st),
         "rece_full_ce_fwd": ([i64, i64, i32, i32, vp, vp, vp, vp, sz, vp, vp, vp, vp], st),
         "rece_full_ce_bwd": ([i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp], st),

@@ -50,8 +50,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_rows(
     const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
     const int32_t* __restrict__ selected, const float* __restrict__ lse,
-    const float* __restrict__ dloss, int64_t N, int64_t C, int d, int k,
-    int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
+    const float* __restrict__ logits, const float* __restrict__ dloss, int64_t N, int64_t C,
+    int d, int k, int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
     uint32_t* status) {
   extern __shared__ __align__(16) float sh_f[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
     int32_t j = s == 0 ? targets[i] : selected[i * k + (s - 1)];
     float g = 0.0f;
     if (j >= 0 && j < C) {
-      const float p = expf(dot_row(xs, Y + int64_t(j) * d, d) - li);
+      const float l = logits ? logits[i * slots + s] : dot_row(xs, Y + int64_t(j) * d, d);
+      const float p = expf(l - li);
       g = (s == 0 ? p - 1.0f : p) * scale;
     } else {
       if (s == 0) raise_flag(status, RECE_DEVICE_BAD_TARGET);
@@ -176,8 +177,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
     const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
     const int32_t* __restrict__ selected, const float* __restrict__ lse,
-    const float* __restrict__ dloss, int64_t N, int64_t C, int d, int k,
-    int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
+    const float* __restrict__ logits, const float* __restrict__ dloss, int64_t N, int64_t C,
+    int d, int k, int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
     uint32_t* status) {
   extern __shared__ __align__(16) float sh_f[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -194,8 +195,26 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
   for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
   __syncwarp();
 
+  if (logits) {
+    // the forward's logits: no dot products; one slot per lane
+    for (int s = lane; s < slots; s += 32) {
+      int32_t j = s == 0 ? targets[i] : selected[i * k + (s - 1)];
+      const bool ok = j >= 0 && j < C;
+      float g = 0.0f;
+      if (ok) {
+        const float p = expf(logits[i * slots + s] - li);
+        g = (s == 0 ? p - 1.0f : p) * scale;
+      } else if (s == 0) {
+        raise_flag(status, RECE_DEVICE_BAD_TARGET);
+      }
+      gs[s] = g;
+      js[s] = ok ? j : -1;
+      e_key[i * slots + s] = ok ? j : int32_t(C);
+      e_g[i * slots + s] = g;
+    }
+  }
   // coefficients: sixteen slots per step, four per quarter, their rows loaded together
-  for (int s0 = 0; s0 < slots; s0 += 16) {
+  for (int s0 = 0; s0 < (logits ? 0 : slots); s0 += 16) {
     int32_t j[4];
     bool ok[4];
     float part[4];
@@ -338,8 +357,8 @@ size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 *
 template <typename T>
 cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
                             const int32_t* targets, const int32_t* selected, const float* lse,
-                            const float* dloss, char* ws, float* dX, float* dY,
-                            uint32_t* status, cudaStream_t st) {
+                            const float* logits, const float* dloss, char* ws, float* dX,
+                            float* dY, uint32_t* status, cudaStream_t st) {
   const auto& c = p.cfg;
   const Layout& L = p.lay;
   const int64_t E = p.entries;
@@ -362,10 +381,12 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
     if (e != cudaSuccess) return e;
     if (v8)
       k_bwd_rows_v8<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
-          X, Y, targets, selected, lse, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX, status);
+          X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX,
+          status);
     else
       k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
-          X, Y, targets, selected, lse, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX, status);
+          X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX,
+          status);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -415,12 +436,12 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
 
 template cudaError_t launch_backward<float>(const rece_plan_s&, const float*, const float*,
                                             const int32_t*, const int32_t*, const float*,
-                                            const float*, char*, float*, float*, uint32_t*,
-                                            cudaStream_t);
+                                            const float*, const float*, char*, float*, float*,
+                                            uint32_t*, cudaStream_t);
 template cudaError_t launch_backward<__nv_bfloat16>(const rece_plan_s&, const __nv_bfloat16*,
                                                     const __nv_bfloat16*, const int32_t*,
                                                     const int32_t*, const float*, const float*,
-                                                    char*, float*, float*, uint32_t*,
-                                                    cudaStream_t);
+                                                    const float*, char*, float*, float*,
+                                                    uint32_t*, cudaStream_t);
 
 }  // namespace rece

@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(kThreads) k_merge_loss(
     const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
     int64_t N, int64_t C, int d, int k, int n_r, int P, const float* __restrict__ list_score,
     const int32_t* __restrict__ list_item, int32_t* __restrict__ selected,
-    float* __restrict__ lse_out, float* __restrict__ row_loss, uint32_t* status) {
+    float* __restrict__ lse_out, float* __restrict__ row_loss, float* __restrict__ logits,
+    uint32_t* status) {
   extern __shared__ __align__(16) uint64_t sk[];  // [2][P]
   uint64_t* tmp = sk + P;
   __shared__ float red[kThreads];
@@ -117,6 +118,12 @@ __global__ void __launch_bounds__(kThreads) k_merge_loss(
   __syncthreads();
   const float lp = red[0];
   __syncthreads();
+  if (logits) {
+    float* lg = logits + i * (int64_t(k) + 1);
+    if (tid == 0) lg[0] = z_ok ? lp : NAN;
+    for (int a = tid; a < k; a += kThreads)
+      lg[1 + a] = a < kk ? key_score(uint32_t((~order[a]) >> 32)) : -INFINITY;
+  }
   const float best = kk > 0 ? key_score(uint32_t((~order[0]) >> 32)) : -INFINITY;
   const float m = fmaxf(lp, best);
   float part = 0.0f;
@@ -162,7 +169,8 @@ template <typename T>
 cudaError_t launch_merge_loss(const rece_plan_s& p, const T* X, const T* Y,
                               const int32_t* targets, const float* list_score,
                               const int32_t* list_item, int32_t* selected, float* lse,
-                              float* row_loss, uint32_t* status, cudaStream_t st) {
+                              float* row_loss, float* logits, uint32_t* status,
+                              cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
   const int P = merge_pow2(c.n_r, c.k);
@@ -172,7 +180,8 @@ cudaError_t launch_merge_loss(const rece_plan_s& p, const T* X, const T* Y,
   if (e != cudaSuccess) return e;
   k_merge_loss<T><<<unsigned(c.N), kThreads, smem, st>>>(X, Y, targets, c.N, c.C, c.d, c.k,
                                                          c.n_r, P, list_score, list_item,
-                                                         selected, lse, row_loss, status);
+                                                         selected, lse, row_loss, logits,
+                                                         status);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -185,11 +194,12 @@ cudaError_t launch_mean(const float* row_loss, int64_t N, float* loss, cudaStrea
 
 template cudaError_t launch_merge_loss<float>(const rece_plan_s&, const float*, const float*,
                                               const int32_t*, const float*, const int32_t*,
-                                              int32_t*, float*, float*, uint32_t*,
+                                              int32_t*, float*, float*, float*, uint32_t*,
                                               cudaStream_t);
 template cudaError_t launch_merge_loss<__nv_bfloat16>(const rece_plan_s&, const __nv_bfloat16*,
                                                       const __nv_bfloat16*, const int32_t*,
                                                       const float*, const int32_t*, int32_t*,
-                                                      float*, float*, uint32_t*, cudaStream_t);
+                                                      float*, float*, float*, uint32_t*,
+                                                      cudaStream_t);
 
 }  // namespace rece

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     const int4* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
     int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap, int P,
     int32_t* __restrict__ selected, float* __restrict__ lse_out, float* __restrict__ row_loss,
-    uint32_t* status) {
+    float* __restrict__ logits, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t sh_raw[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t per_warp = size_t(P) * 8 + size_t(cap) * 8 + 1024;
@@ -240,6 +240,12 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     for (int t = lane; t < d; t += 32) part = fmaf(to_f32(x[t]), to_f32(y[t]), part);
   }
   const float lp = warp_sum(part);
+  if (logits) {
+    float* lg = logits + i * (int64_t(k) + 1);
+    if (lane == 0) lg[0] = z_ok ? lp : NAN;
+    for (int a = lane; a < k; a += 32)
+      lg[1 + a] = a < ns ? key_score(uint32_t((~sel[a]) >> 32)) : -INFINITY;
+  }
   const float best = ns > 0 ? key_score(uint32_t((~sel[0]) >> 32)) : -INFINITY;
   const float m = fmaxf(lp, best);
   float acc = 0.0f;
@@ -277,7 +283,7 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
                             const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, float* lse,
-                            float* row_loss, uint32_t* status, cudaStream_t st) {
+                            float* row_loss, float* logits, uint32_t* status, cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
   int P = 2;
@@ -292,7 +298,7 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   if (e != cudaSuccess) return e;
   k_merge_tc<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
       X, Y, targets, py, invX, chunkY, list, list_count, list_theta, c.N, c.C, c.d, c.k, c.n_r,
-      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), P, selected, lse, row_loss, status);
+      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), P, selected, lse, row_loss, logits, status);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -300,6 +306,6 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
 template cudaError_t launch_merge_tc<__nv_bfloat16>(
     const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
     const int32_t*, const int32_t*, const int32_t*, const int2*, const int4*, const float*,
-    int32_t*, float*, float*, uint32_t*, cudaStream_t);
+    int32_t*, float*, float*, float*, uint32_t*, cudaStream_t);
 
 }  // namespace rece

@@ -113,7 +113,8 @@ template <typename T>
 cudaError_t launch_merge_loss(const rece_plan_s& p, const T* X, const T* Y,
                               const int32_t* targets, const float* list_score,
                               const int32_t* list_item, int32_t* selected, float* lse,
-                              float* row_loss, uint32_t* status, cudaStream_t st);
+                              float* row_loss, float* logits, uint32_t* status,
+                              cudaStream_t st);
 
 // K7: loss[0] = sum(row_loss) / N in a fixed order.
 cudaError_t launch_mean(const float* row_loss, int64_t N, float* loss, cudaStream_t st);
@@ -122,8 +123,8 @@ cudaError_t launch_mean(const float* row_loss, int64_t N, float* loss, cudaStrea
 template <typename T>
 cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
                             const int32_t* targets, const int32_t* selected, const float* lse,
-                            const float* dloss, char* ws, float* dX, float* dY,
-                            uint32_t* status, cudaStream_t st);
+                            const float* logits, const float* dloss, char* ws, float* dX,
+                            float* dY, uint32_t* status, cudaStream_t st);
 
 // K6: exact full cross-entropy.
 template <typename T>

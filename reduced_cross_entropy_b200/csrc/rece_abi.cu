@@ -293,7 +293,7 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
 rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
                             const int32_t* targets, void* workspace, size_t workspace_bytes,
                             float* loss, float* row_loss, int32_t* selected, float* lse,
-                            void* stream) {
+                            float* logits, void* stream) {
   rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
   if (s != RECE_OK) return s;
   const auto& c = plan->cfg;
@@ -315,7 +315,7 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     RECE_CUDA(launch_select_fma(*plan, Xf, Yf, targets, px, py, ls, li, st), "select");
     stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
     stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
-    RECE_CUDA(launch_merge_loss(*plan, Xf, Yf, targets, ls, li, selected, lse, rl, status, st),
+    RECE_CUDA(launch_merge_loss(*plan, Xf, Yf, targets, ls, li, selected, lse, rl, logits, status, st),
               "merge/loss");
   } else if (plan->use_tc) {
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
@@ -331,7 +331,7 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     RECE_CUDA(launch_merge_tc(*plan, Xb, Yb, targets, py,
                               reinterpret_cast<const int32_t*>(ws + L.inv_x),
                               reinterpret_cast<const int32_t*>(ws + L.chunk_y), list, cnt, theta,
-                              selected, lse, rl, status, st),
+                              selected, lse, rl, logits, status, st),
               "merge/loss (tcgen05 lists)");
   } else {
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
@@ -340,7 +340,7 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     RECE_CUDA(launch_select_fma(*plan, Xb, Yb, targets, px, py, ls, li, st), "select");
     stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
     stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
-    RECE_CUDA(launch_merge_loss(*plan, Xb, Yb, targets, ls, li, selected, lse, rl, status, st),
+    RECE_CUDA(launch_merge_loss(*plan, Xb, Yb, targets, ls, li, selected, lse, rl, logits, status, st),
               "merge/loss");
   }
   stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 1, st);
@@ -352,8 +352,8 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
 
 rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
                             const int32_t* targets, const int32_t* selected, const float* lse,
-                            const float* dloss, void* workspace, size_t workspace_bytes,
-                            float* dX, float* dY, void* stream) {
+                            const float* logits, const float* dloss, void* workspace,
+                            size_t workspace_bytes, float* dX, float* dY, void* stream) {
   rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
   if (s != RECE_OK) return s;
   const auto& c = plan->cfg;
@@ -364,12 +364,12 @@ rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan->lay.status);
   if (c.mode == RECE_MODE_FP32_EXACT)
     RECE_CUDA(launch_backward(*plan, static_cast<const float*>(X), static_cast<const float*>(Y),
-                              targets, selected, lse, dloss, ws, dX, dY, status, st),
+                              targets, selected, lse, logits, dloss, ws, dX, dY, status, st),
               "backward");
   else
     RECE_CUDA(launch_backward(*plan, static_cast<const __nv_bfloat16*>(X),
                               static_cast<const __nv_bfloat16*>(Y), targets, selected, lse,
-                              dloss, ws, dX, dY, status, st),
+                              logits, dloss, ws, dX, dY, status, st),
               "backward");
   return RECE_OK;
 }

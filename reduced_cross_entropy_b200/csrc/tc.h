@@ -43,6 +43,6 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
                             const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, float* lse,
-                            float* row_loss, uint32_t* status, cudaStream_t st);
+                            float* row_loss, float* logits, uint32_t* status, cudaStream_t st);
 
 }  // namespace rece

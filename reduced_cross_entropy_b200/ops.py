@@ -113,8 +113,10 @@ def bucketize_sort(plan: Plan, B, X, Y, ws, stream=None):
                "rece_bucketize_sort")
 
 
-def loss_fwd(plan: Plan, X, Y, targets, ws, *, want_row_loss: bool = True, stream=None):
-    """Steps 3-5.  Returns (loss [1], row_loss [N] or None, selected [N,k], lse [N])."""
+def loss_fwd(plan: Plan, X, Y, targets, ws, *, want_row_loss: bool = True,
+             want_logits: bool = True, stream=None):
+    """Steps 3-5.  Returns (loss [1], row_loss [N] or None, selected [N,k], lse [N],
+    logits [N,k+1] or None)."""
     c = plan.cfg
     _need(X, "X", plan.dtype, (c.N, c.d))
     _need(Y, "Y", plan.dtype, (c.C, c.d))
@@ -125,14 +127,16 @@ def loss_fwd(plan: Plan, X, Y, targets, ws, *, want_row_loss: bool = True, strea
     row = torch.empty(c.N, dtype=torch.float32, device=dev) if want_row_loss else None
     sel = torch.empty(c.N, c.k, dtype=torch.int32, device=dev)
     lse = torch.empty(c.N, dtype=torch.float32, device=dev)
+    logits = torch.empty(c.N, c.k + 1, dtype=torch.float32, device=dev) if want_logits else None
     _lib.check(_lib.lib().rece_loss_fwd(plan._h, _vp(X), _vp(Y), _vp(targets), _vp(ws),
                                         ws.numel(), _vp(loss), _vp(row), _vp(sel), _vp(lse),
-                                        _stream(stream)), "rece_loss_fwd")
-    return loss, row, sel, lse
+                                        _vp(logits), _stream(stream)), "rece_loss_fwd")
+    return loss, row, sel, lse, logits
 
 
-def loss_bwd(plan: Plan, X, Y, targets, selected, lse, dloss, ws, stream=None):
-    """Step 6.  Returns (dX [N,d] fp32, dY [C,d] fp32)."""
+def loss_bwd(plan: Plan, X, Y, targets, selected, lse, dloss, ws, logits=None, stream=None):
+    """Step 6.  Returns (dX [N,d] fp32, dY [C,d] fp32).  `logits` from loss_fwd spares
+    recomputing the selected logits (None: recompute them)."""
     c = plan.cfg
     _need(X, "X", plan.dtype, (c.N, c.d))
     _need(Y, "Y", plan.dtype, (c.C, c.d))
@@ -140,12 +144,14 @@ def loss_bwd(plan: Plan, X, Y, targets, selected, lse, dloss, ws, stream=None):
     _need(selected, "selected", torch.int32, (c.N, c.k))
     _need(lse, "lse", torch.float32, (c.N,))
     _need(dloss, "dloss", torch.float32, (1,))
+    if logits is not None:
+        _need(logits, "logits", torch.float32, (c.N, c.k + 1))
     _check_ws(plan, ws)
     dX = torch.empty(c.N, c.d, dtype=torch.float32, device=X.device)
     dY = torch.empty(c.C, c.d, dtype=torch.float32, device=X.device)
     _lib.check(_lib.lib().rece_loss_bwd(plan._h, _vp(X), _vp(Y), _vp(targets), _vp(selected),
-                                        _vp(lse), _vp(dloss), _vp(ws), ws.numel(), _vp(dX),
-                                        _vp(dY), _stream(stream)), "rece_loss_bwd")
+                                        _vp(lse), _vp(logits), _vp(dloss), _vp(ws), ws.numel(),
+                                        _vp(dX), _vp(dY), _stream(stream)), "rece_loss_bwd")
     return dX, dY
 
 
@@ -204,16 +210,16 @@ class _ReceLossFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, X, Y, targets, B, plan, ws):
         bucketize_sort(plan, B, X, Y, ws)
-        loss, _, sel, lse = loss_fwd(plan, X, Y, targets, ws, want_row_loss=False)
-        ctx.save_for_backward(X, Y, targets, sel, lse)
+        loss, _, sel, lse, logits = loss_fwd(plan, X, Y, targets, ws, want_row_loss=False)
+        ctx.save_for_backward(X, Y, targets, sel, lse, logits)
         ctx.plan, ctx.ws = plan, ws
         return loss.reshape(())
 
     @staticmethod
     def backward(ctx, grad):
-        X, Y, targets, sel, lse = ctx.saved_tensors
+        X, Y, targets, sel, lse, logits = ctx.saved_tensors
         dloss = grad.detach().float().reshape(1).contiguous()
-        dX, dY = loss_bwd(ctx.plan, X, Y, targets, sel, lse, dloss, ctx.ws)
+        dX, dY = loss_bwd(ctx.plan, X, Y, targets, sel, lse, dloss, ctx.ws, logits=logits)
         return dX.to(X.dtype), dY.to(Y.dtype), None, None, None, None
 
 

@@ -22,7 +22,7 @@ def max_rel(a, b):
     return float(np.max(np.abs(a - b)) / den)
 
 
-def run_gpu(w: synth.Workload, X, Y, t, B, flags=0, dloss=1.0):
+def run_gpu(w: synth.Workload, X, Y, t, B, flags=0, dloss=1.0, use_logits=True):
     """Whole path on the GPU.  Returns a dict of numpy arrays."""
     plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype,
                     flags=flags)
@@ -32,13 +32,15 @@ def run_gpu(w: synth.Workload, X, Y, t, B, flags=0, dloss=1.0):
     ops.bucketize_sort(plan, Bd, Xd, Yd, ws)
     bx, by = (a.cpu().numpy() for a in plan.bucket_ids(ws))
     px, py = (a.cpu().numpy() for a in plan.permutations(ws))
-    loss, row, sel, lse = ops.loss_fwd(plan, Xd, Yd, td, ws)
+    loss, row, sel, lse, logits = ops.loss_fwd(plan, Xd, Yd, td, ws)
     dl = torch.tensor([dloss], dtype=torch.float32, device="cuda")
-    dX, dY = ops.loss_bwd(plan, Xd, Yd, td, sel, lse, dl, ws)
+    dX, dY = ops.loss_bwd(plan, Xd, Yd, td, sel, lse, dl, ws,
+                          logits=logits if use_logits else None)
     status = ops.device_status(ws)
     return dict(bx=bx, by=by, permX=px, permY=py, loss=float(loss.item()),
                 row_loss=row.cpu().numpy(), selected=sel.cpu().numpy(), lse=lse.cpu().numpy(),
-                dX=dX.cpu().numpy(), dY=dY.cpu().numpy(), status=status, plan=plan)
+                dX=dX.cpu().numpy(), dY=dY.cpu().numpy(), status=status, plan=plan,
+                logits=logits.cpu().numpy())
 
 
 def run_oracle(w: synth.Workload, X, Y, t, B, dloss=1.0):

@@ -167,3 +167,30 @@ def test_sort_many_buckets_and_one_bucket():
         starts = plan.bucket_starts_y(ws).cpu().numpy()[0]
         np.testing.assert_array_equal(starts[:n_b + 1],
                                       np.searchsorted(np.sort(by), np.arange(n_b + 1)))
+
+
+@pytest.mark.parametrize("name", ["ragged", "sasrec_scaled", "d_not_mult8"])
+def test_logits_output_and_both_backward_paths(name):
+    """rece_loss_fwd's logits are the positive's and the selected items' logits; the
+    backward gives the same gradients from them as when it recomputes them."""
+    w = CASES[name]
+    X, Y, t = synth.make_inputs(w, seed=1)
+    B = synth.projections(1, 0, w.n_r, w.n_b, w.d, w.dtype)
+    flags = 1 if w.dtype == "bf16" else 0
+    a = run_gpu(w, X, Y, t, B, flags=flags, use_logits=True)
+    b = run_gpu(w, X, Y, t, B, flags=flags, use_logits=False)
+    o = run_oracle(w, X, Y, t, B)
+    lg = a["logits"]
+    sel = a["selected"]
+    want = np.full_like(lg, -np.inf)
+    X64, Y64 = X.astype(np.float64), Y.astype(np.float64)
+    want[:, 0] = np.einsum("nd,nd->n", X64, Y64[t])
+    for i in range(w.N):
+        s = sel[i][sel[i] >= 0]
+        want[i, 1:1 + len(s)] = Y64[s] @ X64[i]
+    fin = np.isfinite(want)
+    assert np.array_equal(np.isfinite(lg), fin)
+    assert np.abs(lg[fin] - want[fin]).max() <= 1e-5 * max(1.0, np.abs(want[fin]).max())
+    for g in (a, b):
+        assert max_rel(g["dX"], o["dX"]) <= TOL and max_rel(g["dY"], o["dY"]) <= TOL
+    assert max_rel(a["dX"], b["dX"]) <= TOL and max_rel(a["dY"], b["dY"]) <= TOL
