@@ -187,9 +187,9 @@ RECE_API rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t
  *   order        device int32 [M]: element indices by (bucket asc, index asc)
  *   bucket_start device int32 [2^ceil(log2 n_b) + 1] or NULL: first position of every
  *                bucket id (entries from n_b on hold M)
- * Returns RECE_ERR_UNSUPPORTED, having launched nothing, when the histograms of M
- * elements by 2^ceil(log2 n_b) buckets do not fit the 4 MiB (about M * n_b <= 2^30 /
- * 4096 * 4096: e.g. M <= 1,040,000 at n_b = 4096, M <= 16.7M at n_b = 256).
+ * Returns RECE_ERR_UNSUPPORTED, having launched nothing, when the per-2048-element-tile
+ * histograms of M elements by 2^ceil(log2 n_b) buckets do not fit the 4 MiB (about
+ * M * 2^ceil(log2 n_b) <= 2^31: M <= 520,192 at n_b = 4096, M <= 8,384,512 at n_b = 256).
  * The first call on a device looks up the array's device address (make that first call
  * before any stream capture).  All calls share the array: calls whose GPU work can
  * overlap (unordered streams or threads) race; order them. */

@@ -9,8 +9,8 @@
 
 namespace rece {
 
-// Counting-sort geometry: one CTA sorts a tile of kSortTile elements (8 warps x 512).
-constexpr int kSortTile = 4096;
+// Counting-sort geometry: one CTA sorts a tile of kSortTile elements (8 warps x 256).
+constexpr int kSortTile = 2048;
 constexpr int kSortThreads = 256;
 constexpr int kMaxDigitBits = 12;  // up to 4096 buckets in one pass
 

@@ -16,8 +16,8 @@ namespace rece {
 namespace {
 
 constexpr int kWarps = kSortThreads / 32;      // 8
-constexpr int kPerWarp = kSortTile / kWarps;   // 512
-constexpr int kSteps = kPerWarp / 32;          // 16
+constexpr int kPerWarp = kSortTile / kWarps;   // 256
+constexpr int kSteps = kPerWarp / 32;          // 8
 
 __device__ __forceinline__ int32_t elem_id(const int32_t* in_ids, int64_t p) {
   return in_ids ? in_ids[p] : int32_t(p);
@@ -126,7 +126,7 @@ __host__ __device__ constexpr size_t scatter_smem_bytes(int bits) {
          + size_t(kSortTile) * 12;                                        // staged tile
 }
 
-__global__ void __launch_bounds__(kSortThreads) k_sort_scatter(
+__global__ void __launch_bounds__(kSortThreads, 4) k_sort_scatter(
     const int32_t* __restrict__ keys, const int32_t* __restrict__ in_ids, int64_t M, int shift,
     int bits, const int32_t* __restrict__ hist, int64_t tiles,
     const int32_t* __restrict__ digit_start, int32_t* __restrict__ out_ids,
@@ -277,6 +277,8 @@ cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t
   const size_t smem = scatter_smem_bytes(bits);
   cudaError_t e = cudaFuncSetAttribute(k_sort_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(scatter_smem_bytes(kMaxDigitBits)));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_sort_scatter, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   k_sort_scatter<<<unsigned(tiles), kSortThreads, smem, st>>>(
       keys, in_ids, M, shift, bits, hist, tiles, start, out_ids, out_keys, payload, out_payload,
