@@ -135,8 +135,11 @@ RECE_API rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, cons
  *   targets  device int32 [N], positive item of every row, in [0, C)
  *   loss     device fp32 [1]: mean over rows of the per-row loss (0 when N = 0)
  *   row_loss device fp32 [N] or NULL
- *   selected device int32 [N][k]: the kept negatives, best first (score descending,
- *            item id ascending), -1 where a row has fewer than k candidates
+ *   selected device int32 [N][k]: the kept negatives, -1 where a row has fewer than k
+ *            candidates; in RECE_MODE_FP32_EXACT (and with RECE_FLAG_FMA_SCORES) best first
+ *            (score descending, item id ascending), on the tensor-core path in a fixed
+ *            order (by round, then by sorted catalogue position within each selection
+ *            warpgroup's share) -- the set is the same, the order is deterministic
  *   lse      device fp32 [N]: log(exp(l+) + sum over selected exp(l)) per row
  *   logits   device fp32 [N][k+1] or NULL: the logits the loss used, the positive's
  *            first, then those of `selected` (-inf where selected is -1)

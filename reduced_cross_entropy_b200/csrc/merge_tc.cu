@@ -5,14 +5,15 @@
 // j also lies in the row's window of an earlier round r' < r (that round saw the same
 // pair, so the union of the rounds stays de-duplicated -- the RECE paper's ln(count)
 // correction for repeated pairs amounts to counting each pair once).  The k best of the
-// rest by (score descending, item ascending) are found with a warp radix select (4 passes
-// of 8 bits on the score key, then the item ids if the k-th place is tied), ordered best
-// first with a bitonic sort, and give the row's loss (RECE, Algorithm 1's loss lines):
+// rest by (score descending, item ascending) are found with a warp radix select (4-bit
+// digits of the score key from its highest varying bit, then the item ids if the k-th
+// place is tied), kept in the order of the candidate lists (a fixed order), and give the
+// row's loss (RECE, Algorithm 1's loss lines):
 //   lse_i = log(exp(l+) + sum_j exp(l_j)),  loss_i = lse_i - l+.
 // Exactness check: each round recorded the largest score it did not emit; if no list
 // overflowed and every such score is below the k-th kept score, nothing left out could
-// have been selected.  Rows failing the check are counted in the status area (second word) and
-// flagged RECE_DEVICE_INEXACT.
+// have been selected.  Rows failing the check are counted in the status area (second
+// word) and flagged RECE_DEVICE_INEXACT.
 #include "common.cuh"
 #include "plan.h"
 #include "tc.h"
@@ -21,83 +22,88 @@ namespace rece {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kCountBytes = 16 * 32 * 4;  // per-warp digit-count table
 
 struct WarpSel {
-  uint32_t T;
-  int need;
-  int eq;
+  uint32_t T;  // threshold key
+  int need;    // how many keys equal to T are kept
+  int eq;      // how many keys equal T
 };
 
-// Among n elements of the warp (get(q, key) -> in play, its key), the want-th largest key.
+__device__ __forceinline__ uint32_t warp_or(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v |= __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_and(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v &= __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// The want-th largest (1-based) of the warp's keys in play (get(q, key) -> in play, its
+// key; q < n), found four bits at a time from the highest bit in which the keys differ.
+// Each lane counts its own keys in its own column of the 16 x 32 table cnt, so no two
+// lanes ever update one counter.  On return, the kept set is: every key > T, and `need`
+// of the `eq` keys equal to T (all of them when need == eq).  The scan stops early when
+// the digit holding the want-th key is wanted whole; T then carries that digit's prefix
+// with zero bits below it, and every key of the digit is >= T.
 template <typename Get>
-__device__ WarpSel warp_radix_select(int n, int want, Get get, uint32_t* hist) {
+__device__ WarpSel warp_select_kth(int n, int want, Get get, uint32_t* cnt) {
   const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, pmask = 0;
-  int eq = 0;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
+  uint32_t orv = 0u, andv = 0xFFFFFFFFu;
+  int m = 0;
+  for (int q = lane; q < n; q += 32) {
+    uint32_t key;
+    if (get(q, key)) {
+      orv |= key;
+      andv &= key;
+      ++m;
+    }
+  }
+  orv = warp_or(orv);
+  andv = warp_and(andv);
+  m = int(warp_sum(float(m)));  // exact: m <= n < 2^24
+  const uint32_t diff = orv ^ andv;
+  if (diff == 0u) return WarpSel{andv, want, m};
+  int shift = ((31 - __clz(diff)) >> 2) << 2;
+  uint32_t pmask = shift == 28 ? 0u : ~((1u << (shift + 4)) - 1u);
+  uint32_t prefix = andv & pmask;
+  const int hb = lane >> 1, hh = lane & 1;
+  for (;;) {
+#pragma unroll
+    for (int b = 0; b < 16; ++b) cnt[b * 32 + lane] = 0u;
     for (int q = lane; q < n; q += 32) {
       uint32_t key;
-      if (get(q, key) && (key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      if (get(q, key) && (key & pmask) == prefix)
+        atomicAdd(&cnt[((key >> shift) & 15u) * 32 + lane], 1u);
     }
     __syncwarp();
-    int c[8], s = 0;
+    // lanes 2b and 2b+1 add up digit b's 32 columns, half each (rotated: no bank conflict)
+    uint32_t s = 0u;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {  // lane 0 holds the highest 8 bins, highest first
-      c[u] = int(hist[255 - 8 * lane - u]);
-      s += c[u];
-    }
-    int incl = s;
+    for (int t = 0; t < 16; ++t) s += cnt[hb * 32 + hh * 16 + ((t + hb) & 15)];
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
+    // lane l < 16 takes digit 15 - l: digits in descending order along the lanes
+    const uint32_t c0 = __shfl_sync(0xFFFFFFFFu, s, (2 * (15 - lane)) & 31);
+    const int c = lane < 16 ? int(c0) : 0;
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
       if (lane >= o) incl += v;
     }
-    const int excl = incl - s;
-    const bool mine = excl < want && want <= incl;
-    int digit = 0, above = 0, cnt = 0;
-    if (mine) {
-      int run = excl;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (run + c[u] >= want) {
-          digit = 255 - 8 * lane - u;
-          above = run;
-          cnt = c[u];
-          break;
-        }
-        run += c[u];
-      }
-    }
+    const int excl = incl - c;
+    const bool mine = lane < 16 && excl < want && want <= incl;
     const int src = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
-    digit = __shfl_sync(0xFFFFFFFFu, digit, src);
-    above = __shfl_sync(0xFFFFFFFFu, above, src);
-    cnt = __shfl_sync(0xFFFFFFFFu, cnt, src);
+    const int above = __shfl_sync(0xFFFFFFFFu, excl, src);
+    const int count = __shfl_sync(0xFFFFFFFFu, c, src);
     want -= above;
-    eq = cnt;
-    prefix |= uint32_t(digit) << shift;
-    pmask |= 0xFFu << shift;
-    __syncwarp();
-  }
-  return WarpSel{prefix, want, eq};
-}
-
-__device__ void warp_bitonic_sort_asc(uint64_t* a, int P) {
-  const int lane = threadIdx.x & 31;
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int e = lane; e < (P >> 1); e += 32) {
-        const int lo = 2 * stride * (e / stride) + (e % stride), hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const uint64_t x = a[lo], y = a[hi];
-        if ((x > y) == up) {
-          a[lo] = y;
-          a[hi] = x;
-        }
-      }
-      __syncwarp();
-    }
+    prefix |= uint32_t(15 - src) << shift;
+    pmask |= 15u << shift;
+    __syncwarp();  // the table is cleared again by the next pass
+    if (count == want || shift == 0) return WarpSel{prefix, want, count};
+    shift -= 4;
   }
 }
 
@@ -107,17 +113,16 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     const int32_t* __restrict__ py, const int32_t* __restrict__ invX,
     const int32_t* __restrict__ chunkY, const int2* __restrict__ list,
     const int4* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
-    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap, int P,
+    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap,
     int32_t* __restrict__ selected, float* __restrict__ lse_out, float* __restrict__ row_loss,
     float* __restrict__ logits, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t sh_raw[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t per_warp = size_t(P) * 8 + size_t(cap) * 8 + 1024;
+  const size_t per_warp = size_t(cap) * 8 + kCountBytes;
   uint8_t* base = sh_raw + per_warp * wid;
-  uint64_t* sel = reinterpret_cast<uint64_t*>(base);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(base + size_t(P) * 8);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(base);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(base + kCountBytes);
   int32_t* items = reinterpret_cast<int32_t*>(keys + cap);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(items + cap);
 
   const int64_t i = int64_t(blockIdx.x) * warps + wid;
   if (i >= N) return;  // whole warp leaves together; no block-wide barriers below
@@ -128,6 +133,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
   int cx[8];
   for (int r = 0; r < n_r; ++r) cx[r] = int((int64_t(invX[int64_t(r) * N + i]) * n_c) / N);
   int n = 0;
+  uint32_t kmax = 0u;  // largest key buffered by this lane (0: none)
   bool overflow = false;
   float theta_max = -INFINITY;
   for (int r = 0; r < n_r; ++r) {
@@ -173,8 +179,10 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
         if (keep[u]) {
           const int pos = n + __popc(b & ((1u << lane) - 1u));
           if (pos < cap) {
-            keys[pos] = score_key(__int_as_float(e[u].x));
+            const uint32_t key = score_key(__int_as_float(e[u].x));
+            keys[pos] = key;
             items[pos] = jj[u];
+            kmax = key > kmax ? key : kmax;
           }
         }
         n += __popc(b);
@@ -187,52 +195,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
   }
   __syncwarp();
 
-  // the k best
-  const int kk = k < n ? k : n;
-  const bool all = kk >= n;
-  WarpSel s1{0, 0, 0}, s2{0, 0, 0};
-  bool tie = false;
-  if (!all) {
-    s1 = warp_radix_select(
-        n, kk, [&](int q, uint32_t& key) { key = keys[q]; return true; }, hist);
-    if (s1.need != s1.eq) {
-      tie = true;
-      const uint32_t Tk = s1.T;
-      s2 = warp_radix_select(
-          n, s1.need,
-          [&](int q, uint32_t& key) {
-            key = ~uint32_t(items[q]);
-            return keys[q] == Tk;
-          },
-          hist);
-    }
-  }
-  int ns = 0;
-  for (int a0 = 0; a0 < n; a0 += 32) {
-    const int a = a0 + lane;
-    bool take = false;
-    if (a < n) {
-      const uint32_t key = keys[a];
-      take = all || key > s1.T ||
-             (key == s1.T && (!tie || ~uint32_t(items[a]) >= s2.T));
-    }
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, take);
-    if (take) sel[ns + __popc(b & ((1u << lane) - 1u))] = ~cand_key(keys[a], items[a]);
-    ns += __popc(b);
-  }
-  for (int a = ns + lane; a < P; a += 32) sel[a] = ~0ull;
-  __syncwarp();
-  warp_bitonic_sort_asc(sel, P);
-  for (int a = lane; a < k; a += 32) selected[i * k + a] = a < ns ? cand_item(~sel[a]) : -1;
-
-  // theta_max: the largest score some round did not emit (-inf if every round emitted all)
-  const float s_k = ns == k ? key_score(uint32_t((~sel[k - 1]) >> 32)) : -INFINITY;
-  if (lane == 0 && (overflow || (theta_max > -INFINITY && theta_max >= s_k))) {
-    atomicAdd(status + 1, 1u);
-    raise_flag(status, RECE_DEVICE_INEXACT);
-  }
-
-  // loss of the row
+  // the positive's logit
   float part = 0.0f;
   if (z_ok) {
     const T* x = X + i * d;
@@ -240,16 +203,77 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     for (int t = lane; t < d; t += 32) part = fmaf(to_f32(x[t]), to_f32(y[t]), part);
   }
   const float lp = warp_sum(part);
-  if (logits) {
-    float* lg = logits + i * (int64_t(k) + 1);
-    if (lane == 0) lg[0] = z_ok ? lp : NAN;
-    for (int a = lane; a < k; a += 32)
-      lg[1 + a] = a < ns ? key_score(uint32_t((~sel[a]) >> 32)) : -INFINITY;
+
+  // the k best
+  const int kk = k < n ? k : n;
+  const bool all = kk >= n;
+  WarpSel s1{0u, 0, 0}, s2{0u, 0, 0};
+  bool tie = false;
+  if (!all) {
+    s1 = warp_select_kth(
+        n, kk, [&](int q, uint32_t& key) { key = keys[q]; return true; }, cnt);
+    if (s1.need != s1.eq) {
+      tie = true;
+      const uint32_t Tk = s1.T;
+      s2 = warp_select_kth(
+          n, s1.need,
+          [&](int q, uint32_t& key) {
+            key = ~uint32_t(items[q]);
+            return keys[q] == Tk;
+          },
+          cnt);
+    }
   }
-  const float best = ns > 0 ? key_score(uint32_t((~sel[0]) >> 32)) : -INFINITY;
+  // the best candidate is always kept: it bounds the exponentials
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t v = __shfl_xor_sync(0xFFFFFFFFu, kmax, o);
+    kmax = v > kmax ? v : kmax;
+  }
+  const float best = n > 0 ? key_score(kmax) : -INFINITY;
   const float m = fmaxf(lp, best);
-  float acc = 0.0f;
-  for (int a = lane; a < ns; a += 32) acc += expf(key_score(uint32_t((~sel[a]) >> 32)) - m);
+
+  // the kept entries, in the order of the candidate lists (deterministic: rounds, then
+  // each selection warpgroup's emission order), with their logits and exponentials
+  float* lg = logits ? logits + i * (int64_t(k) + 1) : nullptr;
+  int32_t* srow = selected + i * k;
+  int ns = 0;
+  float worst = INFINITY, acc = 0.0f;
+  for (int a0 = 0; a0 < n; a0 += 32) {
+    const int a = a0 + lane;
+    bool take = false;
+    uint32_t key = 0u;
+    if (a < n) {
+      key = keys[a];
+      take = all || key > s1.T || (key == s1.T && (!tie || ~uint32_t(items[a]) >= s2.T));
+    }
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, take);
+    if (take) {
+      const int pos = ns + __popc(b & ((1u << lane) - 1u));
+      const float sc = key_score(key);
+      srow[pos] = items[a];
+      if (lg) lg[1 + pos] = sc;
+      worst = fminf(worst, sc);
+      acc += expf(sc - m);
+    }
+    ns += __popc(b);
+  }
+  worst = -warp_max(-worst);
+  for (int a = ns + lane; a < k; a += 32) {
+    srow[a] = -1;
+    if (lg) lg[1 + a] = -INFINITY;
+  }
+  if (lg && lane == 0) lg[0] = z_ok ? lp : NAN;
+
+  // theta_max: the largest score some round did not emit (-inf if every round emitted
+  // all); the k-th kept score is the smallest kept one
+  const float s_k = ns < k ? -INFINITY : worst;
+  if (lane == 0 && (overflow || (theta_max > -INFINITY && theta_max >= s_k))) {
+    atomicAdd(status + 1, 1u);
+    raise_flag(status, RECE_DEVICE_INEXACT);
+  }
+
+  // loss of the row (RECE, Algorithm 1's loss lines)
   const float tot = warp_sum(acc) + expf(lp - m);
   if (lane == 0) {
     if (!z_ok) {
@@ -273,9 +297,7 @@ int tc_list_capacity(int k);
 int merge_tc_cap(int n_r, int k) { return n_r * (2 * k + 64); }
 
 size_t merge_tc_warp_bytes(int n_r, int k) {
-  int P = 2;
-  while (P < k) P <<= 1;
-  return size_t(P) * 8 + size_t(merge_tc_cap(n_r, k)) * 8 + 1024;
+  return size_t(merge_tc_cap(n_r, k)) * 8 + kCountBytes;
 }
 
 template <typename T>
@@ -286,8 +308,6 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
                             float* row_loss, float* logits, uint32_t* status, cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
-  int P = 2;
-  while (P < c.k) P <<= 1;
   const int Qw = tc_sublist_capacity(c.k);
   const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
   int warps = int((200 * 1024) / per_warp);
@@ -298,7 +318,7 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   if (e != cudaSuccess) return e;
   k_merge_tc<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
       X, Y, targets, py, invX, chunkY, list, list_count, list_theta, c.N, c.C, c.d, c.k, c.n_r,
-      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), P, selected, lse, row_loss, logits, status);
+      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), selected, lse, row_loss, logits, status);
   count_launches(1);
   return cudaGetLastError();
 }

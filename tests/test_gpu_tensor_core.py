@@ -101,3 +101,29 @@ def test_tc_path_recall_and_loss(name):
     oX, oY = oracle.rece_grad(X, Y, t, g["selected"], lse, 1.0)
     assert max_rel(g["dX"], oX) <= 1e-3
     assert max_rel(g["dY"], oY) <= 1e-3
+
+
+@pytest.mark.parametrize("d,n_c,n_ec,n_r,k", [(64, 8, 1, 2, 64), (64, 16, 0, 1, 200),
+                                              (128, 6, 2, 3, 100)])
+def test_tc_path_exact_on_integer_inputs(d, n_c, n_ec, n_r, k):
+    """Integer-valued inputs: every score is exact on the tensor cores and ties are
+    everywhere, so the kept sets (ties to the lower item id) must be the oracle's."""
+    w = synth.Workload("int", N=1000, C=5003, d=d, dtype="bf16", n_b=16, n_c=n_c, n_ec=n_ec,
+                       n_r=n_r, k=k)
+    X, Y, t = synth.integer_inputs(w.N, w.C, d, lo=-2, hi=2, seed=d + k, scale=0.125)
+    B = synth.integer_inputs(n_r * w.n_b, 1, d, lo=-2, hi=2, seed=k, scale=1.0)[0]
+    B = B.reshape(n_r, w.n_b, d)
+    g = run_gpu(w, X, Y, t, B, flags=0, dloss=0.5)
+    o = run_oracle(w, X, Y, t, B, dloss=0.5)
+    assert g["status"] == 0
+    np.testing.assert_array_equal(np.sort(g["selected"], axis=1), np.sort(o["selected"], axis=1))
+    assert abs(g["loss"] - o["loss"]) <= 1e-4 * abs(o["loss"])
+    assert max_rel(g["row_loss"], o["row_loss"]) <= 1e-4
+    assert max_rel(g["dX"], o["dX"]) <= 1e-4 and max_rel(g["dY"], o["dY"]) <= 1e-4
+    # the logits output is the positive's and each kept item's exact score
+    lg, sel = g["logits"], g["selected"]
+    np.testing.assert_array_equal(lg[:, 0], np.einsum("nd,nd->n", X, Y[t]))
+    for i in range(0, w.N, 37):
+        s = sel[i][sel[i] >= 0]
+        np.testing.assert_array_equal(lg[i, 1:1 + len(s)], Y[s] @ X[i])
+        assert np.all(lg[i, 1 + len(s):] == -np.inf)
