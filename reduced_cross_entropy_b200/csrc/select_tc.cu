@@ -4,25 +4,31 @@
 //
 // Work item = (round r, 128 consecutive sorted rows).  Their chunks' windows are a
 // contiguous range of sorted catalogue rows (the union of the windows), streamed by TMA in
-// 256-row tiles; tcgen05.mma forms the 128 x 256 score tile in TMEM.  Each row's thread
+// 128-row tiles; tcgen05.mma forms the 128 x 128 score tile in TMEM.  Each row's thread
 // reads its row of the tile and looks only at columns inside its own window.  The window
 // is streamed three times, the threshold found without any assumption on the scores'
 // distribution:
 //   pass 1  per row: count and max m of its window's scores;
-//   pass 2  per row: exact histogram, in shared memory, of key(m) - key(s) >> 20 where key
-//           is the order-preserving integer image of an fp32 score -- 8 bins per binade
-//           of |s| below m (128 bins, the last one open), so the bins follow the scores'
-//           own scale whatever their distribution;
+//   pass 2  per row: exact histogram, in shared memory, of the distance key(m) - key(s)
+//           >> 20 where key is the order-preserving integer image of an fp32 score -- 8
+//           bins per binade of |s| below m (128 bins, the last one open), so the bins
+//           follow the scores' own scale whatever their distribution.  Scores on the far
+//           side of zero from m fall in the last bin; the distance is one integer
+//           multiply-add on the score's bits (their sign flips with m's);
 //   pass 3  the smallest bin b* whose cumulative count reaches E = 1.25 k + 8 sets the
-//           cut: every score in a bin <= b* is emitted as (score, sorted position) to the
-//           row's list (equal scores share a bin, so a tie is never split); the largest
-//           score NOT emitted is recorded.
+//           cut, turned into the fp32 threshold t at the lower edge of bin b*: every score
+//           >= t is emitted as (score, sorted position) to the row's list (equal scores
+//           share a bin, so a tie is never split).
 // Each of the four epilogue warpgroups (one per 128-column TMEM accumulator, every fourth
 // tile) writes its own sub-list of the row, up to k + 32 entries, and its count of all that
-// passed.  The
-// merge kernel keeps the k best; the selection is exact whenever no list overflowed and
-// every round's largest non-emitted score is below the k-th kept score, which the merge
-// kernel checks row by row.  Score tiles never reach HBM.
+// passed.  The largest fp32 value below t bounds every score not emitted and is recorded
+// per row (-inf when the whole window was emitted).  The merge kernel keeps the k best;
+// the selection is exact whenever no list overflowed and every round's bound is below
+// the k-th kept score, which the merge kernel checks row by row.  Without an overflow
+// the check always passes: the round with the highest threshold emitted at least E > k
+// entries, none of them a duplicate that an earlier round left out (that round's
+// threshold would be higher still), so the k-th kept score is >= every round's
+// threshold.  Score tiles never reach HBM.
 #include "common.cuh"
 #include "plan.h"
 #include "sm100.cuh"
@@ -61,7 +67,6 @@ struct __align__(1024) Smem {
   float part_mx[kAcc][kBM];   // pass 1 partial results of the warpgroups
   int part_cnt[kAcc][kBM];
   int emit_cnt[kAcc][kBM];    // pass 3 entries each warpgroup emitted, per row
-  uint32_t ne_key[kBM];       // pass 3 key of the largest score not emitted, per row
 };
 
 __device__ __forceinline__ void on_timeout(Smem& s, uint32_t* status) {
@@ -73,17 +78,40 @@ struct ItemGeom {
   int r;
   int64_t p0;   // first sorted row of the tile
   int64_t U0;   // union window [U0, U1) in sorted catalogue positions
-  int nt;       // 256-wide tiles covering it
+  int nt;       // kBN-wide tiles covering it
 };
 
-// Order-preserving integer image of an fp32 score (a < b  <=>  key(a) < key(b)).
-__device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return u ^ (uint32_t(int32_t(u) >> 31) | 0x80000000u);
+// Distance bins of pass 2: bin(s) = min((sig * bits(s) + off) >> 20, 127) equals
+// min((key(m) - key(s)) >> 20, 127) for every score s <= m on m's side of zero, where key
+// is the order-preserving integer image of an fp32 value: for m > 0 (or +0),
+// key(m) - key(s) = bits(m) - bits(s); for m < 0 (or -0), it is bits(s) - bits(m).
+// A score on the other side of zero wraps to a distance of at least bits(|m|) + 2^31 -
+// bits(|s|), which puts it in the open last bin unless |s| exceeds |m| by some 2^110;
+// such a score only misplaces the cut (the emission itself compares values, so the
+// exactness check below stays sound).
+struct BinMap {
+  uint32_t sig, off;
+};
+__device__ __forceinline__ BinMap bin_map(float m) {
+  const uint32_t bm = __float_as_uint(m);
+  return (bm & 0x80000000u) ? BinMap{1u, 0u - bm} : BinMap{0xFFFFFFFFu, bm};
 }
 
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+// The fp32 threshold t of the cut "distance < L" (L = (b* + 1) << 20): a score s <= m on
+// m's side of zero has distance < L exactly when s >= t.  -inf when every score passes.
+__device__ __forceinline__ float cut_threshold(float m, uint32_t L) {
+  const uint32_t bm = __float_as_uint(m);
+  if (!(bm & 0x80000000u)) return bm >= L ? __uint_as_float(bm - L + 1u) : 0.0f;
+  const uint64_t tb = uint64_t(bm) + L - 1u;  // a negative value L - 1 ulps beyond m
+  return tb < 0xFF800000ull ? __uint_as_float(uint32_t(tb)) : -INFINITY;
+}
+
+// The largest fp32 value below t (t finite or +0/-0): every score < t is <= it.
+__device__ __forceinline__ float value_below(float t) {
+  const uint32_t b = __float_as_uint(t);
+  if (t > 0.0f) return __uint_as_float(b - 1u);
+  if (t == 0.0f) return __uint_as_float(0x80000001u);
+  return __uint_as_float(b + 1u);
 }
 
 __device__ __forceinline__ int64_t chunk_of(int64_t p, int64_t M, int n_c) {
@@ -226,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
         w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
       }
       int cnt = 0;
-      float mx = -INFINITY, not_emitted = -INFINITY;
-      uint32_t kmx = 0;     // key of the row's max
-      uint32_t limit = 0;   // pass 3 emits a score iff key(m) - key(s) < limit
-      bool histo = false;   // pass 2 needed (else every window score is emitted)
+      float mx = -INFINITY;
+      BinMap bmap{0u, 0u};   // pass 2 distance bins of this row
+      float thr = -INFINITY; // pass 3 emits a score iff score >= thr
+      bool histo = false;    // pass 2 needed (else every window score is emitted)
       uint32_t* hcol = &s.hist[0][row_local];
       int2* out = list + ((int64_t(g.r) * N + (valid ? p : 0)) * kAcc + wg) * Qw;
       int emitted = 0;
@@ -240,7 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           s.part_mx[wg][row_local] = mx;
           s.part_cnt[wg][row_local] = cnt;
           for (int b = wg * (kBins / kAcc); b < (wg + 1) * (kBins / kAcc); ++b) hcol[b * kBM] = 0;
-          if (wg == 0) s.ne_key[row_local] = 0;
           named_barrier(1, kEpiThreads);
           mx = s.part_mx[0][row_local];
           cnt = s.part_cnt[0][row_local];
@@ -250,16 +277,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
             cnt += s.part_cnt[w][row_local];
           }
           histo = valid && cnt > E;
-          kmx = order_key(mx);
-          limit = 0xFFFFFFFFu;  // emit everything unless pass 2 finds a cut
+          bmap = bin_map(mx);
         } else if (pass == 2) {
           named_barrier(1, kEpiThreads);  // every histogram increment has landed
-          if (histo) {
+          if (histo) {  // else thr stays -inf: emit the whole window
             uint32_t cum = 0;
             for (int b = 0; b < kBins - 1; ++b) {
               cum += hcol[b * kBM];
               if (cum >= uint32_t(E)) {
-                limit = uint32_t(b + 1) << 20;
+                thr = cut_threshold(mx, uint32_t(b + 1) << 20);
                 break;
               }
             }
@@ -275,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           }
           tc_fence_after();
           const int64_t q0 = g.U0 + int64_t(t) * kBN;
+          const int32_t q32 = int32_t(q0);  // sorted positions are < C < 2^31
           const uint32_t taddr = tmem + (uint32_t(q4 * 32) << 16) + uint32_t(a * kBN);
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 32) {
@@ -295,16 +322,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
               } else if (pass == 1) {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                  const uint32_t raw = (kmx - order_key(v[u])) >> 20;
+                  const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
                   atomicAdd(&hcol[min(raw, uint32_t(kBins - 1)) * kBM], 1u);
                 }
               } else {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                  const bool e = kmx - order_key(v[u]) < limit;
-                  if (e && emitted < Qw) out[emitted] = make_int2(__float_as_int(v[u]), int32_t(qa + u));
+                  const bool e = v[u] >= thr;
+                  if (e && emitted < Qw)
+                    out[emitted] = make_int2(__float_as_int(v[u]), q32 + c0 + u);
                   emitted += e ? 1 : 0;
-                  not_emitted = e ? not_emitted : fmaxf(not_emitted, v[u]);
                 }
               }
             } else {
@@ -316,13 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
                   ++cnt;
                   mx = fmaxf(mx, v[u]);
                 } else if (pass == 1) {
-                  const uint32_t raw = (kmx - order_key(v[u])) >> 20;
+                  const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
                   atomicAdd(&hcol[min(raw, uint32_t(kBins - 1)) * kBM], 1u);
                 } else {
-                  const bool e = kmx - order_key(v[u]) < limit;
-                  if (e && emitted < Qw) out[emitted] = make_int2(__float_as_int(v[u]), int32_t(qa + u));
+                  const bool e = v[u] >= thr;
+                  if (e && emitted < Qw)
+                    out[emitted] = make_int2(__float_as_int(v[u]), q32 + c0 + u);
                   emitted += e ? 1 : 0;
-                  not_emitted = e ? not_emitted : fmaxf(not_emitted, v[u]);
                 }
               }
             }
@@ -332,14 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           if (lane == 0) mbar_arrive(&s.acc_empty[a]);
         }
       }
-      if (not_emitted > -INFINITY) atomicMax(&s.ne_key[row_local], order_key(not_emitted));
       s.emit_cnt[wg][row_local] = emitted;
       named_barrier(1, kEpiThreads);
       if (wg == 0 && ok && valid) {
-        const uint32_t nk2 = s.ne_key[row_local];
         list_count[int64_t(g.r) * N + p] = make_int4(s.emit_cnt[0][row_local], s.emit_cnt[1][row_local],
                                                      s.emit_cnt[2][row_local], s.emit_cnt[3][row_local]);
-        list_theta[int64_t(g.r) * N + p] = nk2 == 0 ? -INFINITY : key_to_float(nk2);
+        list_theta[int64_t(g.r) * N + p] = thr == -INFINITY ? -INFINITY : value_below(thr);
       }
     }
   }
