@@ -113,25 +113,27 @@ KERNEL_SOURCES = {
     "merge_loss": ["loss.cu"], "mean": ["loss.cu"], "bwd_rows": ["backward.cu"],
     "bwd_sort": ["sort.cu"], "bwd_items": ["backward.cu"],
 }
+KERNEL_SOURCES_TC = dict(KERNEL_SOURCES, bucketize=["bucketize_tc.cu", "permute.cu"],
+                         select=["select_tc.cu", "sm100.cuh"], merge_loss=["merge_tc.cu"])
 
 
-def source_hash(stage):
+def source_hash(stage, tc):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES[stage]:
+    for f in (KERNEL_SOURCES_TC if tc else KERNEL_SOURCES)[stage]:
         h.update(open(os.path.join(ROOT, "reduced_cross_entropy_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(stage, workload):
-    """DRAM bytes per launch of this stage from a committed ncu capture, if the kernel
-    source is unchanged since (else None)."""
+def recorded_traffic(stage, workload, tc):
+    """DRAM bytes per step of this stage (all its launches) from a committed ncu capture,
+    if the kernel source is unchanged since (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(f"{stage}@{workload}")
-    if not d or d.get("source_sha") != source_hash(stage):
+    d = json.load(open(p)).get(f"{stage}@{workload}{'@tc' if tc else ''}")
+    if not d or d.get("source_sha") != source_hash(stage, tc):
         return None
-    return d.get("dram_bytes_per_launch")
+    return d.get("dram_bytes_per_step")
 
 
 # ------------------------------------------------------------------ clocks
@@ -357,26 +359,32 @@ def main():
                 for i, name in enumerate(_lib.STAGES)}
     value = world * w.N * args.steps / (total_ms / 1000.0)
 
-    # roofline of the dominant stage
+    # roofline of every stage, the dominant one reported as the line's roofline
     peaks = load_peaks()
     work = stage_work(w)
-    dom = max(stage_ms, key=stage_ms.get)
-    bound = stage_bound(dom, w, args.flags)
-    flops, bytes_ = work[dom]
-    sec = stage_ms[dom] / 1000.0
-    if bound == "hbm":
-        achieved, peak, unit = bytes_ / sec / 1e9, peaks["hbm_gbs"], "GB/s"
-    elif bound == "tensor":
-        achieved, peak, unit = flops / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    else:  # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
-        achieved, peak, unit = flops / sec / 1e12, 148 * 128 * 2 * peaks["sm_max_mhz"] / 1e6, \
-            "TFLOP/s"
-    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+    tc = uses_tensor_cores(w, args.flags)
+
+    def stage_roofline(name):
+        bound = stage_bound(name, w, args.flags)
+        flops, bytes_ = work[name]
+        sec = stage_ms[name] / 1000.0
+        if bound == "hbm":
+            achieved, peak, unit = bytes_ / sec / 1e9, peaks["hbm_gbs"], "GB/s"
+        elif bound == "tensor":
+            achieved, peak, unit = flops / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        else:  # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+            achieved, peak, unit = (flops / sec / 1e12,
+                                    148 * 128 * 2 * peaks["sm_max_mhz"] / 1e6, "TFLOP/s")
+        return {"bound": bound, "kernel": name, "achieved": achieved, "peak": peak,
                 "unit": unit, "frac": achieved / peak,
                 "peak_source": peaks["source"] if bound != "alu" else
                 "derived: 148 SM x 128 FP32 lanes x 2 x sm_max_mhz",
-                "traffic": recorded_traffic(dom, w.name),
+                "traffic": recorded_traffic(name, w.name, tc),
                 "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
+
+    dom = max(stage_ms, key=stage_ms.get)
+    roofline = stage_roofline(dom)
+    stage_fracs = {name: round(stage_roofline(name)["frac"], 4) for name in stage_ms}
 
     # end to end: host (pinned) inputs copied in, loss copied out, every step
     Xh = torch.from_numpy(X).to(tdt).pin_memory()
@@ -418,7 +426,8 @@ def main():
                        "l2": "flushed between timed steps (256 MiB write)",
                        "scores": "tcgen05" if uses_tensor_cores(w, args.flags)
                        else "fmaf CUDA cores"},
-            "roofline": roofline, "stages_ms": stage_ms, "e2e": e2e, "gpu_launches": int(launches),
+            "roofline": roofline, "stages_ms": stage_ms, "stages_roofline_frac": stage_fracs,
+            "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk.summary()}
 
     if rank == 0 and world == 1 and not args.no_memory:

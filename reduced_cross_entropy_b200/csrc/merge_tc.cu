@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
 
 int tc_list_capacity(int k);
 
-// Candidates buffered per row: the selection emits about 1.25k + (one histogram bin) per
+// Candidates buffered per row: the selection emits about k + 1 + (one histogram bin) per
 // round, so 2k + 64 per round leaves ample room; a row with more is flagged inexact.
 int merge_tc_cap(int n_r, int k) { return n_r * (2 * k + 64); }
 

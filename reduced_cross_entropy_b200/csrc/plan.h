@@ -30,6 +30,32 @@ inline size_t sort_scratch_bytes(int64_t M, int bits) {
          align256(sizeof(int32_t) * size_t(digits + 1));
 }
 
+// One independent counting sort of a batch (see launch_sort_batch): its keys (read by id,
+// or in position order), M elements, histogram scratch (digits x tiles ints), the
+// digits + 1 starts it writes, and its outputs.  `tiles` is filled in by the launcher.
+struct SortSeg {
+  const int32_t* keys;
+  const int32_t* in_ids;
+  int64_t M;
+  int32_t* hist;
+  int64_t tiles;
+  int32_t* start;
+  int32_t* out_ids;
+  int32_t* out_keys;
+  const float* payload;
+  float* out_payload;
+};
+constexpr int kMaxSortSegs = 16;
+struct SortBatch {
+  SortSeg seg[kMaxSortSegs];
+  int n, shift, bits;
+  bool in_order;
+};
+// Histogram scratch of one batch segment of M elements.
+inline size_t sort_hist_bytes(int64_t M, int bits) {
+  return align256(sizeof(int32_t) * size_t(ceil_div(M, kSortTile) << bits));
+}
+
 struct Layout {
   size_t status = 0;
   // forward region (from rece_bucketize_sort to the end of rece_loss_fwd)
@@ -91,6 +117,8 @@ cudaError_t launch_bucketize_fma(const T* V, int64_t M, int d, const T* B, int n
 // digit_start[2^bits] = M).
 // With in_order, element p's key and payload are keys[p] and payload[p] (a previous pass
 // wrote them in the order of its output) instead of being looked up by id.
+cudaError_t launch_sort_batch(const SortSeg* segs, int n, int shift, int bits, bool in_order,
+                              cudaStream_t st);
 cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,
                              int bits, void* scratch, int32_t* out_ids, int32_t* out_keys,
                              int32_t* digit_start, cudaStream_t st,

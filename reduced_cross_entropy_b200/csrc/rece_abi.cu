@@ -71,7 +71,9 @@ void build_layout(rece_plan_s& p) {
   L.py = take(sizeof(int32_t) * c.n_r * c.C);
   L.bstart_x = take(sizeof(int32_t) * c.n_r * nb_stride);
   L.bstart_y = take(sizeof(int32_t) * c.n_r * nb_stride);
-  L.sort_scratch = take(sort_scratch_bytes(c.N > c.C ? c.N : c.C, p.bucket_bits));
+  // the forward sorts (X and Y of every round) run as one batch, a histogram each
+  L.sort_scratch = take(size_t(c.n_r) * (sort_hist_bytes(c.N, p.bucket_bits) +
+                                         sort_hist_bytes(c.C, p.bucket_bits)));
   if (p.use_tc) {
     const size_t Q = size_t(tc_list_capacity(c.k));
     L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
@@ -264,18 +266,23 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   stage_mark(*plan, RECE_STAGE_BUCKETIZE, 1, st);
   stage_mark(*plan, RECE_STAGE_SORT, 0, st);
   const size_t stride = (size_t(1) << plan->bucket_bits) + 1;
+  SortSeg segs[kMaxSortSegs];
+  char* hist = ws + L.sort_scratch;
   for (int r = 0; r < c.n_r; ++r) {
-    RECE_CUDA(launch_sort_pass(bx + int64_t(r) * c.N, nullptr, c.N, 0, plan->bucket_bits,
-                               ws + L.sort_scratch,
-                               reinterpret_cast<int32_t*>(ws + L.px) + int64_t(r) * c.N, nullptr,
-                               reinterpret_cast<int32_t*>(ws + L.bstart_x) + r * stride, st),
-              "sort X");
-    RECE_CUDA(launch_sort_pass(by + int64_t(r) * c.C, nullptr, c.C, 0, plan->bucket_bits,
-                               ws + L.sort_scratch,
-                               reinterpret_cast<int32_t*>(ws + L.py) + int64_t(r) * c.C, nullptr,
-                               reinterpret_cast<int32_t*>(ws + L.bstart_y) + r * stride, st),
-              "sort Y");
+    for (int side = 0; side < 2; ++side) {
+      const int64_t M = side == 0 ? c.N : c.C;
+      SortSeg& g = segs[2 * r + side];
+      g = SortSeg{};
+      g.keys = (side == 0 ? bx : by) + int64_t(r) * M;
+      g.M = M;
+      g.hist = reinterpret_cast<int32_t*>(hist);
+      hist += sort_hist_bytes(M, plan->bucket_bits);
+      g.start = reinterpret_cast<int32_t*>(ws + (side == 0 ? L.bstart_x : L.bstart_y)) + r * stride;
+      g.out_ids = reinterpret_cast<int32_t*>(ws + (side == 0 ? L.px : L.py)) + int64_t(r) * M;
+    }
   }
+  RECE_CUDA(launch_sort_batch(segs, 2 * c.n_r, 0, plan->bucket_bits, false, st),
+            "sort X and Y");
   if (plan->use_tc) {
     RECE_CUDA(launch_permute_rows(X, c.N, c.d, reinterpret_cast<const int32_t*>(ws + L.px),
                                   c.n_r, c.n_c, ws + L.xs,

@@ -8,27 +8,28 @@
 // reads its row of the tile and looks only at columns inside its own window.  The window
 // is streamed three times, the threshold found without any assumption on the scores'
 // distribution:
-//   pass 1  per row: count and max m of its window's scores;
-//   pass 2  per row: exact histogram, in shared memory, of the distance key(m) - key(s)
-//           >> 20 where key is the order-preserving integer image of an fp32 score -- 8
-//           bins per binade of |s| below m (128 bins, the last one open), so the bins
-//           follow the scores' own scale whatever their distribution.  Scores on the far
-//           side of zero from m fall in the last bin; the distance is one integer
-//           multiply-add on the score's bits (their sign flips with m's);
-//   pass 3  the smallest bin b* whose cumulative count reaches E = 1.25 k + 8 sets the
+//   pass 1  per row: max m of a strided quarter of its window's scores (the first 32
+//           columns of every tile; all of them when the window is short);
+//   pass 2  per row: exact histogram, in shared memory, of the distance key(A) - key(s)
+//           >> 20 where key is the order-preserving integer image of an fp32 score and A
+//           lies two binades beyond m -- 8 bins per binade of |s| (128 bins, the last one
+//           open), so the bins follow the scores' own scale whatever their distribution.
+//           The distance is one integer multiply-add on the score's bits;
+//   pass 3  the smallest bin b* whose cumulative count reaches E = k + 1 sets the
 //           cut, turned into the fp32 threshold t at the lower edge of bin b*: every score
 //           >= t is emitted as (score, sorted position) to the row's list (equal scores
-//           share a bin, so a tie is never split).
+//           share a bin, so a tie is never split).  Each thread builds the bit mask of its
+//           32 columns that pass and spends work only on the set bits.
 // Each of the four epilogue warpgroups (one per 128-column TMEM accumulator, every fourth
 // tile) writes its own sub-list of the row, up to k + 32 entries, and its count of all that
 // passed.  The largest fp32 value below t bounds every score not emitted and is recorded
 // per row (-inf when the whole window was emitted).  The merge kernel keeps the k best;
 // the selection is exact whenever no list overflowed and every round's bound is below
 // the k-th kept score, which the merge kernel checks row by row.  Without an overflow
-// the check always passes: the round with the highest threshold emitted at least E > k
-// entries, none of them a duplicate that an earlier round left out (that round's
-// threshold would be higher still), so the k-th kept score is >= every round's
-// threshold.  Score tiles never reach HBM.
+// the check always passes: the round with the highest threshold emitted at least
+// E = k + 1 entries, at least k of them negatives and none of them a duplicate that an
+// earlier round left out (that round's threshold would be higher still), so the k-th
+// kept score is >= every round's threshold.  Score tiles never reach HBM.
 #include "common.cuh"
 #include "plan.h"
 #include "sm100.cuh"
@@ -42,6 +43,8 @@ using namespace sm100;
 constexpr int kStages = 4;
 constexpr int kPasses = 3;
 constexpr int kBins = 128;
+constexpr int kHeadBins = 16;          // bins above the pass 1 max (2 binades)
+constexpr int kSampleAllBelow = 1024;  // windows shorter than this are looked at whole
 constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kBK = 64;
@@ -52,6 +55,7 @@ constexpr int kAcc = 4;       // TMEM accumulators of kBN columns, one per epilo
 constexpr int kEpiWarps = 4 * kAcc;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
+static_assert(kBins * kBM == kEpiThreads * 32, "pass 3 staging fills the histogram space");
 
 struct __align__(1024) Smem {
   uint8_t a[kStages][kStageABytes];
@@ -63,9 +67,9 @@ struct __align__(1024) Smem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  uint32_t hist[kBins][kBM];  // per row (column) histogram of pass 2
-  float part_mx[kAcc][kBM];   // pass 1 partial results of the warpgroups
-  int part_cnt[kAcc][kBM];
+  // per row (column) histogram of pass 2; pass 3 reuses the space to stage scores
+  __align__(16) uint32_t hist[kBins][kBM];
+  float part_mx[kAcc][kBM];   // pass 1 partial maxima of the warpgroups
   int emit_cnt[kAcc][kBM];    // pass 3 entries each warpgroup emitted, per row
 };
 
@@ -81,29 +85,39 @@ struct ItemGeom {
   int nt;       // kBN-wide tiles covering it
 };
 
-// Distance bins of pass 2: bin(s) = min((sig * bits(s) + off) >> 20, 127) equals
-// min((key(m) - key(s)) >> 20, 127) for every score s <= m on m's side of zero, where key
-// is the order-preserving integer image of an fp32 value: for m > 0 (or +0),
-// key(m) - key(s) = bits(m) - bits(s); for m < 0 (or -0), it is bits(s) - bits(m).
-// A score on the other side of zero wraps to a distance of at least bits(|m|) + 2^31 -
-// bits(|s|), which puts it in the open last bin unless |s| exceeds |m| by some 2^110;
-// such a score only misplaces the cut (the emission itself compares values, so the
-// exactness check below stays sound).
+// Distance bins of pass 2.  The anchor A is the bit pattern of a value 16 bins (two
+// binades) beyond the pass 1 max m, away from zero, so that scores a little above m --
+// pass 1 may have looked at a sample only -- still get bins of their own.  For m >= 0 the
+// distance of a score s is A - bits(s), for m < 0 it is bits(s) - A: in both cases
+// key(anchor) - key(s) with key the order-preserving integer image of an fp32 value, as
+// long as s lies between zero and the anchor.  Bin = min(distance >> 20, 127): 8 bins per
+// binade of |s|.  Any other score (beyond the anchor, or on the far side of zero) wraps
+// to a huge distance, normally the open last bin; that only misplaces the cut, since
+// the emission itself compares values and the exactness check below stays sound.
 struct BinMap {
-  uint32_t sig, off;
+  uint32_t sig, off, anchor;
 };
 __device__ __forceinline__ BinMap bin_map(float m) {
+  constexpr uint32_t H = uint32_t(kHeadBins) << 20;
   const uint32_t bm = __float_as_uint(m);
-  return (bm & 0x80000000u) ? BinMap{1u, 0u - bm} : BinMap{0xFFFFFFFFu, bm};
+  if (!(bm & 0x80000000u)) {
+    const uint32_t A = bm > 0x7F7FFFFFu - H ? 0x7F7FFFFFu : bm + H;
+    return BinMap{0xFFFFFFFFu, A, A};
+  }
+  const uint32_t A = bm - H < 0x80000000u ? 0x80000000u : bm - H;
+  return BinMap{1u, 0u - A, A};
 }
 
-// The fp32 threshold t of the cut "distance < L" (L = (b* + 1) << 20): a score s <= m on
-// m's side of zero has distance < L exactly when s >= t.  -inf when every score passes.
-__device__ __forceinline__ float cut_threshold(float m, uint32_t L) {
-  const uint32_t bm = __float_as_uint(m);
-  if (!(bm & 0x80000000u)) return bm >= L ? __uint_as_float(bm - L + 1u) : 0.0f;
-  const uint64_t tb = uint64_t(bm) + L - 1u;  // a negative value L - 1 ulps beyond m
+// The fp32 threshold t of the cut "distance < L" (L = (b* + 1) << 20): a score between
+// zero and the anchor has distance < L exactly when s >= t.  -inf when every score passes.
+__device__ __forceinline__ float cut_threshold(const BinMap& b, uint32_t L) {
+  if (b.sig != 1u) return b.anchor >= L ? __uint_as_float(b.anchor - L + 1u) : 0.0f;
+  const uint64_t tb = uint64_t(b.anchor) + L - 1u;  // L - 1 ulps beyond the anchor
   return tb < 0xFF800000ull ? __uint_as_float(uint32_t(tb)) : -INFINITY;
+}
+
+__device__ __forceinline__ void red_shared_add1(uint32_t addr) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr));
 }
 
 // The largest fp32 value below t (t finite or +0/-0): every score < t is <= it.
@@ -241,55 +255,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
     const int wg = (warp - 2) >> 2;
     const int q4 = warp & 3;  // TMEM lane quarter this warp may access
     const int row_local = q4 * 32 + lane;
+    const int et = threadIdx.x - 64;  // epilogue thread 0..kEpiThreads-1
+    const uint32_t hcol = smem_u32(&s.hist[0][row_local]);
+    // pass 3 staging of this thread's 32 scores (the histogram's space, free by then);
+    // 16-byte slot j of the thread sits at j ^ (et & 7): conflict-free vector stores
+    float* stage = reinterpret_cast<float*>(&s.hist[0][0]) + et * 32;
+    const int swz = et & 7;
     uint32_t acc_it = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
       const ItemGeom g = item_geom(item, tiles_per_round, N, C, n_c, n_ec);
       const int64_t p = g.p0 + row_local;
       const bool valid = p < N;
-      int64_t w0 = 0, w1 = 0;  // this row's window, in sorted catalogue positions
+      int32_t w0 = 0, w1 = 0;  // this row's window, in sorted catalogue positions (< C)
       if (valid) {
         const int64_t c = chunk_of(p, N, n_c);
-        w0 = chunk_start(c - n_ec < 0 ? 0 : c - n_ec, C, n_c);
-        w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
+        w0 = int32_t(chunk_start(c - n_ec < 0 ? 0 : c - n_ec, C, n_c));
+        w1 = int32_t(chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c));
       }
-      int cnt = 0;
-      float mx = -INFINITY;
-      BinMap bmap{0u, 0u};   // pass 2 distance bins of this row
-      float thr = -INFINITY; // pass 3 emits a score iff score >= thr
-      bool histo = false;    // pass 2 needed (else every window score is emitted)
-      uint32_t* hcol = &s.hist[0][row_local];
+      // pass 1 looks at the first 32 columns of every tile (a strided quarter of the
+      // window) unless the window is short, then at all of it
+      const bool sample_all = w1 - w0 < kSampleAllBelow;
+      const bool histo = valid && w1 - w0 > E;  // else every window score is emitted
+      float mx = -INFINITY;  // pass 1: max of the looked-at scores
+      BinMap bmap{0u, 0u, 0u};
+      float thr = -INFINITY;  // pass 3 emits a score iff score >= thr
       int2* out = list + ((int64_t(g.r) * N + (valid ? p : 0)) * kAcc + wg) * Qw;
       int emitted = 0;
       for (int pass = 0; pass < kPasses; ++pass) {
         if (pass == 1) {
-          // combine the warpgroups' max / count; reset this item's shared state
+          // combine the warpgroups' maxima; reset this item's histogram
           named_barrier(1, kEpiThreads);
           s.part_mx[wg][row_local] = mx;
-          s.part_cnt[wg][row_local] = cnt;
-          for (int b = wg * (kBins / kAcc); b < (wg + 1) * (kBins / kAcc); ++b) hcol[b * kBM] = 0;
+          for (int b = wg * (kBins / kAcc); b < (wg + 1) * (kBins / kAcc); ++b)
+            s.hist[b][row_local] = 0;
           named_barrier(1, kEpiThreads);
           mx = s.part_mx[0][row_local];
-          cnt = s.part_cnt[0][row_local];
 #pragma unroll
-          for (int w = 1; w < kAcc; ++w) {
-            mx = fmaxf(mx, s.part_mx[w][row_local]);
-            cnt += s.part_cnt[w][row_local];
-          }
-          histo = valid && cnt > E;
+          for (int w = 1; w < kAcc; ++w) mx = fmaxf(mx, s.part_mx[w][row_local]);
           bmap = bin_map(mx);
         } else if (pass == 2) {
           named_barrier(1, kEpiThreads);  // every histogram increment has landed
-          if (histo) {  // else thr stays -inf: emit the whole window
+          if (histo) {
             uint32_t cum = 0;
             for (int b = 0; b < kBins - 1; ++b) {
-              cum += hcol[b * kBM];
+              cum += s.hist[b][row_local];
               if (cum >= uint32_t(E)) {
-                thr = cut_threshold(mx, uint32_t(b + 1) << 20);
+                thr = cut_threshold(bmap, uint32_t(b + 1) << 20);
                 break;
               }
             }
           }
+          named_barrier(1, kEpiThreads);  // histogram read by all: its space is staging now
         }
         for (int t = 0; t < g.nt; ++t, ++acc_it) {
           const int a = acc_it % kAcc;
@@ -300,57 +317,65 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
             continue;  // keep the loop structure so every barrier is still met
           }
           tc_fence_after();
-          const int64_t q0 = g.U0 + int64_t(t) * kBN;
-          const int32_t q32 = int32_t(q0);  // sorted positions are < C < 2^31
+          const int32_t q0 = int32_t(g.U0) + t * kBN;  // sorted positions are < C < 2^31
           const uint32_t taddr = tmem + (uint32_t(q4 * 32) << 16) + uint32_t(a * kBN);
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 32) {
-            const int64_t qa = q0 + c0;
-            const bool need = valid && qa < w1 && qa + 32 > w0 && (pass != 1 || histo);
+            const int32_t qa = q0 + c0;
+            const bool need = valid && qa < w1 && qa + 32 > w0 &&
+                              (pass != 0 || c0 == 0 || sample_all) && (pass != 1 || histo);
             if (!__any_sync(0xFFFFFFFFu, need)) continue;
             float v[32];
             tmem_load32(taddr + c0, v);
             if (!need) continue;
-            if (qa >= w0 && qa + 32 <= w1) {
-              // chunk entirely inside the row's window: no per-column test
-              if (pass == 0) {
-                cnt += 32;
+            const int lo = w0 > qa ? w0 - qa : 0, hi = w1 < qa + 32 ? w1 - qa : 32;
+            const bool full = lo == 0 && hi == 32;
+            if (pass == 0) {
+              if (full) {
                 float m4[4] = {mx, v[0], v[1], v[2]};
 #pragma unroll
                 for (int u = 3; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
                 mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-              } else if (pass == 1) {
+              } else {
+#pragma unroll
+                for (int u = 0; u < 32; ++u)
+                  if (u >= lo && u < hi) mx = fmaxf(mx, v[u]);
+              }
+            } else if (pass == 1) {
+              if (full) {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
-                  atomicAdd(&hcol[min(raw, uint32_t(kBins - 1)) * kBM], 1u);
+                  red_shared_add1(hcol + min(raw, uint32_t(kBins - 1)) * (kBM * 4));
                 }
               } else {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
-                  const bool e = v[u] >= thr;
-                  if (e && emitted < Qw)
-                    out[emitted] = make_int2(__float_as_int(v[u]), q32 + c0 + u);
-                  emitted += e ? 1 : 0;
+                  if (u < lo || u >= hi) continue;
+                  const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
+                  red_shared_add1(hcol + min(raw, uint32_t(kBins - 1)) * (kBM * 4));
                 }
               }
             } else {
-              const int lo = int(w0 > qa ? w0 - qa : 0), hi = int(w1 < qa + 32 ? w1 - qa : 32);
+              // the bit mask of passing columns (four independent partial masks), then one
+              // step per set bit
+              uint32_t mk[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-              for (int u = 0; u < 32; ++u) {
-                if (u < lo || u >= hi) continue;
-                if (pass == 0) {
-                  ++cnt;
-                  mx = fmaxf(mx, v[u]);
-                } else if (pass == 1) {
-                  const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
-                  atomicAdd(&hcol[min(raw, uint32_t(kBins - 1)) * kBM], 1u);
-                } else {
-                  const bool e = v[u] >= thr;
-                  if (e && emitted < Qw)
-                    out[emitted] = make_int2(__float_as_int(v[u]), q32 + c0 + u);
-                  emitted += e ? 1 : 0;
-                }
+              for (int u = 0; u < 32; ++u) mk[u & 3] |= (v[u] >= thr ? 1u : 0u) << u;
+              uint32_t mask = (mk[0] | mk[1]) | (mk[2] | mk[3]);
+              if (!full) mask &= (hi == 32 ? 0xFFFFFFFFu : (1u << hi) - 1u) & ~((1u << lo) - 1u);
+              if (mask) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  *reinterpret_cast<float4*>(stage + 4 * (j ^ swz)) =
+                      make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                do {
+                  const int u = __ffs(mask) - 1;
+                  mask &= mask - 1u;
+                  const float val = stage[4 * ((u >> 2) ^ swz) + (u & 3)];
+                  if (emitted < Qw) out[emitted] = make_int2(__float_as_int(val), qa + u);
+                  ++emitted;
+                } while (mask);
               }
             }
           }
@@ -380,10 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
 }  // namespace
 
 // Capacity of each warpgroup's sub-list of a (round, row): a warpgroup sees a quarter of
-// the window, so k + 32 leaves wide room above its share of the ~1.25k emitted scores.
+// the window, so k + 32 leaves wide room above its share of the ~k emitted scores.
 int tc_sublist_capacity(int k) { return k + 32; }
 int tc_list_capacity(int k) { return kAcc * tc_sublist_capacity(k); }
-int tc_emit_target(int k) { return k + k / 4 + 8; }
+// k + 1: the positive may be among the emitted, and k others still give the exactness
+// check its margin (see the file comment).
+int tc_emit_target(int k) { return k + 1; }
 
 cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys, int2* list,
                              int4* list_count, float* list_theta, uint32_t* status,

@@ -3,12 +3,14 @@
 // passes of an LSD radix sort of the backward's (item, row) pairs.
 //
 // One pass over M elements with b-bit digits:
-//   hist     per tile of 4096 elements, the count of every digit (digit-major matrix)
+//   hist     per tile of 2048 elements, the count of every digit (digit-major matrix)
 //   scan     exclusive prefix over tiles for every digit, then over digits
-//   scatter  every warp walks its 512 elements in order; __match_any_sync groups the
+//   scatter  every warp walks its 256 elements in order; __match_any_sync groups the
 //            lanes holding the same digit, so an element's rank is the number of
 //            earlier elements with its digit: in earlier tiles, earlier warps of its
 //            tile, earlier steps of its warp, lower lanes of its step.  Stable.
+// Several independent sorts (segments) of one digit width go in one launch sequence:
+// blockIdx.y is the segment, blockIdx.x the tile (or digit) within it.
 #include "common.cuh"
 #include "plan.h"
 
@@ -29,13 +31,12 @@ __device__ __forceinline__ int32_t elem_key(const int32_t* keys, const int32_t* 
   return in_order ? keys[p] : keys[elem_id(in_ids, p)];
 }
 
-__global__ void __launch_bounds__(kSortThreads) k_sort_hist(const int32_t* __restrict__ keys,
-                                                            const int32_t* __restrict__ in_ids,
-                                                            int64_t M, int shift, int bits,
-                                                            int32_t* __restrict__ hist,
-                                                            int64_t tiles, bool in_order) {
+template <bool kMulti>
+__global__ void __launch_bounds__(kSortThreads) k_sort_hist(const __grid_constant__ SortBatch b) {
+  const SortSeg& g = b.seg[kMulti ? blockIdx.y : 0];
+  if (int64_t(blockIdx.x) >= g.tiles) return;
   extern __shared__ int32_t sh_cnt[];
-  const int digits = 1 << bits, mask = digits - 1;
+  const int digits = 1 << b.bits, mask = digits - 1, shift = b.shift;
   for (int i = threadIdx.x; i < digits; i += blockDim.x) sh_cnt[i] = 0;
   __syncthreads();
   const int64_t base = int64_t(blockIdx.x) * kSortTile;
@@ -43,14 +44,14 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_hist(const int32_t* __res
 #pragma unroll
   for (int u = 0; u < kSortTile / kSortThreads; ++u) {
     const int64_t p = base + u * kSortThreads + threadIdx.x;
-    kv[u] = p < M ? elem_key(keys, in_ids, p, in_order) : -1;
+    kv[u] = p < g.M ? elem_key(g.keys, g.in_ids, p, b.in_order) : -1;
   }
 #pragma unroll
   for (int u = 0; u < kSortTile / kSortThreads; ++u)
     if (kv[u] >= 0) atomicAdd(&sh_cnt[(kv[u] >> shift) & mask], 1);
   __syncthreads();
   for (int i = threadIdx.x; i < digits; i += blockDim.x)
-    hist[int64_t(i) * tiles + blockIdx.x] = sh_cnt[i];
+    g.hist[int64_t(i) * g.tiles + blockIdx.x] = sh_cnt[i];
 }
 
 // Exclusive block scan of one value per thread; returns the exclusive prefix and
@@ -82,40 +83,44 @@ __device__ int32_t block_exclusive_scan(int32_t v, int32_t* sh_warp, int32_t* to
   return r;
 }
 
-// grid = digits; row d of hist becomes its exclusive prefix over tiles; total -> out[d].
-__global__ void __launch_bounds__(256) k_sort_scan_tiles(int32_t* __restrict__ hist,
-                                                         int64_t tiles,
-                                                         int32_t* __restrict__ out) {
+// grid = (digits, segments); row d of hist becomes its exclusive prefix over tiles; the
+// total goes to start[d].
+template <bool kMulti>
+__global__ void __launch_bounds__(256) k_sort_scan_tiles(const __grid_constant__ SortBatch b) {
+  const SortSeg& g = b.seg[kMulti ? blockIdx.y : 0];
   __shared__ int32_t sh_warp[32];
   __shared__ int32_t sh_total;
-  int32_t* row = hist + int64_t(blockIdx.x) * tiles;
+  int32_t* row = g.hist + int64_t(blockIdx.x) * g.tiles;
   int32_t carry = 0;
-  for (int64_t c0 = 0; c0 < tiles; c0 += blockDim.x) {
+  for (int64_t c0 = 0; c0 < g.tiles; c0 += blockDim.x) {
     const int64_t i = c0 + threadIdx.x;
-    const int32_t v = i < tiles ? row[i] : 0;
+    const int32_t v = i < g.tiles ? row[i] : 0;
     const int32_t ex = block_exclusive_scan(v, sh_warp, &sh_total);
-    if (i < tiles) row[i] = carry + ex;
+    if (i < g.tiles) row[i] = carry + ex;
     carry += sh_total;
     __syncthreads();
   }
-  if (threadIdx.x == 0) out[blockIdx.x] = carry;
+  if (threadIdx.x == 0) g.start[blockIdx.x] = carry;
 }
 
-// One block: start[0..digits) = exclusive prefix of the totals held there; start[digits] = M.
-__global__ void __launch_bounds__(1024) k_sort_scan_digits(int32_t* __restrict__ start,
-                                                           int digits) {
+// One block per segment: start[0..digits) = exclusive prefix of the totals held there;
+// start[digits] = M.
+template <bool kMulti>
+__global__ void __launch_bounds__(1024) k_sort_scan_digits(const __grid_constant__ SortBatch b) {
+  const SortSeg& g = b.seg[kMulti ? blockIdx.y : 0];
+  const int digits = 1 << b.bits;
   __shared__ int32_t sh_warp[32];
   __shared__ int32_t sh_total;
   int32_t carry = 0;
   for (int c0 = 0; c0 < digits; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
-    const int32_t v = i < digits ? start[i] : 0;
+    const int32_t v = i < digits ? g.start[i] : 0;
     const int32_t ex = block_exclusive_scan(v, sh_warp, &sh_total);
-    if (i < digits) start[i] = carry + ex;
+    if (i < digits) g.start[i] = carry + ex;
     carry += sh_total;
     __syncthreads();
   }
-  if (threadIdx.x == 0) start[digits] = carry;
+  if (threadIdx.x == 0) g.start[digits] = carry;
 }
 
 // Shared memory of the scatter: per-warp digit counts, per-digit offsets, and the tile
@@ -126,14 +131,23 @@ __host__ __device__ constexpr size_t scatter_smem_bytes(int bits) {
          + size_t(kSortTile) * 12;                                        // staged tile
 }
 
-__global__ void __launch_bounds__(kSortThreads, 4) k_sort_scatter(
-    const int32_t* __restrict__ keys, const int32_t* __restrict__ in_ids, int64_t M, int shift,
-    int bits, const int32_t* __restrict__ hist, int64_t tiles,
-    const int32_t* __restrict__ digit_start, int32_t* __restrict__ out_ids,
-    int32_t* __restrict__ out_keys, const float* __restrict__ payload,
-    float* __restrict__ out_payload, bool in_order) {
+template <bool kMulti>
+__global__ void __launch_bounds__(kSortThreads, 4) k_sort_scatter(const __grid_constant__ SortBatch b) {
+  const SortSeg& g = b.seg[kMulti ? blockIdx.y : 0];
+  if (int64_t(blockIdx.x) >= g.tiles) return;
+  const int32_t* __restrict__ keys = g.keys;
+  const int32_t* __restrict__ in_ids = g.in_ids;
+  const int64_t M = g.M, tiles = g.tiles;
+  const int shift = b.shift;
+  const bool in_order = b.in_order;
+  const int32_t* __restrict__ hist = g.hist;
+  const int32_t* __restrict__ digit_start = g.start;
+  int32_t* __restrict__ out_ids = g.out_ids;
+  int32_t* __restrict__ out_keys = g.out_keys;
+  const float* __restrict__ payload = g.payload;
+  float* __restrict__ out_payload = g.out_payload;
   extern __shared__ __align__(16) unsigned char sh_raw[];
-  const int digits = 1 << bits, mask = digits - 1;
+  const int digits = 1 << b.bits, mask = digits - 1;
   uint16_t* cnt = reinterpret_cast<uint16_t*>(sh_raw);  // [kWarps][digits]
   int32_t* gbase = reinterpret_cast<int32_t*>(sh_raw + ((kWarps * digits * 2 + 15) & ~15));
   int32_t* lbase = gbase + digits;   // first staged position of each digit in this tile
@@ -254,37 +268,72 @@ cudaError_t launch_segment_starts(const int32_t* sorted, int64_t M, int32_t n_va
   return cudaGetLastError();
 }
 
+// The single-segment kernels index the segment statically (its fields stay kernel
+// parameters); the batch kernels pick it by blockIdx.y.
+template <bool kMulti>
+cudaError_t run_sort_batch(const SortBatch& b, int64_t max_tiles, int digits, cudaStream_t st) {
+  const unsigned n = unsigned(b.n);
+  // segments with no element still get their starts (all zero) from the scans
+  if (max_tiles > 0)
+    k_sort_hist<kMulti><<<dim3(unsigned(max_tiles), n), kSortThreads, sizeof(int32_t) * digits,
+                          st>>>(b);
+  k_sort_scan_tiles<kMulti><<<dim3(digits, n), 256, 0, st>>>(b);
+  k_sort_scan_digits<kMulti><<<dim3(1, n), 1024, 0, st>>>(b);
+  count_launches(2);
+  if (max_tiles > 0) {
+    // Opt in to the largest dynamic shared memory the scatter can use (per device; cheap).
+    cudaError_t e = cudaFuncSetAttribute(k_sort_scatter<kMulti>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(scatter_smem_bytes(kMaxDigitBits)));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_sort_scatter<kMulti>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    k_sort_scatter<kMulti><<<dim3(unsigned(max_tiles), n), kSortThreads,
+                             scatter_smem_bytes(b.bits), st>>>(b);
+    count_launches(2);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sort_batch(const SortSeg* segs, int n, int shift, int bits, bool in_order,
+                              cudaStream_t st) {
+  if (n < 1 || n > kMaxSortSegs) return cudaErrorInvalidValue;
+  SortBatch b{};
+  int64_t max_tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    b.seg[i] = segs[i];
+    b.seg[i].tiles = ceil_div(segs[i].M, kSortTile);
+    if (b.seg[i].tiles > max_tiles) max_tiles = b.seg[i].tiles;
+  }
+  b.n = n;
+  b.shift = shift;
+  b.bits = bits;
+  b.in_order = in_order;
+  const int digits = 1 << bits;
+  return n > 1 ? run_sort_batch<true>(b, max_tiles, digits, st)
+               : run_sort_batch<false>(b, max_tiles, digits, st);
+}
+
 cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,
                              int bits, void* scratch, int32_t* out_ids, int32_t* out_keys,
                              int32_t* digit_start, cudaStream_t st, const float* payload,
                              float* out_payload, bool in_order) {
   const int digits = 1 << bits;
   const int64_t tiles = ceil_div(M > 0 ? M : 1, kSortTile);
-  int32_t* hist = static_cast<int32_t*>(scratch);
-  int32_t* start = digit_start
-                       ? digit_start
-                       : reinterpret_cast<int32_t*>(static_cast<char*>(scratch) +
-                                                    align256(sizeof(int32_t) * size_t(digits * tiles)));
-  if (M == 0) {
-    if (digit_start) return cudaMemsetAsync(digit_start, 0, sizeof(int32_t) * (digits + 1), st);
-    return cudaSuccess;
-  }
-  k_sort_hist<<<unsigned(tiles), kSortThreads, sizeof(int32_t) * digits, st>>>(
-      keys, in_ids, M, shift, bits, hist, tiles, in_order);
-  k_sort_scan_tiles<<<digits, 256, 0, st>>>(hist, tiles, start);
-  k_sort_scan_digits<<<1, 1024, 0, st>>>(start, digits);
-  // Opt in to the largest dynamic shared memory the scatter can use (per device; cheap).
-  const size_t smem = scatter_smem_bytes(bits);
-  cudaError_t e = cudaFuncSetAttribute(k_sort_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(scatter_smem_bytes(kMaxDigitBits)));
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_sort_scatter, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  if (e != cudaSuccess) return e;
-  k_sort_scatter<<<unsigned(tiles), kSortThreads, smem, st>>>(
-      keys, in_ids, M, shift, bits, hist, tiles, start, out_ids, out_keys, payload, out_payload,
-      in_order);
-  count_launches(4);
-  return cudaGetLastError();
+  SortSeg g{};
+  g.keys = keys;
+  g.in_ids = in_ids;
+  g.M = M;
+  g.hist = static_cast<int32_t*>(scratch);
+  g.start = digit_start ? digit_start
+                        : reinterpret_cast<int32_t*>(static_cast<char*>(scratch) +
+                                                     align256(sizeof(int32_t) * size_t(digits * tiles)));
+  g.out_ids = out_ids;
+  g.out_keys = out_keys;
+  g.payload = payload;
+  g.out_payload = out_payload;
+  return launch_sort_batch(&g, 1, shift, bits, in_order, st);
 }
 
 }  // namespace rece
