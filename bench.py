@@ -229,8 +229,8 @@ def oracle_sample_desc(rows, bucket_frac):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    rank, _, _ = dist_env()
+    if rank != 0:  # the oracle arm runs on rank 0 alone; other ranks exit without work
         return
     import oracle
     from reduced_cross_entropy_b200 import synth
@@ -256,6 +256,33 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    """(rank, local_rank, world) from the launcher's environment (torchrun sets them)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def max_over_ranks(x, device=None):
+    """The largest x over the ranks of the default process group (x itself with no group).
+    Every rank must call it, in the same order.  device: where the reduction tensor
+    lives (the rank's GPU under NCCL, the CPU under gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, rows_per_step, steps, total_ms):
+    """Whole-job rows/s: every rank processes rows_per_step rows per step (weak scaling),
+    timed by the slowest rank's total_ms over `steps` steps."""
+    return world * rows_per_step * steps / (total_ms / 1000.0)
+
+
 # ------------------------------------------------------------------ GPU arm
 def main():
     args = parse()
@@ -267,9 +294,7 @@ def main():
 
     from reduced_cross_entropy_b200 import _lib, ops, synth
 
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank, local_rank, world = dist_env()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
@@ -349,15 +374,11 @@ def main():
     launches = L.rece_kernel_launch_count() - launches0
     L.rece_plan_set_stage_events(plan._h, None)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     stage_ms = {name: statistics.mean(sev[s][2 * i].elapsed_time(sev[s][2 * i + 1])
                                       for s in range(args.steps))
                 for i, name in enumerate(_lib.STAGES)}
-    value = world * w.N * args.steps / (total_ms / 1000.0)
+    value = job_throughput(world, w.N, args.steps, total_ms)
 
     # roofline of every stage, the dominant one reported as the line's roofline
     peaks = load_peaks()
@@ -410,12 +431,8 @@ def main():
         b.synchronize()
         if s >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        tt = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_total = float(tt.item())
-    e2e = {"value": world * w.N * args.steps / (e2e_total / 1000.0), "unit": "rows/s",
+    e2e_total = max_over_ranks(sum(e2e_ms), dev)
+    e2e = {"value": job_throughput(world, w.N, args.steps, e2e_total), "unit": "rows/s",
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4}
 
     line = {"metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
