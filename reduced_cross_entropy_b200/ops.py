@@ -60,8 +60,9 @@ class Plan:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value and _lib._lib is not None:
-            _lib._lib.rece_plan_destroy(h)
+        lib = getattr(_lib, "_lib", None) if _lib is not None else None  # None at exit
+        if h is not None and h.value and lib is not None:
+            lib.rece_plan_destroy(h)
             self._h = None
 
     @property
