@@ -345,7 +345,11 @@ def main():
         flush.zero_()
         step(Bs[s])
     torch.cuda.synchronize(dev)
-    assert ops.device_status(ws) == 0
+    # status area: flags (a bad target or a timed-out wait fails the run; the tensor-core
+    # selection may flag rows it cannot certify exact) and the count of such rows
+    status_words = ws[:16].view(torch.int32).cpu().tolist()
+    assert status_words[0] & ~_lib.DEVICE_INEXACT == 0, f"device status {status_words[0]:#x}"
+    inexact_rows, overflow_rows = int(status_words[1]), int(status_words[2])
 
     # timed region: K steps, each bracketed by events; per-stage events recorded by the
     # library on the same stream
@@ -439,7 +443,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": workload_desc(w),
+            "config": {"workload": workload_desc(w), "inexact_rows_per_step": inexact_rows,
+                       "overflowed_rows_per_step": overflow_rows,
                        "l2": "flushed between timed steps (256 MiB write)",
                        "scores": "tcgen05" if uses_tensor_cores(w, args.flags)
                        else "fmaf CUDA cores"},

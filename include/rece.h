@@ -78,7 +78,8 @@ typedef enum {
 #define RECE_DEVICE_INEXACT 0x4u    /* bf16 tensor-core mode: some rows' top-k could not be
                                        certified exact (a candidate list overflowed or a
                                        threshold was above the k-th kept score); the 32-bit
-                                       word after the status word counts those rows */
+                                       word after the status word counts those rows, the
+                                       next one those whose candidate list overflowed */
 
 typedef struct {
   int64_t N;     /* rows (batch x sequence), >= 0 */

@@ -18,6 +18,7 @@ MODE_BF16 = 1
 FLAG_FMA_SCORES = 0x1
 DEVICE_BAD_TARGET = 0x1
 DEVICE_TIMEOUT = 0x2
+DEVICE_INEXACT = 0x4
 
 # every symbol include/rece.h declares
 EXPORTS = (

@@ -12,8 +12,11 @@
 // Pair e = i*(k+1) + s holds slot s of row i (s = 0: the positive, s >= 1: selected
 // negative s-1); an empty slot carries the key C, which sorts after every item.  Every
 // sum has a fixed order: the gradients are deterministic.
+#include <type_traits>
+
 #include "common.cuh"
 #include "plan.h"
+#include "tc.h"
 
 namespace rece {
 namespace {
@@ -87,6 +90,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
   __syncwarp();
 
   // dX_i: lanes over dimensions (two each), slots in order
+  if (!dX) return;  // dX comes from the tensor cores
   if ((d & 1) == 0) {
     for (int t0 = 0; t0 < d; t0 += 64) {
       const int t = t0 + 2 * lane;
@@ -265,8 +269,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
   }
   __syncwarp();
 
-  // dX_i: quarter q adds the slots s = q (mod 4) in order over its lane's 8 dims
-  for (int t0 = 0; t0 < d; t0 += 64) {
+  // dX_i: quarter q adds the slots s = q (mod 4) in order over its lane's 8 dims (not
+  // here when dX comes from the tensor cores)
+  for (int t0 = 0; t0 < (dX ? d : 0); t0 += 64) {
     const int t = t0 + 8 * sub;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (t < d) {
@@ -354,11 +359,66 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
 
 size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 * (k + 1)); }
 
+// LSD radix sort of E (item key, g) pairs by key (values 0..C), as few passes as the
+// counting sort's 12-bit digit limit allows.  Every pass writes keys and g in its output
+// order, so the next pass reads them contiguously; *sorted_id (perm_a or perm_b) says
+// where each sorted pair came from.  The last pass lands in sorted_key / sorted_g.
+cudaError_t sort_pairs_by_item(const rece_plan_s& p, int64_t E, const int32_t* key,
+                               const float* g, int32_t* perm_a, int32_t* perm_b, int32_t* key_b,
+                               float* g_b, int32_t* sorted_key, float* sorted_g, void* scratch,
+                               const int32_t** sorted_id, cudaStream_t st) {
+  int32_t* key_buf[2] = {key_b, sorted_key};
+  float* g_buf[2] = {g_b, sorted_g};
+  const int passes = p.item_passes;
+  const int32_t* in = nullptr;
+  const int32_t* kin = key;
+  const float* gin = g;
+  int32_t* out = perm_a;
+  int shift = 0;
+  for (int ps = 0; ps < passes; ++ps) {
+    const int bits = (ps + 1 < passes) ? p.item_pass_bits : p.item_bits - shift;
+    const int slot = (passes - 1 - ps) % 2 == 0 ? 1 : 0;
+    cudaError_t e = launch_sort_pass(kin, in, E, shift, bits, scratch, out, key_buf[slot],
+                                     nullptr, st, gin, g_buf[slot], ps > 0);
+    if (e != cudaSuccess) return e;
+    shift += bits;
+    in = out;
+    kin = key_buf[slot];
+    gin = g_buf[slot];
+    out = (out == perm_a) ? perm_b : perm_a;
+  }
+  *sorted_id = in;
+  return cudaSuccess;
+}
+
+// dY_j = sum of g x_row over the pairs of item j (sorted by item; pair id / slots = row),
+// written for every item (0 where it has no pair).
+template <typename T>
+cudaError_t launch_items_from_pairs(const T* X, int64_t C, int d, int slots,
+                                    const int32_t* item_start, const int32_t* sorted_id,
+                                    const float* sorted_g, float* dY, cudaStream_t st) {
+  const int warps = kThreads / 32;
+  if (d % 8 == 0)
+    k_bwd_items_v8<T><<<unsigned(ceil_div(C, warps)), kThreads, 0, st>>>(
+        X, C, d, slots - 1, item_start, sorted_id, sorted_g, dY);
+  else
+    k_bwd_items<T><<<unsigned(ceil_div(C, warps)), kThreads, 0, st>>>(
+        X, C, d, slots - 1, item_start, sorted_id, sorted_g, dY);
+  count_launches(1);
+  return cudaGetLastError();
+}
+template cudaError_t launch_items_from_pairs<__nv_bfloat16>(const __nv_bfloat16*, int64_t, int,
+                                                            int, const int32_t*, const int32_t*,
+                                                            const float*, float*, cudaStream_t);
+
 template <typename T>
 cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
                             const int32_t* targets, const int32_t* selected, const float* lse,
                             const float* logits, const float* dloss, char* ws, float* dX,
                             float* dY, uint32_t* status, cudaStream_t st) {
+  // with dX on the tensor cores the rows kernel only lays out the (item, g) pairs
+  bool dx_tc = false;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) dx_tc = p.tc_dx;
   const auto& c = p.cfg;
   const Layout& L = p.lay;
   const int64_t E = p.entries;
@@ -379,43 +439,34 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
     cudaError_t e = cudaFuncSetAttribute(v8 ? k_bwd_rows_v8<T> : k_bwd_rows<T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
+    float* dx_rows = dx_tc ? nullptr : dX;
     if (v8)
       k_bwd_rows_v8<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
-          X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX,
+          X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dx_rows,
           status);
     else
       k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
-          X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dX,
+          X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dx_rows,
           status);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      if (dx_tc) {
+        e = launch_dx_tc(p, Y, targets, lse, dloss, ws, dX, status, st);
+        if (e != cudaSuccess) return e;
+      }
+    }
   }
   stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
-  // LSD radix sort of the pairs by item key (values 0..C), as few passes as the
-  // counting sort's 12-bit digit limit allows.  Every pass writes keys and g in its output
-  // order, so the next pass reads them contiguously; the ids say where each pair came from.
-  int32_t* key_buf[2] = {reinterpret_cast<int32_t*>(ws + L.e_key_b), sorted_key};
-  float* g_buf[2] = {reinterpret_cast<float*>(ws + L.e_g_b), sorted_g};
-  const int passes = p.item_passes;
   const int32_t* in = nullptr;
-  const int32_t* kin = e_key;
-  const float* gin = e_g;
-  int32_t* out = perm_a;
-  int shift = 0;
-  for (int ps = 0; ps < passes; ++ps) {
-    const int bits = (ps + 1 < passes) ? p.item_pass_bits : p.item_bits - shift;
-    // the last pass lands in sorted_key / sorted_g
-    const int slot = (passes - 1 - ps) % 2 == 0 ? 1 : 0;
-    cudaError_t e = launch_sort_pass(kin, in, E, shift, bits, scratch, out, key_buf[slot],
-                                     nullptr, st, gin, g_buf[slot], ps > 0);
+  {
+    cudaError_t e = sort_pairs_by_item(p, E, e_key, e_g, perm_a, perm_b,
+                                       reinterpret_cast<int32_t*>(ws + L.e_key_b),
+                                       reinterpret_cast<float*>(ws + L.e_g_b), sorted_key,
+                                       sorted_g, scratch, &in, st);
     if (e != cudaSuccess) return e;
-    shift += bits;
-    in = out;
-    kin = key_buf[slot];
-    gin = g_buf[slot];
-    out = (out == perm_a) ? perm_b : perm_a;
   }
   int32_t* item_start = reinterpret_cast<int32_t*>(ws + L.e_item_start);
   cudaError_t e2 = launch_segment_starts(sorted_key, E, int32_t(c.C), item_start, st);

@@ -1,0 +1,410 @@
+// bwd_tc.cu -- dX of step 6 on the tcgen05 tensor cores (bf16 mode): the row gradients of
+// the reduced loss (RECE, equation 4, over the positive and the kept negatives, selection
+// held constant) as dense block products of the sparse coefficient matrix.
+//
+//   g_ij = (exp(l_ij - lse_i) - [j == z_i]) * dloss / N,   dX_i = sum_j g_ij y_j
+//
+// The negatives of round r of a row all lie in that row's window of round r's sorted
+// catalogue, so per round the coefficients form a band: rows of chunk c against the
+// sorted positions of chunks c-n_ec..c+n_ec.  With G_r that band (sorted rows x sorted
+// positions, the round's kept entries only -- the merge kept each pair once, in the
+// earliest round whose window holds it):
+//
+//   dX[rows] += G_r[rows, window] Ys_r[window]     (work item: 128 sorted rows)
+//
+// A work item streams its window in slabs of 64 positions: four builder warps write the
+// slab's 128 x 64 tile of G into shared memory in the 128-byte-swizzled K-major layout
+// (zeros, then the row's entries of the slab, which come grouped by slab) while TMA brings
+// the matching 64-position slab of the d-major sorted copy YsT and one thread issues
+// tcgen05.mma into a TMEM accumulator of 128 x NS fp32 (NS <= 256 columns of d per CTA).
+// The tiles hold the negatives' softmax probabilities p_ij = exp(l_ij - lse_i), which the
+// merge stored split as hi + lo, both bf16 (hi = bf16(p), lo = bf16(p - hi)); both halves
+// are multiplied, so about 16 bits of p survive against 8 for a plain bf16 tile, and the
+// epilogue applies the factor dloss / N.
+//
+// This pays where gathering the catalogue rows does not: at large d, or when the sorted
+// catalogue does not fit in L2.  (The transposed product for dY, G_r^T Xs_r per tile of
+// positions, was measured slower than the pair sort and gather on every shape tried: its
+// K ranges are short and every slice of d rebuilt the same tiles.)
+//
+// Determinism: each dX row is written by one CTA per launch, in a fixed K order; the
+// positive term is written first (dX_i = g_iz y_z), then the rounds add in round order.
+#include "common.cuh"
+#include "plan.h"
+#include "sm100.cuh"
+#include "tc.h"
+
+#define RECE_TRY(x)                          \
+  do {                                       \
+    const cudaError_t err_ = (x);            \
+    if (err_ != cudaSuccess) return err_;    \
+  } while (0)
+
+namespace rece {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;           // rows of G (dX) or of G^T (dY) per work item
+constexpr int kBK = 64;            // K per slab
+constexpr int kAStages = 2;        // G tiles being built / consumed
+constexpr int kMaxBStages = 8;     // TMA slabs in flight
+constexpr int kBuilders = 128;     // warps 0-3: builders, then the epilogue
+constexpr int kThreads = kBuilders + 64;  // warp 4: TMA producer, warp 5: MMA issuer
+constexpr uint32_t kATile = kBM * kBK * 2;  // one bf16 G tile (16 KB)
+constexpr uint64_t kTimeoutNs = 1000000000ull;
+
+struct Ctl {
+  uint64_t bfull[kMaxBStages], bempty[kMaxBStages];
+  uint64_t afull[kAStages], aempty[kAStages];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Dynamic shared memory: A_hi[kAStages], A_lo[kAStages], B[nb] (NS x 128 B each), Ctl.
+__host__ __device__ constexpr size_t smem_bytes(int nb, int ns) {
+  return 1024 + size_t(2 * kAStages) * kATile + size_t(nb) * ns * 128 + sizeof(Ctl);
+}
+
+// Byte offset of element (row, col) of a 128 x 64 bf16 tile in the 128-byte-swizzled
+// K-major layout (what a TMA box {64, rows} with SWIZZLE_128B writes): rows of 128 B in
+// 8-row atoms of 1024 B, the 16-byte chunk index xor-ed with row % 8.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
+  return uint32_t((row >> 3) * 1024 + (row & 7) * 128 + ((((col >> 3) ^ row) & 7) << 4) +
+                  (col & 7) * 2);
+}
+
+// Zeros one 128-byte row; the chunk order is rotated by the row so that the lanes of a
+// warp (32 consecutive rows, 128 B apart) spread over all banks.
+__device__ __forceinline__ void zero_row(uint8_t* tile, int row) {
+  uint4* p = reinterpret_cast<uint4*>(tile + (row >> 3) * 1024 + (row & 7) * 128);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) p[(j + row) & 7] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Writes one coefficient, given as two bf16 halves (hi | lo << 16), into the hi and lo
+// tiles at (row, col).
+__device__ __forceinline__ void put(uint8_t* hi_tile, uint8_t* lo_tile, int row, int col,
+                                    uint32_t packed) {
+  const uint32_t o = sw128_offset(row, col);
+  *reinterpret_cast<uint16_t*>(hi_tile + o) = uint16_t(packed & 0xFFFFu);
+  *reinterpret_cast<uint16_t*>(lo_tile + o) = uint16_t(packed >> 16);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ int64_t chunk_of(int64_t p, int64_t M, int n_c) {
+  return (p * n_c) / M;
+}
+
+// Window [w0, w1) of sorted row p (round's sorted order), in sorted catalogue positions.
+__device__ __forceinline__ void row_window(int64_t p, int64_t N, int64_t C, int n_c, int n_ec,
+                                           int64_t& w0, int64_t& w1) {
+  const int64_t c = chunk_of(p, N, n_c);
+  w0 = chunk_start(c - n_ec < 0 ? 0 : c - n_ec, C, n_c);
+  w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
+}
+
+struct Args {
+  int64_t N, C;
+  int d, k, n_c, n_ec, r, ns, nb, Sp;
+  const int32_t* px;        // [n_r][N] sorted row -> row
+  const int2* kept;         // [n_r][N][k] (sorted position, p as bf16 hi | lo << 16)
+  const int32_t* kept_off;  // [n_r][N][Sp] slice starts within the round's entries
+  const float* dloss;       // [1]
+  float* out;               // dX [N][d], accumulated into
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void on_timeout(Ctl& c, uint32_t* status) {
+  *reinterpret_cast<volatile int*>(&c.abort) = 1;
+  raise_flag(status, RECE_DEVICE_TIMEOUT);
+}
+
+// One work item per CTA: 128 sorted rows of round r (K = the union of their windows);
+// blockIdx.y picks the NS-wide slice of d.
+__global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant__ CUtensorMap tmB,
+                                                        const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* A_hi = base;
+  uint8_t* A_lo = base + kAStages * kATile;
+  uint8_t* Bs = base + 2 * kAStages * kATile;
+  const uint32_t b_bytes = uint32_t(a.ns) * 128u;
+  Ctl& ctl = *reinterpret_cast<Ctl*>(Bs + size_t(a.nb) * b_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  const int nb = a.nb;
+  const int64_t N = a.N, C = a.C;
+  const int r = a.r, n0 = blockIdx.y * a.ns;
+
+  // the item's rows and its K range [lo, hi) in slabs of 64
+  const int64_t m0 = int64_t(blockIdx.x) * kBM;
+  int64_t lo = 0, hi = 0;
+  {
+    const int64_t last = (m0 + kBM - 1 < N - 1) ? m0 + kBM - 1 : N - 1;
+    const int64_t cf = chunk_of(m0, N, a.n_c), cl = chunk_of(last, N, a.n_c);
+    const int64_t k0 = chunk_start(cf - a.n_ec < 0 ? 0 : cf - a.n_ec, C, a.n_c);
+    const int64_t k1 = chunk_start(cl + a.n_ec + 1 > a.n_c ? a.n_c : cl + a.n_ec + 1, C, a.n_c);
+    if (k1 > k0) {
+      lo = k0 >> 6;
+      hi = (k1 + 63) >> 6;
+    }
+  }
+  const int nK = int(hi - lo);
+
+  if (t == 0) {
+    for (int i = 0; i < nb; ++i) {
+      mbar_init(&ctl.bfull[i], 1);
+      mbar_init(&ctl.bempty[i], 1);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&ctl.afull[i], kBuilders / 32);  // one arrival per builder warp
+      mbar_init(&ctl.aempty[i], 1);
+    }
+    mbar_init(&ctl.done, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  const uint32_t tcols = a.ns <= 32 ? 32u : (a.ns <= 64 ? 64u : (a.ns <= 128 ? 128u : 256u));
+  if (warp == 4) {
+    tmem_alloc(&ctl.tmem_base, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmB);
+      int s = 0;
+      for (; s < nK; ++s) {
+        const int slot = s % nb;
+        if (!mbar_wait(&ctl.bempty[slot], ((s / nb) & 1) ^ 1, &ctl.abort, kTimeoutNs)) {
+          on_timeout(ctl, a.status);
+          break;
+        }
+        mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
+        tma_load_2d(Bs + size_t(slot) * b_bytes, &tmB, &ctl.bfull[slot], int((lo + s) * kBK),
+                    r * a.d + n0);
+      }
+      for (int j = (s > nb ? s - nb : 0); j < s; ++j)  // every issued copy has landed
+        mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1, kTimeoutNs);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, a.ns);
+      for (int s = 0; s < nK; ++s) {
+        const int as = s % kAStages, bs = s % nb;
+        if (!mbar_wait(&ctl.afull[as], (s / kAStages) & 1, &ctl.abort, kTimeoutNs) ||
+            !mbar_wait(&ctl.bfull[bs], (s / nb) & 1, &ctl.abort, kTimeoutNs)) {
+          on_timeout(ctl, a.status);
+          break;
+        }
+        tc_fence_after();
+        const uint64_t dh = desc_k_sw128(smem_u32(A_hi + as * kATile));
+        const uint64_t dl = desc_k_sw128(smem_u32(A_lo + as * kATile));
+        const uint64_t db = desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes));
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          mma_bf16(tmem, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
+          mma_bf16(tmem, dl + 2 * kk, db + 2 * kk, idesc, 1);
+        }
+        mma_commit(&ctl.aempty[as]);
+        mma_commit(&ctl.bempty[bs]);
+      }
+      mma_commit(&ctl.done);
+      mbar_wait_limit(&ctl.done, 0, kTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------------------ builders
+    const int64_t rN = int64_t(r) * N;
+    constexpr int2 kNone = {0x7FFFFFFF, 0};  // past the last entry: beyond every slab
+    // This thread's sorted row p = m0 + t.  Its round-r entries are grouped by slice in
+    // ascending order, so the slabs consume them front to back, through a window of two
+    // batches of 8 held in registers: cur = entries [base, base+8), nxt the 8 after, whose
+    // loads are issued a batch ahead of their use.
+    const int64_t p = m0 + t;
+    const bool prow_ok = p < N;
+    const int2* erow = a.kept + (rN + (prow_ok ? p : 0)) * a.k;
+    int count = 0, e = 0, base = 0;
+    int2 cur[8], nxt[8];
+    if (prow_ok) {
+      int64_t w0, w1;
+      row_window(p, N, C, a.n_c, a.n_ec, w0, w1);
+      const int S = w1 > w0 ? int((w1 - 1) >> 6) - int(w0 >> 6) + 1 : 0;
+      count = __ldg(a.kept_off + (rN + p) * a.Sp + S);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cur[u] = u < count ? __ldg(erow + u) : kNone;
+      nxt[u] = 8 + u < count ? __ldg(erow + 8 + u) : kNone;
+    }
+
+    for (int s = 0; s < nK; ++s) {
+      const int as = s % kAStages;
+      const bool waited = mbar_wait(&ctl.aempty[as], ((s / kAStages) & 1) ^ 1, &ctl.abort,
+                                    kTimeoutNs);
+      if (!waited) {  // each thread writes its own row only: no barrier to keep in step
+        on_timeout(ctl, a.status);
+        break;
+      }
+      uint8_t* th = A_hi + as * kATile;
+      uint8_t* tl = A_lo + as * kATile;
+      zero_row(th, t);
+      zero_row(tl, t);
+      const int64_t sig = lo + s;  // absolute slab
+      const int slab_end = int((sig + 1) * kBK);
+      while (e < count) {
+        int used = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (base + u >= e && cur[u].x < slab_end) {
+            const int col = cur[u].x - int(sig * kBK);
+            if (col >= 0 && col < kBK) put(th, tl, t, col, uint32_t(cur[u].y));  // (always)
+            ++used;
+          }
+        }
+        e += used;
+        if (e < base + 8) break;  // the next entry belongs to a later slab
+        // the batch is used up: the next one moves in, the one after is requested
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
+        base += 8;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          nxt[u] = base + 8 + u < count ? __ldg(erow + base + 8 + u) : kNone;
+      }
+      fence_proxy_async_smem();  // this thread's tile writes, visible to the MMA
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.afull[as]);
+    }
+    __syncwarp();
+
+    // ------------------------------------------------------------ epilogue
+    const bool ok = mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && nK > 0;
+    const float scale = a.dloss[0] / float(N);  // G holds p; g = p * dloss / N
+    tc_fence_after();
+    const int64_t row = m0 + t;  // this thread's sorted row
+    const bool live = row < N;
+    const int64_t dst = live ? a.px[rN + row] : 0;
+    float* o = a.out + dst * a.d + n0;
+    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+    for (int c0 = 0; c0 < a.ns; c0 += 32) {
+      float v[32];
+      tmem_load32(taddr + uint32_t(c0), v);
+      if (ok && live) {
+        float4* q = reinterpret_cast<float4*>(o + c0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float4 x = q[u];
+          x.x = fmaf(scale, v[4 * u], x.x);
+          x.y = fmaf(scale, v[4 * u + 1], x.y);
+          x.z = fmaf(scale, v[4 * u + 2], x.z);
+          x.w = fmaf(scale, v[4 * u + 3], x.w);
+          q[u] = x;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
+  }
+}
+
+// One warp per row: the positive's coefficient g_iz and dX_i = g_iz y_z (written, not
+// added: the rounds add after it).
+template <typename T>
+__global__ void __launch_bounds__(256) k_bwd_pos(const T* __restrict__ Y,
+                                                 const int32_t* __restrict__ targets,
+                                                 const float* __restrict__ lse,
+                                                 const float* __restrict__ pos_logit,
+                                                 const float* __restrict__ dloss, int64_t N,
+                                                 int64_t C, int d, float* __restrict__ dX) {
+  const int lane = threadIdx.x & 31;
+  const int64_t i = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= N) return;
+  const int32_t z = targets[i];
+  const bool z_ok = z >= 0 && z < C;
+  float g = 0.0f;
+  if (z_ok) g = (expf(pos_logit[i] - lse[i]) - 1.0f) * (dloss[0] / float(N));
+  const T* y = Y + (z_ok ? int64_t(z) : 0) * d;
+  for (int t = 8 * lane; t < d; t += 256) {
+    float v[8];
+    load8(y + t, v);
+    float4* o = reinterpret_cast<float4*>(dX + i * d + t);
+    o[0] = make_float4(g * v[0], g * v[1], g * v[2], g * v[3]);
+    o[1] = make_float4(g * v[4], g * v[5], g * v[6], g * v[7]);
+  }
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* targets,
+                         const float* lse, const float* dloss, char* ws, float* dX,
+                         uint32_t* status, cudaStream_t st) {
+  const auto& c = p.cfg;
+  const Layout& L = p.lay;
+  if (c.N == 0) return cudaSuccess;
+  // d is split into CTA slices of ns <= 256 columns (one TMEM accumulator each)
+  int ns = c.d;
+  if (ns > 256) ns = (c.d % 256 == 0) ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64));
+  const int slices = c.d / ns;
+  // TMA ring: as deep as lets two CTAs share an SM (at least two slabs)
+  int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(ns) * 128));
+  nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
+  const size_t smem = smem_bytes(nb, ns);
+
+  Args a{};
+  a.N = c.N;
+  a.C = c.C;
+  a.d = c.d;
+  a.k = c.k;
+  a.n_c = c.n_c;
+  a.n_ec = c.n_ec;
+  a.ns = ns;
+  a.nb = nb;
+  a.Sp = p.kept_slices + 1;
+  a.px = reinterpret_cast<const int32_t*>(ws + L.px);
+  a.kept = reinterpret_cast<const int2*>(ws + L.kept);
+  a.kept_off = reinterpret_cast<const int32_t*>(ws + L.kept_off);
+  a.dloss = dloss;
+  a.status = status;
+  a.out = dX;
+
+  k_bwd_pos<T><<<unsigned(ceil_div(c.N, 8)), 256, 0, st>>>(
+      Y, targets, lse, reinterpret_cast<const float*>(ws + L.pos_logit), dloss, c.N, c.C, c.d,
+      dX);
+  count_launches(1);
+  RECE_TRY(cudaGetLastError());
+  RECE_TRY(cudaFuncSetAttribute(k_bwd_dx_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(smem)));
+  CUtensorMap tm;
+  RECE_TRY(make_tmap_bf16_ld(&tm, ws + L.yst, uint64_t(c.n_r) * c.d, uint64_t(c.C), p.ld_c,
+                             uint32_t(ns)));
+  for (int r = 0; r < c.n_r; ++r) {
+    a.r = r;
+    k_bwd_dx_tc<<<dim3(unsigned(ceil_div(c.N, kBM)), unsigned(slices)), kThreads, smem, st>>>(
+        tm, a);
+    count_launches(1);
+    RECE_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+template cudaError_t launch_dx_tc<__nv_bfloat16>(const rece_plan_s&, const __nv_bfloat16*,
+                                                 const int32_t*, const float*, const float*,
+                                                 char*, float*, uint32_t*, cudaStream_t);
+
+}  // namespace rece

@@ -107,22 +107,25 @@ __device__ WarpSel warp_select_kth(int n, int want, Get get, uint32_t* cnt) {
   }
 }
 
-template <typename T>
+// kGrouped: also hand the backward's tensor-core dX its data (entries grouped by slice,
+// probabilities, the positive logit); else the kept entries go out in list order.
+template <typename T, bool kGrouped>
 __global__ void __launch_bounds__(kThreads) k_merge_tc(
     const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
     const int32_t* __restrict__ py, const int32_t* __restrict__ invX,
     const int32_t* __restrict__ chunkY, const int2* __restrict__ list,
     const int4* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
-    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap,
-    int32_t* __restrict__ selected, float* __restrict__ lse_out, float* __restrict__ row_loss,
-    float* __restrict__ logits, uint32_t* status) {
+    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap, int Sp,
+    int32_t* __restrict__ selected, int2* __restrict__ kept, int32_t* __restrict__ kept_off,
+    float* __restrict__ pos_logit, float* __restrict__ lse_out,
+    float* __restrict__ row_loss, float* __restrict__ logits, uint32_t* status) {
   extern __shared__ __align__(16) uint8_t sh_raw[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t per_warp = size_t(cap) * 8 + kCountBytes;
   uint8_t* base = sh_raw + per_warp * wid;
   uint32_t* cnt = reinterpret_cast<uint32_t*>(base);
   uint32_t* keys = reinterpret_cast<uint32_t*>(base + kCountBytes);
-  int32_t* items = reinterpret_cast<int32_t*>(keys + cap);
+  int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);  // sorted position in its round
 
   const int64_t i = int64_t(blockIdx.x) * warps + wid;
   if (i >= N) return;  // whole warp leaves together; no block-wide barriers below
@@ -130,13 +133,18 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
   const bool z_ok = z >= 0 && z < C;
 
   // gather the candidates of all rounds
-  int cx[8];
-  for (int r = 0; r < n_r; ++r) cx[r] = int((int64_t(invX[int64_t(r) * N + i]) * n_c) / N);
+  int cx[8], px_of[8];  // per round: the row's chunk and sorted position
+  for (int r = 0; r < n_r; ++r) {
+    px_of[r] = invX[int64_t(r) * N + i];
+    cx[r] = int((int64_t(px_of[r]) * n_c) / N);
+  }
   int n = 0;
+  int rb[9];           // candidates of round r: [rb[r], rb[r + 1])
   uint32_t kmax = 0u;  // largest key buffered by this lane (0: none)
   bool overflow = false;
   float theta_max = -INFINITY;
   for (int r = 0; r < n_r; ++r) {
+    rb[r] = n < cap ? n : cap;
     const int64_t p = invX[int64_t(r) * N + i];
     // four sub-lists (one per epilogue warpgroup of the selection kernel), read as one
     // concatenated list, four independent entries per lane in flight at a time
@@ -181,7 +189,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
           if (pos < cap) {
             const uint32_t key = score_key(__int_as_float(e[u].x));
             keys[pos] = key;
-            items[pos] = jj[u];
+            poss[pos] = e[u].y;
             kmax = key > kmax ? key : kmax;
           }
         }
@@ -193,6 +201,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     overflow = true;
     n = cap;
   }
+  rb[n_r] = n;
   __syncwarp();
 
   // the positive's logit
@@ -203,6 +212,13 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
     for (int t = lane; t < d; t += 32) part = fmaf(to_f32(x[t]), to_f32(y[t]), part);
   }
   const float lp = warp_sum(part);
+
+  // item id of candidate q (its round found from the boundaries)
+  auto item_of = [&](int q) {
+    int r = 0;
+    while (r + 1 < n_r && q >= rb[r + 1]) ++r;
+    return py[int64_t(r) * C + poss[q]];
+  };
 
   // the k best
   const int kk = k < n ? k : n;
@@ -218,8 +234,9 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
       s2 = warp_select_kth(
           n, s1.need,
           [&](int q, uint32_t& key) {
-            key = ~uint32_t(items[q]);
-            return keys[q] == Tk;
+            if (keys[q] != Tk) return false;
+            key = ~uint32_t(item_of(q));
+            return true;
           },
           cnt);
     }
@@ -233,55 +250,136 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
   const float best = n > 0 ? key_score(kmax) : -INFINITY;
   const float m = fmaxf(lp, best);
 
-  // the kept entries, in the order of the candidate lists (deterministic: rounds, then
-  // each selection warpgroup's emission order), with their logits and exponentials
+  auto take = [&](int a) {
+    const uint32_t key = keys[a];
+    return all || key > s1.T || (key == s1.T && (!tie || ~uint32_t(item_of(a)) >= s2.T));
+  };
+  // the row's loss (RECE, Algorithm 1's loss lines); in grouped mode first, so that the
+  // kept entries can go out with their softmax probabilities
+  float acc = 0.0f, lse = 0.0f;
+  if constexpr (kGrouped) {
+    for (int a = lane; a < n; a += 32)
+      if (take(a)) acc += expf(key_score(keys[a]) - m);
+    lse = m + logf(warp_sum(acc) + expf(lp - m));
+  }
+  // The kept entries, by round and, within a round, grouped by 64-position slice of the
+  // round's sorted catalogue (in candidate-list order inside a slice): a stable counting
+  // sort over the slices of the row's window.  Besides the row's outputs (items, logits),
+  // the backward gets, indexed by (round, sorted row p): the round's entries
+  // kept[r][p][e] = (sorted position, p_ij as two bf16 halves hi | lo << 16, with
+  // p_ij = exp(l_ij - lse_i) = bf16(hi) + bf16(lo) to about 16 bits; 0 for a bad target)
+  // and the slice starts kept_off[r][p][s] (s = 0..S, entry S = the round's count).
   float* lg = logits ? logits + i * (int64_t(k) + 1) : nullptr;
   int32_t* srow = selected + i * k;
+  int32_t* bins = reinterpret_cast<int32_t*>(cnt);  // up to 512 slices (the count table)
   int ns = 0;
-  float worst = INFINITY, acc = 0.0f;
-  for (int a0 = 0; a0 < n; a0 += 32) {
-    const int a = a0 + lane;
-    bool take = false;
-    uint32_t key = 0u;
-    if (a < n) {
-      key = keys[a];
-      take = all || key > s1.T || (key == s1.T && (!tie || ~uint32_t(items[a]) >= s2.T));
+  float worst = INFINITY;
+  for (int r = 0; r < n_r; ++r) {
+    if constexpr (!kGrouped) {
+      // list order: rounds, then each selection warpgroup's emission order
+      for (int a0 = rb[r]; a0 < rb[r + 1]; a0 += 32) {
+        const int a = a0 + lane;
+        const bool tk = a < rb[r + 1] && take(a);
+        const unsigned b = __ballot_sync(0xFFFFFFFFu, tk);
+        if (tk) {
+          const int dest = ns + __popc(b & ((1u << lane) - 1u));
+          const float sc = key_score(keys[a]);
+          srow[dest] = py[int64_t(r) * C + poss[a]];
+          if (lg) lg[1 + dest] = sc;
+          worst = fminf(worst, sc);
+          acc += expf(sc - m);
+        }
+        ns += __popc(b);
+      }
+      continue;
     }
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, take);
-    if (take) {
-      const int pos = ns + __popc(b & ((1u << lane) - 1u));
-      const float sc = key_score(key);
-      srow[pos] = items[a];
-      if (lg) lg[1 + pos] = sc;
-      worst = fminf(worst, sc);
-      acc += expf(sc - m);
+    const int64_t c = cx[r];
+    const int64_t w0 = chunk_start(c - n_ec < 0 ? 0 : c - n_ec, C, n_c);
+    const int64_t w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
+    const int sig0 = int(w0 >> 6);
+    const int S = w1 > w0 ? int((w1 - 1) >> 6) - sig0 + 1 : 0;
+    for (int b = lane; b < S; b += 32) bins[b] = 0;
+    __syncwarp();
+    for (int a = rb[r] + lane; a < rb[r + 1]; a += 32)
+      if (take(a)) atomicAdd(&bins[(poss[a] >> 6) - sig0], 1);
+    __syncwarp();
+    // exclusive scan of the slice counts, lane l holding slices [l*B, l*B + B)
+    const int B = (S + 31) >> 5;
+    int run = 0;
+    for (int b = lane * B; b < S && b < lane * B + B; ++b) run += bins[b];
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
     }
-    ns += __popc(b);
+    const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    int at = ns + incl - run;
+    const int64_t rp = int64_t(r) * N + px_of[r];
+    int32_t* orow = kept_off + rp * Sp;
+    int2* erow = kept + rp * k;  // the round's entries, from 0
+    for (int b = lane * B; b < S && b < lane * B + B; ++b) {
+      const int v = bins[b];
+      bins[b] = at;
+      orow[b] = at - ns;
+      at += v;
+    }
+    if (lane == 0) orow[S] = total;
+    __syncwarp();
+    for (int a0 = rb[r]; a0 < rb[r + 1]; a0 += 32) {
+      const int a = a0 + lane;
+      const bool tk = a < rb[r + 1] && take(a);
+      const int sl = tk ? (poss[a] >> 6) - sig0 : 0;
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, tk ? sl : int(0x40000000 | lane));
+      const int dest = tk ? bins[sl] + __popc(peers & ((1u << lane) - 1u)) : 0;
+      __syncwarp();
+      if (tk && lane == __ffs(peers) - 1) bins[sl] += __popc(peers);
+      __syncwarp();
+      if (tk) {
+        const int32_t pos = poss[a];
+        const float sc = key_score(keys[a]);
+        srow[dest] = py[int64_t(r) * C + pos];
+        uint32_t packed = 0u;
+        if (z_ok) {
+          const float pr = expf(sc - lse);
+          const __nv_bfloat16 h = __float2bfloat16_rn(pr);
+          const __nv_bfloat16 l = __float2bfloat16_rn(pr - __bfloat162float(h));
+          packed = uint32_t(__bfloat16_as_ushort(h)) | (uint32_t(__bfloat16_as_ushort(l)) << 16);
+        }
+        erow[dest - ns] = make_int2(pos, int32_t(packed));
+        if (lg) lg[1 + dest] = sc;
+        worst = fminf(worst, sc);
+      }
+    }
+    ns += total;
+    __syncwarp();
   }
   worst = -warp_max(-worst);
+  if constexpr (!kGrouped) lse = m + logf(warp_sum(acc) + expf(lp - m));
   for (int a = ns + lane; a < k; a += 32) {
     srow[a] = -1;
     if (lg) lg[1 + a] = -INFINITY;
   }
-  if (lg && lane == 0) lg[0] = z_ok ? lp : NAN;
+  if (lane == 0) {
+    if (lg) lg[0] = z_ok ? lp : NAN;
+    if (kGrouped) pos_logit[i] = z_ok ? lp : NAN;
+  }
 
   // theta_max: the largest score some round did not emit (-inf if every round emitted
   // all); the k-th kept score is the smallest kept one
   const float s_k = ns < k ? -INFINITY : worst;
   if (lane == 0 && (overflow || (theta_max > -INFINITY && theta_max >= s_k))) {
     atomicAdd(status + 1, 1u);
+    if (overflow) atomicAdd(status + 2, 1u);
     raise_flag(status, RECE_DEVICE_INEXACT);
   }
 
-  // loss of the row (RECE, Algorithm 1's loss lines)
-  const float tot = warp_sum(acc) + expf(lp - m);
   if (lane == 0) {
     if (!z_ok) {
       raise_flag(status, RECE_DEVICE_BAD_TARGET);
       lse_out[i] = NAN;
       if (row_loss) row_loss[i] = NAN;
     } else {
-      const float lse = m + logf(tot);
       lse_out[i] = lse;
       if (row_loss) row_loss[i] = lse - lp;
     }
@@ -304,8 +402,10 @@ template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
                             const int2* list, const int4* list_count,
-                            const float* list_theta, int32_t* selected, float* lse,
-                            float* row_loss, float* logits, uint32_t* status, cudaStream_t st) {
+                            const float* list_theta, int32_t* selected, int2* kept,
+                            int32_t* kept_off, float* pos_logit, int Sp,
+                            float* lse, float* row_loss, float* logits, uint32_t* status,
+                            cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
   const int Qw = tc_sublist_capacity(c.k);
@@ -313,12 +413,15 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   int warps = int((200 * 1024) / per_warp);
   warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
   const size_t smem = per_warp * warps;
-  cudaError_t e = cudaFuncSetAttribute(k_merge_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool grouped = kept != nullptr;
+  auto kern = grouped ? k_merge_tc<T, true> : k_merge_tc<T, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  k_merge_tc<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
+  kern<<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
       X, Y, targets, py, invX, chunkY, list, list_count, list_theta, c.N, c.C, c.d, c.k, c.n_r,
-      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), selected, lse, row_loss, logits, status);
+      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), Sp, selected, kept, kept_off, pos_logit, lse,
+      row_loss, logits, status);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -326,6 +429,6 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
 template cudaError_t launch_merge_tc<__nv_bfloat16>(
     const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
     const int32_t*, const int32_t*, const int32_t*, const int2*, const int4*, const float*,
-    int32_t*, float*, float*, float*, uint32_t*, cudaStream_t);
+    int32_t*, int2*, int32_t*, float*, int, float*, float*, float*, uint32_t*, cudaStream_t);
 
 }  // namespace rece

@@ -69,6 +69,10 @@ struct Layout {
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_sorted_g = 0,
          e_key_b = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0;
   size_t bwd_end = 0;
+  // tensor-core dX: kept from rece_loss_fwd to rece_loss_bwd (not aliased): the d-major
+  // sorted copy of Y, the kept entries by (round, sorted row) with their slice starts, and
+  // each row's positive logit
+  size_t yst = 0, kept = 0, kept_off = 0, pos_logit = 0;
   size_t total = 0;
 };
 
@@ -86,6 +90,9 @@ struct rece_plan_s {
   int32_t item_pass_bits;  // digit bits of every pass but the last
   int64_t entries;      // N * (k + 1): (row, item) pairs of the backward
   bool use_tc;          // bf16 mode on the tcgen05 kernels
+  bool tc_dx;           // ... and dX of the backward on them too
+  int32_t kept_slices;  // most 64-position slices one window touches
+  int64_t ld_c;         // row pitch (elements) of the d-major copy of Y: C rounded up to 8
   rece::Layout lay;
   void* stage_events[2 * RECE_NUM_STAGES];  // optional timing hook (cudaEvent_t)
   bool timed;
@@ -117,6 +124,14 @@ cudaError_t launch_bucketize_fma(const T* V, int64_t M, int d, const T* B, int n
 // digit_start[2^bits] = M).
 // With in_order, element p's key and payload are keys[p] and payload[p] (a previous pass
 // wrote them in the order of its output) instead of being looked up by id.
+cudaError_t sort_pairs_by_item(const rece_plan_s& p, int64_t E, const int32_t* key,
+                               const float* g, int32_t* perm_a, int32_t* perm_b, int32_t* key_b,
+                               float* g_b, int32_t* sorted_key, float* sorted_g, void* scratch,
+                               const int32_t** sorted_id, cudaStream_t st);
+template <typename T>
+cudaError_t launch_items_from_pairs(const T* X, int64_t C, int d, int slots,
+                                    const int32_t* item_start, const int32_t* sorted_id,
+                                    const float* sorted_g, float* dY, cudaStream_t st);
 cudaError_t launch_sort_batch(const SortSeg* segs, int n, int shift, int bits, bool in_order,
                               cudaStream_t st);
 cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,

@@ -62,13 +62,26 @@ void build_layout(rece_plan_s& p) {
     off += align256(bytes);
     return o;
   };
-  L.status = take(2 * sizeof(uint32_t));  // flags, count of inexact rows
-  const size_t region = off;
+  L.status = take(4 * sizeof(uint32_t));  // flags, inexact rows, of which overflowed
   const size_t nb_stride = (size_t(1) << p.bucket_bits) + 1;
+  if (p.use_tc) {
+    // the orders, kept from rece_loss_fwd until rece_loss_bwd has run
+    L.px = take(sizeof(int32_t) * c.n_r * c.N);
+    L.py = take(sizeof(int32_t) * c.n_r * c.C);
+  }
+  if (p.tc_dx) {
+    L.yst = take(sizeof(uint16_t) * size_t(c.n_r) * c.d * p.ld_c);
+    L.kept = take(sizeof(int2) * size_t(c.n_r) * c.N * c.k);
+    L.kept_off = take(sizeof(int32_t) * size_t(c.n_r) * c.N * (size_t(p.kept_slices) + 1));
+    L.pos_logit = take(sizeof(float) * size_t(c.N));
+  }
+  const size_t region = off;
   L.bx = take(sizeof(int32_t) * c.n_r * c.N);
   L.by = take(sizeof(int32_t) * c.n_r * c.C);
-  L.px = take(sizeof(int32_t) * c.n_r * c.N);
-  L.py = take(sizeof(int32_t) * c.n_r * c.C);
+  if (!p.use_tc) {
+    L.px = take(sizeof(int32_t) * c.n_r * c.N);
+    L.py = take(sizeof(int32_t) * c.n_r * c.C);
+  }
   L.bstart_x = take(sizeof(int32_t) * c.n_r * nb_stride);
   L.bstart_y = take(sizeof(int32_t) * c.n_r * nb_stride);
   // the forward sorts (X and Y of every round) run as one batch, a histogram each
@@ -90,17 +103,19 @@ void build_layout(rece_plan_s& p) {
   L.row_loss_tmp = take(sizeof(float) * c.N);
   L.fwd_end = off;
   off = region;
-  const size_t E = size_t(p.entries);
-  L.e_key = take(sizeof(int32_t) * E);
-  L.e_g = take(sizeof(float) * E);
-  L.e_perm_a = take(sizeof(int32_t) * E);
-  L.e_perm_b = take(sizeof(int32_t) * E);
-  L.e_sorted_key = take(sizeof(int32_t) * E);
-  L.e_sorted_g = take(sizeof(float) * E);
-  L.e_key_b = take(sizeof(int32_t) * E);
-  L.e_g_b = take(sizeof(float) * E);
-  L.e_item_start = take(sizeof(int32_t) * (size_t(c.C) + 1));
-  L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
+  {
+    const size_t E = size_t(p.entries);
+    L.e_key = take(sizeof(int32_t) * E);
+    L.e_g = take(sizeof(float) * E);
+    L.e_perm_a = take(sizeof(int32_t) * E);
+    L.e_perm_b = take(sizeof(int32_t) * E);
+    L.e_sorted_key = take(sizeof(int32_t) * E);
+    L.e_sorted_g = take(sizeof(float) * E);
+    L.e_key_b = take(sizeof(int32_t) * E);
+    L.e_g_b = take(sizeof(float) * E);
+    L.e_item_start = take(sizeof(int32_t) * (size_t(c.C) + 1));
+    L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
+  }
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
@@ -186,7 +201,22 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   p->entries = c.N * (int64_t(c.k) + 1);
   p->timed = false;
   for (void*& e : p->stage_events) e = nullptr;
-  p->use_tc = tc_supported(*p);
+  p->kept_slices = 0;
+  for (int64_t ch = 0; ch < c.n_c; ++ch) {
+    const int64_t w0 = chunk_start(ch - c.n_ec < 0 ? 0 : ch - c.n_ec, c.C, c.n_c);
+    const int64_t w1 = chunk_start(ch + c.n_ec + 1 > c.n_c ? c.n_c : ch + c.n_ec + 1, c.C, c.n_c);
+    const int64_t sl = w1 > w0 ? ((w1 - 1) >> 6) - (w0 >> 6) + 1 : 0;
+    if (sl > p->kept_slices) p->kept_slices = int32_t(sl);
+  }
+  p->ld_c = (c.C + 7) / 8 * 8;
+  // the tensor-core path groups each row's kept entries by slice of its window
+  // (the selection's 16-bit histogram counts hold windows of fewer than 65536 items)
+  p->use_tc = tc_supported(*p) && p->w_max < 65536;
+  // dX on the tensor cores where gathering catalogue rows is the slow way: large d, or a
+  // sorted catalogue that does not fit in half of L2; the merge groups each row's kept
+  // entries by slice of its window for it
+  p->tc_dx = p->use_tc && p->kept_slices <= kMaxKeptSlices &&
+             (c.d >= 256 || 2.0 * double(c.C) * c.d > 64.0 * 1024 * 1024);
   if (p->use_tc && merge_tc_warp_bytes(c.n_r, c.k) > 200 * 1024) {
     delete p;
     return fail(RECE_ERR_UNSUPPORTED, "n_r * k too large for the tensor-core merge");
@@ -240,7 +270,7 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const Layout& L = plan->lay;
-  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, 2 * sizeof(uint32_t), st), "status reset");
+  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, 4 * sizeof(uint32_t), st), "status reset");
   int32_t* bx = reinterpret_cast<int32_t*>(ws + L.bx);
   int32_t* by = reinterpret_cast<int32_t*>(ws + L.by);
   stage_mark(*plan, RECE_STAGE_BUCKETIZE, 0, st);
@@ -292,6 +322,9 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
                                   c.n_r, c.n_c, ws + L.ys, nullptr,
                                   reinterpret_cast<int32_t*>(ws + L.chunk_y), st),
               "permute Y");
+    if (plan->tc_dx)
+      RECE_CUDA(launch_transpose_sorted(ws + L.ys, c.C, c.d, c.n_r, plan->ld_c, ws + L.yst, st),
+                "d-major copy of Y");
   }
   stage_mark(*plan, RECE_STAGE_SORT, 1, st);
   return RECE_OK;
@@ -338,7 +371,11 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     RECE_CUDA(launch_merge_tc(*plan, Xb, Yb, targets, py,
                               reinterpret_cast<const int32_t*>(ws + L.inv_x),
                               reinterpret_cast<const int32_t*>(ws + L.chunk_y), list, cnt, theta,
-                              selected, lse, rl, logits, status, st),
+                              selected,
+                              plan->tc_dx ? reinterpret_cast<int2*>(ws + L.kept) : nullptr,
+                              plan->tc_dx ? reinterpret_cast<int32_t*>(ws + L.kept_off) : nullptr,
+                              plan->tc_dx ? reinterpret_cast<float*>(ws + L.pos_logit) : nullptr,
+                              plan->kept_slices + 1, lse, rl, logits, status, st),
               "merge/loss (tcgen05 lists)");
   } else {
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);

@@ -12,8 +12,10 @@
 //           columns of every tile; all of them when the window is short);
 //   pass 2  per row: exact histogram, in shared memory, of the distance key(A) - key(s)
 //           >> 20 where key is the order-preserving integer image of an fp32 score and A
-//           lies two binades beyond m -- 8 bins per binade of |s| (128 bins, the last one
-//           open), so the bins follow the scores' own scale whatever their distribution.
+//           lies two binades beyond m -- 8 bins per binade of |s| (256 bins, 32 binades,
+//           the last one open), so the bins follow the scores' own scale whatever their
+//           distribution (heavy-tailed item norms put the k-th score a dozen binades and
+//           more below the row's best).
 //           The distance is one integer multiply-add on the score's bits;
 //   pass 3  the smallest bin b* whose cumulative count reaches E = k + 1 sets the
 //           cut, turned into the fp32 threshold t at the lower edge of bin b*: every score
@@ -42,7 +44,8 @@ using namespace sm100;
 
 constexpr int kStages = 4;
 constexpr int kPasses = 3;
-constexpr int kBins = 128;
+constexpr int kBins = 256;                // 8 per binade: 32 binades below the anchor
+constexpr int kBinWords = kBins / 2;      // two 16-bit counts per shared word
 constexpr int kHeadBins = 16;          // bins above the pass 1 max (2 binades)
 constexpr int kSampleAllBelow = 1024;  // windows shorter than this are looked at whole
 constexpr int kBM = 128;
@@ -55,7 +58,7 @@ constexpr int kAcc = 4;       // TMEM accumulators of kBN columns, one per epilo
 constexpr int kEpiWarps = 4 * kAcc;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = 64 + kEpiThreads;
-static_assert(kBins * kBM == kEpiThreads * 32, "pass 3 staging fills the histogram space");
+static_assert(kBinWords * kBM == kEpiThreads * 32, "pass 3 staging fills the histogram space");
 
 struct __align__(1024) Smem {
   uint8_t a[kStages][kStageABytes];
@@ -68,7 +71,9 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort;
   // per row (column) histogram of pass 2; pass 3 reuses the space to stage scores
-  __align__(16) uint32_t hist[kBins][kBM];
+  // (bins 2w and 2w+1 of a row share word w: low and high 16 bits; a window holds fewer
+  // than 65536 scores, so a count never reaches the other half)
+  __align__(16) uint32_t hist[kBinWords][kBM];
   float part_mx[kAcc][kBM];   // pass 1 partial maxima of the warpgroups
   int emit_cnt[kAcc][kBM];    // pass 3 entries each warpgroup emitted, per row
 };
@@ -90,7 +95,7 @@ struct ItemGeom {
 // pass 1 may have looked at a sample only -- still get bins of their own.  For m >= 0 the
 // distance of a score s is A - bits(s), for m < 0 it is bits(s) - A: in both cases
 // key(anchor) - key(s) with key the order-preserving integer image of an fp32 value, as
-// long as s lies between zero and the anchor.  Bin = min(distance >> 20, 127): 8 bins per
+// long as s lies between zero and the anchor.  Bin = min(distance >> 20, 255): 8 bins per
 // binade of |s|.  Any other score (beyond the anchor, or on the far side of zero) wraps
 // to a huge distance, normally the open last bin; that only misplaces the cut, since
 // the emission itself compares values and the exactness check below stays sound.
@@ -116,8 +121,11 @@ __device__ __forceinline__ float cut_threshold(const BinMap& b, uint32_t L) {
   return tb < 0xFF800000ull ? __uint_as_float(uint32_t(tb)) : -INFINITY;
 }
 
-__device__ __forceinline__ void red_shared_add1(uint32_t addr) {
-  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr));
+// One more count in bin b of the row whose column of words starts at shared address hcol.
+__device__ __forceinline__ void bin_add(uint32_t hcol, uint32_t b) {
+  const uint32_t addr = hcol + (b >> 1) * (kBM * 4);
+  const uint32_t inc = 1u << ((b & 1u) << 4);
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(inc));
 }
 
 // The largest fp32 value below t (t finite or +0/-0): every score < t is <= it.
@@ -287,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           // combine the warpgroups' maxima; reset this item's histogram
           named_barrier(1, kEpiThreads);
           s.part_mx[wg][row_local] = mx;
-          for (int b = wg * (kBins / kAcc); b < (wg + 1) * (kBins / kAcc); ++b)
+          for (int b = wg * (kBinWords / kAcc); b < (wg + 1) * (kBinWords / kAcc); ++b)
             s.hist[b][row_local] = 0;
           named_barrier(1, kEpiThreads);
           mx = s.part_mx[0][row_local];
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           if (histo) {
             uint32_t cum = 0;
             for (int b = 0; b < kBins - 1; ++b) {
-              cum += s.hist[b][row_local];
+              cum += (s.hist[b >> 1][row_local] >> ((b & 1) * 16)) & 0xFFFFu;
               if (cum >= uint32_t(E)) {
                 thr = cut_threshold(bmap, uint32_t(b + 1) << 20);
                 break;
@@ -346,14 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
-                  red_shared_add1(hcol + min(raw, uint32_t(kBins - 1)) * (kBM * 4));
+                  bin_add(hcol, min(raw, uint32_t(kBins - 1)));
                 }
               } else {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   if (u < lo || u >= hi) continue;
                   const uint32_t raw = (__float_as_uint(v[u]) * bmap.sig + bmap.off) >> 20;
-                  red_shared_add1(hcol + min(raw, uint32_t(kBins - 1)) * (kBM * 4));
+                  bin_add(hcol, min(raw, uint32_t(kBins - 1)));
                 }
               }
             } else {

@@ -13,6 +13,10 @@ namespace rece {
 // 64 columns x box_rows rows, 128-byte swizzle (the K-major layout the MMA reads).
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows);
+// The same for a matrix whose rows are ld >= cols elements apart (ld * 2 a multiple of
+// 16 bytes) and whose column count is arbitrary: boxes past the last column read zeros.
+cudaError_t make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                              uint64_t ld, uint32_t box_rows);
 int sm_count();
 
 // bf16 mode without RECE_FLAG_FMA_SCORES and d a multiple of 64: the tcgen05 kernels run.
@@ -28,6 +32,10 @@ cudaError_t launch_permute_rows(const void* V, int64_t M, int d, const int32_t* 
                                 int n_c, void* Vs, int32_t* inv, int32_t* chunk,
                                 cudaStream_t st);
 
+// VsT[r][t][p] = Vs[r][p][t]: d-major copies (rows ld elements apart, ld % 8 == 0).
+cudaError_t launch_transpose_sorted(const void* Vs, int64_t M, int d, int n_r, int64_t ld,
+                                    void* VsT, cudaStream_t st);
+
 // K3 on tensor cores: per (round, sorted row) the candidate list (score bits, sorted
 // catalogue position), its count and threshold.
 int tc_list_capacity(int k);      // entries per (round, row): 4 sub-lists
@@ -36,13 +44,28 @@ cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Y
                              int4* list_count, float* list_theta, uint32_t* status,
                              cudaStream_t st);
 
-// K4 for the tensor-core lists: merge, select, order, loss, exactness check.
+// K4 for the tensor-core lists: merge, select, loss, exactness check.  The kept entries
+// go out by round and 64-position slice of the round's sorted catalogue: items
+// (selected [N][k]) and logits ([N][k+1], or NULL), and for the backward, indexed by
+// (round r, sorted row p): kept [n_r][N][k] = (sorted position, softmax probability as
+// bf16 hi | lo << 16), kept_off [n_r][N][Sp] = slice starts of the row's window (entry S
+// = the count); and pos_logit [N], each row's positive logit.
 size_t merge_tc_warp_bytes(int n_r, int k);
+constexpr int kMaxKeptSlices = 512;  // slices of one window the merge can group by
 template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
                             const int2* list, const int4* list_count,
-                            const float* list_theta, int32_t* selected, float* lse,
-                            float* row_loss, float* logits, uint32_t* status, cudaStream_t st);
+                            const float* list_theta, int32_t* selected, int2* kept,
+                            int32_t* kept_off, float* pos_logit, int Sp,
+                            float* lse, float* row_loss, float* logits, uint32_t* status,
+                            cudaStream_t st);
+
+// dX of step 6 on tensor cores (see bwd_tc.cu): written, not accumulated.  Needs the
+// grouped merge outputs (kept, kept_off, pos_logit) and the d-major copy YsT.
+template <typename T>
+cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* targets,
+                         const float* lse, const float* dloss, char* ws, float* dX,
+                         uint32_t* status, cudaStream_t st);
 
 }  // namespace rece

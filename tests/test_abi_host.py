@@ -93,8 +93,13 @@ def test_workspace_size_and_layout():
         assert lay.status == 0
         offs = [lay.bucket_x, lay.bucket_y, lay.perm_x, lay.perm_y, lay.bucket_start_y]
         assert all(o % 256 == 0 for o in offs)
-        assert lay.bucket_y >= lay.bucket_x + 4 * c.n_r * c.N
-        assert lay.perm_x >= lay.bucket_y + 4 * c.n_r * c.C
+        # the arrays the caller may read after rece_bucketize_sort do not overlap
+        spans = sorted([(lay.bucket_x, 4 * c.n_r * c.N), (lay.bucket_y, 4 * c.n_r * c.C),
+                        (lay.perm_x, 4 * c.n_r * c.N), (lay.perm_y, 4 * c.n_r * c.C),
+                        (lay.bucket_start_y, 4 * c.n_r * lay.bucket_start_stride)])
+        for (a, na), (b, _) in zip(spans, spans[1:]):
+            assert a + na <= b
+        assert spans[-1][0] + spans[-1][1] <= p.workspace_bytes
         lists = 8 * c.n_r * c.N * c.k
         pairs = 5 * 4 * c.N * (c.k + 1)
         assert p.workspace_bytes >= max(lists, pairs)
