@@ -6,9 +6,11 @@
 //                                   products for its own slots, then the lanes sweep the
 //                                   dimensions adding the slots in order)
 //   dY_j = sum_i g_ij x_i          (no float atomics: the (item, row) pairs are put in
-//                                   item order by a stable LSD radix sort that carries g
-//                                   along, then one warp per item sums its pairs in row
-//                                   order)
+//                                   item order by a stable LSD radix sort of (item, pair
+//                                   id), then one warp per item sums its pairs in row
+//                                   order, fetching each pair's g by its id -- or, when
+//                                   the g array is too large for L2, g rides along in
+//                                   the sort)
 // Pair e = i*(k+1) + s holds slot s of row i (s = 0: the positive, s >= 1: selected
 // negative s-1); an empty slot carries the key C, which sorts after every item.  Every
 // sum has a fixed order: the gradients are deterministic.
@@ -125,8 +127,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_items(
     const T* __restrict__ X, int64_t C, int d, int k, const int32_t* __restrict__ item_start,
-    const int32_t* __restrict__ sorted_id, const float* __restrict__ sorted_g,
-    float* __restrict__ dY) {
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ pair_g,
+    const float* __restrict__ sorted_g, float* __restrict__ dY) {
   const int lane = threadIdx.x & 31;
   const int64_t j = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
   if (j >= C) return;
@@ -142,8 +144,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items(
       int32_t row = 0;
       float g = 0.0f;
       if (lane < n) {
-        row = sorted_id[b + lane] / slots;
-        g = sorted_g[b + lane];
+        const int32_t id = sorted_id[b + lane];
+        row = id / slots;
+        g = sorted_g ? sorted_g[b + lane] : pair_g[id];
       }
 #pragma unroll 4
       for (int q = 0; q < n; ++q) {
@@ -312,8 +315,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
     const T* __restrict__ X, int64_t C, int d, int k, const int32_t* __restrict__ item_start,
-    const int32_t* __restrict__ sorted_id, const float* __restrict__ sorted_g,
-    float* __restrict__ dY) {
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ pair_g,
+    const float* __restrict__ sorted_g, float* __restrict__ dY) {
   const int lane = threadIdx.x & 31, q = lane >> 3, sub = lane & 7;
   const int64_t j = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
   if (j >= C) return;
@@ -327,8 +330,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
       int32_t row = 0;
       float g = 0.0f;
       if (lane < n) {
-        row = sorted_id[b + lane] / slots;
-        g = sorted_g[b + lane];
+        const int32_t id = sorted_id[b + lane];
+        row = id / slots;
+        g = sorted_g ? sorted_g[b + lane] : pair_g[id];
       }
       for (int e0 = 0; e0 < n; e0 += 4) {
         const int e = e0 + q;
@@ -359,10 +363,10 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
 
 size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 * (k + 1)); }
 
-// LSD radix sort of E (item key, g) pairs by key (values 0..C), as few passes as the
-// counting sort's 12-bit digit limit allows.  Every pass writes keys and g in its output
-// order, so the next pass reads them contiguously; *sorted_id (perm_a or perm_b) says
-// where each sorted pair came from.  The last pass lands in sorted_key / sorted_g.
+// LSD radix sort of E pairs by item key (values 0..C), as few passes as the counting
+// sort's 12-bit digit limit allows.  Every pass writes the keys (and g, when given) in its
+// output order, so the next pass reads them contiguously; *sorted_id (perm_a or perm_b)
+// says where each sorted pair came from.  The last pass lands in sorted_key / sorted_g.
 cudaError_t sort_pairs_by_item(const rece_plan_s& p, int64_t E, const int32_t* key,
                                const float* g, int32_t* perm_a, int32_t* perm_b, int32_t* key_b,
                                float* g_b, int32_t* sorted_key, float* sorted_g, void* scratch,
@@ -379,37 +383,17 @@ cudaError_t sort_pairs_by_item(const rece_plan_s& p, int64_t E, const int32_t* k
     const int bits = (ps + 1 < passes) ? p.item_pass_bits : p.item_bits - shift;
     const int slot = (passes - 1 - ps) % 2 == 0 ? 1 : 0;
     cudaError_t e = launch_sort_pass(kin, in, E, shift, bits, scratch, out, key_buf[slot],
-                                     nullptr, st, gin, g_buf[slot], ps > 0);
+                                     nullptr, st, gin, gin ? g_buf[slot] : nullptr, ps > 0);
     if (e != cudaSuccess) return e;
     shift += bits;
     in = out;
     kin = key_buf[slot];
-    gin = g_buf[slot];
+    gin = gin ? g_buf[slot] : nullptr;
     out = (out == perm_a) ? perm_b : perm_a;
   }
   *sorted_id = in;
   return cudaSuccess;
 }
-
-// dY_j = sum of g x_row over the pairs of item j (sorted by item; pair id / slots = row),
-// written for every item (0 where it has no pair).
-template <typename T>
-cudaError_t launch_items_from_pairs(const T* X, int64_t C, int d, int slots,
-                                    const int32_t* item_start, const int32_t* sorted_id,
-                                    const float* sorted_g, float* dY, cudaStream_t st) {
-  const int warps = kThreads / 32;
-  if (d % 8 == 0)
-    k_bwd_items_v8<T><<<unsigned(ceil_div(C, warps)), kThreads, 0, st>>>(
-        X, C, d, slots - 1, item_start, sorted_id, sorted_g, dY);
-  else
-    k_bwd_items<T><<<unsigned(ceil_div(C, warps)), kThreads, 0, st>>>(
-        X, C, d, slots - 1, item_start, sorted_id, sorted_g, dY);
-  count_launches(1);
-  return cudaGetLastError();
-}
-template cudaError_t launch_items_from_pairs<__nv_bfloat16>(const __nv_bfloat16*, int64_t, int,
-                                                            int, const int32_t*, const int32_t*,
-                                                            const float*, float*, cudaStream_t);
 
 template <typename T>
 cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
@@ -427,7 +411,7 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   int32_t* perm_a = reinterpret_cast<int32_t*>(ws + L.e_perm_a);
   int32_t* perm_b = reinterpret_cast<int32_t*>(ws + L.e_perm_b);
   int32_t* sorted_key = reinterpret_cast<int32_t*>(ws + L.e_sorted_key);
-  float* sorted_g = reinterpret_cast<float*>(ws + L.e_sorted_g);
+  float* sorted_g = p.carry_g ? reinterpret_cast<float*>(ws + L.e_sorted_g) : nullptr;
   void* scratch = ws + L.e_scratch;
   stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
   if (c.N > 0) {
@@ -462,10 +446,10 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
   const int32_t* in = nullptr;
   {
-    cudaError_t e = sort_pairs_by_item(p, E, e_key, e_g, perm_a, perm_b,
-                                       reinterpret_cast<int32_t*>(ws + L.e_key_b),
-                                       reinterpret_cast<float*>(ws + L.e_g_b), sorted_key,
-                                       sorted_g, scratch, &in, st);
+    cudaError_t e = sort_pairs_by_item(
+        p, E, e_key, p.carry_g ? e_g : nullptr, perm_a, perm_b,
+        reinterpret_cast<int32_t*>(ws + L.e_key_b), reinterpret_cast<float*>(ws + L.e_g_b),
+        sorted_key, sorted_g, scratch, &in, st);
     if (e != cudaSuccess) return e;
   }
   int32_t* item_start = reinterpret_cast<int32_t*>(ws + L.e_item_start);
@@ -476,10 +460,10 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   const int warps = kThreads / 32;
   if (c.d % 8 == 0)
     k_bwd_items_v8<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
-        X, c.C, c.d, c.k, item_start, in, sorted_g, dY);
+        X, c.C, c.d, c.k, item_start, in, e_g, sorted_g, dY);
   else
     k_bwd_items<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
-        X, c.C, c.d, c.k, item_start, in, sorted_g, dY);
+        X, c.C, c.d, c.k, item_start, in, e_g, sorted_g, dY);
   count_launches(1);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
   return cudaGetLastError();

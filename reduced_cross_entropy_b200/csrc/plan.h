@@ -66,8 +66,8 @@ struct Layout {
   size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0;
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
-  size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_sorted_g = 0,
-         e_key_b = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0;
+  size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_key_b = 0,
+         e_sorted_g = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0;
   size_t bwd_end = 0;
   // tensor-core dX: kept from rece_loss_fwd to rece_loss_bwd (not aliased): the d-major
   // sorted copy of Y, the kept entries by (round, sorted row) with their slice starts, and
@@ -89,6 +89,7 @@ struct rece_plan_s {
   int32_t item_passes;  // LSD passes of that sort (digits of at most 12 bits)
   int32_t item_pass_bits;  // digit bits of every pass but the last
   int64_t entries;      // N * (k + 1): (row, item) pairs of the backward
+  bool carry_g;         // the pair sort carries g (its array would not stay in L2)
   bool use_tc;          // bf16 mode on the tcgen05 kernels
   bool tc_dx;           // ... and dX of the backward on them too
   int32_t kept_slices;  // most 64-position slices one window touches
@@ -128,10 +129,6 @@ cudaError_t sort_pairs_by_item(const rece_plan_s& p, int64_t E, const int32_t* k
                                const float* g, int32_t* perm_a, int32_t* perm_b, int32_t* key_b,
                                float* g_b, int32_t* sorted_key, float* sorted_g, void* scratch,
                                const int32_t** sorted_id, cudaStream_t st);
-template <typename T>
-cudaError_t launch_items_from_pairs(const T* X, int64_t C, int d, int slots,
-                                    const int32_t* item_start, const int32_t* sorted_id,
-                                    const float* sorted_g, float* dY, cudaStream_t st);
 cudaError_t launch_sort_batch(const SortSeg* segs, int n, int shift, int bits, bool in_order,
                               cudaStream_t st);
 cudaError_t launch_sort_pass(const int32_t* keys, const int32_t* in_ids, int64_t M, int shift,

@@ -110,9 +110,11 @@ void build_layout(rece_plan_s& p) {
     L.e_perm_a = take(sizeof(int32_t) * E);
     L.e_perm_b = take(sizeof(int32_t) * E);
     L.e_sorted_key = take(sizeof(int32_t) * E);
-    L.e_sorted_g = take(sizeof(float) * E);
     L.e_key_b = take(sizeof(int32_t) * E);
-    L.e_g_b = take(sizeof(float) * E);
+    if (p.carry_g) {
+      L.e_sorted_g = take(sizeof(float) * E);
+      L.e_g_b = take(sizeof(float) * E);
+    }
     L.e_item_start = take(sizeof(int32_t) * (size_t(c.C) + 1));
     L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
   }
@@ -199,6 +201,7 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   if (p->item_passes < 1) p->item_passes = 1;
   p->item_pass_bits = (p->item_bits + p->item_passes - 1) / p->item_passes;
   p->entries = c.N * (int64_t(c.k) + 1);
+  p->carry_g = p->entries * int64_t(sizeof(float)) > (int64_t(32) << 20);
   p->timed = false;
   for (void*& e : p->stage_events) e = nullptr;
   p->kept_slices = 0;

@@ -304,14 +304,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           bmap = bin_map(mx);
         } else if (pass == 2) {
           named_barrier(1, kEpiThreads);  // every histogram increment has landed
-          if (histo) {
+          if (histo) {  // else thr stays -inf: emit the whole window
+            // the smallest bin b* (< 255, the last one open) whose cumulative count
+            // reaches E: whole blocks of 16 bins are skipped while their sum falls short
             uint32_t cum = 0;
-            for (int b = 0; b < kBins - 1; ++b) {
-              cum += (s.hist[b >> 1][row_local] >> ((b & 1) * 16)) & 0xFFFFu;
-              if (cum >= uint32_t(E)) {
-                thr = cut_threshold(bmap, uint32_t(b + 1) << 20);
-                break;
+            for (int w0 = 0; w0 < kBinWords; w0 += 8) {
+              uint32_t blk = 0;
+#pragma unroll
+              for (int w = 0; w < 8; ++w) {
+                const uint32_t v = s.hist[w0 + w][row_local];
+                blk += (v & 0xFFFFu) + (v >> 16);
               }
+              if (cum + blk < uint32_t(E)) {
+                cum += blk;
+                continue;
+              }
+              int bstar = -1;
+              for (int b = 2 * w0; b < 2 * w0 + 16 && b < kBins - 1; ++b) {
+                cum += (s.hist[b >> 1][row_local] >> ((b & 1) * 16)) & 0xFFFFu;
+                if (cum >= uint32_t(E)) {
+                  bstar = b;
+                  break;
+                }
+              }
+              if (bstar >= 0) thr = cut_threshold(bmap, uint32_t(bstar + 1) << 20);
+              break;
             }
           }
           named_barrier(1, kEpiThreads);  // histogram read by all: its space is staging now

@@ -128,3 +128,18 @@ def test_tc_path_exact_on_integer_inputs(d, n_c, n_ec, n_r, k):
         s = sel[i][sel[i] >= 0]
         np.testing.assert_array_equal(lg[i, 1:1 + len(s)], Y[s] @ X[i])
         assert np.all(lg[i, 1 + len(s):] == -np.inf)
+
+
+def test_backward_past_the_in_cache_pair_size():
+    """N (k+1) > 8.4M pairs: the pair sort carries each pair's coefficient instead of the
+    item pass gathering it.  Gradients against the oracle's, for the GPU's selection."""
+    w = synth.WORKLOADS["sasrec"].scaled(33_000, 100_000)
+    assert w.N * (w.k + 1) * 4 > (32 << 20)
+    X, Y, t = synth.make_inputs(w, seed=6)
+    B = synth.projections(6, 0, w.n_r, w.n_b, w.d, "bf16")
+    g = run_gpu(w, X, Y, t, B, flags=0, dloss=0.5)
+    assert g["status"] & ~0x4 == 0
+    _, _, lse = oracle.rece_loss(X, Y, t, g["selected"])
+    oX, oY = oracle.rece_grad(X, Y, t, g["selected"], lse, 0.5)
+    assert max_rel(g["dX"], oX) <= 1e-3
+    assert max_rel(g["dY"], oY) <= 1e-3
