@@ -350,6 +350,7 @@ def main():
     status_words = ws[:16].view(torch.int32).cpu().tolist()
     assert status_words[0] & ~_lib.DEVICE_INEXACT == 0, f"device status {status_words[0]:#x}"
     inexact_rows, overflow_rows = int(status_words[1]), int(status_words[2])
+    spilled_rows = int(status_words[3])
 
     # timed region: K steps, each bracketed by events; per-stage events recorded by the
     # library on the same stream
@@ -445,6 +446,7 @@ def main():
             "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": workload_desc(w), "inexact_rows_per_step": inexact_rows,
                        "overflowed_rows_per_step": overflow_rows,
+                       "merge_spilled_rows_per_step": spilled_rows,
                        "l2": "flushed between timed steps (256 MiB write)",
                        "scores": "tcgen05" if uses_tensor_cores(w, args.flags)
                        else "fmaf CUDA cores"},

@@ -107,28 +107,61 @@ __device__ WarpSel warp_select_kth(int n, int want, Get get, uint32_t* cnt) {
   }
 }
 
+template <typename T>
+struct MergeArgs {
+  const T* X;
+  const T* Y;
+  const int32_t* targets;
+  const int32_t* py;
+  const int32_t* invX;
+  const int32_t* chunkY;
+  const int2* list;
+  const int4* list_count;
+  const float* list_theta;
+  int64_t N, C;
+  int d, k, n_r, n_c, n_ec, Qw, Sp;
+  int32_t* selected;
+  int2* kept;
+  int32_t* kept_off;
+  float* pos_logit;
+  float* lse_out;
+  float* row_loss;
+  float* logits;
+  uint32_t* status;
+  int32_t* spill_rows;    // rows whose candidates did not fit the fast path's buffer
+  uint32_t* spill_count;  // how many (status area)
+};
+
+// One row, one warp.  keys / poss: the candidate buffer (cap entries each); cnt: the
+// warp's 16 x 32 count table (shared memory).  When more candidates arrive than the buffer
+// holds, a row with `spill` set is handed to the spill list and nothing is written for it
+// (returns false); without, the first cap are kept and the row is flagged inexact.
 // kGrouped: also hand the backward's tensor-core dX its data (entries grouped by slice,
 // probabilities, the positive logit); else the kept entries go out in list order.
 template <typename T, bool kGrouped>
-__global__ void __launch_bounds__(kThreads) k_merge_tc(
-    const T* __restrict__ X, const T* __restrict__ Y, const int32_t* __restrict__ targets,
-    const int32_t* __restrict__ py, const int32_t* __restrict__ invX,
-    const int32_t* __restrict__ chunkY, const int2* __restrict__ list,
-    const int4* __restrict__ list_count, const float* __restrict__ list_theta, int64_t N,
-    int64_t C, int d, int k, int n_r, int n_c, int n_ec, int Qw, int cap, int Sp,
-    int32_t* __restrict__ selected, int2* __restrict__ kept, int32_t* __restrict__ kept_off,
-    float* __restrict__ pos_logit, float* __restrict__ lse_out,
-    float* __restrict__ row_loss, float* __restrict__ logits, uint32_t* status) {
-  extern __shared__ __align__(16) uint8_t sh_raw[];
-  const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t per_warp = size_t(cap) * 8 + kCountBytes;
-  uint8_t* base = sh_raw + per_warp * wid;
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(base);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(base + kCountBytes);
-  int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);  // sorted position in its round
-
-  const int64_t i = int64_t(blockIdx.x) * warps + wid;
-  if (i >= N) return;  // whole warp leaves together; no block-wide barriers below
+__device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint32_t* cnt,
+                                          uint32_t* keys, int32_t* poss, int cap, bool spill) {
+  const T* __restrict__ X = A.X;
+  const T* __restrict__ Y = A.Y;
+  const int32_t* __restrict__ targets = A.targets;
+  const int32_t* __restrict__ py = A.py;
+  const int32_t* __restrict__ invX = A.invX;
+  const int32_t* __restrict__ chunkY = A.chunkY;
+  const int2* __restrict__ list = A.list;
+  const int4* __restrict__ list_count = A.list_count;
+  const float* __restrict__ list_theta = A.list_theta;
+  const int64_t N = A.N, C = A.C;
+  const int d = A.d, k = A.k, n_r = A.n_r, n_c = A.n_c, n_ec = A.n_ec, Qw = A.Qw, Sp = A.Sp;
+  int32_t* __restrict__ selected = A.selected;
+  int2* __restrict__ kept = A.kept;
+  int32_t* __restrict__ kept_off = A.kept_off;
+  float* __restrict__ pos_logit = A.pos_logit;
+  float* __restrict__ lse_out = A.lse_out;
+  float* __restrict__ row_loss = A.row_loss;
+  float* __restrict__ logits = A.logits;
+  uint32_t* status = A.status;
+  const int lane = threadIdx.x & 31;
+  (void)Y;
   const int32_t z = targets[i];
   const bool z_ok = z >= 0 && z < C;
 
@@ -197,8 +230,12 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
       }
     }
   }
-  if (n > cap) {  // more candidates than the buffer holds: keep the first cap, flag the row
-    overflow = true;
+  if (n > cap) {  // more candidates than the buffer holds
+    if (spill) {
+      if (lane == 0) A.spill_rows[atomicAdd(A.spill_count, 1u)] = int32_t(i);
+      return false;
+    }
+    overflow = true;  // keep the first cap, flag the row
     n = cap;
   }
   rb[n_r] = n;
@@ -384,15 +421,54 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(
       if (row_loss) row_loss[i] = lse - lp;
     }
   }
+  return true;
+}
+
+// Fast path: one row per warp, candidates in shared memory (cap per row).
+template <typename T, bool kGrouped>
+__global__ void __launch_bounds__(kThreads) k_merge_tc(const MergeArgs<T> A, int cap) {
+  extern __shared__ __align__(16) uint8_t sh_raw[];
+  const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5;
+  const size_t per_warp = size_t(cap) * 8 + kCountBytes;
+  uint8_t* base = sh_raw + per_warp * wid;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(base);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(base + kCountBytes);
+  int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);
+  const int64_t i = int64_t(blockIdx.x) * warps + wid;
+  if (i >= A.N) return;  // whole warp leaves together; no block-wide barriers follow
+  merge_row<T, kGrouped>(A, i, cnt, keys, poss, cap, true);
+}
+
+// Spilled rows: the warps walk the spill list with their candidates in global scratch
+// (room for every list entry of every round, so nothing is dropped).
+template <typename T, bool kGrouped>
+__global__ void __launch_bounds__(kThreads) k_merge_tc_spill(const MergeArgs<T> A, int cap,
+                                                             uint32_t* scratch) {
+  __shared__ uint32_t sh_cnt[kThreads / 32][kCountBytes / 4];
+  const int wid = threadIdx.x >> 5;
+  const int64_t gw = int64_t(blockIdx.x) * (blockDim.x >> 5) + wid;
+  const int64_t nw = int64_t(gridDim.x) * (blockDim.x >> 5);
+  uint32_t* keys = scratch + gw * 2 * int64_t(cap);
+  int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);
+  const uint32_t n = *reinterpret_cast<volatile uint32_t*>(A.spill_count);
+  for (int64_t w = gw; w < n; w += nw)
+    merge_row<T, kGrouped>(A, A.spill_rows[w], sh_cnt[wid], keys, poss, cap, false);
 }
 
 }  // namespace
 
 int tc_list_capacity(int k);
 
-// Candidates buffered per row: the selection emits about k + 1 + (one histogram bin) per
-// round, so 2k + 64 per round leaves ample room; a row with more is flagged inexact.
-int merge_tc_cap(int n_r, int k) { return n_r * (2 * k + 64); }
+// Candidates buffered per row in shared memory: a round emits about k + 1 + (one histogram
+// bin) entries, so k + k/4 + 64 per round holds nearly every row; the few that bring more
+// go to the spill path.
+int merge_tc_cap(int n_r, int k) { return n_r * (k + k / 4 + 64); }
+// The spill path's buffer: every list entry of every round.
+int merge_tc_spill_cap(int n_r, int k) { return n_r * tc_list_capacity(k); }
+constexpr int kSpillWarps = 1024;
+size_t merge_tc_spill_bytes(int n_r, int k) {
+  return size_t(kSpillWarps) * size_t(merge_tc_spill_cap(n_r, k)) * 8;
+}
 
 size_t merge_tc_warp_bytes(int n_r, int k) {
   return size_t(merge_tc_cap(n_r, k)) * 8 + kCountBytes;
@@ -403,12 +479,41 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
                             const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, int2* kept,
-                            int32_t* kept_off, float* pos_logit, int Sp,
-                            float* lse, float* row_loss, float* logits, uint32_t* status,
-                            cudaStream_t st) {
+                            int32_t* kept_off, float* pos_logit, int Sp, float* lse,
+                            float* row_loss, float* logits, uint32_t* status, int32_t* spill_rows,
+                            void* spill_scratch, cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
-  const int Qw = tc_sublist_capacity(c.k);
+  MergeArgs<T> A{};
+  A.X = X;
+  A.Y = Y;
+  A.targets = targets;
+  A.py = py;
+  A.invX = invX;
+  A.chunkY = chunkY;
+  A.list = list;
+  A.list_count = list_count;
+  A.list_theta = list_theta;
+  A.N = c.N;
+  A.C = c.C;
+  A.d = c.d;
+  A.k = c.k;
+  A.n_r = c.n_r;
+  A.n_c = c.n_c;
+  A.n_ec = c.n_ec;
+  A.Qw = tc_sublist_capacity(c.k);
+  A.Sp = Sp;
+  A.selected = selected;
+  A.kept = kept;
+  A.kept_off = kept_off;
+  A.pos_logit = pos_logit;
+  A.lse_out = lse;
+  A.row_loss = row_loss;
+  A.logits = logits;
+  A.status = status;
+  A.spill_rows = spill_rows;
+  A.spill_count = status + 3;
+  const int cap = merge_tc_cap(c.n_r, c.k);
   const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
   int warps = int((200 * 1024) / per_warp);
   warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
@@ -418,17 +523,20 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
-  kern<<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
-      X, Y, targets, py, invX, chunkY, list, list_count, list_theta, c.N, c.C, c.d, c.k, c.n_r,
-      c.n_c, c.n_ec, Qw, merge_tc_cap(c.n_r, c.k), Sp, selected, kept, kept_off, pos_logit, lse,
-      row_loss, logits, status);
-  count_launches(1);
+  e = cudaMemsetAsync(A.spill_count, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  kern<<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(A, cap);
+  auto spill = grouped ? k_merge_tc_spill<T, true> : k_merge_tc_spill<T, false>;
+  spill<<<kSpillWarps / (kThreads / 32), kThreads, 0, st>>>(
+      A, merge_tc_spill_cap(c.n_r, c.k), static_cast<uint32_t*>(spill_scratch));
+  count_launches(2);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_merge_tc<__nv_bfloat16>(
     const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
     const int32_t*, const int32_t*, const int32_t*, const int2*, const int4*, const float*,
-    int32_t*, int2*, int32_t*, float*, int, float*, float*, float*, uint32_t*, cudaStream_t);
+    int32_t*, int2*, int32_t*, float*, int, float*, float*, float*, uint32_t*, int32_t*, void*,
+    cudaStream_t);
 
 }  // namespace rece

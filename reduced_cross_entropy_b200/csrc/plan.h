@@ -63,7 +63,8 @@ struct Layout {
   size_t sort_scratch = 0;
   size_t list_score = 0, list_item = 0, row_loss_tmp = 0;
   // tensor-core path (bf16 mode): sorted row copies, inverse orders, candidate lists
-  size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0;
+  size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0,
+         spill_rows = 0, spill_scratch = 0;
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_key_b = 0,

@@ -96,6 +96,8 @@ void build_layout(rece_plan_s& p) {
     L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
     L.tc_count = take(sizeof(int4) * c.n_r * c.N);
     L.tc_theta = take(sizeof(float) * c.n_r * c.N);
+    L.spill_rows = take(sizeof(int32_t) * size_t(c.N));
+    L.spill_scratch = take(merge_tc_spill_bytes(c.n_r, c.k));
   } else {
     L.list_score = take(sizeof(float) * size_t(c.n_r) * c.N * c.k);
     L.list_item = take(sizeof(int32_t) * size_t(c.n_r) * c.N * c.k);
@@ -378,7 +380,9 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
                               plan->tc_dx ? reinterpret_cast<int2*>(ws + L.kept) : nullptr,
                               plan->tc_dx ? reinterpret_cast<int32_t*>(ws + L.kept_off) : nullptr,
                               plan->tc_dx ? reinterpret_cast<float*>(ws + L.pos_logit) : nullptr,
-                              plan->kept_slices + 1, lse, rl, logits, status, st),
+                              plan->kept_slices + 1, lse, rl, logits, status,
+                              reinterpret_cast<int32_t*>(ws + L.spill_rows), ws + L.spill_scratch,
+                              st),
               "merge/loss (tcgen05 lists)");
   } else {
     const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);

@@ -50,16 +50,19 @@ cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Y
 // (round r, sorted row p): kept [n_r][N][k] = (sorted position, softmax probability as
 // bf16 hi | lo << 16), kept_off [n_r][N][Sp] = slice starts of the row's window (entry S
 // = the count); and pos_logit [N], each row's positive logit.
+// Rows with more candidates than the fast path's shared buffer go through a spill list
+// (spill_rows [N]) to a second launch with global scratch (merge_tc_spill_bytes).
 size_t merge_tc_warp_bytes(int n_r, int k);
+size_t merge_tc_spill_bytes(int n_r, int k);
 constexpr int kMaxKeptSlices = 512;  // slices of one window the merge can group by
 template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
                             const int32_t* py, const int32_t* invX, const int32_t* chunkY,
                             const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, int2* kept,
-                            int32_t* kept_off, float* pos_logit, int Sp,
-                            float* lse, float* row_loss, float* logits, uint32_t* status,
-                            cudaStream_t st);
+                            int32_t* kept_off, float* pos_logit, int Sp, float* lse,
+                            float* row_loss, float* logits, uint32_t* status, int32_t* spill_rows,
+                            void* spill_scratch, cudaStream_t st);
 
 // dX of step 6 on tensor cores (see bwd_tc.cu): written, not accumulated.  Needs the
 // grouped merge outputs (kept, kept_off, pos_logit) and the d-major copy YsT.

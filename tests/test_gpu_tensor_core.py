@@ -117,6 +117,7 @@ def test_tc_path_exact_on_integer_inputs(d, n_c, n_ec, n_r, k):
     g = run_gpu(w, X, Y, t, B, flags=0, dloss=0.5)
     o = run_oracle(w, X, Y, t, B, dloss=0.5)
     assert g["status"] == 0
+    print("rows spilled to the merge's global-memory path:", int(g["words"][3]))
     np.testing.assert_array_equal(np.sort(g["selected"], axis=1), np.sort(o["selected"], axis=1))
     assert abs(g["loss"] - o["loss"]) <= 1e-4 * abs(o["loss"])
     assert max_rel(g["row_loss"], o["row_loss"]) <= 1e-4
@@ -143,3 +144,27 @@ def test_backward_past_the_in_cache_pair_size():
     oX, oY = oracle.rece_grad(X, Y, t, g["selected"], lse, 0.5)
     assert max_rel(g["dX"], oX) <= 1e-3
     assert max_rel(g["dY"], oY) <= 1e-3
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_merge_spill_path_on_tied_scores(d):
+    """Every score equal: each round emits its whole window (one histogram bin), more
+    candidates than the merge's shared-memory buffer, so the rows go through the spill
+    path (global-memory buffers).  Ties go to the lower item id: the oracle's sets."""
+    w = synth.Workload("tied", N=300, C=1000, d=d, dtype="bf16", n_b=8, n_c=6, n_ec=1,
+                       n_r=2, k=100)
+    X = np.full((w.N, d), 0.125, np.float32)
+    Y = np.full((w.C, d), 0.25, np.float32)
+    t = np.random.default_rng(5).integers(0, w.C, w.N).astype(np.int32)
+    B = synth.projections(5, 0, w.n_r, w.n_b, d, "bf16")
+    g = run_gpu(w, X, Y, t, B, flags=0, dloss=1.0)
+    o = run_oracle(w, X, Y, t, B, dloss=1.0)
+    assert g["status"] == 0
+    assert g["words"][3] > 0  # rows that took the spill path
+    np.testing.assert_array_equal(np.sort(g["selected"], axis=1), np.sort(o["selected"], axis=1))
+    assert abs(g["loss"] - o["loss"]) <= 1e-4 * abs(o["loss"])
+    # with every y equal, dX_i = y * sum_j g_ij vanishes (the softmax sums to 1): measure
+    # it against the size of its terms, dloss / N * |y|
+    term = 1.0 / w.N * float(np.abs(Y).max())
+    assert np.abs(g["dX"] - o["dX"]).max() <= 1e-4 * term
+    assert max_rel(g["dY"], o["dY"]) <= 1e-4
