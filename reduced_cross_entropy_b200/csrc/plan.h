@@ -64,7 +64,7 @@ struct Layout {
   size_t list_score = 0, list_item = 0, row_loss_tmp = 0;
   // tensor-core path (bf16 mode): sorted row copies, inverse orders, candidate lists
   size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0,
-         spill_rows = 0, spill_scratch = 0;
+         spill_rows = 0, spill_scratch = 0, scores = 0;
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_key_b = 0,
@@ -93,6 +93,8 @@ struct rece_plan_s {
   bool carry_g;         // the pair sort carries g (its array would not stay in L2)
   bool use_tc;          // bf16 mode on the tcgen05 kernels
   bool tc_dx;           // ... and dX of the backward on them too
+  bool tc_scores;       // ... with the window scores computed once and stored (large d)
+  int64_t score_width;  // columns of the stored scores per row (longest union, padded)
   int32_t kept_slices;  // most 64-position slices one window touches
   int64_t ld_c;         // row pitch (elements) of the d-major copy of Y: C rounded up to 8
   rece::Layout lay;

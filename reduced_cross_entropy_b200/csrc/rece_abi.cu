@@ -96,6 +96,7 @@ void build_layout(rece_plan_s& p) {
     L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
     L.tc_count = take(sizeof(int4) * c.n_r * c.N);
     L.tc_theta = take(sizeof(float) * c.n_r * c.N);
+    if (p.tc_scores) L.scores = take(sizeof(float) * size_t(c.n_r) * c.N * p.score_width);
     L.spill_rows = take(sizeof(int32_t) * size_t(c.N));
     L.spill_scratch = take(merge_tc_spill_bytes(c.n_r, c.k));
   } else {
@@ -220,6 +221,10 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   // dX on the tensor cores where gathering catalogue rows is the slow way: large d, or a
   // sorted catalogue that does not fit in half of L2; the merge groups each row's kept
   // entries by slice of its window for it
+  // at large d the window scores are computed once and stored (a d-deep dot product per
+  // score outweighs writing and reading it back)
+  p->tc_scores = p->use_tc && c.d >= 1024;
+  p->score_width = p->tc_scores ? scores_tc_width(*p) : 0;
   p->tc_dx = p->use_tc && p->kept_slices <= kMaxKeptSlices &&
              (c.d >= 256 || 2.0 * double(c.C) * c.d > 64.0 * 1024 * 1024);
   if (p->use_tc && merge_tc_warp_bytes(c.n_r, c.k) > 200 * 1024) {
@@ -369,8 +374,14 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     int4* cnt = reinterpret_cast<int4*>(ws + L.tc_count);
     float* theta = reinterpret_cast<float*>(ws + L.tc_theta);
     stage_mark(*plan, RECE_STAGE_SELECT, 0, st);
-    RECE_CUDA(launch_select_tc(*plan, ws + L.xs, ws + L.ys, list, cnt, theta, status, st),
-              "select (tcgen05)");
+    if (plan->tc_scores)
+      RECE_CUDA(launch_scores_select_tc(*plan, ws + L.xs, ws + L.ys,
+                                        reinterpret_cast<float*>(ws + L.scores), list, cnt, theta,
+                                        status, st),
+                "scores + select (tcgen05)");
+    else
+      RECE_CUDA(launch_select_tc(*plan, ws + L.xs, ws + L.ys, list, cnt, theta, status, st),
+                "select (tcgen05)");
     stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
     stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
     RECE_CUDA(launch_merge_tc(*plan, Xb, Yb, targets, py,

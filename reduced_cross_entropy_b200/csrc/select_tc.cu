@@ -36,11 +36,13 @@
 #include "plan.h"
 #include "sm100.cuh"
 #include "tc.h"
+#include "tc_bins.cuh"
 
 namespace rece {
 namespace {
 
 using namespace sm100;
+using namespace tcsel;
 
 constexpr int kStages = 4;
 constexpr int kPasses = 3;
@@ -90,37 +92,6 @@ struct ItemGeom {
   int nt;       // kBN-wide tiles covering it
 };
 
-// Distance bins of pass 2.  The anchor A is the bit pattern of a value 16 bins (two
-// binades) beyond the pass 1 max m, away from zero, so that scores a little above m --
-// pass 1 may have looked at a sample only -- still get bins of their own.  For m >= 0 the
-// distance of a score s is A - bits(s), for m < 0 it is bits(s) - A: in both cases
-// key(anchor) - key(s) with key the order-preserving integer image of an fp32 value, as
-// long as s lies between zero and the anchor.  Bin = min(distance >> 20, 255): 8 bins per
-// binade of |s|.  Any other score (beyond the anchor, or on the far side of zero) wraps
-// to a huge distance, normally the open last bin; that only misplaces the cut, since
-// the emission itself compares values and the exactness check below stays sound.
-struct BinMap {
-  uint32_t sig, off, anchor;
-};
-__device__ __forceinline__ BinMap bin_map(float m) {
-  constexpr uint32_t H = uint32_t(kHeadBins) << 20;
-  const uint32_t bm = __float_as_uint(m);
-  if (!(bm & 0x80000000u)) {
-    const uint32_t A = bm > 0x7F7FFFFFu - H ? 0x7F7FFFFFu : bm + H;
-    return BinMap{0xFFFFFFFFu, A, A};
-  }
-  const uint32_t A = bm - H < 0x80000000u ? 0x80000000u : bm - H;
-  return BinMap{1u, 0u - A, A};
-}
-
-// The fp32 threshold t of the cut "distance < L" (L = (b* + 1) << 20): a score between
-// zero and the anchor has distance < L exactly when s >= t.  -inf when every score passes.
-__device__ __forceinline__ float cut_threshold(const BinMap& b, uint32_t L) {
-  if (b.sig != 1u) return b.anchor >= L ? __uint_as_float(b.anchor - L + 1u) : 0.0f;
-  const uint64_t tb = uint64_t(b.anchor) + L - 1u;  // L - 1 ulps beyond the anchor
-  return tb < 0xFF800000ull ? __uint_as_float(uint32_t(tb)) : -INFINITY;
-}
-
 // One more count in bin b of the row whose column of words starts at shared address hcol.
 __device__ __forceinline__ void bin_add(uint32_t hcol, uint32_t b) {
   const uint32_t addr = hcol + (b >> 1) * (kBM * 4);
@@ -128,13 +99,6 @@ __device__ __forceinline__ void bin_add(uint32_t hcol, uint32_t b) {
   asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(inc));
 }
 
-// The largest fp32 value below t (t finite or +0/-0): every score < t is <= it.
-__device__ __forceinline__ float value_below(float t) {
-  const uint32_t b = __float_as_uint(t);
-  if (t > 0.0f) return __uint_as_float(b - 1u);
-  if (t == 0.0f) return __uint_as_float(0x80000001u);
-  return __uint_as_float(b + 1u);
-}
 
 __device__ __forceinline__ int64_t chunk_of(int64_t p, int64_t M, int n_c) {
   return (p * n_c) / M;
@@ -301,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
           mx = s.part_mx[0][row_local];
 #pragma unroll
           for (int w = 1; w < kAcc; ++w) mx = fmaxf(mx, s.part_mx[w][row_local]);
-          bmap = bin_map(mx);
+          bmap = bin_map(mx, uint32_t(kHeadBins));
         } else if (pass == 2) {
           named_barrier(1, kEpiThreads);  // every histogram increment has landed
           if (histo) {  // else thr stays -inf: emit the whole window

@@ -44,6 +44,13 @@ cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Y
                              int4* list_count, float* list_theta, uint32_t* status,
                              cudaStream_t st);
 
+// Steps 3-4 for large d (see scores_tc.cu): window scores once into S [n_r][N][width],
+// then the exact per-row selection into the same lists as launch_select_tc.
+int64_t scores_tc_width(const rece_plan_s& p);
+cudaError_t launch_scores_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys,
+                                    float* S, int2* list, int4* list_count, float* list_theta,
+                                    uint32_t* status, cudaStream_t st);
+
 // K4 for the tensor-core lists: merge, select, loss, exactness check.  The kept entries
 // go out by round and 64-position slice of the round's sorted catalogue: items
 // (selected [N][k]) and logits ([N][k+1], or NULL), and for the backward, indexed by

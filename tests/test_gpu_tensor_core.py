@@ -68,6 +68,8 @@ TC_CASES = {
     "lm_scaled": synth.WORKLOADS["lm"].scaled(512, 4000, n_c=4, n_b=64, k=128, d=256),
     "very_large_scaled": synth.WORKLOADS["very_large"].scaled(4096, 40000, n_c=64, n_b=256,
                                                               k=256),
+    # d >= 1024: window scores computed once and stored, then selected row by row
+    "lm_scaled_d1024": synth.WORKLOADS["lm"].scaled(512, 4000, n_c=4, n_b=64, k=128, d=1024),
 }
 
 
@@ -104,11 +106,13 @@ def test_tc_path_recall_and_loss(name):
 
 
 @pytest.mark.parametrize("d,n_c,n_ec,n_r,k", [(64, 8, 1, 2, 64), (64, 16, 0, 1, 200),
-                                              (128, 6, 2, 3, 100), (256, 8, 1, 2, 96)])
+                                              (128, 6, 2, 3, 100), (256, 8, 1, 2, 96),
+                                              (1024, 8, 1, 2, 96)])
 def test_tc_path_exact_on_integer_inputs(d, n_c, n_ec, n_r, k):
     """Integer-valued inputs: every score is exact on the tensor cores and ties are
     everywhere, so the kept sets (ties to the lower item id) must be the oracle's.  At
-    d = 256 dX also comes from the tensor cores (band products of the coefficients)."""
+    d >= 256 dX also comes from the tensor cores (band products of the coefficients); at
+    d = 1024 the window scores are stored once and selected row by row."""
     w = synth.Workload("int", N=1000, C=5003, d=d, dtype="bf16", n_b=16, n_c=n_c, n_ec=n_ec,
                        n_r=n_r, k=k)
     X, Y, t = synth.integer_inputs(w.N, w.C, d, lo=-2, hi=2, seed=d + k, scale=0.125)
