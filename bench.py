@@ -97,14 +97,13 @@ def stage_work(w):
     }
 
 
-def uses_tensor_cores(w, flags):
-    """bf16 mode without RECE_FLAG_FMA_SCORES and d a multiple of 64: tcgen05 kernels."""
-    return w.dtype == "bf16" and not (flags & 1) and w.d % 64 == 0
-
-
-def stage_bound(stage, w, flags):
+def stage_bound(stage, paths):
+    """The roofline a stage is held to, given the plan's kernels (rece_plan_paths)."""
+    from reduced_cross_entropy_b200 import _lib
     if stage in ("bucketize", "select"):
-        return "tensor" if uses_tensor_cores(w, flags) else "alu"
+        return "tensor" if paths & _lib.PATH_TENSOR_CORES else "alu"
+    if stage == "bwd_rows" and paths & _lib.PATH_DX_TENSORS:
+        return "tensor"
     return "hbm"
 
 
@@ -113,25 +112,37 @@ KERNEL_SOURCES = {
     "merge_loss": ["loss.cu"], "mean": ["loss.cu"], "bwd_rows": ["backward.cu"],
     "bwd_sort": ["sort.cu"], "bwd_items": ["backward.cu"],
 }
-KERNEL_SOURCES_TC = dict(KERNEL_SOURCES, bucketize=["bucketize_tc.cu", "permute.cu"],
-                         select=["select_tc.cu", "sm100.cuh"], merge_loss=["merge_tc.cu"])
 
 
-def source_hash(stage, tc):
+def kernel_sources(stage, paths):
+    from reduced_cross_entropy_b200 import _lib
+    src = dict(KERNEL_SOURCES)
+    if paths & _lib.PATH_TENSOR_CORES:
+        src.update(bucketize=["bucketize_tc.cu", "permute.cu"],
+                   select=["select_tc.cu", "sm100.cuh", "tc_bins.cuh"],
+                   merge_loss=["merge_tc.cu"])
+    if paths & _lib.PATH_STORED_SCORES:
+        src["select"] = ["scores_tc.cu", "sm100.cuh", "tc_bins.cuh"]
+    if paths & _lib.PATH_DX_TENSORS:
+        src["bwd_rows"] = ["backward.cu", "bwd_tc.cu", "sm100.cuh"]
+    return src[stage]
+
+
+def source_hash(stage, paths):
     h = hashlib.sha256()
-    for f in (KERNEL_SOURCES_TC if tc else KERNEL_SOURCES)[stage]:
+    for f in kernel_sources(stage, paths):
         h.update(open(os.path.join(ROOT, "reduced_cross_entropy_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(stage, workload, tc):
+def recorded_traffic(stage, workload, paths):
     """DRAM bytes per step of this stage (all its launches) from a committed ncu capture,
-    if the kernel source is unchanged since (else None)."""
+    if the kernel sources are unchanged since (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(f"{stage}@{workload}{'@tc' if tc else ''}")
-    if not d or d.get("source_sha") != source_hash(stage, tc):
+    d = json.load(open(p)).get(f"{stage}@{workload}@paths{paths}")
+    if not d or d.get("source_sha") != source_hash(stage, paths):
         return None
     return d.get("dram_bytes_per_step")
 
@@ -388,10 +399,10 @@ def main():
     # roofline of every stage, the dominant one reported as the line's roofline
     peaks = load_peaks()
     work = stage_work(w)
-    tc = uses_tensor_cores(w, args.flags)
+    paths = plan.paths
 
     def stage_roofline(name):
-        bound = stage_bound(name, w, args.flags)
+        bound = stage_bound(name, paths)
         flops, bytes_ = work[name]
         sec = stage_ms[name] / 1000.0
         if bound == "hbm":
@@ -405,7 +416,7 @@ def main():
                 "unit": unit, "frac": achieved / peak,
                 "peak_source": peaks["source"] if bound != "alu" else
                 "derived: 148 SM x 128 FP32 lanes x 2 x sm_max_mhz",
-                "traffic": recorded_traffic(name, w.name, tc),
+                "traffic": recorded_traffic(name, w.name, paths),
                 "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
 
     dom = max(stage_ms, key=stage_ms.get)
@@ -448,8 +459,11 @@ def main():
                        "overflowed_rows_per_step": overflow_rows,
                        "merge_spilled_rows_per_step": spilled_rows,
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "scores": "tcgen05" if uses_tensor_cores(w, args.flags)
-                       else "fmaf CUDA cores"},
+                       "scores": ("tcgen05" + (", stored" if paths & _lib.PATH_STORED_SCORES
+                                                 else ", recomputed per pass")
+                                  if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),
+                       "dX": "tcgen05 band products" if paths & _lib.PATH_DX_TENSORS
+                       else "gathered rows"},
             "roofline": roofline, "stages_ms": stage_ms, "stages_roofline_frac": stage_fracs,
             "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk.summary()}

@@ -122,6 +122,19 @@ RECE_API void rece_plan_destroy(rece_plan_t plan);
 RECE_API rece_status_t rece_plan_workspace_size(rece_plan_t plan, size_t* bytes);
 RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspace_layout_t* layout);
 
+/* Which kernels a plan runs (host-side; no device work).  *paths receives the OR of:
+ *   RECE_PATH_TENSOR_CORES  bf16 mode on tcgen05: bucketing and the window scores with
+ *                           their selection (else the fmaf kernels);
+ *   RECE_PATH_DX_TENSORS    dX of the backward as tcgen05 band products (large d or a
+ *                           catalogue beyond half of L2; else gathered rows);
+ *   RECE_PATH_STORED_SCORES window scores computed once and stored, then selected row by
+ *                           row (d >= 1024; else recomputed in the fused selection).
+ * RECE_ERR_INVALID_ARG for a NULL argument. */
+#define RECE_PATH_TENSOR_CORES 0x1u
+#define RECE_PATH_DX_TENSORS 0x2u
+#define RECE_PATH_STORED_SCORES 0x4u
+RECE_API rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths);
+
 /* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].
  *   B  device, [n_r][n_b][d] random vectors (one set per round; the caller draws them,
  *      N(0,1), afresh for every call as the paper does)

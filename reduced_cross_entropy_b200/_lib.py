@@ -19,6 +19,9 @@ FLAG_FMA_SCORES = 0x1
 DEVICE_BAD_TARGET = 0x1
 DEVICE_TIMEOUT = 0x2
 DEVICE_INEXACT = 0x4
+PATH_TENSOR_CORES = 0x1
+PATH_DX_TENSORS = 0x2
+PATH_STORED_SCORES = 0x4
 
 # every symbol include/rece.h declares
 EXPORTS = (
@@ -27,6 +30,7 @@ EXPORTS = (
     "rece_full_ce_workspace_size", "rece_full_ce_fwd", "rece_full_ce_bwd",
     "rece_get_device_status", "rece_status_string", "rece_last_error_string",
     "rece_plan_set_stage_events", "rece_kernel_launch_count", "rece_bucket_sort_static",
+    "rece_plan_paths",
 )
 STAGES = ("bucketize", "sort", "select", "merge_loss", "mean", "bwd_rows", "bwd_sort",
           "bwd_items")
@@ -72,6 +76,7 @@ def lib():
         "rece_plan_destroy": ([vp], None),
         "rece_plan_workspace_size": ([vp, ctypes.POINTER(sz)], st),
         "rece_plan_workspace_layout": ([vp, ctypes.POINTER(WorkspaceLayout)], st),
+        "rece_plan_paths": ([vp, ctypes.POINTER(ctypes.c_uint32)], st),
         "rece_bucketize_sort": ([vp, vp, vp, vp, vp, sz, vp], st),
         "rece_loss_fwd": ([vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp, vp], st),
         "rece_loss_bwd": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp], st),

@@ -271,6 +271,14 @@ rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspace_layout
   return RECE_OK;
 }
 
+rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
+  if (!plan || !paths) return fail(RECE_ERR_INVALID_ARG, "NULL argument");
+  *paths = (plan->use_tc ? RECE_PATH_TENSOR_CORES : 0u) |
+           (plan->tc_dx ? RECE_PATH_DX_TENSORS : 0u) |
+           (plan->tc_scores ? RECE_PATH_STORED_SCORES : 0u);
+  return RECE_OK;
+}
+
 rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X, const void* Y,
                                   void* workspace, size_t workspace_bytes, void* stream) {
   rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);

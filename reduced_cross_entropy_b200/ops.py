@@ -69,6 +69,13 @@ class Plan:
     def dtype(self):
         return _DTYPES[self.mode]
 
+    @property
+    def paths(self) -> int:
+        """OR of _lib.PATH_* flags: which kernels this plan runs."""
+        v = ctypes.c_uint32()
+        _lib.check(_lib.lib().rece_plan_paths(self._h, ctypes.byref(v)), "rece_plan_paths")
+        return int(v.value)
+
     def __getattr__(self, name):
         if name in ("N", "C", "d", "n_b", "n_c", "n_ec", "n_r", "k", "flags"):
             return getattr(self.cfg, name)
