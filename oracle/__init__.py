@@ -13,6 +13,8 @@ upcast) and follows the definitions cited in ``rece_oracle.c``:
                        de-duplicated, the k best by (score desc, item asc) (SCE abstract)
 * ``rece_loss`` / ``rece_grad``       -- Algorithm 1's loss, equation (4) on the subset
 * ``full_ce_loss`` / ``full_ce_grad`` -- equations (3) and (4) over the whole catalogue
+* ``sampled_loss`` / ``sampled_grad`` -- the sampled baselines of section 2: CE- (eq. 2,
+                       kind 0) and BCE+ (eq. 1, kind 1) over given negatives
 * ``rece_forward``  -- the whole forward path, steps 1 to 5, given the random vectors B
 """
 import ctypes
@@ -56,6 +58,12 @@ def _load():
         lib.oracle_full_ce_grad.argtypes = [f32p, f32p, i32p, i64, i64, i32, f64p,
                                             ctypes.c_double, f64p, f64p]
         lib.oracle_full_ce_grad.restype = None
+        lib.oracle_sampled_loss.argtypes = [i32, f32p, f32p, i32p, i64, i32, i32, i32p, f64p,
+                                            f64p, f64p]
+        lib.oracle_sampled_loss.restype = None
+        lib.oracle_sampled_grad.argtypes = [i32, f32p, f32p, i32p, i64, i64, i32, i32, i32p,
+                                            f64p, ctypes.c_double, f64p, f64p]
+        lib.oracle_sampled_grad.restype = None
         lib.oracle_dot_f32.argtypes = [f32p, f32p, i32]
         lib.oracle_dot_f32.restype = ctypes.c_float
         lib.oracle_num_threads.argtypes = []
@@ -167,6 +175,39 @@ def full_ce_grad(X, Y, target, lse, dloss=1.0):
     dY = np.empty((C, d), np.float64)
     _load().oracle_full_ce_grad(X, Y, target, N, C, d, np.ascontiguousarray(lse, np.float64),
                                 float(dloss), dX, dY)
+    return dX, dY
+
+
+SAMPLED_CE_MINUS = 0  # equation (2)
+SAMPLED_BCE_PLUS = 1  # equation (1)
+
+
+def sampled_loss(kind, X, Y, target, negatives):
+    """Sampled baseline loss (section 2, eq. 2 for kind 0, eq. 1 for kind 1) over the
+    given negatives [N, n] (ids < 0 are padding).  Returns (loss, row_loss, lse); lse
+    is meaningful for CE- only."""
+    X, Y, target, neg = _f32(X), _f32(Y), _i32(target), _i32(negatives)
+    N, d = X.shape
+    n = neg.shape[1] if neg.ndim == 2 else 0
+    neg = neg.reshape(N, n) if N * n else np.zeros((max(N, 1), max(n, 1)), np.int32)
+    row = np.empty(N, np.float64)
+    lse = np.zeros(N, np.float64)
+    loss = np.zeros(1, np.float64)
+    _load().oracle_sampled_loss(int(kind), X, Y, target, N, d, n, neg, row, lse, loss)
+    return float(loss[0]), row, lse
+
+
+def sampled_grad(kind, X, Y, target, negatives, lse, dloss=1.0):
+    """(dX, dY) of the sampled baseline, the negatives held constant (fp64)."""
+    X, Y, target, neg = _f32(X), _f32(Y), _i32(target), _i32(negatives)
+    N, d = X.shape
+    C = Y.shape[0]
+    n = neg.shape[1] if neg.ndim == 2 else 0
+    neg = neg.reshape(N, n) if N * n else np.zeros((max(N, 1), max(n, 1)), np.int32)
+    dX = np.empty((N, d), np.float64)
+    dY = np.empty((C, d), np.float64)
+    _load().oracle_sampled_grad(int(kind), X, Y, target, N, C, d, n, neg,
+                                np.ascontiguousarray(lse, np.float64), float(dloss), dX, dY)
     return dX, dY
 
 

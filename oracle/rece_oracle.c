@@ -11,6 +11,8 @@
  *           Recommenders", section 3 (Reduced Cross-Entropy): equations (3) and (4),
  *           Algorithm 1, and the paragraph before Algorithm 1 (rounds, duplicate pairs,
  *           neighbouring chunks).
+ *           Section 2 (Related Work): equations (1) BCE+ and (2) CE-, the sampled
+ *           baselines.
  *   [SCE]   "Scalable Cross-Entropy Loss for Sequential Recommendations with Large
  *           Item Catalogs", abstract (softmax approximated over a subset found by
  *           maximum inner product search, i.e. the top-k negatives per row).
@@ -296,6 +298,79 @@ void oracle_full_ce_grad(const float* X, const float* Y, const int32_t* target, 
       const float* y = Y + j * d;
       double g = (exp(dot_f64(x, y, d) - lse[i]) - (j == target[i] ? 1.0 : 0.0)) * scale;
       double* dy = dY + j * d;
+      for (int32_t t = 0; t < d; ++t) {
+        dx[t] += g * (double)y[t];
+        dy[t] += g * (double)x[t];
+      }
+    }
+  }
+}
+
+/* log(1 + exp(u)) without overflow: for u > 0 it is u + log(1 + exp(-u)). */
+static double softplus(double u) { return u > 0.0 ? u + log1p(exp(-u)) : log1p(exp(u)); }
+
+/* Sampled baselines, [RECE] section 2 (Related Work), equations (1) and (2).  Row i has
+ * the positive z_i and n sampled negatives neg[i][0..n) (ids < 0 are padding and take no
+ * part; a sample equal to the positive is a negative like any other, as the sums are
+ * written):
+ *   kind 0, CE-  (2):  lse_i  = log(exp(l+) + sum_j exp(l_ij)),  loss_i = lse_i - l+
+ *   kind 1, BCE+ (1):  loss_i = -log sigmoid(l+) - sum_j log(1 - sigmoid(l_ij))
+ *                             = softplus(-l+) + sum_j softplus(l_ij)
+ * with l = <x_i, y_j> in fp64; L = mean_i loss_i.  lse is written for kind 0 only. */
+void oracle_sampled_loss(int32_t kind, const float* X, const float* Y, const int32_t* target,
+                         int64_t N, int32_t d, int32_t n, const int32_t* neg,
+                         double* row_loss, double* lse, double* loss) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    const int32_t* ng = neg + i * (int64_t)n;
+    double lp = dot_f64(x, Y + (int64_t)target[i] * d, d);
+    if (kind == 0) {
+      double m = lp;
+      for (int32_t a = 0; a < n; ++a) {
+        if (ng[a] < 0) continue;
+        double l = dot_f64(x, Y + (int64_t)ng[a] * d, d);
+        if (l > m) m = l;
+      }
+      double s = exp(lp - m);
+      for (int32_t a = 0; a < n; ++a)
+        if (ng[a] >= 0) s += exp(dot_f64(x, Y + (int64_t)ng[a] * d, d) - m);
+      lse[i] = m + log(s);
+      row_loss[i] = lse[i] - lp;
+    } else {
+      double r = softplus(-lp);
+      for (int32_t a = 0; a < n; ++a)
+        if (ng[a] >= 0) r += softplus(dot_f64(x, Y + (int64_t)ng[a] * d, d));
+      row_loss[i] = r;
+    }
+  }
+  double total = 0.0;
+  for (int64_t i = 0; i < N; ++i) total += row_loss[i];
+  *loss = N > 0 ? total / (double)N : 0.0;
+}
+
+/* Gradients of equations (1) and (2), the sampled negatives held constant:
+ *   CE-:   g_i+ = (p_i+ - 1) dloss/N,      g_ij = p_ij dloss/N,   p = exp(l - lse_i)
+ *   BCE+:  g_i+ = (sigmoid(l+) - 1) dloss/N,  g_ij = sigmoid(l_ij) dloss/N
+ *   dX_i = g_i+ y_{z_i} + sum_j g_ij y_j,   dY_j = sum over the pairs naming j of g x_i
+ * (a negative sampled twice contributes twice), in fp64. */
+void oracle_sampled_grad(int32_t kind, const float* X, const float* Y, const int32_t* target,
+                         int64_t N, int64_t C, int32_t d, int32_t n, const int32_t* neg,
+                         const double* lse, double dloss, double* dX, double* dY) {
+  double scale = N > 0 ? dloss / (double)N : 0.0;
+  memset(dY, 0, sizeof(double) * (size_t)C * (size_t)d);
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    double* dx = dX + i * (int64_t)d;
+    for (int32_t t = 0; t < d; ++t) dx[t] = 0.0;
+    for (int32_t a = -1; a < n; ++a) {
+      int32_t j = a < 0 ? target[i] : neg[i * (int64_t)n + a];
+      if (j < 0) continue;
+      const float* y = Y + (int64_t)j * d;
+      double l = dot_f64(x, y, d);
+      double p = kind == 0 ? exp(l - lse[i]) : 1.0 / (1.0 + exp(-l));
+      double g = (a < 0 ? p - 1.0 : p) * scale;
+      double* dy = dY + (int64_t)j * d;
       for (int32_t t = 0; t < d; ++t) {
         dx[t] += g * (double)y[t];
         dy[t] += g * (double)x[t];

@@ -325,6 +325,138 @@ def test_full_ce_grad_matches_torch_autograd():
     assert rel_err(dY, Yt.grad.numpy()) < 1e-12
 
 
+# --------------------------------------------------------------------------- sampled baselines
+def _sampled_case(N=24, C=60, d=7, n=9, seed=5, pad=True):
+    X, Y, z, _ = _random_case(N=N, C=C, d=d)
+    rng = np.random.default_rng(seed)
+    neg = rng.integers(0, C, size=(N, n)).astype(np.int32)
+    neg[0, :] = z[0]                      # the positive sampled as a negative
+    neg[1, 1] = neg[1, 0]                 # a negative drawn twice
+    if pad:
+        neg[2, -3:] = -1                  # padding
+    return X, Y, z, neg
+
+
+def _torch_sampled_rows(kind, X, Y, z, neg):
+    """Row losses from torch's own loss routines on the [positive, negatives] logits."""
+    Xt, Yt = torch.from_numpy(X).double(), torch.from_numpy(Y).double()
+    rows = []
+    for i in range(len(X)):
+        js = [int(z[i])] + [int(j) for j in neg[i] if j >= 0]
+        lg = Xt[i] @ Yt[js].T
+        if kind == oracle.SAMPLED_CE_MINUS:
+            rows.append(torch.nn.functional.cross_entropy(lg[None], torch.zeros(1).long()))
+        else:
+            lab = torch.zeros_like(lg)
+            lab[0] = 1.0
+            rows.append(torch.nn.functional.binary_cross_entropy_with_logits(
+                lg, lab, reduction="sum"))
+    return torch.stack(rows) if rows else torch.zeros(0, dtype=torch.float64)
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_sampled_loss_matches_torch_losses(kind):
+    """Equation (2) is torch's cross-entropy over [l+, l_neg...] with class 0; equation
+    (1) is torch's BCE-with-logits with label 1 on l+ and 0 on every sampled negative."""
+    X, Y, z, neg = _sampled_case()
+    loss, row, lse = oracle.sampled_loss(kind, X, Y, z, neg)
+    ref = _torch_sampled_rows(kind, X, Y, z, neg).numpy()
+    np.testing.assert_allclose(row, ref, rtol=1e-12, atol=1e-12)
+    assert loss == pytest.approx(float(ref.mean()), rel=1e-12)
+
+
+def test_bce_plus_far_tails_stay_finite():
+    """Logits of +-800: -log sigmoid(800) ~ 0 and -log(1 - sigmoid(800)) = 800 + ~0,
+    where a naive log(1 + exp(l)) overflows."""
+    X = np.array([[1.0]], np.float32)
+    Y = np.array([[800.0], [-800.0]], np.float32)
+    loss, row, _ = oracle.sampled_loss(1, X, Y, np.array([0], np.int32),
+                                       np.array([[0, 1, 0]], np.int32))
+    assert row[0] == pytest.approx(2 * 800.0, rel=1e-15)
+
+
+def test_ce_minus_over_the_rest_of_the_catalogue_is_full_ce():
+    """Every item but the positive sampled once: equation (2) is equation (3)."""
+    X, Y, z, _ = _random_case(N=20, C=40, d=6)
+    neg = np.array([[j for j in range(len(Y)) if j != z[i]] for i in range(len(X))],
+                   np.int32)
+    loss, row, lse = oracle.sampled_loss(0, X, Y, z, neg)
+    floss, frow, flse = oracle.full_ce_loss(X, Y, z)
+    np.testing.assert_allclose(row, frow, rtol=1e-12)
+    np.testing.assert_allclose(lse, flse, rtol=1e-13)
+    dX, dY = oracle.sampled_grad(0, X, Y, z, neg, lse, 0.9)
+    fX, fY = oracle.full_ce_grad(X, Y, z, flse, 0.9)
+    assert rel_err(dX, fX) < 1e-12 and rel_err(dY, fY) < 1e-12
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_sampled_grad_matches_torch_autograd(kind):
+    X, Y, z, neg = _sampled_case(N=12, C=30, d=5, n=6)
+    _, _, lse = oracle.sampled_loss(kind, X, Y, z, neg)
+    dX, dY = oracle.sampled_grad(kind, X, Y, z, neg, lse, 1.7)
+    Xt = torch.from_numpy(X).double().requires_grad_()
+    Yt = torch.from_numpy(Y).double().requires_grad_()
+    rows = []
+    for i in range(len(X)):
+        js = [int(z[i])] + [int(j) for j in neg[i] if j >= 0]
+        lg = Xt[i] @ Yt[js].T
+        if kind == 0:
+            rows.append(torch.logsumexp(lg, 0) - lg[0])
+        else:
+            rows.append(-torch.nn.functional.logsigmoid(lg[0])
+                        - torch.nn.functional.logsigmoid(-lg[1:]).sum())
+    (1.7 * torch.stack(rows).mean()).backward()
+    assert rel_err(dX, Xt.grad.numpy()) < 1e-12
+    assert rel_err(dY, Yt.grad.numpy()) < 1e-12
+
+
+@pytest.mark.parametrize("kind", [0, 1])
+def test_sampled_grad_finite_differences(kind):
+    X, Y, z, _ = _dyadic_case(N=5, C=12, d=3)
+    neg = np.random.default_rng(3).integers(0, 12, size=(5, 4)).astype(np.int32)
+    _, _, lse = oracle.sampled_loss(kind, X, Y, z, neg)
+    dloss = 0.6
+    dX, dY = oracle.sampled_grad(kind, X, Y, z, neg, lse, dloss)
+    h = 2.0 ** -10
+    for name, A, G in (("X", X, dX), ("Y", Y, dY)):
+        for idx in np.ndindex(A.shape):
+            ls = []
+            for sgn in (+1, -1):
+                P = A.copy()
+                P[idx] = P[idx] + np.float32(sgn * h)
+                XX, YY = (P, Y) if name == "X" else (X, P)
+                ls.append(oracle.sampled_loss(kind, XX, YY, z, neg)[0])
+            fd = dloss * (ls[0] - ls[1]) / (2 * h)
+            assert fd == pytest.approx(G[idx], abs=1e-6 * max(1.0, np.abs(G).max()))
+
+
+def test_sampled_invariants():
+    X, Y, z, neg = _sampled_case(pad=False)
+    N = len(X)
+    # padding takes no part
+    padded = np.concatenate([neg, np.full((N, 4), -1, np.int32)], 1)
+    for kind in (0, 1):
+        assert np.array_equal(oracle.sampled_loss(kind, X, Y, z, neg)[1],
+                              oracle.sampled_loss(kind, X, Y, z, padded)[1])
+    # BCE+: the negatives' terms are independent, so the loss is additive over a split
+    a, b = neg[:, :4], neg[:, 4:]
+    none = np.zeros((N, 0), np.int32)
+    r_ab = oracle.sampled_loss(1, X, Y, z, neg)[1]
+    r_a = oracle.sampled_loss(1, X, Y, z, a)[1]
+    r_b = oracle.sampled_loss(1, X, Y, z, b)[1]
+    r_0 = oracle.sampled_loss(1, X, Y, z, none)[1]
+    np.testing.assert_allclose(r_ab, r_a + r_b - r_0, rtol=1e-12)
+    # CE- with no negatives: the softmax over the positive alone, loss exactly 0
+    assert np.all(oracle.sampled_loss(0, X, Y, z, none)[1] == 0.0)
+    # CE-: more negatives never lower a row's loss (the denominator only grows)
+    assert np.all(oracle.sampled_loss(0, X, Y, z, a)[1] <=
+                  oracle.sampled_loss(0, X, Y, z, neg)[1] + 1e-15)
+    # every row's CE- coefficients sum to zero -> the dY rows sum to the zero vector
+    _, _, lse = oracle.sampled_loss(0, X, Y, z, neg)
+    _, dY = oracle.sampled_grad(0, X, Y, z, neg, lse, 1.0)
+    assert np.abs(dY.sum(0)).max() < 1e-12
+
+
 # --------------------------------------------------------------------------- inputs
 def test_bf16_rounding_is_round_to_nearest_even():
     vals = np.array([1.0, 1.00390625, 1.005859375, 1.0078125 + 2 ** -9, -3.3, 0.0],
