@@ -192,6 +192,45 @@ RECE_API rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t
                                const float* dloss, void* workspace, size_t workspace_bytes,
                                float* dX, float* dY, void* stream);
 
+/* Sampled baselines [RECE section 2, Related Work, equations (1) and (2)]: the loss of
+ * row i over its positive z_i and n given negatives, with l = <x_i, y_j>:
+ *   RECE_SAMPLED_CE_MINUS (eq. 2): loss_i = log(exp(l+) + sum_j exp(l_ij)) - l+
+ *   RECE_SAMPLED_BCE_PLUS (eq. 1): loss_i = -log sigmoid(l+) - sum_j log(1 - sigmoid(l_ij))
+ * L = (1/N) sum_i loss_i.  The caller draws the negatives (uniformly, in the pages'
+ * setting); the library takes them as given:
+ *   negatives  device int32 [N][n] (NULL when n = 0): ids in [0, C) or < 0 for padding
+ *              (no term).  A sample equal to the row's positive is a negative like any
+ *              other, and a repeated sample counts once per occurrence, as the sums are
+ *              written.  Ids >= C and targets outside [0, C) set RECE_DEVICE_BAD_TARGET.
+ *   mode       element type of X and Y (fp32 or bf16), arithmetic in fp32
+ * Workspace (rece_sampled_workspace_size bytes, 256-byte aligned): the status word, then
+ * the backward's pair arrays.  fwd writes loss [1], row_loss [N] (or NULL), logits
+ * [N][n+1] (slot 0 the positive, slot s the negative s-1; padding 0; or NULL) and, for
+ * CE-, lse [N] (required; unused and may be NULL for BCE+).  bwd takes fwd's logits (or
+ * NULL: they are recomputed) and lse, and overwrites dX [N][d] and dY [C][d]:
+ *   g_i+ = (p_i+ - 1) dloss/N,  g_ij = p_ij dloss/N,  p = exp(l - lse) (CE-), sigmoid(l) (BCE+)
+ *   dX_i = g_i+ y_{z_i} + sum_j g_ij y_j,  dY_j = sum of g x_i over the pairs naming j,
+ * deterministic (no floating-point atomics).  Limits: N (n+1) < 2^31, d + 2(n+1) <= 51200.
+ * Host errors (bad sizes, kind or mode, NULL pointers, small workspace) return before
+ * anything is launched. */
+#define RECE_SAMPLED_CE_MINUS 0
+#define RECE_SAMPLED_BCE_PLUS 1
+RECE_API rece_status_t rece_sampled_workspace_size(int32_t kind, int64_t N, int64_t C, int32_t d,
+                                                   int32_t n, int32_t mode, size_t* bytes);
+RECE_API rece_status_t rece_sampled_fwd(int32_t kind, int64_t N, int64_t C, int32_t d, int32_t n,
+                                        int32_t mode, const void* X, const void* Y,
+                                        const int32_t* targets, const int32_t* negatives,
+                                        void* workspace, size_t workspace_bytes, float* loss,
+                                        float* row_loss, float* logits, float* lse,
+                                        void* stream);
+RECE_API rece_status_t rece_sampled_bwd(int32_t kind, int64_t N, int64_t C, int32_t d, int32_t n,
+                                        int32_t mode, const void* X, const void* Y,
+                                        const int32_t* targets, const int32_t* negatives,
+                                        const float* logits, const float* lse,
+                                        const float* dloss, void* workspace,
+                                        size_t workspace_bytes, float* dX, float* dY,
+                                        void* stream);
+
 /* Stable bucket sort that allocates nothing (the pages have no counterpart: this is an
  * interface for callers, not a step of the method).  It is step 2's sort on its own, for
  * callers that cannot give the library device memory: code running inside another

@@ -30,8 +30,10 @@ EXPORTS = (
     "rece_full_ce_workspace_size", "rece_full_ce_fwd", "rece_full_ce_bwd",
     "rece_get_device_status", "rece_status_string", "rece_last_error_string",
     "rece_plan_set_stage_events", "rece_kernel_launch_count", "rece_bucket_sort_static",
-    "rece_plan_paths",
+    "rece_plan_paths", "rece_sampled_workspace_size", "rece_sampled_fwd", "rece_sampled_bwd",
 )
+SAMPLED_CE_MINUS = 0  # RECE section 2, equation (2)
+SAMPLED_BCE_PLUS = 1  # RECE section 2, equation (1)
 STAGES = ("bucketize", "sort", "select", "merge_loss", "mean", "bwd_rows", "bwd_sort",
           "bwd_items")
 
@@ -89,6 +91,11 @@ def lib():
         "rece_plan_set_stage_events": ([vp, ctypes.POINTER(vp)], st),
         "rece_kernel_launch_count": ([], ctypes.c_uint64),
         "rece_bucket_sort_static": ([vp, i64, i32, vp, vp, vp], st),
+        "rece_sampled_workspace_size": ([i32, i64, i64, i32, i32, i32, ctypes.POINTER(sz)], st),
+        "rece_sampled_fwd": ([i32, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp, vp,
+                              vp, vp], st),
+        "rece_sampled_bwd": ([i32, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                              vp, vp, vp], st),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)

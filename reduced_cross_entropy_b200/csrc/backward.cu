@@ -2,6 +2,8 @@
 // restricted to the positive and the kept negatives; selection held constant).
 //
 //   g_ij = (exp(l_ij - lse_i) - [j == z_i]) * dloss / N
+//   (the sampled baselines reuse it: CE- with its sampled negatives in the slots, BCE+
+//   with sigmoid(l_ij) in place of the softmax term; see sampled.cu)
 //   dX_i = sum_j g_ij y_j          (one warp per row: every lane computes whole dot
 //                                   products for its own slots, then the lanes sweep the
 //                                   dimensions adding the slots in order)
@@ -33,6 +35,12 @@ __device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
+// The coefficient's probability term: the softmax exp(l - lse) of the reduced loss and of
+// CE-, or the sigmoid of BCE+ (its g is sigmoid(l) - [positive] likewise).
+__device__ __forceinline__ float coef_p(float l, float li, bool sigmoid) {
+  return sigmoid ? 1.0f / (1.0f + expf(-l)) : expf(l - li);
+}
+
 // <x, y> with x in shared memory (fp32) and y a catalogue row, t ascending.
 template <typename T>
 __device__ __forceinline__ float dot_row(const float* xs, const T* __restrict__ y, int d) {
@@ -57,7 +65,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
     const int32_t* __restrict__ selected, const float* __restrict__ lse,
     const float* __restrict__ logits, const float* __restrict__ dloss, int64_t N, int64_t C,
     int d, int k, int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
-    uint32_t* status) {
+    uint32_t* status, bool sigmoid) {
   extern __shared__ __align__(16) float sh_f[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slots = k + 1;
@@ -68,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
   const int64_t i = int64_t(blockIdx.x) * warps + wid;
   if (i >= N) return;  // the warp leaves together; no block-wide barrier follows
   const float scale = dloss[0] / float(N);
-  const float li = lse[i];
+  const float li = sigmoid ? 0.0f : lse[i];
   for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
   __syncwarp();
 
@@ -78,7 +86,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
     float g = 0.0f;
     if (j >= 0 && j < C) {
       const float l = logits ? logits[i * slots + s] : dot_row(xs, Y + int64_t(j) * d, d);
-      const float p = expf(l - li);
+      const float p = coef_p(l, li, sigmoid);
       g = (s == 0 ? p - 1.0f : p) * scale;
     } else {
       if (s == 0) raise_flag(status, RECE_DEVICE_BAD_TARGET);
@@ -186,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
     const int32_t* __restrict__ selected, const float* __restrict__ lse,
     const float* __restrict__ logits, const float* __restrict__ dloss, int64_t N, int64_t C,
     int d, int k, int32_t* __restrict__ e_key, float* __restrict__ e_g, float* __restrict__ dX,
-    uint32_t* status) {
+    uint32_t* status, bool sigmoid) {
   extern __shared__ __align__(16) float sh_f[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = lane >> 3, sub = lane & 7;
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
   const int64_t i = int64_t(blockIdx.x) * warps + wid;
   if (i >= N) return;  // the warp leaves together; no block-wide barrier follows
   const float scale = dloss[0] / float(N);
-  const float li = lse[i];
+  const float li = sigmoid ? 0.0f : lse[i];
   for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
   __syncwarp();
 
@@ -209,7 +217,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
       const bool ok = j >= 0 && j < C;
       float g = 0.0f;
       if (ok) {
-        const float p = expf(logits[i * slots + s] - li);
+        const float p = coef_p(logits[i * slots + s], li, sigmoid);
         g = (s == 0 ? p - 1.0f : p) * scale;
       } else if (s == 0) {
         raise_flag(status, RECE_DEVICE_BAD_TARGET);
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
         if (s >= slots) continue;
         float g = 0.0f;
         if (ok[u]) {
-          const float p = expf(part[u] - li);
+          const float p = coef_p(part[u], li, sigmoid);
           g = (s == 0 ? p - 1.0f : p) * scale;
         } else if (s == 0) {
           raise_flag(status, RECE_DEVICE_BAD_TARGET);
@@ -427,11 +435,11 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
     if (v8)
       k_bwd_rows_v8<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
           X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dx_rows,
-          status);
+          status, p.sigmoid_g);
     else
       k_bwd_rows<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(
           X, Y, targets, selected, lse, logits, dloss, c.N, c.C, c.d, c.k, e_key, e_g, dx_rows,
-          status);
+          status, p.sigmoid_g);
     count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

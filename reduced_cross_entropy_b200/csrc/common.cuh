@@ -72,6 +72,19 @@ __device__ __forceinline__ void raise_flag(uint32_t* status, uint32_t bit) {
 }
 
 // ---------------------------------------------------------------- warp helpers
+// Lanes of the warp whose value dg (in [0, 2^bits)) equals this lane's, from one ballot
+// per bit (the peers agree with it on every bit); lanes with !ok match only themselves.
+// All 32 lanes must call it.
+__device__ __forceinline__ unsigned digit_peers(int dg, int bits, bool ok, int lane) {
+  unsigned m = __ballot_sync(0xFFFFFFFFu, ok);
+  for (int b = 0; b < bits; ++b) {
+    const bool bit = (dg >> b) & 1;
+    const unsigned v = __ballot_sync(0xFFFFFFFFu, bit);
+    m &= bit ? v : ~v;
+  }
+  return ok ? m : (1u << lane);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);

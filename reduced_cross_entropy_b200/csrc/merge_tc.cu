@@ -342,6 +342,8 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
     __syncwarp();
     // exclusive scan of the slice counts, lane l holding slices [l*B, l*B + B)
     const int B = (S + 31) >> 5;
+    int sbits = 0;  // bits of the slice ids 0..S-1
+    while ((1 << sbits) < S) ++sbits;
     int run = 0;
     for (int b = lane * B; b < S && b < lane * B + B; ++b) run += bins[b];
     int incl = run;
@@ -367,7 +369,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
       const int a = a0 + lane;
       const bool tk = a < rb[r + 1] && take(a);
       const int sl = tk ? (poss[a] >> 6) - sig0 : 0;
-      const unsigned peers = __match_any_sync(0xFFFFFFFFu, tk ? sl : int(0x40000000 | lane));
+      const unsigned peers = digit_peers(sl, sbits, tk, lane);
       const int dest = tk ? bins[sl] + __popc(peers & ((1u << lane) - 1u)) : 0;
       __syncwarp();
       if (tk && lane == __ffs(peers) - 1) bins[sl] += __popc(peers);

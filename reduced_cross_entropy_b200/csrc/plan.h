@@ -91,6 +91,7 @@ struct rece_plan_s {
   int32_t item_pass_bits;  // digit bits of every pass but the last
   int64_t entries;      // N * (k + 1): (row, item) pairs of the backward
   bool carry_g;         // the pair sort carries g (its array would not stay in L2)
+  bool sigmoid_g;       // backward coefficients sigmoid(l) - [positive] (BCE+), else softmax
   bool use_tc;          // bf16 mode on the tcgen05 kernels
   bool tc_dx;           // ... and dX of the backward on them too
   bool tc_scores;       // ... with the window scores computed once and stored (large d)
@@ -168,6 +169,14 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
                             const int32_t* targets, const int32_t* selected, const float* lse,
                             const float* logits, const float* dloss, char* ws, float* dX,
                             float* dY, uint32_t* status, cudaStream_t st);
+
+// Sampled baselines (sampled.cu): logits [N][n+1], lse (CE-) and row losses.
+size_t sampled_fwd_warp_bytes(int d, int n);
+template <typename T>
+cudaError_t launch_sampled_fwd(int kind, int64_t N, int64_t C, int d, int n, const T* X,
+                               const T* Y, const int32_t* targets, const int32_t* neg,
+                               float* logits, float* lse, float* row_loss, uint32_t* status,
+                               cudaStream_t st);
 
 // K6: exact full cross-entropy.
 template <typename T>

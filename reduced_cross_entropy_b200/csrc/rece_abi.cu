@@ -53,6 +53,40 @@ int64_t window_len(int64_t c, int64_t C, int64_t n_c, int64_t n_ec) {
   return chunk_start(hi, C, n_c) - chunk_start(lo, C, n_c);
 }
 
+// The backward's (item, row) pair arrays from offset `off` on.
+void layout_pairs(rece_plan_s& p, size_t& off) {
+  Layout& L = p.lay;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t E = size_t(p.entries);
+  L.e_key = take(sizeof(int32_t) * E);
+  L.e_g = take(sizeof(float) * E);
+  L.e_perm_a = take(sizeof(int32_t) * E);
+  L.e_perm_b = take(sizeof(int32_t) * E);
+  L.e_sorted_key = take(sizeof(int32_t) * E);
+  L.e_key_b = take(sizeof(int32_t) * E);
+  if (p.carry_g) {
+    L.e_sorted_g = take(sizeof(float) * E);
+    L.e_g_b = take(sizeof(float) * E);
+  }
+  L.e_item_start = take(sizeof(int32_t) * (size_t(p.cfg.C) + 1));
+  L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
+}
+
+// Item-sort geometry of the backward's pairs (keys 0..C: C marks an empty slot).
+void set_pair_sort(rece_plan_s& p) {
+  const auto& c = p.cfg;
+  p.item_bits = bits_for(c.C + 1);
+  p.item_passes = int32_t((p.item_bits + kMaxDigitBits - 1) / kMaxDigitBits);
+  if (p.item_passes < 1) p.item_passes = 1;
+  p.item_pass_bits = (p.item_bits + p.item_passes - 1) / p.item_passes;
+  p.entries = c.N * (int64_t(c.k) + 1);
+  p.carry_g = p.entries * int64_t(sizeof(float)) > (int64_t(32) << 20);
+}
+
 void build_layout(rece_plan_s& p) {
   const auto& c = p.cfg;
   Layout& L = p.lay;
@@ -106,21 +140,7 @@ void build_layout(rece_plan_s& p) {
   L.row_loss_tmp = take(sizeof(float) * c.N);
   L.fwd_end = off;
   off = region;
-  {
-    const size_t E = size_t(p.entries);
-    L.e_key = take(sizeof(int32_t) * E);
-    L.e_g = take(sizeof(float) * E);
-    L.e_perm_a = take(sizeof(int32_t) * E);
-    L.e_perm_b = take(sizeof(int32_t) * E);
-    L.e_sorted_key = take(sizeof(int32_t) * E);
-    L.e_key_b = take(sizeof(int32_t) * E);
-    if (p.carry_g) {
-      L.e_sorted_g = take(sizeof(float) * E);
-      L.e_g_b = take(sizeof(float) * E);
-    }
-    L.e_item_start = take(sizeof(int32_t) * (size_t(c.C) + 1));
-    L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
-  }
+  layout_pairs(p, off);
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
@@ -131,6 +151,45 @@ rece_status_t check_plan_ws(rece_plan_t plan, const void* ws, size_t ws_bytes) {
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
     return fail(RECE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
   if (ws_bytes < plan->lay.total) return fail(RECE_ERR_WORKSPACE, "workspace too small");
+  return RECE_OK;
+}
+
+// Plan of a sampled baseline (CE- / BCE+): the reduced loss's CUDA-core backward over
+// k = n sampled slots.  Workspace: the status words, then the pair arrays (the forward's
+// row-loss scratch shares their start: forward and backward are separate calls).
+rece_status_t sampled_plan(int32_t kind, int64_t N, int64_t C, int32_t d, int32_t n,
+                           int32_t mode, rece_plan_s& p) {
+  if (kind != RECE_SAMPLED_CE_MINUS && kind != RECE_SAMPLED_BCE_PLUS)
+    return fail(RECE_ERR_INVALID_ARG, "unknown sampled-loss kind");
+  if (N < 0 || C < 1 || C >= kInt32Max || d < 1 || n < 0)
+    return fail(RECE_ERR_INVALID_ARG, "bad sampled-loss sizes");
+  if (mode != RECE_MODE_FP32_EXACT && mode != RECE_MODE_BF16)
+    return fail(RECE_ERR_INVALID_ARG, "unknown mode");
+  if (N * (int64_t(n) + 1) >= kInt32Max || N * int64_t(d) >= (int64_t(1) << 40))
+    return fail(RECE_ERR_UNSUPPORTED, "sizes exceed 32-bit pair indexing");
+  if (int64_t(d) + 2 * (int64_t(n) + 1) > 51200)
+    return fail(RECE_ERR_UNSUPPORTED, "d + 2(n + 1) must be <= 51200");
+  p = rece_plan_s();
+  p.cfg.N = N;
+  p.cfg.C = C;
+  p.cfg.d = d;
+  p.cfg.n_b = 1;
+  p.cfg.n_c = 1;
+  p.cfg.n_ec = 0;
+  p.cfg.n_r = 1;
+  p.cfg.k = n;
+  p.cfg.mode = static_cast<rece_mode_t>(mode);
+  set_pair_sort(p);
+  p.sigmoid_g = kind == RECE_SAMPLED_BCE_PLUS;
+  size_t off = 0;
+  p.lay.status = off;
+  off += align256(4 * sizeof(uint32_t));
+  p.lay.row_loss_tmp = off;
+  const size_t fwd_end = off + align256(sizeof(float) * size_t(N));
+  layout_pairs(p, off);
+  p.lay.bwd_end = off;
+  p.lay.fwd_end = fwd_end;
+  p.lay.total = fwd_end > off ? fwd_end : off;
   return RECE_OK;
 }
 
@@ -199,12 +258,8 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     return fail(RECE_ERR_UNSUPPORTED, "chunk window too long for the selection kernel");
   }
   p->bucket_bits = bits_for(c.n_b);
-  p->item_bits = bits_for(c.C + 1);
-  p->item_passes = int32_t((p->item_bits + kMaxDigitBits - 1) / kMaxDigitBits);
-  if (p->item_passes < 1) p->item_passes = 1;
-  p->item_pass_bits = (p->item_bits + p->item_passes - 1) / p->item_passes;
-  p->entries = c.N * (int64_t(c.k) + 1);
-  p->carry_g = p->entries * int64_t(sizeof(float)) > (int64_t(32) << 20);
+  set_pair_sort(*p);
+  p->sigmoid_g = false;
   p->timed = false;
   for (void*& e : p->stage_events) e = nullptr;
   p->kept_slices = 0;
@@ -500,6 +555,79 @@ rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
                                  static_cast<const __nv_bfloat16*>(Y), targets, lse, dloss, dX,
                                  dY, st),
               "full CE backward");
+  return RECE_OK;
+}
+
+rece_status_t rece_sampled_workspace_size(int32_t kind, int64_t N, int64_t C, int32_t d,
+                                          int32_t n, int32_t mode, size_t* bytes) {
+  if (!bytes) return fail(RECE_ERR_INVALID_ARG, "bytes is NULL");
+  rece_plan_s p;
+  rece_status_t s = sampled_plan(kind, N, C, d, n, mode, p);
+  if (s != RECE_OK) return s;
+  *bytes = p.lay.total;
+  return RECE_OK;
+}
+
+rece_status_t rece_sampled_fwd(int32_t kind, int64_t N, int64_t C, int32_t d, int32_t n,
+                               int32_t mode, const void* X, const void* Y,
+                               const int32_t* targets, const int32_t* negatives,
+                               void* workspace, size_t workspace_bytes, float* loss,
+                               float* row_loss, float* logits, float* lse, void* stream) {
+  rece_plan_s p;
+  rece_status_t s = sampled_plan(kind, N, C, d, n, mode, p);
+  if (s != RECE_OK) return s;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < p.lay.total)
+    return fail(RECE_ERR_WORKSPACE, "workspace NULL, unaligned or too small");
+  if (!loss || !Y || (N > 0 && (!X || !targets || (n > 0 && !negatives) ||
+                                (kind == RECE_SAMPLED_CE_MINUS && !lse))))
+    return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.lay.status);
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + p.lay.row_loss_tmp);
+  RECE_CUDA(cudaMemsetAsync(status, 0, 4 * sizeof(uint32_t), st), "status reset");
+  if (mode == RECE_MODE_FP32_EXACT)
+    RECE_CUDA(launch_sampled_fwd(kind, N, C, d, n, static_cast<const float*>(X),
+                                 static_cast<const float*>(Y), targets, negatives, logits, lse,
+                                 rl, status, st),
+              "sampled forward");
+  else
+    RECE_CUDA(launch_sampled_fwd(kind, N, C, d, n, static_cast<const __nv_bfloat16*>(X),
+                                 static_cast<const __nv_bfloat16*>(Y), targets, negatives,
+                                 logits, lse, rl, status, st),
+              "sampled forward");
+  RECE_CUDA(launch_mean(rl, N, loss, st), "mean");
+  return RECE_OK;
+}
+
+rece_status_t rece_sampled_bwd(int32_t kind, int64_t N, int64_t C, int32_t d, int32_t n,
+                               int32_t mode, const void* X, const void* Y,
+                               const int32_t* targets, const int32_t* negatives,
+                               const float* logits, const float* lse, const float* dloss,
+                               void* workspace, size_t workspace_bytes, float* dX, float* dY,
+                               void* stream) {
+  rece_plan_s p;
+  rece_status_t s = sampled_plan(kind, N, C, d, n, mode, p);
+  if (s != RECE_OK) return s;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < p.lay.total)
+    return fail(RECE_ERR_WORKSPACE, "workspace NULL, unaligned or too small");
+  if (!Y || !dY || (N > 0 && (!X || !targets || (n > 0 && !negatives) || !dloss || !dX ||
+                              (kind == RECE_SAMPLED_CE_MINUS && !lse))))
+    return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.lay.status);
+  if (mode == RECE_MODE_FP32_EXACT)
+    RECE_CUDA(launch_backward(p, static_cast<const float*>(X), static_cast<const float*>(Y),
+                              targets, negatives, lse, logits, dloss, ws, dX, dY, status, st),
+              "sampled backward");
+  else
+    RECE_CUDA(launch_backward(p, static_cast<const __nv_bfloat16*>(X),
+                              static_cast<const __nv_bfloat16*>(Y), targets, negatives, lse,
+                              logits, dloss, ws, dX, dY, status, st),
+              "sampled backward");
   return RECE_OK;
 }
 

@@ -5,10 +5,11 @@
 // One pass over M elements with b-bit digits:
 //   hist     per tile of 2048 elements, the count of every digit (digit-major matrix)
 //   scan     exclusive prefix over tiles for every digit, then over digits
-//   scatter  every warp walks its 256 elements in order; __match_any_sync groups the
-//            lanes holding the same digit, so an element's rank is the number of
-//            earlier elements with its digit: in earlier tiles, earlier warps of its
-//            tile, earlier steps of its warp, lower lanes of its step.  Stable.
+//   scatter  every warp walks its 256 elements in order; one ballot per digit bit
+//            gives every lane the mask of lanes holding its digit, so an element's rank
+//            is the number of earlier elements with its digit: in earlier tiles,
+//            earlier warps of its tile, earlier steps of its warp, lower lanes of its
+//            step.  Stable.
 // Several independent sorts (segments) of one digit width go in one launch sequence:
 // blockIdx.y is the segment, blockIdx.x the tile (or digit) within it.
 #include "common.cuh"
@@ -185,11 +186,13 @@ __global__ void __launch_bounds__(kSortThreads, 4) k_sort_scatter(const __grid_c
     }
   }
   // pass 1: this warp's count of every digit
+  unsigned r_peers[kSteps];
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
     const bool ok = wbase + s * 32 + lane < M;
-    const int dg = ok ? ((r_key[s] >> shift) & mask) : (0x40000000 | lane);
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
+    const int dg = (r_key[s] >> shift) & mask;
+    const unsigned peers = digit_peers(dg, b.bits, ok, lane);
+    r_peers[s] = peers;
     if (ok && lane == __ffs(peers) - 1) wcnt[dg] += uint16_t(__popc(peers));
     __syncwarp();
   }
@@ -220,8 +223,8 @@ __global__ void __launch_bounds__(kSortThreads, 4) k_sort_scatter(const __grid_c
   for (int s = 0; s < kSteps; ++s) {
     const bool ok = wbase + s * 32 + lane < M;
     const int32_t key = r_key[s];
-    const int dg = ok ? ((key >> shift) & mask) : (0x40000000 | lane);
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, dg);
+    const int dg = (key >> shift) & mask;
+    const unsigned peers = r_peers[s];
     const int base = ok ? int(wcnt[dg]) : 0;
     __syncwarp();
     if (ok) {

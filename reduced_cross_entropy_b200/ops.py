@@ -214,6 +214,67 @@ def full_ce_bwd(X, Y, targets, lse, dloss, ws, stream=None):
     return dX, dY
 
 
+_KINDS = {"ce_minus": _lib.SAMPLED_CE_MINUS, "bce_plus": _lib.SAMPLED_BCE_PLUS}
+
+
+def _kind(kind) -> int:
+    return _KINDS[kind] if isinstance(kind, str) else int(kind)
+
+
+def sampled_workspace_bytes(kind, N, C, d, n, mode="bf16") -> int:
+    size = ctypes.c_size_t()
+    m = _MODES[mode] if isinstance(mode, str) else int(mode)
+    _lib.check(_lib.lib().rece_sampled_workspace_size(_kind(kind), N, C, d, n, m,
+                                                      ctypes.byref(size)),
+               "rece_sampled_workspace_size")
+    return int(size.value)
+
+
+def sampled_fwd(kind, X, Y, targets, negatives, ws=None, stream=None):
+    """Sampled baseline forward: kind "ce_minus" (RECE section 2, eq. 2) or "bce_plus"
+    (eq. 1) over negatives [N, n] int32 (ids < 0: padding).
+    Returns (loss [1], row_loss [N], logits [N, n+1], lse [N], ws)."""
+    N, d = X.shape
+    C = Y.shape[0]
+    n = negatives.shape[1]
+    mode = _lib.MODE_BF16 if X.dtype == torch.bfloat16 else _lib.MODE_FP32_EXACT
+    _need(X, "X", _DTYPES[mode], (N, d))
+    _need(Y, "Y", _DTYPES[mode], (C, d))
+    _need(targets, "targets", torch.int32, (N,))
+    _need(negatives, "negatives", torch.int32, (N, n))
+    nbytes = sampled_workspace_bytes(kind, N, C, d, n, mode)
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
+    loss = torch.empty(1, dtype=torch.float32, device=X.device)
+    row = torch.empty(N, dtype=torch.float32, device=X.device)
+    logits = torch.empty(N, n + 1, dtype=torch.float32, device=X.device)
+    lse = torch.empty(N, dtype=torch.float32, device=X.device)
+    _lib.check(_lib.lib().rece_sampled_fwd(_kind(kind), N, C, d, n, mode, _vp(X), _vp(Y),
+                                           _vp(targets), _vp(negatives), _vp(ws), ws.numel(),
+                                           _vp(loss), _vp(row), _vp(logits), _vp(lse),
+                                           _stream(stream)), "rece_sampled_fwd")
+    return loss, row, logits, lse, ws
+
+
+def sampled_bwd(kind, X, Y, targets, negatives, lse, dloss, ws, logits=None, stream=None):
+    """Gradients of the sampled baseline (negatives held constant): (dX, dY) fp32."""
+    N, d = X.shape
+    C = Y.shape[0]
+    n = negatives.shape[1]
+    mode = _lib.MODE_BF16 if X.dtype == torch.bfloat16 else _lib.MODE_FP32_EXACT
+    _need(lse, "lse", torch.float32, (N,))
+    _need(dloss, "dloss", torch.float32, (1,))
+    if logits is not None:
+        _need(logits, "logits", torch.float32, (N, n + 1))
+    dX = torch.empty(N, d, dtype=torch.float32, device=X.device)
+    dY = torch.empty(C, d, dtype=torch.float32, device=X.device)
+    _lib.check(_lib.lib().rece_sampled_bwd(_kind(kind), N, C, d, n, mode, _vp(X), _vp(Y),
+                                           _vp(targets), _vp(negatives), _vp(logits), _vp(lse),
+                                           _vp(dloss), _vp(ws), ws.numel(), _vp(dX), _vp(dY),
+                                           _stream(stream)), "rece_sampled_bwd")
+    return dX, dY
+
+
 class _ReceLossFn(torch.autograd.Function):
     @staticmethod
     def forward(ctx, X, Y, targets, B, plan, ws):

@@ -118,6 +118,15 @@ def projections(seed: int, step: int, n_r: int, n_b: int, d: int, dtype: str = "
     return round_bf16(B) if dtype == "bf16" else B
 
 
+def uniform_negatives(seed: int, N: int, C: int, n: int) -> np.ndarray:
+    """n negatives per row drawn uniformly from the catalogue [0, C), with replacement
+    (the uniform sampling of the sampled baselines, RECE section 2), int32 [N, n].  The
+    draw may hit the row's positive or repeat an item; the losses take the ids as given."""
+    ss = np.random.SeedSequence([seed, 0x5A4D])
+    rng = np.random.Generator(np.random.PCG64(ss))
+    return rng.integers(0, C, size=(N, n), dtype=np.int64).astype(np.int32)
+
+
 def integer_inputs(N: int, C: int, d: int, lo: int = -3, hi: int = 3, seed: int = 0,
                    scale: float = 0.25):
     """Small-integer multiples of `scale` (a power of two): every product and partial
