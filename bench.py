@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="sasrec")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-memory", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true",
+                    help="skip timing the sampled CE- / BCE+ comparison ops")
     ap.add_argument("--flags", type=int, default=0, help="rece_config_t.flags")
     return ap.parse_args()
 
@@ -470,6 +472,9 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_memory:
         line["peak_hbm"] = measure_memory(torch, ops, plan, w, Xd, Yd, td, Bs[0], dev)
+    if rank == 0 and world == 1 and not args.no_baselines:
+        line["baselines"] = measure_baselines(torch, ops, w, Xd, Yd, td, flush, dev,
+                                              load_peaks())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         rows, frac = 256, 16
@@ -482,6 +487,44 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def measure_baselines(torch, ops, w, Xd, Yd, td, flush, dev, peaks, reps=10, warm=3):
+    """The pages' sampled comparison points (RECE section 2: CE- eq. 2, BCE+ eq. 1) on the
+    same resident inputs, n = k uniform negatives per row (as many as RECE keeps):
+    fwd+bwd rows/s (L2 flushed between steps, CUDA events), and the forward's gather
+    rate: its algorithmic bytes are the N (n+1) catalogue rows it reads, x, and the
+    logits it writes."""
+    from reduced_cross_entropy_b200 import synth
+    n = w.k
+    neg = torch.from_numpy(synth.uniform_negatives(1, w.N, w.C, n)).to(dev)
+    dl = torch.ones(1, dtype=torch.float32, device=dev)
+    e = 2 if w.dtype == "bf16" else 4
+    fwd_bytes = w.N * (n + 1) * w.d * e + w.N * w.d * e + w.N * (n + 1) * 4
+    out = {"negatives_per_row": n, "sampling": "uniform over [0, C), with replacement"}
+    stream = torch.cuda.current_stream(dev)
+    for kind in ("ce_minus", "bce_plus"):
+        ws = torch.empty(ops.sampled_workspace_bytes(kind, w.N, w.C, w.d, n, w.dtype),
+                         dtype=torch.uint8, device=dev)
+        fw, tot = [], []
+        for r in range(warm + reps):
+            flush.zero_()
+            a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record(stream)
+            _, _, lg, lse, _ = ops.sampled_fwd(kind, Xd, Yd, td, neg, ws)
+            m.record(stream)
+            ops.sampled_bwd(kind, Xd, Yd, td, neg, lse, dl, ws, logits=lg)
+            b.record(stream)
+            b.synchronize()
+            if r >= warm:
+                fw.append(a.elapsed_time(m))
+                tot.append(a.elapsed_time(b))
+        assert ops.device_status(ws) == 0
+        ms, fms = statistics.median(tot), statistics.median(fw)
+        gbs = fwd_bytes / (fms / 1e3) / 1e9
+        out[kind] = {"rows_per_s": w.N / (ms / 1e3), "ms_fwd_bwd": ms, "ms_fwd": fms,
+                     "fwd_gather_gbs": gbs, "fwd_frac_of_hbm": gbs / peaks["hbm_gbs"]}
+    return out
 
 
 def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
@@ -527,6 +570,14 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
     out["ratio_vs_materialised"] = ref / max(out["rece_bytes"], 1)
     if out["full_ce_fused_bytes"] is not None:
         out["ratio_vs_fused"] = out["full_ce_fused_bytes"] / max(out["rece_bytes"], 1)
+    # the pages' memory model of Algorithm 1 (every chunk's logits stored) at this
+    # workload's alpha_bc = n_b / n_c, and the bucket count it calls optimal
+    a = w.n_b / w.n_c
+    nb, nc = ops.optimal_buckets(w.N, w.C, w.n_ec, a)
+    el = ops.memory_model_elements(w.N, w.C, w.n_ec, w.n_r, a)
+    out["pages_memory_model"] = {"alpha_bc": a, "n_b_star": nb, "n_c_star": nc,
+                                 "logit_elements": el, "bytes_fp32": 4 * el,
+                                 "rece_bytes_over_model": out["rece_bytes"] / (4 * el)}
     out["note"] = "bytes above the resident inputs; torch.cuda.max_memory_allocated"
     return out
 

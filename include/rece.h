@@ -192,6 +192,20 @@ RECE_API rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t
                                const float* dloss, void* workspace, size_t workspace_bytes,
                                float* dX, float* dY, void* stream);
 
+/* Bucket count for the least memory [RECE section 3, the paragraph before Algorithm 1]:
+ *   n_b* = sqrt(4 alpha_bc (1 + 2 n_ec) min(C, N)),   alpha_bc = n_b / n_c,
+ * rounded to the nearest integer and clamped to [1, 4096]; n_c* = n_b* / alpha_bc rounded,
+ * clamped to [1, min(N, C)].  N is the row count (the pages' s * l).  Host only. */
+RECE_API rece_status_t rece_optimal_buckets(int64_t N, int64_t C, int32_t n_ec, double alpha_bc,
+                                            int32_t* n_b, int32_t* n_c);
+/* The pages' memory model of the method at n_b* [same paragraph], in logit elements:
+ *   2 r sqrt(alpha_bc (1 + 2 n_ec) min(C, N)) max(C, N),
+ * against N * C for the full cross-entropy (ratio sqrt(min) / (2 r sqrt(alpha_bc (1 + 2 n_ec)))).
+ * A model of Algorithm 1, which stores every chunk's logits; this library keeps them on
+ * chip, so its workspace sits below the model.  Host only. */
+RECE_API rece_status_t rece_memory_model_elements(int64_t N, int64_t C, int32_t n_ec, int32_t n_r,
+                                                  double alpha_bc, double* elements);
+
 /* Sampled baselines [RECE section 2, Related Work, equations (1) and (2)]: the loss of
  * row i over its positive z_i and n given negatives, with l = <x_i, y_j>:
  *   RECE_SAMPLED_CE_MINUS (eq. 2): loss_i = log(exp(l+) + sum_j exp(l_ij)) - l+

@@ -13,11 +13,13 @@ upcast) and follows the definitions cited in ``rece_oracle.c``:
                        de-duplicated, the k best by (score desc, item asc) (SCE abstract)
 * ``rece_loss`` / ``rece_grad``       -- Algorithm 1's loss, equation (4) on the subset
 * ``full_ce_loss`` / ``full_ce_grad`` -- equations (3) and (4) over the whole catalogue
+* ``optimal_buckets`` / ``memory_model_elements`` -- section 3's n_b* and memory model
 * ``sampled_loss`` / ``sampled_grad`` -- the sampled baselines of section 2: CE- (eq. 2,
                        kind 0) and BCE+ (eq. 1, kind 1) over given negatives
 * ``rece_forward``  -- the whole forward path, steps 1 to 5, given the random vectors B
 """
 import ctypes
+import math
 import os
 
 import numpy as np
@@ -176,6 +178,24 @@ def full_ce_grad(X, Y, target, lse, dloss=1.0):
     _load().oracle_full_ce_grad(X, Y, target, N, C, d, np.ascontiguousarray(lse, np.float64),
                                 float(dloss), dX, dY)
     return dX, dY
+
+
+def optimal_buckets(N, C, n_ec, alpha_bc):
+    """RECE section 3, the paragraph before Algorithm 1: the bucket count of least peak
+    memory, n_b* = sqrt(4 alpha_bc (1 + 2 n_ec) min(C, N)) with alpha_bc = n_b / n_c,
+    rounded to the nearest integer (halves up) and held to [1, 4096]; n_c* = n_b* /
+    alpha_bc rounded the same way and held to [1, min(N, C)]."""
+    m = min(C, N)
+    b = math.floor(math.sqrt(4.0 * alpha_bc * (1 + 2 * n_ec) * m) + 0.5)
+    b = min(max(b, 1), 4096)
+    c = min(max(math.floor(b / alpha_bc + 0.5), 1), m)
+    return b, c
+
+
+def memory_model_elements(N, C, n_ec, n_r, alpha_bc):
+    """The same paragraph's memory complexity at n_b*, in logit elements:
+    2 r sqrt(alpha_bc (1 + 2 n_ec) min(C, N)) max(C, N)."""
+    return 2.0 * n_r * math.sqrt(alpha_bc * (1 + 2 * n_ec) * min(C, N)) * max(C, N)
 
 
 SAMPLED_CE_MINUS = 0  # equation (2)

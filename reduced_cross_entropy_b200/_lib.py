@@ -31,6 +31,7 @@ EXPORTS = (
     "rece_get_device_status", "rece_status_string", "rece_last_error_string",
     "rece_plan_set_stage_events", "rece_kernel_launch_count", "rece_bucket_sort_static",
     "rece_plan_paths", "rece_sampled_workspace_size", "rece_sampled_fwd", "rece_sampled_bwd",
+    "rece_optimal_buckets", "rece_memory_model_elements",
 )
 SAMPLED_CE_MINUS = 0  # RECE section 2, equation (2)
 SAMPLED_BCE_PLUS = 1  # RECE section 2, equation (1)
@@ -92,6 +93,10 @@ def lib():
         "rece_kernel_launch_count": ([], ctypes.c_uint64),
         "rece_bucket_sort_static": ([vp, i64, i32, vp, vp, vp], st),
         "rece_sampled_workspace_size": ([i32, i64, i64, i32, i32, i32, ctypes.POINTER(sz)], st),
+        "rece_optimal_buckets": ([i64, i64, i32, ctypes.c_double, ctypes.POINTER(i32),
+                                  ctypes.POINTER(i32)], st),
+        "rece_memory_model_elements": ([i64, i64, i32, i32, ctypes.c_double,
+                                        ctypes.POINTER(ctypes.c_double)], st),
         "rece_sampled_fwd": ([i32, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp, vp,
                               vp, vp], st),
         "rece_sampled_bwd": ([i32, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz,

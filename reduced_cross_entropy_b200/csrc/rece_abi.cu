@@ -2,6 +2,7 @@
 // layout and the launch sequence of every entry point.  No device memory is allocated
 // here: every device buffer, the workspace included, belongs to the caller.
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -555,6 +556,29 @@ rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
                                  static_cast<const __nv_bfloat16*>(Y), targets, lse, dloss, dX,
                                  dY, st),
               "full CE backward");
+  return RECE_OK;
+}
+
+rece_status_t rece_optimal_buckets(int64_t N, int64_t C, int32_t n_ec, double alpha_bc,
+                                   int32_t* n_b, int32_t* n_c) {
+  if (!n_b || !n_c || N < 1 || C < 1 || n_ec < 0 || !(alpha_bc > 0.0))
+    return fail(RECE_ERR_INVALID_ARG, "bad optimal-bucket arguments");
+  const double mn = double(N < C ? N : C);
+  double b = std::floor(std::sqrt(4.0 * alpha_bc * (1.0 + 2.0 * n_ec) * mn) + 0.5);
+  b = b < 1.0 ? 1.0 : (b > double(1 << kMaxDigitBits) ? double(1 << kMaxDigitBits) : b);
+  double c = std::floor(b / alpha_bc + 0.5);
+  c = c < 1.0 ? 1.0 : (c > mn ? mn : c);
+  *n_b = int32_t(b);
+  *n_c = int32_t(c);
+  return RECE_OK;
+}
+
+rece_status_t rece_memory_model_elements(int64_t N, int64_t C, int32_t n_ec, int32_t n_r,
+                                         double alpha_bc, double* elements) {
+  if (!elements || N < 1 || C < 1 || n_ec < 0 || n_r < 1 || !(alpha_bc > 0.0))
+    return fail(RECE_ERR_INVALID_ARG, "bad memory-model arguments");
+  const double mn = double(N < C ? N : C), mx = double(N < C ? C : N);
+  *elements = 2.0 * n_r * std::sqrt(alpha_bc * (1.0 + 2.0 * n_ec) * mn) * mx;
   return RECE_OK;
 }
 

@@ -214,6 +214,23 @@ def full_ce_bwd(X, Y, targets, lse, dloss, ws, stream=None):
     return dX, dY
 
 
+def optimal_buckets(N: int, C: int, n_ec: int, alpha_bc: float):
+    """(n_b*, n_c*) of the least memory (RECE section 3), for alpha_bc = n_b / n_c."""
+    nb, nc = ctypes.c_int32(), ctypes.c_int32()
+    _lib.check(_lib.lib().rece_optimal_buckets(N, C, n_ec, float(alpha_bc), ctypes.byref(nb),
+                                               ctypes.byref(nc)), "rece_optimal_buckets")
+    return int(nb.value), int(nc.value)
+
+
+def memory_model_elements(N: int, C: int, n_ec: int, n_r: int, alpha_bc: float) -> float:
+    """The pages' memory model of the method at n_b*, in logit elements."""
+    v = ctypes.c_double()
+    _lib.check(_lib.lib().rece_memory_model_elements(N, C, n_ec, n_r, float(alpha_bc),
+                                                     ctypes.byref(v)),
+               "rece_memory_model_elements")
+    return float(v.value)
+
+
 _KINDS = {"ce_minus": _lib.SAMPLED_CE_MINUS, "bce_plus": _lib.SAMPLED_BCE_PLUS}
 
 

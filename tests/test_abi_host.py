@@ -139,3 +139,39 @@ def test_plan_paths_follow_the_shape():
     assert paths(W["sasrec"], d=48) == 0              # d not a multiple of 64
     p = Plan(256, 4096, 64, 16, 8, 1, 1, 32, mode="bf16", flags=_lib.FLAG_FMA_SCORES)
     assert p.paths == 0                               # fmaf scores on request
+
+
+def test_optimal_buckets_and_memory_model_match_the_oracle():
+    import oracle
+    from reduced_cross_entropy_b200 import ops
+    for N, C, n_ec, n_r, a in [(25600, 100000, 1, 2, 4.0), (51200, 10 ** 6, 1, 2, 1.0),
+                               (300, 200, 0, 1, 0.5), (16384, 128000, 2, 3, 2.0),
+                               (7, 10 ** 9, 2, 1, 2.0), (10 ** 9, 10 ** 9, 3, 1, 4.0),
+                               (1, 1, 0, 1, 1.0), (2500, 3000, 0, 1, 0.25)]:
+        assert ops.optimal_buckets(N, C, n_ec, a) == oracle.optimal_buckets(N, C, n_ec, a)
+        assert ops.memory_model_elements(N, C, n_ec, n_r, a) == pytest.approx(
+            oracle.memory_model_elements(N, C, n_ec, n_r, a), rel=1e-12)
+    L = _lib.lib()
+    nb, nc, v = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_double()
+    assert L.rece_optimal_buckets(10, 10, 0, 0.0, ctypes.byref(nb), ctypes.byref(nc)) == 1
+    assert L.rece_optimal_buckets(0, 10, 0, 1.0, ctypes.byref(nb), ctypes.byref(nc)) == 1
+    assert L.rece_memory_model_elements(10, 10, -1, 1, 1.0, ctypes.byref(v)) == 1
+
+
+def test_sampled_workspace_and_validation():
+    from reduced_cross_entropy_b200 import ops
+    small = ops.sampled_workspace_bytes("ce_minus", 1000, 5000, 64, 10, "bf16")
+    large = ops.sampled_workspace_bytes("ce_minus", 1000, 5000, 64, 100, "bf16")
+    assert 0 < small < large
+    assert ops.sampled_workspace_bytes("bce_plus", 0, 5000, 64, 10, "fp32") > 0
+    L = _lib.lib()
+    sz = ctypes.c_size_t()
+    assert L.rece_sampled_workspace_size(2, 10, 10, 8, 1, 0, ctypes.byref(sz)) == 1  # kind
+    assert L.rece_sampled_workspace_size(0, 10, 10, 8, -1, 0, ctypes.byref(sz)) == 1  # n
+    assert L.rece_sampled_workspace_size(0, 10, 10, 8, 1, 7, ctypes.byref(sz)) == 1  # mode
+    assert L.rece_sampled_workspace_size(0, 10, 10, 50000, 1000, 0, ctypes.byref(sz)) == 2
+    assert L.rece_sampled_workspace_size(0, 2 ** 20, 10, 8, 4096, 0, ctypes.byref(sz)) == 2
+    # a workspace smaller than asked for is refused before anything is launched
+    one = ctypes.c_void_p(256)
+    assert L.rece_sampled_fwd(0, 10, 10, 8, 1, 0, one, one, one, one, one, 16, one, None,
+                              None, one, None) == 3

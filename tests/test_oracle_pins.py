@@ -467,3 +467,26 @@ def test_bf16_rounding_is_round_to_nearest_even():
     v = rng.standard_normal(10000).astype(np.float32)
     np.testing.assert_array_equal(synth.round_bf16(v),
                                   torch.from_numpy(v).to(torch.bfloat16).float().numpy())
+
+
+# --------------------------------------------------------------------------- memory model
+def test_optimal_buckets_closed_forms():
+    # 4 * 1 * (1 + 2) * 10000 = 120000 -> sqrt = 346.41 -> 346, n_c = 346 / 1 = 346
+    assert oracle.optimal_buckets(10000, 10 ** 6, 1, 1.0) == (346, 346)
+    # alpha_bc = 0.25, n_ec = 0, min = 2500: sqrt(2500) = 50, n_c = 200
+    assert oracle.optimal_buckets(2500, 3000, 0, 0.25) == (50, 200)
+    # the count is symmetric in N and C (min of the two), clamped at 4096
+    assert oracle.optimal_buckets(7, 10 ** 9, 2, 2.0) == oracle.optimal_buckets(10 ** 9, 7, 2, 2.0)
+    assert oracle.optimal_buckets(10 ** 9, 10 ** 9, 3, 4.0)[0] == 4096
+
+
+def test_memory_model_matches_the_stated_ratio():
+    """The pages state the model is sqrt(min) / (2 r sqrt(alpha_bc (1 + 2 n_ec))) times
+    below the full cross-entropy's N * C logits; check that ratio on a grid."""
+    for N, C, n_ec, n_r, a in [(25600, 100000, 1, 2, 4.0), (51200, 10 ** 6, 1, 2, 1.0),
+                               (300, 200, 0, 1, 0.5), (16384, 128000, 2, 3, 2.0)]:
+        model = oracle.memory_model_elements(N, C, n_ec, n_r, a)
+        ratio = math.sqrt(min(N, C)) / (2 * n_r * math.sqrt(a * (1 + 2 * n_ec)))
+        assert N * C / model == pytest.approx(ratio, rel=1e-12)
+    # the minimised quantity: at alpha_bc = 1, n_ec = 0, r = 1, min = max = M: 2 M^1.5
+    assert oracle.memory_model_elements(400, 400, 0, 1, 1.0) == pytest.approx(2 * 400 ** 1.5)
