@@ -13,6 +13,8 @@ upcast) and follows the definitions cited in ``rece_oracle.c``:
                        de-duplicated, the k best by (score desc, item asc) (SCE abstract)
 * ``rece_loss`` / ``rece_grad``       -- Algorithm 1's loss, equation (4) on the subset
 * ``full_ce_loss`` / ``full_ce_grad`` -- equations (3) and (4) over the whole catalogue
+* ``window_loss`` / ``window_grad`` -- Algorithm 1 as printed: every window item a
+                       negative, duplicates across rounds corrected by ln(count)
 * ``optimal_buckets`` / ``memory_model_elements`` -- section 3's n_b* and memory model
 * ``sampled_loss`` / ``sampled_grad`` -- the sampled baselines of section 2: CE- (eq. 2,
                        kind 0) and BCE+ (eq. 1, kind 1) over given negatives
@@ -66,6 +68,12 @@ def _load():
         lib.oracle_sampled_grad.argtypes = [i32, f32p, f32p, i32p, i64, i64, i32, i32, i32p,
                                             f64p, ctypes.c_double, f64p, f64p]
         lib.oracle_sampled_grad.restype = None
+        lib.oracle_window_loss.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32,
+                                           i32p, i32p, f64p, f64p, f64p]
+        lib.oracle_window_loss.restype = None
+        lib.oracle_window_grad.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32,
+                                           i32p, i32p, f64p, ctypes.c_double, f64p, f64p]
+        lib.oracle_window_grad.restype = None
         lib.oracle_dot_f32.argtypes = [f32p, f32p, i32]
         lib.oracle_dot_f32.restype = ctypes.c_float
         lib.oracle_num_threads.argtypes = []
@@ -228,6 +236,39 @@ def sampled_grad(kind, X, Y, target, negatives, lse, dloss=1.0):
     dY = np.empty((C, d), np.float64)
     _load().oracle_sampled_grad(int(kind), X, Y, target, N, C, d, n, neg,
                                 np.ascontiguousarray(lse, np.float64), float(dloss), dX, dY)
+    return dX, dY
+
+
+def window_loss(X, Y, target, permX, permY, n_c, n_ec):
+    """Algorithm 1 as printed (every window item a negative) over the rounds' stable
+    orders permX [n_r, N], permY [n_r, C], duplicates across rounds corrected by
+    ln(count).  Returns (loss, row_loss, lse)."""
+    X, Y, target = _f32(X), _f32(Y), _i32(target)
+    permX, permY = _i32(permX), _i32(permY)
+    N, d = X.shape
+    n_r = permY.shape[0]
+    row = np.empty(N, np.float64)
+    lse = np.empty(N, np.float64)
+    loss = np.zeros(1, np.float64)
+    _load().oracle_window_loss(X, Y, target, N, Y.shape[0], d, n_c, n_ec, n_r,
+                               permX.reshape(-1) if N else np.zeros(1, np.int32),
+                               permY.reshape(-1), row, lse, loss)
+    return float(loss[0]), row, lse
+
+
+def window_grad(X, Y, target, permX, permY, n_c, n_ec, lse, dloss=1.0):
+    """(dX, dY) of window_loss, the buckets and windows held constant (fp64)."""
+    X, Y, target = _f32(X), _f32(Y), _i32(target)
+    permX, permY = _i32(permX), _i32(permY)
+    N, d = X.shape
+    C = Y.shape[0]
+    n_r = permY.shape[0]
+    dX = np.empty((N, d), np.float64)
+    dY = np.empty((C, d), np.float64)
+    _load().oracle_window_grad(X, Y, target, N, C, d, n_c, n_ec, n_r,
+                               permX.reshape(-1) if N else np.zeros(1, np.int32),
+                               permY.reshape(-1), np.ascontiguousarray(lse, np.float64),
+                               float(dloss), dX, dY)
     return dX, dY
 
 

@@ -306,6 +306,136 @@ void oracle_full_ce_grad(const float* X, const float* Y, const int32_t* target, 
   }
 }
 
+/* Algorithm 1 as printed [RECE section 3], every window item a negative (no top-k),
+ * over n_r rounds with the rounds paragraph's duplicate correction: a pair (i, j)
+ * computed in cnt_ij of the rounds enters every round's sum as exp(l_ij - ln cnt_ij).
+ * Row i's window in round r: the sorted catalogue positions of chunks c-n_ec..c+n_ec
+ * (clipped) of the chunk c that holds its sorted position; its positive is left out of
+ * the window sums (it enters once, as l+):
+ *   lse_i  = log(exp(l+) + sum_r sum_{j in W_r(i), j != z_i} exp(l_ij - ln cnt_ij))
+ *   loss_i = lse_i - l+,   L = mean_i loss_i          (fp64)
+ * permX [n_r*N], permY [n_r*C]: the rounds' stable bucket orders. */
+static void window_of(int64_t i, int32_t r, const int64_t* posX, int64_t N, int64_t C,
+                      int32_t n_c, int32_t n_ec, int64_t* q_lo, int64_t* q_hi) {
+  int64_t c = chunk_of(posX[(int64_t)r * N + i], N, n_c);
+  int64_t c_lo = c - n_ec < 0 ? 0 : c - n_ec;
+  int64_t c_hi = c + n_ec + 1 > n_c ? n_c : c + n_ec + 1;
+  *q_lo = oracle_chunk_start(c_lo, C, n_c);
+  *q_hi = oracle_chunk_start(c_hi, C, n_c);
+}
+
+static int64_t* positions(const int32_t* permX, int64_t N, int32_t n_r) {
+  int64_t* posX = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N * n_r > 0 ? N * n_r : 1));
+  for (int32_t r = 0; r < n_r; ++r)
+    for (int64_t p = 0; p < N; ++p) posX[(int64_t)r * N + permX[(int64_t)r * N + p]] = p;
+  return posX;
+}
+
+void oracle_window_loss(const float* X, const float* Y, const int32_t* target, int64_t N,
+                        int64_t C, int32_t d, int32_t n_c, int32_t n_ec, int32_t n_r,
+                        const int32_t* permX, const int32_t* permY, double* row_loss,
+                        double* lse, double* loss) {
+  int64_t* posX = positions(permX, N, n_r);
+#pragma omp parallel
+  {
+    int32_t* cnt = (int32_t*)calloc((size_t)C, sizeof(int32_t));
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t i = 0; i < N; ++i) {
+      const float* x = X + i * (int64_t)d;
+      int64_t q_lo, q_hi;
+      /* how many rounds compute each pair of this row */
+      for (int32_t r = 0; r < n_r; ++r) {
+        window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+        for (int64_t q = q_lo; q < q_hi; ++q) {
+          int32_t j = permY[(int64_t)r * C + q];
+          if (j != target[i]) ++cnt[j];
+        }
+      }
+      double lp = dot_f64(x, Y + (int64_t)target[i] * d, d);
+      double m = lp;
+      for (int32_t r = 0; r < n_r; ++r) {
+        window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+        for (int64_t q = q_lo; q < q_hi; ++q) {
+          int32_t j = permY[(int64_t)r * C + q];
+          if (j == target[i]) continue;
+          double l = dot_f64(x, Y + (int64_t)j * d, d) - log((double)cnt[j]);
+          if (l > m) m = l;
+        }
+      }
+      double s = exp(lp - m);
+      for (int32_t r = 0; r < n_r; ++r) {
+        window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+        for (int64_t q = q_lo; q < q_hi; ++q) {
+          int32_t j = permY[(int64_t)r * C + q];
+          if (j == target[i]) continue;
+          s += exp(dot_f64(x, Y + (int64_t)j * d, d) - log((double)cnt[j]) - m);
+        }
+      }
+      lse[i] = m + log(s);
+      row_loss[i] = lse[i] - lp;
+      for (int32_t r = 0; r < n_r; ++r) {
+        window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+        for (int64_t q = q_lo; q < q_hi; ++q) cnt[permY[(int64_t)r * C + q]] = 0;
+      }
+    }
+    free(cnt);
+  }
+  free(posX);
+  double total = 0.0;
+  for (int64_t i = 0; i < N; ++i) total += row_loss[i];
+  *loss = N > 0 ? total / (double)N : 0.0;
+}
+
+/* Its gradients, the buckets and windows held constant: every computed copy of a pair
+ * carries g = exp(l_ij - ln cnt_ij - lse_i) dloss/N, the positive (exp(l+ - lse_i) - 1)
+ * dloss/N;  dX_i = sum of g y_j,  dY_j = sum of g x_i over all copies  (fp64). */
+void oracle_window_grad(const float* X, const float* Y, const int32_t* target, int64_t N,
+                        int64_t C, int32_t d, int32_t n_c, int32_t n_ec, int32_t n_r,
+                        const int32_t* permX, const int32_t* permY, const double* lse,
+                        double dloss, double* dX, double* dY) {
+  double scale = N > 0 ? dloss / (double)N : 0.0;
+  int64_t* posX = positions(permX, N, n_r);
+  int32_t* cnt = (int32_t*)calloc((size_t)C, sizeof(int32_t));
+  memset(dY, 0, sizeof(double) * (size_t)C * (size_t)d);
+  for (int64_t i = 0; i < N; ++i) {
+    const float* x = X + i * (int64_t)d;
+    double* dx = dX + i * (int64_t)d;
+    int64_t q_lo, q_hi;
+    for (int32_t r = 0; r < n_r; ++r) {
+      window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+      for (int64_t q = q_lo; q < q_hi; ++q) {
+        int32_t j = permY[(int64_t)r * C + q];
+        if (j != target[i]) ++cnt[j];
+      }
+    }
+    const float* yz = Y + (int64_t)target[i] * d;
+    double gp = (exp(dot_f64(x, yz, d) - lse[i]) - 1.0) * scale;
+    for (int32_t t = 0; t < d; ++t) dx[t] = gp * (double)yz[t];
+    double* dyz = dY + (int64_t)target[i] * d;
+    for (int32_t t = 0; t < d; ++t) dyz[t] += gp * (double)x[t];
+    for (int32_t r = 0; r < n_r; ++r) {
+      window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+      for (int64_t q = q_lo; q < q_hi; ++q) {
+        int32_t j = permY[(int64_t)r * C + q];
+        if (j == target[i]) continue;
+        const float* y = Y + (int64_t)j * d;
+        double g = exp(dot_f64(x, y, d) - log((double)cnt[j]) - lse[i]) * scale;
+        double* dy = dY + (int64_t)j * d;
+        for (int32_t t = 0; t < d; ++t) {
+          dx[t] += g * (double)y[t];
+          dy[t] += g * (double)x[t];
+        }
+      }
+    }
+    for (int32_t r = 0; r < n_r; ++r) {
+      window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
+      for (int64_t q = q_lo; q < q_hi; ++q) cnt[permY[(int64_t)r * C + q]] = 0;
+    }
+  }
+  free(cnt);
+  free(posX);
+}
+
 /* log(1 + exp(u)) without overflow: for u > 0 it is u + log(1 + exp(-u)). */
 static double softplus(double u) { return u > 0.0 ? u + log1p(exp(-u)) : log1p(exp(u)); }
 

@@ -490,3 +490,67 @@ def test_memory_model_matches_the_stated_ratio():
         assert N * C / model == pytest.approx(ratio, rel=1e-12)
     # the minimised quantity: at alpha_bc = 1, n_ec = 0, r = 1, min = max = M: 2 M^1.5
     assert oracle.memory_model_elements(400, 400, 0, 1, 1.0) == pytest.approx(2 * 400 ** 1.5)
+
+
+# --------------------------------------------------------------------------- Algorithm 1 as printed
+@pytest.mark.parametrize("n_c,n_ec,n_r", [(4, 1, 2), (5, 0, 3), (3, 2, 1), (6, 1, 2)])
+def test_window_loss_ln_count_equals_deduplicated_union(n_c, n_ec, n_r):
+    """The rounds paragraph's ln(count) correction makes every duplicated pair count once:
+    the literal loss equals the top-k path with k at least the number of candidates (the
+    de-duplicated union), a separately written selection-based oracle."""
+    X, Y, z, B = _random_case(N=48, C=120, d=8, n_b=3, n_c=n_c, n_r=n_r, seed=n_c + n_r)
+    top = oracle.rece_forward(X, Y, z, B, n_c, n_ec, len(Y))
+    assert np.all(top["n_cand"] <= len(Y))
+    loss, row, lse = oracle.window_loss(X, Y, z, top["permX"], top["permY"], n_c, n_ec)
+    np.testing.assert_allclose(row, top["row_loss"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, top["lse"], rtol=1e-13)
+    dX, dY = oracle.window_grad(X, Y, z, top["permX"], top["permY"], n_c, n_ec, lse, 0.8)
+    tX, tY = oracle.rece_grad(X, Y, z, top["selected"], top["lse"], 0.8)
+    assert rel_err(dX, tX) < 1e-12 and rel_err(dY, tY) < 1e-12
+
+
+def test_window_loss_one_bucket_one_chunk_is_full_ce():
+    X, Y, z, B = _random_case(N=30, C=70, d=6, n_b=1, n_c=1, n_r=2)
+    top = oracle.rece_forward(X, Y, z, B, 1, 0, 1)
+    loss, row, lse = oracle.window_loss(X, Y, z, top["permX"], top["permY"], 1, 0)
+    f_loss, f_row, f_lse = oracle.full_ce_loss(X, Y, z)
+    np.testing.assert_allclose(row, f_row, rtol=1e-12)
+    dX, dY = oracle.window_grad(X, Y, z, top["permX"], top["permY"], 1, 0, lse)
+    fX, fY = oracle.full_ce_grad(X, Y, z, f_lse)
+    assert rel_err(dX, fX) < 1e-12 and rel_err(dY, fY) < 1e-12
+
+
+def test_window_loss_identical_rounds_equal_one_round():
+    """r identical rounds compute every pair r times, each copy weighted by 1/r."""
+    X, Y, z, B = _random_case(N=40, C=100, d=8, n_b=4, n_c=4, n_r=1)
+    one = oracle.rece_forward(X, Y, z, B, 4, 1, 1)
+    three_px = np.repeat(one["permX"], 3, 0)
+    three_py = np.repeat(one["permY"], 3, 0)
+    _, r1, l1 = oracle.window_loss(X, Y, z, one["permX"], one["permY"], 4, 1)
+    _, r3, l3 = oracle.window_loss(X, Y, z, three_px, three_py, 4, 1)
+    np.testing.assert_allclose(r3, r1, rtol=1e-12)
+    g1 = oracle.window_grad(X, Y, z, one["permX"], one["permY"], 4, 1, l1)
+    g3 = oracle.window_grad(X, Y, z, three_px, three_py, 4, 1, l3)
+    assert rel_err(g3[0], g1[0]) < 1e-12 and rel_err(g3[1], g1[1]) < 1e-12
+
+
+def test_window_grad_finite_differences_and_invariants():
+    X, Y, z, B = _dyadic_case(N=6, C=20, d=3)
+    top = oracle.rece_forward(X, Y, z, B, 3, 0, 1)
+    px, py = top["permX"], top["permY"]
+    _, _, lse = oracle.window_loss(X, Y, z, px, py, 3, 0)
+    dloss = 0.9
+    dX, dY = oracle.window_grad(X, Y, z, px, py, 3, 0, lse, dloss)
+    h = 2.0 ** -10
+    for name, A, G in (("X", X, dX), ("Y", Y, dY)):
+        for idx in np.ndindex(A.shape):
+            ls = []
+            for sgn in (+1, -1):
+                P = A.copy()
+                P[idx] = P[idx] + np.float32(sgn * h)
+                XX, YY = (P, Y) if name == "X" else (X, P)
+                ls.append(oracle.window_loss(XX, YY, z, px, py, 3, 0)[0])
+            fd = dloss * (ls[0] - ls[1]) / (2 * h)
+            assert fd == pytest.approx(G[idx], abs=1e-6 * max(1.0, np.abs(G).max()))
+    # every row's coefficients sum to zero -> the dY rows sum to the zero vector
+    assert np.abs(dY.sum(0)).max() < 1e-12
