@@ -71,6 +71,16 @@ typedef enum {
 /* rece_config_t.flags */
 #define RECE_FLAG_FMA_SCORES 0x1u /* bf16 mode: use the fmaf-chain CUDA-core kernels for
                                      the scores as well (bit-exact on bf16 inputs) */
+/* Algorithm 1 as printed [RECE section 3]: every item of a row's chunk windows is a
+ * negative (no top-k; k is not used), and a pair computed in cnt of the n_r rounds
+ * enters each round's sum as exp(l - ln cnt) [the rounds paragraph], the positive left
+ * out of the window sums (it enters once, as l+):
+ *   lse_i = log(exp(l+) + sum_r sum_{j in W_r(i), j != z_i} exp(l_ij) / cnt_ij).
+ * The window sums are formed on the tcgen05 tensor cores and never stored; the backward
+ * recomputes them.  bf16 mode, d a multiple of 64 and at most 256 (else
+ * RECE_ERR_UNSUPPORTED).  rece_loss_fwd writes no logits and fills `selected` (which may
+ * be NULL) with -1; rece_loss_bwd ignores `selected` and `logits` (either may be NULL). */
+#define RECE_FLAG_ALL_NEGATIVES 0x2u
 
 /* Bits of the device status word (rece_get_device_status). */
 #define RECE_DEVICE_BAD_TARGET 0x1u /* some target outside [0, C) */
@@ -128,11 +138,13 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
  *   RECE_PATH_DX_TENSORS    dX of the backward as tcgen05 band products (large d or a
  *                           catalogue beyond half of L2; else gathered rows);
  *   RECE_PATH_STORED_SCORES window scores computed once and stored, then selected row by
- *                           row (d >= 1024; else recomputed in the fused selection).
+ *                           row (d >= 1024; else recomputed in the fused selection);
+ *   RECE_PATH_ALL_NEGATIVES the all-negatives mode (RECE_FLAG_ALL_NEGATIVES).
  * RECE_ERR_INVALID_ARG for a NULL argument. */
 #define RECE_PATH_TENSOR_CORES 0x1u
 #define RECE_PATH_DX_TENSORS 0x2u
 #define RECE_PATH_STORED_SCORES 0x4u
+#define RECE_PATH_ALL_NEGATIVES 0x8u  /* RECE_FLAG_ALL_NEGATIVES: window sums on tcgen05 */
 RECE_API rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths);
 
 /* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].

@@ -88,7 +88,56 @@ void set_pair_sort(rece_plan_s& p) {
   p.carry_g = p.entries * int64_t(sizeof(float)) > (int64_t(32) << 20);
 }
 
+// All-negatives mode: what the backward reads stays from rece_bucketize_sort on (sorted
+// copies, their d-major copies, orders, chunk tables, positives' sorted positions, lse by
+// round); the forward's scratch and the positives' pair arrays share the rest.
+void build_layout_all_neg(rece_plan_s& p) {
+  const auto& c = p.cfg;
+  Layout& L = p.lay;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.status = take(4 * sizeof(uint32_t));
+  const size_t nb_stride = (size_t(1) << p.bucket_bits) + 1;
+  const size_t nr = size_t(c.n_r);
+  L.px = take(sizeof(int32_t) * nr * c.N);
+  L.py = take(sizeof(int32_t) * nr * c.C);
+  L.xs = take(sizeof(uint16_t) * nr * c.N * c.d);
+  L.ys = take(sizeof(uint16_t) * nr * c.C * c.d);
+  L.xst = take(sizeof(uint16_t) * nr * c.d * p.ld_n);
+  L.yst = take(sizeof(uint16_t) * nr * c.d * p.ld_c);
+  L.itemc = take(sizeof(int32_t) * nr * nr * c.C);
+  L.rowc = take(sizeof(int32_t) * nr * nr * c.N);
+  L.pz = take(sizeof(int32_t) * nr * c.N);
+  L.lse_sorted = take(sizeof(float) * nr * c.N);
+  const size_t region = off;
+  L.bx = take(sizeof(int32_t) * nr * c.N);
+  L.by = take(sizeof(int32_t) * nr * c.C);
+  L.bstart_x = take(sizeof(int32_t) * nr * nb_stride);
+  L.bstart_y = take(sizeof(int32_t) * nr * nb_stride);
+  L.sort_scratch = take(nr * (sort_hist_bytes(c.N, p.bucket_bits) +
+                              sort_hist_bytes(c.C, p.bucket_bits)));
+  L.inv_x = take(sizeof(int32_t) * nr * c.N);
+  L.inv_y = take(sizeof(int32_t) * nr * c.C);
+  L.ms = take(sizeof(float) * 2 * nr * c.N);
+  L.row_loss_tmp = take(sizeof(float) * c.N);
+  L.fwd_end = off;
+  off = region;
+  rece_plan_s& q = *p.pos_plan;
+  q.lay.status = L.status;
+  layout_pairs(q, off);
+  L.bwd_end = off;
+  L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
+}
+
 void build_layout(rece_plan_s& p) {
+  if (p.all_neg) {
+    build_layout_all_neg(p);
+    return;
+  }
   const auto& c = p.cfg;
   Layout& L = p.lay;
   size_t off = 0;
@@ -194,6 +243,76 @@ rece_status_t sampled_plan(int32_t kind, int64_t N, int64_t C, int32_t d, int32_
   return RECE_OK;
 }
 
+// Forward of the all-negatives mode: chunk tables, the rounds' window sums on the tensor
+// cores, their combination with l+, the mean.  `selected`, when given, is set to -1 (no
+// subset is chosen); the logits are not produced.
+rece_status_t all_neg_fwd(const rece_plan_s& p, const void* X, const void* Y,
+                          const int32_t* targets, char* ws, float* loss, float* row_loss,
+                          int32_t* selected, float* lse, cudaStream_t st) {
+  const auto& c = p.cfg;
+  const Layout& L = p.lay;
+  auto I = [&](size_t o) { return reinterpret_cast<int32_t*>(ws + o); };
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + L.row_loss_tmp);
+  float2* ms = reinterpret_cast<float2*>(ws + L.ms);
+  stage_mark(p, RECE_STAGE_SELECT, 0, st);
+  RECE_CUDA(launch_window_meta(I(L.py), I(L.inv_y), c.C, c.n_c, c.n_r, I(L.itemc), nullptr,
+                               nullptr, c.C, nullptr, st),
+            "item chunk tables");
+  RECE_CUDA(launch_window_meta(I(L.px), I(L.inv_x), c.N, c.n_c, c.n_r, I(L.rowc), targets,
+                               I(L.inv_y), c.C, I(L.pz), st),
+            "row chunk tables");
+  RECE_CUDA(launch_window_lse_tc(p, ws + L.xs, ws + L.ys, I(L.itemc), I(L.rowc), I(L.pz), ms,
+                                 status, st),
+            "window sums (tcgen05)");
+  stage_mark(p, RECE_STAGE_SELECT, 1, st);
+  stage_mark(p, RECE_STAGE_MERGE_LOSS, 0, st);
+  RECE_CUDA(launch_window_combine(p, static_cast<const __nv_bfloat16*>(X),
+                                  static_cast<const __nv_bfloat16*>(Y), targets, I(L.inv_x), ms,
+                                  lse, rl, reinterpret_cast<float*>(ws + L.lse_sorted), status,
+                                  st),
+            "rounds' log-sum-exp");
+  if (selected && c.N > 0)
+    RECE_CUDA(cudaMemsetAsync(selected, 0xFF, sizeof(int32_t) * size_t(c.N) * c.k, st),
+              "selected");
+  stage_mark(p, RECE_STAGE_MERGE_LOSS, 1, st);
+  stage_mark(p, RECE_STAGE_MEAN, 0, st);
+  RECE_CUDA(launch_mean(rl, c.N, loss, st), "mean");
+  stage_mark(p, RECE_STAGE_MEAN, 1, st);
+  return RECE_OK;
+}
+
+// Backward of the all-negatives mode: the positives' terms (written), then the window
+// terms of dX and of dY, added round by round.
+rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
+                          const int32_t* targets, const float* lse, const float* dloss,
+                          char* ws, float* dX, float* dY, cudaStream_t st) {
+  const auto& c = p.cfg;
+  const Layout& L = p.lay;
+  auto I = [&](size_t o) { return reinterpret_cast<const int32_t*>(ws + o); };
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  const float* ls = reinterpret_cast<const float*>(ws + L.lse_sorted);
+  stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
+  RECE_CUDA(launch_backward(*p.pos_plan, static_cast<const __nv_bfloat16*>(X),
+                            static_cast<const __nv_bfloat16*>(Y), targets, nullptr, lse, nullptr,
+                            dloss, ws, dX, dY, status, st),
+            "positives' backward");
+  RECE_CUDA(launch_window_grad_tc(p, false, ws + L.xs, ws + L.ys, ws + L.xst, ws + L.yst,
+                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.px), dloss, dX, status,
+                                  st),
+            "window dX (tcgen05)");
+  stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
+  stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
+  stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
+  stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
+  RECE_CUDA(launch_window_grad_tc(p, true, ws + L.xs, ws + L.ys, ws + L.xst, ws + L.yst,
+                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.py), dloss, dY, status,
+                                  st),
+            "window dY (tcgen05)");
+  stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
+  return RECE_OK;
+}
+
 }  // namespace
 
 void rece::set_last_error(const char* msg) { fail(RECE_OK, msg); }
@@ -231,7 +350,8 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     return fail(RECE_ERR_INVALID_ARG, "n_c must be in [1, min(N, C)]");
   if (c.mode != RECE_MODE_FP32_EXACT && c.mode != RECE_MODE_BF16)
     return fail(RECE_ERR_INVALID_ARG, "unknown mode");
-  if ((c.flags & ~RECE_FLAG_FMA_SCORES) != 0) return fail(RECE_ERR_INVALID_ARG, "unknown flag");
+  if ((c.flags & ~(RECE_FLAG_FMA_SCORES | RECE_FLAG_ALL_NEGATIVES)) != 0)
+    return fail(RECE_ERR_INVALID_ARG, "unknown flag");
   if (c.N * (int64_t(c.k) + 1) >= kInt32Max || c.N * c.n_r >= kInt32Max ||
       c.C * c.n_r >= kInt32Max || c.N * c.d >= (int64_t(1) << 40))
     return fail(RECE_ERR_UNSUPPORTED, "sizes exceed 32-bit pair indexing");
@@ -271,6 +391,9 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     if (sl > p->kept_slices) p->kept_slices = int32_t(sl);
   }
   p->ld_c = (c.C + 7) / 8 * 8;
+  p->ld_n = (c.N + 7) / 8 * 8;
+  p->all_neg = (c.flags & RECE_FLAG_ALL_NEGATIVES) != 0;
+  p->pos_plan = nullptr;
   // the tensor-core path groups each row's kept entries by slice of its window
   // (the selection's 16-bit histogram counts hold windows of fewer than 65536 items)
   p->use_tc = tc_supported(*p) && p->w_max < 65536;
@@ -283,7 +406,30 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   p->score_width = p->tc_scores ? scores_tc_width(*p) : 0;
   p->tc_dx = p->use_tc && p->kept_slices <= kMaxKeptSlices &&
              (c.d >= 256 || 2.0 * double(c.C) * c.d > 64.0 * 1024 * 1024);
-  if (p->use_tc && merge_tc_warp_bytes(c.n_r, c.k) > 200 * 1024) {
+  if (p->all_neg) {
+    if (!window_tc_supported(*p)) {
+      delete p;
+      return fail(RECE_ERR_UNSUPPORTED,
+                  "all-negatives mode needs bf16 on tcgen05 with d a multiple of 64, <= 256");
+    }
+    p->tc_dx = false;
+    p->tc_scores = false;
+    p->score_width = 0;
+    // the positives' coefficients and their dY go through the pair backward (k = 0)
+    rece_plan_s* q = new (std::nothrow) rece_plan_s();
+    if (!q) {
+      delete p;
+      return fail(RECE_ERR_INVALID_ARG, "out of host memory");
+    }
+    *q = *p;
+    q->cfg.k = 0;
+    q->all_neg = false;
+    q->use_tc = false;
+    q->timed = false;
+    q->pos_plan = nullptr;
+    set_pair_sort(*q);
+    p->pos_plan = q;
+  } else if (p->use_tc && merge_tc_warp_bytes(c.n_r, c.k) > 200 * 1024) {
     delete p;
     return fail(RECE_ERR_UNSUPPORTED, "n_r * k too large for the tensor-core merge");
   }
@@ -292,7 +438,10 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   return RECE_OK;
 }
 
-void rece_plan_destroy(rece_plan_t plan) { delete plan; }
+void rece_plan_destroy(rece_plan_t plan) {
+  if (plan) delete plan->pos_plan;
+  delete plan;
+}
 
 rece_status_t rece_plan_set_stage_events(rece_plan_t plan, void* const* events) {
   if (!plan) return fail(RECE_ERR_INVALID_ARG, "plan is NULL");
@@ -331,7 +480,8 @@ rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
   if (!plan || !paths) return fail(RECE_ERR_INVALID_ARG, "NULL argument");
   *paths = (plan->use_tc ? RECE_PATH_TENSOR_CORES : 0u) |
            (plan->tc_dx ? RECE_PATH_DX_TENSORS : 0u) |
-           (plan->tc_scores ? RECE_PATH_STORED_SCORES : 0u);
+           (plan->tc_scores ? RECE_PATH_STORED_SCORES : 0u) |
+           (plan->all_neg ? RECE_PATH_ALL_NEGATIVES : 0u);
   return RECE_OK;
 }
 
@@ -387,7 +537,20 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   }
   RECE_CUDA(launch_sort_batch(segs, 2 * c.n_r, 0, plan->bucket_bits, false, st),
             "sort X and Y");
-  if (plan->use_tc) {
+  if (plan->all_neg) {
+    RECE_CUDA(launch_permute_rows(X, c.N, c.d, reinterpret_cast<const int32_t*>(ws + L.px),
+                                  c.n_r, c.n_c, ws + L.xs,
+                                  reinterpret_cast<int32_t*>(ws + L.inv_x), nullptr, st),
+              "permute X");
+    RECE_CUDA(launch_permute_rows(Y, c.C, c.d, reinterpret_cast<const int32_t*>(ws + L.py),
+                                  c.n_r, c.n_c, ws + L.ys,
+                                  reinterpret_cast<int32_t*>(ws + L.inv_y), nullptr, st),
+              "permute Y");
+    RECE_CUDA(launch_transpose_sorted(ws + L.xs, c.N, c.d, c.n_r, plan->ld_n, ws + L.xst, st),
+              "d-major copy of X");
+    RECE_CUDA(launch_transpose_sorted(ws + L.ys, c.C, c.d, c.n_r, plan->ld_c, ws + L.yst, st),
+              "d-major copy of Y");
+  } else if (plan->use_tc) {
     RECE_CUDA(launch_permute_rows(X, c.N, c.d, reinterpret_cast<const int32_t*>(ws + L.px),
                                   c.n_r, c.n_c, ws + L.xs,
                                   reinterpret_cast<int32_t*>(ws + L.inv_x), nullptr, st),
@@ -411,11 +574,12 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
   rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
   if (s != RECE_OK) return s;
   const auto& c = plan->cfg;
-  if (!loss || !Y || (c.N > 0 && (!X || !targets || !selected || !lse)))
+  if (!loss || !Y || (c.N > 0 && (!X || !targets || (!selected && !plan->all_neg) || !lse)))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const Layout& L = plan->lay;
+  if (plan->all_neg) return all_neg_fwd(*plan, X, Y, targets, ws, loss, row_loss, selected, lse, st);
   const int32_t* px = reinterpret_cast<const int32_t*>(ws + L.px);
   const int32_t* py = reinterpret_cast<const int32_t*>(ws + L.py);
   float* ls = reinterpret_cast<float*>(ws + L.list_score);
@@ -483,11 +647,13 @@ rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
   rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);
   if (s != RECE_OK) return s;
   const auto& c = plan->cfg;
-  if (!Y || !dY || (c.N > 0 && (!X || !targets || !selected || !lse || !dloss || !dX)))
+  if (!Y || !dY ||
+      (c.N > 0 && (!X || !targets || (!selected && !plan->all_neg) || !lse || !dloss || !dX)))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan->lay.status);
+  if (plan->all_neg) return all_neg_bwd(*plan, X, Y, targets, lse, dloss, ws, dX, dY, st);
   if (c.mode == RECE_MODE_FP32_EXACT)
     RECE_CUDA(launch_backward(*plan, static_cast<const float*>(X), static_cast<const float*>(Y),
                               targets, selected, lse, logits, dloss, ws, dX, dY, status, st),

@@ -78,4 +78,31 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
                          const float* lse, const float* dloss, char* ws, float* dX,
                          uint32_t* status, cudaStream_t st);
 
+// All-negatives mode (Algorithm 1 as printed; window.cu, window_tc.cu).  Per-round chunk
+// tables chunks[(r * n_r + s) * M + p] of the row (item) at sorted position p of round r,
+// and for the rows the sorted position of their positive (pz [n_r][N], -1 for none).
+cudaError_t launch_window_meta(const int32_t* perm, const int32_t* inv, int64_t M, int n_c,
+                               int n_r, int32_t* chunks, const int32_t* targets,
+                               const int32_t* invY, int64_t C, int32_t* pz, cudaStream_t st);
+// bf16, d a multiple of 64 up to 256, at most 8 rounds.
+bool window_tc_supported(const rece_plan_s& p);
+// ms [n_r][N]: per round and sorted row, (max, sum) of exp(s)/cnt over its window terms.
+cudaError_t launch_window_lse_tc(const rece_plan_s& p, const void* Xs, const void* Ys,
+                                 const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
+                                 float2* ms, uint32_t* status, cudaStream_t st);
+// lse and row losses from l+ and the rounds' (max, sum); lse also per round, sorted.
+template <typename T>
+cudaError_t launch_window_combine(const rece_plan_s& p, const T* X, const T* Y,
+                                  const int32_t* targets, const int32_t* invX, const float2* ms,
+                                  float* lse, float* row_loss, float* lse_sorted,
+                                  uint32_t* status, cudaStream_t st);
+// The window terms of dX (dy = false, perm = px) or dY (dy = true, perm = py), added
+// into `out` round by round.
+cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
+                                  const void* Ys, const void* XsT, const void* YsT,
+                                  const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
+                                  const float* lse_sorted, const int32_t* perm,
+                                  const float* dloss, float* out, uint32_t* status,
+                                  cudaStream_t st);
+
 }  // namespace rece

@@ -175,3 +175,16 @@ def test_sampled_workspace_and_validation():
     one = ctypes.c_void_p(256)
     assert L.rece_sampled_fwd(0, 10, 10, 8, 1, 0, one, one, one, one, one, 16, one, None,
                               None, one, None) == 3
+
+
+def test_all_negatives_mode_support():
+    flags = _lib.FLAG_ALL_NEGATIVES
+    p = Plan(1000, 5000, 128, 16, 8, 1, 2, 8, mode="bf16", flags=flags)
+    assert p.paths == _lib.PATH_TENSOR_CORES | _lib.PATH_ALL_NEGATIVES
+    assert p.workspace_bytes > 0
+    for bad in (dict(mode="fp32"), dict(d=512), dict(d=96)):
+        kw = dict(N=1000, C=5000, d=128, n_b=16, n_c=8, n_ec=1, n_r=2, k=8, mode="bf16")
+        kw.update(bad)
+        with pytest.raises(RuntimeError):
+            Plan(kw["N"], kw["C"], kw["d"], kw["n_b"], kw["n_c"], kw["n_ec"], kw["n_r"],
+                 kw["k"], mode=kw["mode"], flags=flags)
