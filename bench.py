@@ -82,10 +82,26 @@ def pairs_per_round(w):
     return tot
 
 
-def stage_work(w):
+def stage_work(w, paths=0):
     """Algorithmic (flops, bytes) of every stage, per step (one launch sequence)."""
+    from reduced_cross_entropy_b200 import _lib
     e = 2 if w.dtype == "bf16" else 4
     N, C, d, nb, nr, k = w.N, w.C, w.d, w.n_b, w.n_r, w.k
+    if paths & _lib.PATH_ALL_NEGATIVES:
+        # Algorithm 1 as printed: every window pair scored in the forward, and in the
+        # backward scored again and multiplied twice (dX = P Y, dY = P^T X); the positives
+        # through the pair backward
+        pr = pairs_per_round(w) * nr
+        return {
+            "bucketize": (2 * (N + C) * nb * d * nr, nr * (N + C) * (d * e + 4)),
+            "sort": (0, nr * (N + C) * (16 + 2 * d * e)),
+            "select": (2 * d * pr, nr * (N + C) * d * e + 8 * nr * N),
+            "merge_loss": (0, 8 * nr * N + 2 * N * d * e + 8 * N),
+            "mean": (0, 4 * N),
+            "bwd_rows": (4 * d * pr + 2 * N * d, nr * (N + C) * d * e + 2 * N * d * 4),
+            "bwd_sort": (0, 0),
+            "bwd_items": (4 * d * pr, nr * (N + C) * d * e + 2 * C * d * 4),
+        }
     return {
         "bucketize": (2 * (N + C) * nb * d * nr, nr * (N + C) * (d * e + 4)),
         "sort": (0, nr * (N + C) * 16),
@@ -104,6 +120,8 @@ def stage_bound(stage, paths):
     from reduced_cross_entropy_b200 import _lib
     if stage in ("bucketize", "select"):
         return "tensor" if paths & _lib.PATH_TENSOR_CORES else "alu"
+    if stage in ("bwd_rows", "bwd_items") and paths & _lib.PATH_ALL_NEGATIVES:
+        return "tensor"
     if stage == "bwd_rows" and paths & _lib.PATH_DX_TENSORS:
         return "tensor"
     return "hbm"
@@ -127,6 +145,10 @@ def kernel_sources(stage, paths):
         src["select"] = ["scores_tc.cu", "sm100.cuh", "tc_bins.cuh"]
     if paths & _lib.PATH_DX_TENSORS:
         src["bwd_rows"] = ["backward.cu", "bwd_tc.cu", "sm100.cuh"]
+    if paths & _lib.PATH_ALL_NEGATIVES:
+        src.update(select=["window_tc.cu", "window.cu", "sm100.cuh"],
+                   merge_loss=["window.cu"], bwd_rows=["backward.cu", "window_tc.cu"],
+                   bwd_sort=["sort.cu"], bwd_items=["window_tc.cu"])
     return src[stage]
 
 
@@ -206,7 +228,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_step_seconds(w, X, Y, t, B, rows=256, bucket_frac=16):
+def oracle_step_seconds(w, X, Y, t, B, rows=256, bucket_frac=16, all_negatives=False):
     """Estimated seconds of one whole step of the CPU oracle, from a bounded sample:
     bucketing of every bucket_frac-th row of X and Y (scaled up), the full stable sorts,
     and selection + loss + gradient of `rows` rows (scaled by N / rows)."""
@@ -229,6 +251,10 @@ def oracle_step_seconds(w, X, Y, t, B, rows=256, bucket_frac=16):
     t_sort = time.perf_counter() - t0
     sample = np.linspace(0, w.N - 1, rows).astype(np.int64)
     t0 = time.perf_counter()
+    if all_negatives:  # Algorithm 1 as printed: every window item a negative
+        _, _, lse = oracle.window_loss(X, Y, t, px, py, w.n_c, w.n_ec, rows=sample)
+        oracle.window_grad(X, Y, t, px, py, w.n_c, w.n_ec, lse, 1.0, rows=sample)
+        return t_bucket + t_sort + (time.perf_counter() - t0) * w.N / rows
     sel, _, _ = oracle.select(X, Y, t, px, py, w.n_c, w.n_ec, w.k, rows=sample)
     _, _, lse = oracle.rece_loss(X[sample], Y, t[sample], sel)
     oracle.rece_grad(X[sample], Y, t[sample], sel, lse, 1.0)
@@ -251,9 +277,11 @@ def run_reference(args):
     X, Y, t = synth.make_inputs(w, seed=0)
     B = synth.projections(0, 0, w.n_r, w.n_b, w.d, w.dtype)
     rows, frac = 128, 32
+    alln = bool(args.flags & 0x2)  # RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed
     for _ in range(args.warmup):
-        oracle_step_seconds(w, X, Y, t, B, rows, frac)
-    secs = [oracle_step_seconds(w, X, Y, t, B, rows, frac) for _ in range(args.steps)]
+        oracle_step_seconds(w, X, Y, t, B, rows, frac, all_negatives=alln)
+    secs = [oracle_step_seconds(w, X, Y, t, B, rows, frac, all_negatives=alln)
+            for _ in range(args.steps)]
     total = sum(secs)
     value = w.N * args.steps / total
     cores = oracle.num_threads()
@@ -400,13 +428,13 @@ def main():
 
     # roofline of every stage, the dominant one reported as the line's roofline
     peaks = load_peaks()
-    work = stage_work(w)
     paths = plan.paths
+    work = stage_work(w, paths)
 
     def stage_roofline(name):
         bound = stage_bound(name, paths)
         flops, bytes_ = work[name]
-        sec = stage_ms[name] / 1000.0
+        sec = max(stage_ms[name], 1e-9) / 1000.0
         if bound == "hbm":
             achieved, peak, unit = bytes_ / sec / 1e9, peaks["hbm_gbs"], "GB/s"
         elif bound == "tensor":
@@ -465,7 +493,11 @@ def main():
                                                  else ", recomputed per pass")
                                   if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),
                        "dX": "tcgen05 band products" if paths & _lib.PATH_DX_TENSORS
-                       else "gathered rows"},
+                       else "gathered rows",
+                       "negatives": ("every window item (Algorithm 1 as printed), window "
+                                     "sums and gradients on tcgen05"
+                                     if paths & _lib.PATH_ALL_NEGATIVES
+                                     else f"top-{w.k} per row")},
             "roofline": roofline, "stages_ms": stage_ms, "stages_roofline_frac": stage_fracs,
             "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk.summary()}
@@ -479,7 +511,8 @@ def main():
         import oracle
         rows, frac = 256, 16
         secs = oracle_step_seconds(w, X, Y, t, synth.projections(0, 0, w.n_r, w.n_b, w.d,
-                                                                   w.dtype), rows, frac)
+                                                                   w.dtype), rows, frac,
+                                   all_negatives=bool(paths & _lib.PATH_ALL_NEGATIVES))
         line["cpu_baseline"] = {"value": w.N / secs, "unit": "rows/s",
                                 "cores": oracle.num_threads(), "kind": "oracle",
                                 "sample": oracle_sample_desc(rows, frac)}

@@ -69,10 +69,11 @@ def _load():
                                             f64p, ctypes.c_double, f64p, f64p]
         lib.oracle_sampled_grad.restype = None
         lib.oracle_window_loss.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32,
-                                           i32p, i32p, f64p, f64p, f64p]
+                                           i32p, i32p, i64p_or_null, i64, f64p, f64p, f64p]
         lib.oracle_window_loss.restype = None
         lib.oracle_window_grad.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32,
-                                           i32p, i32p, f64p, ctypes.c_double, f64p, f64p]
+                                           i32p, i32p, i64p_or_null, i64, f64p,
+                                           ctypes.c_double, f64p, f64p]
         lib.oracle_window_grad.restype = None
         lib.oracle_dot_f32.argtypes = [f32p, f32p, i32]
         lib.oracle_dot_f32.restype = ctypes.c_float
@@ -239,35 +240,48 @@ def sampled_grad(kind, X, Y, target, negatives, lse, dloss=1.0):
     return dX, dY
 
 
-def window_loss(X, Y, target, permX, permY, n_c, n_ec):
+def _rows_arg(rows, N):
+    if rows is None:
+        return None, N
+    r = np.ascontiguousarray(rows, np.int64)
+    return r.ctypes.data_as(ctypes.c_void_p), len(r)
+
+
+def window_loss(X, Y, target, permX, permY, n_c, n_ec, rows=None):
     """Algorithm 1 as printed (every window item a negative) over the rounds' stable
     orders permX [n_r, N], permY [n_r, C], duplicates across rounds corrected by
-    ln(count).  Returns (loss, row_loss, lse)."""
+    ln(count).  rows: optional sample of row ids (outputs follow the sample, the mean is
+    over it).  Returns (loss, row_loss, lse)."""
     X, Y, target = _f32(X), _f32(Y), _i32(target)
     permX, permY = _i32(permX), _i32(permY)
     N, d = X.shape
     n_r = permY.shape[0]
-    row = np.empty(N, np.float64)
-    lse = np.empty(N, np.float64)
+    keep = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    rp, n = _rows_arg(keep, N)
+    row = np.empty(n, np.float64)
+    lse = np.empty(n, np.float64)
     loss = np.zeros(1, np.float64)
     _load().oracle_window_loss(X, Y, target, N, Y.shape[0], d, n_c, n_ec, n_r,
                                permX.reshape(-1) if N else np.zeros(1, np.int32),
-                               permY.reshape(-1), row, lse, loss)
+                               permY.reshape(-1), rp, n, row, lse, loss)
     return float(loss[0]), row, lse
 
 
-def window_grad(X, Y, target, permX, permY, n_c, n_ec, lse, dloss=1.0):
-    """(dX, dY) of window_loss, the buckets and windows held constant (fp64)."""
+def window_grad(X, Y, target, permX, permY, n_c, n_ec, lse, dloss=1.0, rows=None):
+    """(dX, dY) of window_loss, the buckets and windows held constant (fp64); with a
+    row sample, dX follows the sample and dY sums over it."""
     X, Y, target = _f32(X), _f32(Y), _i32(target)
     permX, permY = _i32(permX), _i32(permY)
     N, d = X.shape
     C = Y.shape[0]
     n_r = permY.shape[0]
-    dX = np.empty((N, d), np.float64)
+    keep = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    rp, n = _rows_arg(keep, N)
+    dX = np.empty((n, d), np.float64)
     dY = np.empty((C, d), np.float64)
     _load().oracle_window_grad(X, Y, target, N, C, d, n_c, n_ec, n_r,
                                permX.reshape(-1) if N else np.zeros(1, np.int32),
-                               permY.reshape(-1), np.ascontiguousarray(lse, np.float64),
+                               permY.reshape(-1), rp, n, np.ascontiguousarray(lse, np.float64),
                                float(dloss), dX, dY)
     return dX, dY
 

@@ -314,7 +314,9 @@ void oracle_full_ce_grad(const float* X, const float* Y, const int32_t* target, 
  * the window sums (it enters once, as l+):
  *   lse_i  = log(exp(l+) + sum_r sum_{j in W_r(i), j != z_i} exp(l_ij - ln cnt_ij))
  *   loss_i = lse_i - l+,   L = mean_i loss_i          (fp64)
- * permX [n_r*N], permY [n_r*C]: the rounds' stable bucket orders. */
+ * permX [n_r*N], permY [n_r*C]: the rounds' stable bucket orders.  rows [n_rows]: the
+ * rows to compute (NULL: all N, n_rows = N); outputs are indexed by the sample, and the
+ * mean is over the sample.  The gradient takes the same sample (dY sums over it). */
 static void window_of(int64_t i, int32_t r, const int64_t* posX, int64_t N, int64_t C,
                       int32_t n_c, int32_t n_ec, int64_t* q_lo, int64_t* q_hi) {
   int64_t c = chunk_of(posX[(int64_t)r * N + i], N, n_c);
@@ -333,14 +335,15 @@ static int64_t* positions(const int32_t* permX, int64_t N, int32_t n_r) {
 
 void oracle_window_loss(const float* X, const float* Y, const int32_t* target, int64_t N,
                         int64_t C, int32_t d, int32_t n_c, int32_t n_ec, int32_t n_r,
-                        const int32_t* permX, const int32_t* permY, double* row_loss,
-                        double* lse, double* loss) {
+                        const int32_t* permX, const int32_t* permY, const int64_t* rows,
+                        int64_t n_rows, double* row_loss, double* lse, double* loss) {
   int64_t* posX = positions(permX, N, n_r);
 #pragma omp parallel
   {
     int32_t* cnt = (int32_t*)calloc((size_t)C, sizeof(int32_t));
 #pragma omp for schedule(dynamic, 16)
-    for (int64_t i = 0; i < N; ++i) {
+    for (int64_t o = 0; o < n_rows; ++o) {
+      const int64_t i = rows ? rows[o] : o;
       const float* x = X + i * (int64_t)d;
       int64_t q_lo, q_hi;
       /* how many rounds compute each pair of this row */
@@ -371,8 +374,8 @@ void oracle_window_loss(const float* X, const float* Y, const int32_t* target, i
           s += exp(dot_f64(x, Y + (int64_t)j * d, d) - log((double)cnt[j]) - m);
         }
       }
-      lse[i] = m + log(s);
-      row_loss[i] = lse[i] - lp;
+      lse[o] = m + log(s);
+      row_loss[o] = lse[o] - lp;
       for (int32_t r = 0; r < n_r; ++r) {
         window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
         for (int64_t q = q_lo; q < q_hi; ++q) cnt[permY[(int64_t)r * C + q]] = 0;
@@ -382,8 +385,8 @@ void oracle_window_loss(const float* X, const float* Y, const int32_t* target, i
   }
   free(posX);
   double total = 0.0;
-  for (int64_t i = 0; i < N; ++i) total += row_loss[i];
-  *loss = N > 0 ? total / (double)N : 0.0;
+  for (int64_t o = 0; o < n_rows; ++o) total += row_loss[o];
+  *loss = n_rows > 0 ? total / (double)n_rows : 0.0;
 }
 
 /* Its gradients, the buckets and windows held constant: every computed copy of a pair
@@ -391,15 +394,17 @@ void oracle_window_loss(const float* X, const float* Y, const int32_t* target, i
  * dloss/N;  dX_i = sum of g y_j,  dY_j = sum of g x_i over all copies  (fp64). */
 void oracle_window_grad(const float* X, const float* Y, const int32_t* target, int64_t N,
                         int64_t C, int32_t d, int32_t n_c, int32_t n_ec, int32_t n_r,
-                        const int32_t* permX, const int32_t* permY, const double* lse,
-                        double dloss, double* dX, double* dY) {
+                        const int32_t* permX, const int32_t* permY, const int64_t* rows,
+                        int64_t n_rows, const double* lse, double dloss, double* dX,
+                        double* dY) {
   double scale = N > 0 ? dloss / (double)N : 0.0;
   int64_t* posX = positions(permX, N, n_r);
   int32_t* cnt = (int32_t*)calloc((size_t)C, sizeof(int32_t));
   memset(dY, 0, sizeof(double) * (size_t)C * (size_t)d);
-  for (int64_t i = 0; i < N; ++i) {
+  for (int64_t o = 0; o < n_rows; ++o) {
+    const int64_t i = rows ? rows[o] : o;
     const float* x = X + i * (int64_t)d;
-    double* dx = dX + i * (int64_t)d;
+    double* dx = dX + o * (int64_t)d;
     int64_t q_lo, q_hi;
     for (int32_t r = 0; r < n_r; ++r) {
       window_of(i, r, posX, N, C, n_c, n_ec, &q_lo, &q_hi);
@@ -409,7 +414,7 @@ void oracle_window_grad(const float* X, const float* Y, const int32_t* target, i
       }
     }
     const float* yz = Y + (int64_t)target[i] * d;
-    double gp = (exp(dot_f64(x, yz, d) - lse[i]) - 1.0) * scale;
+    double gp = (exp(dot_f64(x, yz, d) - lse[o]) - 1.0) * scale;
     for (int32_t t = 0; t < d; ++t) dx[t] = gp * (double)yz[t];
     double* dyz = dY + (int64_t)target[i] * d;
     for (int32_t t = 0; t < d; ++t) dyz[t] += gp * (double)x[t];
@@ -419,7 +424,7 @@ void oracle_window_grad(const float* X, const float* Y, const int32_t* target, i
         int32_t j = permY[(int64_t)r * C + q];
         if (j == target[i]) continue;
         const float* y = Y + (int64_t)j * d;
-        double g = exp(dot_f64(x, y, d) - log((double)cnt[j]) - lse[i]) * scale;
+        double g = exp(dot_f64(x, y, d) - log((double)cnt[j]) - lse[o]) * scale;
         double* dy = dY + (int64_t)j * d;
         for (int32_t t = 0; t < d; ++t) {
           dx[t] += g * (double)y[t];

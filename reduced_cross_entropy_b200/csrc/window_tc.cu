@@ -50,6 +50,7 @@ constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kSlab = kBM * kBK * 2;    // one 128 x 64 bf16 box: 16 KB
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr int kMaxRounds = 8;
+constexpr int kMetaPer = ((kMaxRounds + 2) * 128 + 511) / 512;  // metadata loads per thread
 
 struct Ctl {
   uint64_t ab_full[kAB], ab_empty[kAB];
@@ -60,6 +61,7 @@ struct Ctl {
   uint32_t tmem_base;
   int abort;
   float part_m[4][kBM], part_s[4][kBM];  // LSE: the warpgroups' partial (max, sum)
+  int32_t meta[2][(kMaxRounds + 2) * kBN];  // column metadata of two K tiles
 };
 
 // Dynamic shared memory: AB stages, then (gradient roles) V stages and the P tiles.
@@ -102,6 +104,14 @@ __device__ __forceinline__ uint32_t sw128_chunk(int row, int ch) {
   return uint32_t((row >> 3) * 1024 + (row & 7) * 128 + (((ch ^ row) & 7) << 4));
 }
 
+// 2^x (the hardware approximation; subnormal results flush to zero).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
          (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
@@ -123,7 +133,8 @@ __device__ __forceinline__ void k_range(const Args& a, int64_t m0, int64_t& k0a,
   nK = k1 > k0 ? int((k1 - k0a + kBN - 1) / kBN) : 0;
 }
 
-template <int kRole>
+// kR: the round count the kernel is specialised for (1 or 2), 0 for any up to kMaxRounds.
+template <int kRole, int kR>
 __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const __grid_constant__ CUtensorMap tmV, const Args a) {
@@ -290,118 +301,212 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
     const int m = q4 * 32 + lane;   // this thread's position in the M tile
     const int64_t mi = m0 + m;
     const bool mvalid = mi < Mside;
-    const int n_r = a.n_r, n_ec = a.n_ec;
+    const int n_r = kR ? kR : a.n_r, n_ec = a.n_ec;
+    const int o = kR == 2 ? 1 - r : 0;  // the other round (two rounds)
     const int64_t rN = int64_t(r) * a.N;
-    // this thread's own side: window, positive and lse of a row (LSE, DX); its chunk in
-    // every round (rows: rowc, items: itemc)
+    // This thread's own side.  Rows (LSE, DX): window, positive, lse, and the row's chunk
+    // in every round; items (DY): the item's chunk in every round.
     int64_t w0 = 0, w1 = 0;
-    int32_t my_pz = -1;
-    float my_lse = 0.0f;
-    int32_t myc[kMaxRounds];
-    if (mvalid && kRole != kRoleDy) {
-      const int64_t cm = chunk_of(mi, a.N, a.n_c);
-      w0 = chunk_start(cm - n_ec < 0 ? 0 : cm - n_ec, a.C, a.n_c);
-      w1 = chunk_start(cm + n_ec + 1 > a.n_c ? a.n_c : cm + n_ec + 1, a.C, a.n_c);
-      my_pz = a.pz[rN + mi];
-      if (kRole == kRoleDx) my_lse = a.lse_sorted[rN + mi];
+    int64_t my_pz = -1;
+    float my_nl = 0.0f;  // -lse * log2(e)
+    int32_t myc_r = 0, myc_o = 0;
+    int32_t myc[kR == 0 ? kMaxRounds : 1];
+    const int32_t* own = kRole == kRoleDy ? a.itemc : a.rowc;
+    const int64_t ownM = kRole == kRoleDy ? a.C : a.N;
+    if (mvalid) {
+      if (kRole != kRoleDy) {
+        const int64_t cm = chunk_of(mi, a.N, a.n_c);
+        w0 = chunk_start(cm - n_ec < 0 ? 0 : cm - n_ec, a.C, a.n_c);
+        w1 = chunk_start(cm + n_ec + 1 > a.n_c ? a.n_c : cm + n_ec + 1, a.C, a.n_c);
+        my_pz = a.pz[rN + mi];
+        if (kRole == kRoleDx) my_nl = -a.lse_sorted[rN + mi] * kLog2e;
+      } else {
+        myc_r = int32_t(chunk_of(mi, a.C, a.n_c));
+      }
+      if (kR == 2) myc_o = own[(int64_t(r) * 2 + o) * ownM + mi];
     }
+    if (kR == 0) {
 #pragma unroll
-    for (int s2 = 0; s2 < kMaxRounds; ++s2) {
-      myc[s2] = 0;
-      if (s2 < n_r && mvalid)
-        myc[s2] = kRole == kRoleDy ? a.itemc[(int64_t(r) * n_r + s2) * a.C + mi]
-                                   : a.rowc[(int64_t(r) * n_r + s2) * a.N + mi];
+      for (int s2 = 0; s2 < (kR == 0 ? kMaxRounds : 1); ++s2)
+        myc[s2] = (s2 < n_r && mvalid) ? own[(int64_t(r) * n_r + s2) * ownM + mi] : 0;
     }
     const int32_t* oc_tab = kRole == kRoleDy ? a.rowc : a.itemc;  // the other side's chunks
-    const int64_t oc_M = kRole == kRoleDy ? a.N : a.C;
-    float run_m = -INFINITY, run_s = 0.0f;  // LSE: online max and sum
+    // Column metadata of every K tile, staged in shared memory (two buffers) by all
+    // epilogue threads, each tile's loads issued one tile ahead:
+    //   kR = 1, 2: DY one int4 per column (row's chunk in round r, its positive's
+    //              position, its lse, its chunk in the other round); LSE / DX one int per
+    //              column (the item's chunk in the other round; none for one round);
+    //   kR = 0:    [round][column] chunks (and, DY, [n_r] positives, [n_r + 1] lse).
+    const int n_meta = kR == 0 ? (kRole == kRoleDy ? (n_r + 2) * kBN : n_r * kBN)
+                               : (kRole == kRoleDy ? 4 * kBN : (kR == 2 ? kBN : 0));
+    const int et = threadIdx.x - 64;
+    int32_t pre[kMetaPer];
+    auto meta_load = [&](int t) {
+#pragma unroll
+      for (int j = 0; j < kMetaPer; ++j) {
+        const int v = et + j * kEpiThreads;
+        pre[j] = 0;
+        if (v >= n_meta || t >= nK) continue;
+        int arr, c;
+        if (kR != 0 && kRole == kRoleDy) {  // packed: field v & 3 of column v >> 2
+          arr = v & 3;
+          c = v >> 2;
+        } else {
+          arr = v >> 7;
+          c = v & (kBN - 1);
+        }
+        const int64_t kk = k0a + int64_t(t) * kBN + c;
+        if (kk >= Kside) continue;
+        if (kR != 0) {
+          if (kRole == kRoleDy) {
+            if (arr == 0) pre[j] = __ldg(a.rowc + (int64_t(r) * n_r + r) * a.N + kk);
+            else if (arr == 1) pre[j] = __ldg(a.pz + rN + kk);
+            else if (arr == 2) pre[j] = __float_as_int(-__ldg(a.lse_sorted + rN + kk) * kLog2e);
+            else if (kR == 2) pre[j] = __ldg(a.rowc + (int64_t(r) * 2 + o) * a.N + kk);
+          } else {
+            pre[j] = __ldg(a.itemc + (int64_t(r) * 2 + o) * a.C + kk);
+          }
+        } else if (arr < n_r) {
+          if (kRole != kRoleDy && arr == r) continue;  // a row's own round: positions decide
+          pre[j] = __ldg(oc_tab + (int64_t(r) * n_r + arr) * Kside + kk);
+        } else if (arr == n_r) {
+          pre[j] = __ldg(a.pz + rN + kk);
+        } else {
+          pre[j] = __float_as_int(-__ldg(a.lse_sorted + rN + kk) * kLog2e);
+        }
+      }
+    };
+    auto meta_store = [&](int t) {
+      int32_t* dst = ctl.meta[t & 1];
+#pragma unroll
+      for (int j = 0; j < kMetaPer; ++j)
+        if (et + j * kEpiThreads < n_meta) dst[et + j * kEpiThreads] = pre[j];
+    };
+    meta_load(0);
+    meta_store(0);
+    meta_load(1);
+    named_barrier(1, kEpiThreads);
+    float run_m = -INFINITY, run_s = 0.0f;  // LSE: online max (log2 units) and sum
     const uint32_t trow = tmem + (uint32_t(q4 * 32) << 16);
     const int col0 = 32 * g;
     bool ok = true;
+    // Every epilogue thread runs every iteration to the named barrier at its end, also
+    // after a timed-out wait (then without touching TMEM or the tiles).
     for (int kt = 0; kt < nK; ++kt) {
       const int sb = kt & 1;
       bool got = ok && mbar_wait(&ctl.s_full[sb], (kt >> 1) & 1, &ctl.abort, kTimeoutNs);
       got = __all_sync(0xFFFFFFFFu, got);  // the warp's TMEM load is collective
-      if (!got) {
-        if (ok && lane == 0) on_timeout(ctl, a.status);
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float v[32];
-      tmem_load32(trow + uint32_t(sb * kBN + col0), v);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.s_empty[sb]);
-      const int64_t kb = k0a + int64_t(kt) * kBN + col0;  // K index of v[0]
-      // v[u] becomes the column's weight 1/cnt times exp(s - lse) (gradient roles), or
-      // its weight alone with -1 for a dead column (LSE)
-      float wgt[32];
-#pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        const int64_t kk = kb + u;
-        bool live;
-        float lse_k = my_lse;
-        if (kRole == kRoleDy) {  // kk is a sorted row, this thread an item
-          live = mvalid && kk < a.N;
-          if (live)
-            live = abs(__ldg(a.rowc + (int64_t(r) * n_r + r) * a.N + kk) - myc[r]) <= n_ec &&
-                   __ldg(a.pz + rN + kk) != int32_t(mi);
-          if (live) lse_k = __ldg(a.lse_sorted + rN + kk);
-        } else {  // kk is a sorted catalogue position, this thread a row
-          live = mvalid && kk >= w0 && kk < w1 && kk != my_pz;
-        }
-        float cnt = 1.0f;
-        if (live && n_r > 1) {
-          for (int s2 = 0; s2 < n_r; ++s2)
-            if (s2 != r &&
-                abs(__ldg(oc_tab + (int64_t(r) * n_r + s2) * oc_M + kk) - myc[s2]) <= n_ec)
-              cnt += 1.0f;
-        }
-        wgt[u] = live ? 1.0f / cnt : 0.0f;
-        if (kGrad) v[u] = live ? expf(v[u] - lse_k) * wgt[u] : 0.0f;
-      }
-      if (kRole == kRoleLse) {
-        float bm = -INFINITY;
-#pragma unroll
-        for (int u = 0; u < 32; ++u)
-          if (wgt[u] > 0.0f) bm = fmaxf(bm, v[u]);
-        if (bm > run_m) {
-          run_s *= expf(run_m - bm);
-          run_m = bm;
-        }
-#pragma unroll
-        for (int u = 0; u < 32; ++u)
-          if (wgt[u] > 0.0f) run_s += expf(v[u] - run_m) * wgt[u];
-        continue;
-      }
-      // gradient roles: P into the shared tiles once the previous product has read them
-      got = mbar_wait(&ctl.p_empty, uint32_t(kt & 1) ^ 1u, &ctl.abort, kTimeoutNs);
-      if (!__all_sync(0xFFFFFFFFu, got)) {
+      if (!got && ok) {
         if (lane == 0) on_timeout(ctl, a.status);
         ok = false;
-        break;
       }
-      uint8_t* th = phi + (col0 >> 6) * kSlab;
-      uint8_t* tl = plo + (col0 >> 6) * kSlab;
-      const int cb = (col0 & 63) >> 3;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t h[4], l[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = v[8 * j + 2 * e], x1 = v[8 * j + 2 * e + 1];
-          const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
-          h[e] = pack_bf16(h0, h1);
-          l[e] = pack_bf16(x0 - h0, x1 - h1);
+      if (ok) {
+        tc_fence_after();
+        float v[32];
+        tmem_load32(trow + uint32_t(sb * kBN + col0), v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.s_empty[sb]);
+        const int32_t* md = ctl.meta[kt & 1];
+        const int64_t kb = k0a + int64_t(kt) * kBN + col0;  // K index of v[0]
+        // the live columns of this block: [lo, hi) minus the positive's column
+        int lo = 0, hi = 0, pzc = -1;
+        if (mvalid) {
+          if (kRole == kRoleDy) {
+            const int64_t rest = a.N - kb;
+            hi = rest <= 0 ? 0 : (rest >= 32 ? 32 : int(rest));
+          } else {
+            const int64_t l = w0 - kb, h = w1 - kb;
+            lo = l <= 0 ? 0 : (l >= 32 ? 32 : int(l));
+            hi = h <= 0 ? 0 : (h >= 32 ? 32 : int(h));
+            if (my_pz >= kb && my_pz < kb + 32) pzc = int(my_pz - kb);
+          }
         }
-        *reinterpret_cast<uint4*>(th + sw128_chunk(m, cb + j)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(tl + sw128_chunk(m, cb + j)) = make_uint4(l[0], l[1], l[2], l[3]);
+        // v[u] becomes, per live column, log2(e) times the score plus (gradient roles)
+        // the row's -lse * log2(e); w[u] the column's weight 1/cnt (0: dead)
+        float w[kGrad ? 1 : 32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int c = col0 + u;
+          bool live = u >= lo && u < hi && u != pzc;
+          float nl = my_nl;
+          float wt = 1.0f;
+          if (kRole == kRoleDy && kR != 0) {
+            const int4 mc = reinterpret_cast<const int4*>(md)[c];
+            live = live && abs(mc.x - myc_r) <= n_ec && mc.y != int32_t(mi);
+            nl = __int_as_float(mc.z);
+            if (kR == 2 && abs(mc.w - myc_o) <= n_ec) wt = 0.5f;
+          } else if (kRole == kRoleDy) {
+            live = live && abs(md[r * kBN + c] - myc_r) <= n_ec && md[n_r * kBN + c] != int32_t(mi);
+            nl = __int_as_float(md[(n_r + 1) * kBN + c]);
+          } else if (kR == 2) {
+            if (abs(md[c] - myc_o) <= n_ec) wt = 0.5f;
+          }
+          if (kR == 0) {
+            int cnt = 1;
+            for (int s2 = 0; s2 < n_r; ++s2)
+              if (s2 != r && abs(md[s2 * kBN + c] - myc[s2]) <= n_ec) ++cnt;
+            wt = __fdividef(1.0f, float(cnt));
+          }
+          if (kGrad) {
+            v[u] = live ? wt * ex2(fmaf(v[u], kLog2e, nl)) : 0.0f;  // p / cnt
+          } else {
+            w[u] = live ? wt : 0.0f;
+            v[u] = live ? fmaf(v[u], kLog2e, nl) : -INFINITY;
+          }
+        }
+        if (kRole == kRoleLse) {
+          float bm = -INFINITY;
+#pragma unroll
+          for (int u = 0; u < 32; ++u) bm = fmaxf(bm, v[u]);
+          if (bm != -INFINITY) {
+            if (bm > run_m) {
+              run_s *= ex2(run_m - bm);
+              run_m = bm;
+            }
+            float acc = 0.0f;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) acc = fmaf(w[u], ex2(v[u] - run_m), acc);
+            run_s += acc;
+          }
+        } else {
+          // P into the shared tiles once the previous product has read them
+          got = mbar_wait(&ctl.p_empty, uint32_t(kt & 1) ^ 1u, &ctl.abort, kTimeoutNs);
+          if (!__all_sync(0xFFFFFFFFu, got)) {
+            if (lane == 0) on_timeout(ctl, a.status);
+            ok = false;
+          } else {
+            uint8_t* th = phi + (col0 >> 6) * kSlab;
+            uint8_t* tl = plo + (col0 >> 6) * kSlab;
+            const int cb = (col0 & 63) >> 3;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t h[4], l[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float x0 = v[8 * j + 2 * e], x1 = v[8 * j + 2 * e + 1];
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+                const float2 hf = __bfloat1622float2(hb);
+                const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+                h[e] = *reinterpret_cast<const uint32_t*>(&hb);
+                l[e] = *reinterpret_cast<const uint32_t*>(&lb);
+              }
+              *reinterpret_cast<uint4*>(th + sw128_chunk(m, cb + j)) =
+                  make_uint4(h[0], h[1], h[2], h[3]);
+              *reinterpret_cast<uint4*>(tl + sw128_chunk(m, cb + j)) =
+                  make_uint4(l[0], l[1], l[2], l[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl.p_full);
+          }
+        }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.p_full);
+      // tile kt+1's metadata in (its buffer was last read during tile kt-1, which every
+      // thread finished before the barrier that ended it); tile kt+2's loads out
+      meta_store(kt + 1);
+      meta_load(kt + 2);
+      named_barrier(1, kEpiThreads);
     }
     if (kRole == kRoleLse) {
       // the four warpgroups' partials of every row
@@ -409,14 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
       ctl.part_s[g][m] = run_s;
       named_barrier(1, kEpiThreads);
       if (g == 0 && mvalid) {
-        float M = -INFINITY, S = 0.0f;
+        float M = -INFINITY, S = 0.0f;  // M in log2 units, as the partials
 #pragma unroll
         for (int w = 0; w < 4; ++w)
           if (ctl.part_s[w][m] > 0.0f) M = fmaxf(M, ctl.part_m[w][m]);
 #pragma unroll
         for (int w = 0; w < 4; ++w)
-          if (ctl.part_s[w][m] > 0.0f) S += ctl.part_s[w][m] * expf(ctl.part_m[w][m] - M);
-        a.ms[rN + mi] = make_float2(S > 0.0f ? M : 0.0f, S);
+          if (ctl.part_s[w][m] > 0.0f) S += ctl.part_s[w][m] * ex2(ctl.part_m[w][m] - M);
+        a.ms[rN + mi] = make_float2(S > 0.0f ? M / kLog2e : 0.0f, S);
       }
     } else {
       bool fin = ok && mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && nK > 0;
@@ -455,19 +560,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
 }
 
 
-template <int kRole>
-cudaError_t run_window(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& V,
-                       const Args& a, unsigned gx, unsigned gy, cudaStream_t st) {
+template <int kRole, int kR>
+cudaError_t run_window_r(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& V,
+                         const Args& a, unsigned gx, unsigned gy, cudaStream_t st) {
   size_t smem = window_smem(kRole, a.d, a.nv);
   // at most two CTAs per SM: their TMEM allocations (256 columns each in the LSE role,
   // 512 in the gradient roles, one CTA) always fit
   if (smem < 80 * 1024) smem = 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_window_tc<kRole>,
+  cudaError_t e = cudaFuncSetAttribute(k_window_tc<kRole, kR>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  k_window_tc<kRole><<<dim3(gx, gy), kThreads, smem, st>>>(A, B, V, a);
+  k_window_tc<kRole, kR><<<dim3(gx, gy), kThreads, smem, st>>>(A, B, V, a);
   count_launches(1);
   return cudaGetLastError();
+}
+
+template <int kRole>
+cudaError_t run_window(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& V,
+                       const Args& a, unsigned gx, unsigned gy, cudaStream_t st) {
+  if (a.n_r == 1) return run_window_r<kRole, 1>(A, B, V, a, gx, gy, st);
+  if (a.n_r == 2) return run_window_r<kRole, 2>(A, B, V, a, gx, gy, st);
+  return run_window_r<kRole, 0>(A, B, V, a, gx, gy, st);
 }
 
 Args base_args(const rece_plan_s& p, const int32_t* itemc, const int32_t* rowc,

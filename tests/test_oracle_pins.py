@@ -554,3 +554,16 @@ def test_window_grad_finite_differences_and_invariants():
             assert fd == pytest.approx(G[idx], abs=1e-6 * max(1.0, np.abs(G).max()))
     # every row's coefficients sum to zero -> the dY rows sum to the zero vector
     assert np.abs(dY.sum(0)).max() < 1e-12
+
+
+def test_window_row_sample_matches_the_full_computation():
+    X, Y, z, B = _random_case(N=50, C=140, d=8, n_b=3, n_c=5, n_r=2)
+    top = oracle.rece_forward(X, Y, z, B, 5, 1, 1)
+    px, py = top["permX"], top["permY"]
+    _, row, lse = oracle.window_loss(X, Y, z, px, py, 5, 1)
+    dX, _ = oracle.window_grad(X, Y, z, px, py, 5, 1, lse, 0.5)
+    sample = np.array([3, 17, 49, 0, 22])
+    _, srow, slse = oracle.window_loss(X, Y, z, px, py, 5, 1, rows=sample)
+    np.testing.assert_array_equal(srow, row[sample])
+    sX, _ = oracle.window_grad(X, Y, z, px, py, 5, 1, slse, 0.5, rows=sample)
+    np.testing.assert_array_equal(sX, dX[sample])
