@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="sasrec")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-memory", action="store_true")
+    ap.add_argument("--no-allreduce-dy", action="store_true",
+                    help="N > 1: run independent replicas, without summing dY across ranks")
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip timing the sampled CE- / BCE+ comparison ops")
     ap.add_argument("--flags", type=int, default=0, help="rece_config_t.flags")
@@ -277,7 +279,7 @@ def run_reference(args):
     X, Y, t = synth.make_inputs(w, seed=0)
     B = synth.projections(0, 0, w.n_r, w.n_b, w.d, w.dtype)
     rows, frac = 128, 32
-    alln = bool(args.flags & 0x2)  # RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed
+    alln = bool(getattr(args, "flags", 0) & 0x2)  # RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed
     for _ in range(args.warmup):
         oracle_step_seconds(w, X, Y, t, B, rows, frac, all_negatives=alln)
     secs = [oracle_step_seconds(w, X, Y, t, B, rows, frac, all_negatives=alln)
@@ -318,6 +320,15 @@ def max_over_ranks(x, device=None):
     return float(t.item())
 
 
+def allreduce_dy(dY):
+    """Data-parallel replicas share the catalogue Y: the one exchange of a training step
+    is the sum of the ranks' dY (NCCL over NVLink under torchrun; any backend of the
+    default group).  Every rank calls it once per step, in the same place."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(dY, op=dist.ReduceOp.SUM)
+
+
 def job_throughput(world, rows_per_step, steps, total_ms):
     """Whole-job rows/s: every rank processes rows_per_step rows per step (weak scaling),
     timed by the slowest rank's total_ms over `steps` steps."""
@@ -346,6 +357,8 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
+
+    exchange = world > 1 and not args.no_allreduce_dy
 
     L = _lib.lib()
     w = synth.WORKLOADS[args.workload]
@@ -381,6 +394,8 @@ def main():
         _lib.check(L.rece_loss_bwd(plan._h, vp(Xd), vp(Yd), vp(td), vp(sel), vp(lse),
                                    vp(logits), vp(dloss), vp(ws), nbytes, vp(dX), vp(dY), sp),
                    "loss_bwd")
+        if exchange:
+            allreduce_dy(dY)
 
     for s in range(args.warmup):
         flush.zero_()
@@ -489,6 +504,9 @@ def main():
                        "overflowed_rows_per_step": overflow_rows,
                        "merge_spilled_rows_per_step": spilled_rows,
                        "l2": "flushed between timed steps (256 MiB write)",
+                       "parallelism": f"dp{world}",
+                       "exchange": ("all-reduce of dY [C x d] fp32 every step (NCCL)"
+                                    if exchange else "none"),
                        "scores": ("tcgen05" + (", stored" if paths & _lib.PATH_STORED_SCORES
                                                  else ", recomputed per pass")
                                   if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),

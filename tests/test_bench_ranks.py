@@ -1,9 +1,10 @@
 """Host logic of bench.py's multi-GPU run, on CPU ranks over gloo (world size 2).
 
-The path does not shard: every rank runs the whole loss on its own problem (weak
-scaling) and the job's time is the slowest rank's.  These tests run that timing
-reduction, the throughput formula and the reference arm's rank rule as two gloo
-processes, no GPU involved.
+Data-parallel replicas: every rank runs the whole loss on its own batch against the
+shared catalogue (weak scaling), the ranks sum their dY once per step, and the job's time
+is the slowest rank's.  These tests run that exchange, the timing reduction, the
+throughput formula and the reference arm's rank rule as two gloo processes, no GPU
+involved.
 """
 import contextlib
 import importlib.util
@@ -43,6 +44,11 @@ def _rank_main(rank, world, port, out):
         # each rank's own total time; the job is as slow as its slowest rank
         mine = 10.0 + 5.0 * rank
         slowest = bench.max_over_ranks(mine)
+        # the data-parallel exchange: every rank ends with the sum of the ranks' dY
+        import torch
+        dY = torch.full((5, 3), float(rank + 1))
+        bench.allreduce_dy(dY)
+        assert torch.equal(dY, torch.full((5, 3), float(world * (world + 1) // 2)))
         rows = bench.job_throughput(world, 25_600, 4, slowest)
         # the reference (oracle) arm: rank 0 alone works and prints
         buf = io.StringIO()
