@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "plan.h"
+#include "sm100.cuh"
 #include "tc.h"
 
 namespace rece {
@@ -367,6 +368,100 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
   }
 }
 
+// dY for wide rows (1024 <= d <= 4096, d % 16 == 0): one CTA per item.  Warp 0 streams
+// the item's pairs' x rows, each one contiguous bulk copy, through a ring of shared-memory
+// stages; every other thread owns 16 dimensions and adds g * x for each pair in order.
+// The rows reach the SM without passing through registers, so far more bytes are in
+// flight than a register-gathering warp can hold.  Each dimension is summed by one
+// thread in the pairs' (row) order: deterministic.  Waits are bounded; a timeout sets
+// the device flag and ends the CTA's work.
+constexpr int kWideMaxStages = 8;
+constexpr uint64_t kWideTimeoutNs = 1000000000ull;
+
+int wide_stages(int d, size_t elem) {
+  const size_t rb = size_t(d) * elem;
+  int st = int((64 * 1024) / rb);
+  return st < 2 ? 2 : (st > kWideMaxStages ? kWideMaxStages : st);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(288) k_bwd_items_wide(
+    const T* __restrict__ X, int d, int k, int stages, const int32_t* __restrict__ item_start,
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ pair_g,
+    const float* __restrict__ sorted_g, float* __restrict__ dY, uint32_t* status) {
+  extern __shared__ __align__(128) uint8_t wsm[];
+  __shared__ uint64_t full[kWideMaxStages], empty[kWideMaxStages];
+  __shared__ float s_g[kWideMaxStages];
+  __shared__ int abort_flag;
+  const uint32_t rb = uint32_t(d) * sizeof(T);
+  const int64_t j = blockIdx.x;
+  const int64_t lo = item_start[j];
+  const int n = int(item_start[j + 1] - lo);
+  const int consumers = (blockDim.x >> 5) - 1;  // warps
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages; ++st) {
+      sm100::mbar_init(&full[st], 1);
+      sm100::mbar_init(&empty[st], consumers);
+    }
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // ------------------------------------------------------------ producer
+    if (threadIdx.x == 0) {
+      const int slots = k + 1;
+      int q = 0;
+      for (; q < n; ++q) {
+        const int st = q % stages;
+        if (q >= stages &&
+            !sm100::mbar_wait(&empty[st], uint32_t((q / stages) - 1) & 1u, &abort_flag,
+                              kWideTimeoutNs)) {
+          abort_flag = 1;
+          raise_flag(status, RECE_DEVICE_TIMEOUT);
+          break;
+        }
+        const int32_t id = sorted_id[lo + q];
+        s_g[st] = sorted_g ? sorted_g[lo + q] : pair_g[id];
+        sm100::mbar_arrive_expect_tx(&full[st], rb);
+        sm100::bulk_load(wsm + size_t(st) * rb, X + int64_t(id / slots) * d, rb, &full[st]);
+      }
+      // every issued copy has landed before the CTA may exit
+      for (int p = (q > stages ? q - stages : 0); p < q; ++p)
+        sm100::mbar_wait_limit(&full[p % stages], uint32_t(p / stages) & 1u, kWideTimeoutNs);
+    }
+    return;
+  }
+  // -------------------------------------------------------------- consumers
+  const int t0 = (threadIdx.x - 32) * 16;
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+  for (int q = 0; q < n; ++q) {
+    const int st = q % stages;
+    if (!sm100::mbar_wait(&full[st], uint32_t(q / stages) & 1u, &abort_flag, kWideTimeoutNs)) {
+      abort_flag = 1;
+      raise_flag(status, RECE_DEVICE_TIMEOUT);
+      break;
+    }
+    const T* row = reinterpret_cast<const T*>(wsm + size_t(st) * rb) + t0;
+    const float g = s_g[st];
+    float v[16];
+    load8(row, *reinterpret_cast<float(*)[8]>(&v[0]));
+    load8(row + 8, *reinterpret_cast<float(*)[8]>(&v[8]));
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = fmaf(g, v[e], acc[e]);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) sm100::mbar_arrive(&empty[st]);
+  }
+  // streaming stores: dY is written once, and should not push the gathered rows of X
+  // out of L2
+  float4* o = reinterpret_cast<float4*>(dY + j * d + t0);
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    __stcs(o + e, make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]));
+}
+
 }  // namespace
 
 size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 * (k + 1)); }
@@ -466,7 +561,15 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
   const int warps = kThreads / 32;
-  if (c.d % 8 == 0)
+  if (c.d >= 1024 && c.d <= 4096 && c.d % 16 == 0) {
+    const int stages = wide_stages(c.d, sizeof(T));
+    const size_t smem = size_t(stages) * c.d * sizeof(T);
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_items_wide<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    k_bwd_items_wide<T><<<unsigned(c.C), 32 + c.d / 16, smem, st>>>(
+        X, c.d, c.k, stages, item_start, in, e_g, sorted_g, dY, status);
+  } else if (c.d % 8 == 0)
     k_bwd_items_v8<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
         X, c.C, c.d, c.k, item_start, in, e_g, sorted_g, dY);
   else
