@@ -77,7 +77,8 @@ struct Layout {
   // all-negatives mode, kept from rece_loss_fwd to rece_loss_bwd: the d-major copy of X,
   // the chunk tables, positives' sorted positions, lse per round in sorted order; forward
   // only: the rounds' (max, sum) pairs and the inverse orders of Y
-  size_t xst = 0, itemc = 0, rowc = 0, pz = 0, lse_sorted = 0, ms = 0, inv_y = 0;
+  size_t xst = 0, itemc = 0, rowc = 0, pz = 0, lse_sorted = 0, ms = 0, inv_y = 0,
+         dx_parts = 0;
   size_t total = 0;
 };
 

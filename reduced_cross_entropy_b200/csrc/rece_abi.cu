@@ -129,6 +129,7 @@ void build_layout_all_neg(rece_plan_s& p) {
   rece_plan_s& q = *p.pos_plan;
   q.lay.status = L.status;
   layout_pairs(q, off);
+  L.dx_parts = take(sizeof(float) * nr * c.N * c.d);  // each round's part of dX
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
@@ -298,16 +299,16 @@ rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
                             dloss, ws, dX, dY, status, st),
             "positives' backward");
   RECE_CUDA(launch_window_grad_tc(p, false, ws + L.xs, ws + L.ys, ws + L.xst, ws + L.yst,
-                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.px), dloss, dX, status,
-                                  st),
+                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.px), dloss, dX,
+                                  reinterpret_cast<float*>(ws + L.dx_parts), status, st),
             "window dX (tcgen05)");
   stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
   RECE_CUDA(launch_window_grad_tc(p, true, ws + L.xs, ws + L.ys, ws + L.xst, ws + L.yst,
-                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.py), dloss, dY, status,
-                                  st),
+                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.py), dloss, dY,
+                                  nullptr, status, st),
             "window dY (tcgen05)");
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
   return RECE_OK;

@@ -97,12 +97,13 @@ cudaError_t launch_window_combine(const rece_plan_s& p, const T* X, const T* Y,
                                   float* lse, float* row_loss, float* lse_sorted,
                                   uint32_t* status, cudaStream_t st);
 // The window terms of dX (dy = false, perm = px) or dY (dy = true, perm = py), added
-// into `out` round by round.
+// into `out` round by round (dX with `scratch` [n_r][N][d]: all rounds in one grid, then
+// added in round order).
 cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
                                   const void* Ys, const void* XsT, const void* YsT,
                                   const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
                                   const float* lse_sorted, const int32_t* perm,
-                                  const float* dloss, float* out, uint32_t* status,
-                                  cudaStream_t st);
+                                  const float* dloss, float* out, float* scratch,
+                                  uint32_t* status, cudaStream_t st);
 
 }  // namespace rece

@@ -82,6 +82,7 @@ struct Args {
   const int32_t* perm;       // px (DX) or py (DY): sorted position -> row / item
   const float* dloss;
   float* out;                // dX [N][d] or dY [C][d], added into
+  float* scratch;            // DX with all rounds in one grid: [n_r][N][d], written
   float2* ms;                // LSE: [n_r][N] (max, sum) of the window terms
   uint32_t* status;
 };
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
   Ctl& ctl = *reinterpret_cast<Ctl*>(plo + (kGrad ? 2 * kSlab : 0));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = a.d, nk = d / kBK;
-  const int r = kRole == kRoleLse ? int(blockIdx.y) : a.r;
+  const int r = (kRole == kRoleLse || a.scratch) ? int(blockIdx.y) : a.r;
   const int64_t Mside = kRole == kRoleDy ? a.C : a.N;
   const int64_t Kside = kRole == kRoleDy ? a.N : a.C;
   const int64_t m0 = int64_t(blockIdx.x) * kBM;
@@ -534,7 +535,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
         for (int oc = col0; oc < d; oc += 128) {
           float v[32];
           tmem_load32(trow + 256u + uint32_t(oc), v);
-          if (mvalid) {
+          if (mvalid && a.scratch) {  // this round's part, written; the rounds add later
+            float4* q = reinterpret_cast<float4*>(a.scratch + (rN + dst) * d + oc);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              q[u] = make_float4(scale * v[4 * u], scale * v[4 * u + 1], scale * v[4 * u + 2],
+                                 scale * v[4 * u + 3]);
+          } else if (mvalid) {
             float4* q = reinterpret_cast<float4*>(o + oc);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -559,6 +566,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
   }
 }
 
+
+// out[i][:] += sum over rounds r of part[r][i][:], rounds in order.
+__global__ void __launch_bounds__(256) k_window_add(const float4* __restrict__ part,
+                                                    int64_t n4, int n_r,
+                                                    float4* __restrict__ out) {
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    float4 x = out[e];
+    for (int r = 0; r < n_r; ++r) {
+      const float4 p = part[int64_t(r) * n4 + e];
+      x.x += p.x;
+      x.y += p.y;
+      x.z += p.z;
+      x.w += p.w;
+    }
+    out[e] = x;
+  }
+}
 
 template <int kRole, int kR>
 cudaError_t run_window_r(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& V,
@@ -626,8 +651,8 @@ cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
                                   const void* Ys, const void* XsT, const void* YsT,
                                   const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
                                   const float* lse_sorted, const int32_t* perm,
-                                  const float* dloss, float* out, uint32_t* status,
-                                  cudaStream_t st) {
+                                  const float* dloss, float* out, float* scratch,
+                                  uint32_t* status, cudaStream_t st) {
   const auto& c = p.cfg;
   if (c.N == 0) return cudaSuccess;
   CUtensorMap tX, tY, tV;
@@ -645,6 +670,19 @@ cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
   a.perm = perm;
   a.dloss = dloss;
   a.out = out;
+  if (!dy && scratch) {
+    // dX: every round in one grid (the rows' tiles alone would not fill the GPU), each
+    // writing its part; then the parts are added into dX in round order
+    a.scratch = scratch;
+    e = run_window<kRoleDx>(tX, tY, tV, a, unsigned(ceil_div(c.N, kBM)), unsigned(c.n_r), st);
+    if (e != cudaSuccess) return e;
+    const int64_t n4 = c.N * int64_t(c.d) / 4;
+    const int64_t want = (n4 + 255) / 256;
+    k_window_add<<<unsigned(want < 8 * 148 ? want : 8 * 148), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(scratch), n4, c.n_r, reinterpret_cast<float4*>(out));
+    count_launches(1);
+    return cudaGetLastError();
+  }
   for (int r = 0; r < c.n_r; ++r) {  // rounds in order: each adds into the same rows
     a.r = r;
     e = dy ? run_window<kRoleDy>(tY, tX, tV, a, unsigned(ceil_div(c.C, kBM)), 1u, st)
