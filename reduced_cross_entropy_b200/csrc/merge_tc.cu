@@ -138,7 +138,9 @@ struct MergeArgs {
 // (returns false); without, the first cap are kept and the row is flagged inexact.
 // kGrouped: also hand the backward's tensor-core dX its data (entries grouped by slice,
 // probabilities, the positive logit); else the kept entries go out in list order.
-template <typename T, bool kGrouped>
+// kGather: candidates per lane gathered together (list entry, then item, then chunk):
+// 8 pays at k >= 384, where a round's candidates fill the wider batches; else 4.
+template <typename T, bool kGrouped, int kGather>
 __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint32_t* cnt,
                                           uint32_t* keys, int32_t* poss, int cap, bool spill) {
   const T* __restrict__ X = A.X;
@@ -180,7 +182,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
     rb[r] = n < cap ? n : cap;
     const int64_t p = invX[int64_t(r) * N + i];
     // four sub-lists (one per epilogue warpgroup of the selection kernel), read as one
-    // concatenated list, four independent entries per lane in flight at a time
+    // concatenated list, kGather independent entries per lane in flight at a time
     const int4 c4 = list_count[int64_t(r) * N + p];
     theta_max = fmaxf(theta_max, list_theta[int64_t(r) * N + p]);
     const int cs[4] = {c4.x < Qw ? c4.x : Qw, c4.y < Qw ? c4.y : Qw, c4.z < Qw ? c4.z : Qw,
@@ -188,12 +190,12 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
     overflow |= c4.x > Qw || c4.y > Qw || c4.z > Qw || c4.w > Qw;
     const int total = cs[0] + cs[1] + cs[2] + cs[3];
     const int2* L = list + (int64_t(r) * N + p) * 4 * Qw;
-    for (int a0 = 0; a0 < total; a0 += 128) {
-      int2 e[4];
-      int32_t jj[4];
-      bool in[4];
+    for (int a0 = 0; a0 < total; a0 += 32 * kGather) {
+      int2 e[kGather];
+      int32_t jj[kGather];
+      bool in[kGather];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kGather; ++u) {
         int a = a0 + 32 * u + lane;
         in[u] = a < total;
         int w = 0;
@@ -204,10 +206,10 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
         e[u] = in[u] ? L[w * Qw + a] : make_int2(0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) jj[u] = in[u] ? py[int64_t(r) * C + e[u].y] : -1;
-      bool keep[4];
+      for (int u = 0; u < kGather; ++u) jj[u] = in[u] ? py[int64_t(r) * C + e[u].y] : -1;
+      bool keep[kGather];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kGather; ++u) {
         keep[u] = in[u] && jj[u] != z;
         for (int rp = 0; rp < r && keep[u]; ++rp) {
           const int dc = chunkY[int64_t(rp) * C + jj[u]] - cx[rp];
@@ -215,7 +217,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kGather; ++u) {
         const unsigned b = __ballot_sync(0xFFFFFFFFu, keep[u]);
         if (keep[u]) {
           const int pos = n + __popc(b & ((1u << lane) - 1u));
@@ -427,7 +429,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
 }
 
 // Fast path: one row per warp, candidates in shared memory (cap per row).
-template <typename T, bool kGrouped>
+template <typename T, bool kGrouped, int kGather>
 __global__ void __launch_bounds__(kThreads) k_merge_tc(const MergeArgs<T> A, int cap) {
   extern __shared__ __align__(16) uint8_t sh_raw[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5;
@@ -438,12 +440,12 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(const MergeArgs<T> A, int
   int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);
   const int64_t i = int64_t(blockIdx.x) * warps + wid;
   if (i >= A.N) return;  // whole warp leaves together; no block-wide barriers follow
-  merge_row<T, kGrouped>(A, i, cnt, keys, poss, cap, true);
+  merge_row<T, kGrouped, kGather>(A, i, cnt, keys, poss, cap, true);
 }
 
 // Spilled rows: the warps walk the spill list with their candidates in global scratch
 // (room for every list entry of every round, so nothing is dropped).
-template <typename T, bool kGrouped>
+template <typename T, bool kGrouped, int kGather>
 __global__ void __launch_bounds__(kThreads) k_merge_tc_spill(const MergeArgs<T> A, int cap,
                                                              uint32_t* scratch) {
   __shared__ uint32_t sh_cnt[kThreads / 32][kCountBytes / 4];
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc_spill(const MergeArgs<T> 
   int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);
   const uint32_t n = *reinterpret_cast<volatile uint32_t*>(A.spill_count);
   for (int64_t w = gw; w < n; w += nw)
-    merge_row<T, kGrouped>(A, A.spill_rows[w], sh_cnt[wid], keys, poss, cap, false);
+    merge_row<T, kGrouped, kGather>(A, A.spill_rows[w], sh_cnt[wid], keys, poss, cap, false);
 }
 
 }  // namespace
@@ -521,14 +523,17 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
   const size_t smem = per_warp * warps;
   const bool grouped = kept != nullptr;
-  auto kern = grouped ? k_merge_tc<T, true> : k_merge_tc<T, false>;
+  const bool wide = c.k >= 384;
+  auto kern = grouped ? (wide ? k_merge_tc<T, true, 8> : k_merge_tc<T, true, 4>)
+                      : (wide ? k_merge_tc<T, false, 8> : k_merge_tc<T, false, 4>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(A.spill_count, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return e;
   kern<<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(A, cap);
-  auto spill = grouped ? k_merge_tc_spill<T, true> : k_merge_tc_spill<T, false>;
+  auto spill = grouped ? (wide ? k_merge_tc_spill<T, true, 8> : k_merge_tc_spill<T, true, 4>)
+                       : (wide ? k_merge_tc_spill<T, false, 8> : k_merge_tc_spill<T, false, 4>);
   spill<<<kSpillWarps / (kThreads / 32), kThreads, 0, st>>>(
       A, merge_tc_spill_cap(c.n_r, c.k), static_cast<uint32_t*>(spill_scratch));
   count_launches(2);
