@@ -104,16 +104,20 @@ def stage_work(w, paths=0):
             "bwd_sort": (0, 0),
             "bwd_items": (4 * d * pr, nr * (N + C) * d * e + 2 * C * d * 4),
         }
+    # Step 6 charges what the scope table does: F = 4 N (k+1) d, B = (N+C) d e + 8 N k +
+    # (N+C) d 4 -- X and Y read once, dX and dY written once -- split between the dX
+    # stage (Y, the coefficients' inputs, dX) and the dY stage (X, dY); re-reading a
+    # gathered row and the pair sort are the implementation's cost, not charged.
+    tc = paths & _lib.PATH_TENSOR_CORES
     return {
         "bucketize": (2 * (N + C) * nb * d * nr, nr * (N + C) * (d * e + 4)),
-        "sort": (0, nr * (N + C) * 16),
+        "sort": (0, nr * (N + C) * (16 + (2 * d * e if tc else 0))),
         "select": (2 * d * pairs_per_round(w) * nr, nr * (N + C) * d * e + nr * N * k * 8),
-        "merge_loss": (0, nr * N * k * 8 + N * k * 4 + 8 * N + N * d * e),
+        "merge_loss": (0, nr * N * k * 8 + N * k * 4 + 8 * N),
         "mean": (0, 4 * N),
-        "bwd_rows": (4 * N * (k + 1) * d, N * d * e + N * (k + 1) * d * e + 4 * N * k
-                     + N * d * 4 + 8 * N * (k + 1)),
-        "bwd_sort": (0, 3 * N * (k + 1) * 16),
-        "bwd_items": (2 * N * (k + 1) * d, N * (k + 1) * 8 + N * (k + 1) * d * e + C * d * 4),
+        "bwd_rows": (2 * N * (k + 1) * d, C * d * e + 8 * N * k + N * d * 4),
+        "bwd_sort": (0, 0),
+        "bwd_items": (2 * N * (k + 1) * d, N * d * e + C * d * 4),
     }
 
 
@@ -126,7 +130,7 @@ def stage_bound(stage, paths):
         return "tensor"
     if stage == "bwd_rows" and paths & _lib.PATH_DX_TENSORS:
         return "tensor"
-    return "hbm"
+    return "hbm"  # (the pair sort has no algorithmic work: its fraction reads 0)
 
 
 KERNEL_SOURCES = {
