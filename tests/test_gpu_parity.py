@@ -29,6 +29,9 @@ CASES = {
     "sasrec_scaled": W["sasrec"].scaled(3200, 12500, n_c=8),
     "lm_scaled": W["lm"].scaled(512, 4000, n_c=4, n_b=64, k=128, d=256),
     "large_norms_scaled": W["large"].scaled(2000, 20000, n_c=10, n_b=128, k=128),
+    # C >= 2^18: the backward's pair sort takes three passes of at most 9-bit digits
+    "three_pass_pair_sort": synth.Workload("p3", N=256, C=300001, d=16, dtype="fp32", n_b=8,
+                                           n_c=16, n_ec=1, n_r=2, k=16),
     # wide rows: dY through the shared-memory ring of bulk row copies (d >= 1024)
     "lm_wide_fp32": W["lm"].scaled(384, 3000, n_c=3, n_b=32, k=64, d=2048, dtype="fp32"),
     "lm_wide_bf16": W["lm"].scaled(384, 3000, n_c=3, n_b=32, k=64, d=4096),
