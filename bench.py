@@ -133,10 +133,10 @@ def stage_bound(stage, paths):
     return "hbm"  # (the pair sort has no algorithmic work: its fraction reads 0)
 
 
-KERNEL_SOURCES = {
+KERNEL_SOURCES = {  # the pair sort's pass geometry is decided in rece_abi.cu
     "bucketize": ["bucketize.cu"], "sort": ["sort.cu"], "select": ["select.cu"],
     "merge_loss": ["loss.cu"], "mean": ["loss.cu"], "bwd_rows": ["backward.cu"],
-    "bwd_sort": ["sort.cu"], "bwd_items": ["backward.cu"],
+    "bwd_sort": ["sort.cu", "rece_abi.cu"], "bwd_items": ["backward.cu"],
 }
 
 
@@ -154,7 +154,7 @@ def kernel_sources(stage, paths):
     if paths & _lib.PATH_ALL_NEGATIVES:
         src.update(select=["window_tc.cu", "window.cu", "sm100.cuh"],
                    merge_loss=["window.cu"], bwd_rows=["backward.cu", "window_tc.cu"],
-                   bwd_sort=["sort.cu"], bwd_items=["window_tc.cu"])
+                   bwd_sort=["sort.cu", "rece_abi.cu"], bwd_items=["window_tc.cu"])
     return src[stage]
 
 
