@@ -23,6 +23,7 @@ PATH_TENSOR_CORES = 0x1
 PATH_DX_TENSORS = 0x2
 PATH_STORED_SCORES = 0x4
 PATH_ALL_NEGATIVES = 0x8
+PATH_DY_TENSORS = 0x10
 FLAG_ALL_NEGATIVES = 0x2  # Algorithm 1 as printed: every window item a negative
 
 # every symbol include/rece.h declares

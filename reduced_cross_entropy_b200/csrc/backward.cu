@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows(
   if (i >= N) return;  // the warp leaves together; no block-wide barrier follows
   const float scale = dloss[0] / float(N);
   const float li = sigmoid ? 0.0f : lse[i];
-  for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
+  if (!logits)  // x takes part only in the dot products
+    for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
   __syncwarp();
 
   // coefficients: one slot per lane at a time
@@ -208,7 +209,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
   if (i >= N) return;  // the warp leaves together; no block-wide barrier follows
   const float scale = dloss[0] / float(N);
   const float li = sigmoid ? 0.0f : lse[i];
-  for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
+  if (!logits)  // x takes part only in the dot products
+    for (int t = lane; t < d; t += 32) xs[t] = to_f32(X[i * d + t]);
   __syncwarp();
 
   if (logits) {
@@ -398,6 +400,14 @@ __global__ void __launch_bounds__(288) k_bwd_items_wide(
   const int64_t lo = item_start[j];
   const int n = int(item_start[j + 1] - lo);
   const int consumers = (blockDim.x >> 5) - 1;  // warps
+  if (n == 0) {  // an item no pair names: zeros, without setting up the ring
+    if (threadIdx.x >= 32) {
+      float4* o = reinterpret_cast<float4*>(dY + j * d + (threadIdx.x - 32) * 16);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) __stcs(o + e, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+    }
+    return;
+  }
   if (threadIdx.x == 0) {
     for (int st = 0; st < stages; ++st) {
       sm100::mbar_init(&full[st], 1);
@@ -516,6 +526,26 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   int32_t* sorted_key = reinterpret_cast<int32_t*>(ws + L.e_sorted_key);
   float* sorted_g = p.carry_g ? reinterpret_cast<float*>(ws + L.e_sorted_g) : nullptr;
   void* scratch = ws + L.e_scratch;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (p.tc_dy) {
+      // dX and dY as band products on the tensor cores; the positives' dY by their pairs
+      stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
+      cudaError_t e = launch_dx_tc(p, Y, targets, lse, dloss, ws, dX, status, st);
+      if (e != cudaSuccess) return e;
+      stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
+      stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
+      // the merge stored each row's positive logit: a k = 0 plan's logits [N][1]
+      e = launch_backward(*p.pos_plan, X, Y, targets, selected, lse,
+                          reinterpret_cast<const float*>(ws + L.pos_logit), dloss, ws,
+                          static_cast<float*>(nullptr), dY, status, st);
+      if (e != cudaSuccess) return e;
+      stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
+      stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
+      e = launch_dy_tc(p, dloss, ws, dY, status, st);
+      stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
+      return e;
+    }
+  }
   stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
   if (c.N > 0) {
     const size_t per_warp = bwd_rows_warp_bytes(c.d, c.k);

@@ -111,7 +111,7 @@ __device__ __forceinline__ void row_window(int64_t p, int64_t N, int64_t C, int 
 struct Args {
   int64_t N, C;
   int d, k, n_c, n_ec, r, ns, nb, Sp;
-  const int32_t* px;        // [n_r][N] sorted row -> row
+  const int32_t* px;        // [n_r][N] sorted row -> row (dY: py, sorted position -> item)
   const int2* kept;         // [n_r][N][k] (sorted position, p as bf16 hi | lo << 16)
   const int32_t* kept_off;  // [n_r][N][Sp] slice starts within the round's entries
   const float* dloss;       // [1]
@@ -322,6 +322,195 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
   }
 }
 
+// dY of step 6 on the tensor cores: per (round r, 128 sorted catalogue positions) the
+// band product G_r[rows, positions]^T Xs_r[rows].  K = the rows whose windows cover the
+// positions, in slabs of 64 rows.  Each builder thread owns one row of the slab and one
+// 64-position half of the tile: it writes its row's kept entries there into the tile
+// (items x rows, K-major: another thread's M row, so the tile is cleared, all builders
+// meet at a named barrier, then fill it).  TMA streams the slab of the d-major sorted copy
+// XsT, the MMAs and the epilogue are the dX kernel's; the epilogue adds into dY at the
+// positions' item ids.  The positives' terms are written first (pair path), the rounds
+// add in round order: deterministic.
+__global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant__ CUtensorMap tmB,
+                                                        const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* A_hi = base;
+  uint8_t* A_lo = base + kAStages * kATile;
+  uint8_t* Bs = base + 2 * kAStages * kATile;
+  const uint32_t b_bytes = uint32_t(a.ns) * 128u;
+  Ctl& ctl = *reinterpret_cast<Ctl*>(Bs + size_t(a.nb) * b_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  const int nb = a.nb;
+  const int64_t N = a.N, C = a.C;
+  const int r = a.r, n0 = blockIdx.y * a.ns;
+
+  // the tile's positions and its K range [lo, hi) of 64-row slabs
+  const int64_t q0 = int64_t(blockIdx.x) * kBM;
+  int64_t k0 = 0, k1 = 0, lo = 0, hi = 0;
+  {
+    const int64_t last = (q0 + kBM - 1 < C - 1) ? q0 + kBM - 1 : C - 1;
+    const int64_t cf = chunk_of(q0, C, a.n_c), cl = chunk_of(last, C, a.n_c);
+    k0 = chunk_start(cf - a.n_ec < 0 ? 0 : cf - a.n_ec, N, a.n_c);
+    k1 = chunk_start(cl + a.n_ec + 1 > a.n_c ? a.n_c : cl + a.n_ec + 1, N, a.n_c);
+    if (k1 > k0) {
+      lo = k0 >> 6;
+      hi = (k1 + 63) >> 6;
+    }
+  }
+  const int nK = int(hi - lo);
+
+  if (t == 0) {
+    for (int i = 0; i < nb; ++i) {
+      mbar_init(&ctl.bfull[i], 1);
+      mbar_init(&ctl.bempty[i], 1);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&ctl.afull[i], kBuilders / 32);
+      mbar_init(&ctl.aempty[i], 1);
+    }
+    mbar_init(&ctl.done, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  const uint32_t tcols = a.ns <= 32 ? 32u : (a.ns <= 64 ? 64u : (a.ns <= 128 ? 128u : 256u));
+  if (warp == 4) {
+    tmem_alloc(&ctl.tmem_base, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmB);
+      int s = 0;
+      for (; s < nK; ++s) {
+        const int slot = s % nb;
+        if (!mbar_wait(&ctl.bempty[slot], ((s / nb) & 1) ^ 1, &ctl.abort, kTimeoutNs)) {
+          on_timeout(ctl, a.status);
+          break;
+        }
+        mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
+        tma_load_2d(Bs + size_t(slot) * b_bytes, &tmB, &ctl.bfull[slot], int((lo + s) * kBK),
+                    r * a.d + n0);
+      }
+      for (int j = (s > nb ? s - nb : 0); j < s; ++j)
+        mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1, kTimeoutNs);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, a.ns);
+      for (int s = 0; s < nK; ++s) {
+        const int as = s % kAStages, bs = s % nb;
+        if (!mbar_wait(&ctl.afull[as], (s / kAStages) & 1, &ctl.abort, kTimeoutNs) ||
+            !mbar_wait(&ctl.bfull[bs], (s / nb) & 1, &ctl.abort, kTimeoutNs)) {
+          on_timeout(ctl, a.status);
+          break;
+        }
+        tc_fence_after();
+        const uint64_t dh = desc_k_sw128(smem_u32(A_hi + as * kATile));
+        const uint64_t dl = desc_k_sw128(smem_u32(A_lo + as * kATile));
+        const uint64_t db = desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes));
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          mma_bf16(tmem, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
+          mma_bf16(tmem, dl + 2 * kk, db + 2 * kk, idesc, 1);
+        }
+        mma_commit(&ctl.aempty[as]);
+        mma_commit(&ctl.bempty[bs]);
+      }
+      mma_commit(&ctl.done);
+      mbar_wait_limit(&ctl.done, 0, kTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------------------ builders
+    const int64_t rN = int64_t(r) * N;
+    const int kc = t & (kBK - 1);  // this thread's row within a slab (the tile's K column)
+    const int half = t >> 6;       // and its 64-position half of the tile
+    const int64_t slice = (q0 >> 6) + half;
+    bool ok = true;
+    for (int s = 0; s < nK; ++s) {
+      const int as = s % kAStages;
+      // every builder runs every slab to the named barriers, also after a timeout
+      if (ok && !mbar_wait(&ctl.aempty[as], ((s / kAStages) & 1) ^ 1, &ctl.abort, kTimeoutNs)) {
+        on_timeout(ctl, a.status);
+        ok = false;
+      }
+      uint8_t* th = A_hi + as * kATile;
+      uint8_t* tl = A_lo + as * kATile;
+      if (ok) {
+        zero_row(th, t);
+        zero_row(tl, t);
+      }
+      named_barrier(1, kBuilders);  // the whole tile is clear before anyone fills it
+      const int64_t p = (lo + s) * kBK + kc;  // sorted row
+      if (ok && p >= k0 && p < k1 && p < N) {
+        int64_t w0, w1;
+        row_window(p, N, C, a.n_c, a.n_ec, w0, w1);
+        const int64_t sig0 = w0 >> 6;
+        const int S = w1 > w0 ? int((w1 - 1) >> 6) - int(sig0) + 1 : 0;
+        const int64_t idx = slice - sig0;
+        if (idx >= 0 && idx < S) {
+          const int32_t* off = a.kept_off + (rN + p) * a.Sp;
+          const int e0 = __ldg(off + idx), e1 = __ldg(off + idx + 1);
+          const int2* ent = a.kept + (rN + p) * a.k;
+          for (int e = e0; e < e1; ++e) {
+            const int2 en = __ldg(ent + e);
+            const int m = int(en.x - q0);  // in [64 half, 64 half + 64)
+            put(th, tl, m, kc, uint32_t(en.y));
+          }
+        }
+      }
+      fence_proxy_async_smem();  // this thread's tile writes, visible to the MMA
+      named_barrier(1, kBuilders);  // nobody clears the next tile into this one's readers
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&ctl.afull[as]);
+    }
+    __syncwarp();
+
+    // ------------------------------------------------------------ epilogue
+    bool fin = ok && mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && nK > 0;
+    fin = __all_sync(0xFFFFFFFFu, fin);
+    tc_fence_after();
+    const float scale = a.dloss[0] / float(N);  // G holds p; g = p * dloss / N
+    const int64_t q = q0 + t;                   // this thread's sorted position
+    const bool live = q < C;
+    const int64_t dst = live ? a.px[int64_t(r) * C + q] : 0;
+    float* o = a.out + dst * a.d + n0;
+    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+    if (fin) {
+      for (int c0 = 0; c0 < a.ns; c0 += 32) {
+        float v[32];
+        tmem_load32(taddr + uint32_t(c0), v);
+        if (live) {
+          float4* qq = reinterpret_cast<float4*>(o + c0);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4 x = qq[u];
+            x.x = fmaf(scale, v[4 * u], x.x);
+            x.y = fmaf(scale, v[4 * u + 1], x.y);
+            x.z = fmaf(scale, v[4 * u + 2], x.z);
+            x.w = fmaf(scale, v[4 * u + 3], x.w);
+            qq[u] = x;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
+  }
+}
+
 // One warp per row: the positive's coefficient g_iz and dX_i = g_iz y_z (written, not
 // added: the rounds add after it).
 template <typename T>
@@ -396,6 +585,49 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
     k_bwd_dx_tc<<<dim3(unsigned(ceil_div(c.N, kBM)), unsigned(slices)), kThreads, smem, st>>>(
+        tm, a);
+    count_launches(1);
+    RECE_TRY(cudaGetLastError());
+  }
+  return cudaSuccess;
+}
+
+// The window terms of dY, added into dY round by round (its positives' terms first).
+cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, float* dY,
+                         uint32_t* status, cudaStream_t st) {
+  const auto& c = p.cfg;
+  const Layout& L = p.lay;
+  if (c.N == 0) return cudaSuccess;
+  int ns = c.d;
+  if (ns > 256) ns = (c.d % 256 == 0) ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64));
+  const int slices = c.d / ns;
+  int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(ns) * 128));
+  nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
+  const size_t smem = smem_bytes(nb, ns);
+  Args a{};
+  a.N = c.N;
+  a.C = c.C;
+  a.d = c.d;
+  a.k = c.k;
+  a.n_c = c.n_c;
+  a.n_ec = c.n_ec;
+  a.ns = ns;
+  a.nb = nb;
+  a.Sp = p.kept_slices + 1;
+  a.px = reinterpret_cast<const int32_t*>(ws + L.py);
+  a.kept = reinterpret_cast<const int2*>(ws + L.kept);
+  a.kept_off = reinterpret_cast<const int32_t*>(ws + L.kept_off);
+  a.dloss = dloss;
+  a.status = status;
+  a.out = dY;
+  RECE_TRY(cudaFuncSetAttribute(k_bwd_dy_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(smem)));
+  CUtensorMap tm;
+  RECE_TRY(make_tmap_bf16_ld(&tm, ws + L.xst, uint64_t(c.n_r) * c.d, uint64_t(c.N), p.ld_n,
+                             uint32_t(ns)));
+  for (int r = 0; r < c.n_r; ++r) {
+    a.r = r;
+    k_bwd_dy_tc<<<dim3(unsigned(ceil_div(c.C, kBM)), unsigned(slices)), kThreads, smem, st>>>(
         tm, a);
     count_launches(1);
     RECE_TRY(cudaGetLastError());

@@ -99,13 +99,15 @@ struct rece_plan_s {
   bool sigmoid_g;       // backward coefficients sigmoid(l) - [positive] (BCE+), else softmax
   bool use_tc;          // bf16 mode on the tcgen05 kernels
   bool tc_dx;           // ... and dX of the backward on them too
+  bool tc_dy;           // ... and dY (band products; positives through pos_plan's pairs)
   bool tc_scores;       // ... with the window scores computed once and stored (large d)
   int64_t score_width;  // columns of the stored scores per row (longest union, padded)
   int32_t kept_slices;  // most 64-position slices one window touches
   int64_t ld_c;         // row pitch (elements) of the d-major copy of Y: C rounded up to 8
   int64_t ld_n;         // ... and of X (all-negatives mode): N rounded up to 8
   bool all_neg;         // RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed, no top-k
-  rece_plan_s* pos_plan;  // all-negatives mode: the positives' pair backward (k = 0)
+  rece_plan_s* pos_plan;  // all-negatives mode and tensor-core dY: the positives' pair
+                          // backward (k = 0)
   rece::Layout lay;
   void* stage_events[2 * RECE_NUM_STAGES];  // optional timing hook (cudaEvent_t)
   bool timed;

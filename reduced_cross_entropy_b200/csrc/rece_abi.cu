@@ -158,6 +158,7 @@ void build_layout(rece_plan_s& p) {
     L.px = take(sizeof(int32_t) * c.n_r * c.N);
     L.py = take(sizeof(int32_t) * c.n_r * c.C);
   }
+  if (p.tc_dy) L.xst = take(sizeof(uint16_t) * size_t(c.n_r) * c.d * p.ld_n);
   if (p.tc_dx) {
     L.yst = take(sizeof(uint16_t) * size_t(c.n_r) * c.d * p.ld_c);
     L.kept = take(sizeof(int2) * size_t(c.n_r) * c.N * c.k);
@@ -438,7 +439,31 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     delete p;
     return fail(RECE_ERR_UNSUPPORTED, "n_r * k too large for the tensor-core merge");
   }
+  p->tc_dy = false;
+  if (p->tc_dx && !p->all_neg && c.d >= 1024) {
+    // dY as band products too (at large d: each x row gathered per pair is 2d bytes,
+    // while the band's builders cost the same per slab whatever d); the positives' dY
+    // through a pair backward of k = 0 that shares the pair region (N pairs fit where
+    // N (k + 1) do)
+    rece_plan_s* q = new (std::nothrow) rece_plan_s();
+    if (!q) {
+      delete p;
+      return fail(RECE_ERR_INVALID_ARG, "out of host memory");
+    }
+    *q = *p;
+    q->cfg.k = 0;
+    q->use_tc = q->tc_dx = q->tc_dy = q->tc_scores = false;
+    q->timed = false;
+    q->pos_plan = nullptr;
+    set_pair_sort(*q);
+    p->pos_plan = q;
+    p->tc_dy = true;
+  }
   build_layout(*p);
+  if (p->tc_dy) {
+    p->pos_plan->lay = p->lay;  // the main plan's pair arrays and status words
+    p->pos_plan->carry_g = p->carry_g && p->pos_plan->carry_g;
+  }
   *out = p;
   return RECE_OK;
 }
@@ -486,7 +511,8 @@ rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
   *paths = (plan->use_tc ? RECE_PATH_TENSOR_CORES : 0u) |
            (plan->tc_dx ? RECE_PATH_DX_TENSORS : 0u) |
            (plan->tc_scores ? RECE_PATH_STORED_SCORES : 0u) |
-           (plan->all_neg ? RECE_PATH_ALL_NEGATIVES : 0u);
+           (plan->all_neg ? RECE_PATH_ALL_NEGATIVES : 0u) |
+           (plan->tc_dy ? RECE_PATH_DY_TENSORS : 0u);
   return RECE_OK;
 }
 
@@ -567,6 +593,9 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
     if (plan->tc_dx)
       RECE_CUDA(launch_transpose_sorted(ws + L.ys, c.C, c.d, c.n_r, plan->ld_c, ws + L.yst, st),
                 "d-major copy of Y");
+    if (plan->tc_dy)
+      RECE_CUDA(launch_transpose_sorted(ws + L.xs, c.N, c.d, c.n_r, plan->ld_n, ws + L.xst, st),
+                "d-major copy of X");
   }
   stage_mark(*plan, RECE_STAGE_SORT, 1, st);
   return RECE_OK;

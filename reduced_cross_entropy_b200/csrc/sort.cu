@@ -250,23 +250,31 @@ __global__ void __launch_bounds__(kSortThreads, 4) k_sort_scatter(const __grid_c
 }
 
 // start[j] = first position p of sorted (non-decreasing) keys with key >= j, j in [0, n_vals]:
-// thread p fills the starts of the values between key[p-1] and key[p].
+// one thread per value, a binary search.  (Filling the gap below each key from the key's
+// own thread left one thread to write every value above the largest key, millions of them
+// when the keys are few and crowd the low values, as a batch's Zipf-drawn targets do.)
 __global__ void __launch_bounds__(256) k_segment_starts(const int32_t* __restrict__ sorted,
                                                         int64_t M, int32_t n_vals,
                                                         int32_t* __restrict__ start) {
-  const int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (p > M) return;
-  const int32_t prev = p > 0 ? sorted[p - 1] : -1;
-  int32_t cur = p < M ? sorted[p] : n_vals;
-  if (cur > n_vals) cur = n_vals;
-  for (int32_t j = prev + 1; j <= cur; ++j) start[j] = int32_t(p);
+  for (int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; j <= n_vals;
+       j += int64_t(gridDim.x) * blockDim.x) {
+    int64_t lo = 0, hi = M;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi) >> 1;
+      if (__ldg(sorted + mid) < j) lo = mid + 1;
+      else hi = mid;
+    }
+    start[j] = int32_t(lo);
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_segment_starts(const int32_t* sorted, int64_t M, int32_t n_vals,
                                   int32_t* start, cudaStream_t st) {
-  k_segment_starts<<<unsigned(ceil_div(M + 1, 256)), 256, 0, st>>>(sorted, M, n_vals, start);
+  const int64_t want = ceil_div(int64_t(n_vals) + 1, 256);
+  k_segment_starts<<<unsigned(want < 32 * 148 ? want : 32 * 148), 256, 0, st>>>(sorted, M,
+                                                                               n_vals, start);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -78,6 +78,11 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
                          const float* lse, const float* dloss, char* ws, float* dX,
                          uint32_t* status, cudaStream_t st);
 
+// dY of step 6 on tensor cores: the rounds' window terms, added into dY (the positives'
+// terms already in it).  Needs the grouped kept entries and the d-major copy XsT.
+cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, float* dY,
+                         uint32_t* status, cudaStream_t st);
+
 // All-negatives mode (Algorithm 1 as printed; window.cu, window_tc.cu).  Per-round chunk
 // tables chunks[(r * n_r + s) * M + p] of the row (item) at sorted position p of round r,
 // and for the rows the sorted position of their positive (pz [n_r][N], -1 for none).
