@@ -433,6 +433,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
     const int kc = t & (kBK - 1);  // this thread's row within a slab (the tile's K column)
     const int half = t >> 6;       // and its 64-position half of the tile
     const int64_t slice = (q0 >> 6) + half;
+    // the entries of slab s's row in this half: [e0, e1) of its kept list, found a slab
+    // ahead so that the offsets' load latency overlaps the previous slab
+    auto entry_range = [&](int s2, int& e0, int& e1) {
+      e0 = e1 = 0;
+      const int64_t p = (lo + s2) * kBK + kc;  // sorted row
+      if (s2 >= nK || p < k0 || p >= k1 || p >= N) return;
+      int64_t w0, w1;
+      row_window(p, N, C, a.n_c, a.n_ec, w0, w1);
+      const int64_t sig0 = w0 >> 6;
+      const int S = w1 > w0 ? int((w1 - 1) >> 6) - int(sig0) + 1 : 0;
+      const int64_t idx = slice - sig0;
+      if (idx < 0 || idx >= S) return;
+      const int32_t* off = a.kept_off + (rN + p) * a.Sp;
+      e0 = __ldg(off + idx);
+      e1 = __ldg(off + idx + 1);
+    };
+    int nx0, nx1;
+    entry_range(0, nx0, nx1);
     bool ok = true;
     for (int s = 0; s < nK; ++s) {
       const int as = s % kAStages;
@@ -448,22 +466,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
         zero_row(tl, t);
       }
       named_barrier(1, kBuilders);  // the whole tile is clear before anyone fills it
-      const int64_t p = (lo + s) * kBK + kc;  // sorted row
-      if (ok && p >= k0 && p < k1 && p < N) {
-        int64_t w0, w1;
-        row_window(p, N, C, a.n_c, a.n_ec, w0, w1);
-        const int64_t sig0 = w0 >> 6;
-        const int S = w1 > w0 ? int((w1 - 1) >> 6) - int(sig0) + 1 : 0;
-        const int64_t idx = slice - sig0;
-        if (idx >= 0 && idx < S) {
-          const int32_t* off = a.kept_off + (rN + p) * a.Sp;
-          const int e0 = __ldg(off + idx), e1 = __ldg(off + idx + 1);
-          const int2* ent = a.kept + (rN + p) * a.k;
-          for (int e = e0; e < e1; ++e) {
-            const int2 en = __ldg(ent + e);
-            const int m = int(en.x - q0);  // in [64 half, 64 half + 64)
-            put(th, tl, m, kc, uint32_t(en.y));
-          }
+      const int e0 = nx0, e1 = nx1;
+      entry_range(s + 1, nx0, nx1);
+      if (ok && e1 > e0) {
+        const int2* ent = a.kept + (rN + (lo + s) * kBK + kc) * a.k;
+        for (int e = e0; e < e1; e += 8) {  // eight loads in flight
+          int2 en[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) en[u] = e + u < e1 ? __ldg(ent + e + u) : make_int2(0, 0);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (e + u < e1) put(th, tl, int(en[u].x - q0), kc, uint32_t(en[u].y));
         }
       }
       fence_proxy_async_smem();  // this thread's tile writes, visible to the MMA
