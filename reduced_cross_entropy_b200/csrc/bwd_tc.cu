@@ -168,7 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
     ctl.abort = 0;
     fence_mbar_init();
   }
-  const uint32_t tcols = a.ns <= 32 ? 32u : (a.ns <= 64 ? 64u : (a.ns <= 128 ? 128u : 256u));
+  const uint32_t tcols =
+      a.ns <= 32 ? 32u : (a.ns <= 64 ? 64u : (a.ns <= 128 ? 128u : (a.ns <= 256 ? 256u : 512u)));
   if (warp == 4) {
     tmem_alloc(&ctl.tmem_base, tcols);
     tmem_relinquish();
@@ -190,8 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
           break;
         }
         mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
-        tma_load_2d(Bs + size_t(slot) * b_bytes, &tmB, &ctl.bfull[slot], int((lo + s) * kBK),
-                    r * a.d + n0);
+        for (int h = 0; h < a.ns; h += 256)  // boxes of at most 256 rows of d
+          tma_load_2d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
+                      int((lo + s) * kBK), r * a.d + n0 + h);
       }
       for (int j = (s > nb ? s - nb : 0); j < s; ++j)  // every issued copy has landed
         mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1, kTimeoutNs);
@@ -199,7 +201,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, a.ns);
+      // a slice of 512 columns is two MMAs of N = 256 into two accumulators
+      const int nh = a.ns > 256 ? 2 : 1, nsh = a.ns / nh;
+      const uint32_t idesc = idesc_bf16_f32(kBM, nsh);
       for (int s = 0; s < nK; ++s) {
         const int as = s % kAStages, bs = s % nb;
         if (!mbar_wait(&ctl.afull[as], (s / kAStages) & 1, &ctl.abort, kTimeoutNs) ||
@@ -210,11 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
         tc_fence_after();
         const uint64_t dh = desc_k_sw128(smem_u32(A_hi + as * kATile));
         const uint64_t dl = desc_k_sw128(smem_u32(A_lo + as * kATile));
-        const uint64_t db = desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes));
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
-          mma_bf16(tmem, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
-          mma_bf16(tmem, dl + 2 * kk, db + 2 * kk, idesc, 1);
+          for (int h = 0; h < nh; ++h) {
+            const uint64_t db =
+                desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128));
+            const uint32_t acc = tmem + uint32_t(h * nsh);
+            mma_bf16(acc, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
+            mma_bf16(acc, dl + 2 * kk, db + 2 * kk, idesc, 1);
+          }
         }
         mma_commit(&ctl.aempty[as]);
         mma_commit(&ctl.bempty[bs]);
@@ -373,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
     ctl.abort = 0;
     fence_mbar_init();
   }
-  const uint32_t tcols = a.ns <= 32 ? 32u : (a.ns <= 64 ? 64u : (a.ns <= 128 ? 128u : 256u));
+  const uint32_t tcols =
+      a.ns <= 32 ? 32u : (a.ns <= 64 ? 64u : (a.ns <= 128 ? 128u : (a.ns <= 256 ? 256u : 512u)));
   if (warp == 4) {
     tmem_alloc(&ctl.tmem_base, tcols);
     tmem_relinquish();
@@ -395,8 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
           break;
         }
         mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
-        tma_load_2d(Bs + size_t(slot) * b_bytes, &tmB, &ctl.bfull[slot], int((lo + s) * kBK),
-                    r * a.d + n0);
+        for (int h = 0; h < a.ns; h += 256)  // boxes of at most 256 rows of d
+          tma_load_2d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
+                      int((lo + s) * kBK), r * a.d + n0 + h);
       }
       for (int j = (s > nb ? s - nb : 0); j < s; ++j)
         mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1, kTimeoutNs);
@@ -404,7 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, a.ns);
+      // a slice of 512 columns is two MMAs of N = 256 into two accumulators
+      const int nh = a.ns > 256 ? 2 : 1, nsh = a.ns / nh;
+      const uint32_t idesc = idesc_bf16_f32(kBM, nsh);
       for (int s = 0; s < nK; ++s) {
         const int as = s % kAStages, bs = s % nb;
         if (!mbar_wait(&ctl.afull[as], (s / kAStages) & 1, &ctl.abort, kTimeoutNs) ||
@@ -415,11 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
         tc_fence_after();
         const uint64_t dh = desc_k_sw128(smem_u32(A_hi + as * kATile));
         const uint64_t dl = desc_k_sw128(smem_u32(A_lo + as * kATile));
-        const uint64_t db = desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes));
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
-          mma_bf16(tmem, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
-          mma_bf16(tmem, dl + 2 * kk, db + 2 * kk, idesc, 1);
+          for (int h = 0; h < nh; ++h) {
+            const uint64_t db =
+                desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128));
+            const uint32_t acc = tmem + uint32_t(h * nsh);
+            mma_bf16(acc, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
+            mma_bf16(acc, dl + 2 * kk, db + 2 * kk, idesc, 1);
+          }
         }
         mma_commit(&ctl.aempty[as]);
         mma_commit(&ctl.bempty[bs]);
@@ -559,9 +575,11 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   const auto& c = p.cfg;
   const Layout& L = p.lay;
   if (c.N == 0) return cudaSuccess;
-  // d is split into CTA slices of ns <= 256 columns (one TMEM accumulator each)
+  // d is split into CTA slices of ns <= 512 columns (two TMEM accumulators past 256)
   int ns = c.d;
-  if (ns > 256) ns = (c.d % 256 == 0) ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64));
+  if (ns > 256)
+    ns = (c.d % 512 == 0) ? 512
+                          : (c.d % 256 == 0 ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64)));
   const int slices = c.d / ns;
   // TMA ring: as deep as lets two CTAs share an SM (at least two slabs)
   int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(ns) * 128));
@@ -594,7 +612,7 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
                                 int(smem)));
   CUtensorMap tm;
   RECE_TRY(make_tmap_bf16_ld(&tm, ws + L.yst, uint64_t(c.n_r) * c.d, uint64_t(c.C), p.ld_c,
-                             uint32_t(ns)));
+                             uint32_t(ns < 256 ? ns : 256)));
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
     k_bwd_dx_tc<<<dim3(unsigned(ceil_div(c.N, kBM)), unsigned(slices)), kThreads, smem, st>>>(
@@ -611,8 +629,11 @@ cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, flo
   const auto& c = p.cfg;
   const Layout& L = p.lay;
   if (c.N == 0) return cudaSuccess;
+  // d is split into CTA slices of ns <= 512 columns (two TMEM accumulators past 256)
   int ns = c.d;
-  if (ns > 256) ns = (c.d % 256 == 0) ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64));
+  if (ns > 256)
+    ns = (c.d % 512 == 0) ? 512
+                          : (c.d % 256 == 0 ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64)));
   const int slices = c.d / ns;
   int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(ns) * 128));
   nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
@@ -637,7 +658,7 @@ cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, flo
                                 int(smem)));
   CUtensorMap tm;
   RECE_TRY(make_tmap_bf16_ld(&tm, ws + L.xst, uint64_t(c.n_r) * c.d, uint64_t(c.N), p.ld_n,
-                             uint32_t(ns)));
+                             uint32_t(ns < 256 ? ns : 256)));
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
     k_bwd_dy_tc<<<dim3(unsigned(ceil_div(c.C, kBM)), unsigned(slices)), kThreads, smem, st>>>(
