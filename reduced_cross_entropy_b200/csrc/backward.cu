@@ -472,6 +472,104 @@ __global__ void __launch_bounds__(288) k_bwd_items_wide(
     __stcs(o + e, make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]));
 }
 
+// The run of equal keys holding position p: run_lo[p] its first position, run_hi[p] the
+// first past it (two binary searches per position).
+__global__ void __launch_bounds__(256) k_runs(const int32_t* __restrict__ key, int64_t E,
+                                              int32_t* __restrict__ run_lo,
+                                              int32_t* __restrict__ run_hi) {
+  const int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (p >= E) return;
+  const int32_t j = key[p];
+  int64_t lo = 0, hi = p;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (key[mid] < j) lo = mid + 1;
+    else hi = mid;
+  }
+  run_lo[p] = int32_t(lo);
+  lo = p + 1;
+  hi = E;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (key[mid] <= j) lo = mid + 1;
+    else hi = mid;
+  }
+  run_hi[p] = int32_t(lo);
+}
+
+constexpr int kSeg = 32;  // pairs per segment of a run
+
+// The positives' terms of dY, in two levels so that a popular target's long run (the
+// targets are Zipf-drawn) is summed in parallel.  Level 1: one warp per (segment of up to
+// 32 pairs of a run, 256 columns of d), eight pairs' rows in flight, pairs in order; a run
+// of one segment adds its sum into the item's row, a longer run leaves each segment's sum
+// in part[first position of the segment].  Level 2 (k_pos_dy_runs): the run's first
+// position adds the parts in order.  Deterministic.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_pos_dy_seg(
+    const T* __restrict__ X, int64_t C, int d, int slots, const int32_t* __restrict__ key,
+    const int32_t* __restrict__ run_lo, const int32_t* __restrict__ run_hi,
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ pair_g, int64_t E,
+    float* __restrict__ part, float* __restrict__ dY) {
+  const int lane = threadIdx.x & 31;
+  const int64_t p = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  if (p >= E) return;
+  const int32_t j = key[p];
+  const int64_t r0 = run_lo[p], r1 = run_hi[p];
+  if (j >= C || (p - r0) % kSeg != 0) return;
+  const int t0 = blockIdx.y * 256 + 8 * lane;
+  if (t0 >= d) return;
+  const int64_t q1 = p + kSeg < r1 ? p + kSeg : r1;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int64_t q = p; q < q1; q += 8) {
+    float v[8][8], gq[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      gq[u] = 0.0f;
+      if (q + u < q1) {
+        const int32_t id = sorted_id[q + u];
+        gq[u] = pair_g[id];
+        load8(X + int64_t(id / slots) * d + t0, v[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (q + u < q1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(gq[u], v[u][e], acc[e]);
+      }
+  }
+  float4* o = reinterpret_cast<float4*>(r1 - r0 <= kSeg ? dY + int64_t(j) * d + t0
+                                                         : part + p * d + t0);
+  if (r1 - r0 <= kSeg) {
+    float4 a0 = o[0], a1 = o[1];
+    a0.x += acc[0]; a0.y += acc[1]; a0.z += acc[2]; a0.w += acc[3];
+    a1.x += acc[4]; a1.y += acc[5]; a1.z += acc[6]; a1.w += acc[7];
+    o[0] = a0;
+    o[1] = a1;
+  } else {
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) k_pos_dy_runs(
+    int64_t C, int d, const int32_t* __restrict__ key, const int32_t* __restrict__ run_lo,
+    const int32_t* __restrict__ run_hi, int64_t E, const float* __restrict__ part,
+    float* __restrict__ dY) {
+  const int lane = threadIdx.x & 31;
+  const int64_t p = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  if (p >= E) return;
+  const int32_t j = key[p];
+  const int64_t r1 = run_hi[p];
+  if (j >= C || run_lo[p] != p || r1 - p <= kSeg) return;
+  for (int t = blockIdx.y * 256 + lane; t < d && t < int(blockIdx.y + 1) * 256; t += 32) {
+    float sum = 0.0f;
+    for (int64_t q = p; q < r1; q += kSeg) sum += part[q * d + t];
+    dY[int64_t(j) * d + t] += sum;
+  }
+}
+
 }  // namespace
 
 size_t bwd_rows_warp_bytes(int d, int k) { return sizeof(float) * size_t(d + 2 * (k + 1)); }
@@ -528,22 +626,52 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
   void* scratch = ws + L.e_scratch;
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     if (p.tc_dy) {
-      // dX and dY as band products on the tensor cores; the positives' dY by their pairs
+      // dX and dY as band products on the tensor cores (dY written by round 0, added by
+      // the others), then the positives' dY terms added from their sorted pairs
       stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
       cudaError_t e = launch_dx_tc(p, Y, targets, lse, dloss, ws, dX, status, st);
       if (e != cudaSuccess) return e;
       stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
-      stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
-      // the merge stored each row's positive logit: a k = 0 plan's logits [N][1]
-      e = launch_backward(*p.pos_plan, X, Y, targets, selected, lse,
-                          reinterpret_cast<const float*>(ws + L.pos_logit), dloss, ws,
-                          static_cast<float*>(nullptr), dY, status, st);
-      if (e != cudaSuccess) return e;
-      stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
       stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
       e = launch_dy_tc(p, dloss, ws, dY, status, st);
+      if (e != cudaSuccess) return e;
       stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
-      return e;
+      stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
+      const rece_plan_s& q = *p.pos_plan;  // k = 0: one slot per row, its positive
+      if (c.N > 0) {
+        const size_t per_warp = bwd_rows_warp_bytes(c.d, 0);
+        int warps = int((200 * 1024) / per_warp);
+        warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
+        // the merge stored each row's positive logit: a k = 0 plan's logits [N][1]
+        const float* plog = reinterpret_cast<const float*>(ws + L.pos_logit);
+        e = cudaFuncSetAttribute(k_bwd_rows_v8<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(per_warp * warps));
+        if (e != cudaSuccess) return e;
+        k_bwd_rows_v8<T><<<unsigned(ceil_div(c.N, warps)), warps * 32, per_warp * warps, st>>>(
+            X, Y, targets, selected, lse, plog, dloss, c.N, c.C, c.d, 0, e_key, e_g, nullptr,
+            status, false);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int32_t* in = nullptr;
+        e = sort_pairs_by_item(q, c.N, e_key, nullptr, perm_a, perm_b,
+                               reinterpret_cast<int32_t*>(ws + L.e_key_b), nullptr, sorted_key,
+                               nullptr, scratch, &in, st);
+        if (e != cudaSuccess) return e;
+        // the runs of equal targets, in the arrays the sort no longer needs
+        int32_t* run_lo = reinterpret_cast<int32_t*>(ws + L.e_key_b);
+        int32_t* run_hi = const_cast<int32_t*>(in) == perm_a ? perm_b : perm_a;
+        float* part = reinterpret_cast<float*>(ws + L.pos_parts);
+        const dim3 grid(unsigned(ceil_div(c.N, kThreads / 32)), unsigned(ceil_div(c.d, 256)));
+        k_runs<<<unsigned(ceil_div(c.N, 256)), 256, 0, st>>>(sorted_key, c.N, run_lo, run_hi);
+        k_pos_dy_seg<T><<<grid, kThreads, 0, st>>>(X, c.C, c.d, 1, sorted_key, run_lo, run_hi,
+                                                   in, e_g, c.N, part, dY);
+        k_pos_dy_runs<<<grid, kThreads, 0, st>>>(c.C, c.d, sorted_key, run_lo, run_hi, c.N,
+                                                 part, dY);
+        count_launches(3);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      }
+      stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
+      return cudaSuccess;
     }
   }
   stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);

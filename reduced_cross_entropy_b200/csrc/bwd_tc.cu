@@ -117,6 +117,7 @@ struct Args {
   const float* dloss;       // [1]
   float* out;               // dX [N][d], accumulated into
   uint32_t* status;
+  int write;                // dY: store (round 0, which covers every position), else add
 };
 
 __device__ __forceinline__ void on_timeout(Ctl& c, uint32_t* status) {
@@ -516,7 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
       for (int c0 = 0; c0 < a.ns; c0 += 32) {
         float v[32];
         tmem_load32(taddr + uint32_t(c0), v);
-        if (live) {
+        if (live && a.write) {
+          float4* qq = reinterpret_cast<float4*>(o + c0);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            qq[u] = make_float4(scale * v[4 * u], scale * v[4 * u + 1], scale * v[4 * u + 2],
+                                scale * v[4 * u + 3]);
+        } else if (live) {
           float4* qq = reinterpret_cast<float4*>(o + c0);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -623,7 +630,8 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   return cudaSuccess;
 }
 
-// The window terms of dY, added into dY round by round (its positives' terms first).
+// The window terms of dY: round 0 stores them (its tiles cover every catalogue position),
+// the later rounds add.
 cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, float* dY,
                          uint32_t* status, cudaStream_t st) {
   const auto& c = p.cfg;
@@ -661,6 +669,7 @@ cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, flo
                              uint32_t(ns < 256 ? ns : 256)));
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
+    a.write = r == 0;
     k_bwd_dy_tc<<<dim3(unsigned(ceil_div(c.C, kBM)), unsigned(slices)), kThreads, smem, st>>>(
         tm, a);
     count_launches(1);

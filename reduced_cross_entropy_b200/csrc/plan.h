@@ -79,6 +79,8 @@ struct Layout {
   // only: the rounds' (max, sum) pairs and the inverse orders of Y
   size_t xst = 0, itemc = 0, rowc = 0, pz = 0, lse_sorted = 0, ms = 0, inv_y = 0,
          dx_parts = 0;
+  // tensor-core dY: the positives' per-segment partial sums [N][d] (backward region)
+  size_t pos_parts = 0;
   size_t total = 0;
 };
 

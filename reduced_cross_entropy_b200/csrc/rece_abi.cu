@@ -197,6 +197,7 @@ void build_layout(rece_plan_s& p) {
   L.fwd_end = off;
   off = region;
   layout_pairs(p, off);
+  if (p.tc_dy) L.pos_parts = take(sizeof(float) * size_t(c.N) * c.d);
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }

@@ -78,8 +78,9 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
                          const float* lse, const float* dloss, char* ws, float* dX,
                          uint32_t* status, cudaStream_t st);
 
-// dY of step 6 on tensor cores: the rounds' window terms, added into dY (the positives'
-// terms already in it).  Needs the grouped kept entries and the d-major copy XsT.
+// dY of step 6 on tensor cores: the rounds' window terms, written by round 0 and added by
+// the others (the positives' terms are added after).  Needs the grouped kept entries and
+// the d-major copy XsT.
 cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, float* dY,
                          uint32_t* status, cudaStream_t st);
 
