@@ -23,9 +23,10 @@
 // epilogue applies the factor dloss / N.
 //
 // This pays where gathering the catalogue rows does not: at large d, or when the sorted
-// catalogue does not fit in L2.  (The transposed product for dY, G_r^T Xs_r per tile of
-// positions, was measured slower than the pair sort and gather on every shape tried: its
-// K ranges are short and every slice of d rebuilt the same tiles.)
+// catalogue does not fit in L2.  The transposed product for dY, G_r^T Xs_r per tile of
+// positions (k_bwd_dy_tc below), pays only at large d (d >= 1024): its K ranges are short
+// and every slice of d rebuilds the same tiles, against a pair sort and gather whose cost
+// per pair grows with d.
 //
 // Determinism: each dX row is written by one CTA per launch, in a fixed K order; the
 // positive term is written first (dX_i = g_iz y_z), then the rounds add in round order.
@@ -108,6 +109,45 @@ __device__ __forceinline__ void row_window(int64_t p, int64_t N, int64_t C, int 
   w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
 }
 
+// Epilogue of both band kernels: this thread's accumulator row (TMEM lane of the thread,
+// ns columns) times `scale` into out row o -- stored when `write`, else added.  The rows
+// are scattered (item ids or row ids of sorted positions), so each thread stages its row in
+// pieces of W columns in shared memory (two buffers over the G tiles and B ring, free once
+// the MMAs are done; rows padded by 16 B so that the float4 writes of 8 consecutive rows
+// hit distinct banks) and hands each piece to the bulk-copy engine: full lines reach
+// memory, and an add is done at L2 (the old values never come back to the SM).  One add
+// per element per launch: deterministic.  `fin` must be uniform across the warp (the TMEM
+// loads are warp-collective); rows with `live` false load but write nothing.
+__device__ __forceinline__ void epilogue_rows(uint8_t* stage, size_t avail, int t,
+                                              uint32_t taddr, int ns, float scale, bool live,
+                                              float* o, bool write) {
+  const int W = (ns % 128 == 0 && avail >= 2u * kBM * (128 * 4 + 16)) ? 128 : 64;
+  const int stride = W * 4 + 16;
+  for (int c0 = 0, piece = 0; c0 < ns; c0 += W, ++piece) {
+    float* srow =
+        reinterpret_cast<float*>(stage + size_t(piece & 1) * kBM * stride + size_t(t) * stride);
+    bulk_wait_read<1>();  // this thread's copy out of that buffer (two pieces ago)
+    for (int cc = 0; cc < W; cc += 32) {
+      float v[32];
+      tmem_load32(taddr + uint32_t(c0 + cc), v);
+      float4* s4 = reinterpret_cast<float4*>(srow + cc);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        s4[u] = make_float4(scale * v[4 * u], scale * v[4 * u + 1], scale * v[4 * u + 2],
+                            scale * v[4 * u + 3]);
+    }
+    if (live) {
+      fence_proxy_async_smem();
+      if (write)
+        bulk_store(o + c0, srow, uint32_t(W) * 4u);
+      else
+        bulk_reduce_add_f32(o + c0, srow, uint32_t(W) * 4u);
+      bulk_commit();
+    }
+  }
+  bulk_wait_all();
+}
+
 struct Args {
   int64_t N, C;
   int d, k, n_c, n_ec, r, ns, nb, Sp;
@@ -130,10 +170,10 @@ __device__ __forceinline__ void on_timeout(Ctl& c, uint32_t* status) {
 __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant__ CUtensorMap tmB,
                                                         const Args a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* A_hi = base;
-  uint8_t* A_lo = base + kAStages * kATile;
-  uint8_t* Bs = base + 2 * kAStages * kATile;
+  uint8_t* sbase = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* A_hi = sbase;
+  uint8_t* A_lo = sbase + kAStages * kATile;
+  uint8_t* Bs = sbase + 2 * kAStages * kATile;
   const uint32_t b_bytes = uint32_t(a.ns) * 128u;
   Ctl& ctl = *reinterpret_cast<Ctl*>(Bs + size_t(a.nb) * b_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
@@ -297,30 +337,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
     __syncwarp();
 
     // ------------------------------------------------------------ epilogue
-    const bool ok = mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && nK > 0;
+    bool ok = mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && nK > 0;
+    ok = __all_sync(0xFFFFFFFFu, ok);
     const float scale = a.dloss[0] / float(N);  // G holds p; g = p * dloss / N
     tc_fence_after();
     const int64_t row = m0 + t;  // this thread's sorted row
     const bool live = row < N;
     const int64_t dst = live ? a.px[rN + row] : 0;
-    float* o = a.out + dst * a.d + n0;
-    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
-    for (int c0 = 0; c0 < a.ns; c0 += 32) {
-      float v[32];
-      tmem_load32(taddr + uint32_t(c0), v);
-      if (ok && live) {
-        float4* q = reinterpret_cast<float4*>(o + c0);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          float4 x = q[u];
-          x.x = fmaf(scale, v[4 * u], x.x);
-          x.y = fmaf(scale, v[4 * u + 1], x.y);
-          x.z = fmaf(scale, v[4 * u + 2], x.z);
-          x.w = fmaf(scale, v[4 * u + 3], x.w);
-          q[u] = x;
-        }
-      }
-    }
+    if (ok)
+      epilogue_rows(sbase, size_t(2 * kAStages) * kATile + size_t(nb) * b_bytes, t,
+                    tmem + (uint32_t(warp * 32) << 16), a.ns, scale, live,
+                    a.out + dst * a.d + n0, false);
   }
   tc_fence_before();
   __syncthreads();
@@ -338,8 +365,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
 // (items x rows, K-major: another thread's M row, so the tile is cleared, all builders
 // meet at a named barrier, then fill it).  TMA streams the slab of the d-major sorted copy
 // XsT, the MMAs and the epilogue are the dX kernel's; the epilogue adds into dY at the
-// positions' item ids.  The positives' terms are written first (pair path), the rounds
-// add in round order: deterministic.
+// positions' item ids.  Round 0 writes every catalogue row (its tiles cover all positions),
+// the later rounds add in round order, and the positives' terms are added after them (pair
+// path): deterministic.
 __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant__ CUtensorMap tmB,
                                                         const Args a) {
   extern __shared__ uint8_t smem_raw[];
@@ -511,32 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
     const int64_t q = q0 + t;                   // this thread's sorted position
     const bool live = q < C;
     const int64_t dst = live ? a.px[int64_t(r) * C + q] : 0;
-    float* o = a.out + dst * a.d + n0;
-    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
-    if (fin) {
-      for (int c0 = 0; c0 < a.ns; c0 += 32) {
-        float v[32];
-        tmem_load32(taddr + uint32_t(c0), v);
-        if (live && a.write) {
-          float4* qq = reinterpret_cast<float4*>(o + c0);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            qq[u] = make_float4(scale * v[4 * u], scale * v[4 * u + 1], scale * v[4 * u + 2],
-                                scale * v[4 * u + 3]);
-        } else if (live) {
-          float4* qq = reinterpret_cast<float4*>(o + c0);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            float4 x = qq[u];
-            x.x = fmaf(scale, v[4 * u], x.x);
-            x.y = fmaf(scale, v[4 * u + 1], x.y);
-            x.z = fmaf(scale, v[4 * u + 2], x.z);
-            x.w = fmaf(scale, v[4 * u + 3], x.w);
-            qq[u] = x;
-          }
-        }
-      }
-    }
+    if (fin)
+      epilogue_rows(base, size_t(2 * kAStages) * kATile + size_t(nb) * b_bytes, t,
+                    tmem + (uint32_t(warp * 32) << 16), a.ns, scale, live,
+                    a.out + dst * a.d + n0, a.write);
   }
   tc_fence_before();
   __syncthreads();
