@@ -15,8 +15,10 @@
 // A work item streams its window in slabs of 64 positions: four builder warps write the
 // slab's 128 x 64 tile of G into shared memory in the 128-byte-swizzled K-major layout
 // (zeros, then the row's entries of the slab, which come grouped by slab) while TMA brings
-// the matching 64-position slab of the d-major sorted copy YsT and one thread issues
-// tcgen05.mma into a TMEM accumulator of 128 x NS fp32 (NS <= 256 columns of d per CTA).
+// the matching 64 rows of the sorted copy Ys (64-column boxes, which the MMA reads as an
+// MN-major B operand: no transposed copy) and one thread issues
+// tcgen05.mma into TMEM accumulators of 128 x NS fp32 (NS <= 512 columns of d per CTA:
+// two accumulators of N = 256 past 256).
 // The tiles hold the negatives' softmax probabilities p_ij = exp(l_ij - lse_i), which the
 // merge stored split as hi + lo, both bf16 (hi = bf16(p), lo = bf16(p - hi)); both halves
 // are multiplied, so about 16 bits of p survive against 8 for a plain bf16 tile, and the
@@ -232,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
           break;
         }
         mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
-        for (int h = 0; h < a.ns; h += 256)  // boxes of at most 256 rows of d
-          tma_load_2d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
-                      int((lo + s) * kBK), r * a.d + n0 + h);
+        for (int h = 0; h < a.ns; h += 64)  // boxes of 64 columns of d x 64 positions
+          tma_load_3d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
+                      n0 + h, int((lo + s) * kBK), r);
       }
       for (int j = (s > nb ? s - nb : 0); j < s; ++j)  // every issued copy has landed
         mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1, kTimeoutNs);
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
     if (lane == 0) {
       // a slice of 512 columns is two MMAs of N = 256 into two accumulators
       const int nh = a.ns > 256 ? 2 : 1, nsh = a.ns / nh;
-      const uint32_t idesc = idesc_bf16_f32(kBM, nsh);
+      const uint32_t idesc = idesc_bf16_f32_bmn(kBM, nsh);  // B (rows of d) MN-major
       for (int s = 0; s < nK; ++s) {
         const int as = s % kAStages, bs = s % nb;
         if (!mbar_wait(&ctl.afull[as], (s / kAStages) & 1, &ctl.abort, kTimeoutNs) ||
@@ -258,11 +260,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           for (int h = 0; h < nh; ++h) {
+            // B: 64-column boxes 8 KB apart; 16 K rows of 128 B per MMA
             const uint64_t db =
-                desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128));
+                desc_mn_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128),
+                              8192u) + 128u * kk;
             const uint32_t acc = tmem + uint32_t(h * nsh);
-            mma_bf16(acc, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
-            mma_bf16(acc, dl + 2 * kk, db + 2 * kk, idesc, 1);
+            mma_bf16(acc, dh + 2 * kk, db, idesc, (s | kk) != 0);
+            mma_bf16(acc, dl + 2 * kk, db, idesc, 1);
           }
         }
         mma_commit(&ctl.aempty[as]);
@@ -363,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
 // positions, in slabs of 64 rows.  Each builder thread owns one row of the slab and one
 // 64-position half of the tile: it writes its row's kept entries there into the tile
 // (items x rows, K-major: another thread's M row, so the tile is cleared, all builders
-// meet at a named barrier, then fill it).  TMA streams the slab of the d-major sorted copy
-// XsT, the MMAs and the epilogue are the dX kernel's; the epilogue adds into dY at the
+// meet at a named barrier, then fill it).  TMA streams the slab's 64 rows of the sorted
+// copy Xs (MN-major B, as in the dX kernel), the MMAs and the epilogue are the dX kernel's; the epilogue adds into dY at the
 // positions' item ids.  Round 0 writes every catalogue row (its tiles cover all positions),
 // the later rounds add in round order, and the positives' terms are added after them (pair
 // path): deterministic.
@@ -433,9 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
           break;
         }
         mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
-        for (int h = 0; h < a.ns; h += 256)  // boxes of at most 256 rows of d
-          tma_load_2d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
-                      int((lo + s) * kBK), r * a.d + n0 + h);
+        for (int h = 0; h < a.ns; h += 64)  // boxes of 64 columns of d x 64 positions
+          tma_load_3d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
+                      n0 + h, int((lo + s) * kBK), r);
       }
       for (int j = (s > nb ? s - nb : 0); j < s; ++j)
         mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1, kTimeoutNs);
@@ -445,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
     if (lane == 0) {
       // a slice of 512 columns is two MMAs of N = 256 into two accumulators
       const int nh = a.ns > 256 ? 2 : 1, nsh = a.ns / nh;
-      const uint32_t idesc = idesc_bf16_f32(kBM, nsh);
+      const uint32_t idesc = idesc_bf16_f32_bmn(kBM, nsh);  // B (rows of d) MN-major
       for (int s = 0; s < nK; ++s) {
         const int as = s % kAStages, bs = s % nb;
         if (!mbar_wait(&ctl.afull[as], (s / kAStages) & 1, &ctl.abort, kTimeoutNs) ||
@@ -459,11 +463,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           for (int h = 0; h < nh; ++h) {
+            // B: 64-column boxes 8 KB apart; 16 K rows of 128 B per MMA
             const uint64_t db =
-                desc_k_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128));
+                desc_mn_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128),
+                              8192u) + 128u * kk;
             const uint32_t acc = tmem + uint32_t(h * nsh);
-            mma_bf16(acc, dh + 2 * kk, db + 2 * kk, idesc, (s | kk) != 0);
-            mma_bf16(acc, dl + 2 * kk, db + 2 * kk, idesc, 1);
+            mma_bf16(acc, dh + 2 * kk, db, idesc, (s | kk) != 0);
+            mma_bf16(acc, dl + 2 * kk, db, idesc, 1);
           }
         }
         mma_commit(&ctl.aempty[as]);
@@ -623,9 +629,9 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   RECE_TRY(cudaGetLastError());
   RECE_TRY(cudaFuncSetAttribute(k_bwd_dx_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(smem)));
-  CUtensorMap tm;
-  RECE_TRY(make_tmap_bf16_ld(&tm, ws + L.yst, uint64_t(c.n_r) * c.d, uint64_t(c.C), p.ld_c,
-                             uint32_t(ns < 256 ? ns : 256)));
+  CUtensorMap tm;  // the sorted rows of Y of every round, read MN-major
+  RECE_TRY(make_tmap_bf16_3d(&tm, ws + L.ys, uint64_t(c.d), uint64_t(c.C), uint64_t(c.n_r),
+                             uint32_t(kBK)));
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
     k_bwd_dx_tc<<<dim3(unsigned(ceil_div(c.N, kBM)), unsigned(slices)), kThreads, smem, st>>>(
@@ -670,9 +676,9 @@ cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, flo
   a.out = dY;
   RECE_TRY(cudaFuncSetAttribute(k_bwd_dy_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(smem)));
-  CUtensorMap tm;
-  RECE_TRY(make_tmap_bf16_ld(&tm, ws + L.xst, uint64_t(c.n_r) * c.d, uint64_t(c.N), p.ld_n,
-                             uint32_t(ns < 256 ? ns : 256)));
+  CUtensorMap tm;  // the sorted rows of X of every round, read MN-major
+  RECE_TRY(make_tmap_bf16_3d(&tm, ws + L.xs, uint64_t(c.d), uint64_t(c.N), uint64_t(c.n_r),
+                             uint32_t(kBK)));
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
     a.write = r == 0;

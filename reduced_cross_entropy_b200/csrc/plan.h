@@ -70,9 +70,10 @@ struct Layout {
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_key_b = 0,
          e_sorted_g = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0;
   size_t bwd_end = 0;
-  // tensor-core dX: kept from rece_loss_fwd to rece_loss_bwd (not aliased): the d-major
-  // sorted copy of Y, the kept entries by (round, sorted row) with their slice starts, and
-  // each row's positive logit
+  // tensor-core dX (and dY): kept from rece_loss_fwd to rece_loss_bwd (not aliased): the
+  // sorted copies of Y (and X) -- xs, ys above, placed here then -- the kept entries by
+  // (round, sorted row) with their slice starts, and each row's positive logit; the
+  // all-negatives mode keeps d-major copies of Y and X (yst, xst)
   size_t yst = 0, kept = 0, kept_off = 0, pos_logit = 0;
   // all-negatives mode, kept from rece_loss_fwd to rece_loss_bwd: the d-major copy of X,
   // the chunk tables, positives' sorted positions, lse per round in sorted order; forward

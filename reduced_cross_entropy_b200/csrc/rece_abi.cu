@@ -158,9 +158,11 @@ void build_layout(rece_plan_s& p) {
     L.px = take(sizeof(int32_t) * c.n_r * c.N);
     L.py = take(sizeof(int32_t) * c.n_r * c.C);
   }
-  if (p.tc_dy) L.xst = take(sizeof(uint16_t) * size_t(c.n_r) * c.d * p.ld_n);
+  // the sorted copies that the backward's band products read (the B operands) outlive
+  // the forward
+  if (p.tc_dy) L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
   if (p.tc_dx) {
-    L.yst = take(sizeof(uint16_t) * size_t(c.n_r) * c.d * p.ld_c);
+    L.ys = take(sizeof(uint16_t) * size_t(c.n_r) * c.C * c.d);
     L.kept = take(sizeof(int2) * size_t(c.n_r) * c.N * c.k);
     L.kept_off = take(sizeof(int32_t) * size_t(c.n_r) * c.N * (size_t(p.kept_slices) + 1));
     L.pos_logit = take(sizeof(float) * size_t(c.N));
@@ -179,8 +181,8 @@ void build_layout(rece_plan_s& p) {
                                          sort_hist_bytes(c.C, p.bucket_bits)));
   if (p.use_tc) {
     const size_t Q = size_t(tc_list_capacity(c.k));
-    L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
-    L.ys = take(sizeof(uint16_t) * size_t(c.n_r) * c.C * c.d);
+    if (!p.tc_dy) L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
+    if (!p.tc_dx) L.ys = take(sizeof(uint16_t) * size_t(c.n_r) * c.C * c.d);
     L.inv_x = take(sizeof(int32_t) * c.n_r * c.N);
     L.chunk_y = take(sizeof(int32_t) * c.n_r * c.C);
     L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
@@ -591,12 +593,6 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
                                   c.n_r, c.n_c, ws + L.ys, nullptr,
                                   reinterpret_cast<int32_t*>(ws + L.chunk_y), st),
               "permute Y");
-    if (plan->tc_dx)
-      RECE_CUDA(launch_transpose_sorted(ws + L.ys, c.C, c.d, c.n_r, plan->ld_c, ws + L.yst, st),
-                "d-major copy of Y");
-    if (plan->tc_dy)
-      RECE_CUDA(launch_transpose_sorted(ws + L.xs, c.N, c.d, c.n_r, plan->ld_n, ws + L.xst, st),
-                "d-major copy of X");
   }
   stage_mark(*plan, RECE_STAGE_SORT, 1, st);
   return RECE_OK;

@@ -87,6 +87,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+// 3D tile load (no multicast): box at element coordinates (x, y, z) of `map`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 // 1-D bulk copy (no multicast) of `bytes` (a multiple of 16; both addresses 16-byte
 // aligned) from global memory into shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
@@ -218,6 +227,18 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
          | (uint64_t(2) << 61);             // 128-byte swizzle
 }
 
+// Shared-memory descriptor of an MN-major bf16 operand written by TMA boxes {64, rows}
+// with the 128-byte swizzle: each box holds 64 consecutive elements of M or N (128 B) for
+// each K index, K rows 128 B apart in 8-row atoms of 1024 B (the stride byte offset); the
+// next 64 elements of M or N lie `lbo` bytes further (the leading byte offset).
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4)      // start address, 16-byte units
+         | (uint64_t((lbo >> 4) & 0x3FFFu) << 16)  // leading byte offset: next 64 of M/N
+         | (uint64_t(1024 >> 4) << 32)          // stride byte offset: next 8 K rows
+         | (uint64_t(1) << 46)                  // descriptor version of sm_100
+         | (uint64_t(2) << 61);                 // 128-byte swizzle
+}
+
 // Instruction descriptor: bf16 A and B (K-major), fp32 accumulator, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                             // D format fp32
@@ -225,6 +246,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                          // B format bf16
          | (uint32_t(N >> 3) << 17)            // N / 8
          | (uint32_t(M >> 4) << 24);           // M / 16
+}
+// The same with B MN-major (its N elements contiguous in the tile).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
 }  // namespace sm100

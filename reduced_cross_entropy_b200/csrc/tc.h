@@ -17,6 +17,10 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
 // 16 bytes) and whose column count is arbitrary: boxes past the last column read zeros.
 cudaError_t make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                               uint64_t ld, uint32_t box_rows);
+// rows x cols bf16 matrices, `planes` of them one after another (cols a multiple of 64);
+// box {64, box_rows, 1}, 128-byte swizzle; rows past the end read as zeros.
+cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
+                              uint64_t rows, uint64_t planes, uint32_t box_rows);
 int sm_count();
 
 // bf16 mode without RECE_FLAG_FMA_SCORES and d a multiple of 64: the tcgen05 kernels run.
