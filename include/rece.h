@@ -20,7 +20,8 @@
  *
  * Conventions shared by every call
  *   - Pointers marked "device" point to GPU memory the caller owns; the library never
- *     allocates device memory.  Matrices are row-major and contiguous.
+ *     allocates device memory.  Matrices are row-major and contiguous, and X, Y, B, dX
+ *     and dY start on a 16-byte boundary (RECE_ERR_INVALID_ARG otherwise).
  *   - Element type of X, Y, B: fp32 in RECE_MODE_FP32_EXACT, bf16 in RECE_MODE_BF16.
  *     Losses, log-sum-exps and gradients are always fp32.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <new>
 
 #include "common.cuh"
@@ -203,6 +204,15 @@ void build_layout(rece_plan_s& p) {
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
+
+// The kernels read X, Y, B with 16-byte vector loads and write dX, dY with 16-byte stores
+// and bulk copies: every matrix must start on a 16-byte boundary (NULL ones are skipped).
+bool aligned16(std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if (q && (reinterpret_cast<uintptr_t>(q) & 15u) != 0) return false;
+  return true;
+}
+constexpr const char* kMisaligned = "X, Y, B, dX and dY must be 16-byte aligned";
 
 rece_status_t check_plan_ws(rece_plan_t plan, const void* ws, size_t ws_bytes) {
   if (!plan) return fail(RECE_ERR_INVALID_ARG, "plan is NULL");
@@ -525,6 +535,7 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   if (s != RECE_OK) return s;
   const auto& c = plan->cfg;
   if (!B || !Y || (c.N > 0 && !X)) return fail(RECE_ERR_INVALID_ARG, "NULL input");
+  if (!aligned16({B, X, Y})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const Layout& L = plan->lay;
@@ -607,6 +618,7 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
   const auto& c = plan->cfg;
   if (!loss || !Y || (c.N > 0 && (!X || !targets || (!selected && !plan->all_neg) || !lse)))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  if (!aligned16({X, Y})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const Layout& L = plan->lay;
@@ -681,6 +693,7 @@ rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void* Y,
   if (!Y || !dY ||
       (c.N > 0 && (!X || !targets || (!selected && !plan->all_neg) || !lse || !dloss || !dX)))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  if (!aligned16({X, Y, dX, dY})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan->lay.status);
@@ -715,6 +728,7 @@ rece_status_t rece_full_ce_fwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
   if (!workspace || workspace_bytes < need) return fail(RECE_ERR_WORKSPACE, "workspace too small");
   if (!loss || !Y || (N > 0 && (!X || !targets || !lse)))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  if (!aligned16({X, Y})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
@@ -743,6 +757,7 @@ rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
   if (!workspace || workspace_bytes < need) return fail(RECE_ERR_WORKSPACE, "workspace too small");
   if (!Y || !dY || (N > 0 && (!X || !targets || !lse || !dloss || !dX)))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  if (!aligned16({X, Y, dX, dY})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mode == RECE_MODE_FP32_EXACT)
     RECE_CUDA(launch_full_ce_bwd(N, C, d, static_cast<const float*>(X),
@@ -803,6 +818,7 @@ rece_status_t rece_sampled_fwd(int32_t kind, int64_t N, int64_t C, int32_t d, in
   if (!loss || !Y || (N > 0 && (!X || !targets || (n > 0 && !negatives) ||
                                 (kind == RECE_SAMPLED_CE_MINUS && !lse))))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  if (!aligned16({X, Y})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.lay.status);
@@ -837,6 +853,7 @@ rece_status_t rece_sampled_bwd(int32_t kind, int64_t N, int64_t C, int32_t d, in
   if (!Y || !dY || (N > 0 && (!X || !targets || (n > 0 && !negatives) || !dloss || !dX ||
                               (kind == RECE_SAMPLED_CE_MINUS && !lse))))
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
+  if (!aligned16({X, Y, dX, dY})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + p.lay.status);

@@ -122,6 +122,21 @@ def test_calls_reject_small_workspace_without_gpu():
     assert s == 3
 
 
+def test_calls_reject_misaligned_matrices_without_gpu():
+    # the kernels use 16-byte vector loads, stores and bulk copies on X, Y, B, dX, dY
+    p = Plan(N=256, C=4096, d=64, n_b=16, n_c=8, n_r=1, k=32, mode="fp32")
+    L = _lib.lib()
+    ws = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected on the host first
+    ok, bad = ctypes.c_void_p(1 << 16), ctypes.c_void_p((1 << 16) + 8)
+    n = p.workspace_bytes
+    assert L.rece_bucketize_sort(p._h, ok, bad, ok, ws, n, None) == 1
+    assert L.rece_bucketize_sort(p._h, bad, ok, ok, ws, n, None) == 1
+    assert b"16-byte aligned" in L.rece_last_error_string()
+    args = [ok] * 7  # X, Y, targets, selected, lse, logits, dloss
+    assert L.rece_loss_bwd(p._h, *args, ws, n, ok, bad, None) == 1
+    assert L.rece_loss_bwd(p._h, bad, *args[1:], ws, n, ok, ok, None) == 1
+
+
 def test_plan_paths_follow_the_shape():
     """rece_plan_paths: which kernels a plan runs (decided on the host, no GPU needed)."""
     TC, DX, SC = _lib.PATH_TENSOR_CORES, _lib.PATH_DX_TENSORS, _lib.PATH_STORED_SCORES
