@@ -72,13 +72,12 @@ struct Layout {
   size_t bwd_end = 0;
   // tensor-core dX (and dY): kept from rece_loss_fwd to rece_loss_bwd (not aliased): the
   // sorted copies of Y (and X) -- xs, ys above, placed here then -- the kept entries by
-  // (round, sorted row) with their slice starts, and each row's positive logit; the
-  // all-negatives mode keeps d-major copies of Y and X (yst, xst)
-  size_t yst = 0, kept = 0, kept_off = 0, pos_logit = 0;
-  // all-negatives mode, kept from rece_loss_fwd to rece_loss_bwd: the d-major copy of X,
-  // the chunk tables, positives' sorted positions, lse per round in sorted order; forward
-  // only: the rounds' (max, sum) pairs and the inverse orders of Y
-  size_t xst = 0, itemc = 0, rowc = 0, pz = 0, lse_sorted = 0, ms = 0, inv_y = 0,
+  // (round, sorted row) with their slice starts, and each row's positive logit
+  size_t kept = 0, kept_off = 0, pos_logit = 0;
+  // all-negatives mode, kept from rece_loss_fwd to rece_loss_bwd: the chunk tables, the
+  // positives' sorted positions, lse per round in sorted order; forward only: the rounds'
+  // (max, sum) pairs and the inverse orders of Y
+  size_t itemc = 0, rowc = 0, pz = 0, lse_sorted = 0, ms = 0, inv_y = 0,
          dx_parts = 0;
   // tensor-core dY: the positives' per-segment partial sums [N][d] (backward region)
   size_t pos_parts = 0;
@@ -106,8 +105,6 @@ struct rece_plan_s {
   bool tc_scores;       // ... with the window scores computed once and stored (large d)
   int64_t score_width;  // columns of the stored scores per row (longest union, padded)
   int32_t kept_slices;  // most 64-position slices one window touches
-  int64_t ld_c;         // row pitch (elements) of the d-major copy of Y: C rounded up to 8
-  int64_t ld_n;         // ... and of X (all-negatives mode): N rounded up to 8
   bool all_neg;         // RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed, no top-k
   rece_plan_s* pos_plan;  // all-negatives mode and tensor-core dY: the positives' pair
                           // backward (k = 0)

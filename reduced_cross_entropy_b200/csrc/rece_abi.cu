@@ -94,7 +94,7 @@ void set_pair_sort(rece_plan_s& p) {
 }
 
 // All-negatives mode: what the backward reads stays from rece_bucketize_sort on (sorted
-// copies, their d-major copies, orders, chunk tables, positives' sorted positions, lse by
+// copies, orders, chunk tables, positives' sorted positions, lse by
 // round); the forward's scratch and the positives' pair arrays share the rest.
 void build_layout_all_neg(rece_plan_s& p) {
   const auto& c = p.cfg;
@@ -112,8 +112,6 @@ void build_layout_all_neg(rece_plan_s& p) {
   L.py = take(sizeof(int32_t) * nr * c.C);
   L.xs = take(sizeof(uint16_t) * nr * c.N * c.d);
   L.ys = take(sizeof(uint16_t) * nr * c.C * c.d);
-  L.xst = take(sizeof(uint16_t) * nr * c.d * p.ld_n);
-  L.yst = take(sizeof(uint16_t) * nr * c.d * p.ld_c);
   L.itemc = take(sizeof(int32_t) * nr * nr * c.C);
   L.rowc = take(sizeof(int32_t) * nr * nr * c.N);
   L.pz = take(sizeof(int32_t) * nr * c.N);
@@ -316,7 +314,7 @@ rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
                             static_cast<const __nv_bfloat16*>(Y), targets, nullptr, lse, nullptr,
                             dloss, ws, dX, dY, status, st),
             "positives' backward");
-  RECE_CUDA(launch_window_grad_tc(p, false, ws + L.xs, ws + L.ys, ws + L.xst, ws + L.yst,
+  RECE_CUDA(launch_window_grad_tc(p, false, ws + L.xs, ws + L.ys,
                                   I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.px), dloss, dX,
                                   reinterpret_cast<float*>(ws + L.dx_parts), status, st),
             "window dX (tcgen05)");
@@ -324,7 +322,7 @@ rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
   stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
-  RECE_CUDA(launch_window_grad_tc(p, true, ws + L.xs, ws + L.ys, ws + L.xst, ws + L.yst,
+  RECE_CUDA(launch_window_grad_tc(p, true, ws + L.xs, ws + L.ys,
                                   I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.py), dloss, dY,
                                   nullptr, status, st),
             "window dY (tcgen05)");
@@ -409,8 +407,6 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     const int64_t sl = w1 > w0 ? ((w1 - 1) >> 6) - (w0 >> 6) + 1 : 0;
     if (sl > p->kept_slices) p->kept_slices = int32_t(sl);
   }
-  p->ld_c = (c.C + 7) / 8 * 8;
-  p->ld_n = (c.N + 7) / 8 * 8;
   p->all_neg = (c.flags & RECE_FLAG_ALL_NEGATIVES) != 0;
   p->pos_plan = nullptr;
   // the tensor-core path groups each row's kept entries by slice of its window
@@ -591,10 +587,6 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
                                   c.n_r, c.n_c, ws + L.ys,
                                   reinterpret_cast<int32_t*>(ws + L.inv_y), nullptr, st),
               "permute Y");
-    RECE_CUDA(launch_transpose_sorted(ws + L.xs, c.N, c.d, c.n_r, plan->ld_n, ws + L.xst, st),
-              "d-major copy of X");
-    RECE_CUDA(launch_transpose_sorted(ws + L.ys, c.C, c.d, c.n_r, plan->ld_c, ws + L.yst, st),
-              "d-major copy of Y");
   } else if (plan->use_tc) {
     RECE_CUDA(launch_permute_rows(X, c.N, c.d, reinterpret_cast<const int32_t*>(ws + L.px),
                                   c.n_r, c.n_c, ws + L.xs,

@@ -13,10 +13,6 @@ namespace rece {
 // 64 columns x box_rows rows, 128-byte swizzle (the K-major layout the MMA reads).
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                            uint32_t box_rows);
-// The same for a matrix whose rows are ld >= cols elements apart (ld * 2 a multiple of
-// 16 bytes) and whose column count is arbitrary: boxes past the last column read zeros.
-cudaError_t make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                              uint64_t ld, uint32_t box_rows);
 // rows x cols bf16 matrices, `planes` of them one after another (cols a multiple of 64);
 // box {64, box_rows, 1}, 128-byte swizzle; rows past the end read as zeros.
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
@@ -35,10 +31,6 @@ cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void*
 cudaError_t launch_permute_rows(const void* V, int64_t M, int d, const int32_t* perm, int n_r,
                                 int n_c, void* Vs, int32_t* inv, int32_t* chunk,
                                 cudaStream_t st);
-
-// VsT[r][t][p] = Vs[r][p][t]: d-major copies (rows ld elements apart, ld % 8 == 0).
-cudaError_t launch_transpose_sorted(const void* Vs, int64_t M, int d, int n_r, int64_t ld,
-                                    void* VsT, cudaStream_t st);
 
 // K3 on tensor cores: per (round, sorted row) the candidate list (score bits, sorted
 // catalogue position), its count and threshold.
@@ -75,8 +67,9 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
                             float* row_loss, float* logits, uint32_t* status, int32_t* spill_rows,
                             void* spill_scratch, cudaStream_t st);
 
-// dX of step 6 on tensor cores (see bwd_tc.cu): written, not accumulated.  Needs the
-// grouped merge outputs (kept, kept_off, pos_logit) and the d-major copy YsT.
+// dX of step 6 on tensor cores (see bwd_tc.cu): the positives' terms written, the
+// rounds' added.  Needs the grouped merge outputs (kept, kept_off, pos_logit) and the
+// sorted copy Ys.
 template <typename T>
 cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* targets,
                          const float* lse, const float* dloss, char* ws, float* dX,
@@ -84,7 +77,7 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
 
 // dY of step 6 on tensor cores: the rounds' window terms, written by round 0 and added by
 // the others (the positives' terms are added after).  Needs the grouped kept entries and
-// the d-major copy XsT.
+// the sorted copy Xs.
 cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, float* dY,
                          uint32_t* status, cudaStream_t st);
 
@@ -110,8 +103,7 @@ cudaError_t launch_window_combine(const rece_plan_s& p, const T* X, const T* Y,
 // into `out` round by round (dX with `scratch` [n_r][N][d]: all rounds in one grid, then
 // added in round order).
 cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
-                                  const void* Ys, const void* XsT, const void* YsT,
-                                  const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
+                                  const void* Ys, const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
                                   const float* lse_sorted, const int32_t* perm,
                                   const float* dloss, float* out, float* scratch,
                                   uint32_t* status, cudaStream_t st);

@@ -44,24 +44,6 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t make_tmap_bf16_ld(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                              uint64_t ld, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return cudaErrorNotSupported;
-  if (rows == 0 || cols == 0 || ld < cols || (ld * 2) % 16 != 0 || box_rows == 0 ||
-      box_rows > 256 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0)
-    return cudaErrorInvalidValue;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                  strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
                               uint64_t rows, uint64_t planes, uint32_t box_rows) {
   auto fn = encode_fn();

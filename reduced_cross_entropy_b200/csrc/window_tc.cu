@@ -11,10 +11,10 @@
 //   LSE  M = rows, K = items.  Each row's thread keeps an online (max, sum) of
 //        exp(s) / cnt over its window columns; out: the round's (max, sum) per row.
 //   DX   M = rows, K = items.  P = exp(s - lse_row) / cnt on the row's window columns,
-//        O += P V with V = the K tile of the d-major sorted catalogue copy; at the end
+//        O += P V with V = the K tile of the sorted catalogue copy (read MN-major); at the end
 //        dX[row] += O * dloss / N.
 //   DY   M = items, K = rows.  The same with the roles swapped (the pair is live when the
-//        item lies in the row's window), V = the d-major sorted copy of X; dY[item] +=.
+//        item lies in the row's window), V = the sorted copy of X; dY[item] +=.
 // The round count of a pair (row p, item q) is 1 plus the number of other rounds s in
 // which the item's chunk is within n_ec of the row's chunk: both come from per-round
 // tables of every row's and item's chunk in every round.
@@ -119,8 +119,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // The K range of an M tile: the union of the windows of its 128 positions, as a start
-// rounded down to 64 (TMA column coordinates of the d-major copies stay 16-byte aligned)
-// and a count of 128-wide tiles.
+// rounded down to 64 and a count of 128-wide tiles.
 template <int kRole>
 __device__ __forceinline__ void k_range(const Args& a, int64_t m0, int64_t& k0a, int& nK) {
   const int64_t Mside = kRole == kRoleDy ? a.C : a.N;
@@ -220,8 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
           uint8_t* sv = vbuf + size_t(vs) * vb;
           const int32_t kx = int32_t(k0a + int64_t(kt) * kBN);
           mbar_arrive_expect_tx(&ctl.v_full[vs], vb);
-          tma_load_2d(sv, &tmV, &ctl.v_full[vs], kx, r * d);
-          tma_load_2d(sv + vb / 2, &tmV, &ctl.v_full[vs], kx + kBK, r * d);
+          // two K atoms of 64 positions, each d/64 boxes of 64 columns (8 KB apart)
+          for (int at = 0; at < 2; ++at)
+            for (int h = 0; h < d; h += 64)
+              tma_load_3d(sv + at * (vb / 2) + size_t(h) * 128, &tmV, &ctl.v_full[vs], h,
+                          kx + at * kBK, r);
           ++nv_issued;
         }
       }
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN);
-      const uint32_t idesc_o = idesc_bf16_f32(kBM, d);
+      const uint32_t idesc_o = idesc_bf16_f32_bmn(kBM, d);  // V MN-major
       uint32_t it = 0;
       bool ok = true;
       auto mma_pv = [&](int j) {  // O += P_j V_j (hi and lo halves)
@@ -252,11 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
         for (int at = 0; at < 2; ++at) {
           const uint64_t dh = desc_k_sw128(smem_u32(phi + at * kSlab));
           const uint64_t dl = desc_k_sw128(smem_u32(plo + at * kSlab));
-          const uint64_t dv = desc_k_sw128(smem_u32(sv + at * (vb / 2)));
+          const uint64_t dv = desc_mn_sw128(smem_u32(sv + at * (vb / 2)), 8192u);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            mma_bf16(tmem + 256, dh + 2 * kk, dv + 2 * kk, idesc_o, (j | at | kk) != 0);
-            mma_bf16(tmem + 256, dl + 2 * kk, dv + 2 * kk, idesc_o, 1);
+          for (int kk = 0; kk < kBK / 16; ++kk) {  // 16 K rows of 128 B per MMA
+            mma_bf16(tmem + 256, dh + 2 * kk, dv + 128u * kk, idesc_o, (j | at | kk) != 0);
+            mma_bf16(tmem + 256, dl + 2 * kk, dv + 128u * kk, idesc_o, 1);
           }
         }
         mma_commit(&ctl.p_empty);
@@ -648,8 +650,7 @@ cudaError_t launch_window_lse_tc(const rece_plan_s& p, const void* Xs, const voi
 }
 
 cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
-                                  const void* Ys, const void* XsT, const void* YsT,
-                                  const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
+                                  const void* Ys, const int32_t* itemc, const int32_t* rowc, const int32_t* pz,
                                   const float* lse_sorted, const int32_t* perm,
                                   const float* dloss, float* out, float* scratch,
                                   uint32_t* status, cudaStream_t st) {
@@ -660,10 +661,11 @@ cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tY, Ys, uint64_t(c.n_r) * c.C, c.d, kBM);
   if (e != cudaSuccess) return e;
+  // V: the sorted rows of X (dY) or Y (dX) of every round, read MN-major
   if (dy)
-    e = make_tmap_bf16_ld(&tV, XsT, uint64_t(c.n_r) * c.d, c.N, p.ld_n, uint32_t(c.d));
+    e = make_tmap_bf16_3d(&tV, Xs, uint64_t(c.d), uint64_t(c.N), uint64_t(c.n_r), kBK);
   else
-    e = make_tmap_bf16_ld(&tV, YsT, uint64_t(c.n_r) * c.d, c.C, p.ld_c, uint32_t(c.d));
+    e = make_tmap_bf16_3d(&tV, Ys, uint64_t(c.d), uint64_t(c.C), uint64_t(c.n_r), kBK);
   if (e != cudaSuccess) return e;
   Args a = base_args(p, itemc, rowc, pz, status);
   a.lse_sorted = lse_sorted;
