@@ -544,8 +544,10 @@ def main():
                        "scores": ("tcgen05" + (", stored" if paths & _lib.PATH_STORED_SCORES
                                                  else ", recomputed per pass")
                                   if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),
-                       "dX": "tcgen05 band products" if paths & _lib.PATH_DX_TENSORS
-                       else "gathered rows",
+                       "dX": ("tcgen05 band products" +
+                              (", rounds in one launch, parts summed in order"
+                               if paths & _lib.PATH_DX_PARTS else "")
+                              if paths & _lib.PATH_DX_TENSORS else "gathered rows"),
                        "negatives": ("every window item (Algorithm 1 as printed), window "
                                      "sums and gradients on tcgen05"
                                      if paths & _lib.PATH_ALL_NEGATIVES

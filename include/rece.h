@@ -142,13 +142,18 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
  *                           row (d >= 1024; else recomputed in the fused selection);
  *   RECE_PATH_ALL_NEGATIVES the all-negatives mode (RECE_FLAG_ALL_NEGATIVES);
  *   RECE_PATH_DY_TENSORS    dY as tcgen05 band products as well (with RECE_PATH_DX_TENSORS;
- *                           else a stable pair sort and gathered rows).
+ *                           else a stable pair sort and gathered rows);
+ *   RECE_PATH_DX_PARTS      (with RECE_PATH_DX_TENSORS) the dX band products of all rounds
+ *                           in one launch, each row tile's window split in parts that are
+ *                           stored and then summed in a fixed order (when per-round
+ *                           launches would leave their last wave part-empty).
  * RECE_ERR_INVALID_ARG for a NULL argument. */
 #define RECE_PATH_TENSOR_CORES 0x1u
 #define RECE_PATH_DX_TENSORS 0x2u
 #define RECE_PATH_STORED_SCORES 0x4u
 #define RECE_PATH_ALL_NEGATIVES 0x8u  /* RECE_FLAG_ALL_NEGATIVES: window sums on tcgen05 */
 #define RECE_PATH_DY_TENSORS 0x10u
+#define RECE_PATH_DX_PARTS 0x20u
 RECE_API rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths);
 
 /* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].

@@ -12,6 +12,8 @@ upcast) and follows the definitions cited in ``rece_oracle.c``:
 * ``select``        -- candidates of the chunk windows over all rounds, positive removed,
                        de-duplicated, the k best by (score desc, item asc) (SCE abstract)
 * ``rece_loss`` / ``rece_grad``       -- Algorithm 1's loss, equation (4) on the subset
+* ``rece_grad_rows`` / ``rece_grad_items`` -- rece_grad's dX rows / dY rows for a sample of
+                       row or item ids only (the same sums, restricted; numpy fp64)
 * ``full_ce_loss`` / ``full_ce_grad`` -- equations (3) and (4) over the whole catalogue
 * ``window_loss`` / ``window_grad`` -- Algorithm 1 as printed: every window item a
                        negative, duplicates across rounds corrected by ln(count)
@@ -166,6 +168,52 @@ def rece_grad(X, Y, target, selected, lse, dloss=1.0):
     _load().oracle_rece_grad(X, Y, target, N, C, d, k, selected,
                              np.ascontiguousarray(lse, np.float64), float(dloss), dX, dY)
     return dX, dY
+
+
+def rece_grad_rows(X, Y, target, rows, selected, lse, dloss=1.0):
+    """dX rows of ``rece_grad`` for the row ids ``rows`` only: for each sampled row i,
+    dX_i = sum over j in (z_i, then the selected entries as listed) of g_ij y_j with
+    g_ij = (exp(l_ij - lse_i) - [entry is the positive]) * dloss / N, N = len(X) (RECE
+    paper, equation (4) on the subset, the selection held constant).  ``selected`` [R, k]
+    (-1 padded) and ``lse`` [R] follow ``rows``.  fp64 [R, d]."""
+    X, Y = np.asarray(X, np.float32), np.asarray(Y, np.float32)
+    N, d = X.shape
+    scale = dloss / N if N else 0.0
+    out = np.zeros((len(rows), d), np.float64)
+    for a, i in enumerate(np.asarray(rows, np.int64)):
+        js = [int(target[i])] + [int(j) for j in selected[a] if j >= 0]
+        Yj = Y[js].astype(np.float64)
+        g = np.exp(Yj @ X[i].astype(np.float64) - lse[a])
+        g[0] -= 1.0  # the positive
+        out[a] = (g * scale) @ Yj
+    return out
+
+
+def rece_grad_items(X, Y, target, rows, selected, lse, items, dloss=1.0):
+    """dY rows of ``rece_grad`` for the item ids ``items`` only: dY_j = sum over rows i
+    and entries (z_i, then the selected ones as listed) equal to j of g_ij x_i, g_ij as in
+    ``rece_grad_rows``.  ``rows`` must hold every row whose positive or selection holds one
+    of the items (other rows add nothing); ``selected`` [R, k] and ``lse`` [R] follow it.
+    fp64 [len(items), d]."""
+    X, Y = np.asarray(X, np.float32), np.asarray(Y, np.float32)
+    N, d = X.shape
+    scale = dloss / N if N else 0.0
+    rows = np.asarray(rows, np.int64)
+    sel = np.asarray(selected, np.int64).reshape(len(rows), -1)
+    z = np.asarray(target, np.int64)[rows]
+    out = np.zeros((len(items), d), np.float64)
+    for b, j in enumerate(items):
+        y = Y[j].astype(np.float64)
+        n_sel = (sel == j).sum(axis=1)     # entries of the selection equal to j
+        is_pos = (z == j).astype(np.int64)  # and the positive
+        idx = np.nonzero(n_sel + is_pos)[0]
+        if len(idx) == 0:
+            continue
+        Xi = X[rows[idx]].astype(np.float64)
+        p = np.exp(Xi @ y - np.asarray(lse, np.float64)[idx])
+        g = (p * (n_sel[idx] + is_pos[idx]) - is_pos[idx]) * scale
+        out[b] = g @ Xi
+    return out
 
 
 def full_ce_loss(X, Y, target):

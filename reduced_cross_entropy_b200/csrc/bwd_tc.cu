@@ -32,6 +32,8 @@
 //
 // Determinism: each dX row is written by one CTA per launch, in a fixed K order; the
 // positive term is written first (dX_i = g_iz y_z), then the rounds add in round order.
+#include <cmath>
+
 #include "common.cuh"
 #include "plan.h"
 #include "sm100.cuh"
@@ -119,10 +121,11 @@ __device__ __forceinline__ void row_window(int64_t p, int64_t N, int64_t C, int 
 // hit distinct banks) and hands each piece to the bulk-copy engine: full lines reach
 // memory, and an add is done at L2 (the old values never come back to the SM).  One add
 // per element per launch: deterministic.  `fin` must be uniform across the warp (the TMEM
-// loads are warp-collective); rows with `live` false load but write nothing.
+// loads are warp-collective); rows with `live` false load but write nothing; `zero`
+// (uniform across the CTA) writes zeros without reading TMEM.
 __device__ __forceinline__ void epilogue_rows(uint8_t* stage, size_t avail, int t,
                                               uint32_t taddr, int ns, float scale, bool live,
-                                              float* o, bool write) {
+                                              float* o, bool write, bool zero = false) {
   const int W = (ns % 128 == 0 && avail >= 2u * kBM * (128 * 4 + 16)) ? 128 : 64;
   const int stride = W * 4 + 16;
   for (int c0 = 0, piece = 0; c0 < ns; c0 += W, ++piece) {
@@ -131,7 +134,12 @@ __device__ __forceinline__ void epilogue_rows(uint8_t* stage, size_t avail, int 
     bulk_wait_read<1>();  // this thread's copy out of that buffer (two pieces ago)
     for (int cc = 0; cc < W; cc += 32) {
       float v[32];
-      tmem_load32(taddr + uint32_t(c0 + cc), v);
+      if (zero) {  // no K slab: nothing was accumulated (CTA-uniform)
+#pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] = 0.0f;
+      } else {
+        tmem_load32(taddr + uint32_t(c0 + cc), v);
+      }
       float4* s4 = reinterpret_cast<float4*>(srow + cc);
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -147,7 +155,7 @@ __device__ __forceinline__ void epilogue_rows(uint8_t* stage, size_t avail, int 
       bulk_commit();
     }
   }
-  bulk_wait_all();
+  bulk_wait_read<0>();  // the shared memory may go; the writes finish on their own
 }
 
 struct Args {
@@ -160,6 +168,10 @@ struct Args {
   float* out;               // dX [N][d], accumulated into
   uint32_t* status;
   int write;                // dY: store (round 0, which covers every position), else add
+  // dX with parts: one grid over (round, K split): blockIdx.z = round * ksplit + split;
+  // each CTA stores its part to parts[z][row][:] (rows by id), added in z order after
+  float* parts;
+  int ksplit;
 };
 
 __device__ __forceinline__ void on_timeout(Ctl& c, uint32_t* status) {
@@ -181,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
   const int nb = a.nb;
   const int64_t N = a.N, C = a.C;
-  const int r = a.r, n0 = blockIdx.y * a.ns;
+  const int r = a.parts ? int(blockIdx.z) / a.ksplit : a.r, n0 = blockIdx.y * a.ns;
 
   // the item's rows and its K range [lo, hi) in slabs of 64
   const int64_t m0 = int64_t(blockIdx.x) * kBM;
@@ -194,6 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
     if (k1 > k0) {
       lo = k0 >> 6;
       hi = (k1 + 63) >> 6;
+    }
+    if (a.parts && a.ksplit > 1) {  // this CTA's share of the slabs
+      const int64_t n = hi - lo, sp = int64_t(blockIdx.z) % a.ksplit;
+      hi = lo + n * (sp + 1) / a.ksplit;
+      lo = lo + n * sp / a.ksplit;
     }
   }
   const int nK = int(hi - lo);
@@ -292,12 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
       int64_t w0, w1;
       row_window(p, N, C, a.n_c, a.n_ec, w0, w1);
       const int S = w1 > w0 ? int((w1 - 1) >> 6) - int(w0 >> 6) + 1 : 0;
-      count = __ldg(a.kept_off + (rN + p) * a.Sp + S);
+      const int32_t* offs = a.kept_off + (rN + p) * a.Sp;
+      count = __ldg(offs + S);
+      // the first entry at or past slab lo (a K split may start inside the window)
+      const int64_t idx = lo - (w0 >> 6);
+      e = idx <= 0 ? 0 : (idx >= S ? count : __ldg(offs + idx));
+      base = e;
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      cur[u] = u < count ? __ldg(erow + u) : kNone;
-      nxt[u] = 8 + u < count ? __ldg(erow + 8 + u) : kNone;
+      cur[u] = e + u < count ? __ldg(erow + e + u) : kNone;
+      nxt[u] = e + 8 + u < count ? __ldg(erow + e + 8 + u) : kNone;
     }
 
     for (int s = 0; s < nK; ++s) {
@@ -341,17 +363,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
     __syncwarp();
 
     // ------------------------------------------------------------ epilogue
-    bool ok = mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && nK > 0;
+    bool ok = mbar_wait(&ctl.done, 0, &ctl.abort, kTimeoutNs) && (nK > 0 || a.parts);
     ok = __all_sync(0xFFFFFFFFu, ok);
     const float scale = a.dloss[0] / float(N);  // G holds p; g = p * dloss / N
     tc_fence_after();
     const int64_t row = m0 + t;  // this thread's sorted row
     const bool live = row < N;
     const int64_t dst = live ? a.px[rN + row] : 0;
+    // parts: every CTA stores its part (zeros when its split has no slab); else add
+    float* o = a.parts ? a.parts + (int64_t(blockIdx.z) * N + dst) * a.d + n0
+                       : a.out + dst * a.d + n0;
     if (ok)
       epilogue_rows(sbase, size_t(2 * kAStages) * kATile + size_t(nb) * b_bytes, t,
-                    tmem + (uint32_t(warp * 32) << 16), a.ns, scale, live,
-                    a.out + dst * a.d + n0, false);
+                    tmem + (uint32_t(warp * 32) << 16), a.ns, scale, live, o,
+                    a.parts != nullptr, nK == 0);
   }
   tc_fence_before();
   __syncthreads();
@@ -587,6 +612,27 @@ __global__ void __launch_bounds__(256) k_bwd_pos(const T* __restrict__ Y,
 
 }  // namespace
 
+// Band-product geometry for d: CTA slices of ns <= 512 columns (two TMEM accumulators
+// past 256) and a TMA ring as deep as lets two CTAs share an SM (at least two slabs).
+struct BandGeometry {
+  int ns, slices, nb;
+  size_t smem;
+  uint32_t tcols;
+};
+BandGeometry band_geometry(int d) {
+  BandGeometry g;
+  g.ns = d;
+  if (g.ns > 256)
+    g.ns = (d % 512 == 0) ? 512
+                          : (d % 256 == 0 ? 256 : (d % 192 == 0 ? 192 : (d % 128 == 0 ? 128 : 64)));
+  g.slices = d / g.ns;
+  int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(g.ns) * 128));
+  g.nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
+  g.smem = smem_bytes(g.nb, g.ns);
+  g.tcols = g.ns <= 32 ? 32u : (g.ns <= 64 ? 64u : (g.ns <= 128 ? 128u : (g.ns <= 256 ? 256u : 512u)));
+  return g;
+}
+
 template <typename T>
 cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* targets,
                          const float* lse, const float* dloss, char* ws, float* dX,
@@ -594,16 +640,9 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   const auto& c = p.cfg;
   const Layout& L = p.lay;
   if (c.N == 0) return cudaSuccess;
-  // d is split into CTA slices of ns <= 512 columns (two TMEM accumulators past 256)
-  int ns = c.d;
-  if (ns > 256)
-    ns = (c.d % 512 == 0) ? 512
-                          : (c.d % 256 == 0 ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64)));
-  const int slices = c.d / ns;
-  // TMA ring: as deep as lets two CTAs share an SM (at least two slabs)
-  int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(ns) * 128));
-  nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
-  const size_t smem = smem_bytes(nb, ns);
+  const BandGeometry g = band_geometry(c.d);
+  const int ns = g.ns, slices = g.slices, nb = g.nb;
+  const size_t smem = g.smem;
 
   Args a{};
   a.N = c.N;
@@ -632,7 +671,18 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   CUtensorMap tm;  // the sorted rows of Y of every round, read MN-major
   RECE_TRY(make_tmap_bf16_3d(&tm, ws + L.ys, uint64_t(c.d), uint64_t(c.C), uint64_t(c.n_r),
                              uint32_t(kBK)));
-  for (int r = 0; r < c.n_r; ++r) {
+  if (p.dx_split > 0) {
+    // one grid over (round, K split), parts stored, then added into dX in order
+    a.parts = reinterpret_cast<float*>(ws + L.dx_parts);
+    a.ksplit = p.dx_split;
+    const int nz = c.n_r * p.dx_split;
+    k_bwd_dx_tc<<<dim3(unsigned(ceil_div(c.N, kBM)), unsigned(slices), unsigned(nz)), kThreads,
+                  smem, st>>>(tm, a);
+    count_launches(1);
+    RECE_TRY(cudaGetLastError());
+    return launch_add_parts(a.parts, c.N * int64_t(c.d), nz, dX, st);
+  }
+  for (int r = 0; r < c.n_r; ++r) {  // rounds in order, each adding into dX
     a.r = r;
     k_bwd_dx_tc<<<dim3(unsigned(ceil_div(c.N, kBM)), unsigned(slices)), kThreads, smem, st>>>(
         tm, a);
@@ -642,6 +692,35 @@ cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* target
   return cudaSuccess;
 }
 
+// How the dX band products cover the rounds.  Per-round launches (0) leave the last wave
+// of each launch part-empty when a round has few work items; one launch over (round, K
+// split) with S splits of every work item's window (S >= 1) fills the waves at the price
+// of n_r S parts of dX written and summed in order.  Chosen from the wave counts, in units
+// of one whole-window work item; a split keeps at least 8 slabs of the narrowest window.
+int dx_tc_split(const rece_plan_s& p) {
+  const auto& c = p.cfg;
+  if (c.N == 0 || c.n_c < 1) return 0;
+  const BandGeometry g = band_geometry(c.d);
+  int per_sm = int((228 * 1024) / (g.smem + 1024));
+  if (per_sm > int(512 / g.tcols)) per_sm = int(512 / g.tcols);
+  if (per_sm < 1) per_sm = 1;
+  const double slots = double(sm_count()) * per_sm;
+  const double items = double(ceil_div(c.N, kBM)) * g.slices;  // per round
+  double best = c.n_r * std::ceil(items / slots);
+  int pick = 0;
+  const int64_t edge_chunks = c.n_ec + 1 < c.n_c ? c.n_ec + 1 : c.n_c;
+  const int64_t min_slabs = (c.C * edge_chunks / c.n_c) / kBK;
+  for (int S = 1; S <= 4; ++S) {
+    if (S > 1 && min_slabs / S < 8) break;
+    const double cost = std::ceil(c.n_r * items * S / slots) / S;
+    if (cost < 0.9 * best) {
+      best = cost;
+      pick = S;
+    }
+  }
+  return pick;
+}
+
 // The window terms of dY: round 0 stores them (its tiles cover every catalogue position),
 // the later rounds add.
 cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, float* dY,
@@ -649,15 +728,9 @@ cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, flo
   const auto& c = p.cfg;
   const Layout& L = p.lay;
   if (c.N == 0) return cudaSuccess;
-  // d is split into CTA slices of ns <= 512 columns (two TMEM accumulators past 256)
-  int ns = c.d;
-  if (ns > 256)
-    ns = (c.d % 512 == 0) ? 512
-                          : (c.d % 256 == 0 ? 256 : (c.d % 192 == 0 ? 192 : (c.d % 128 == 0 ? 128 : 64)));
-  const int slices = c.d / ns;
-  int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(ns) * 128));
-  nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
-  const size_t smem = smem_bytes(nb, ns);
+  const BandGeometry g = band_geometry(c.d);
+  const int ns = g.ns, slices = g.slices, nb = g.nb;
+  const size_t smem = g.smem;
   Args a{};
   a.N = c.N;
   a.C = c.C;

@@ -78,7 +78,7 @@ struct Layout {
   // positives' sorted positions, lse per round in sorted order; forward only: the rounds'
   // (max, sum) pairs and the inverse orders of Y
   size_t itemc = 0, rowc = 0, pz = 0, lse_sorted = 0, ms = 0, inv_y = 0,
-         dx_parts = 0;
+         dx_parts = 0;  // (also the tensor-core dX's parts when split, backward region)
   // tensor-core dY: the positives' per-segment partial sums [N][d] (backward region)
   size_t pos_parts = 0;
   size_t total = 0;
@@ -102,6 +102,7 @@ struct rece_plan_s {
   bool use_tc;          // bf16 mode on the tcgen05 kernels
   bool tc_dx;           // ... and dX of the backward on them too
   bool tc_dy;           // ... and dY (band products; positives through pos_plan's pairs)
+  int dx_split;         // tensor-core dX: 0 one launch per round, S > 0 K splits into parts
   bool tc_scores;       // ... with the window scores computed once and stored (large d)
   int64_t score_width;  // columns of the stored scores per row (longest union, padded)
   int32_t kept_slices;  // most 64-position slices one window touches

@@ -199,6 +199,8 @@ void build_layout(rece_plan_s& p) {
   off = region;
   layout_pairs(p, off);
   if (p.tc_dy) L.pos_parts = take(sizeof(float) * size_t(c.N) * c.d);
+  if (p.dx_split > 0)
+    L.dx_parts = take(sizeof(float) * size_t(c.n_r) * p.dx_split * size_t(c.N) * c.d);
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
@@ -304,7 +306,6 @@ rece_status_t all_neg_fwd(const rece_plan_s& p, const void* X, const void* Y,
 rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
                           const int32_t* targets, const float* lse, const float* dloss,
                           char* ws, float* dX, float* dY, cudaStream_t st) {
-  const auto& c = p.cfg;
   const Layout& L = p.lay;
   auto I = [&](size_t o) { return reinterpret_cast<const int32_t*>(ws + o); };
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
@@ -468,6 +469,7 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     p->pos_plan = q;
     p->tc_dy = true;
   }
+  p->dx_split = p->tc_dx ? dx_tc_split(*p) : 0;
   build_layout(*p);
   if (p->tc_dy) {
     p->pos_plan->lay = p->lay;  // the main plan's pair arrays and status words
@@ -521,7 +523,8 @@ rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
            (plan->tc_dx ? RECE_PATH_DX_TENSORS : 0u) |
            (plan->tc_scores ? RECE_PATH_STORED_SCORES : 0u) |
            (plan->all_neg ? RECE_PATH_ALL_NEGATIVES : 0u) |
-           (plan->tc_dy ? RECE_PATH_DY_TENSORS : 0u);
+           (plan->tc_dy ? RECE_PATH_DY_TENSORS : 0u) |
+           (plan->dx_split > 0 ? RECE_PATH_DX_PARTS : 0u);
   return RECE_OK;
 }
 

@@ -18,6 +18,10 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
                               uint64_t rows, uint64_t planes, uint32_t box_rows);
 int sm_count();
+// out[i] += parts[0][i] + parts[1][i] + ... (n floats each, n % 4 == 0), in that order.
+cudaError_t launch_add_parts(const float* parts, int64_t n, int nparts, float* out,
+                             cudaStream_t st);
+
 
 // bf16 mode without RECE_FLAG_FMA_SCORES and d a multiple of 64: the tcgen05 kernels run.
 bool tc_supported(const rece_plan_s& p);
@@ -74,6 +78,10 @@ template <typename T>
 cudaError_t launch_dx_tc(const rece_plan_s& p, const T* Y, const int32_t* targets,
                          const float* lse, const float* dloss, char* ws, float* dX,
                          uint32_t* status, cudaStream_t st);
+
+// 0: dX band products one launch per round, each adding into dX; S >= 1: one launch over
+// (round, K split) into n_r S parts of dX (Layout::dx_parts), summed in order after.
+int dx_tc_split(const rece_plan_s& p);
 
 // dY of step 6 on tensor cores: the rounds' window terms, written by round 0 and added by
 // the others (the positives' terms are added after).  Needs the grouped kept entries and

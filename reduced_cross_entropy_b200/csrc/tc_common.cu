@@ -1,6 +1,6 @@
 // tc_common.cu -- host helpers of the tensor-core kernels: TMA descriptors (tensor maps)
-// for row-major bf16 matrices (2-D, or 3-D: planes of rows, one per round) and the SM
-// count of the current device.
+// for row-major bf16 matrices (2-D, or 3-D: planes of rows, one per round), the SM count
+// of the current device, and the ordered sum of partial results.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -60,6 +60,37 @@ cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+
+__global__ void __launch_bounds__(256) k_add_parts(const float4* __restrict__ parts, int64_t n4,
+                                                   int nparts, float4* __restrict__ out) {
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    float4 x = out[e];
+    for (int z = 0; z < nparts; ++z) {
+      const float4 q = parts[int64_t(z) * n4 + e];
+      x.x += q.x;
+      x.y += q.y;
+      x.z += q.z;
+      x.w += q.w;
+    }
+    out[e] = x;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_add_parts(const float* parts, int64_t n, int nparts, float* out,
+                             cudaStream_t st) {
+  if (n == 0 || nparts == 0) return cudaSuccess;
+  if (n % 4 != 0) return cudaErrorInvalidValue;
+  const int64_t n4 = n / 4, want = (n4 + 255) / 256;
+  k_add_parts<<<unsigned(want < 8 * 148 ? want : 8 * 148), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(parts), n4, nparts, reinterpret_cast<float4*>(out));
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 int sm_count() {

@@ -113,11 +113,6 @@ __device__ __forceinline__ float ex2(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  return uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
-         (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
-}
-
 // The K range of an M tile: the union of the windows of its 128 positions, as a start
 // rounded down to 64 and a count of 128-wide tiles.
 template <int kRole>
@@ -569,24 +564,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_window_tc(
 }
 
 
-// out[i][:] += sum over rounds r of part[r][i][:], rounds in order.
-__global__ void __launch_bounds__(256) k_window_add(const float4* __restrict__ part,
-                                                    int64_t n4, int n_r,
-                                                    float4* __restrict__ out) {
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    float4 x = out[e];
-    for (int r = 0; r < n_r; ++r) {
-      const float4 p = part[int64_t(r) * n4 + e];
-      x.x += p.x;
-      x.y += p.y;
-      x.z += p.z;
-      x.w += p.w;
-    }
-    out[e] = x;
-  }
-}
-
 template <int kRole, int kR>
 cudaError_t run_window_r(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& V,
                          const Args& a, unsigned gx, unsigned gy, cudaStream_t st) {
@@ -678,12 +655,7 @@ cudaError_t launch_window_grad_tc(const rece_plan_s& p, bool dy, const void* Xs,
     a.scratch = scratch;
     e = run_window<kRoleDx>(tX, tY, tV, a, unsigned(ceil_div(c.N, kBM)), unsigned(c.n_r), st);
     if (e != cudaSuccess) return e;
-    const int64_t n4 = c.N * int64_t(c.d) / 4;
-    const int64_t want = (n4 + 255) / 256;
-    k_window_add<<<unsigned(want < 8 * 148 ? want : 8 * 148), 256, 0, st>>>(
-        reinterpret_cast<const float4*>(scratch), n4, c.n_r, reinterpret_cast<float4*>(out));
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_add_parts(scratch, c.N * int64_t(c.d), c.n_r, out, st);
   }
   for (int r = 0; r < c.n_r; ++r) {  // rounds in order: each adds into the same rows
     a.r = r;

@@ -3,7 +3,10 @@
 This module only draws numbers: it holds none of the loss's arithmetic, so both the
 CUDA path and the CPU oracle can be fed from it.  Everything is drawn with numpy's
 PCG64 from an explicit seed, in a fixed order (X, then Y, then the targets), in fp32,
-then rounded to bf16 (round to nearest even) where a workload is bf16.
+then rounded to bf16 (round to nearest even) where a workload is bf16.  A matrix of more
+than 2^24 elements is drawn instead in blocks of 2^22 elements, block b from its own
+PCG64 stream (the b-th child of SeedSequence([seed, 0 for X / 1 for Y])), filled by a
+thread pool: the values depend on the seed only, never on the thread count.
 
 Workloads follow the shapes of the RECE paper's experiments (section 4, Table 1:
 catalogues of 22k to 174k items, SASRec outputs of batch x sequence rows) and extend
@@ -21,6 +24,8 @@ stream keyed by (seed, step), and are passed to both sides as an input.
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Optional
 
 import numpy as np
@@ -62,11 +67,19 @@ WORKLOADS = {
 }
 
 
+def _bf16_rounded_u32(a: np.ndarray) -> np.ndarray:
+    """fp32 bit patterns rounded to nearest even at bit 16 (low 16 bits left as they are
+    after the add; finite inputs: the largest sum, 0xFF7FFFFF + 0x8000, stays in 32 bits)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    r += u
+    r += np.uint32(0x7FFF)
+    return r
+
+
 def bf16_bits(a: np.ndarray) -> np.ndarray:
     """fp32 -> bf16 bit patterns (uint16), round to nearest even (finite inputs)."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return r.astype(np.uint16)
+    return (_bf16_rounded_u32(a) >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -76,7 +89,9 @@ def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
 
 
 def round_bf16(a: np.ndarray) -> np.ndarray:
-    return bf16_to_f32(bf16_bits(a))
+    r = _bf16_rounded_u32(a)
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32).reshape(np.shape(a))
 
 
 def zipf_targets(rng: np.random.Generator, n: int, C: int, alpha: float) -> np.ndarray:
@@ -90,13 +105,37 @@ def zipf_targets(rng: np.random.Generator, n: int, C: int, alpha: float) -> np.n
     return np.minimum(np.searchsorted(cdf, u, side="right"), C - 1).astype(np.int32)
 
 
+_BLOCK = 1 << 22
+_SINGLE_STREAM_MAX = 1 << 24
+
+
+def _standard_normal(rng: np.random.Generator, seed: int, tag: int, shape) -> np.ndarray:
+    """fp32 N(0, 1) draws: from `rng` for up to 2^24 elements, else block by block."""
+    n = int(np.prod(shape))
+    if n <= _SINGLE_STREAM_MAX:
+        return rng.standard_normal(shape, dtype=np.float32)
+    out = np.empty(n, np.float32)
+    nb = (n + _BLOCK - 1) // _BLOCK
+    kids = np.random.SeedSequence([seed, tag]).spawn(nb)
+
+    def fill(b):
+        np.random.Generator(np.random.PCG64(kids[b])).standard_normal(
+            out=out[b * _BLOCK:(b + 1) * _BLOCK], dtype=np.float32)
+
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        list(ex.map(fill, range(nb)))
+    return out.reshape(shape)
+
+
 def make_inputs(w: Workload, seed: int = 0):
     """(X, Y, targets) as fp32 numpy arrays (bf16 workloads already rounded to bf16)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     xs = w.x_std if w.x_std is not None else w.d ** -0.5
     ys = w.y_std if w.y_std is not None else w.d ** -0.5
-    X = (rng.standard_normal((w.N, w.d), dtype=np.float32) * np.float32(xs))
-    Y = (rng.standard_normal((w.C, w.d), dtype=np.float32) * np.float32(ys))
+    X = _standard_normal(rng, seed, 0, (w.N, w.d))
+    X *= np.float32(xs)
+    Y = _standard_normal(rng, seed, 1, (w.C, w.d))
+    Y *= np.float32(ys)
     if w.y_norm_alpha > 0.0:
         s = np.arange(1, w.C + 1, dtype=np.float64) ** (-w.y_norm_alpha)
         s /= np.sqrt(np.mean(s * s))

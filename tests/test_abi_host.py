@@ -140,7 +140,7 @@ def test_calls_reject_misaligned_matrices_without_gpu():
 def test_plan_paths_follow_the_shape():
     """rece_plan_paths: which kernels a plan runs (decided on the host, no GPU needed)."""
     TC, DX, SC = _lib.PATH_TENSOR_CORES, _lib.PATH_DX_TENSORS, _lib.PATH_STORED_SCORES
-    DY = _lib.PATH_DY_TENSORS
+    DY, PARTS = _lib.PATH_DY_TENSORS, _lib.PATH_DX_PARTS
     from reduced_cross_entropy_b200 import synth
     W = synth.WORKLOADS
 
@@ -150,9 +150,12 @@ def test_plan_paths_follow_the_shape():
 
     assert paths(W["tiny"]) == 0                      # fp32 exact mode: fmaf kernels
     assert paths(W["sasrec"]) == TC                   # catalogue in L2: gathered dX
-    assert paths(W["large"]) == TC | DX               # 256 MB catalogue: dX on tcgen05
-    assert paths(W["lm"]) == TC | DX | SC | DY        # d = 4096: stored scores, dY on tcgen05
-    assert paths(W["very_large"]) == TC | DX          # d = 256: dY by the pair sort
+    # 256 MB catalogue: dX on tcgen05; 400 row tiles a round, two CTAs an SM: both rounds
+    # in one launch (parts summed in order) fill the waves better than a launch a round
+    assert paths(W["large"]) == TC | DX | PARTS
+    # d = 4096: stored scores, dY on tcgen05; 1024 work items a round: a launch a round
+    assert paths(W["lm"]) == TC | DX | SC | DY
+    assert paths(W["very_large"]) == TC | DX | PARTS  # d = 256: dY by the pair sort
     assert paths(W["sasrec"], d=48) == 0              # d not a multiple of 64
     p = Plan(256, 4096, 64, 16, 8, 1, 1, 32, mode="bf16", flags=_lib.FLAG_FMA_SCORES)
     assert p.paths == 0                               # fmaf scores on request

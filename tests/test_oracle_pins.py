@@ -304,6 +304,33 @@ def test_rece_grad_invariants():
     assert len(untouched) > 0 and np.all(dY[untouched] == 0.0)
 
 
+def test_rece_grad_row_and_item_samples_match_the_full_gradient():
+    """rece_grad_rows / rece_grad_items (the full-size parity checks' expected values)
+    against rece_grad, which finite differences and autograd pin; a planted duplicate entry
+    and an item nobody selects cover the counting rules."""
+    X, Y, z, B = _random_case(N=60, C=300, d=8)
+    out = oracle.rece_forward(X, Y, z, B, 6, 1, 5)
+    sel, lse = out["selected"].copy(), out["lse"]
+    sel[3, 0] = sel[3, 1]  # a duplicate entry counts twice, as rece_grad counts it
+    _, _, lse = oracle.rece_loss(X, Y, z, sel)
+    dX, dY = oracle.rece_grad(X, Y, z, sel, lse, 0.7)
+    rows = np.array([0, 3, 17, 59])
+    gX = oracle.rece_grad_rows(X, Y, z, rows, sel[rows], lse[rows], 0.7)
+    assert rel_err(gX, dX[rows]) < 1e-12
+    touched = set(z.tolist()) | set(sel[sel >= 0].tolist())
+    nobody = min(set(range(len(Y))) - touched)
+    items = [int(z[0]), int(sel[3, 1]), int(sel[10, 2]), nobody, len(Y) - 1]
+    every = np.arange(len(X))
+    gY = oracle.rece_grad_items(X, Y, z, every, sel, lse, items, 0.7)
+    assert rel_err(gY, dY[items]) < 1e-12
+    assert np.all(gY[3] == 0.0)
+    # rows that hold none of the items may be left out
+    keep = np.nonzero(np.isin(sel, items).any(axis=1) | np.isin(z, items))[0]
+    assert len(keep) < len(X)
+    gY2 = oracle.rece_grad_items(X, Y, z, keep, sel[keep], lse[keep], items, 0.7)
+    assert rel_err(gY2, dY[items]) < 1e-12
+
+
 def test_rece_grad_equals_full_ce_grad_in_full_case():
     X, Y, z, B = _random_case(N=20, C=50, d=6, n_b=1, n_r=1)
     out = oracle.rece_forward(X, Y, z, B, 1, 0, len(Y) - 1)
