@@ -525,8 +525,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
       e0 = __ldg(off + idx);
       e1 = __ldg(off + idx + 1);
     };
-    int nx0, nx1;
-    entry_range(0, nx0, nx1);
+    // Slab s's first kPre entries wait in registers, loaded while slab s - 1 was built
+    // (its range known a slab earlier still), so the entry loads overlap the MMAs and
+    // the clearing instead of following them; a longer run is loaded on the spot.
+    constexpr int kPre = 16;
+    auto slab_entries = [&](int s2) {
+      return a.kept + (rN + (lo + s2) * kBK + kc) * a.k;
+    };
+    int a0, a1, b0, b1;  // entry ranges of slabs s and s + 1
+    entry_range(0, a0, a1);
+    entry_range(1, b0, b1);
+    int2 pre[kPre];
+    {
+      const int2* ent = slab_entries(0);
+#pragma unroll
+      for (int u = 0; u < kPre; ++u)
+        pre[u] = a0 + u < a1 ? __ldg(ent + a0 + u) : make_int2(0, 0);
+    }
     bool ok = true;
     for (int s = 0; s < nK; ++s) {
       const int as = s % kAStages;
@@ -542,19 +557,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
         zero_row(tl, t);
       }
       named_barrier(1, kBuilders);  // the whole tile is clear before anyone fills it
-      const int e0 = nx0, e1 = nx1;
-      entry_range(s + 1, nx0, nx1);
-      if (ok && e1 > e0) {
-        const int2* ent = a.kept + (rN + (lo + s) * kBK + kc) * a.k;
-        for (int e = e0; e < e1; e += 8) {  // eight loads in flight
+      int c0, c1;
+      entry_range(s + 2, c0, c1);
+      if (ok && a1 > a0) {
+#pragma unroll
+        for (int u = 0; u < kPre; ++u)
+          if (a0 + u < a1) put(th, tl, int(pre[u].x - q0), kc, uint32_t(pre[u].y));
+        const int2* ent = slab_entries(s);
+        for (int e = a0 + kPre; e < a1; e += 8) {  // the rest, eight loads in flight
           int2 en[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) en[u] = e + u < e1 ? __ldg(ent + e + u) : make_int2(0, 0);
+          for (int u = 0; u < 8; ++u) en[u] = e + u < a1 ? __ldg(ent + e + u) : make_int2(0, 0);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            if (e + u < e1) put(th, tl, int(en[u].x - q0), kc, uint32_t(en[u].y));
+            if (e + u < a1) put(th, tl, int(en[u].x - q0), kc, uint32_t(en[u].y));
         }
       }
+      {  // slab s + 1's first entries
+        const int2* ent = slab_entries(s + 1);
+#pragma unroll
+        for (int u = 0; u < kPre; ++u)
+          pre[u] = b0 + u < b1 ? __ldg(ent + b0 + u) : make_int2(0, 0);
+      }
+      a0 = b0;
+      a1 = b1;
+      b0 = c0;
+      b1 = c1;
       fence_proxy_async_smem();  // this thread's tile writes, visible to the MMA
       named_barrier(1, kBuilders);  // nobody clears the next tile into this one's readers
       __syncwarp();
