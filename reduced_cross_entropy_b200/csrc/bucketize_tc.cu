@@ -207,6 +207,223 @@ __global__ void __launch_bounds__(kThreads, 1) k_bucketize_tc(
   }
 }
 
+// The same for d <= 256, with the rows kept resident: work item = (round, 256-row tile of
+// X or Y) whose two 128-row blocks (all of d: at most 4 slices of 64) are loaded once,
+// while only B_r streams, in 128-vector x 64 slices.  Each B slice feeds both row blocks
+// (two MMAs of M = 128, N = 128), so a B element is read once per 256 rows and an input
+// row once per round: three times fewer L2 bytes per multiply-add than the streamed
+// kernel, whose (128 + 256)-element slices fed one 128 x 256 tile.  TMEM: one
+// accumulator of 128 columns per (row block, buffer).  Eight epilogue warps, a row each.
+constexpr int kRBStages = 4;
+constexpr int kRBN = 128;                                  // B vectors per slice
+constexpr int kRMaxK = 4;                                  // d <= 256
+constexpr uint32_t kRSliceA = kBM * kBK * 2;               // 16 KB
+constexpr uint32_t kRSliceB = kRBN * kBK * 2;              // 16 KB
+constexpr int kRThreads = 64 + 256;
+
+struct __align__(1024) SmemRes {
+  uint8_t a[2][kRMaxK][kRSliceA];  // [row block][k slice]
+  uint8_t b[kRBStages][kRSliceB];
+  uint64_t full[kRBStages];
+  uint64_t empty[kRBStages];
+  uint64_t a_full, a_empty;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void on_timeout_res(SmemRes& s, uint32_t* status) {
+  *reinterpret_cast<volatile int*>(&s.abort) = 1;
+  raise_flag(status, RECE_DEVICE_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kRThreads, 1) k_bucketize_tc_res(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+    const __grid_constant__ CUtensorMap tmB, int64_t N, int64_t C, int d, int n_b, int n_r,
+    int bn, int32_t* __restrict__ bx, int32_t* __restrict__ by, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemRes& s = *reinterpret_cast<SmemRes*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kRows = 2 * kBM;
+  const int64_t tX = (N + kRows - 1) / kRows, tY = (C + kRows - 1) / kRows;
+  const int64_t per_round = tX + tY, items = per_round * n_r;
+  const int n_nt = (n_b + kRBN - 1) / kRBN;
+  const int nk = d / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRBStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    mbar_init(&s.a_full, 1);
+    mbar_init(&s.a_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 8);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abortp = &s.abort;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    uint32_t it = 0, ni = 0;
+    bool ok = true;
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmY);
+      prefetch_tmap(&tmB);
+      for (int64_t item = blockIdx.x; item < items && ok && !*abortp;
+           item += gridDim.x, ++ni) {
+        const int r = int(item / per_round);
+        const int64_t t = item % per_round;
+        const bool isY = t >= tX;
+        const int64_t row0 = (isY ? t - tX : t) * kRows;
+        // the rows, once the previous item's MMAs are done with them
+        if (!mbar_wait(&s.a_empty, (ni & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+          on_timeout_res(s, status);
+          break;
+        }
+        mbar_arrive_expect_tx(&s.a_full, 2u * uint32_t(nk) * kRSliceA);
+        for (int rb = 0; rb < 2; ++rb)
+          for (int ks = 0; ks < nk; ++ks)
+            tma_load_2d(s.a[rb][ks], isY ? &tmY : &tmX, &s.a_full, ks * kBK,
+                        int32_t(row0 + rb * kBM));
+        for (int nt = 0; nt < n_nt && ok; ++nt) {
+          for (int ks = 0; ks < nk; ++ks, ++it) {
+            const int st = it % kRBStages;
+            if (!mbar_wait(&s.empty[st], ((it / kRBStages) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+              on_timeout_res(s, status);
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&s.full[st], uint32_t(bn) * kBK * 2);
+            tma_load_2d(s.b[st], &tmB, &s.full[st], ks * kBK, r * n_b + nt * kRBN);
+          }
+        }
+      }
+      // teardown: the last loads have landed (or we give up after the limit)
+      for (uint32_t j = (it > kRBStages ? it - kRBStages : 0); j < it; ++j)
+        mbar_wait_limit(&s.full[j % kRBStages], (j / kRBStages) & 1u, kTimeoutNs);
+      if (ni > 0) mbar_wait_limit(&s.a_full, (ni - 1) & 1u, kTimeoutNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, bn);
+      uint32_t it = 0, acc_it = 0, ni = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < items && ok && !*abortp;
+           item += gridDim.x, ++ni) {
+        if (!mbar_wait(&s.a_full, ni & 1u, &s.abort, kTimeoutNs)) {
+          on_timeout_res(s, status);
+          break;
+        }
+        for (int nt = 0; nt < n_nt && ok; ++nt, ++acc_it) {
+          const int a = acc_it & 1;
+          if (!mbar_wait(&s.acc_empty[a], ((acc_it >> 1) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+            on_timeout_res(s, status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int ks = 0; ks < nk; ++ks, ++it) {
+            const int st = it % kRBStages;
+            if (!mbar_wait(&s.full[st], (it / kRBStages) & 1u, &s.abort, kTimeoutNs)) {
+              on_timeout_res(s, status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t db = desc_k_sw128(smem_u32(s.b[st]));
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb) {
+              const uint64_t da = desc_k_sw128(smem_u32(s.a[rb][ks]));
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                mma_bf16(tmem + uint32_t(rb * 256 + a * kRBN), da + 2 * kk, db + 2 * kk, idesc,
+                         (ks | kk) != 0);
+            }
+            mma_commit(&s.empty[st]);
+          }
+          if (!ok) break;
+          mma_commit(&s.acc_full[a]);
+        }
+        if (!ok) break;
+        mma_commit(&s.a_empty);  // the rows may be replaced
+      }
+      // teardown: every MMA issued so far has completed
+      mma_commit(&s.drain);
+      mbar_wait_limit(&s.drain, 0, kTimeoutNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int rb = (warp - 2) >> 2;  // and its row block
+    const int row_local = rb * kBM + q * 32 + lane;
+    uint32_t acc_it = 0;
+    for (int64_t item = blockIdx.x; item < items && !*abortp; item += gridDim.x) {
+      const int r = int(item / per_round);
+      const int64_t t = item % per_round;
+      const bool isY = t >= tX;
+      const int64_t row0 = (isY ? t - tX : t) * kRows;
+      float best = -INFINITY;
+      int best_b = INT_MAX;
+      bool ok = true;
+      for (int nt = 0; nt < n_nt; ++nt, ++acc_it) {
+        const int a = acc_it & 1;
+        if (!mbar_wait(&s.acc_full[a], (acc_it >> 1) & 1u, &s.abort, kTimeoutNs)) {
+          on_timeout_res(s, status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem + (uint32_t(q * 32) << 16) + uint32_t(rb * 256 + a * kRBN);
+        for (int c0 = 0; c0 < bn; c0 += 32) {
+          float v[32];
+          tmem_load32(taddr + c0, v);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int b = nt * kRBN + c0 + u;
+            if (b < n_b && v[u] > best) {
+              best = v[u];
+              best_b = b;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.acc_empty[a]);
+      }
+      if (!ok) break;
+      const int64_t row = row0 + row_local;
+      const int64_t M = isY ? C : N;
+      if (row < M) (isY ? by : bx)[int64_t(r) * M + row] = best_b;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void* Y,
@@ -223,6 +440,22 @@ cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void*
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tmB, B, uint64_t(c.n_r) * c.n_b, c.d, bn);
   if (e != cudaSuccess) return e;
+  if (c.d <= kRMaxK * kBK) {
+    // rows resident, B streamed once per 256 rows
+    const int bnr = c.n_b >= kRBN ? kRBN : ((c.n_b + 15) / 16) * 16;
+    e = make_tmap_bf16(&tmB, B, uint64_t(c.n_r) * c.n_b, c.d, bnr);
+    if (e != cudaSuccess) return e;
+    const int64_t items = (ceil_div(c.N, 2 * kBM) + ceil_div(c.C, 2 * kBM)) * c.n_r;
+    const int grid = int(items < sm_count() ? items : sm_count());
+    const size_t smem = sizeof(SmemRes) + 1024;
+    e = cudaFuncSetAttribute(k_bucketize_tc_res, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    k_bucketize_tc_res<<<grid, kRThreads, smem, st>>>(tmX, tmY, tmB, c.N, c.C, c.d, c.n_b,
+                                                      c.n_r, bnr, bx, by, status);
+    count_launches(1);
+    return cudaGetLastError();
+  }
   const int64_t items = (ceil_div(c.N, kBM) + ceil_div(c.C, kBM)) * c.n_r;
   const int grid = int(items < sm_count() ? items : sm_count());
   const size_t smem = sizeof(Smem) + 1024;
