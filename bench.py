@@ -144,16 +144,20 @@ def kernel_sources(stage, paths):
     from reduced_cross_entropy_b200 import _lib
     src = dict(KERNEL_SOURCES)
     if paths & _lib.PATH_TENSOR_CORES:
-        src.update(bucketize=["bucketize_tc.cu", "permute.cu"],
+        src.update(bucketize=["bucketize_tc.cu", "sm100.cuh"], sort=["sort.cu", "permute.cu"],
                    select=["select_tc.cu", "sm100.cuh", "tc_bins.cuh"],
                    merge_loss=["merge_tc.cu"])
     if paths & _lib.PATH_STORED_SCORES:
         src["select"] = ["scores_tc.cu", "sm100.cuh", "tc_bins.cuh"]
     if paths & _lib.PATH_DX_TENSORS:
-        src["bwd_rows"] = ["backward.cu", "bwd_tc.cu", "sm100.cuh"]
+        src["bwd_rows"] = ["backward.cu", "bwd_tc.cu", "sm100.cuh", "tc_common.cu"]
+    if paths & _lib.PATH_DY_TENSORS:  # the positives' pair backward, then the band products
+        src.update(bwd_sort=["backward.cu", "sort.cu", "rece_abi.cu"],
+                   bwd_items=["bwd_tc.cu", "sm100.cuh"])
     if paths & _lib.PATH_ALL_NEGATIVES:
         src.update(select=["window_tc.cu", "window.cu", "sm100.cuh"],
-                   merge_loss=["window.cu"], bwd_rows=["backward.cu", "window_tc.cu"],
+                   merge_loss=["window.cu"],
+                   bwd_rows=["backward.cu", "window_tc.cu", "tc_common.cu"],
                    bwd_sort=["sort.cu", "rece_abi.cu"], bwd_items=["window_tc.cu"])
     return src[stage]
 

@@ -45,6 +45,39 @@ struct __align__(1024) Smem {
   int abort;
 };
 
+// Running (max, argmax) over the scores v[0..32) of vectors b0..b0+31 (those >= n_b
+// excluded), ties to the lowest b: the earlier chunk keeps a tie (strict >), and inside a
+// chunk the first u whose score equals the chunk's maximum wins.  A full chunk costs a
+// max tree (one instruction a score); the index is searched only when the chunk beats
+// the running best, which gets rare as the best rises.  NaN scores never win.
+__device__ __forceinline__ void argmax32(const float (&v)[32], int b0, int n_b, float& best,
+                                         int& best_b) {
+  if (b0 + 32 <= n_b) {
+    float m[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) m[u] = fmaxf(v[2 * u], v[2 * u + 1]);
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+      for (int u = 0; u < w; ++u) m[u] = fmaxf(m[u], m[u + w]);
+    if (m[0] > best) {
+      int idx = 31;
+#pragma unroll
+      for (int u = 31; u >= 0; --u)
+        if (v[u] == m[0]) idx = u;
+      best = m[0];
+      best_b = b0 + idx;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 32; ++u)
+      if (b0 + u < n_b && v[u] > best) {
+        best = v[u];
+        best_b = b0 + u;
+      }
+  }
+}
+
 __device__ __forceinline__ void on_timeout(Smem& s, uint32_t* status) {
   *reinterpret_cast<volatile int*>(&s.abort) = 1;
   raise_flag(status, RECE_DEVICE_TIMEOUT);
@@ -179,14 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bucketize_tc(
         for (int c0 = 0; c0 < bn; c0 += 32) {
           float v[32];
           tmem_load32(taddr + c0, v);
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int b = nt * kBN + c0 + u;
-            if (b < n_b && v[u] > best) {
-              best = v[u];
-              best_b = b;
-            }
-          }
+          argmax32(v, nt * kBN + c0, n_b, best, best_b);
         }
         tc_fence_before();
         __syncwarp();
@@ -396,14 +422,7 @@ __global__ void __launch_bounds__(kRThreads, 1) k_bucketize_tc_res(
         for (int c0 = 0; c0 < bn; c0 += 32) {
           float v[32];
           tmem_load32(taddr + c0, v);
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int b = nt * kRBN + c0 + u;
-            if (b < n_b && v[u] > best) {
-              best = v[u];
-              best_b = b;
-            }
-          }
+          argmax32(v, nt * kRBN + c0, n_b, best, best_b);
         }
         tc_fence_before();
         __syncwarp();
