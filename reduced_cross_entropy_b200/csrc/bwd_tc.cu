@@ -511,16 +511,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
     const int64_t slice = (q0 >> 6) + half;
     // the entries of slab s's row in this half: [e0, e1) of its kept list, found a slab
     // ahead so that the offsets' load latency overlaps the previous slab
+    // the window of this thread's row, tracked as the slabs advance (the row only grows):
+    // the 64-bit divisions of the chunk arithmetic run when the row enters a new chunk,
+    // not at every slab
+    int64_t wc = -1, wc_hi = 0, sig0 = 0;  // the row's chunk, its end, its window's slab
+    int wS = 0;                             // and the window's slab count
+    auto set_chunk = [&](int64_t c) {
+      wc = c;
+      wc_hi = chunk_start(c + 1, N, a.n_c);
+      const int64_t w0 = chunk_start(c - a.n_ec < 0 ? 0 : c - a.n_ec, C, a.n_c);
+      const int64_t w1 = chunk_start(c + a.n_ec + 1 > a.n_c ? a.n_c : c + a.n_ec + 1, C, a.n_c);
+      sig0 = w0 >> 6;
+      wS = w1 > w0 ? int((w1 - 1) >> 6) - int(sig0) + 1 : 0;
+    };
     auto entry_range = [&](int s2, int& e0, int& e1) {
       e0 = e1 = 0;
-      const int64_t p = (lo + s2) * kBK + kc;  // sorted row
+      const int64_t p = (lo + s2) * kBK + kc;  // sorted row (grows with s2)
       if (s2 >= nK || p < k0 || p >= k1 || p >= N) return;
-      int64_t w0, w1;
-      row_window(p, N, C, a.n_c, a.n_ec, w0, w1);
-      const int64_t sig0 = w0 >> 6;
-      const int S = w1 > w0 ? int((w1 - 1) >> 6) - int(sig0) + 1 : 0;
+      if (wc < 0) set_chunk(chunk_of(p, N, a.n_c));
+      while (p >= wc_hi) set_chunk(wc + 1);
       const int64_t idx = slice - sig0;
-      if (idx < 0 || idx >= S) return;
+      if (idx < 0 || idx >= wS) return;
       const int32_t* off = a.kept_off + (rN + p) * a.Sp;
       e0 = __ldg(off + idx);
       e1 = __ldg(off + idx + 1);
