@@ -327,11 +327,16 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
     const T* __restrict__ X, int64_t C, int d, int k, const int32_t* __restrict__ item_start,
     const int32_t* __restrict__ sorted_id, const float* __restrict__ pair_g,
-    const float* __restrict__ sorted_g, float* __restrict__ dY) {
+    const float* __restrict__ sorted_g, int32_t* __restrict__ long_items,
+    float* __restrict__ dY) {
   const int lane = threadIdx.x & 31, q = lane >> 3, sub = lane & 7;
   const int64_t j = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
   if (j >= C) return;
   const int64_t lo = item_start[j], hi = item_start[j + 1];
+  if (long_items && hi - lo > kLongRunPairs) {  // a popular item: k_bwd_items_long sums it
+    if (lane == 0) long_items[1 + atomicAdd(long_items, 1)] = int32_t(j);
+    return;
+  }
   const int slots = k + 1;
   for (int t0 = 0; t0 < d; t0 += 64) {
     const int t = t0 + 8 * sub;
@@ -366,6 +371,73 @@ __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
       float4* o = reinterpret_cast<float4*>(dY + j * d + t);
       o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
       o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+}
+
+// dY of the items k_bwd_items_v8 left out (runs of more than kLongRunPairs pairs: the
+// targets are Zipf-drawn, and the most popular item's run would keep one warp busy long
+// after the others finished).  A CTA per listed item: warp w sums the w-th of kLongWarps
+// contiguous parts of the run (pairs in order, four rows in flight, as k_bwd_items_v8),
+// then one thread per dimension adds the warps' parts in warp order: deterministic.
+// long_items[0] is the count, the ids follow (their order does not matter: each item is
+// summed by one CTA alone).
+constexpr int kLongWarps = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(kLongWarps * 32) k_bwd_items_long(
+    const T* __restrict__ X, int d, int k, const int32_t* __restrict__ item_start,
+    const int32_t* __restrict__ sorted_id, const float* __restrict__ pair_g,
+    const float* __restrict__ sorted_g, const int32_t* __restrict__ long_items,
+    float* __restrict__ dY) {
+  __shared__ float part[kLongWarps][64];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane >> 3, sub = lane & 7;
+  const int count = long_items[0];
+  const int slots = k + 1;
+  for (int li = blockIdx.x; li < count; li += gridDim.x) {
+    const int64_t j = long_items[1 + li];
+    const int64_t lo = item_start[j], n = item_start[j + 1] - lo;
+    const int64_t a0 = lo + n * warp / kLongWarps, a1 = lo + n * (warp + 1) / kLongWarps;
+    for (int t0 = 0; t0 < d; t0 += 64) {
+      const int t = t0 + 8 * sub;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int64_t b = a0; b < a1; b += 32) {
+        const int m = int(a1 - b < 32 ? a1 - b : 32);
+        int32_t row = 0;
+        float g = 0.0f;
+        if (lane < m) {
+          const int32_t id = sorted_id[b + lane];
+          row = id / slots;
+          g = sorted_g ? sorted_g[b + lane] : pair_g[id];
+        }
+        for (int e0 = 0; e0 < m; e0 += 4) {
+          const int e = e0 + q;
+          const int32_t r = __shfl_sync(0xFFFFFFFFu, row, e & 31);
+          const float ge = __shfl_sync(0xFFFFFFFFu, g, e & 31);
+          if (e < m && t < d) {
+            float v[8];
+            load8v(X + int64_t(r) * d + t, v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = fmaf(ge, v[u], acc[u]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], 8);
+        acc[u] += __shfl_xor_sync(0xFFFFFFFFu, acc[u], 16);
+      }
+      __syncthreads();  // the last slice's parts are added
+      if (q == 0) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part[warp][8 * sub + u] = acc[u];
+      }
+      __syncthreads();
+      if (threadIdx.x < 64 && t0 + int(threadIdx.x) < d) {
+        float s = 0.0f;
+        for (int w = 0; w < kLongWarps; ++w) s += part[w][threadIdx.x];
+        dY[j * d + t0 + threadIdx.x] = s;
+      }
     }
   }
 }
@@ -727,10 +799,18 @@ cudaError_t launch_backward(const rece_plan_s& p, const T* X, const T* Y,
     if (e != cudaSuccess) return e;
     k_bwd_items_wide<T><<<unsigned(c.C), 32 + c.d / 16, smem, st>>>(
         X, c.d, c.k, stages, item_start, in, e_g, sorted_g, dY, status);
-  } else if (c.d % 8 == 0)
+  } else if (c.d % 8 == 0) {
+    // popular items go to a list that k_bwd_items_long sums, a CTA per item
+    int32_t* long_items = reinterpret_cast<int32_t*>(ws + L.e_long);
+    cudaError_t e = cudaMemsetAsync(long_items, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
     k_bwd_items_v8<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
-        X, c.C, c.d, c.k, item_start, in, e_g, sorted_g, dY);
-  else
+        X, c.C, c.d, c.k, item_start, in, e_g, sorted_g, long_items, dY);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_items_long<T><<<unsigned(2 * sm_count()), kLongWarps * 32, 0, st>>>(
+        X, c.d, c.k, item_start, in, e_g, sorted_g, long_items, dY);
+  } else
     k_bwd_items<T><<<unsigned(ceil_div(c.C, warps)), kThreads, 0, st>>>(
         X, c.C, c.d, c.k, item_start, in, e_g, sorted_g, dY);
   count_launches(1);

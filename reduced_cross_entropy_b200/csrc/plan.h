@@ -56,6 +56,10 @@ inline size_t sort_hist_bytes(int64_t M, int bits) {
   return align256(sizeof(int32_t) * size_t(ceil_div(M, kSortTile) << bits));
 }
 
+// dY by gathered rows: an item whose run holds more pairs than this is summed by a whole
+// CTA (its run split among the warps, the parts added in warp order) instead of one warp.
+constexpr int kLongRunPairs = 256;
+
 struct Layout {
   size_t status = 0;
   // forward region (from rece_bucketize_sort to the end of rece_loss_fwd)
@@ -68,7 +72,8 @@ struct Layout {
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_key_b = 0,
-         e_sorted_g = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0;
+         e_sorted_g = 0, e_g_b = 0, e_item_start = 0, e_scratch = 0,
+         e_long = 0;  // dY: count and list of the items with runs of > kLongRunPairs pairs
   size_t bwd_end = 0;
   // tensor-core dX (and dY): kept from rece_loss_fwd to rece_loss_bwd (not aliased): the
   // sorted copies of Y (and X) -- xs, ys above, placed here then -- the kept entries by

@@ -76,6 +76,7 @@ void layout_pairs(rece_plan_s& p, size_t& off) {
   }
   L.e_item_start = take(sizeof(int32_t) * (size_t(p.cfg.C) + 1));
   L.e_scratch = take(sort_scratch_bytes(p.entries, p.item_pass_bits));
+  L.e_long = take(sizeof(int32_t) * (E / kLongRunPairs + 2));
 }
 
 // Item-sort geometry of the backward's pairs (keys 0..C: C marks an empty slot).  Digits
