@@ -12,7 +12,8 @@
 //                                   id), then one warp per item sums its pairs in row
 //                                   order, fetching each pair's g by its id -- or, when
 //                                   the g array is too large for L2, g rides along in
-//                                   the sort)
+//                                   the sort; an item with a long run is summed by a
+//                                   CTA, its warps' parts added in warp order)
 // Pair e = i*(k+1) + s holds slot s of row i (s = 0: the positive, s >= 1: selected
 // negative s-1); an empty slot carries the key C, which sorts after every item.  Every
 // sum has a fixed order: the gradients are deterministic.
@@ -322,7 +323,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd_rows_v8(
   }
 }
 
-// One warp per item; quarter q adds the pairs b = lo + q (mod 4) in row order.
+// One warp per item; quarter q adds the pairs b = lo + q (mod 4) in row order.  With
+// `long_items`, an item of more than kLongRunPairs pairs is only listed there (count in
+// long_items[0]) for k_bwd_items_long.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_bwd_items_v8(
     const T* __restrict__ X, int64_t C, int d, int k, const int32_t* __restrict__ item_start,
