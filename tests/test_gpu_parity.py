@@ -155,6 +155,22 @@ def test_backward_is_deterministic():
     assert a["loss"] == b["loss"]
 
 
+def test_popular_items_summed_by_a_cta():
+    """Items whose (item, row) runs exceed 256 pairs take the dY kernel that splits a run
+    among a CTA's warps: here every row's positive is one of three items (runs of 300 to
+    600 pairs and more) in the fp32 exact mode, against the oracle, and twice for
+    determinism."""
+    w = synth.Workload("popular", N=1200, C=2500, d=24, dtype="fp32", n_b=8, n_c=6, n_ec=1,
+                       n_r=2, k=40)
+    X, Y, _ = synth.make_inputs(w, seed=8)
+    t = np.array([(0, 0, 7, 1999)[i % 4] for i in range(w.N)], dtype=np.int32)
+    B = synth.projections(8, 0, w.n_r, w.n_b, w.d, w.dtype)
+    g = run_gpu(w, X, Y, t, B, dloss=1.25)
+    compare(w, g, run_oracle(w, X, Y, t, B, dloss=1.25))
+    again = run_gpu(w, X, Y, t, B, dloss=1.25)
+    np.testing.assert_array_equal(g["dY"], again["dY"])
+
+
 def test_sort_many_buckets_and_one_bucket():
     for n_b in (4096, 1):
         w = synth.Workload("sort", N=20000, C=30011, d=16, dtype="fp32", n_b=n_b, n_c=16,
