@@ -165,7 +165,7 @@ struct Args {
   const int2* kept;         // [n_r][N][k] (sorted position, p as bf16 hi | lo << 16)
   const int32_t* kept_off;  // [n_r][N][Sp] slice starts within the round's entries
   const float* dloss;       // [1]
-  float* out;               // dX [N][d], accumulated into
+  float* out;               // dX [N][d] (added into) or dY [C][d] (stored or added into)
   uint32_t* status;
   int write;                // dY: store (round 0, which covers every position), else add
   // dX with parts: one grid over (round, K split): blockIdx.z = round * ksplit + split;
