@@ -224,7 +224,9 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
           if (pos < cap) {
             const uint32_t key = score_key(__int_as_float(e[u].x));
             keys[pos] = key;
-            poss[pos] = e[u].y;
+            // grouped output needs the sorted position; otherwise keep the item id, which
+            // the output then reads without a second gather
+            poss[pos] = kGrouped ? e[u].y : jj[u];
             kmax = key > kmax ? key : kmax;
           }
         }
@@ -254,6 +256,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
 
   // item id of candidate q (its round found from the boundaries)
   auto item_of = [&](int q) {
+    if constexpr (!kGrouped) return poss[q];
     int r = 0;
     while (r + 1 < n_r && q >= rb[r + 1]) ++r;
     return py[int64_t(r) * C + poss[q]];
@@ -323,7 +326,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
         if (tk) {
           const int dest = ns + __popc(b & ((1u << lane) - 1u));
           const float sc = key_score(keys[a]);
-          srow[dest] = py[int64_t(r) * C + poss[a]];
+          srow[dest] = poss[a];  // the item id (not grouped)
           if (lg) lg[1 + dest] = sc;
           worst = fminf(worst, sc);
           acc += expf(sc - m);
