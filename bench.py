@@ -41,7 +41,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="sasrec")
+    ap.add_argument("--workload", default="very_large",
+                    help="the headline workload (synth.WORKLOADS)")
+    ap.add_argument("--also", default="large,sasrec",
+                    help="one GPU: more workloads measured in the same run, reported under "
+                         "'workloads' (comma-separated; empty for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-memory", action="store_true")
     ap.add_argument("--no-allreduce-dy", action="store_true",
@@ -193,6 +197,8 @@ class ClockSampler:
         self.lines = []
 
     def __enter__(self):
+        if self.index is None:  # not sampled
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -238,43 +244,89 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_step_seconds(w, X, Y, t, B, rows=256, bucket_frac=16, all_negatives=False):
-    """Estimated seconds of one whole step of the CPU oracle, from a bounded sample:
-    bucketing of every bucket_frac-th row of X and Y (scaled up), the full stable sorts,
-    and selection + loss + gradient of `rows` rows (scaled by N / rows)."""
+def oracle_rate():
+    """Multiply-adds per second of the CPU oracle's scoring loops on this host (a short
+    bucketing run), used only to size the slices below."""
     import oracle
-    n_r = w.n_r
+    rng = np.random.Generator(np.random.PCG64(7))
+    V = rng.standard_normal((4096, 256), dtype=np.float32)
+    B = rng.standard_normal((256, 256), dtype=np.float32)
+    oracle.bucketize(V[:256], B)
     t0 = time.perf_counter()
-    for r in range(n_r):
-        oracle.bucketize(X[::bucket_frac], B[r])
-        oracle.bucketize(Y[::bucket_frac], B[r])
-    t_bucket = (time.perf_counter() - t0) * bucket_frac
-    # valid orders for the sampled rows come from a full (untimed) bucketing, once
-    if not hasattr(oracle_step_seconds, "_perm"):
-        bx = np.stack([oracle.bucketize(X, B[r]) for r in range(n_r)])
-        by = np.stack([oracle.bucketize(Y, B[r]) for r in range(n_r)])
-        oracle_step_seconds._perm = (bx, by)
-    bx, by = oracle_step_seconds._perm
+    oracle.bucketize(V, B)
+    return V.shape[0] * B.shape[0] * V.shape[1] / (time.perf_counter() - t0)
+
+
+def oracle_slice(w, seconds, rate):
+    """A proportional slice of workload w for the CPU oracle: N, C and n_c divided by the
+    same power of two f, so that chunks keep their sizes (N/n_c rows, C/n_c items) and
+    rows keep their windows, their n_b projections and their k; each row's and item's
+    work is then that of the whole workload (bar the clipped windows of the two end
+    chunks), and the slice's rows/s stands for the whole workload's.  f is the smallest
+    that brings the slice's multiply-adds (bucketing plus window scores) within `seconds`
+    at `rate`, keeping n_c >= 8; f = 1 (the workload itself) when it fits."""
+    from reduced_cross_entropy_b200 import synth
+
+    def fmaf(N, C, n_c):
+        ws = synth.Workload(w.name, N=N, d=w.d, C=C, dtype=w.dtype, n_b=w.n_b, n_c=n_c,
+                            n_ec=w.n_ec, n_r=w.n_r, k=w.k)
+        return (N + C) * w.n_b * w.d * w.n_r + pairs_per_round(ws) * w.d * w.n_r
+
+    f = 1
+    while (fmaf(w.N // f, w.C // f, w.n_c // f) > seconds * rate and w.n_c // (2 * f) >= 8
+           and w.N % (2 * f) == 0 and w.C % (2 * f) == 0 and w.n_c % (2 * f) == 0):
+        f *= 2
+    if f == 1:
+        return w, 1
+    return w.scaled(w.N // f, w.C // f, n_c=w.n_c // f), f
+
+
+def mean_window(w):
+    """Window items per row, averaged over the rows (edge chunks see clipped windows)."""
+    return pairs_per_round(w) / max(w.N, 1)
+
+
+def oracle_step(ws, X, Y, t, B, all_negatives=False):
+    """One whole step of the CPU oracle on workload ws (bucketing, stable sorts, the
+    selection or Algorithm 1's window sums, loss, gradients); returns its seconds."""
+    import oracle
     t0 = time.perf_counter()
-    px = np.stack([oracle.stable_argsort(bx[r]) for r in range(n_r)])
-    py = np.stack([oracle.stable_argsort(by[r]) for r in range(n_r)])
-    t_sort = time.perf_counter() - t0
-    sample = np.linspace(0, w.N - 1, rows).astype(np.int64)
-    t0 = time.perf_counter()
+    bx = [oracle.bucketize(X, B[r]) for r in range(ws.n_r)]
+    by = [oracle.bucketize(Y, B[r]) for r in range(ws.n_r)]
+    px = np.stack([oracle.stable_argsort(b) for b in bx])
+    py = np.stack([oracle.stable_argsort(b) for b in by])
     if all_negatives:  # Algorithm 1 as printed: every window item a negative
-        _, _, lse = oracle.window_loss(X, Y, t, px, py, w.n_c, w.n_ec, rows=sample)
-        oracle.window_grad(X, Y, t, px, py, w.n_c, w.n_ec, lse, 1.0, rows=sample)
-        return t_bucket + t_sort + (time.perf_counter() - t0) * w.N / rows
-    sel, _, _ = oracle.select(X, Y, t, px, py, w.n_c, w.n_ec, w.k, rows=sample)
-    _, _, lse = oracle.rece_loss(X[sample], Y, t[sample], sel)
-    oracle.rece_grad(X[sample], Y, t[sample], sel, lse, 1.0)
-    t_rows = (time.perf_counter() - t0) * w.N / rows
-    return t_bucket + t_sort + t_rows
+        _, _, lse = oracle.window_loss(X, Y, t, px, py, ws.n_c, ws.n_ec)
+        oracle.window_grad(X, Y, t, px, py, ws.n_c, ws.n_ec, lse, 1.0)
+    else:
+        sel, _, _ = oracle.select(X, Y, t, px, py, ws.n_c, ws.n_ec, ws.k)
+        _, _, lse = oracle.rece_loss(X, Y, t, sel)
+        oracle.rece_grad(X, Y, t, sel, lse, 1.0)
+    return time.perf_counter() - t0
 
 
-def oracle_sample_desc(rows, bucket_frac):
-    return (f"bucketing of every {bucket_frac}th row of X and Y (x{bucket_frac}), full stable "
-            f"sorts, selection+loss+gradient of {rows} evenly spaced rows (x N/{rows})")
+def oracle_sample_desc(w, ws, f):
+    if f == 1:
+        return f"the whole workload ({w.N} rows, {w.C} items): the oracle's full step, timed"
+    return (f"a 1/{f} slice of the workload, its whole step timed: N={ws.N} rows, C={ws.C} "
+            f"items, n_c={ws.n_c} (chunks of {w.N // w.n_c} rows and {w.C / w.n_c:g} items; "
+            f"n_b, d, k, n_ec as in the workload; {mean_window(ws):.0f} window items per row "
+            f"against the workload's {mean_window(w):.0f}); the slice's rows/s is reported "
+            f"for the whole workload (extrapolated, linear in N and C)")
+
+
+def cpu_baseline(w, seed, all_negatives=False, seconds=20.0):
+    """rows/s of the CPU oracle on workload w (or its proportional slice), one step of
+    about `seconds`."""
+    import oracle
+    from reduced_cross_entropy_b200 import synth
+    ws, f = oracle_slice(w, seconds, oracle_rate())
+    X, Y, t = synth.make_inputs(ws, seed=seed)
+    B = synth.projections(seed, 0, ws.n_r, ws.n_b, ws.d, ws.dtype)
+    sec = oracle_step(ws, X, Y, t, B, all_negatives)
+    return {"value": ws.N / sec, "unit": "rows/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "method": "extrapolated" if f > 1 else "full",
+            "sample": oracle_sample_desc(w, ws, f), "seconds": sec}
 
 
 def run_reference(args):
@@ -284,24 +336,28 @@ def run_reference(args):
     import oracle
     from reduced_cross_entropy_b200 import synth
     w = synth.WORKLOADS[args.workload]
-    X, Y, t = synth.make_inputs(w, seed=0)
-    B = synth.projections(0, 0, w.n_r, w.n_b, w.d, w.dtype)
-    rows, frac = 128, 32
+    # every step is one whole oracle step on a slice sized so that all warm-up and timed
+    # steps take about two minutes
+    ws, f = oracle_slice(w, 120.0 / max(args.steps + args.warmup, 1), oracle_rate())
+    X, Y, t = synth.make_inputs(ws, seed=0)
     alln = bool(getattr(args, "flags", 0) & 0x2)  # RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed
-    for _ in range(args.warmup):
-        oracle_step_seconds(w, X, Y, t, B, rows, frac, all_negatives=alln)
-    secs = [oracle_step_seconds(w, X, Y, t, B, rows, frac, all_negatives=alln)
-            for _ in range(args.steps)]
+    for s in range(args.warmup):
+        oracle_step(ws, X, Y, t, synth.projections(0, s, ws.n_r, ws.n_b, ws.d, ws.dtype), alln)
+    secs = [oracle_step(ws, X, Y, t,
+                        synth.projections(0, args.warmup + s, ws.n_r, ws.n_b, ws.d, ws.dtype),
+                        alln)
+            for s in range(args.steps)]
     total = sum(secs)
-    value = w.N * args.steps / total
+    value = ws.N * args.steps / total  # each step is the slice's whole step: ws.N rows
     cores = oracle.num_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000 * total / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "ms_per_step": 1000 * total / args.steps, "rows_per_step": ws.N,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workload_desc(w)},
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
-                             "sample": oracle_sample_desc(rows, frac)},
+                             "method": "extrapolated" if f > 1 else "full",
+                             "sample": oracle_sample_desc(w, ws, f)},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -344,6 +400,239 @@ def job_throughput(world, rows_per_step, steps, total_ms):
 
 
 # ------------------------------------------------------------------ GPU arm
+class WorkloadRun:
+    """One workload on one GPU: seeded inputs resident in HBM, a plan, its workspace and
+    outputs, and the step (rece_bucketize_sort + rece_loss_fwd + rece_loss_bwd, and the
+    ranks' dY exchange when there is one) timed with CUDA events on the launching stream."""
+
+    def __init__(self, torch, w, seed, dev, flags, n_steps, exchange):
+        from reduced_cross_entropy_b200 import _lib, ops, synth
+        self.torch, self.w, self.dev, self.exchange = torch, w, dev, exchange
+        self.L, self._lib = _lib.lib(), _lib
+        self.X, self.Y, self.t = synth.make_inputs(w, seed=seed)
+        self.tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype,
+                             flags=flags)
+        self.paths = self.plan.paths
+        self.Xd = torch.from_numpy(self.X).to(dev).to(self.tdt)
+        self.Yd = torch.from_numpy(self.Y).to(dev).to(self.tdt)
+        self.td = torch.from_numpy(self.t).to(dev)
+        # B is drawn afresh for every step (the method's randn inside the loss), keyed by
+        # (seed 0, step) on every rank so that the replicas bucket alike
+        self.Bs = [torch.from_numpy(synth.projections(0, s, w.n_r, w.n_b, w.d, w.dtype))
+                   .to(dev).to(self.tdt) for s in range(n_steps)]
+        self.ws = self.plan.workspace(dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.loss = torch.empty(1, **f32)
+        self.sel = torch.empty(w.N, w.k, dtype=torch.int32, device=dev)
+        self.lse = torch.empty(w.N, **f32)
+        self.logits = torch.empty(w.N, w.k + 1, **f32)
+        self.dloss = torch.ones(1, **f32)
+        self.dX = torch.empty(w.N, w.d, **f32)
+        self.dY = torch.empty(w.C, w.d, **f32)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.sp = ctypes.c_void_p(self.stream.cuda_stream)
+        self.nbytes = ctypes.c_size_t(self.ws.numel())
+
+    def step(self, Bt, Xc=None, Yc=None, tc=None):
+        vp = lambda x: ctypes.c_void_p(x.data_ptr())  # noqa: E731
+        L, h, sp, ck = self.L, self.plan._h, self.sp, self._lib.check
+        Xc = self.Xd if Xc is None else Xc
+        Yc = self.Yd if Yc is None else Yc
+        tc = self.td if tc is None else tc
+        ck(L.rece_bucketize_sort(h, vp(Bt), vp(Xc), vp(Yc), vp(self.ws), self.nbytes, sp),
+           "bucketize_sort")
+        ck(L.rece_loss_fwd(h, vp(Xc), vp(Yc), vp(tc), vp(self.ws), self.nbytes, vp(self.loss),
+                           None, vp(self.sel), vp(self.lse), vp(self.logits), sp), "loss_fwd")
+        ck(L.rece_loss_bwd(h, vp(Xc), vp(Yc), vp(tc), vp(self.sel), vp(self.lse),
+                           vp(self.logits), vp(self.dloss), vp(self.ws), self.nbytes,
+                           vp(self.dX), vp(self.dY), sp), "loss_bwd")
+        if self.exchange:
+            allreduce_dy(self.dY)
+
+    def warm(self, warmup):
+        for s in range(warmup):
+            self.flush.zero_()
+            self.step(self.Bs[s])
+        self.torch.cuda.synchronize(self.dev)
+        # status area: flags (a bad target or a timed-out wait fails the run; the
+        # tensor-core selection may flag rows it cannot certify exact) and row counts
+        words = self.ws[:16].view(self.torch.int32).cpu().tolist()
+        assert words[0] & ~self._lib.DEVICE_INEXACT == 0, f"device status {words[0]:#x}"
+        self.status_words = {"inexact_rows_per_step": int(words[1]),
+                             "overflowed_rows_per_step": int(words[2]),
+                             "merge_spilled_rows_per_step": int(words[3])}
+
+    def timed(self, first, steps, barrier=lambda: None, clock_index=None):
+        """`steps` steps from B number `first`, L2 flushed before each; per-step and
+        per-stage CUDA events (the library records the stage events on the same stream).
+        Returns (per-step ms, mean ms per stage, kernel launches, clock summary)."""
+        torch, _lib, stream = self.torch, self._lib, self.stream
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        n_st = len(_lib.STAGES)
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_st)]
+               for _ in range(steps)]
+        for row in sev:  # torch creates the CUDA event at its first record
+            for e in row:
+                e.record(stream)
+        sev_h = [(ctypes.c_void_p * (2 * n_st))(*[ctypes.c_void_p(e.cuda_event) for e in row])
+                 for row in sev]
+        launches0 = self.L.rece_kernel_launch_count()
+        barrier()
+        torch.cuda.synchronize(self.dev)
+        with ClockSampler(clock_index) as clk:
+            for s in range(steps):
+                self.flush.zero_()
+                _lib.check(self.L.rece_plan_set_stage_events(self.plan._h, sev_h[s]),
+                           "stage events")
+                ev[s][0].record(stream)
+                self.step(self.Bs[first + s])
+                ev[s][1].record(stream)
+            torch.cuda.synchronize(self.dev)
+        barrier()
+        launches = self.L.rece_kernel_launch_count() - launches0
+        self.L.rece_plan_set_stage_events(self.plan._h, None)
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        stage_ms = {name: statistics.mean(sev[s][2 * i].elapsed_time(sev[s][2 * i + 1])
+                                          for s in range(steps))
+                    for i, name in enumerate(_lib.STAGES)}
+        return step_ms, stage_ms, launches, (clk.summary() if clock_index is not None else None)
+
+    def rooflines(self, stage_ms):
+        """(roofline of the dominant stage, every stage's fraction of its roofline)."""
+        peaks = load_peaks()
+        work = stage_work(self.w, self.paths)
+
+        def one(name):
+            bound = stage_bound(name, self.paths)
+            flops, bytes_ = work[name]
+            sec = max(stage_ms[name], 1e-9) / 1000.0
+            if bound == "hbm":
+                achieved, peak, unit = bytes_ / sec / 1e9, peaks["hbm_gbs"], "GB/s"
+            elif bound == "tensor":
+                achieved, peak, unit = flops / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+            else:  # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
+                achieved, peak, unit = (flops / sec / 1e12,
+                                        148 * 128 * 2 * peaks["sm_max_mhz"] / 1e6, "TFLOP/s")
+            return {"bound": bound, "kernel": name, "achieved": achieved, "peak": peak,
+                    "unit": unit, "frac": achieved / peak,
+                    "peak_source": peaks["source"] if bound != "alu" else
+                    "derived: 148 SM x 128 FP32 lanes x 2 x sm_max_mhz",
+                    "traffic": recorded_traffic(name, self.w.name, self.paths),
+                    "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
+
+        dom = max(stage_ms, key=stage_ms.get)
+        return one(dom), {name: round(one(name)["frac"], 4) for name in stage_ms}
+
+    def path_roofline(self, ms_per_step):
+        """The whole step against the sum of every stage's roofline time."""
+        peaks = load_peaks()
+        t = 0.0
+        for name, (flops, bytes_) in stage_work(self.w, self.paths).items():
+            t += max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+        return {"roofline_ms": 1000 * t, "measured_ms": ms_per_step,
+                "frac": 1000 * t / ms_per_step}
+
+    def describe(self):
+        _lib, w, paths = self._lib, self.w, self.paths
+        return {"workload": workload_desc(w), **self.status_words,
+                "l2": "flushed between timed steps (256 MiB write)",
+                "scores": ("tcgen05" + (", stored" if paths & _lib.PATH_STORED_SCORES
+                                          else ", recomputed per pass")
+                           if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),
+                "dX": ("tcgen05 band products" +
+                       (", rounds in one launch, parts summed in order"
+                        if paths & _lib.PATH_DX_PARTS else "")
+                       if paths & _lib.PATH_DX_TENSORS else "gathered rows"),
+                "dY": ("tcgen05 band products" if paths & _lib.PATH_DY_TENSORS
+                       else "pairs sorted by item, gathered rows"),
+                "negatives": ("every window item (Algorithm 1 as printed), window "
+                              "sums and gradients on tcgen05"
+                              if paths & _lib.PATH_ALL_NEGATIVES else f"top-{w.k} per row")}
+
+    def e2e(self, warmup, steps, barrier=lambda: None):
+        """End to end through the same C-ABI calls: every step's inputs copied in from
+        pinned host memory and its loss copied out.  Step s+1's copies (a copy stream,
+        two device input sets) overlap step s's compute, as a training input pipeline
+        does; the L2 flush stays in the timeline; one pair of events spans all timed
+        steps.  Returns (total ms of the timed steps, h2d bytes per step, d2h bytes)."""
+        torch, dev, stream = self.torch, self.dev, self.stream
+        tdt = self.tdt
+        Xh = torch.from_numpy(self.X).to(tdt).pin_memory()
+        Yh = torch.from_numpy(self.Y).to(tdt).pin_memory()
+        th = torch.from_numpy(self.t).pin_memory()
+        Bh = [b.cpu().pin_memory() for b in self.Bs]
+        loss_h = torch.empty(len(self.Bs), dtype=torch.float32).pin_memory()
+        h2d = Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size() + \
+            th.numel() * 4 + Bh[0].numel() * Bh[0].element_size()
+        sets = [(self.Xd, self.Yd, self.td, torch.empty_like(self.Bs[0])),
+                (torch.empty_like(self.Xd), torch.empty_like(self.Yd),
+                 torch.empty_like(self.td), torch.empty_like(self.Bs[0]))]
+        cstream = torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event() for _ in range(2)]
+        consumed = [torch.cuda.Event() for _ in range(2)]
+
+        def issue_copy(s, j):
+            k = s % 2
+            with torch.cuda.stream(cstream):
+                if j >= 2:  # the set's previous step has finished with it
+                    cstream.wait_event(consumed[k])
+                for dst, src in zip(sets[k], (Xh, Yh, th, Bh[s])):
+                    dst.copy_(src, non_blocking=True)
+                copied[k].record(cstream)
+
+        def run(first, count):
+            torch.cuda.synchronize(dev)
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(cstream)
+            issue_copy(first, 0)
+            for j in range(count):
+                s = first + j
+                if j + 1 < count:
+                    issue_copy(s + 1, j + 1)
+                k = s % 2
+                stream.wait_event(copied[k])
+                self.flush.zero_()
+                Xc, Yc, tc, Bc = sets[k]
+                self.step(Bc, Xc, Yc, tc)
+                consumed[k].record(stream)
+                loss_h[s].copy_(self.loss[0], non_blocking=True)
+            t1.record(stream)
+            t1.synchronize()
+            return t0.elapsed_time(t1)
+
+        run(0, warmup)
+        barrier()
+        ms = run(warmup, steps)
+        assert np.all(np.isfinite(loss_h.numpy())), "non-finite loss"
+        del sets
+        return ms, int(h2d), 4
+
+
+def extra_workload(torch, name, args, dev):
+    """Another workload measured in the same process (one GPU): ms per step, rows/s, the
+    dominant stage's roofline, every stage's fraction and peak HBM against full CE."""
+    from reduced_cross_entropy_b200 import ops, synth
+    w = synth.WORKLOADS[name]
+    run = WorkloadRun(torch, w, 0, dev, args.flags, args.warmup + args.steps, False)
+    run.warm(args.warmup)
+    step_ms, stage_ms, launches, _ = run.timed(args.warmup, args.steps)
+    ms = sum(step_ms) / args.steps
+    roof, fracs = run.rooflines(stage_ms)
+    out = {"config": run.describe(), "ms_per_step": ms, "value": w.N / (ms / 1000.0),
+           "unit": "rows/s", "steps": args.steps, "warmup": args.warmup,
+           "roofline": roof, "path_roofline": run.path_roofline(ms), "stages_ms": stage_ms,
+           "stages_roofline_frac": fracs, "gpu_launches": int(launches)}
+    if not args.no_memory:
+        out["peak_hbm"] = measure_memory(torch, ops, run.plan, w, run.Xd, run.Yd, run.td,
+                                         run.Bs[0], dev)
+    del run
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -367,213 +656,45 @@ def main():
             dist.barrier()
 
     exchange = world > 1 and not args.no_allreduce_dy
-
-    L = _lib.lib()
     w = synth.WORKLOADS[args.workload]
-    X, Y, t = synth.make_inputs(w, seed=rank)
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype,
-                    flags=args.flags)
-    Xd = torch.from_numpy(X).to(dev).to(tdt)
-    Yd = torch.from_numpy(Y).to(dev).to(tdt)
-    td = torch.from_numpy(t).to(dev)
-    n_steps = args.warmup + args.steps
-    Bs = [torch.from_numpy(synth.projections(0, s, w.n_r, w.n_b, w.d, w.dtype)).to(dev).to(tdt)
-          for s in range(n_steps)]
-    ws = plan.workspace(dev)
-    loss = torch.empty(1, dtype=torch.float32, device=dev)
-    sel = torch.empty(w.N, w.k, dtype=torch.int32, device=dev)
-    lse = torch.empty(w.N, dtype=torch.float32, device=dev)
-    logits = torch.empty(w.N, w.k + 1, dtype=torch.float32, device=dev)
-    dloss = torch.ones(1, dtype=torch.float32, device=dev)
-    dX = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
-    dY = torch.empty(w.C, w.d, dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    vp = lambda x: ctypes.c_void_p(x.data_ptr())  # noqa: E731
-    nbytes = ctypes.c_size_t(ws.numel())
-
-    def step(Bt, Xc=None, Yc=None, tc=None):
-        Xc = Xd if Xc is None else Xc
-        Yc = Yd if Yc is None else Yc
-        tc = td if tc is None else tc
-        _lib.check(L.rece_bucketize_sort(plan._h, vp(Bt), vp(Xc), vp(Yc), vp(ws), nbytes, sp),
-                   "bucketize_sort")
-        _lib.check(L.rece_loss_fwd(plan._h, vp(Xc), vp(Yc), vp(tc), vp(ws), nbytes, vp(loss),
-                                   None, vp(sel), vp(lse), vp(logits), sp), "loss_fwd")
-        _lib.check(L.rece_loss_bwd(plan._h, vp(Xc), vp(Yc), vp(tc), vp(sel), vp(lse),
-                                   vp(logits), vp(dloss), vp(ws), nbytes, vp(dX), vp(dY), sp),
-                   "loss_bwd")
-        if exchange:
-            allreduce_dy(dY)
-
-    for s in range(args.warmup):
-        flush.zero_()
-        step(Bs[s])
-    torch.cuda.synchronize(dev)
-    # status area: flags (a bad target or a timed-out wait fails the run; the tensor-core
-    # selection may flag rows it cannot certify exact) and the count of such rows
-    status_words = ws[:16].view(torch.int32).cpu().tolist()
-    assert status_words[0] & ~_lib.DEVICE_INEXACT == 0, f"device status {status_words[0]:#x}"
-    inexact_rows, overflow_rows = int(status_words[1]), int(status_words[2])
-    spilled_rows = int(status_words[3])
-
-    # timed region: K steps, each bracketed by events; per-stage events recorded by the
-    # library on the same stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    n_st = len(_lib.STAGES)
-    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_st)]
-           for _ in range(args.steps)]
-    for row in sev:  # torch creates the CUDA event at its first record
-        for e in row:
-            e.record(stream)
-    sev_h = [(ctypes.c_void_p * (2 * n_st))(*[ctypes.c_void_p(e.cuda_event) for e in row])
-             for row in sev]
-    launches0 = L.rece_kernel_launch_count()
-    barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clk:
-        for s in range(args.steps):
-            flush.zero_()
-            _lib.check(L.rece_plan_set_stage_events(plan._h, sev_h[s]), "stage events")
-            ev[s][0].record(stream)
-            step(Bs[args.warmup + s])
-            ev[s][1].record(stream)
-        torch.cuda.synchronize(dev)
-    barrier()
-    launches = L.rece_kernel_launch_count() - launches0
-    L.rece_plan_set_stage_events(plan._h, None)
-    step_ms = [a.elapsed_time(b) for a, b in ev]
+    run = WorkloadRun(torch, w, rank, dev, args.flags, args.warmup + args.steps, exchange)
+    run.warm(args.warmup)
+    step_ms, stage_ms, launches, clocks = run.timed(args.warmup, args.steps, barrier,
+                                                    clock_index=local_rank)
     total_ms = max_over_ranks(sum(step_ms), dev)
-    stage_ms = {name: statistics.mean(sev[s][2 * i].elapsed_time(sev[s][2 * i + 1])
-                                      for s in range(args.steps))
-                for i, name in enumerate(_lib.STAGES)}
     value = job_throughput(world, w.N, args.steps, total_ms)
-
-    # roofline of every stage, the dominant one reported as the line's roofline
-    peaks = load_peaks()
-    paths = plan.paths
-    work = stage_work(w, paths)
-
-    def stage_roofline(name):
-        bound = stage_bound(name, paths)
-        flops, bytes_ = work[name]
-        sec = max(stage_ms[name], 1e-9) / 1000.0
-        if bound == "hbm":
-            achieved, peak, unit = bytes_ / sec / 1e9, peaks["hbm_gbs"], "GB/s"
-        elif bound == "tensor":
-            achieved, peak, unit = flops / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        else:  # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flop x max SM clock
-            achieved, peak, unit = (flops / sec / 1e12,
-                                    148 * 128 * 2 * peaks["sm_max_mhz"] / 1e6, "TFLOP/s")
-        return {"bound": bound, "kernel": name, "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak,
-                "peak_source": peaks["source"] if bound != "alu" else
-                "derived: 148 SM x 128 FP32 lanes x 2 x sm_max_mhz",
-                "traffic": recorded_traffic(name, w.name, paths),
-                "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
-
-    dom = max(stage_ms, key=stage_ms.get)
-    roofline = stage_roofline(dom)
-    stage_fracs = {name: round(stage_roofline(name)["frac"], 4) for name in stage_ms}
-
-    # end to end: every step's inputs copied in from pinned host memory and its loss
-    # copied out, through the same C-ABI calls.  Step s+1's copies (a copy stream, two
-    # device input sets) overlap step s's compute, as a training input pipeline does; the
-    # L2 flush stays in the timeline; one pair of events spans all timed steps.
-    Xh = torch.from_numpy(X).to(tdt).pin_memory()
-    Yh = torch.from_numpy(Y).to(tdt).pin_memory()
-    th = torch.from_numpy(t).pin_memory()
-    Bh = [b.cpu().pin_memory() for b in Bs]
-    loss_h = torch.empty(n_steps, dtype=torch.float32).pin_memory()
-    h2d = Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size() + th.numel() * 4 \
-        + Bh[0].numel() * Bh[0].element_size()
-    sets = [(Xd, Yd, td, torch.empty_like(Bs[0])),
-            (torch.empty_like(Xd), torch.empty_like(Yd), torch.empty_like(td),
-             torch.empty_like(Bs[0]))]
-    cstream = torch.cuda.Stream(dev)
-    copied = [torch.cuda.Event() for _ in range(2)]
-    consumed = [torch.cuda.Event() for _ in range(2)]
-
-    def issue_copy(s, j):
-        k = s % 2
-        with torch.cuda.stream(cstream):
-            if j >= 2:  # the set's previous step has finished with it
-                cstream.wait_event(consumed[k])
-            for dst, src in zip(sets[k], (Xh, Yh, th, Bh[s])):
-                dst.copy_(src, non_blocking=True)
-            copied[k].record(cstream)
-
-    def e2e_run(first, count):
-        torch.cuda.synchronize(dev)
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(cstream)
-        issue_copy(first, 0)
-        for j in range(count):
-            s = first + j
-            if j + 1 < count:
-                issue_copy(s + 1, j + 1)
-            k = s % 2
-            stream.wait_event(copied[k])
-            flush.zero_()
-            Xc, Yc, tc, Bc = sets[k]
-            step(Bc, Xc, Yc, tc)
-            consumed[k].record(stream)
-            loss_h[s].copy_(loss[0], non_blocking=True)
-        t1.record(stream)
-        t1.synchronize()
-        return t0.elapsed_time(t1)
-
-    e2e_run(0, args.warmup)
-    barrier()
-    e2e_ms = [e2e_run(args.warmup, args.steps)]
-    assert np.all(np.isfinite(loss_h.numpy())), "non-finite loss"
-    e2e_total = max_over_ranks(sum(e2e_ms), dev)
+    roofline, stage_fracs = run.rooflines(stage_ms)
+    e2e_ms, h2d, d2h = run.e2e(args.warmup, args.steps, barrier)
+    e2e_total = max_over_ranks(e2e_ms, dev)
     e2e = {"value": job_throughput(world, w.N, args.steps, e2e_total), "unit": "rows/s",
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4}
-
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    paths = run.paths
+    config = run.describe()
+    config.update({"parallelism": f"dp{world}",
+                   "exchange": ("all-reduce of dY [C x d] fp32 every step (NCCL)"
+                                if exchange else "none")})
     line = {"metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": workload_desc(w), "inexact_rows_per_step": inexact_rows,
-                       "overflowed_rows_per_step": overflow_rows,
-                       "merge_spilled_rows_per_step": spilled_rows,
-                       "l2": "flushed between timed steps (256 MiB write)",
-                       "parallelism": f"dp{world}",
-                       "exchange": ("all-reduce of dY [C x d] fp32 every step (NCCL)"
-                                    if exchange else "none"),
-                       "scores": ("tcgen05" + (", stored" if paths & _lib.PATH_STORED_SCORES
-                                                 else ", recomputed per pass")
-                                  if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),
-                       "dX": ("tcgen05 band products" +
-                              (", rounds in one launch, parts summed in order"
-                               if paths & _lib.PATH_DX_PARTS else "")
-                              if paths & _lib.PATH_DX_TENSORS else "gathered rows"),
-                       "negatives": ("every window item (Algorithm 1 as printed), window "
-                                     "sums and gradients on tcgen05"
-                                     if paths & _lib.PATH_ALL_NEGATIVES
-                                     else f"top-{w.k} per row")},
-            "roofline": roofline, "stages_ms": stage_ms, "stages_roofline_frac": stage_fracs,
-            "e2e": e2e, "gpu_launches": int(launches),
-            "clocks": clk.summary()}
+            "config": config, "roofline": roofline,
+            "path_roofline": run.path_roofline(total_ms / args.steps),
+            "stages_ms": stage_ms, "stages_roofline_frac": stage_fracs,
+            "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks}
 
     if rank == 0 and world == 1 and not args.no_memory:
-        line["peak_hbm"] = measure_memory(torch, ops, plan, w, Xd, Yd, td, Bs[0], dev)
+        line["peak_hbm"] = measure_memory(torch, ops, run.plan, w, run.Xd, run.Yd, run.td,
+                                          run.Bs[0], dev)
     if rank == 0 and world == 1 and not args.no_baselines:
-        line["baselines"] = measure_baselines(torch, ops, w, Xd, Yd, td, flush, dev,
-                                              load_peaks())
+        line["baselines"] = measure_baselines(torch, ops, w, run.Xd, run.Yd, run.td, run.flush,
+                                              dev, load_peaks())
+    del run
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and args.also:
+        line["workloads"] = {name: extra_workload(torch, name, args, dev)
+                             for name in args.also.split(",") if name and name != w.name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        rows, frac = 256, 16
-        secs = oracle_step_seconds(w, X, Y, t, synth.projections(0, 0, w.n_r, w.n_b, w.d,
-                                                                   w.dtype), rows, frac,
-                                   all_negatives=bool(paths & _lib.PATH_ALL_NEGATIVES))
-        line["cpu_baseline"] = {"value": w.N / secs, "unit": "rows/s",
-                                "cores": oracle.num_threads(), "kind": "oracle",
-                                "sample": oracle_sample_desc(rows, frac)}
+        line["cpu_baseline"] = cpu_baseline(w, 0, bool(paths & _lib.PATH_ALL_NEGATIVES))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -669,6 +790,14 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
     out["pages_memory_model"] = {"alpha_bc": a, "n_b_star": nb, "n_c_star": nc,
                                  "logit_elements": el, "bytes_fp32": 4 * el,
                                  "rece_bytes_over_model": out["rece_bytes"] / (4 * el)}
+    # the plan the library makes when asked for the pages' optimum (n_b = n_c = 0:
+    # n_b* at alpha_bc = 1) and its workspace, against the model at alpha_bc = 1
+    auto = ops.Plan(w.N, w.C, w.d, 0, 0, w.n_ec, w.n_r, w.k, mode=w.dtype,
+                    flags=plan.cfg.flags)
+    el1 = ops.memory_model_elements(w.N, w.C, w.n_ec, w.n_r, 1.0)
+    out["pages_memory_model"]["auto_plan"] = {
+        "n_b": auto.n_b, "n_c": auto.n_c, "workspace_bytes": auto.workspace_bytes,
+        "model_bytes_fp32": 4 * el1, "workspace_over_model": auto.workspace_bytes / (4 * el1)}
     out["note"] = "bytes above the resident inputs; torch.cuda.max_memory_allocated"
     return out
 

@@ -96,8 +96,9 @@ typedef struct {
   int64_t N;     /* rows (batch x sequence), >= 0 */
   int64_t C;     /* catalogue size, >= 1 */
   int32_t d;     /* embedding width, >= 1 (bf16 mode: multiple of 16 for tcgen05) */
-  int32_t n_b;   /* random vectors per round, 1 .. 4096 */
-  int32_t n_c;   /* chunks, 1 .. min(N, C) (any n_c <= C when N = 0) */
+  int32_t n_b;   /* random vectors per round, 1 .. 4096; 0 together with n_c = 0: the
+                    pages' n_b* at alpha_bc = 1 (see rece_plan_create) */
+  int32_t n_c;   /* chunks, 1 .. min(N, C) (any n_c <= C when N = 0); 0 with n_b = 0 */
   int32_t n_ec;  /* neighbouring chunks on each side, >= 0 */
   int32_t n_r;   /* rounds, 1 .. 8 */
   int32_t k;     /* negatives kept per row, 1 .. 4096 */
@@ -123,9 +124,18 @@ typedef struct {
 
 /* Validate cfg and build a host-side plan (no CUDA call, no device memory).
  * cfg, plan: host pointers.  On success *plan owns a host object freed by
- * rece_plan_destroy.  RECE_ERR_INVALID_ARG / RECE_ERR_UNSUPPORTED on a bad config. */
+ * rece_plan_destroy.  RECE_ERR_INVALID_ARG / RECE_ERR_UNSUPPORTED on a bad config.
+ * n_b = n_c = 0 asks for the bucket count the RECE paper calls optimal for peak memory
+ * [RECE section 3, the paragraph before Algorithm 1]: n_b* at alpha_bc = n_b / n_c = 1
+ * (section 5: n_c = n_b gave the best quality for a memory budget), i.e. n_b = n_c =
+ * rece_optimal_buckets(N, C, n_ec, 1.0) (1 when N = 0); only one of them 0 is
+ * RECE_ERR_INVALID_ARG.  rece_plan_get_config returns the values chosen. */
 RECE_API rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* plan);
 RECE_API void rece_plan_destroy(rece_plan_t plan);
+
+/* The plan's configuration as resolved by rece_plan_create (n_b and n_c filled in when
+ * they were 0).  cfg: host pointer.  RECE_ERR_INVALID_ARG for a NULL argument. */
+RECE_API rece_status_t rece_plan_get_config(rece_plan_t plan, rece_config_t* cfg);
 
 /* Device workspace bytes the plan needs (one buffer, caller-allocated, 256-byte
  * aligned).  The same buffer serves rece_bucketize_sort, rece_loss_fwd and
@@ -274,7 +284,9 @@ RECE_API rece_status_t rece_sampled_bwd(int32_t kind, int64_t N, int64_t C, int3
  * synchronisation.  Its scratch (per-tile histograms) is a 4 MiB array of device memory
  * inside the library image; every GPU the library is used on holds it until the process
  * exits.
- *   bucket_ids   device int32 [M], values in [0, n_b) (others sort by their low bits)
+ *   bucket_ids   device int32 [M], values in [0, n_b); any other value, negative ones
+ *                included, is sorted by its low ceil(log2 n_b) bits (two's complement),
+ *                i.e. as the key (value & (2^ceil(log2 n_b) - 1)), stably
  *   order        device int32 [M]: element indices by (bucket asc, index asc)
  *   bucket_start device int32 [2^ceil(log2 n_b) + 1] or NULL: first position of every
  *                bucket id (entries from n_b on hold M)
@@ -282,8 +294,11 @@ RECE_API rece_status_t rece_sampled_bwd(int32_t kind, int64_t N, int64_t C, int3
  * histograms of M elements by 2^ceil(log2 n_b) buckets do not fit the 4 MiB (about
  * M * 2^ceil(log2 n_b) <= 2^31: M <= 520,192 at n_b = 4096, M <= 8,384,512 at n_b = 256).
  * The first call on a device looks up the array's device address (make that first call
- * before any stream capture).  All calls share the array: calls whose GPU work can
- * overlap (unordered streams or threads) race; order them. */
+ * before any stream capture) and keeps it for the rest of the process: after
+ * cudaDeviceReset (or anything else that tears the device's primary context down) the kept
+ * address is stale, so do not call this function again in that process.  All calls share
+ * the array: calls whose GPU work can overlap (unordered streams or threads) race; order
+ * them. */
 RECE_API rece_status_t rece_bucket_sort_static(const int32_t* bucket_ids, int64_t M,
                                                int32_t n_b, int32_t* order,
                                                int32_t* bucket_start, void* stream);

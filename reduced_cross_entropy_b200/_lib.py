@@ -35,7 +35,7 @@ EXPORTS = (
     "rece_get_device_status", "rece_status_string", "rece_last_error_string",
     "rece_plan_set_stage_events", "rece_kernel_launch_count", "rece_bucket_sort_static",
     "rece_plan_paths", "rece_sampled_workspace_size", "rece_sampled_fwd", "rece_sampled_bwd",
-    "rece_optimal_buckets", "rece_memory_model_elements",
+    "rece_optimal_buckets", "rece_memory_model_elements", "rece_plan_get_config",
 )
 SAMPLED_CE_MINUS = 0  # RECE section 2, equation (2)
 SAMPLED_BCE_PLUS = 1  # RECE section 2, equation (1)
@@ -82,6 +82,7 @@ def lib():
         "rece_plan_create": ([ctypes.POINTER(Config), ctypes.POINTER(vp)], st),
         "rece_plan_destroy": ([vp], None),
         "rece_plan_workspace_size": ([vp, ctypes.POINTER(sz)], st),
+        "rece_plan_get_config": ([vp, ctypes.POINTER(Config)], st),
         "rece_plan_workspace_layout": ([vp, ctypes.POINTER(WorkspaceLayout)], st),
         "rece_plan_paths": ([vp, ctypes.POINTER(ctypes.c_uint32)], st),
         "rece_bucketize_sort": ([vp, vp, vp, vp, vp, sz, vp], st),

@@ -357,7 +357,22 @@ const char* rece_last_error_string(void) { return g_last_error; }
 rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   if (!cfg || !out) return fail(RECE_ERR_INVALID_ARG, "cfg or plan pointer is NULL");
   *out = nullptr;
-  const rece_config_t& c = *cfg;
+  rece_config_t c = *cfg;
+  if (c.n_b == 0 || c.n_c == 0) {
+    // n_b = n_c = 0: the bucket count the RECE paper calls optimal for peak memory,
+    // n_b* = sqrt(4 alpha_bc (1 + 2 n_ec) min(C, N)), at alpha_bc = 1 (n_c = n_b, the
+    // ratio its experiments found best), as rece_optimal_buckets rounds and clamps it
+    if (c.n_b != 0 || c.n_c != 0)
+      return fail(RECE_ERR_INVALID_ARG,
+                  "n_b and n_c must both be 0 (the pages' n_b* at alpha_bc = 1) or both >= 1");
+    if (c.N >= 0 && c.C >= 1 && c.n_ec >= 0) {
+      int32_t nb = 1, nc = 1;
+      if (c.N > 0 && rece_optimal_buckets(c.N, c.C, c.n_ec, 1.0, &nb, &nc) != RECE_OK)
+        return RECE_ERR_INVALID_ARG;
+      c.n_b = nb;
+      c.n_c = nc;
+    }
+  }
   if (c.N < 0 || c.C < 1 || c.C >= kInt32Max) return fail(RECE_ERR_INVALID_ARG, "N or C out of range");
   if (c.d < 1) return fail(RECE_ERR_INVALID_ARG, "d must be >= 1");
   if (c.n_b < 1 || c.n_b > (1 << kMaxDigitBits))
@@ -499,6 +514,12 @@ rece_status_t rece_plan_set_stage_events(rece_plan_t plan, void* const* events) 
 }
 
 uint64_t rece_kernel_launch_count(void) { return g_launches.load(); }
+
+rece_status_t rece_plan_get_config(rece_plan_t plan, rece_config_t* cfg) {
+  if (!plan || !cfg) return fail(RECE_ERR_INVALID_ARG, "NULL argument");
+  *cfg = plan->cfg;
+  return RECE_OK;
+}
 
 rece_status_t rece_plan_workspace_size(rece_plan_t plan, size_t* bytes) {
   if (!plan || !bytes) return fail(RECE_ERR_INVALID_ARG, "NULL argument");

@@ -41,15 +41,19 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_hist(const __grid_constan
   for (int i = threadIdx.x; i < digits; i += blockDim.x) sh_cnt[i] = 0;
   __syncthreads();
   const int64_t base = int64_t(blockIdx.x) * kSortTile;
+  // an element counts when it lies inside the segment (p < M), whatever its key: the
+  // scatter ranks exactly those elements by the same digit expression, so a key outside
+  // [0, 2^bits) -- a negative one included -- is sorted by its low bits on both sides
   int32_t kv[kSortTile / kSortThreads];
 #pragma unroll
   for (int u = 0; u < kSortTile / kSortThreads; ++u) {
     const int64_t p = base + u * kSortThreads + threadIdx.x;
-    kv[u] = p < g.M ? elem_key(g.keys, g.in_ids, p, b.in_order) : -1;
+    kv[u] = p < g.M ? elem_key(g.keys, g.in_ids, p, b.in_order) : 0;
   }
 #pragma unroll
   for (int u = 0; u < kSortTile / kSortThreads; ++u)
-    if (kv[u] >= 0) atomicAdd(&sh_cnt[(kv[u] >> shift) & mask], 1);
+    if (base + u * kSortThreads + threadIdx.x < g.M)
+      atomicAdd(&sh_cnt[(kv[u] >> shift) & mask], 1);
   __syncthreads();
   for (int i = threadIdx.x; i < digits; i += blockDim.x)
     g.hist[int64_t(i) * g.tiles + blockIdx.x] = sh_cnt[i];

@@ -52,6 +52,8 @@ class Plan:
         _lib.check(L.rece_plan_create(ctypes.byref(self.cfg), ctypes.byref(h)),
                    "rece_plan_create")
         self._h = h
+        # the configuration as the library resolved it (n_b = n_c = 0: the pages' n_b*)
+        _lib.check(L.rece_plan_get_config(h, ctypes.byref(self.cfg)), "rece_plan_get_config")
         size = ctypes.c_size_t()
         _lib.check(L.rece_plan_workspace_size(h, ctypes.byref(size)), "workspace_size")
         self.workspace_bytes = int(size.value)

@@ -22,10 +22,14 @@ def max_rel(a, b):
     return float(np.max(np.abs(a - b)) / den)
 
 
-def run_gpu(w: synth.Workload, X, Y, t, B, flags=0, dloss=1.0, use_logits=True):
-    """Whole path on the GPU.  Returns a dict of numpy arrays."""
-    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype,
-                    flags=flags)
+def run_gpu(w: synth.Workload, X, Y, t, B, flags=0, dloss=1.0, use_logits=True,
+            auto_buckets=False):
+    """Whole path on the GPU.  Returns a dict of numpy arrays.  auto_buckets: the plan is
+    created with n_b = n_c = 0 (the library picks the pages' n_b*), which must resolve to
+    w's n_b and n_c."""
+    plan = ops.Plan(w.N, w.C, w.d, 0 if auto_buckets else w.n_b, 0 if auto_buckets else w.n_c,
+                    w.n_ec, w.n_r, w.k, mode=w.dtype, flags=flags)
+    assert (plan.n_b, plan.n_c) == (w.n_b, w.n_c)
     Xd, Yd, Bd = to_dev(X, w.dtype), to_dev(Y, w.dtype), to_dev(B, w.dtype)
     td = torch.from_numpy(t).cuda()
     ws = plan.workspace()

@@ -55,6 +55,7 @@ def create(c):
 @pytest.mark.parametrize("bad", [
     dict(N=-1), dict(C=0), dict(d=0), dict(n_b=0), dict(n_b=4097), dict(n_r=0), dict(n_r=9),
     dict(k=0), dict(k=4097), dict(n_ec=-1), dict(n_c=0), dict(n_c=257), dict(C=100, n_c=101),
+    dict(n_b=0, n_c=0, N=-1), dict(n_b=0, n_c=0, C=0), dict(n_b=0, n_c=0, n_ec=-1),
     dict(mode=2), dict(flags=0x80),
 ])
 def test_invalid_configs_rejected(bad):
@@ -208,3 +209,34 @@ def test_all_negatives_mode_support():
         with pytest.raises(RuntimeError):
             Plan(kw["N"], kw["C"], kw["d"], kw["n_b"], kw["n_c"], kw["n_ec"], kw["n_r"],
                  kw["k"], mode=kw["mode"], flags=flags)
+
+
+@pytest.mark.parametrize("N,C,n_ec", [(256, 4096, 1), (25_600, 100_000, 1),
+                                      (65_536, 4_000_000, 2), (3, 100, 0), (0, 50, 1),
+                                      (10**6, 2 * 10**6, 8)])
+def test_zero_buckets_and_chunks_mean_the_pages_optimum(N, C, n_ec):
+    """n_b = n_c = 0: n_b* = sqrt(4 alpha_bc (1 + 2 n_ec) min(C, N)) at alpha_bc = 1, rounded
+    to the nearest integer, n_b held to [1, 4096] and n_c = n_b to [1, min(N, C)] (RECE
+    section 3, the paragraph before Algorithm 1; section 5 for alpha_bc = 1)."""
+    import math
+    p = Plan(N, C, 64, 0, 0, n_ec, 1, 8, mode="fp32")
+    m = min(N, C)
+    want = min(max(int(math.floor(math.sqrt(4 * (1 + 2 * n_ec) * m) + 0.5)), 1), 4096)
+    want_c = min(max(want, 1), max(m, 1))
+    assert (p.n_b, p.n_c) == (want, want_c)
+    assert (p.N, p.C, p.n_ec) == (N, C, n_ec)
+    # the same numbers as the helper the library exports
+    nb, nc = ctypes.c_int32(), ctypes.c_int32()
+    if N > 0:
+        assert _lib.lib().rece_optimal_buckets(N, C, n_ec, 1.0, ctypes.byref(nb),
+                                               ctypes.byref(nc)) == 0
+        assert (nb.value, nc.value) == (p.n_b, p.n_c)
+    # an explicit plan with those numbers is the same plan
+    q = Plan(N, C, 64, p.n_b, p.n_c, n_ec, 1, 8, mode="fp32")
+    assert q.workspace_bytes == p.workspace_bytes
+
+
+def test_zero_buckets_needs_zero_chunks_too():
+    assert create(cfg(n_b=0, n_c=8)) == 1
+    assert create(cfg(n_b=16, n_c=0)) == 1
+    assert b"both" in _lib.lib().rece_last_error_string()

@@ -63,6 +63,35 @@ def test_parity_fma_path(name):
             run_oracle(w, X, Y, t, B, dloss=0.75))
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_auto_bucket_plan_matches_oracle(dtype):
+    """n_b = n_c = 0: the library takes the pages' n_b* at alpha_bc = 1 (RECE section 3,
+    the paragraph before Algorithm 1): sqrt(4 * 3 * 600) = 84.9 -> n_b = n_c = 85 here; the
+    path through that plan equals the oracle run at those values."""
+    w = synth.Workload("auto", N=600, C=5000, d=64, dtype=dtype, n_b=85, n_c=85, n_ec=1,
+                       n_r=2, k=40)
+    X, Y, t = synth.make_inputs(w, seed=5)
+    B = synth.projections(5, 0, w.n_r, w.n_b, w.d, w.dtype)
+    g = run_gpu(w, X, Y, t, B, flags=1 if dtype == "bf16" else 0, auto_buckets=True)
+    compare(w, g, run_oracle(w, X, Y, t, B))
+    if dtype == "bf16":  # and on the tensor cores (tcgen05 sums: loss within 1e-2)
+        o = run_oracle(w, X, Y, t, B)
+        g = run_gpu(w, X, Y, t, B, auto_buckets=True)
+        assert g["status"] & ~0x4 == 0
+        assert abs(g["loss"] - o["loss"]) <= 1e-2 * abs(o["loss"])
+
+
+def test_fp32_exact_whole_arrays_at_sasrec_scale():
+    """The fp32 exact mode at the SASRec-scale benchmark shape (N = 25,600, C = 100,000,
+    n_b = 256, n_c = 64, n_ec = 1, n_r = 2, k = 256), the whole arrays against the whole
+    oracle: bucket ids, orders and selected sets bit for bit, losses and gradients
+    within 1e-4."""
+    w = W["sasrec"].scaled(25_600, 100_000, dtype="fp32")
+    X, Y, t = synth.make_inputs(w, seed=0)
+    B = synth.projections(0, 0, w.n_r, w.n_b, w.d, w.dtype)
+    compare(w, run_gpu(w, X, Y, t, B), run_oracle(w, X, Y, t, B))
+
+
 def test_parity_ties_on_exact_inputs():
     """Integer-valued inputs: every score is exact and ties are everywhere, so the
     lowest-index tie rules of argmax, sort and selection are all exercised."""

@@ -67,13 +67,19 @@ def test_full_size_sampled_parity(name):
     if len(untouched):
         items.append(int(untouched[len(untouched) // 2]))
 
-    # step 1: bucket ids of the sampled rows and items, against the oracle's argmax
+    # step 1: bucket ids of a sample of rows and items (8192 of each, the checked rows and
+    # items among them) against the oracle's argmax: a differing id must be a near-tie,
+    # and at most 1e-3 of them may differ
+    many_rows = np.union1d(rows, rng.choice(w.N, min(w.N, 8192), replace=False))
+    many_items = np.union1d(items, rng.choice(w.C, min(w.C, 8192), replace=False))
     for r in range(w.n_r):
-        for V, ids, got in ((X, rows, bx[r]), (Y, np.array(items), by[r])):
+        for V, ids, got in ((X, many_rows, bx[r]), (Y, many_items, by[r])):
             want = oracle.bucketize(V[ids], B[r])
-            P = V[ids].astype(np.float64) @ B[r].astype(np.float64).T
-            for a in np.nonzero(got[ids] != want)[0]:
-                assert abs(P[a, got[ids[a]]] - P[a, want[a]]) <= 1e-5 * np.abs(P[a]).max()
+            diff = np.nonzero(got[ids] != want)[0]
+            assert len(diff) <= 1e-3 * len(ids), (len(diff), len(ids))
+            P = V[ids[diff]].astype(np.float64) @ B[r].astype(np.float64).T
+            for a, j in enumerate(diff):
+                assert abs(P[a, got[ids[j]]] - P[a, want[j]]) <= 1e-5 * np.abs(P[a]).max()
     # step 2: the orders are the stable argsort of the GPU's bucket ids (whole arrays)
     for r in range(w.n_r):
         np.testing.assert_array_equal(px[r], oracle.stable_argsort(bx[r]))

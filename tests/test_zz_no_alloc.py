@@ -71,3 +71,28 @@ def test_static_sort_rejects_sizes_beyond_its_scratch():
     assert s == 0
     torch.cuda.synchronize()
     assert torch.equal(order, torch.arange(16, dtype=torch.int32, device="cuda"))
+
+
+@pytest.mark.parametrize("M,n_b", [(5000, 300), (2048 * 3 + 17, 4096), (1, 1), (777, 2)])
+def test_static_sort_out_of_range_keys_sort_by_their_low_bits(M, n_b):
+    # hand-made keys: in range, at and above n_b, and negative; M off the 2048-element tile
+    rng = np.random.Generator(np.random.PCG64(M + n_b))
+    keys = rng.integers(-3 * n_b - 5, 3 * n_b + 5, size=M).astype(np.int32)
+    keys[: min(M, 4)] = np.array([-1, n_b, -2147483648, 2147483647][: min(M, 4)], np.int32)
+    bits = max(int(np.ceil(np.log2(n_b))), 0) if n_b > 1 else 0
+    digit = (keys.astype(np.int64) & ((1 << bits) - 1)).astype(np.int64)
+    want = np.argsort(digit, kind="stable").astype(np.int32)
+    stride = (1 << bits) + 1
+    want_starts = np.searchsorted(digit[want], np.arange(stride), side="left").astype(np.int32)
+
+    L = _lib.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    kd = torch.from_numpy(keys).cuda()
+    for _ in range(2):  # twice in a row: the shared scratch keeps the first call's contents
+        order = torch.full((M,), -1, dtype=torch.int32, device="cuda")
+        starts = torch.full((stride,), -7, dtype=torch.int32, device="cuda")
+        s = L.rece_bucket_sort_static(_vp(kd), M, n_b, _vp(order), _vp(starts), stream)
+        assert s == 0, L.rece_last_error_string()
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(order.cpu().numpy(), want)
+        np.testing.assert_array_equal(starts.cpu().numpy(), want_starts)
