@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip timing the sampled CE- / BCE+ comparison ops")
     ap.add_argument("--flags", type=int, default=0, help="rece_config_t.flags")
+    ap.add_argument("--slice", type=int, default=1,
+                    help="run a proportional 1/F slice of the workload (N, C and n_c divided "
+                         "by F: the same chunks and windows), e.g. for profiler captures")
     return ap.parse_args()
 
 
@@ -458,11 +461,15 @@ class WorkloadRun:
         self.torch.cuda.synchronize(self.dev)
         # status area: flags (a bad target or a timed-out wait fails the run; the
         # tensor-core selection may flag rows it cannot certify exact) and row counts
-        words = self.ws[:16].view(self.torch.int32).cpu().tolist()
+        words = self.ws[:32].view(self.torch.int32).cpu().tolist()
         assert words[0] & ~self._lib.DEVICE_INEXACT == 0, f"device status {words[0]:#x}"
         self.status_words = {"inexact_rows_per_step": int(words[1]),
                              "overflowed_rows_per_step": int(words[2]),
                              "merge_spilled_rows_per_step": int(words[3])}
+        if self.paths & self._lib.PATH_SAMPLED_SELECT:
+            # work items (128 rows of a round) the sampled selection could not certify
+            # and handed to the exact kernel
+            self.status_words["select_redo_items_per_step"] = int(words[4])
 
     def timed(self, first, steps, barrier=lambda: None, clock_index=None):
         """`steps` steps from B number `first`, L2 flushed before each; per-step and
@@ -540,7 +547,9 @@ class WorkloadRun:
         return {"workload": workload_desc(w), **self.status_words,
                 "l2": "flushed between timed steps (256 MiB write)",
                 "scores": ("tcgen05" + (", stored" if paths & _lib.PATH_STORED_SCORES
-                                          else ", recomputed per pass")
+                                          else ", threshold from a 1/8 sample, one pass"
+                                          if paths & _lib.PATH_SAMPLED_SELECT
+                                          else ", exact threshold, three passes")
                            if paths & _lib.PATH_TENSOR_CORES else "fmaf CUDA cores"),
                 "dX": ("tcgen05 band products" +
                        (", rounds in one launch, parts summed in order"
@@ -657,6 +666,11 @@ def main():
 
     exchange = world > 1 and not args.no_allreduce_dy
     w = synth.WORKLOADS[args.workload]
+    if args.slice > 1:
+        f = args.slice
+        if w.N % f or w.C % f or w.n_c % f:
+            raise SystemExit(f"--slice {f} must divide N, C and n_c of {w.name}")
+        w = w.scaled(w.N // f, w.C // f, n_c=w.n_c // f)
     run = WorkloadRun(torch, w, rank, dev, args.flags, args.warmup + args.steps, exchange)
     run.warm(args.warmup)
     step_ms, stage_ms, launches, clocks = run.timed(args.warmup, args.steps, barrier,

@@ -156,7 +156,11 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
  *   RECE_PATH_DX_PARTS      (with RECE_PATH_DX_TENSORS) the dX band products of all rounds
  *                           in one launch, each row tile's window split in parts that are
  *                           stored and then summed in a fixed order (when per-round
- *                           launches would leave their last wave part-empty).
+ *                           launches would leave their last wave part-empty);
+ *   RECE_PATH_SAMPLED_SELECT the fused selection sets each row's threshold from a 1/8
+ *                           sample of its window and streams the window once (d >= 256);
+ *                           rows it cannot certify are selected again by the exact
+ *                           three-pass kernel, so the result is the same either way.
  * RECE_ERR_INVALID_ARG for a NULL argument. */
 #define RECE_PATH_TENSOR_CORES 0x1u
 #define RECE_PATH_DX_TENSORS 0x2u
@@ -164,6 +168,7 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
 #define RECE_PATH_ALL_NEGATIVES 0x8u  /* RECE_FLAG_ALL_NEGATIVES: window sums on tcgen05 */
 #define RECE_PATH_DY_TENSORS 0x10u
 #define RECE_PATH_DX_PARTS 0x20u
+#define RECE_PATH_SAMPLED_SELECT 0x40u
 RECE_API rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths);
 
 /* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].

@@ -25,6 +25,7 @@ PATH_STORED_SCORES = 0x4
 PATH_ALL_NEGATIVES = 0x8
 PATH_DY_TENSORS = 0x10
 PATH_DX_PARTS = 0x20
+PATH_SAMPLED_SELECT = 0x40
 FLAG_ALL_NEGATIVES = 0x2  # Algorithm 1 as printed: every window item a negative
 
 # every symbol include/rece.h declares

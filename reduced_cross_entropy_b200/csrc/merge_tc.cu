@@ -184,7 +184,9 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
     // four sub-lists (one per epilogue warpgroup of the selection kernel), read as one
     // concatenated list, kGather independent entries per lane in flight at a time
     const int4 c4 = list_count[int64_t(r) * N + p];
-    theta_max = fmaxf(theta_max, list_theta[int64_t(r) * N + p]);
+    // every entry at or below the round's theta lies below its cut: not a candidate
+    const float theta_r = list_theta[int64_t(r) * N + p];
+    theta_max = fmaxf(theta_max, theta_r);
     const int cs[4] = {c4.x < Qw ? c4.x : Qw, c4.y < Qw ? c4.y : Qw, c4.z < Qw ? c4.z : Qw,
                        c4.w < Qw ? c4.w : Qw};
     overflow |= c4.x > Qw || c4.y > Qw || c4.z > Qw || c4.w > Qw;
@@ -204,6 +206,7 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
           ++w;
         }
         e[u] = in[u] ? L[w * Qw + a] : make_int2(0, 0);
+        in[u] = in[u] && __int_as_float(e[u].x) > theta_r;
       }
 #pragma unroll
       for (int u = 0; u < kGather; ++u) jj[u] = in[u] ? py[int64_t(r) * C + e[u].y] : -1;

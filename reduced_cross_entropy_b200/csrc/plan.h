@@ -68,7 +68,8 @@ struct Layout {
   size_t list_score = 0, list_item = 0, row_loss_tmp = 0;
   // tensor-core path (bf16 mode): sorted row copies, inverse orders, candidate lists
   size_t xs = 0, ys = 0, inv_x = 0, chunk_y = 0, tc_list = 0, tc_count = 0, tc_theta = 0,
-         spill_rows = 0, spill_scratch = 0, scores = 0;
+         spill_rows = 0, spill_scratch = 0, scores = 0,
+         redo_list = 0;  // work items the sampled selection hands to the exact one
   size_t fwd_end = 0;
   // backward region (rece_loss_bwd), overlaps the forward region
   size_t e_key = 0, e_g = 0, e_perm_a = 0, e_perm_b = 0, e_sorted_key = 0, e_key_b = 0,
@@ -109,6 +110,8 @@ struct rece_plan_s {
   bool tc_dy;           // ... and dY (band products; positives through pos_plan's pairs)
   int dx_split;         // tensor-core dX: 0 one launch per round, S > 0 K splits into parts
   bool tc_scores;       // ... with the window scores computed once and stored (large d)
+  bool tc_sampled;      // ... else the fused selection's threshold from a 1/8 sample of
+                        // the window (one streaming pass; d >= 256), or exact (three)
   int64_t score_width;  // columns of the stored scores per row (longest union, padded)
   int32_t kept_slices;  // most 64-position slices one window touches
   bool all_neg;         // RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed, no top-k

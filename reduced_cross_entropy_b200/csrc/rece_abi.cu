@@ -151,7 +151,9 @@ void build_layout(rece_plan_s& p) {
     off += align256(bytes);
     return o;
   };
-  L.status = take(4 * sizeof(uint32_t));  // flags, inexact rows, of which overflowed
+  // flags, inexact rows, of which overflowed, rows the merge spilled, items the sampled
+  // selection handed to the exact one
+  L.status = take(8 * sizeof(uint32_t));
   const size_t nb_stride = (size_t(1) << p.bucket_bits) + 1;
   if (p.use_tc) {
     // the orders, kept from rece_loss_fwd until rece_loss_bwd has run
@@ -162,7 +164,7 @@ void build_layout(rece_plan_s& p) {
   // the forward
   if (p.tc_dy) L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
   if (p.tc_dx) {
-    L.ys = take(sizeof(uint16_t) * size_t(c.n_r) * c.C * c.d);
+    L.ys = take(sizeof(uint16_t) * size_t(tc_ys_rows(int64_t(c.n_r) * c.C)) * c.d);
     L.kept = take(sizeof(int2) * size_t(c.n_r) * c.N * c.k);
     L.kept_off = take(sizeof(int32_t) * size_t(c.n_r) * c.N * (size_t(p.kept_slices) + 1));
     L.pos_logit = take(sizeof(float) * size_t(c.N));
@@ -182,7 +184,7 @@ void build_layout(rece_plan_s& p) {
   if (p.use_tc) {
     const size_t Q = size_t(tc_list_capacity(c.k));
     if (!p.tc_dy) L.xs = take(sizeof(uint16_t) * size_t(c.n_r) * c.N * c.d);
-    if (!p.tc_dx) L.ys = take(sizeof(uint16_t) * size_t(c.n_r) * c.C * c.d);
+    if (!p.tc_dx) L.ys = take(sizeof(uint16_t) * size_t(tc_ys_rows(int64_t(c.n_r) * c.C)) * c.d);
     L.inv_x = take(sizeof(int32_t) * c.n_r * c.N);
     L.chunk_y = take(sizeof(int32_t) * c.n_r * c.C);
     L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
@@ -190,6 +192,7 @@ void build_layout(rece_plan_s& p) {
     L.tc_theta = take(sizeof(float) * c.n_r * c.N);
     if (p.tc_scores) L.scores = take(sizeof(float) * size_t(c.n_r) * c.N * p.score_width);
     L.spill_rows = take(sizeof(int32_t) * size_t(c.N));
+    if (p.tc_sampled) L.redo_list = take(sizeof(int32_t) * size_t(tc_select_items(p)));
     L.spill_scratch = take(merge_tc_spill_bytes(c.n_r, c.k));
   } else {
     L.list_score = take(sizeof(float) * size_t(c.n_r) * c.N * c.k);
@@ -435,6 +438,11 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   // at large d the window scores are computed once and stored (a d-deep dot product per
   // score outweighs writing and reading it back)
   p->tc_scores = p->use_tc && c.d >= 1024;
+  // the fused selection: a sampled threshold and one streaming pass where each pass's
+  // multiply and stream cost outweigh emitting about twice k entries per row instead of
+  // about k (measured: 4.2 -> 2.4 ms at the 4M-item workload, d = 256; no gain at d = 64
+  // or 128, where the epilogue's per-score work, not the passes, bounds the kernel)
+  p->tc_sampled = p->use_tc && !p->tc_scores && c.d >= 256;
   p->score_width = p->tc_scores ? scores_tc_width(*p) : 0;
   p->tc_dx = p->use_tc && p->kept_slices <= kMaxKeptSlices &&
              (c.d >= 256 || 2.0 * double(c.C) * c.d > 64.0 * 1024 * 1024);
@@ -446,6 +454,7 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     }
     p->tc_dx = false;
     p->tc_scores = false;
+    p->tc_sampled = false;
     p->score_width = 0;
     // the positives' coefficients and their dY go through the pair backward (k = 0)
     rece_plan_s* q = new (std::nothrow) rece_plan_s();
@@ -466,11 +475,12 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
     return fail(RECE_ERR_UNSUPPORTED, "n_r * k too large for the tensor-core merge");
   }
   p->tc_dy = false;
-  if (p->tc_dx && !p->all_neg && c.d >= 1024) {
-    // dY as band products too (at large d: each x row gathered per pair is 2d bytes,
-    // while the band's builders cost the same per slab whatever d); the positives' dY
-    // through a pair backward of k = 0 that shares the pair region (N pairs fit where
-    // N (k + 1) do)
+  if (p->tc_dx && !p->all_neg && c.d >= 128) {
+    // dY as band products too wherever dX is (from d = 128: each x row gathered per pair
+    // is 2d bytes and the pairs need a sort by item, while the band's builders cost the
+    // same per slab whatever d; measured 8.4 -> 4.8 ms at the 4M-item workload, d = 256);
+    // the positives' dY through a pair backward of k = 0 that shares the pair region (N
+    // pairs fit where N (k + 1) do)
     rece_plan_s* q = new (std::nothrow) rece_plan_s();
     if (!q) {
       delete p;
@@ -546,7 +556,8 @@ rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
            (plan->tc_scores ? RECE_PATH_STORED_SCORES : 0u) |
            (plan->all_neg ? RECE_PATH_ALL_NEGATIVES : 0u) |
            (plan->tc_dy ? RECE_PATH_DY_TENSORS : 0u) |
-           (plan->dx_split > 0 ? RECE_PATH_DX_PARTS : 0u);
+           (plan->dx_split > 0 ? RECE_PATH_DX_PARTS : 0u) |
+           (plan->tc_sampled ? RECE_PATH_SAMPLED_SELECT : 0u);
   return RECE_OK;
 }
 
@@ -560,7 +571,7 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const Layout& L = plan->lay;
-  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, 4 * sizeof(uint32_t), st), "status reset");
+  RECE_CUDA(cudaMemsetAsync(ws + L.status, 0, 8 * sizeof(uint32_t), st), "status reset");
   int32_t* bx = reinterpret_cast<int32_t*>(ws + L.bx);
   int32_t* by = reinterpret_cast<int32_t*>(ws + L.by);
   stage_mark(*plan, RECE_STAGE_BUCKETIZE, 0, st);
@@ -621,6 +632,12 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
                                   c.n_r, c.n_c, ws + L.ys, nullptr,
                                   reinterpret_cast<int32_t*>(ws + L.chunk_y), st),
               "permute Y");
+    // the copy's padding to whole 128-row groups (read by the selection's tiles, masked)
+    const int64_t rows = int64_t(c.n_r) * c.C, padded = tc_ys_rows(rows);
+    if (padded > rows)
+      RECE_CUDA(cudaMemsetAsync(ws + L.ys + size_t(rows) * c.d * 2, 0,
+                                size_t(padded - rows) * c.d * 2, st),
+                "pad Y copy");
   }
   stage_mark(*plan, RECE_STAGE_SORT, 1, st);
   return RECE_OK;
@@ -668,7 +685,9 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
                                         status, st),
                 "scores + select (tcgen05)");
     else
-      RECE_CUDA(launch_select_tc(*plan, ws + L.xs, ws + L.ys, list, cnt, theta, status, st),
+      RECE_CUDA(launch_select_tc(*plan, ws + L.xs, ws + L.ys, list, cnt, theta,
+                                 reinterpret_cast<int32_t*>(ws + L.redo_list), status + 4,
+                                 status, st),
                 "select (tcgen05)");
     stage_mark(*plan, RECE_STAGE_SELECT, 1, st);
     stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);

@@ -17,6 +17,13 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
 // box {64, box_rows, 1}, 128-byte swizzle; rows past the end read as zeros.
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
                               uint64_t rows, uint64_t planes, uint32_t box_rows);
+// A row-major bf16 matrix of groups x group_rows rows (cols a multiple of 64) seen as
+// [groups][group_rows][cols]: one box is the first box_rows rows of box_groups consecutive
+// groups, which lands in shared memory as box_rows * box_groups rows of a 128-byte-swizzled
+// K-major tile; groups past the end read as zeros.
+cudaError_t make_tmap_bf16_groups(CUtensorMap* map, const void* base, uint64_t cols,
+                                  uint64_t groups, uint32_t group_rows, uint32_t box_rows,
+                                  uint32_t box_groups);
 int sm_count();
 // out[i] += parts[0][i] + parts[1][i] + ... (n floats each, n % 4 == 0), in that order.
 cudaError_t launch_add_parts(const float* parts, int64_t n, int nparts, float* out,
@@ -38,11 +45,18 @@ cudaError_t launch_permute_rows(const void* V, int64_t M, int d, const int32_t* 
 
 // K3 on tensor cores: per (round, sorted row) the candidate list (score bits, sorted
 // catalogue position), its count and threshold.
+// The sorted copy Ys that the selection reads is padded to whole 128-row groups
+// (tc_ys_rows of the n_r * C rows; the padding is zeroed by rece_bucketize_sort).  With
+// p.tc_sampled a sampled pass sets each row's threshold and one pass emits; the items it
+// could not certify (redo_list, *redo_count, at most tc_select_items) are done again by
+// the exact kernel, which otherwise runs alone over every item.
 int tc_list_capacity(int k);      // entries per (round, row): 4 sub-lists
 int tc_sublist_capacity(int k);   // entries per sub-list
+int64_t tc_ys_rows(int64_t rows);
+int64_t tc_select_items(const rece_plan_s& p);
 cudaError_t launch_select_tc(const rece_plan_s& p, const void* Xs, const void* Ys, int2* list,
-                             int4* list_count, float* list_theta, uint32_t* status,
-                             cudaStream_t st);
+                             int4* list_count, float* list_theta, int32_t* redo_list,
+                             uint32_t* redo_count, uint32_t* status, cudaStream_t st);
 
 // Steps 3-4 for large d (see scores_tc.cu): window scores once into S [n_r][N][width],
 // then the exact per-row selection into the same lists as launch_select_tc.

@@ -62,6 +62,26 @@ cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t cols,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_tmap_bf16_groups(CUtensorMap* map, const void* base, uint64_t cols,
+                                  uint64_t groups, uint32_t group_rows, uint32_t box_rows,
+                                  uint32_t box_groups) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (groups == 0 || cols % 64 != 0 || box_rows == 0 || box_rows > group_rows ||
+      box_rows > 256 || box_groups == 0 || box_groups > 256 ||
+      (reinterpret_cast<uintptr_t>(base) & 15u) != 0)
+    return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {cols, group_rows, groups};
+  cuuint64_t strides[2] = {cols * 2, uint64_t(group_rows) * cols * 2};
+  cuuint32_t box[3] = {64, box_rows, box_groups};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 namespace {
 
 __global__ void __launch_bounds__(256) k_add_parts(const float4* __restrict__ parts, int64_t n4,

@@ -41,8 +41,9 @@ def run_gpu(w: synth.Workload, X, Y, t, B, flags=0, dloss=1.0, use_logits=True,
     dX, dY = ops.loss_bwd(plan, Xd, Yd, td, sel, lse, dl, ws,
                           logits=logits if use_logits else None)
     status = ops.device_status(ws)
-    # status area: flags, inexact rows, overflowed lists, rows the merge spilled
-    words = ws[:16].view(torch.int32).cpu().numpy()
+    # status area: flags, inexact rows, overflowed lists, rows the merge spilled, items
+    # the sampled selection handed to the exact kernel
+    words = ws[:32].view(torch.int32).cpu().numpy()
     return dict(bx=bx, by=by, permX=px, permY=py, loss=float(loss.item()), words=words,
                 row_loss=row.cpu().numpy(), selected=sel.cpu().numpy(), lse=lse.cpu().numpy(),
                 dX=dX.cpu().numpy(), dY=dY.cpu().numpy(), status=status, plan=plan,

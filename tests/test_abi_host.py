@@ -151,12 +151,17 @@ def test_plan_paths_follow_the_shape():
 
     assert paths(W["tiny"]) == 0                      # fp32 exact mode: fmaf kernels
     assert paths(W["sasrec"]) == TC                   # catalogue in L2: gathered dX
-    # 256 MB catalogue: dX on tcgen05; 400 row tiles a round, two CTAs an SM: both rounds
-    # in one launch (parts summed in order) fill the waves better than a launch a round
-    assert paths(W["large"]) == TC | DX | PARTS
+    # 256 MB catalogue: dX and dY on tcgen05; 400 row tiles a round, two CTAs an SM: both
+    # rounds in one launch (parts summed in order) fill the waves better than a launch a round
+    assert paths(W["large"]) == TC | DX | DY | PARTS
     # d = 4096: stored scores, dY on tcgen05; 1024 work items a round: a launch a round
     assert paths(W["lm"]) == TC | DX | SC | DY
-    assert paths(W["very_large"]) == TC | DX | PARTS  # d = 256: dY by the pair sort
+    # d = 256: the selection's threshold from a sample of the window, one streaming pass
+    assert paths(W["very_large"]) == TC | DX | DY | PARTS | _lib.PATH_SAMPLED_SELECT
+    # catalogues beyond half of L2 at small d: dX on tcgen05, dY too from d = 128 on
+    big = W["sasrec"].scaled(25_600, 600_000)
+    assert paths(big) & (DX | DY) == DX                 # d = 64: dY by the pair sort
+    assert paths(big, d=128) & (DX | DY) == DX | DY
     assert paths(W["sasrec"], d=48) == 0              # d not a multiple of 64
     p = Plan(256, 4096, 64, 16, 8, 1, 1, 32, mode="bf16", flags=_lib.FLAG_FMA_SCORES)
     assert p.paths == 0                               # fmaf scores on request

@@ -172,3 +172,29 @@ def test_merge_spill_path_on_tied_scores(d):
     term = 1.0 / w.N * float(np.abs(Y).max())
     assert np.abs(g["dX"] - o["dX"]).max() <= 1e-4 * term
     assert max_rel(g["dY"], o["dY"]) <= 1e-4
+
+
+def test_sampled_selection_hands_misled_rows_to_the_exact_kernel():
+    """d >= 256: each row's threshold comes from a sample of its window (the first 16
+    positions of every 128-position tile).  With one bucket the sorted order is the item
+    order, so making exactly the sampled items score high misleads the sample: fewer than
+    k + 1 scores pass its threshold, the rows cannot be certified and go to the exact
+    three-pass kernel.  The kept sets must still be the oracle's (ties to the lower id)."""
+    from reduced_cross_entropy_b200 import _lib
+    w = synth.Workload("misled", N=256, C=4096, d=256, dtype="bf16", n_b=1, n_c=2, n_ec=0,
+                       n_r=1, k=400)
+    X = np.full((w.N, w.d), 0.125, np.float32)
+    j = np.arange(w.C)
+    sampled = (j % 128) < 16
+    Y = np.where(sampled[:, None], 0.25 * (1 + j[:, None] % 3), 0.125 * (j[:, None] % 5 - 2))
+    Y = np.ascontiguousarray(np.broadcast_to(Y, (w.C, w.d)), dtype=np.float32)
+    t = np.random.default_rng(9).integers(0, w.C, w.N).astype(np.int32)
+    B = np.ones((1, 1, w.d), np.float32)
+    g = run_gpu(w, X, Y, t, B, flags=0, dloss=1.0)
+    assert g["plan"].paths & _lib.PATH_SAMPLED_SELECT
+    assert g["status"] & ~0x4 == 0 and g["words"][1] == 0   # certified exact
+    assert g["words"][4] > 0                                 # items redone exactly
+    o = run_oracle(w, X, Y, t, B, dloss=1.0)
+    np.testing.assert_array_equal(np.sort(g["selected"], axis=1), np.sort(o["selected"], axis=1))
+    assert abs(g["loss"] - o["loss"]) <= 1e-4 * abs(o["loss"])
+    assert max_rel(g["dX"], o["dX"]) <= 1e-4 and max_rel(g["dY"], o["dY"]) <= 1e-4
