@@ -652,7 +652,9 @@ __global__ void __launch_bounds__(256) k_bwd_pos(const T* __restrict__ Y,
 }  // namespace
 
 // Band-product geometry for d: CTA slices of ns <= 512 columns (two TMEM accumulators
-// past 256) and a TMA ring as deep as lets two CTAs share an SM (at least two slabs).
+// past 256) and a TMA ring as deep as lets two CTAs share an SM (at least two slabs), or,
+// where two cannot share one (ns >= 256), as deep as one CTA's shared memory allows (at
+// the 4M-item workload, d = 256: dY 4.16 -> 3.76 ms, its CTAs' few slabs all in flight).
 struct BandGeometry {
   int ns, slices, nb;
   size_t smem;
@@ -666,6 +668,8 @@ BandGeometry band_geometry(int d) {
                           : (d % 256 == 0 ? 256 : (d % 192 == 0 ? 192 : (d % 128 == 0 ? 128 : 64)));
   g.slices = d / g.ns;
   int nb = int((110 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(g.ns) * 128));
+  if (nb < 2)  // two CTAs cannot share an SM anyway: one CTA takes the SM's shared memory
+    nb = int((227 * 1024 - 2 * kAStages * kATile - 1024 - sizeof(Ctl)) / (size_t(g.ns) * 128));
   g.nb = nb > kMaxBStages ? kMaxBStages : (nb < 2 ? 2 : nb);
   g.smem = smem_bytes(g.nb, g.ns);
   g.tcols = g.ns <= 32 ? 32u : (g.ns <= 64 ? 64u : (g.ns <= 128 ? 128u : (g.ns <= 256 ? 256u : 512u)));
