@@ -777,12 +777,16 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
         ops.full_ce_bwd(Xd, Yd, td, l, torch.ones(1, device=dev), ws)
 
     out["rece_bytes"] = peak(rece)
-    # the fused exact op runs on the CUDA cores: past ~3e13 flops (minutes) it is skipped
+    # the fused exact op's memory is its outputs (lse, row losses, dX, dY in fp32) and its
+    # workspace, whatever the run time; it is run where its 6 N C d flops take seconds
+    ws_bytes = ops.full_ce_workspace_bytes(w.N, w.C, w.d, w.dtype)
+    out["full_ce_fused_bytes_computed"] = 4 * (2 * w.N + w.N * w.d + w.C * w.d + 1) + ws_bytes
     if 6.0 * w.N * w.C * w.d <= 3e13:
         out["full_ce_fused_bytes"] = peak(fused)
     else:
         out["full_ce_fused_bytes"] = None
-        out["full_ce_fused_note"] = "skipped: 6 N C d flops on the CUDA cores would take minutes"
+        out["full_ce_fused_note"] = (f"not run: {6.0 * w.N * w.C * w.d:.1e} flops; its allocations "
+                                     f"are full_ce_fused_bytes_computed")
     mat = 8 * w.N * w.C
     out["full_ce_materialised_bytes_computed"] = mat
     free = torch.cuda.mem_get_info(dev)[0]
@@ -794,8 +798,8 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
         out["full_ce_materialised_bytes_measured"] = peak(materialised)
     ref = out.get("full_ce_materialised_bytes_measured", mat)
     out["ratio_vs_materialised"] = ref / max(out["rece_bytes"], 1)
-    if out["full_ce_fused_bytes"] is not None:
-        out["ratio_vs_fused"] = out["full_ce_fused_bytes"] / max(out["rece_bytes"], 1)
+    fused_ref = out["full_ce_fused_bytes"] or out["full_ce_fused_bytes_computed"]
+    out["ratio_vs_fused"] = fused_ref / max(out["rece_bytes"], 1)
     # the pages' memory model of Algorithm 1 (every chunk's logits stored) at this
     # workload's alpha_bc = n_b / n_c, and the bucket count it calls optimal
     a = w.n_b / w.n_c

@@ -77,10 +77,12 @@ typedef enum {
  * enters each round's sum as exp(l - ln cnt) [the rounds paragraph], the positive left
  * out of the window sums (it enters once, as l+):
  *   lse_i = log(exp(l+) + sum_r sum_{j in W_r(i), j != z_i} exp(l_ij) / cnt_ij).
- * The window sums are formed on the tcgen05 tensor cores and never stored; the backward
- * recomputes them.  bf16 mode, d a multiple of 64 and at most 256 (else
- * RECE_ERR_UNSUPPORTED).  rece_loss_fwd writes no logits and fills `selected` (which may
- * be NULL) with -1; rece_loss_bwd ignores `selected` and `logits` (either may be NULL). */
+ * The window sums are never stored; the backward recomputes them: on the tcgen05 tensor
+ * cores in bf16 mode with d a multiple of 64 up to 256, else (fp32 mode, bf16 with
+ * RECE_FLAG_FMA_SCORES, other widths) on the CUDA cores with the fixed-order fmaf chain of
+ * the scores (RECE_PATH_WINDOW_FMA).  rece_loss_fwd writes no logits and fills `selected`
+ * (which may be NULL) with -1; rece_loss_bwd ignores `selected` and `logits` (either may be
+ * NULL). */
 #define RECE_FLAG_ALL_NEGATIVES 0x2u
 
 /* Bits of the device status word (rece_get_device_status). */
@@ -160,7 +162,11 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
  *   RECE_PATH_SAMPLED_SELECT the fused selection sets each row's threshold from a 1/8
  *                           sample of its window and streams the window once (d >= 256);
  *                           rows it cannot certify are selected again by the exact
- *                           three-pass kernel, so the result is the same either way.
+ *                           three-pass kernel, so the result is the same either way;
+ *   RECE_PATH_WINDOW_FMA    (with RECE_PATH_ALL_NEGATIVES) the window sums and their
+ *                           gradients on the CUDA cores, with the fixed-order fmaf chain
+ *                           of RECE_MODE_FP32_EXACT (fp32 mode, RECE_FLAG_FMA_SCORES, or a
+ *                           width the tcgen05 window kernels do not take).
  * RECE_ERR_INVALID_ARG for a NULL argument. */
 #define RECE_PATH_TENSOR_CORES 0x1u
 #define RECE_PATH_DX_TENSORS 0x2u
@@ -169,6 +175,8 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
 #define RECE_PATH_DY_TENSORS 0x10u
 #define RECE_PATH_DX_PARTS 0x20u
 #define RECE_PATH_SAMPLED_SELECT 0x40u
+#define RECE_PATH_WINDOW_FMA 0x80u  /* with RECE_PATH_ALL_NEGATIVES: window sums on the CUDA
+                                       cores (fmaf chains), not tcgen05 */
 RECE_API rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths);
 
 /* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].

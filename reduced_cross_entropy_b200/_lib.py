@@ -26,6 +26,7 @@ PATH_ALL_NEGATIVES = 0x8
 PATH_DY_TENSORS = 0x10
 PATH_DX_PARTS = 0x20
 PATH_SAMPLED_SELECT = 0x40
+PATH_WINDOW_FMA = 0x80  # with PATH_ALL_NEGATIVES: window sums on the CUDA cores
 FLAG_ALL_NEGATIVES = 0x2  # Algorithm 1 as printed: every window item a negative
 
 # every symbol include/rece.h declares

@@ -5,6 +5,7 @@
 //   Vs[r][p][:]       = V[perm[r][p]][:]                (bf16, 16-byte vector copies)
 //   inv[r][perm[r][p]] = p
 //   chunk[r][perm[r][p]] = chunk holding sorted position p (start of chunk c = ceil(cM/n_c))
+// (Vs may be NULL: then only the inverse orders and chunks are written.)
 // The backward's tensor-core products read Vs too, as MN-major operands.
 #include "common.cuh"
 #include "plan.h"
@@ -25,9 +26,11 @@ __global__ void __launch_bounds__(256) k_permute_rows(const uint4* __restrict__ 
        w += warps) {
     const int64_t r = w / M, p = w % M;
     const int32_t id = perm[w];
-    const uint4* src = V + int64_t(id) * vec_per_row;
-    uint4* dst = Vs + w * vec_per_row;
-    for (int c = lane; c < vec_per_row; c += 32) dst[c] = src[c];
+    if (Vs) {  // (no copy wanted: the inverse order and chunks only)
+      const uint4* src = V + int64_t(id) * vec_per_row;
+      uint4* dst = Vs + w * vec_per_row;
+      for (int c = lane; c < vec_per_row; c += 32) dst[c] = src[c];
+    }
     if (lane == 0) {
       if (inv) inv[r * M + id] = int32_t(p);
       if (chunk) chunk[r * M + id] = int32_t((p * n_c) / M);

@@ -115,6 +115,7 @@ struct rece_plan_s {
   int64_t score_width;  // columns of the stored scores per row (longest union, padded)
   int32_t kept_slices;  // most 64-position slices one window touches
   bool all_neg;         // RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed, no top-k
+  bool window_tc;       // ... its window sums and gradients on tcgen05 (else CUDA cores)
   rece_plan_s* pos_plan;  // all-negatives mode and tensor-core dY: the positives' pair
                           // backward (k = 0)
   rece::Layout lay;

@@ -111,8 +111,10 @@ void build_layout_all_neg(rece_plan_s& p) {
   const size_t nr = size_t(c.n_r);
   L.px = take(sizeof(int32_t) * nr * c.N);
   L.py = take(sizeof(int32_t) * nr * c.C);
-  L.xs = take(sizeof(uint16_t) * nr * c.N * c.d);
-  L.ys = take(sizeof(uint16_t) * nr * c.C * c.d);
+  if (p.window_tc) {  // the tcgen05 kernels' sorted copies (the CUDA-core ones read X, Y)
+    L.xs = take(sizeof(uint16_t) * nr * c.N * c.d);
+    L.ys = take(sizeof(uint16_t) * nr * c.C * c.d);
+  }
   L.itemc = take(sizeof(int32_t) * nr * nr * c.C);
   L.rowc = take(sizeof(int32_t) * nr * nr * c.N);
   L.pz = take(sizeof(int32_t) * nr * c.N);
@@ -133,7 +135,7 @@ void build_layout_all_neg(rece_plan_s& p) {
   rece_plan_s& q = *p.pos_plan;
   q.lay.status = L.status;
   layout_pairs(q, off);
-  L.dx_parts = take(sizeof(float) * nr * c.N * c.d);  // each round's part of dX
+  if (p.window_tc) L.dx_parts = take(sizeof(float) * nr * c.N * c.d);  // each round's part of dX
   L.bwd_end = off;
   L.total = L.fwd_end > L.bwd_end ? L.fwd_end : L.bwd_end;
 }
@@ -278,6 +280,8 @@ rece_status_t all_neg_fwd(const rece_plan_s& p, const void* X, const void* Y,
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
   float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + L.row_loss_tmp);
   float2* ms = reinterpret_cast<float2*>(ws + L.ms);
+  float* ls = reinterpret_cast<float*>(ws + L.lse_sorted);
+  const bool f32 = c.mode == RECE_MODE_FP32_EXACT;
   stage_mark(p, RECE_STAGE_SELECT, 0, st);
   RECE_CUDA(launch_window_meta(I(L.py), I(L.inv_y), c.C, c.n_c, c.n_r, I(L.itemc), nullptr,
                                nullptr, c.C, nullptr, st),
@@ -285,16 +289,32 @@ rece_status_t all_neg_fwd(const rece_plan_s& p, const void* X, const void* Y,
   RECE_CUDA(launch_window_meta(I(L.px), I(L.inv_x), c.N, c.n_c, c.n_r, I(L.rowc), targets,
                                I(L.inv_y), c.C, I(L.pz), st),
             "row chunk tables");
-  RECE_CUDA(launch_window_lse_tc(p, ws + L.xs, ws + L.ys, I(L.itemc), I(L.rowc), I(L.pz), ms,
-                                 status, st),
-            "window sums (tcgen05)");
+  if (p.window_tc)
+    RECE_CUDA(launch_window_lse_tc(p, ws + L.xs, ws + L.ys, I(L.itemc), I(L.rowc), I(L.pz), ms,
+                                   status, st),
+              "window sums (tcgen05)");
+  else if (f32)
+    RECE_CUDA(launch_window_lse_fma(p, static_cast<const float*>(X),
+                                    static_cast<const float*>(Y), I(L.px), I(L.py), targets,
+                                    I(L.itemc), I(L.rowc), ms, st),
+              "window sums (fmaf)");
+  else
+    RECE_CUDA(launch_window_lse_fma(p, static_cast<const __nv_bfloat16*>(X),
+                                    static_cast<const __nv_bfloat16*>(Y), I(L.px), I(L.py),
+                                    targets, I(L.itemc), I(L.rowc), ms, st),
+              "window sums (fmaf)");
   stage_mark(p, RECE_STAGE_SELECT, 1, st);
   stage_mark(p, RECE_STAGE_MERGE_LOSS, 0, st);
-  RECE_CUDA(launch_window_combine(p, static_cast<const __nv_bfloat16*>(X),
-                                  static_cast<const __nv_bfloat16*>(Y), targets, I(L.inv_x), ms,
-                                  lse, rl, reinterpret_cast<float*>(ws + L.lse_sorted), status,
-                                  st),
-            "rounds' log-sum-exp");
+  if (f32)
+    RECE_CUDA(launch_window_combine(p, static_cast<const float*>(X),
+                                    static_cast<const float*>(Y), targets, I(L.inv_x), ms, lse,
+                                    rl, ls, status, st),
+              "rounds' log-sum-exp");
+  else
+    RECE_CUDA(launch_window_combine(p, static_cast<const __nv_bfloat16*>(X),
+                                    static_cast<const __nv_bfloat16*>(Y), targets, I(L.inv_x),
+                                    ms, lse, rl, ls, status, st),
+              "rounds' log-sum-exp");
   if (selected && c.N > 0)
     RECE_CUDA(cudaMemsetAsync(selected, 0xFF, sizeof(int32_t) * size_t(c.N) * c.k, st),
               "selected");
@@ -307,32 +327,51 @@ rece_status_t all_neg_fwd(const rece_plan_s& p, const void* X, const void* Y,
 
 // Backward of the all-negatives mode: the positives' terms (written), then the window
 // terms of dX and of dY, added round by round.
-rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
-                          const int32_t* targets, const float* lse, const float* dloss,
-                          char* ws, float* dX, float* dY, cudaStream_t st) {
+template <typename T>
+rece_status_t all_neg_bwd_t(const rece_plan_s& p, const T* X, const T* Y,
+                            const int32_t* targets, const float* lse, const float* dloss,
+                            char* ws, float* dX, float* dY, cudaStream_t st) {
   const Layout& L = p.lay;
   auto I = [&](size_t o) { return reinterpret_cast<const int32_t*>(ws + o); };
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
   const float* ls = reinterpret_cast<const float*>(ws + L.lse_sorted);
   stage_mark(p, RECE_STAGE_BWD_ROWS, 0, st);
-  RECE_CUDA(launch_backward(*p.pos_plan, static_cast<const __nv_bfloat16*>(X),
-                            static_cast<const __nv_bfloat16*>(Y), targets, nullptr, lse, nullptr,
-                            dloss, ws, dX, dY, status, st),
+  RECE_CUDA(launch_backward(*p.pos_plan, X, Y, targets, nullptr, lse, nullptr, dloss, ws, dX,
+                            dY, status, st),
             "positives' backward");
-  RECE_CUDA(launch_window_grad_tc(p, false, ws + L.xs, ws + L.ys,
-                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.px), dloss, dX,
-                                  reinterpret_cast<float*>(ws + L.dx_parts), status, st),
-            "window dX (tcgen05)");
+  if (p.window_tc)
+    RECE_CUDA(launch_window_grad_tc(p, false, ws + L.xs, ws + L.ys, I(L.itemc), I(L.rowc),
+                                    I(L.pz), ls, I(L.px), dloss, dX,
+                                    reinterpret_cast<float*>(ws + L.dx_parts), status, st),
+              "window dX (tcgen05)");
+  else
+    RECE_CUDA(launch_window_grad_fma(p, false, X, Y, I(L.px), I(L.py), targets, I(L.itemc),
+                                     I(L.rowc), lse, dloss, dX, st),
+              "window dX (fmaf)");
   stage_mark(p, RECE_STAGE_BWD_ROWS, 1, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 0, st);
   stage_mark(p, RECE_STAGE_BWD_SORT, 1, st);
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 0, st);
-  RECE_CUDA(launch_window_grad_tc(p, true, ws + L.xs, ws + L.ys,
-                                  I(L.itemc), I(L.rowc), I(L.pz), ls, I(L.py), dloss, dY,
-                                  nullptr, status, st),
-            "window dY (tcgen05)");
+  if (p.window_tc)
+    RECE_CUDA(launch_window_grad_tc(p, true, ws + L.xs, ws + L.ys, I(L.itemc), I(L.rowc),
+                                    I(L.pz), ls, I(L.py), dloss, dY, nullptr, status, st),
+              "window dY (tcgen05)");
+  else
+    RECE_CUDA(launch_window_grad_fma(p, true, X, Y, I(L.px), I(L.py), targets, I(L.itemc),
+                                     I(L.rowc), lse, dloss, dY, st),
+              "window dY (fmaf)");
   stage_mark(p, RECE_STAGE_BWD_ITEMS, 1, st);
   return RECE_OK;
+}
+
+rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
+                          const int32_t* targets, const float* lse, const float* dloss,
+                          char* ws, float* dX, float* dY, cudaStream_t st) {
+  if (p.cfg.mode == RECE_MODE_FP32_EXACT)
+    return all_neg_bwd_t(p, static_cast<const float*>(X), static_cast<const float*>(Y), targets,
+                         lse, dloss, ws, dX, dY, st);
+  return all_neg_bwd_t(p, static_cast<const __nv_bfloat16*>(X),
+                       static_cast<const __nv_bfloat16*>(Y), targets, lse, dloss, ws, dX, dY, st);
 }
 
 }  // namespace
@@ -411,7 +450,7 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
       break;
     }
   }
-  if (p->sel_rows == 0) {
+  if (p->sel_rows == 0 && !(c.flags & RECE_FLAG_ALL_NEGATIVES)) {
     delete p;
     return fail(RECE_ERR_UNSUPPORTED, "chunk window too long for the selection kernel");
   }
@@ -446,12 +485,11 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   p->score_width = p->tc_scores ? scores_tc_width(*p) : 0;
   p->tc_dx = p->use_tc && p->kept_slices <= kMaxKeptSlices &&
              (c.d >= 256 || 2.0 * double(c.C) * c.d > 64.0 * 1024 * 1024);
+  p->window_tc = false;
   if (p->all_neg) {
-    if (!window_tc_supported(*p)) {
-      delete p;
-      return fail(RECE_ERR_UNSUPPORTED,
-                  "all-negatives mode needs bf16 on tcgen05 with d a multiple of 64, <= 256");
-    }
+    // the window sums on tcgen05 where those kernels take the shape (bf16, d a multiple of
+    // 64 up to 256), else on the CUDA cores (fmaf chains: fp32 mode, the FMA flag, wide d)
+    p->window_tc = window_tc_supported(*p);
     p->tc_dx = false;
     p->tc_scores = false;
     p->tc_sampled = false;
@@ -557,7 +595,8 @@ rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
            (plan->all_neg ? RECE_PATH_ALL_NEGATIVES : 0u) |
            (plan->tc_dy ? RECE_PATH_DY_TENSORS : 0u) |
            (plan->dx_split > 0 ? RECE_PATH_DX_PARTS : 0u) |
-           (plan->tc_sampled ? RECE_PATH_SAMPLED_SELECT : 0u);
+           (plan->tc_sampled ? RECE_PATH_SAMPLED_SELECT : 0u) |
+           (plan->all_neg && !plan->window_tc ? RECE_PATH_WINDOW_FMA : 0u);
   return RECE_OK;
 }
 
@@ -615,12 +654,15 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
   RECE_CUDA(launch_sort_batch(segs, 2 * c.n_r, 0, plan->bucket_bits, false, st),
             "sort X and Y");
   if (plan->all_neg) {
-    RECE_CUDA(launch_permute_rows(X, c.N, c.d, reinterpret_cast<const int32_t*>(ws + L.px),
-                                  c.n_r, c.n_c, ws + L.xs,
+    // sorted bf16 copies for the tcgen05 window kernels; the inverse orders either way
+    RECE_CUDA(launch_permute_rows(X, c.N, plan->window_tc ? c.d : 0,
+                                  reinterpret_cast<const int32_t*>(ws + L.px), c.n_r, c.n_c,
+                                  plan->window_tc ? ws + L.xs : nullptr,
                                   reinterpret_cast<int32_t*>(ws + L.inv_x), nullptr, st),
               "permute X");
-    RECE_CUDA(launch_permute_rows(Y, c.C, c.d, reinterpret_cast<const int32_t*>(ws + L.py),
-                                  c.n_r, c.n_c, ws + L.ys,
+    RECE_CUDA(launch_permute_rows(Y, c.C, plan->window_tc ? c.d : 0,
+                                  reinterpret_cast<const int32_t*>(ws + L.py), c.n_r, c.n_c,
+                                  plan->window_tc ? ws + L.ys : nullptr,
                                   reinterpret_cast<int32_t*>(ws + L.inv_y), nullptr, st),
               "permute Y");
   } else if (plan->use_tc) {

@@ -121,6 +121,20 @@ cudaError_t launch_window_combine(const rece_plan_s& p, const T* X, const T* Y,
                                   const int32_t* targets, const int32_t* invX, const float2* ms,
                                   float* lse, float* row_loss, float* lse_sorted,
                                   uint32_t* status, cudaStream_t st);
+// The all-negatives mode on the CUDA cores (window_fma.cu: fp32 mode, RECE_FLAG_FMA_SCORES,
+// or bf16 widths the tcgen05 window kernels do not take), reading X and Y in place through
+// the orders px, py: ms [n_r][N] as launch_window_lse_tc writes it, and the window terms
+// of dX (dy = false) or dY (dy = true) added into `out` one round after another.
+template <typename T>
+cudaError_t launch_window_lse_fma(const rece_plan_s& p, const T* X, const T* Y,
+                                  const int32_t* px, const int32_t* py, const int32_t* targets,
+                                  const int32_t* itemc, const int32_t* rowc, float2* ms,
+                                  cudaStream_t st);
+template <typename T>
+cudaError_t launch_window_grad_fma(const rece_plan_s& p, bool dy, const T* X, const T* Y,
+                                   const int32_t* px, const int32_t* py, const int32_t* targets,
+                                   const int32_t* itemc, const int32_t* rowc, const float* lse,
+                                   const float* dloss, float* out, cudaStream_t st);
 // The window terms of dX (dy = false, perm = px) or dY (dy = true, perm = py), added
 // into `out` round by round (dX with `scratch` [n_r][N][d]: all rounds in one grid, then
 // added in round order).

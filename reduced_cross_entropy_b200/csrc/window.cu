@@ -105,6 +105,9 @@ cudaError_t launch_window_combine(const rece_plan_s& p, const T* X, const T* Y,
   return cudaGetLastError();
 }
 
+template cudaError_t launch_window_combine<float>(
+    const rece_plan_s&, const float*, const float*, const int32_t*, const int32_t*,
+    const float2*, float*, float*, float*, uint32_t*, cudaStream_t);
 template cudaError_t launch_window_combine<__nv_bfloat16>(
     const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
     const int32_t*, const float2*, float*, float*, float*, uint32_t*, cudaStream_t);

@@ -204,16 +204,29 @@ def test_sampled_workspace_and_validation():
 
 
 def test_all_negatives_mode_support():
+    """Algorithm 1 as printed: window sums on tcgen05 for bf16 with d a multiple of 64 up
+    to 256, on the CUDA cores (fmaf chains) for every other shape and mode."""
     flags = _lib.FLAG_ALL_NEGATIVES
+    TC, AN, FMA = _lib.PATH_TENSOR_CORES, _lib.PATH_ALL_NEGATIVES, _lib.PATH_WINDOW_FMA
     p = Plan(1000, 5000, 128, 16, 8, 1, 2, 8, mode="bf16", flags=flags)
-    assert p.paths == _lib.PATH_TENSOR_CORES | _lib.PATH_ALL_NEGATIVES
+    assert p.paths == TC | AN
     assert p.workspace_bytes > 0
-    for bad in (dict(mode="fp32"), dict(d=512), dict(d=96)):
+
+    def paths(**over):
         kw = dict(N=1000, C=5000, d=128, n_b=16, n_c=8, n_ec=1, n_r=2, k=8, mode="bf16")
-        kw.update(bad)
-        with pytest.raises(RuntimeError):
-            Plan(kw["N"], kw["C"], kw["d"], kw["n_b"], kw["n_c"], kw["n_ec"], kw["n_r"],
-                 kw["k"], mode=kw["mode"], flags=flags)
+        kw.update(over)
+        return Plan(kw["N"], kw["C"], kw["d"], kw["n_b"], kw["n_c"], kw["n_ec"], kw["n_r"],
+                    kw["k"], mode=kw["mode"], flags=kw.get("flags", flags)).paths
+
+    assert paths(mode="fp32") == AN | FMA                   # fp32 exact mode
+    assert paths(d=512) == TC | AN | FMA                    # bucketing on tcgen05 only
+    assert paths(d=4096, N=16_384, C=128_000, n_b=512, n_c=128) == TC | AN | FMA  # LM shape
+    assert paths(d=96) == AN | FMA                          # d not a multiple of 64
+    assert paths(flags=flags | _lib.FLAG_FMA_SCORES) == AN | FMA
+    # the CUDA-core mode keeps no sorted copies: a smaller workspace than the tcgen05 one
+    a = Plan(1000, 5000, 128, 16, 8, 1, 2, 8, mode="bf16", flags=flags)
+    b = Plan(1000, 5000, 128, 16, 8, 1, 2, 8, mode="bf16", flags=flags | _lib.FLAG_FMA_SCORES)
+    assert b.workspace_bytes < a.workspace_bytes
 
 
 @pytest.mark.parametrize("N,C,n_ec", [(256, 4096, 1), (25_600, 100_000, 1),

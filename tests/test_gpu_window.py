@@ -31,11 +31,11 @@ CASES = {
 }
 
 
-def run_window_gpu(w, X, Y, t, B, dloss=1.0):
-    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode="bf16",
-                    flags=_lib.FLAG_ALL_NEGATIVES)
+def run_window_gpu(w, X, Y, t, B, dloss=1.0, extra_flags=0):
+    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype,
+                    flags=_lib.FLAG_ALL_NEGATIVES | extra_flags)
     assert plan.paths & _lib.PATH_ALL_NEGATIVES
-    Xd, Yd, Bd = to_dev(X, "bf16"), to_dev(Y, "bf16"), to_dev(B, "bf16")
+    Xd, Yd, Bd = to_dev(X, w.dtype), to_dev(Y, w.dtype), to_dev(B, w.dtype)
     td = torch.from_numpy(t).cuda()
     ws = plan.workspace()
     ops.bucketize_sort(plan, Bd, Xd, Yd, ws)
@@ -46,7 +46,7 @@ def run_window_gpu(w, X, Y, t, B, dloss=1.0):
     dX, dY = ops.loss_bwd(plan, Xd, Yd, td, sel, lse, dl, ws)
     return dict(bx=bx, by=by, px=px, py=py, loss=float(loss.item()), row=row.cpu().numpy(),
                 lse=lse.cpu().numpy(), sel=sel.cpu().numpy(), dX=dX.cpu().numpy(),
-                dY=dY.cpu().numpy(), status=ops.device_status(ws))
+                dY=dY.cpu().numpy(), status=ops.device_status(ws), paths=plan.paths)
 
 
 def check_orders(g, n_r):
@@ -115,3 +115,75 @@ def test_window_identical_rounds_and_determinism():
     assert max_rel(b["dX"], a["dX"]) <= 1e-4 and max_rel(b["dY"], a["dY"]) <= 1e-4
     for key in ("row", "lse", "dX", "dY"):
         assert np.array_equal(b[key], c[key]), key
+
+
+# ---------------------------------------------------------------- on the CUDA cores
+# fp32 exact mode, bf16 with RECE_FLAG_FMA_SCORES and bf16 widths the tcgen05 window
+# kernels do not take: every score is the fixed-order fmaf chain, so the orders are the
+# oracle's bit for bit (fmaf bucketing) and every value is within 1e-4 of its fp64 sums.
+FMA_CASES = {
+    "fp32_d64_rounds2": W("f1", N=600, C=3000, d=64, dtype="fp32", n_b=16, n_c=6, n_ec=1,
+                          n_r=2, k=8),
+    "fp32_d48_rounds3_ragged": W("f2", N=333, C=2001, d=48, dtype="fp32", n_b=7, n_c=5,
+                                 n_ec=2, n_r=3, k=8, target_alpha=1.0),
+    "fp32_d7_no_neighbours": W("f3", N=200, C=999, d=7, dtype="fp32", n_b=5, n_c=4, n_ec=0,
+                               n_r=1, k=8),
+    "bf16_fma_flag_d128": W("f4", N=500, C=2500, d=128, dtype="bf16", n_b=16, n_c=5, n_ec=1,
+                            n_r=2, k=8),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FMA_CASES))
+def test_window_fma_parity(name):
+    w = FMA_CASES[name]
+    X, Y, t = synth.make_inputs(w, seed=12)
+    B = synth.projections(12, 0, w.n_r, w.n_b, w.d, w.dtype)
+    extra = _lib.FLAG_FMA_SCORES if w.dtype == "bf16" else 0
+    g = run_window_gpu(w, X, Y, t, B, dloss=0.75, extra_flags=extra)
+    assert g["paths"] & _lib.PATH_WINDOW_FMA
+    assert g["status"] == 0
+    full = oracle.rece_forward(X, Y, t, B, w.n_c, w.n_ec, 1)  # the oracle's own orders
+    np.testing.assert_array_equal(g["bx"], full["bx"])
+    np.testing.assert_array_equal(g["by"], full["by"])
+    np.testing.assert_array_equal(g["px"], full["permX"])
+    np.testing.assert_array_equal(g["py"], full["permY"])
+    o_loss, o_row, o_lse = oracle.window_loss(X, Y, t, full["permX"], full["permY"], w.n_c,
+                                              w.n_ec)
+    assert max_rel(g["row"], o_row) <= 1e-4 and max_rel(g["lse"], o_lse) <= 1e-4
+    assert abs(g["loss"] - o_loss) <= 1e-4 * abs(o_loss)
+    oX, oY = oracle.window_grad(X, Y, t, full["permX"], full["permY"], w.n_c, w.n_ec, o_lse,
+                                0.75)
+    assert max_rel(g["dX"], oX) <= 1e-4 and max_rel(g["dY"], oY) <= 1e-4
+    assert np.all(g["sel"] == -1)
+
+
+def test_window_fma_wide_rows_and_determinism():
+    """bf16 at d = 1024 (past the tcgen05 window kernels): bucketing on tcgen05, the window
+    sums on the CUDA cores; the oracle on the GPU's orders, values within 1e-4; two runs
+    agree bit for bit."""
+    w = W("fw", N=256, C=1500, d=1024, dtype="bf16", n_b=16, n_c=3, n_ec=1, n_r=2, k=8)
+    X, Y, t = synth.make_inputs(w, seed=13)
+    B = synth.projections(13, 0, w.n_r, w.n_b, w.d, w.dtype)
+    g = run_window_gpu(w, X, Y, t, B)
+    assert g["paths"] & _lib.PATH_WINDOW_FMA and g["status"] == 0
+    check_orders(g, w.n_r)
+    _, o_row, o_lse = oracle.window_loss(X, Y, t, g["px"], g["py"], w.n_c, w.n_ec)
+    assert max_rel(g["row"], o_row) <= 1e-4
+    oX, oY = oracle.window_grad(X, Y, t, g["px"], g["py"], w.n_c, w.n_ec, o_lse)
+    assert max_rel(g["dX"], oX) <= 1e-4 and max_rel(g["dY"], oY) <= 1e-4
+    h = run_window_gpu(w, X, Y, t, B)
+    for key in ("row", "lse", "dX", "dY"):
+        assert np.array_equal(g[key], h[key]), key
+
+
+def test_window_fma_one_bucket_one_chunk_is_full_ce():
+    """fp32, n_b = n_c = 1: every item is in every row's window, once per round: the full
+    cross-entropy (equation 3) and its gradient (equation 4), within 1e-4."""
+    w = W("ff", N=200, C=700, d=32, dtype="fp32", n_b=1, n_c=1, n_ec=0, n_r=2, k=8)
+    X, Y, t = synth.make_inputs(w, seed=14)
+    B = synth.projections(14, 0, w.n_r, w.n_b, w.d)
+    g = run_window_gpu(w, X, Y, t, B)
+    f_loss, f_row, f_lse = oracle.full_ce_loss(X, Y, t)
+    assert max_rel(g["row"], f_row) <= 1e-4
+    fX, fY = oracle.full_ce_grad(X, Y, t, f_lse)
+    assert max_rel(g["dX"], fX) <= 1e-4 and max_rel(g["dY"], fY) <= 1e-4
