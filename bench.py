@@ -772,17 +772,30 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
         _, _, s, l, lg = ops.loss_fwd(plan, Xd, Yd, td, ws, want_row_loss=False)
         ops.loss_bwd(plan, Xd, Yd, td, s, l, torch.ones(1, device=dev), ws, logits=lg)
 
+    fused_ms = []
+
     def fused():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
         _, _, l, ws = ops.full_ce_fwd(Xd, Yd, td)
         ops.full_ce_bwd(Xd, Yd, td, l, torch.ones(1, device=dev), ws)
+        b.record()
+        b.synchronize()
+        fused_ms.append(a.elapsed_time(b))
 
     out["rece_bytes"] = peak(rece)
     # the fused exact op's memory is its outputs (lse, row losses, dX, dY in fp32) and its
     # workspace, whatever the run time; it is run where its 6 N C d flops take seconds
     ws_bytes = ops.full_ce_workspace_bytes(w.N, w.C, w.d, w.dtype)
     out["full_ce_fused_bytes_computed"] = 4 * (2 * w.N + w.N * w.d + w.C * w.d + 1) + ws_bytes
-    if 6.0 * w.N * w.C * w.d <= 3e13:
+    # the op runs on tcgen05 for bf16 with d a multiple of 64 up to 256, else on the CUDA
+    # cores: run it (and time one fwd+bwd, after one untimed) where that takes seconds
+    tc = w.dtype == "bf16" and w.d % 64 == 0 and w.d <= 256
+    if 6.0 * w.N * w.C * w.d <= (2e15 if tc else 3e13):
+        fused()
         out["full_ce_fused_bytes"] = peak(fused)
+        out["full_ce_fused_ms_fwd_bwd"] = fused_ms[-1]
+        out["full_ce_fused_kernels"] = "tcgen05" if tc else "CUDA cores"
     else:
         out["full_ce_fused_bytes"] = None
         out["full_ce_fused_note"] = (f"not run: {6.0 * w.N * w.C * w.d:.1e} flops; its allocations "

@@ -223,8 +223,13 @@ RECE_API rece_status_t rece_loss_bwd(rece_plan_t plan, const void* X, const void
 
 /* Exact full cross-entropy [RECE equations (3) and (4)], fused: the logits are formed
  * tile by tile on chip and never stored.  Arguments as above; mode picks the input
- * element type.  The workspace (rece_full_ce_workspace_size bytes) holds the status
- * word. */
+ * element type.  In bf16 mode with d a multiple of 64 up to 256 the op runs on the tcgen05
+ * tensor cores as the all-negatives mode (RECE_FLAG_ALL_NEGATIVES) at n_b = n_c = n_r = 1
+ * -- every item in every row's window, counted once, which is equation (3) -- and its
+ * workspace then holds that mode's sorted copies and tables: rece_full_ce_bwd must get the
+ * workspace rece_full_ce_fwd used, unchanged in between.  Elsewhere (fp32 mode, other
+ * widths) it runs on the CUDA cores and the workspace holds the status word and the row
+ * losses.  rece_full_ce_workspace_size gives the bytes for the shape and mode. */
 RECE_API rece_status_t rece_full_ce_workspace_size(int64_t N, int64_t C, int32_t d, int32_t mode,
                                           size_t* bytes);
 RECE_API rece_status_t rece_full_ce_fwd(int64_t N, int64_t C, int32_t d, int32_t mode, const void* X,

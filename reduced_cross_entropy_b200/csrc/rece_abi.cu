@@ -374,6 +374,43 @@ rece_status_t all_neg_bwd(const rece_plan_s& p, const void* X, const void* Y,
                        static_cast<const __nv_bfloat16*>(Y), targets, lse, dloss, ws, dX, dY, st);
 }
 
+// The exact full cross-entropy on the tcgen05 tensor cores, where their window kernels
+// take the shape (bf16, d a multiple of 64 up to 256): the all-negatives mode with one
+// bucket, one chunk and one round is the full cross-entropy -- every item is in every
+// row's window, counted once, the positive entering once as l+ -- so the op runs that
+// mode's kernels through an internal plan.  The workspace holds the plan's workspace,
+// then the one (zero) random vector its bucketing reads.  Returns NULL elsewhere (the
+// CUDA-core kernels of full_ce.cu run).
+rece_plan_t full_ce_window_plan(int64_t N, int64_t C, int32_t d, int32_t mode) {
+  if (mode != RECE_MODE_BF16 || N < 1 || C < 1 || d % 64 != 0 || d > 256) return nullptr;
+  rece_config_t cfg{};
+  cfg.N = N;
+  cfg.C = C;
+  cfg.d = d;
+  cfg.n_b = 1;
+  cfg.n_c = 1;
+  cfg.n_ec = 0;
+  cfg.n_r = 1;
+  cfg.k = 1;
+  cfg.mode = RECE_MODE_BF16;
+  cfg.flags = RECE_FLAG_ALL_NEGATIVES;
+  rece_plan_t p = nullptr;
+  char saved[sizeof(g_last_error)];
+  memcpy(saved, g_last_error, sizeof(saved));
+  if (rece_plan_create(&cfg, &p) != RECE_OK) p = nullptr;
+  memcpy(g_last_error, saved, sizeof(saved));  // a shape it does not take is no error
+  if (p && !p->window_tc) {
+    rece_plan_destroy(p);
+    p = nullptr;
+  }
+  return p;
+}
+
+struct FullCeWindow {
+  rece_plan_t plan = nullptr;
+  ~FullCeWindow() { rece_plan_destroy(plan); }
+};
+
 }  // namespace
 
 void rece::set_last_error(const char* msg) { fail(RECE_OK, msg); }
@@ -470,7 +507,8 @@ rece_status_t rece_plan_create(const rece_config_t* cfg, rece_plan_t* out) {
   p->pos_plan = nullptr;
   // the tensor-core path groups each row's kept entries by slice of its window
   // (the selection's 16-bit histogram counts hold windows of fewer than 65536 items)
-  p->use_tc = tc_supported(*p) && p->w_max < 65536;
+  p->use_tc = tc_supported(*p) &&
+              (p->w_max < 65536 || (c.flags & RECE_FLAG_ALL_NEGATIVES) != 0);
   // dX on the tensor cores where gathering catalogue rows is the slow way: large d, or a
   // sorted catalogue that does not fit in half of L2; the merge groups each row's kept
   // entries by slice of its window for it
@@ -792,7 +830,12 @@ rece_status_t rece_full_ce_workspace_size(int64_t N, int64_t C, int32_t d, int32
                                           size_t* bytes) {
   if (!bytes || N < 0 || C < 1 || d < 1 || (mode != RECE_MODE_FP32_EXACT && mode != RECE_MODE_BF16))
     return fail(RECE_ERR_INVALID_ARG, "bad full-CE arguments");
-  *bytes = align256(2 * sizeof(uint32_t)) + align256(sizeof(float) * size_t(N));
+  FullCeWindow w;
+  w.plan = full_ce_window_plan(N, C, d, mode);
+  if (w.plan)
+    *bytes = align256(w.plan->lay.total) + align256(sizeof(uint16_t) * size_t(d));
+  else
+    *bytes = align256(2 * sizeof(uint32_t)) + align256(sizeof(float) * size_t(N));
   return RECE_OK;
 }
 
@@ -809,6 +852,17 @@ rece_status_t rece_full_ce_fwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
   if (!aligned16({X, Y})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
+  FullCeWindow w;
+  w.plan = full_ce_window_plan(N, C, d, mode);
+  if (w.plan) {  // tcgen05: the all-negatives kernels at one bucket, chunk and round
+    const size_t pb = align256(w.plan->lay.total);
+    char* B = ws + pb;
+    RECE_CUDA(cudaMemsetAsync(B, 0, sizeof(uint16_t) * size_t(d), st), "unit vector");
+    rece_status_t r = rece_bucketize_sort(w.plan, B, X, Y, ws, pb, stream);
+    if (r != RECE_OK) return r;
+    return rece_loss_fwd(w.plan, X, Y, targets, ws, pb, loss, row_loss, nullptr, lse, nullptr,
+                         stream);
+  }
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + align256(2 * sizeof(uint32_t)));
   RECE_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), st), "status reset");
@@ -837,6 +891,11 @@ rece_status_t rece_full_ce_bwd(int64_t N, int64_t C, int32_t d, int32_t mode, co
     return fail(RECE_ERR_INVALID_ARG, "NULL input or output");
   if (!aligned16({X, Y, dX, dY})) return fail(RECE_ERR_INVALID_ARG, kMisaligned);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FullCeWindow w;
+  w.plan = full_ce_window_plan(N, C, d, mode);
+  if (w.plan)  // the forward left the sorted copies and tables in the workspace
+    return rece_loss_bwd(w.plan, X, Y, targets, nullptr, lse, nullptr, dloss, workspace,
+                         align256(w.plan->lay.total), dX, dY, stream);
   if (mode == RECE_MODE_FP32_EXACT)
     RECE_CUDA(launch_full_ce_bwd(N, C, d, static_cast<const float*>(X),
                                  static_cast<const float*>(Y), targets, lse, dloss, dX, dY, st),

@@ -141,6 +141,31 @@ def test_full_ce_op_parity(dtype):
     assert max_rel(dY.cpu().numpy(), fY) <= TOL
 
 
+@pytest.mark.parametrize("N,C,d", [(333, 2049, 64), (200, 70_001, 64), (130, 3000, 256)])
+def test_full_ce_op_on_tensor_cores(N, C, d):
+    """bf16 with d a multiple of 64 up to 256: the fused exact full CE runs on tcgen05, as
+    the all-negatives mode at one bucket, one chunk and one round (every item in every
+    row's window, counted once; RECE equations 3 and 4).  Loss, row losses and lse within
+    1e-4; gradients within 1e-3 (the probabilities reach the tensor cores as hi + lo
+    bf16).  A catalogue past 2^16 items included."""
+    w = synth.Workload("fce_tc", N=N, C=C, d=d, dtype="bf16", n_b=1, n_c=1, n_ec=0, n_r=1,
+                       k=1, target_alpha=1.0)
+    X, Y, t = synth.make_inputs(w, seed=21)
+    Xd, Yd, td = to_dev(X, "bf16"), to_dev(Y, "bf16"), torch.from_numpy(t).cuda()
+    assert ops.full_ce_workspace_bytes(N, C, d, "bf16") > ops.full_ce_workspace_bytes(N, C, 40,
+                                                                                      "bf16")
+    loss, row, lse, ws = ops.full_ce_fwd(Xd, Yd, td)
+    o_loss, o_row, o_lse = oracle.full_ce_loss(X, Y, t)
+    assert abs(loss.item() - o_loss) <= TOL * o_loss
+    assert max_rel(row.cpu().numpy(), o_row) <= TOL
+    assert max_rel(lse.cpu().numpy(), o_lse) <= TOL
+    dX, dY = ops.full_ce_bwd(Xd, Yd, td, lse, torch.full((1,), 2.0, device="cuda"), ws)
+    fX, fY = oracle.full_ce_grad(X, Y, t, o_lse, 2.0)
+    assert max_rel(dX.cpu().numpy(), fX) <= 1e-3
+    assert max_rel(dY.cpu().numpy(), fY) <= 1e-3
+    assert ops.device_status(ws) == 0
+
+
 def test_empty_batch():
     w = synth.Workload("empty", N=0, C=100, d=8, dtype="fp32", n_b=4, n_c=5, n_ec=1, n_r=1, k=3)
     X = np.zeros((0, 8), np.float32)
