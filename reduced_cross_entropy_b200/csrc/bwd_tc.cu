@@ -623,6 +623,328 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
   }
 }
 
+// Persistent dY (slices of 256 columns of d): one CTA per SM loops over work items
+// (128 sorted catalogue positions x one slice of d), so the fixed cost of a CTA -- barrier
+// set-up, TMEM allocation, the first entry loads, the epilogue's tail -- is paid once per
+// SM instead of once per item, and one item's epilogue overlaps the next one's tiles and
+// MMAs: TMEM holds two accumulators (item parity), four epilogue warps drain one while the
+// MMAs fill the other, and stage their rows in a shared-memory area of their own.  The
+// builders, the TMA producer and the MMA issuer run the items' slabs through the rings
+// back to back.  Per item the computation is k_bwd_dy_tc's (each dY row written or added
+// by one CTA per launch, K in a fixed order): deterministic.
+constexpr int kPEpi = 128;                       // epilogue threads (warps 6-9)
+constexpr int kPThreads = kBuilders + 64 + kPEpi;
+constexpr int kPW = 32;                          // epilogue piece: 32 columns a row
+constexpr int kPStride = kPW * 4 + 16;           // staged row piece, padded by 16 B
+
+struct CtlP {
+  uint64_t bfull[kMaxBStages], bempty[kMaxBStages];
+  uint64_t afull[kAStages], aempty[kAStages];
+  uint64_t accfull[2], accempty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__host__ __device__ constexpr size_t smem_bytes_p(int nb, int ns) {
+  return 1024 + size_t(2 * kAStages) * kATile + size_t(nb) * ns * 128 +
+         size_t(2) * kPEpi * kPStride + sizeof(CtlP);
+}
+
+struct DyItem {
+  int64_t q0, k0, k1, lo;
+  int nK, n0;
+};
+__device__ __forceinline__ DyItem dy_item(int64_t it, int slices, int ns, int64_t N,
+                                          int64_t C, int n_c, int n_ec) {
+  DyItem g;
+  g.q0 = (it / slices) * kBM;
+  g.n0 = int(it % slices) * ns;
+  const int64_t last = (g.q0 + kBM - 1 < C - 1) ? g.q0 + kBM - 1 : C - 1;
+  const int64_t cf = chunk_of(g.q0, C, n_c), cl = chunk_of(last, C, n_c);
+  g.k0 = chunk_start(cf - n_ec < 0 ? 0 : cf - n_ec, N, n_c);
+  g.k1 = chunk_start(cl + n_ec + 1 > n_c ? n_c : cl + n_ec + 1, N, n_c);
+  g.lo = 0;
+  g.nK = 0;
+  if (g.k1 > g.k0) {
+    g.lo = g.k0 >> 6;
+    g.nK = int(((g.k1 + 63) >> 6) - g.lo);
+  }
+  return g;
+}
+
+__device__ __forceinline__ void on_timeout_p(CtlP& c, uint32_t* status) {
+  *reinterpret_cast<volatile int*>(&c.abort) = 1;
+  raise_flag(status, RECE_DEVICE_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kPThreads, 1) k_bwd_dy_tc_p(const __grid_constant__ CUtensorMap tmB,
+                                                          const Args a, int64_t items,
+                                                          int slices) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* A_hi = base;
+  uint8_t* A_lo = base + kAStages * kATile;
+  uint8_t* Bs = base + 2 * kAStages * kATile;
+  const uint32_t b_bytes = uint32_t(a.ns) * 128u;
+  uint8_t* stage = Bs + size_t(a.nb) * b_bytes;
+  CtlP& ctl = *reinterpret_cast<CtlP*>(stage + size_t(2) * kPEpi * kPStride);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  const int nb = a.nb, ns = a.ns;
+  const int64_t N = a.N, C = a.C;
+  const int r = a.r;
+
+  if (t == 0) {
+    for (int i = 0; i < nb; ++i) {
+      mbar_init(&ctl.bfull[i], 1);
+      mbar_init(&ctl.bempty[i], 1);
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&ctl.afull[i], kBuilders / 32);
+      mbar_init(&ctl.aempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl.accfull[i], 1);
+      mbar_init(&ctl.accempty[i], kPEpi / 32);
+    }
+    mbar_init(&ctl.done, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  const uint32_t tcols = ns <= 32 ? 64u : (ns <= 64 ? 128u : (ns <= 128 ? 256u : 512u));
+  if (warp == 4) {
+    tmem_alloc(&ctl.tmem_base, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmB);
+      uint32_t sg = 0;  // slabs issued so far (all items)
+      bool ok = true;
+      for (int64_t it = blockIdx.x; it < items && ok; it += gridDim.x) {
+        const DyItem g = dy_item(it, slices, ns, N, C, a.n_c, a.n_ec);
+        for (int s = 0; s < g.nK; ++s, ++sg) {
+          const int slot = int(sg % uint32_t(nb));
+          if (!mbar_wait(&ctl.bempty[slot], ((sg / nb) & 1u) ^ 1u, &ctl.abort, kTimeoutNs)) {
+            on_timeout_p(ctl, a.status);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl.bfull[slot], b_bytes);
+          for (int h = 0; h < ns; h += 64)  // boxes of 64 columns of d x 64 rows
+            tma_load_3d(Bs + size_t(slot) * b_bytes + size_t(h) * 128, &tmB, &ctl.bfull[slot],
+                        g.n0 + h, int((g.lo + s) * kBK), r);
+        }
+      }
+      for (uint32_t j = (sg > uint32_t(nb) ? sg - nb : 0); j < sg; ++j)
+        mbar_wait_limit(&ctl.bfull[j % nb], (j / nb) & 1u, kTimeoutNs);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32_bmn(kBM, ns);  // B (rows of d) MN-major
+      uint32_t sg = 0, il = 0;  // slabs consumed, items begun by this CTA
+      bool ok = true;
+      for (int64_t it = blockIdx.x; it < items && ok; it += gridDim.x, ++il) {
+        const DyItem g = dy_item(it, slices, ns, N, C, a.n_c, a.n_ec);
+        const int acc = int(il & 1u);
+        if (!mbar_wait(&ctl.accempty[acc], ((il >> 1) & 1u) ^ 1u, &ctl.abort, kTimeoutNs)) {
+          on_timeout_p(ctl, a.status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_acc = tmem + uint32_t(acc * ns);
+        for (int s = 0; s < g.nK; ++s, ++sg) {
+          const int as = int(sg % kAStages), bs = int(sg % uint32_t(nb));
+          if (!mbar_wait(&ctl.afull[as], (sg / kAStages) & 1u, &ctl.abort, kTimeoutNs) ||
+              !mbar_wait(&ctl.bfull[bs], (sg / nb) & 1u, &ctl.abort, kTimeoutNs)) {
+            on_timeout_p(ctl, a.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dh = desc_k_sw128(smem_u32(A_hi + as * kATile));
+          const uint64_t dl = desc_k_sw128(smem_u32(A_lo + as * kATile));
+          const uint64_t db0 = desc_mn_sw128(smem_u32(Bs + size_t(bs) * b_bytes), 8192u);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t db = db0 + 128u * kk;  // 16 K rows of 128 B per MMA
+            mma_bf16(d_acc, dh + 2 * kk, db, idesc, (s | kk) != 0);
+            mma_bf16(d_acc, dl + 2 * kk, db, idesc, 1);
+          }
+          mma_commit(&ctl.aempty[as]);
+          mma_commit(&ctl.bempty[bs]);
+        }
+        if (!ok) break;
+        mma_commit(&ctl.accfull[acc]);
+      }
+      mma_commit(&ctl.done);
+      mbar_wait_limit(&ctl.done, 0, kTimeoutNs);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ builders
+    // As in k_bwd_dy_tc: thread t owns row kc = t % 64 of every slab and the 64-position
+    // half t / 64 of the tile; it clears its row of both halves' tiles, all builders meet,
+    // then each writes its row's kept entries that fall in its half.  Every builder runs
+    // every item and slab to the named barriers, also after a timeout.
+    const int64_t rN = int64_t(r) * N;
+    const int kc = t & (kBK - 1);
+    const int half = t >> 6;
+    uint32_t sg = 0;
+    bool ok = true;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+      const DyItem g = dy_item(it, slices, ns, N, C, a.n_c, a.n_ec);
+      const int64_t slice = (g.q0 >> 6) + half;
+      int64_t wc = -1, wc_hi = 0, sig0 = 0;
+      int wS = 0;
+      auto set_chunk = [&](int64_t c) {
+        wc = c;
+        wc_hi = chunk_start(c + 1, N, a.n_c);
+        const int64_t w0 = chunk_start(c - a.n_ec < 0 ? 0 : c - a.n_ec, C, a.n_c);
+        const int64_t w1 =
+            chunk_start(c + a.n_ec + 1 > a.n_c ? a.n_c : c + a.n_ec + 1, C, a.n_c);
+        sig0 = w0 >> 6;
+        wS = w1 > w0 ? int((w1 - 1) >> 6) - int(sig0) + 1 : 0;
+      };
+      auto entry_range = [&](int s2, int& e0, int& e1) {
+        e0 = e1 = 0;
+        const int64_t p = (g.lo + s2) * kBK + kc;  // sorted row (grows with s2)
+        if (s2 >= g.nK || p < g.k0 || p >= g.k1 || p >= N) return;
+        if (wc < 0) set_chunk(chunk_of(p, N, a.n_c));
+        while (p >= wc_hi) set_chunk(wc + 1);
+        const int64_t idx = slice - sig0;
+        if (idx < 0 || idx >= wS) return;
+        const int32_t* off = a.kept_off + (rN + p) * a.Sp;
+        e0 = __ldg(off + idx);
+        e1 = __ldg(off + idx + 1);
+      };
+      constexpr int kPre = 16;
+      auto slab_entries = [&](int s2) { return a.kept + (rN + (g.lo + s2) * kBK + kc) * a.k; };
+      int a0, a1, b0, b1;
+      entry_range(0, a0, a1);
+      entry_range(1, b0, b1);
+      int2 pre[kPre];
+      {
+        const int2* ent = slab_entries(0);
+#pragma unroll
+        for (int u = 0; u < kPre; ++u)
+          pre[u] = a0 + u < a1 ? __ldg(ent + a0 + u) : make_int2(0, 0);
+      }
+      for (int s = 0; s < g.nK; ++s, ++sg) {
+        const int as = int(sg % kAStages);
+        if (ok && !mbar_wait(&ctl.aempty[as], ((sg / kAStages) & 1u) ^ 1u, &ctl.abort,
+                             kTimeoutNs)) {
+          on_timeout_p(ctl, a.status);
+          ok = false;
+        }
+        uint8_t* th = A_hi + as * kATile;
+        uint8_t* tl = A_lo + as * kATile;
+        if (ok) {
+          zero_row(th, t);
+          zero_row(tl, t);
+        }
+        named_barrier(1, kBuilders);  // the whole tile is clear before anyone fills it
+        int c0, c1;
+        entry_range(s + 2, c0, c1);
+        if (ok && a1 > a0) {
+#pragma unroll
+          for (int u = 0; u < kPre; ++u)
+            if (a0 + u < a1) put(th, tl, int(pre[u].x - g.q0), kc, uint32_t(pre[u].y));
+          const int2* ent = slab_entries(s);
+          for (int e = a0 + kPre; e < a1; e += 8) {
+            int2 en[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) en[u] = e + u < a1 ? __ldg(ent + e + u) : make_int2(0, 0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              if (e + u < a1) put(th, tl, int(en[u].x - g.q0), kc, uint32_t(en[u].y));
+          }
+        }
+        {
+          const int2* ent = slab_entries(s + 1);
+#pragma unroll
+          for (int u = 0; u < kPre; ++u)
+            pre[u] = b0 + u < b1 ? __ldg(ent + b0 + u) : make_int2(0, 0);
+        }
+        a0 = b0;
+        a1 = b1;
+        b0 = c0;
+        b1 = c1;
+        fence_proxy_async_smem();
+        named_barrier(1, kBuilders);  // nobody clears the next tile into this one's readers
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&ctl.afull[as]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int row = ((warp & 3) << 5) + lane;  // this thread's TMEM lane (tile row)
+    float* const buf0 = reinterpret_cast<float*>(stage + size_t(row) * kPStride);
+    float* const buf1 = reinterpret_cast<float*>(stage + size_t(kPEpi + row) * kPStride);
+    const float scale = a.dloss[0] / float(N);  // G holds p; g = p * dloss / N
+    uint32_t il = 0, piece = 0;
+    bool ok = true;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x, ++il) {
+      const DyItem g = dy_item(it, slices, ns, N, C, a.n_c, a.n_ec);
+      const int acc = int(il & 1u);
+      bool fin = ok && mbar_wait(&ctl.accfull[acc], (il >> 1) & 1u, &ctl.abort, kTimeoutNs);
+      fin = __all_sync(0xFFFFFFFFu, fin);
+      if (!fin) {
+        if (ok) on_timeout_p(ctl, a.status);
+        ok = false;
+        continue;
+      }
+      tc_fence_after();
+      const int64_t q = g.q0 + row;
+      const bool live = q < C;
+      const int64_t dst = live ? a.px[int64_t(r) * C + q] : 0;
+      float* o = a.out + dst * a.d + g.n0;
+      const uint32_t taddr = tmem + (uint32_t((warp & 3) * 32) << 16) + uint32_t(acc * ns);
+      for (int c0 = 0; c0 < ns; c0 += kPW, ++piece) {
+        float* srow = (piece & 1u) ? buf1 : buf0;
+        bulk_wait_read<1>();  // this thread's copy out of that buffer (two pieces ago)
+        float v[32];
+        if (g.nK == 0) {  // no rows cover the item: nothing accumulated (uniform)
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = 0.0f;
+        } else {
+          tmem_load32(taddr + uint32_t(c0), v);
+        }
+        float4* s4 = reinterpret_cast<float4*>(srow);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          s4[u] = make_float4(scale * v[4 * u], scale * v[4 * u + 1], scale * v[4 * u + 2],
+                              scale * v[4 * u + 3]);
+        if (live) {
+          fence_proxy_async_smem();
+          if (a.write)
+            bulk_store(o + c0, srow, uint32_t(kPW) * 4u);
+          else
+            bulk_reduce_add_f32(o + c0, srow, uint32_t(kPW) * 4u);
+          bulk_commit();
+        }
+      }
+      tc_fence_before();  // the accumulator's reads are done: the MMAs may refill it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.accempty[acc]);
+    }
+    bulk_wait_read<0>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, tcols);
+  }
+}
+
 // One warp per row: the positive's coefficient g_iz and dX_i = g_iz y_z (written, not
 // added: the rounds add after it).
 template <typename T>
@@ -790,11 +1112,37 @@ cudaError_t launch_dy_tc(const rece_plan_s& p, const float* dloss, char* ws, flo
   a.dloss = dloss;
   a.status = status;
   a.out = dY;
-  RECE_TRY(cudaFuncSetAttribute(k_bwd_dy_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(smem)));
   CUtensorMap tm;  // the sorted rows of X of every round, read MN-major
   RECE_TRY(make_tmap_bf16_3d(&tm, ws + L.xs, uint64_t(c.d), uint64_t(c.N), uint64_t(c.n_r),
                              uint32_t(kBK)));
+  if (ns == 256) {
+    // persistent: a CTA per SM over (position tile, slice) items, the B ring as deep as
+    // the shared memory left beside the G stages and the epilogue's staging allows (at
+    // the 4M-item workload, d = 256: 3.76 -> 2.79 ms; at d = 128 two CTAs of the
+    // per-item kernel share an SM and their builders outrun one persistent CTA's:
+    // 1.35 -> 2.01 ms there, so narrower slices keep k_bwd_dy_tc)
+    const size_t fixed = smem_bytes_p(0, ns);
+    int nbp = int((227 * 1024 - fixed) / (size_t(ns) * 128));
+    nbp = nbp > kMaxBStages ? kMaxBStages : nbp;
+    if (nbp >= 2) {
+      a.nb = nbp;
+      const size_t smem_p = smem_bytes_p(nbp, ns);
+      RECE_TRY(cudaFuncSetAttribute(k_bwd_dy_tc_p, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(smem_p)));
+      const int64_t items = ceil_div(c.C, kBM) * slices;
+      const int grid = int(items < sm_count() ? items : sm_count());
+      for (int r = 0; r < c.n_r; ++r) {
+        a.r = r;
+        a.write = r == 0;
+        k_bwd_dy_tc_p<<<grid, kPThreads, smem_p, st>>>(tm, a, items, slices);
+        count_launches(1);
+        RECE_TRY(cudaGetLastError());
+      }
+      return cudaSuccess;
+    }
+  }
+  RECE_TRY(cudaFuncSetAttribute(k_bwd_dy_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(smem)));
   for (int r = 0; r < c.n_r; ++r) {
     a.r = r;
     a.write = r == 0;
