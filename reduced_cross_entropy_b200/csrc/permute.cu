@@ -19,21 +19,38 @@ __global__ void __launch_bounds__(256) k_permute_rows(const uint4* __restrict__ 
                                                       int n_r, int n_c, uint4* __restrict__ Vs,
                                                       int32_t* __restrict__ inv,
                                                       int32_t* __restrict__ chunk) {
+  // a warp copies kRows rows at a time, all their loads in flight before the stores
+  // (one row of d <= 256 bf16 is one 16-byte vector per lane or less)
+  constexpr int kRows = 4;
   const int lane = threadIdx.x & 31;
   const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
   const int64_t total = int64_t(n_r) * M;
-  for (int64_t w = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total;
-       w += warps) {
-    const int64_t r = w / M, p = w % M;
-    const int32_t id = perm[w];
+  for (int64_t w0 = (int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kRows;
+       w0 < total; w0 += warps * kRows) {
+    int32_t id[kRows];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) id[u] = w0 + u < total ? perm[w0 + u] : 0;
     if (Vs) {  // (no copy wanted: the inverse order and chunks only)
-      const uint4* src = V + int64_t(id) * vec_per_row;
-      uint4* dst = Vs + w * vec_per_row;
-      for (int c = lane; c < vec_per_row; c += 32) dst[c] = src[c];
+      for (int c0 = 0; c0 < vec_per_row; c0 += 32) {
+        const int c = c0 + lane;
+        uint4 v[kRows];
+#pragma unroll
+        for (int u = 0; u < kRows; ++u)
+          if (w0 + u < total && c < vec_per_row) v[u] = V[int64_t(id[u]) * vec_per_row + c];
+#pragma unroll
+        for (int u = 0; u < kRows; ++u)
+          if (w0 + u < total && c < vec_per_row) Vs[(w0 + u) * vec_per_row + c] = v[u];
+      }
     }
-    if (lane == 0) {
-      if (inv) inv[r * M + id] = int32_t(p);
-      if (chunk) chunk[r * M + id] = int32_t((p * n_c) / M);
+    if (lane < kRows && w0 + lane < total) {
+      const int64_t w = w0 + lane;
+      const int64_t r = w / M, p = w % M;
+      int32_t myid = id[0];
+#pragma unroll
+      for (int u = 1; u < kRows; ++u)
+        if (lane == u) myid = id[u];
+      if (inv) inv[r * M + myid] = int32_t(p);
+      if (chunk) chunk[r * M + myid] = int32_t((p * n_c) / M);
     }
   }
 }
@@ -45,7 +62,7 @@ cudaError_t launch_permute_rows(const void* V, int64_t M, int d, const int32_t* 
                                 cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const int64_t rows = int64_t(n_r) * M;
-  const int64_t want = (rows + 7) / 8;
+  const int64_t want = (rows + 31) / 32;  // 8 warps of 4 rows a block
   const int grid = int(want < 8 * 148 ? want : 8 * 148);
   k_permute_rows<<<grid, 256, 0, st>>>(static_cast<const uint4*>(V), M, d / 8, perm, n_r, n_c,
                                        static_cast<uint4*>(Vs), inv, chunk);

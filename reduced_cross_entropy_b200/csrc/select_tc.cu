@@ -466,7 +466,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
                   if (emitted < Qw) out[emitted] = make_int2(__float_as_int(val), qa + u);
                   ++emitted;
                   if (kSampled) {
-                    const uint32_t fb = (ord_key(val) - thr_key) >> 20;
+                    // (a -0 score passing a +0 threshold has the lower key: bin 0)
+                    const uint32_t kv = ord_key(val);
+                    const uint32_t fb = kv > thr_key ? (kv - thr_key) >> 20 : 0u;
                     bin_add(fcol, fb < kFineBins - 1 ? fb : uint32_t(kFineBins - 1));
                   }
                 } while (mask);
