@@ -579,7 +579,8 @@ constexpr int kSeg = 32;  // pairs per segment of a run
 // 32 pairs of a run, 256 columns of d), eight pairs' rows in flight, pairs in order; a run
 // of one segment adds its sum into the item's row, a longer run leaves each segment's sum
 // in part[first position of the segment].  Level 2 (k_pos_dy_runs): the run's first
-// position adds the parts in order.  Deterministic.
+// position adds the parts into eight partial sums (part u, u + 8, ...) and those in a
+// fixed tree.  Deterministic.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_pos_dy_seg(
     const T* __restrict__ X, int64_t C, int d, int slots, const int32_t* __restrict__ key,
@@ -638,10 +639,17 @@ __global__ void __launch_bounds__(kThreads) k_pos_dy_runs(
   const int32_t j = key[p];
   const int64_t r1 = run_hi[p];
   if (j >= C || run_lo[p] != p || r1 - p <= kSeg) return;
+  // eight parts' loads in flight at a time, into eight partial sums added in a fixed tree
+  // (a Zipf-drawn target's run holds thousands of positives: hundreds of parts)
   for (int t = blockIdx.y * 256 + lane; t < d && t < int(blockIdx.y + 1) * 256; t += 32) {
-    float sum = 0.0f;
-    for (int64_t q = p; q < r1; q += kSeg) sum += part[q * d + t];
-    dY[int64_t(j) * d + t] += sum;
+    float s[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    int64_t q = p;
+    for (; q + 7 * kSeg < r1; q += 8 * kSeg) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s[u] += part[(q + u * kSeg) * d + t];
+    }
+    for (; q < r1; q += kSeg) s[0] += part[q * d + t];
+    dY[int64_t(j) * d + t] += ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
   }
 }
 

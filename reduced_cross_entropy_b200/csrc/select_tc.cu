@@ -383,6 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
             const int bstar = cut_bin(s.hist, row_local, want);
             if (bstar >= 0) thr = cut_threshold(bmap, uint32_t(bstar + 1) << 20);
           }
+          // a zero threshold as -0: every score that passes it (+0 and -0 included) then
+          // has an order key at or above thr_key, so the fine bins below never wrap
+          if (thr == 0.0f) thr = -0.0f;
           thr_key = ord_key(thr);
           if (kSampled && wg == 0)
             for (int b = 0; b < kFineBins / 2; ++b) s.fine[b][row_local] = 0;
@@ -466,9 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_select_tc(
                   if (emitted < Qw) out[emitted] = make_int2(__float_as_int(val), qa + u);
                   ++emitted;
                   if (kSampled) {
-                    // (a -0 score passing a +0 threshold has the lower key: bin 0)
-                    const uint32_t kv = ord_key(val);
-                    const uint32_t fb = kv > thr_key ? (kv - thr_key) >> 20 : 0u;
+                    const uint32_t fb = (ord_key(val) - thr_key) >> 20;
                     bin_add(fcol, fb < kFineBins - 1 ? fb : uint32_t(kFineBins - 1));
                   }
                 } while (mask);
