@@ -133,6 +133,8 @@ def stage_bound(stage, paths):
     from reduced_cross_entropy_b200 import _lib
     if stage in ("bucketize", "select"):
         return "tensor" if paths & _lib.PATH_TENSOR_CORES else "alu"
+    if paths & _lib.PATH_ALL_NEGATIVES and paths & _lib.PATH_WINDOW_FMA:
+        return "alu" if stage in ("select", "bwd_rows", "bwd_items") else "hbm"
     if stage in ("bwd_rows", "bwd_items") and paths & _lib.PATH_ALL_NEGATIVES:
         return "tensor"
     if stage == "bwd_rows" and paths & _lib.PATH_DX_TENSORS:
@@ -166,6 +168,9 @@ def kernel_sources(stage, paths):
                    merge_loss=["window.cu"],
                    bwd_rows=["backward.cu", "window_tc.cu", "tc_common.cu"],
                    bwd_sort=["sort.cu", "rece_abi.cu"], bwd_items=["window_tc.cu"])
+        if paths & _lib.PATH_WINDOW_FMA:
+            src.update(select=["window_fma.cu", "window.cu"],
+                       bwd_rows=["backward.cu", "window_fma.cu"], bwd_items=["window_fma.cu"])
     return src[stage]
 
 
