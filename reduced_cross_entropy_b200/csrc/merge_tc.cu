@@ -114,6 +114,7 @@ struct MergeArgs {
   const int32_t* targets;
   const int32_t* py;
   const int32_t* invX;
+  const int32_t* invY;  // sorted position of each item, per round
   const int32_t* chunkY;
   const int2* list;
   const int4* list_count;
@@ -465,6 +466,425 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc_spill(const MergeArgs<T> 
     merge_row<T, kGrouped, kGather>(A, A.spill_rows[w], sh_cnt[wid], keys, poss, cap, false);
 }
 
+// ---------------------------------------------------------------- one row per CTA
+// The same merge with the row's work spread over four warps: warp w reads sub-list w of
+// every round (the entries of selection warpgroup w) into its own shared-memory region,
+// the k-th key is found with 8-bit digits over a shared 256-bin histogram, and in grouped
+// mode the kept entries of a round go out ordered by sorted position (a bit map of the
+// round's window: an entry's place is the count of kept positions before it), which
+// groups them by 64-position slice with no sort.  Without grouping they go out by round,
+// then warp, lane and place in the region.  Every sum is taken in a fixed order.  A row
+// whose entries do not fit a warp's region is handed to the spill list (the warp-per-row
+// path above finishes it).
+constexpr int kCtaThreads = 128;
+constexpr int kCtaWarps = kCtaThreads / 32;
+constexpr int kGatherCta = 4;  // list entries per lane in flight
+
+struct CtaShared {
+  uint32_t u[kCtaWarps][3];  // per warp: or, and, largest of its keys
+  int cnt[kCtaWarps];        // per warp: entries that passed (uncapped)
+  int rb[kCtaWarps][9];      // per warp: where each round's entries start in its region
+  float f[kCtaWarps][3];     // per warp: positive-logit part, sum of exponentials, worst
+  int scan[kCtaWarps];       // warp totals of a block scan
+  int res[3];                // selection pass: digit, keys above it, keys in it
+  int px[8], cx[8];          // the row's sorted position and chunk, per round
+};
+
+struct CtaSel {
+  uint32_t T;
+  int need;
+  int eq;
+};
+
+// Exclusive scan of v over the block (thread order); total gets the sum.  Starts and ends
+// with every thread past a barrier, so cs.scan may be reused right after.
+__device__ __forceinline__ int cta_excl_scan(int v, CtaShared& cs, int& total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) cs.scan[wid] = incl;
+  __syncthreads();
+  int base = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kCtaWarps; ++w) {
+    base += w < wid ? cs.scan[w] : 0;
+    all += cs.scan[w];
+  }
+  total = all;
+  __syncthreads();
+  return base + incl - v;
+}
+
+// The want-th largest (1-based) of the keys in play over the four warps' regions
+// (get(q, key) -> in play, its key; q < nq in this warp's region); orv / andv / m: the OR,
+// AND and count of those keys.  Digits of 8 bits from the highest bit in which the keys
+// differ; same result convention as warp_select_kth.
+template <typename Get>
+__device__ CtaSel cta_select_kth(int nq, int want, uint32_t orv, uint32_t andv, int m, Get get,
+                                 uint32_t* hist, CtaShared& cs) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t diff = orv ^ andv;
+  if (diff == 0u) return CtaSel{andv, want, m};
+  const int hb = 31 - __clz(diff);
+  int shift = hb >= 7 ? hb - 7 : 0;
+  uint32_t pmask = shift + 8 >= 32 ? 0u : ~((1u << (shift + 8)) - 1u);
+  uint32_t prefix = andv & pmask;
+  for (;;) {
+    hist[tid] = 0u;
+    hist[tid + kCtaThreads] = 0u;
+    __syncthreads();
+    for (int q = lane; q < nq; q += 32) {
+      uint32_t key;
+      if (get(q, key) && (key & pmask) == prefix)
+        atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    // thread t: digits 255 - 2t and 254 - 2t, i.e. the digits in descending order
+    const int c0 = int(hist[255 - 2 * tid]), c1 = int(hist[254 - 2 * tid]);
+    int total;
+    const int excl = cta_excl_scan(c0 + c1, cs, total);
+    if (excl < want && want <= excl + c0) {
+      cs.res[0] = 255 - 2 * tid;
+      cs.res[1] = excl;
+      cs.res[2] = c0;
+    } else if (excl + c0 < want && want <= excl + c0 + c1) {
+      cs.res[0] = 254 - 2 * tid;
+      cs.res[1] = excl + c0;
+      cs.res[2] = c1;
+    }
+    __syncthreads();
+    const int dg = cs.res[0], above = cs.res[1], count = cs.res[2];
+    want -= above;
+    // (a digit below 8 bits wide at the bottom overlaps bits the prefix already fixed;
+    // every key counted agrees with the prefix there, so the OR changes nothing there)
+    prefix |= uint32_t(dg) << shift;
+    pmask |= 255u << shift;
+    if (count == want || shift == 0) return CtaSel{prefix, want, count};
+    shift = shift >= 8 ? shift - 8 : 0;
+  }
+}
+
+template <typename T, bool kGrouped>
+__global__ void __launch_bounds__(kCtaThreads, 8) k_merge_cta(const MergeArgs<T> A, int capw) {
+  extern __shared__ __align__(16) uint8_t sh_raw[];
+  __shared__ CtaShared cs;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int64_t i = blockIdx.x;
+  const int64_t N = A.N, C = A.C;
+  const int k = A.k, n_r = A.n_r, n_c = A.n_c, n_ec = A.n_ec, Qw = A.Qw, Sp = A.Sp;
+  const int32_t* __restrict__ py = A.py;
+  const int32_t* __restrict__ invX = A.invX;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sh_raw) + size_t(wid) * 2 * capw;
+  int32_t* poss = reinterpret_cast<int32_t*>(keys + capw);
+  uint32_t* aux = reinterpret_cast<uint32_t*>(sh_raw) + size_t(kCtaWarps) * 2 * capw;
+  const int aux_words = kGrouped && 2 * Sp > 256 ? 2 * Sp : 256;
+  int32_t* sliceoff = reinterpret_cast<int32_t*>(aux + aux_words);
+
+  const int32_t z = A.targets[i];
+  const bool z_ok = z >= 0 && z < C;
+  // the row's sorted position and chunk in each round
+  if (tid < n_r) {
+    const int px = invX[int64_t(tid) * N + i];
+    cs.px[tid] = px;
+    cs.cx[tid] = int((int64_t(px) * n_c) / N);
+  }
+  __syncthreads();
+
+  // 1. this warp's sub-list of every round: entries above the round's theta, not the
+  //    positive, not in an earlier round's window; their keys and sorted positions
+  int n = 0;
+  uint32_t orv = 0u, andv = 0xFFFFFFFFu, kmax = 0u;
+  bool over = false;
+  float theta_max = -INFINITY;
+  for (int r = 0; r < n_r; ++r) {
+    if (lane == 0) cs.rb[wid][r] = n < capw ? n : capw;
+    const int64_t rp = int64_t(r) * N + cs.px[r];
+    const int4 c4 = A.list_count[rp];
+    const float th = A.list_theta[rp];
+    theta_max = fmaxf(theta_max, th);
+    over |= c4.x > Qw || c4.y > Qw || c4.z > Qw || c4.w > Qw;
+    const int cw0 = wid == 0 ? c4.x : wid == 1 ? c4.y : wid == 2 ? c4.z : c4.w;
+    const int cw = cw0 < Qw ? cw0 : Qw;
+    const int32_t pz = z_ok ? A.invY[int64_t(r) * C + z] : -1;
+    const int2* L = A.list + (rp * 4 + wid) * Qw;
+    for (int a0 = 0; a0 < cw; a0 += 32 * kGatherCta) {
+      int2 e[kGatherCta];
+      bool keep[kGatherCta];
+#pragma unroll
+      for (int u = 0; u < kGatherCta; ++u) {
+        const int a = a0 + 32 * u + lane;
+        e[u] = a < cw ? L[a] : make_int2(0, 0);
+        keep[u] = a < cw && __int_as_float(e[u].x) > th && e[u].y != pz;
+      }
+      if (r > 0) {  // an item an earlier round's window held was that round's to select
+#pragma unroll
+        for (int u = 0; u < kGatherCta; ++u) {
+          const int32_t jj = keep[u] ? py[int64_t(r) * C + e[u].y] : 0;
+          for (int q = 0; q < r && keep[u]; ++q) {
+            const int dc = A.chunkY[int64_t(q) * C + jj] - cs.cx[q];
+            if (dc >= -n_ec && dc <= n_ec) keep[u] = false;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherCta; ++u) {
+        const unsigned b = __ballot_sync(0xFFFFFFFFu, keep[u]);
+        if (keep[u]) {
+          const int at = n + __popc(b & ((1u << lane) - 1u));
+          const uint32_t key = score_key(__int_as_float(e[u].x));
+          if (at < capw) {
+            keys[at] = key;
+            poss[at] = e[u].y;
+          }
+          orv |= key;
+          andv &= key;
+          kmax = key > kmax ? key : kmax;
+        }
+        n += __popc(b);
+      }
+    }
+  }
+  // the positive's logit, over the block
+  float part = 0.0f;
+  if (z_ok) {
+    const T* x = A.X + i * A.d;
+    const T* y = A.Y + int64_t(z) * A.d;
+    for (int t = tid; t < A.d; t += kCtaThreads) part = fmaf(to_f32(x[t]), to_f32(y[t]), part);
+  }
+  part = warp_sum(part);
+  orv = warp_or(orv);
+  andv = warp_and(andv);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t v = __shfl_xor_sync(0xFFFFFFFFu, kmax, o);
+    kmax = v > kmax ? v : kmax;
+  }
+  if (lane == 0) {
+    cs.rb[wid][n_r] = n < capw ? n : capw;
+    cs.cnt[wid] = n;
+    cs.u[wid][0] = orv;
+    cs.u[wid][1] = andv;
+    cs.u[wid][2] = kmax;
+    cs.f[wid][0] = part;
+  }
+  __syncthreads();
+  int ntot = 0;
+  bool spill = false;
+  float lp = 0.0f;
+  orv = 0u;
+  andv = 0xFFFFFFFFu;
+  kmax = 0u;
+#pragma unroll
+  for (int w = 0; w < kCtaWarps; ++w) {
+    ntot += cs.cnt[w];
+    spill |= cs.cnt[w] > capw;
+    lp += cs.f[w][0];
+    if (cs.cnt[w] > 0) {
+      orv |= cs.u[w][0];
+      andv &= cs.u[w][1];
+      kmax = cs.u[w][2] > kmax ? cs.u[w][2] : kmax;
+    }
+  }
+  if (spill) {  // (the whole block leaves)
+    if (tid == 0) A.spill_rows[atomicAdd(A.spill_count, 1u)] = int32_t(i);
+    return;
+  }
+  const int* rbw = cs.rb[wid];  // (not written again)
+  const int nq = rbw[n_r];
+  auto item_of = [&](int q) {
+    int r = 0;
+    while (r + 1 < n_r && q >= rbw[r + 1]) ++r;
+    return py[int64_t(r) * C + poss[q]];
+  };
+
+  // 2. the k best
+  const int kk = k < ntot ? k : ntot;
+  const bool all = kk >= ntot;
+  CtaSel s1{0u, 0, 0}, s2{0u, 0, 0};
+  bool tie = false;
+  if (!all) {
+    s1 = cta_select_kth(
+        nq, kk, orv, andv, ntot, [&](int q, uint32_t& key) { key = keys[q]; return true; }, aux,
+        cs);
+    if (s1.need != s1.eq) {
+      tie = true;
+      const uint32_t Tk = s1.T;
+      uint32_t o2 = 0u, a2 = 0xFFFFFFFFu;
+      int m2 = 0;
+      for (int q = lane; q < nq; q += 32)
+        if (keys[q] == Tk) {
+          const uint32_t v = ~uint32_t(item_of(q));
+          o2 |= v;
+          a2 &= v;
+          ++m2;
+        }
+      o2 = warp_or(o2);
+      a2 = warp_and(a2);
+      m2 = int(warp_sum(float(m2)));
+      __syncthreads();  // cs.u was read above by every thread
+      if (lane == 0) {
+        cs.u[wid][0] = o2;
+        cs.u[wid][1] = a2;
+        cs.cnt[wid] = m2;
+      }
+      __syncthreads();
+      o2 = 0u;
+      a2 = 0xFFFFFFFFu;
+      m2 = 0;
+#pragma unroll
+      for (int w = 0; w < kCtaWarps; ++w) {
+        m2 += cs.cnt[w];
+        if (cs.cnt[w] > 0) {
+          o2 |= cs.u[w][0];
+          a2 &= cs.u[w][1];
+        }
+      }
+      s2 = cta_select_kth(
+          nq, s1.need, o2, a2, m2,
+          [&](int q, uint32_t& key) {
+            if (keys[q] != Tk) return false;
+            key = ~uint32_t(item_of(q));
+            return true;
+          },
+          aux, cs);
+    }
+  }
+  auto take = [&](int q) {
+    const uint32_t key = keys[q];
+    return all || key > s1.T || (key == s1.T && (!tie || ~uint32_t(item_of(q)) >= s2.T));
+  };
+
+  // 3. the row's loss (RECE, Algorithm 1's loss lines); the best candidate is always kept
+  const float best = ntot > 0 ? key_score(kmax) : -INFINITY;
+  const float m = fmaxf(lp, best);
+  float acc = 0.0f, worst = INFINITY;
+  for (int q = lane; q < nq; q += 32)
+    if (take(q)) {
+      const float sc = key_score(keys[q]);
+      acc += expf(sc - m);
+      worst = fminf(worst, sc);
+    }
+  acc = warp_sum(acc);
+  worst = warp_max(-worst);
+  if (lane == 0) {
+    cs.f[wid][1] = acc;
+    cs.f[wid][2] = worst;
+  }
+  __syncthreads();
+  float sum = 0.0f;
+  worst = INFINITY;
+#pragma unroll
+  for (int w = 0; w < kCtaWarps; ++w) {
+    sum += cs.f[w][1];
+    worst = fminf(worst, -cs.f[w][2]);
+  }
+  const float lse = m + logf(sum + expf(lp - m));
+
+  // 4. the kept entries, round by round
+  float* lg = A.logits ? A.logits + i * (int64_t(k) + 1) : nullptr;
+  int32_t* srow = A.selected + i * k;
+  int ns = 0;
+  for (int r = 0; r < n_r; ++r) {
+    const int px = cs.px[r];
+    if constexpr (kGrouped) {
+      // ordered by sorted position: a bit per position of the round's window, from the
+      // start of its first 64-position slice
+      const int64_t c = cs.cx[r];
+      const int64_t w0 = chunk_start(c - n_ec < 0 ? 0 : c - n_ec, C, n_c);
+      const int64_t w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
+      const int sig0 = int(w0 >> 6);
+      const int S = w1 > w0 ? int((w1 - 1) >> 6) - sig0 + 1 : 0;
+      const int32_t base = sig0 << 6;
+      uint32_t* bits = aux;
+      for (int b = tid; b < 2 * S; b += kCtaThreads) bits[b] = 0u;
+      __syncthreads();
+      for (int q = rbw[r] + lane; q < rbw[r + 1]; q += 32)
+        if (take(q)) {
+          const int o = poss[q] - base;
+          atomicOr(&bits[o >> 5], 1u << (o & 31));
+        }
+      __syncthreads();
+      // slices [t*B, t*B + B) per thread: counts, then their starts
+      const int B = (S + kCtaThreads - 1) / kCtaThreads;
+      const int s0 = tid * B, s1e = s0 + B < S ? s0 + B : S;
+      int run = 0;
+      for (int s = s0; s < s1e; ++s) run += __popc(bits[2 * s]) + __popc(bits[2 * s + 1]);
+      int total;
+      int at = cta_excl_scan(run, cs, total);
+      const int64_t rp = int64_t(r) * N + px;
+      int32_t* orow = A.kept_off + rp * Sp;
+      for (int s = s0; s < s1e; ++s) {
+        sliceoff[s] = at;
+        orow[s] = at;
+        at += __popc(bits[2 * s]) + __popc(bits[2 * s + 1]);
+      }
+      if (tid == 0) orow[S] = total;
+      __syncthreads();
+      int2* erow = A.kept + rp * k;
+      for (int q = rbw[r] + lane; q < rbw[r + 1]; q += 32) {
+        if (!take(q)) continue;
+        const int32_t pos = poss[q];
+        const int o = pos - base, wi = o >> 5;
+        const int dest = sliceoff[o >> 6] + __popc(bits[wi] & ((1u << (o & 31)) - 1u)) +
+                         ((wi & 1) ? __popc(bits[wi - 1]) : 0);
+        const float sc = key_score(keys[q]);
+        uint32_t packed = 0u;
+        if (z_ok) {
+          const float pr = expf(sc - lse);
+          const __nv_bfloat16 h = __float2bfloat16_rn(pr);
+          const __nv_bfloat16 l = __float2bfloat16_rn(pr - __bfloat162float(h));
+          packed = uint32_t(__bfloat16_as_ushort(h)) | (uint32_t(__bfloat16_as_ushort(l)) << 16);
+        }
+        erow[dest] = make_int2(pos, int32_t(packed));
+        srow[ns + dest] = py[int64_t(r) * C + pos];
+        if (lg) lg[1 + ns + dest] = sc;
+      }
+      ns += total;
+      __syncthreads();  // the bit map is cleared again by the next round
+    } else {
+      int mine = 0;
+      for (int q = rbw[r] + lane; q < rbw[r + 1]; q += 32) mine += take(q) ? 1 : 0;
+      int total;
+      int at = ns + cta_excl_scan(mine, cs, total);
+      for (int q = rbw[r] + lane; q < rbw[r + 1]; q += 32) {
+        if (!take(q)) continue;
+        const float sc = key_score(keys[q]);
+        srow[at] = py[int64_t(r) * C + poss[q]];
+        if (lg) lg[1 + at] = sc;
+        ++at;
+      }
+      ns += total;
+    }
+  }
+  for (int a = ns + tid; a < k; a += kCtaThreads) {
+    srow[a] = -1;
+    if (lg) lg[1 + a] = -INFINITY;
+  }
+  if (tid == 0) {
+    if (lg) lg[0] = z_ok ? lp : NAN;
+    if (kGrouped) A.pos_logit[i] = z_ok ? lp : NAN;
+    // exactness: theta_max is the largest score some round did not emit
+    const float s_k = ns < k ? -INFINITY : worst;
+    if (over || (theta_max > -INFINITY && theta_max >= s_k)) {
+      atomicAdd(A.status + 1, 1u);
+      if (over) atomicAdd(A.status + 2, 1u);
+      raise_flag(A.status, RECE_DEVICE_INEXACT);
+    }
+    if (!z_ok) {
+      raise_flag(A.status, RECE_DEVICE_BAD_TARGET);
+      A.lse_out[i] = NAN;
+      if (A.row_loss) A.row_loss[i] = NAN;
+    } else {
+      A.lse_out[i] = lse;
+      if (A.row_loss) A.row_loss[i] = lse - lp;
+    }
+  }
+}
+
 }  // namespace
 
 int tc_list_capacity(int k);
@@ -484,10 +904,35 @@ size_t merge_tc_warp_bytes(int n_r, int k) {
   return size_t(merge_tc_cap(n_r, k)) * 8 + kCountBytes;
 }
 
+// One-row-per-CTA path: the 256-bin histogram, which the grouped output's bit map (two
+// words per slice) reuses, and the slice starts; then each warp's region for the entries
+// of its sub-lists that pass, as large as eight CTAs per SM allow (the registers allow
+// eight), but never more than the sub-lists can hold.  The path is taken when k >= 512
+// (smaller rows are done faster a warp each, more rows in flight) and the region holds at
+// least a quarter of the warp path's buffer plus 32 (the sub-lists hold every fourth tile
+// of the window, so their shares stay close to a quarter).
+constexpr size_t kCtaSmemBudget = 26 * 1024;
+size_t merge_cta_aux_bytes(int Sp) {
+  const size_t aux = 2 * size_t(Sp) > 256 ? 2 * size_t(Sp) : 256;
+  return aux * 4 + size_t(Sp) * 4;
+}
+int merge_cta_region(int n_r, int k, int Sp) {
+  const size_t aux = merge_cta_aux_bytes(Sp);
+  if (aux >= kCtaSmemBudget) return 0;
+  const int64_t fit = int64_t((kCtaSmemBudget - aux) / (size_t(kCtaWarps) * 8));
+  const int64_t most = int64_t(n_r) * tc_sublist_capacity(k);
+  const int64_t want = int64_t(n_r) * ((k + k / 4 + 64 + 3) / 4) + 32;
+  if (k < 512 || fit < want) return 0;
+  return int(fit < most ? fit : most);
+}
+size_t merge_cta_smem(int capw, int Sp) {
+  return size_t(kCtaWarps) * 8 * size_t(capw) + merge_cta_aux_bytes(Sp);
+}
+
 template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
-                            const int32_t* py, const int32_t* invX, const int32_t* chunkY,
-                            const int2* list, const int4* list_count,
+                            const int32_t* py, const int32_t* invX, const int32_t* invY,
+                            const int32_t* chunkY, const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, int2* kept,
                             int32_t* kept_off, float* pos_logit, int Sp, float* lse,
                             float* row_loss, float* logits, uint32_t* status, int32_t* spill_rows,
@@ -500,6 +945,7 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   A.targets = targets;
   A.py = py;
   A.invX = invX;
+  A.invY = invY;
   A.chunkY = chunkY;
   A.list = list;
   A.list_count = list_count;
@@ -523,21 +969,29 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   A.status = status;
   A.spill_rows = spill_rows;
   A.spill_count = status + 3;
-  const int cap = merge_tc_cap(c.n_r, c.k);
-  const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
-  int warps = int((200 * 1024) / per_warp);
-  warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
-  const size_t smem = per_warp * warps;
   const bool grouped = kept != nullptr;
   const bool wide = c.k >= 384;
-  auto kern = grouped ? (wide ? k_merge_tc<T, true, 8> : k_merge_tc<T, true, 4>)
-                      : (wide ? k_merge_tc<T, false, 8> : k_merge_tc<T, false, 4>);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  cudaError_t e = cudaMemsetAsync(A.spill_count, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(A.spill_count, 0, sizeof(uint32_t), st);
-  if (e != cudaSuccess) return e;
-  kern<<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(A, cap);
+  const int capw = merge_cta_region(c.n_r, c.k, grouped ? Sp : 0);
+  const size_t cta_smem = merge_cta_smem(capw, grouped ? Sp : 0);
+  if (invY && capw > 0) {
+    auto kern = grouped ? k_merge_cta<T, true> : k_merge_cta<T, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(cta_smem));
+    if (e != cudaSuccess) return e;
+    kern<<<unsigned(c.N), kCtaThreads, cta_smem, st>>>(A, capw);
+  } else {
+    const int cap = merge_tc_cap(c.n_r, c.k);
+    const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
+    int warps = int((200 * 1024) / per_warp);
+    warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
+    const size_t smem = per_warp * warps;
+    auto kern = grouped ? (wide ? k_merge_tc<T, true, 8> : k_merge_tc<T, true, 4>)
+                        : (wide ? k_merge_tc<T, false, 8> : k_merge_tc<T, false, 4>);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<unsigned(ceil_div(c.N, warps)), warps * 32, smem, st>>>(A, cap);
+  }
   auto spill = grouped ? (wide ? k_merge_tc_spill<T, true, 8> : k_merge_tc_spill<T, true, 4>)
                        : (wide ? k_merge_tc_spill<T, false, 8> : k_merge_tc_spill<T, false, 4>);
   spill<<<kSpillWarps / (kThreads / 32), kThreads, 0, st>>>(
@@ -548,7 +1002,8 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
 
 template cudaError_t launch_merge_tc<__nv_bfloat16>(
     const rece_plan_s&, const __nv_bfloat16*, const __nv_bfloat16*, const int32_t*,
-    const int32_t*, const int32_t*, const int32_t*, const int2*, const int4*, const float*,
+    const int32_t*, const int32_t*, const int32_t*, const int32_t*, const int2*, const int4*,
+    const float*,
     int32_t*, int2*, int32_t*, float*, int, float*, float*, float*, uint32_t*, int32_t*, void*,
     cudaStream_t);
 

@@ -189,6 +189,7 @@ void build_layout(rece_plan_s& p) {
     if (!p.tc_dx) L.ys = take(sizeof(uint16_t) * size_t(tc_ys_rows(int64_t(c.n_r) * c.C)) * c.d);
     L.inv_x = take(sizeof(int32_t) * c.n_r * c.N);
     L.chunk_y = take(sizeof(int32_t) * c.n_r * c.C);
+    L.inv_y = take(sizeof(int32_t) * c.n_r * c.C);  // the merge's test for the positive
     L.tc_list = take(sizeof(int2) * size_t(c.n_r) * c.N * Q);
     L.tc_count = take(sizeof(int4) * c.n_r * c.N);
     L.tc_theta = take(sizeof(float) * c.n_r * c.N);
@@ -709,7 +710,8 @@ rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X
                                   reinterpret_cast<int32_t*>(ws + L.inv_x), nullptr, st),
               "permute X");
     RECE_CUDA(launch_permute_rows(Y, c.C, c.d, reinterpret_cast<const int32_t*>(ws + L.py),
-                                  c.n_r, c.n_c, ws + L.ys, nullptr,
+                                  c.n_r, c.n_c, ws + L.ys,
+                                  reinterpret_cast<int32_t*>(ws + L.inv_y),
                                   reinterpret_cast<int32_t*>(ws + L.chunk_y), st),
               "permute Y");
     // the copy's padding to whole 128-row groups (read by the selection's tiles, masked)
@@ -773,6 +775,7 @@ rece_status_t rece_loss_fwd(rece_plan_t plan, const void* X, const void* Y,
     stage_mark(*plan, RECE_STAGE_MERGE_LOSS, 0, st);
     RECE_CUDA(launch_merge_tc(*plan, Xb, Yb, targets, py,
                               reinterpret_cast<const int32_t*>(ws + L.inv_x),
+                              reinterpret_cast<const int32_t*>(ws + L.inv_y),
                               reinterpret_cast<const int32_t*>(ws + L.chunk_y), list, cnt, theta,
                               selected,
                               plan->tc_dx ? reinterpret_cast<int2*>(ws + L.kept) : nullptr,

@@ -21,8 +21,9 @@
 //                   (score, sorted position) into the row's lists, with the largest fp32
 //                   value below t as the bound of what was left out.
 //
-// The lists have the fused kernel's format (four sub-lists of Qw entries, filled in
-// order), so the merge and its exactness check are shared.  The scores pass through HBM
+// The lists have the fused kernel's format (four sub-lists of Qw entries, entry e of the
+// row in sub-list e mod 4, so their shares are even as the fused kernel's are), so the
+// merge and its exactness check are shared.  The scores pass through HBM
 // once (4 bytes per window score); that is far cheaper than recomputing d-deep dot
 // products at the sizes this path is chosen for.
 #include "common.cuh"
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select_scores(
     }
     if (bmin < kSelBins - 1) thr = cut_threshold(bm, uint32_t(bmin + 1) << 20);
   }
-  // emission, in column order: entry e goes to sub-list e / Qw, slot e % Qw
+  // emission, in column order: entry e goes to sub-list e mod 4, slot e / 4
   int2* out = list + w * 4 * int64_t(Qw);
   int n = 0;
   for (int c0 = 0; c0 < W; c0 += 32) {
@@ -332,18 +333,14 @@ __global__ void __launch_bounds__(kSelThreads) k_select_scores(
     const unsigned b = __ballot_sync(0xFFFFFFFFu, e);
     if (e) {
       const int idx = n + __popc(b & ((1u << lane) - 1u));
-      if (idx < 4 * Qw) out[idx] = make_int2(__float_as_int(v), int32_t(w0 + c));
+      if ((idx >> 2) < Qw)
+        out[(idx & 3) * Qw + (idx >> 2)] = make_int2(__float_as_int(v), int32_t(w0 + c));
     }
     n += __popc(b);
   }
   if (lane == 0) {
-    int cnt[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int rest = n - q * Qw;
-      cnt[q] = rest < 0 ? 0 : (q < 3 && rest > Qw ? Qw : rest);  // the last one shows overflow
-    }
-    list_count[w] = make_int4(cnt[0], cnt[1], cnt[2], cnt[3]);
+    // entries per sub-list (more than Qw: the list overflowed)
+    list_count[w] = make_int4((n + 3) >> 2, (n + 2) >> 2, (n + 1) >> 2, n >> 2);
     list_theta[w] = thr == -INFINITY ? -INFINITY : value_below(thr);
   }
 }

@@ -78,8 +78,8 @@ size_t merge_tc_spill_bytes(int n_r, int k);
 constexpr int kMaxKeptSlices = 512;  // slices of one window the merge can group by
 template <typename T>
 cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const int32_t* targets,
-                            const int32_t* py, const int32_t* invX, const int32_t* chunkY,
-                            const int2* list, const int4* list_count,
+                            const int32_t* py, const int32_t* invX, const int32_t* invY,
+                            const int32_t* chunkY, const int2* list, const int4* list_count,
                             const float* list_theta, int32_t* selected, int2* kept,
                             int32_t* kept_off, float* pos_logit, int Sp, float* lse,
                             float* row_loss, float* logits, uint32_t* status, int32_t* spill_rows,

@@ -107,12 +107,14 @@ def test_tc_path_recall_and_loss(name):
 
 @pytest.mark.parametrize("d,n_c,n_ec,n_r,k", [(64, 8, 1, 2, 64), (64, 16, 0, 1, 200),
                                               (128, 6, 2, 3, 100), (256, 8, 1, 2, 96),
-                                              (1024, 8, 1, 2, 96)])
+                                              (1024, 8, 1, 2, 96), (64, 8, 1, 2, 600),
+                                              (256, 8, 1, 1, 600)])
 def test_tc_path_exact_on_integer_inputs(d, n_c, n_ec, n_r, k):
     """Integer-valued inputs: every score is exact on the tensor cores and ties are
     everywhere, so the kept sets (ties to the lower item id) must be the oracle's.  At
     d >= 256 dX also comes from the tensor cores (band products of the coefficients); at
-    d = 1024 the window scores are stored once and selected row by row."""
+    d = 1024 the window scores are stored once and selected row by row.  At k >= 512 the
+    merge spreads each row over four warps."""
     w = synth.Workload("int", N=1000, C=5003, d=d, dtype="bf16", n_b=16, n_c=n_c, n_ec=n_ec,
                        n_r=n_r, k=k)
     X, Y, t = synth.integer_inputs(w.N, w.C, d, lo=-2, hi=2, seed=d + k, scale=0.125)
@@ -152,11 +154,11 @@ def test_backward_past_the_in_cache_pair_size():
 
 @pytest.mark.parametrize("d", [64, 256])
 def test_merge_spill_path_on_tied_scores(d):
-    """Every score equal: each round emits its whole window (one histogram bin), more
-    candidates than the merge's shared-memory buffer, so the rows go through the spill
-    path (global-memory buffers).  Ties go to the lower item id: the oracle's sets."""
+    """Every score equal: each row's whole window is emitted (one histogram bin, about 500
+    positions), more candidates than the merge's shared-memory buffers, so the rows go
+    through the spill path (global-memory buffers).  Ties go to the lower item id: the oracle's sets."""
     w = synth.Workload("tied", N=300, C=1000, d=d, dtype="bf16", n_b=8, n_c=6, n_ec=1,
-                       n_r=2, k=100)
+                       n_r=1, k=100)
     X = np.full((w.N, d), 0.125, np.float32)
     Y = np.full((w.C, d), 0.25, np.float32)
     t = np.random.default_rng(5).integers(0, w.C, w.N).astype(np.int32)
@@ -172,6 +174,32 @@ def test_merge_spill_path_on_tied_scores(d):
     term = 1.0 / w.N * float(np.abs(Y).max())
     assert np.abs(g["dX"] - o["dX"]).max() <= 1e-4 * term
     assert max_rel(g["dY"], o["dY"]) <= 1e-4
+
+
+def test_merge_four_warp_rows_spill_on_tied_scores():
+    """k >= 512: each row is merged by four warps, each holding one selection sub-list.
+    Every score tied (x = e_0, y_0 = 1/4, the other coordinates of y random, so the
+    catalogue's buckets still differ from round to round): each round emits its whole
+    window, about 1930 positions, and two rounds' entries overfill the warps' regions, so
+    rows go through the spill path.  Ties go to the lower item id: the oracle's sets."""
+    w = synth.Workload("tied4", N=300, C=9000, d=64, dtype="bf16", n_b=8, n_c=14, n_ec=1,
+                       n_r=2, k=512)
+    X = np.zeros((w.N, w.d), np.float32)
+    X[:, 0] = 1.0
+    rng = np.random.default_rng(12)
+    Y = rng.integers(-2, 3, (w.C, w.d)).astype(np.float32) * 0.125
+    Y[:, 0] = 0.25
+    t = rng.integers(0, w.C, w.N).astype(np.int32)
+    # integer projections: every projection exact on both sides, ties to the lower bucket
+    B = synth.integer_inputs(w.n_r * w.n_b, 1, w.d, lo=-2, hi=2, seed=12, scale=1.0)[0]
+    B = B.reshape(w.n_r, w.n_b, w.d)
+    g = run_gpu(w, X, Y, t, B, flags=0, dloss=1.0)
+    o = run_oracle(w, X, Y, t, B, dloss=1.0)
+    assert g["status"] == 0
+    assert g["words"][3] > 0  # rows that took the spill path
+    np.testing.assert_array_equal(np.sort(g["selected"], axis=1), np.sort(o["selected"], axis=1))
+    assert abs(g["loss"] - o["loss"]) <= 1e-4 * abs(o["loss"])
+    assert max_rel(g["dX"], o["dX"]) <= 1e-4 and max_rel(g["dY"], o["dY"]) <= 1e-4
 
 
 def test_sampled_selection_hands_misled_rows_to_the_exact_kernel():
