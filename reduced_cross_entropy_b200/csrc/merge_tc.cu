@@ -24,6 +24,13 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCountBytes = 16 * 32 * 4;  // per-warp digit-count table
 
+// A warp's table: the digit counts, and in grouped mode the bit map of a window (two words
+// a slice) and its slice starts, whichever is larger.
+__host__ __device__ __forceinline__ size_t merge_table_bytes(bool grouped, int Sp) {
+  const size_t g = grouped ? size_t(3) * size_t(Sp) * 4 : 0;
+  return g > size_t(kCountBytes) ? (g + 15) / 16 * 16 : size_t(kCountBytes);
+}
+
 struct WarpSel {
   uint32_t T;  // threshold key
   int need;    // how many keys equal to T are kept
@@ -308,16 +315,17 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
       if (take(a)) acc += expf(key_score(keys[a]) - m);
     lse = m + logf(warp_sum(acc) + expf(lp - m));
   }
-  // The kept entries, by round and, within a round, grouped by 64-position slice of the
-  // round's sorted catalogue (in candidate-list order inside a slice): a stable counting
-  // sort over the slices of the row's window.  Besides the row's outputs (items, logits),
-  // the backward gets, indexed by (round, sorted row p): the round's entries
+  // The kept entries, by round and, within a round, in order of sorted position (so
+  // grouped by 64-position slice of the round's sorted catalogue): a bit map of the
+  // round's window from the start of its first slice, an entry's place being the count of
+  // kept positions before it.  Besides the row's outputs (items, logits), the backward
+  // gets, indexed by (round, sorted row p): the round's entries
   // kept[r][p][e] = (sorted position, p_ij as two bf16 halves hi | lo << 16, with
   // p_ij = exp(l_ij - lse_i) = bf16(hi) + bf16(lo) to about 16 bits; 0 for a bad target)
   // and the slice starts kept_off[r][p][s] (s = 0..S, entry S = the round's count).
+  // The table cnt holds the bit map (2 S words) and the slice starts (S words).
   float* lg = logits ? logits + i * (int64_t(k) + 1) : nullptr;
   int32_t* srow = selected + i * k;
-  int32_t* bins = reinterpret_cast<int32_t*>(cnt);  // up to 512 slices (the count table)
   int ns = 0;
   float worst = INFINITY;
   for (int r = 0; r < n_r; ++r) {
@@ -344,17 +352,22 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
     const int64_t w1 = chunk_start(c + n_ec + 1 > n_c ? n_c : c + n_ec + 1, C, n_c);
     const int sig0 = int(w0 >> 6);
     const int S = w1 > w0 ? int((w1 - 1) >> 6) - sig0 + 1 : 0;
-    for (int b = lane; b < S; b += 32) bins[b] = 0;
+    const int32_t pbase = sig0 << 6;
+    uint32_t* bits = cnt;
+    int32_t* soff = reinterpret_cast<int32_t*>(cnt) + 2 * S;
+    for (int b = lane; b < 2 * S; b += 32) bits[b] = 0u;
     __syncwarp();
     for (int a = rb[r] + lane; a < rb[r + 1]; a += 32)
-      if (take(a)) atomicAdd(&bins[(poss[a] >> 6) - sig0], 1);
+      if (take(a)) {
+        const int o = poss[a] - pbase;
+        atomicOr(&bits[o >> 5], 1u << (o & 31));
+      }
     __syncwarp();
     // exclusive scan of the slice counts, lane l holding slices [l*B, l*B + B)
     const int B = (S + 31) >> 5;
-    int sbits = 0;  // bits of the slice ids 0..S-1
-    while ((1 << sbits) < S) ++sbits;
     int run = 0;
-    for (int b = lane * B; b < S && b < lane * B + B; ++b) run += bins[b];
+    for (int b = lane * B; b < S && b < lane * B + B; ++b)
+      run += __popc(bits[2 * b]) + __popc(bits[2 * b + 1]);
     int incl = run;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -362,42 +375,35 @@ __device__ __forceinline__ bool merge_row(const MergeArgs<T>& A, int64_t i, uint
       if (lane >= o) incl += v;
     }
     const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    int at = ns + incl - run;
+    int at = incl - run;
     const int64_t rp = int64_t(r) * N + px_of[r];
     int32_t* orow = kept_off + rp * Sp;
     int2* erow = kept + rp * k;  // the round's entries, from 0
     for (int b = lane * B; b < S && b < lane * B + B; ++b) {
-      const int v = bins[b];
-      bins[b] = at;
-      orow[b] = at - ns;
-      at += v;
+      soff[b] = at;
+      orow[b] = at;
+      at += __popc(bits[2 * b]) + __popc(bits[2 * b + 1]);
     }
     if (lane == 0) orow[S] = total;
     __syncwarp();
-    for (int a0 = rb[r]; a0 < rb[r + 1]; a0 += 32) {
-      const int a = a0 + lane;
-      const bool tk = a < rb[r + 1] && take(a);
-      const int sl = tk ? (poss[a] >> 6) - sig0 : 0;
-      const unsigned peers = digit_peers(sl, sbits, tk, lane);
-      const int dest = tk ? bins[sl] + __popc(peers & ((1u << lane) - 1u)) : 0;
-      __syncwarp();
-      if (tk && lane == __ffs(peers) - 1) bins[sl] += __popc(peers);
-      __syncwarp();
-      if (tk) {
-        const int32_t pos = poss[a];
-        const float sc = key_score(keys[a]);
-        srow[dest] = py[int64_t(r) * C + pos];
-        uint32_t packed = 0u;
-        if (z_ok) {
-          const float pr = expf(sc - lse);
-          const __nv_bfloat16 h = __float2bfloat16_rn(pr);
-          const __nv_bfloat16 l = __float2bfloat16_rn(pr - __bfloat162float(h));
-          packed = uint32_t(__bfloat16_as_ushort(h)) | (uint32_t(__bfloat16_as_ushort(l)) << 16);
-        }
-        erow[dest - ns] = make_int2(pos, int32_t(packed));
-        if (lg) lg[1 + dest] = sc;
-        worst = fminf(worst, sc);
+    for (int a = rb[r] + lane; a < rb[r + 1]; a += 32) {
+      if (!take(a)) continue;
+      const int32_t pos = poss[a];
+      const int o = pos - pbase, wi = o >> 5;
+      const int dest = soff[o >> 6] + __popc(bits[wi] & ((1u << (o & 31)) - 1u)) +
+                       ((wi & 1) ? __popc(bits[wi - 1]) : 0);
+      const float sc = key_score(keys[a]);
+      srow[ns + dest] = py[int64_t(r) * C + pos];
+      uint32_t packed = 0u;
+      if (z_ok) {
+        const float pr = expf(sc - lse);
+        const __nv_bfloat16 h = __float2bfloat16_rn(pr);
+        const __nv_bfloat16 l = __float2bfloat16_rn(pr - __bfloat162float(h));
+        packed = uint32_t(__bfloat16_as_ushort(h)) | (uint32_t(__bfloat16_as_ushort(l)) << 16);
       }
+      erow[dest] = make_int2(pos, int32_t(packed));
+      if (lg) lg[1 + ns + dest] = sc;
+      worst = fminf(worst, sc);
     }
     ns += total;
     __syncwarp();
@@ -440,10 +446,11 @@ template <typename T, bool kGrouped, int kGather>
 __global__ void __launch_bounds__(kThreads) k_merge_tc(const MergeArgs<T> A, int cap) {
   extern __shared__ __align__(16) uint8_t sh_raw[];
   const int warps = blockDim.x >> 5, wid = threadIdx.x >> 5;
-  const size_t per_warp = size_t(cap) * 8 + kCountBytes;
+  const size_t tab = merge_table_bytes(kGrouped, A.Sp);
+  const size_t per_warp = size_t(cap) * 8 + tab;
   uint8_t* base = sh_raw + per_warp * wid;
   uint32_t* cnt = reinterpret_cast<uint32_t*>(base);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(base + kCountBytes);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(base + tab);
   int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);
   const int64_t i = int64_t(blockIdx.x) * warps + wid;
   if (i >= A.N) return;  // whole warp leaves together; no block-wide barriers follow
@@ -455,15 +462,16 @@ __global__ void __launch_bounds__(kThreads) k_merge_tc(const MergeArgs<T> A, int
 template <typename T, bool kGrouped, int kGather>
 __global__ void __launch_bounds__(kThreads) k_merge_tc_spill(const MergeArgs<T> A, int cap,
                                                              uint32_t* scratch) {
-  __shared__ uint32_t sh_cnt[kThreads / 32][kCountBytes / 4];
+  extern __shared__ __align__(16) uint8_t sh_raw[];
   const int wid = threadIdx.x >> 5;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(sh_raw + merge_table_bytes(kGrouped, A.Sp) * wid);
   const int64_t gw = int64_t(blockIdx.x) * (blockDim.x >> 5) + wid;
   const int64_t nw = int64_t(gridDim.x) * (blockDim.x >> 5);
   uint32_t* keys = scratch + gw * 2 * int64_t(cap);
   int32_t* poss = reinterpret_cast<int32_t*>(keys + cap);
   const uint32_t n = *reinterpret_cast<volatile uint32_t*>(A.spill_count);
   for (int64_t w = gw; w < n; w += nw)
-    merge_row<T, kGrouped, kGather>(A, A.spill_rows[w], sh_cnt[wid], keys, poss, cap, false);
+    merge_row<T, kGrouped, kGather>(A, A.spill_rows[w], cnt, keys, poss, cap, false);
 }
 
 // ---------------------------------------------------------------- one row per CTA
@@ -900,8 +908,9 @@ size_t merge_tc_spill_bytes(int n_r, int k) {
   return size_t(kSpillWarps) * size_t(merge_tc_spill_cap(n_r, k)) * 8;
 }
 
+// (the largest table: grouped, the widest window the plan accepts)
 size_t merge_tc_warp_bytes(int n_r, int k) {
-  return size_t(merge_tc_cap(n_r, k)) * 8 + kCountBytes;
+  return size_t(merge_tc_cap(n_r, k)) * 8 + merge_table_bytes(true, kMaxKeptSlices + 1);
 }
 
 // One-row-per-CTA path: the 256-bin histogram, which the grouped output's bit map (two
@@ -982,7 +991,7 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
     kern<<<unsigned(c.N), kCtaThreads, cta_smem, st>>>(A, capw);
   } else {
     const int cap = merge_tc_cap(c.n_r, c.k);
-    const size_t per_warp = merge_tc_warp_bytes(c.n_r, c.k);
+    const size_t per_warp = size_t(cap) * 8 + merge_table_bytes(grouped, Sp);
     int warps = int((200 * 1024) / per_warp);
     warps = warps < 1 ? 1 : (warps > kThreads / 32 ? kThreads / 32 : warps);
     const size_t smem = per_warp * warps;
@@ -994,7 +1003,10 @@ cudaError_t launch_merge_tc(const rece_plan_s& p, const T* X, const T* Y, const 
   }
   auto spill = grouped ? (wide ? k_merge_tc_spill<T, true, 8> : k_merge_tc_spill<T, true, 4>)
                        : (wide ? k_merge_tc_spill<T, false, 8> : k_merge_tc_spill<T, false, 4>);
-  spill<<<kSpillWarps / (kThreads / 32), kThreads, 0, st>>>(
+  const size_t spill_smem = size_t(kThreads / 32) * merge_table_bytes(grouped, Sp);
+  e = cudaFuncSetAttribute(spill, cudaFuncAttributeMaxDynamicSharedMemorySize, int(spill_smem));
+  if (e != cudaSuccess) return e;
+  spill<<<kSpillWarps / (kThreads / 32), kThreads, spill_smem, st>>>(
       A, merge_tc_spill_cap(c.n_r, c.k), static_cast<uint32_t*>(spill_scratch));
   count_launches(2);
   return cudaGetLastError();
