@@ -21,6 +21,8 @@ upcast) and follows the definitions cited in ``rece_oracle.c``:
 * ``sampled_loss`` / ``sampled_grad`` -- the sampled baselines of section 2: CE- (eq. 2,
                        kind 0) and BCE+ (eq. 1, kind 1) over given negatives
 * ``rece_forward``  -- the whole forward path, steps 1 to 5, given the random vectors B
+* ``draw_projections`` / ``splitmix64`` -- Algorithm 1's randn step as a counter-based
+                       stream of (seed, step): SplitMix64 outputs, Box-Muller normals
 """
 import ctypes
 import math
@@ -49,6 +51,11 @@ def _load():
         lib.oracle_stable_argsort.restype = None
         lib.oracle_chunk_start.argtypes = [i64, i64, i64]
         lib.oracle_chunk_start.restype = i64
+        u64 = ctypes.c_uint64
+        lib.oracle_splitmix64.argtypes = [u64, u64]
+        lib.oracle_splitmix64.restype = u64
+        lib.oracle_draw_projections.argtypes = [u64, u64, i64, f32p]
+        lib.oracle_draw_projections.restype = None
         i64p_or_null = ctypes.c_void_p
         lib.oracle_select.argtypes = [f32p, f32p, i32p, i64, i64, i32, i32, i32, i32, i32,
                                       i32p, i32p, i64p_or_null, i64, i32p, f32p, i64p]
@@ -235,6 +242,22 @@ def full_ce_grad(X, Y, target, lse, dloss=1.0):
     _load().oracle_full_ce_grad(X, Y, target, N, C, d, np.ascontiguousarray(lse, np.float64),
                                 float(dloss), dX, dY)
     return dX, dY
+
+
+def splitmix64(state, i):
+    """The i-th output (from 0) of SplitMix64 started at `state` (Steele, Lea and Flood,
+    OOPSLA 2014): mix(state + (i + 1) * 0x9E3779B97F4A7C15)."""
+    return int(_load().oracle_splitmix64(state & (2**64 - 1), i & (2**64 - 1)))
+
+
+def draw_projections(seed, step, n_r, n_b, d):
+    """Algorithm 1's random vectors B [n_r, n_b, d] (fp32) of call `step` of a run seeded
+    with `seed`: standard normals by Box-Muller from the SplitMix64 stream of state
+    mix(mix(seed) ^ step), elements in B's row-major order (rece_oracle.c gives every
+    constant)."""
+    out = np.empty(n_r * n_b * d, np.float32)
+    _load().oracle_draw_projections(seed & (2**64 - 1), step & (2**64 - 1), out.size, out)
+    return out.reshape(n_r, n_b, d)
 
 
 def optimal_buckets(N, C, n_ec, alpha_bc):

@@ -516,3 +516,44 @@ void oracle_sampled_grad(int32_t kind, const float* X, const float* Y, const int
 
 /* Exposed for the tests: the fp32 fmaf-chain score of one pair. */
 float oracle_dot_f32(const float* a, const float* b, int32_t d) { return dot_f32(a, b, d); }
+
+/* [RECE] Algorithm 1, the randn step: the random vectors B of one call of the loss,
+ * drawn from (seed, step) by a counter-based stream, so that the library and this oracle,
+ * each written from the stream's published definition, draw the same numbers.
+ *   SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom number generators",
+ *   OOPSLA 2014): for state s and gamma G = 0x9E3779B97F4A7C15 the i-th output (from 0)
+ *   is mix(s + (i + 1) G), where mix(z) is z ^= z >> 30; z *= 0xBF58476D1CE4E5B9;
+ *   z ^= z >> 27; z *= 0x94D049BB133111EB; z ^= z >> 31 (arithmetic mod 2^64).
+ *   A call's state: s = mix(mix(seed) ^ step).
+ *   A uniform from an output x: u = ((x >> 11) + 1) 2^-53, in (0, 1].
+ *   Box-Muller (Box and Muller, Ann. Math. Statist. 1958), pair q of elements: from
+ *   u1 = u(x_2q) and u2 = u(x_2q+1), rho = sqrt(-2 ln u1), theta = 2 pi u2 (2 pi as the
+ *   double 6.283185307179586), element 2q = rho cos(theta), element 2q+1 = rho sin(theta),
+ *   in fp64, rounded to fp32.  Elements follow B's row-major order [n_r][n_b][d]; with an
+ *   odd count the last sine is not used. */
+static uint64_t splitmix_mix(uint64_t z) {
+  z ^= z >> 30;
+  z *= 0xBF58476D1CE4E5B9ull;
+  z ^= z >> 27;
+  z *= 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return z;
+}
+
+uint64_t oracle_splitmix64(uint64_t s, uint64_t i) {
+  return splitmix_mix(s + (i + 1) * 0x9E3779B97F4A7C15ull);
+}
+
+void oracle_draw_projections(uint64_t seed, uint64_t step, int64_t count, float* B) {
+  const uint64_t s = splitmix_mix(splitmix_mix(seed) ^ step);
+  for (int64_t q = 0; 2 * q < count; ++q) {
+    const uint64_t x1 = oracle_splitmix64(s, (uint64_t)(2 * q));
+    const uint64_t x2 = oracle_splitmix64(s, (uint64_t)(2 * q + 1));
+    const double u1 = (double)((x1 >> 11) + 1) * 0x1.0p-53;
+    const double u2 = (double)((x2 >> 11) + 1) * 0x1.0p-53;
+    const double rho = sqrt(-2.0 * log(u1));
+    const double theta = 6.283185307179586 * u2;
+    B[2 * q] = (float)(rho * cos(theta));
+    if (2 * q + 1 < count) B[2 * q + 1] = (float)(rho * sin(theta));
+  }
+}

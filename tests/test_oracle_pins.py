@@ -594,3 +594,38 @@ def test_window_row_sample_matches_the_full_computation():
     np.testing.assert_array_equal(srow, row[sample])
     sX, _ = oracle.window_grad(X, Y, z, px, py, 5, 1, slse, 0.5, rows=sample)
     np.testing.assert_array_equal(sX, dX[sample])
+
+
+# --------------------------------------------------------------------------- randn draw
+def test_splitmix64_first_outputs_from_state_zero():
+    """SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) started at state 0: its first three
+    outputs as published with the generator (0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4,
+    0x06C45D188009454F)."""
+    assert oracle.splitmix64(0, 0) == 0xE220A8397B1DCDAF
+    assert oracle.splitmix64(0, 1) == 0x6E789E6AA1B965F4
+    assert oracle.splitmix64(0, 2) == 0x06C45D188009454F
+
+
+def test_draw_projections_is_a_standard_normal_stream():
+    """Algorithm 1's randn step as drawn by the oracle: against the normal law and the
+    Box-Muller construction's own laws (Box and Muller 1958: for a pair (z0, z1),
+    z0^2 + z1^2 is exponential with mean 2 and atan2(z1, z0) is uniform on (-pi, pi],
+    independently), by Kolmogorov-Smirnov tests; independent pairs, calls and seeds."""
+    from scipy import stats
+    B = oracle.draw_projections(7, 3, 4, 1024, 256).ravel().astype(np.float64)
+    n = B.size  # 2^20
+    assert abs(B.mean()) < 5 / math.sqrt(n)
+    assert abs(B.var() - 1.0) < 5 * math.sqrt(2.0 / n)
+    assert stats.kstest(B, "norm").pvalue > 1e-3
+    z0, z1 = B[0::2], B[1::2]
+    assert stats.kstest(z0 ** 2 + z1 ** 2, "expon", args=(0, 2)).pvalue > 1e-3
+    assert stats.kstest(np.arctan2(z1, z0), "uniform", args=(-math.pi, 2 * math.pi)).pvalue > 1e-3
+    assert abs(np.corrcoef(z0, z1)[0, 1]) < 5 / math.sqrt(z0.size)
+    # another call (step) and another seed: fresh, uncorrelated numbers
+    B2 = oracle.draw_projections(7, 4, 4, 1024, 256).ravel().astype(np.float64)
+    B3 = oracle.draw_projections(8, 3, 4, 1024, 256).ravel().astype(np.float64)
+    assert abs(np.corrcoef(B, B2)[0, 1]) < 5 / math.sqrt(n)
+    assert abs(np.corrcoef(B, B3)[0, 1]) < 5 / math.sqrt(n)
+    # the same (seed, step) draws the same numbers; a shape is a prefix of the stream
+    np.testing.assert_array_equal(oracle.draw_projections(7, 3, 4, 1024, 256).ravel(), B)
+    np.testing.assert_array_equal(oracle.draw_projections(7, 3, 1, 1, 99).ravel(), B[:99])
