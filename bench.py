@@ -323,6 +323,15 @@ def oracle_sample_desc(w, ws, f):
             f"for the whole workload (extrapolated, linear in N and C)")
 
 
+def oracle_projections(ws, seed, step):
+    """The oracle's draw of a step's random vectors (the library's stream), in the
+    workload's element type."""
+    import oracle
+    from reduced_cross_entropy_b200 import synth
+    B = oracle.draw_projections(seed, step, ws.n_r, ws.n_b, ws.d)
+    return synth.round_bf16(B) if ws.dtype == "bf16" else B
+
+
 def cpu_baseline(w, seed, all_negatives=False, seconds=20.0):
     """rows/s of the CPU oracle on workload w (or its proportional slice), one step of
     about `seconds`."""
@@ -330,8 +339,7 @@ def cpu_baseline(w, seed, all_negatives=False, seconds=20.0):
     from reduced_cross_entropy_b200 import synth
     ws, f = oracle_slice(w, seconds, oracle_rate())
     X, Y, t = synth.make_inputs(ws, seed=seed)
-    B = synth.projections(seed, 0, ws.n_r, ws.n_b, ws.d, ws.dtype)
-    sec = oracle_step(ws, X, Y, t, B, all_negatives)
+    sec = oracle_step(ws, X, Y, t, oracle_projections(ws, 0, 0), all_negatives)
     return {"value": ws.N / sec, "unit": "rows/s", "cores": oracle.num_threads(),
             "kind": "oracle", "method": "extrapolated" if f > 1 else "full",
             "sample": oracle_sample_desc(w, ws, f), "seconds": sec}
@@ -350,10 +358,8 @@ def run_reference(args):
     X, Y, t = synth.make_inputs(ws, seed=0)
     alln = bool(getattr(args, "flags", 0) & 0x2)  # RECE_FLAG_ALL_NEGATIVES: Algorithm 1 as printed
     for s in range(args.warmup):
-        oracle_step(ws, X, Y, t, synth.projections(0, s, ws.n_r, ws.n_b, ws.d, ws.dtype), alln)
-    secs = [oracle_step(ws, X, Y, t,
-                        synth.projections(0, args.warmup + s, ws.n_r, ws.n_b, ws.d, ws.dtype),
-                        alln)
+        oracle_step(ws, X, Y, t, oracle_projections(ws, 0, s), alln)
+    secs = [oracle_step(ws, X, Y, t, oracle_projections(ws, 0, args.warmup + s), alln)
             for s in range(args.steps)]
     total = sum(secs)
     value = ws.N * args.steps / total  # each step is the slice's whole step: ws.N rows
@@ -425,10 +431,11 @@ class WorkloadRun:
         self.Xd = torch.from_numpy(self.X).to(dev).to(self.tdt)
         self.Yd = torch.from_numpy(self.Y).to(dev).to(self.tdt)
         self.td = torch.from_numpy(self.t).to(dev)
-        # B is drawn afresh for every step (the method's randn inside the loss), keyed by
-        # (seed 0, step) on every rank so that the replicas bucket alike
-        self.Bs = [torch.from_numpy(synth.projections(0, s, w.n_r, w.n_b, w.d, w.dtype))
-                   .to(dev).to(self.tdt) for s in range(n_steps)]
+        # B is drawn afresh on the device in every step (the method's randn inside the
+        # loss, rece_draw_projections), keyed by (seed 0, step) on every rank so that the
+        # replicas bucket alike
+        self.Bd = torch.empty((w.n_r, w.n_b, w.d), dtype=self.tdt, device=dev)
+        self.n_steps = n_steps
         self.ws = self.plan.workspace(dev)
         f32 = dict(dtype=torch.float32, device=dev)
         self.loss = torch.empty(1, **f32)
@@ -443,13 +450,14 @@ class WorkloadRun:
         self.sp = ctypes.c_void_p(self.stream.cuda_stream)
         self.nbytes = ctypes.c_size_t(self.ws.numel())
 
-    def step(self, Bt, Xc=None, Yc=None, tc=None):
+    def step(self, s, Xc=None, Yc=None, tc=None):
         vp = lambda x: ctypes.c_void_p(x.data_ptr())  # noqa: E731
         L, h, sp, ck = self.L, self.plan._h, self.sp, self._lib.check
         Xc = self.Xd if Xc is None else Xc
         Yc = self.Yd if Yc is None else Yc
         tc = self.td if tc is None else tc
-        ck(L.rece_bucketize_sort(h, vp(Bt), vp(Xc), vp(Yc), vp(self.ws), self.nbytes, sp),
+        ck(L.rece_draw_projections(h, 0, s, vp(self.Bd), sp), "draw_projections")
+        ck(L.rece_bucketize_sort(h, vp(self.Bd), vp(Xc), vp(Yc), vp(self.ws), self.nbytes, sp),
            "bucketize_sort")
         ck(L.rece_loss_fwd(h, vp(Xc), vp(Yc), vp(tc), vp(self.ws), self.nbytes, vp(self.loss),
                            None, vp(self.sel), vp(self.lse), vp(self.logits), sp), "loss_fwd")
@@ -462,7 +470,7 @@ class WorkloadRun:
     def warm(self, warmup):
         for s in range(warmup):
             self.flush.zero_()
-            self.step(self.Bs[s])
+            self.step(s)
         self.torch.cuda.synchronize(self.dev)
         # status area: flags (a bad target or a timed-out wait fails the run; the
         # tensor-core selection may flag rows it cannot certify exact) and row counts
@@ -500,7 +508,7 @@ class WorkloadRun:
                 _lib.check(self.L.rece_plan_set_stage_events(self.plan._h, sev_h[s]),
                            "stage events")
                 ev[s][0].record(stream)
-                self.step(self.Bs[first + s])
+                self.step(first + s)
                 ev[s][1].record(stream)
             torch.cuda.synchronize(self.dev)
         barrier()
@@ -577,13 +585,11 @@ class WorkloadRun:
         Xh = torch.from_numpy(self.X).to(tdt).pin_memory()
         Yh = torch.from_numpy(self.Y).to(tdt).pin_memory()
         th = torch.from_numpy(self.t).pin_memory()
-        Bh = [b.cpu().pin_memory() for b in self.Bs]
-        loss_h = torch.empty(len(self.Bs), dtype=torch.float32).pin_memory()
-        h2d = Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size() + \
-            th.numel() * 4 + Bh[0].numel() * Bh[0].element_size()
-        sets = [(self.Xd, self.Yd, self.td, torch.empty_like(self.Bs[0])),
+        loss_h = torch.empty(self.n_steps, dtype=torch.float32).pin_memory()
+        h2d = Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size() + th.numel() * 4
+        sets = [(self.Xd, self.Yd, self.td),
                 (torch.empty_like(self.Xd), torch.empty_like(self.Yd),
-                 torch.empty_like(self.td), torch.empty_like(self.Bs[0]))]
+                 torch.empty_like(self.td))]
         cstream = torch.cuda.Stream(dev)
         copied = [torch.cuda.Event() for _ in range(2)]
         consumed = [torch.cuda.Event() for _ in range(2)]
@@ -593,7 +599,7 @@ class WorkloadRun:
             with torch.cuda.stream(cstream):
                 if j >= 2:  # the set's previous step has finished with it
                     cstream.wait_event(consumed[k])
-                for dst, src in zip(sets[k], (Xh, Yh, th, Bh[s])):
+                for dst, src in zip(sets[k], (Xh, Yh, th)):
                     dst.copy_(src, non_blocking=True)
                 copied[k].record(cstream)
 
@@ -609,8 +615,8 @@ class WorkloadRun:
                 k = s % 2
                 stream.wait_event(copied[k])
                 self.flush.zero_()
-                Xc, Yc, tc, Bc = sets[k]
-                self.step(Bc, Xc, Yc, tc)
+                Xc, Yc, tc = sets[k]
+                self.step(s, Xc, Yc, tc)
                 consumed[k].record(stream)
                 loss_h[s].copy_(self.loss[0], non_blocking=True)
             t1.record(stream)
@@ -641,7 +647,7 @@ def extra_workload(torch, name, args, dev):
            "stages_roofline_frac": fracs, "gpu_launches": int(launches)}
     if not args.no_memory:
         out["peak_hbm"] = measure_memory(torch, ops, run.plan, w, run.Xd, run.Yd, run.td,
-                                         run.Bs[0], dev)
+                                         run.Bd, dev)
     del run
     torch.cuda.empty_cache()
     return out
@@ -703,7 +709,7 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_memory:
         line["peak_hbm"] = measure_memory(torch, ops, run.plan, w, run.Xd, run.Yd, run.td,
-                                          run.Bs[0], dev)
+                                          run.Bd, dev)
     if rank == 0 and world == 1 and not args.no_baselines:
         line["baselines"] = measure_baselines(torch, ops, w, run.Xd, run.Yd, run.td, run.flush,
                                               dev, load_peaks())

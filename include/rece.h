@@ -179,9 +179,26 @@ RECE_API rece_status_t rece_plan_workspace_layout(rece_plan_t plan, rece_workspa
                                        cores (fmaf chains), not tcgen05 */
 RECE_API rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths);
 
+/* Algorithm 1's randn step [RECE section 3, Algorithm 1: the random vectors], drawn on
+ * the device: B [n_r][n_b][d] (device, in the plan's element type: fp32, or bf16 rounded
+ * to nearest even from the fp32 value; caller-owned, any alignment rece_bucketize_sort
+ * accepts) is filled with standard normals of call `step` of a run seeded with `seed`.
+ * The stream is counter-based, so any element can be drawn alone and a call repeats
+ * exactly: SplitMix64 [Steele, Lea, Flood, OOPSLA 2014] started at
+ * s = mix(mix(seed) ^ step), whose i-th output is mix(s + (i+1) * 0x9E3779B97F4A7C15)
+ * with mix(z) = z ^= z >> 30; z *= 0xBF58476D1CE4E5B9; z ^= z >> 27;
+ * z *= 0x94D049BB133111EB; z ^= z >> 31; outputs x -> uniforms ((x >> 11) + 1) 2^-53 in
+ * (0, 1]; element pair q by Box-Muller from outputs 2q and 2q+1: rho = sqrt(-2 ln u1),
+ * theta = 6.283185307179586 u2, elements rho cos(theta), rho sin(theta) (fp64, then fp32),
+ * in B's row-major order.  Enqueued on `stream`; B may be passed to rece_bucketize_sort
+ * on the same stream right after.  Errors: NULL plan or B (RECE_ERR_INVALID_ARG), a
+ * launch failure (RECE_ERR_CUDA). */
+RECE_API rece_status_t rece_draw_projections(rece_plan_t plan, uint64_t seed, uint64_t step,
+                                             void* B, void* stream);
+
 /* Steps 1-2 [RECE section 3, Algorithm 1: random vectors, argmax bucketing, argsort].
- *   B  device, [n_r][n_b][d] random vectors (one set per round; the caller draws them,
- *      N(0,1), afresh for every call as the paper does)
+ *   B  device, [n_r][n_b][d] random vectors (one set per round, N(0,1), afresh for every
+ *      call as the paper does: rece_draw_projections draws them, or the caller does)
  *   X  device, [N][d];  Y device, [C][d]
  * Writes bucket ids and stable per-round orders into the workspace, and clears the
  * status word.  Must precede rece_loss_fwd on the same workspace and stream. */

@@ -38,6 +38,7 @@ EXPORTS = (
     "rece_plan_set_stage_events", "rece_kernel_launch_count", "rece_bucket_sort_static",
     "rece_plan_paths", "rece_sampled_workspace_size", "rece_sampled_fwd", "rece_sampled_bwd",
     "rece_optimal_buckets", "rece_memory_model_elements", "rece_plan_get_config",
+    "rece_draw_projections",
 )
 SAMPLED_CE_MINUS = 0  # RECE section 2, equation (2)
 SAMPLED_BCE_PLUS = 1  # RECE section 2, equation (1)
@@ -88,6 +89,7 @@ def lib():
         "rece_plan_workspace_layout": ([vp, ctypes.POINTER(WorkspaceLayout)], st),
         "rece_plan_paths": ([vp, ctypes.POINTER(ctypes.c_uint32)], st),
         "rece_bucketize_sort": ([vp, vp, vp, vp, vp, sz, vp], st),
+        "rece_draw_projections": ([vp, ctypes.c_uint64, ctypes.c_uint64, vp, vp], st),
         "rece_loss_fwd": ([vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp, vp], st),
         "rece_loss_bwd": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp], st),
         "rece_full_ce_workspace_size": ([i64, i64, i32, i32, ctypes.POINTER(sz)], st),

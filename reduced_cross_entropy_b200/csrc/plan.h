@@ -136,6 +136,11 @@ inline void stage_mark(const rece_plan_s& p, int stage, int end, cudaStream_t st
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `st` and return the launch error (cudaSuccess if none).
 
+// The random vectors B [n_r][n_b][d] (count elements) of call `step` of a run seeded with
+// `seed`: SplitMix64 outputs, Box-Muller normals (projections.cu), fp32 or bf16.
+cudaError_t launch_draw_projections(uint64_t seed, uint64_t step, int64_t count, bool bf16,
+                                    void* B, cudaStream_t st);
+
 // K1: bucket[r][i] = argmax_b <B[r][b], V[i]> (fmaf chain, ties to lowest b).
 template <typename T>
 cudaError_t launch_bucketize_fma(const T* V, int64_t M, int d, const T* B, int n_b, int n_r,

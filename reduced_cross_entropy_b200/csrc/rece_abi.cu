@@ -639,6 +639,18 @@ rece_status_t rece_plan_paths(rece_plan_t plan, uint32_t* paths) {
   return RECE_OK;
 }
 
+rece_status_t rece_draw_projections(rece_plan_t plan, uint64_t seed, uint64_t step, void* B,
+                                    void* stream) {
+  if (!plan) return fail(RECE_ERR_INVALID_ARG, "NULL plan");
+  if (!B) return fail(RECE_ERR_INVALID_ARG, "NULL B");
+  const auto& c = plan->cfg;
+  const int64_t count = int64_t(c.n_r) * c.n_b * c.d;
+  RECE_CUDA(launch_draw_projections(seed, step, count, c.mode == RECE_MODE_BF16, B,
+                                    static_cast<cudaStream_t>(stream)),
+            "draw projections");
+  return RECE_OK;
+}
+
 rece_status_t rece_bucketize_sort(rece_plan_t plan, const void* B, const void* X, const void* Y,
                                   void* workspace, size_t workspace_bytes, void* stream) {
   rece_status_t s = check_plan_ws(plan, workspace, workspace_bytes);

@@ -111,6 +111,20 @@ def _check_ws(plan: Plan, ws: torch.Tensor):
         raise ValueError("workspace must be a CUDA uint8 tensor of plan.workspace_bytes bytes")
 
 
+def draw_projections(plan: Plan, seed: int, step: int, out=None, stream=None):
+    """Algorithm 1's random vectors B [n_r, n_b, d] of call `step` of a run seeded with
+    `seed`, drawn on the device (rece_draw_projections).  Returns `out` (allocated when
+    None) in the plan's element type."""
+    c = plan.cfg
+    if out is None:
+        out = torch.empty((c.n_r, c.n_b, c.d), dtype=plan.dtype, device="cuda")
+    _need(out, "B", plan.dtype, (c.n_r, c.n_b, c.d))
+    _lib.check(_lib.lib().rece_draw_projections(plan._h, seed & (2**64 - 1), step & (2**64 - 1),
+                                                _vp(out), _stream(stream)),
+               "rece_draw_projections")
+    return out
+
+
 def bucketize_sort(plan: Plan, B, X, Y, ws, stream=None):
     """Steps 1-2: bucket ids and stable per-round orders (into the workspace)."""
     c = plan.cfg

@@ -81,6 +81,32 @@ def test_auto_bucket_plan_matches_oracle(dtype):
         assert abs(g["loss"] - o["loss"]) <= 1e-2 * abs(o["loss"])
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_draw_projections_match_oracle(dtype):
+    """Algorithm 1's randn step drawn by the library (rece_draw_projections) against the
+    oracle's draw of the same (seed, step) stream: the same fp32 numbers (one unit in the
+    last place where the two sides' fp64 log / cos / sin differ at an fp32 rounding
+    boundary, at most one element in 10^4), bf16 as the oracle's fp32 rounded to nearest
+    even; then the fp32 path bucketized with the drawn vectors equals the oracle run."""
+    w = synth.Workload("draw", N=700, C=4000, d=64, dtype=dtype, n_b=64, n_c=16, n_ec=1,
+                       n_r=3, k=50)
+    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype)
+    for seed, step in [(0, 0), (12345, 7), (2**63 + 5, 2**40)]:
+        g = ops.draw_projections(plan, seed, step).float().cpu().numpy()
+        o = oracle.draw_projections(seed, step, w.n_r, w.n_b, w.d)
+        if dtype == "bf16":
+            o = synth.round_bf16(o)
+        diff = g != o
+        assert diff.mean() <= 1e-4
+        ulp = np.spacing(np.abs(o[diff])) * (2 ** 16 if dtype == "bf16" else 1)
+        assert np.all(np.abs(g[diff] - o[diff]) <= ulp)
+    if dtype == "fp32":
+        X, Y, t = synth.make_inputs(w, seed=9)
+        B = ops.draw_projections(plan, 9, 1).cpu().numpy()
+        np.testing.assert_array_equal(B, oracle.draw_projections(9, 1, w.n_r, w.n_b, w.d))
+        compare(w, run_gpu(w, X, Y, t, B), run_oracle(w, X, Y, t, B))
+
+
 def test_fp32_exact_whole_arrays_at_sasrec_scale():
     """The fp32 exact mode at the SASRec-scale benchmark shape (N = 25,600, C = 100,000,
     n_b = 256, n_c = 64, n_ec = 1, n_r = 2, k = 256), the whole arrays against the whole
