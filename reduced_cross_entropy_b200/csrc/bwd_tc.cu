@@ -88,13 +88,38 @@ __device__ __forceinline__ void zero_row(uint8_t* tile, int row) {
   for (int j = 0; j < 8; ++j) p[(j + row) & 7] = make_uint4(0u, 0u, 0u, 0u);
 }
 
+
+// The dX kernel's G tiles use the K-major layout without swizzle instead: 8 x 16-byte
+// core matrices, the 8 of a row group along K 128 B apart (leading byte offset), row
+// groups 1024 B apart (stride byte offset).  Element (row, col) then sits in bank
+// 4 (row % 8) + (col % 8) / 2, so the lanes of a warp (32 consecutive rows, one entry
+// each) can only collide four at a time, where the 128-byte swizzle spreads their random
+// columns over all 32 banks.
+__device__ __forceinline__ uint32_t plain_offset(int row, int col) {
+  return uint32_t((row >> 3) * 1024 + (col >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2);
+}
+__device__ __forceinline__ void zero_row_plain(uint8_t* tile, int row) {
+  uint8_t* p = tile + (row >> 3) * 1024 + (row & 7) * 16;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(p + j * 128) = make_uint4(0u, 0u, 0u, 0u);
+}
+// A 16-bit shared store that only happens when `p` holds (one predicated instruction).
+__device__ __forceinline__ void st_shared_b16_if(uint32_t addr, uint32_t v, bool p) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t"
+      "@q st.shared.b16 [%0], %1;\n\t}" ::"r"(addr), "h"(uint16_t(v)), "r"(int(p))
+      : "memory");
+}
+
 // Writes one coefficient, given as two bf16 halves (hi | lo << 16), into the hi and lo
-// tiles at (row, col).
-__device__ __forceinline__ void put(uint8_t* hi_tile, uint8_t* lo_tile, int row, int col,
-                                    uint32_t packed) {
-  const uint32_t o = sw128_offset(row, col);
-  *reinterpret_cast<uint16_t*>(hi_tile + o) = uint16_t(packed & 0xFFFFu);
-  *reinterpret_cast<uint16_t*>(lo_tile + o) = uint16_t(packed >> 16);
+// tiles at (row, col) when `p` holds: two predicated stores, no branch (a branch around
+// every entry's stores left the builder warps' tile writes several times slower).
+__device__ __forceinline__ void put_if(uint8_t* hi_tile, uint8_t* lo_tile, int row, int col,
+                                       uint32_t packed, bool p) {
+  const uint32_t o = sw128_offset(row & (kBM - 1), col);
+  st_shared_b16_if(smem_u32(hi_tile) + o, packed & 0xFFFFu, p);
+  st_shared_b16_if(smem_u32(lo_tile) + o, packed >> 16, p);
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -272,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
           break;
         }
         tc_fence_after();
-        const uint64_t dh = desc_k_sw128(smem_u32(A_hi + as * kATile));
-        const uint64_t dl = desc_k_sw128(smem_u32(A_lo + as * kATile));
+        const uint64_t dh = desc_k_plain(smem_u32(A_hi + as * kATile), 128u, 1024u);
+        const uint64_t dl = desc_k_plain(smem_u32(A_lo + as * kATile), 128u, 1024u);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           for (int h = 0; h < nh; ++h) {
@@ -282,8 +307,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
                 desc_mn_sw128(smem_u32(Bs + size_t(bs) * b_bytes + size_t(h) * nsh * 128),
                               8192u) + 128u * kk;
             const uint32_t acc = tmem + uint32_t(h * nsh);
-            mma_bf16(acc, dh + 2 * kk, db, idesc, (s | kk) != 0);
-            mma_bf16(acc, dl + 2 * kk, db, idesc, 1);
+            // K step kk: core matrices 2kk and 2kk + 1 along K, 256 B further
+            mma_bf16(acc, dh + 16 * kk, db, idesc, (s | kk) != 0);
+            mma_bf16(acc, dl + 16 * kk, db, idesc, 1);
           }
         }
         mma_commit(&ctl.aempty[as]);
@@ -332,19 +358,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dx_tc(const __grid_constant
       }
       uint8_t* th = A_hi + as * kATile;
       uint8_t* tl = A_lo + as * kATile;
-      zero_row(th, t);
-      zero_row(tl, t);
+      zero_row_plain(th, t);
+      zero_row_plain(tl, t);
       const int64_t sig = lo + s;  // absolute slab
       const int slab_end = int((sig + 1) * kBK);
       while (e < count) {
         int used = 0;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          if (base + u >= e && cur[u].x < slab_end) {
-            const int col = cur[u].x - int(sig * kBK);
-            if (col >= 0 && col < kBK) put(th, tl, t, col, uint32_t(cur[u].y));  // (always)
-            ++used;
-          }
+          // branch-free: the slot's two halves are stored under a predicate
+          const bool in = base + u >= e && cur[u].x < slab_end;
+          const int col = cur[u].x - int(sig * kBK);
+          const bool put = in && col >= 0 && col < kBK;
+          const uint32_t o = plain_offset(t, col & (kBK - 1));
+          const uint32_t v = uint32_t(cur[u].y);
+          st_shared_b16_if(smem_u32(th) + o, v & 0xFFFFu, put);
+          st_shared_b16_if(smem_u32(tl) + o, v >> 16, put);
+          used += in ? 1 : 0;
         }
         e += used;
         if (e < base + 8) break;  // the next entry belongs to a later slab
@@ -573,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
       if (ok && a1 > a0) {
 #pragma unroll
         for (int u = 0; u < kPre; ++u)
-          if (a0 + u < a1) put(th, tl, int(pre[u].x - q0), kc, uint32_t(pre[u].y));
+          put_if(th, tl, int(pre[u].x - q0), kc, uint32_t(pre[u].y), a0 + u < a1);
         const int2* ent = slab_entries(s);
         for (int e = a0 + kPre; e < a1; e += 8) {  // the rest, eight loads in flight
           int2 en[8];
@@ -581,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dy_tc(const __grid_constant
           for (int u = 0; u < 8; ++u) en[u] = e + u < a1 ? __ldg(ent + e + u) : make_int2(0, 0);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            if (e + u < a1) put(th, tl, int(en[u].x - q0), kc, uint32_t(en[u].y));
+            put_if(th, tl, int(en[u].x - q0), kc, uint32_t(en[u].y), e + u < a1);
         }
       }
       {  // slab s + 1's first entries
@@ -855,7 +885,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_bwd_dy_tc_p(const __grid_const
         if (ok && a1 > a0) {
 #pragma unroll
           for (int u = 0; u < kPre; ++u)
-            if (a0 + u < a1) put(th, tl, int(pre[u].x - g.q0), kc, uint32_t(pre[u].y));
+            put_if(th, tl, int(pre[u].x - g.q0), kc, uint32_t(pre[u].y), a0 + u < a1);
           const int2* ent = slab_entries(s);
           for (int e = a0 + kPre; e < a1; e += 8) {
             int2 en[8];
@@ -863,7 +893,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_bwd_dy_tc_p(const __grid_const
             for (int u = 0; u < 8; ++u) en[u] = e + u < a1 ? __ldg(ent + e + u) : make_int2(0, 0);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-              if (e + u < a1) put(th, tl, int(en[u].x - g.q0), kc, uint32_t(en[u].y));
+              put_if(th, tl, int(en[u].x - g.q0), kc, uint32_t(en[u].y), e + u < a1);
           }
         }
         {

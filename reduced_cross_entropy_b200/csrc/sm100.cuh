@@ -227,6 +227,16 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
          | (uint64_t(2) << 61);             // 128-byte swizzle
 }
 
+// Shared-memory descriptor of a K-major bf16 operand without swizzle: 8-row x 16-byte
+// core matrices (rows 16 B apart), `lbo` bytes between core matrices adjacent along K,
+// `sbo` bytes between 8-row groups.  One MMA's K = 16 spans two core matrices along K.
+__device__ __forceinline__ uint64_t desc_k_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4)        // start address, 16-byte units
+         | (uint64_t((lbo >> 4) & 0x3FFFu) << 16)  // leading byte offset: along K
+         | (uint64_t((sbo >> 4) & 0x3FFFu) << 32)  // stride byte offset: next 8 rows
+         | (uint64_t(1) << 46);                    // descriptor version of sm_100; no swizzle
+}
+
 // Shared-memory descriptor of an MN-major bf16 operand written by TMA boxes {64, rows}
 // with the 128-byte swizzle: each box holds 64 consecutive elements of M or N (128 B) for
 // each K index, K rows 128 B apart in 8-row atoms of 1024 B (the stride byte offset); the
