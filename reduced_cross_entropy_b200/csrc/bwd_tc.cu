@@ -854,7 +854,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_bwd_dy_tc_p(const __grid_const
         e0 = __ldg(off + idx);
         e1 = __ldg(off + idx + 1);
       };
-      constexpr int kPre = 16;
+      constexpr int kPre = 8;  // entries prefetched per (row, half); more take the loop below
       auto slab_entries = [&](int s2) { return a.kept + (rN + (g.lo + s2) * kBK + kc) * a.k; };
       int a0, a1, b0, b1;
       entry_range(0, a0, a1);
@@ -933,12 +933,13 @@ __global__ void __launch_bounds__(kPThreads, 1) k_bwd_dy_tc_p(const __grid_const
       tc_fence_after();
       const int64_t q = g.q0 + row;
       const bool live = q < C;
-      const int64_t dst = live ? a.px[int64_t(r) * C + q] : 0;
-      float* o = a.out + dst * a.d + g.n0;
+      const int64_t dst = live ? a.px[int64_t(r) * C + q] : -1;
       const uint32_t taddr = tmem + (uint32_t((warp & 3) * 32) << 16) + uint32_t(acc * ns);
+      // Each piece of 32 columns goes through the warp's staging rows and out as whole
+      // 128-byte row segments: lanes 8j..8j+7 write 16 B each of one row, four rows a store
+      // (the rows are items, scattered); the warp's rows' destinations come by shuffle.
       for (int c0 = 0; c0 < ns; c0 += kPW, ++piece) {
         float* srow = (piece & 1u) ? buf1 : buf0;
-        bulk_wait_read<1>();  // this thread's copy out of that buffer (two pieces ago)
         float v[32];
         if (g.nK == 0) {  // no rows cover the item: nothing accumulated (uniform)
 #pragma unroll
@@ -951,20 +952,28 @@ __global__ void __launch_bounds__(kPThreads, 1) k_bwd_dy_tc_p(const __grid_const
         for (int u = 0; u < 8; ++u)
           s4[u] = make_float4(scale * v[4 * u], scale * v[4 * u + 1], scale * v[4 * u + 2],
                               scale * v[4 * u + 3]);
-        if (live) {
-          fence_proxy_async_smem();
-          if (a.write)
-            bulk_store(o + c0, srow, uint32_t(kPW) * 4u);
-          else
-            bulk_reduce_add_f32(o + c0, srow, uint32_t(kPW) * 4u);
-          bulk_commit();
+        __syncwarp();
+        const uint8_t* wbase = reinterpret_cast<const uint8_t*>(srow) - size_t(lane) * kPStride;
+#pragma unroll
+        for (int it4 = 0; it4 < 8; ++it4) {
+          const int rr = 4 * it4 + (lane >> 3), ch = lane & 7;
+          const int64_t drow = __shfl_sync(0xFFFFFFFFu, dst, rr);
+          const float4 x = *reinterpret_cast<const float4*>(wbase + size_t(rr) * kPStride + ch * 16);
+          if (drow >= 0) {
+            float4* out = reinterpret_cast<float4*>(a.out + drow * a.d + g.n0 + c0) + ch;
+            if (a.write) {
+              *out = x;
+            } else {  // later rounds add (one writer per element and launch: a fixed order)
+              const float4 y = *out;
+              *out = make_float4(y.x + x.x, y.y + x.y, y.z + x.z, y.w + x.w);
+            }
+          }
         }
       }
       tc_fence_before();  // the accumulator's reads are done: the MMAs may refill it
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.accempty[acc]);
     }
-    bulk_wait_read<0>();
   }
   tc_fence_before();
   __syncthreads();
