@@ -800,9 +800,10 @@ def measure_memory(torch, ops, plan, w, Xd, Yd, td, B, dev):
     ws_bytes = ops.full_ce_workspace_bytes(w.N, w.C, w.d, w.dtype)
     out["full_ce_fused_bytes_computed"] = 4 * (2 * w.N + w.N * w.d + w.C * w.d + 1) + ws_bytes
     # the op runs on tcgen05 for bf16 with d a multiple of 64 up to 256, else on the CUDA
-    # cores: run it (and time one fwd+bwd, after one untimed) where that takes a few seconds
+    # cores (measured: about 112 s for one fwd+bwd at N = 16,384, C = 128,000, d = 4096):
+    # run it (and time one fwd+bwd, after one untimed) where that takes seconds
     tc = w.dtype == "bf16" and w.d % 64 == 0 and w.d <= 256
-    if 6.0 * w.N * w.C * w.d <= (2e15 if tc else 6e13):
+    if 6.0 * w.N * w.C * w.d <= (2e15 if tc else 3e13):
         fused()
         out["full_ce_fused_bytes"] = peak(fused)
         out["full_ce_fused_ms_fwd_bwd"] = fused_ms[-1]
