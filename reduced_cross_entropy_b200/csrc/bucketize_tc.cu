@@ -443,6 +443,259 @@ __global__ void __launch_bounds__(kRThreads, 1) k_bucketize_tc_res(
   }
 }
 
+
+// The same for d <= 256 on pairs of SMs (a cluster of two CTAs, tcgen05 cta_group::2):
+// work item = (round, 256-row tile), CTA r of the pair holding rows [128r, 128r + 128) of
+// it resident (all of d) and, of every slice of 256 vectors, vectors [128r, 128r + 128)
+// (64 K elements a stage); the even CTA issues M = 256 x N = 256 MMAs, each CTA's TMEM
+// receiving its own 128 rows (two 256-column accumulators).  An MMA then reads from each
+// SM's shared memory half the bytes the single-SM kernel's M = 128 x N = 128 MMAs read
+// for the same work, which had shared-memory bandwidth, not the tensor pipe, bound the
+// bucketing; the rows of the next item load into a second buffer meanwhile.  Loads of
+// both CTAs complete on the even CTA's barriers; the MMA commits (a stage or a row buffer
+// free, an accumulator full, all done) arrive on both CTAs' barriers at once (forwarding
+// them from the even CTA's threads instead made the kernel 1.6 times slower).  Eight
+// epilogue warps a CTA: warps q and q + 4 share TMEM lanes 32(q mod 4) and take column
+// halves, combined at the end of the item (ties to the lower vector).
+constexpr int kPStages = 6;
+constexpr int kPBN = 256;                        // vectors per slice (N of the pair MMA)
+constexpr uint32_t kPSliceA = kBM * kBK * 2;     // 16 KB: 128 rows x 64 K
+constexpr uint32_t kPSliceB = 128 * kBK * 2;     // 16 KB: this CTA's 128 vectors x 64 K
+constexpr int kPThreads = 96 + 256;              // B loads, MMA, row loads, 8 epilogue warps
+
+struct __align__(1024) SmemPair {
+  uint8_t a[2][kRMaxK][kPSliceA];  // [row buffer][k slice]
+  uint8_t b[kPStages][kPSliceB];
+  uint64_t full[kPStages];
+  uint64_t empty[kPStages];
+  uint64_t a_full[2], a_empty[2];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  float cmb_v[kBM];
+  int cmb_i[kBM];
+};
+static_assert(sizeof(SmemPair) + 1024 <= 232448, "pair kernel shared memory");
+
+__device__ __forceinline__ void on_timeout_pair(SmemPair& s, uint32_t* status) {
+  *reinterpret_cast<volatile int*>(&s.abort) = 1;
+  raise_flag(status, RECE_DEVICE_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kPThreads, 1) k_bucketize_tc_pair(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+    const __grid_constant__ CUtensorMap tmB, int64_t N, int64_t C, int d, int n_b, int n_r,
+    int32_t* __restrict__ bx, int32_t* __restrict__ by, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemPair& s = *reinterpret_cast<SmemPair*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool lead = rank == 0;
+  constexpr int kRows = 2 * kBM;
+  const int64_t tX = (N + kRows - 1) / kRows, tY = (C + kRows - 1) / kRows;
+  const int64_t per_round = tX + tY, items = per_round * n_r;
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int n_nt = (n_b + kPBN - 1) / kPBN;
+  const int nk = d / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.a_full[i], 1);
+      mbar_init(&s.a_empty[i], 1);
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 16);  // the pair's 16 epilogue warps (even CTA's)
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s.tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers and TMEM ready before either touches the other
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abortp = &s.abort;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- B loads
+    uint32_t it = 0;
+    if (lane == 0) {
+      prefetch_tmap(&tmB);
+      bool ok = true;
+      for (int64_t item = pair; item < items && ok && !*abortp; item += npairs) {
+        const int r = int(item / per_round);
+        for (int nt = 0; nt < n_nt && ok; ++nt) {
+          for (int ks = 0; ks < nk; ++ks, ++it) {
+            const int st = it % kPStages;
+            if (!mbar_wait_cluster(&s.empty[st], ((it / kPStages) & 1u) ^ 1u, &s.abort,
+                                   kTimeoutNs)) {
+              on_timeout_pair(s, status);
+              ok = false;
+              break;
+            }
+            if (lead) mbar_arrive_expect_tx(&s.full[st], 2 * kPSliceB);  // both halves
+            tma_load_2d_pair(s.b[st], &tmB, &s.full[st], ks * kBK,
+                             r * n_b + nt * kPBN + int(rank) * 128);
+          }
+        }
+      }
+      if (lead)  // teardown: the last stages' loads (both CTAs') have landed
+        for (uint32_t j = (it > kPStages ? it - kPStages : 0); j < it; ++j)
+          mbar_wait_limit(&s.full[j % kPStages], (j / kPStages) & 1u, kTimeoutNs);
+    }
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- row loads
+    uint32_t ni = 0;
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmY);
+      for (int64_t item = pair; item < items && !*abortp; item += npairs, ++ni) {
+        const int64_t t = item % per_round;
+        const bool isY = t >= tX;
+        const int64_t row0 = (isY ? t - tX : t) * kRows + int64_t(rank) * kBM;
+        const int slot = int(ni & 1u);
+        if (!mbar_wait_cluster(&s.a_empty[slot], ((ni >> 1) & 1u) ^ 1u, &s.abort, kTimeoutNs)) {
+          on_timeout_pair(s, status);
+          break;
+        }
+        if (lead) mbar_arrive_expect_tx(&s.a_full[slot], 2u * uint32_t(nk) * kPSliceA);
+        for (int ks = 0; ks < nk; ++ks)
+          tma_load_2d_pair(s.a[slot][ks], isY ? &tmY : &tmX, &s.a_full[slot], ks * kBK,
+                           int32_t(row0));
+      }
+      if (lead)
+        for (uint32_t j = (ni > 2 ? ni - 2 : 0); j < ni; ++j)
+          mbar_wait_limit(&s.a_full[j & 1u], (j >> 1) & 1u, kTimeoutNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (even CTA)
+    if (lane == 0) {
+      if (lead) {
+        const uint32_t idesc = idesc_bf16_f32(2 * kBM, kPBN);
+        uint32_t it = 0, acc_it = 0, ni = 0;
+        bool ok = true;
+        for (int64_t item = pair; item < items && ok && !*abortp; item += npairs, ++ni) {
+          const int slot = int(ni & 1u);
+          if (!mbar_wait(&s.a_full[slot], (ni >> 1) & 1u, &s.abort, kTimeoutNs)) {
+            on_timeout_pair(s, status);
+            break;
+          }
+          for (int nt = 0; nt < n_nt && ok; ++nt, ++acc_it) {
+            const int a = int(acc_it & 1u);
+            if (!mbar_wait_cluster(&s.acc_empty[a], ((acc_it >> 1) & 1u) ^ 1u, &s.abort,
+                                   kTimeoutNs)) {
+              on_timeout_pair(s, status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int ks = 0; ks < nk; ++ks, ++it) {
+              const int st = it % kPStages;
+              if (!mbar_wait(&s.full[st], (it / kPStages) & 1u, &s.abort, kTimeoutNs)) {
+                on_timeout_pair(s, status);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t da = desc_k_sw128(smem_u32(s.a[slot][ks]));
+              const uint64_t db = desc_k_sw128(smem_u32(s.b[st]));
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk)
+                mma_bf16_pair(tmem + uint32_t(a * kPBN), da + 2 * kk, db + 2 * kk, idesc,
+                              (ks | kk) != 0);
+              mma_commit_pair(&s.empty[st]);
+            }
+            if (!ok) break;
+            mma_commit_pair(&s.acc_full[a]);
+          }
+          if (!ok) break;
+          mma_commit_pair(&s.a_empty[slot]);  // the rows may be replaced
+        }
+        // teardown: every MMA issued so far has completed, in both SMs
+        mma_commit_pair(&s.drain);
+      }
+      const int never = 0;
+      mbar_wait_cluster(&s.drain, 0, &never, kTimeoutNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int ew = warp - 3;           // 0..7
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int h = ew >> 2;             // column half of the slice
+    const int row_local = q * 32 + lane;
+    uint32_t acc_it = 0;
+    bool ok = true;
+    // every epilogue warp walks every item (meeting every named barrier), doing no more
+    // waits once one has timed out
+    for (int64_t item = pair; item < items; item += npairs) {
+      const int r = int(item / per_round);
+      const int64_t t = item % per_round;
+      const bool isY = t >= tX;
+      const int64_t row0 = (isY ? t - tX : t) * kRows + int64_t(rank) * kBM;
+      float best = -INFINITY;
+      int best_b = INT_MAX;
+      for (int nt = 0; nt < n_nt; ++nt, ++acc_it) {
+        const int a = int(acc_it & 1u);
+        if (ok && (*abortp || !mbar_wait_cluster(&s.acc_full[a], (acc_it >> 1) & 1u, &s.abort,
+                                                 kTimeoutNs))) {
+          if (!*abortp) on_timeout_pair(s, status);
+          ok = false;
+        }
+        if (!ok) continue;
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem + (uint32_t(q * 32) << 16) + uint32_t(a * kPBN + h * 128);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 64) {
+          float v[64];
+          tmem_load64(taddr + c0, v);
+          argmax32(*reinterpret_cast<float(*)[32]>(v), nt * kPBN + h * 128 + c0, n_b, best,
+                   best_b);
+          argmax32(*reinterpret_cast<float(*)[32]>(v + 32), nt * kPBN + h * 128 + c0 + 32, n_b,
+                   best, best_b);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(&s.acc_empty[a], 0);
+      }
+      // the two column halves of the row: the lower vector wins a tie
+      if (h == 1) {
+        s.cmb_v[row_local] = best;
+        s.cmb_i[row_local] = best_b;
+      }
+      named_barrier(1, 256);
+      if (h == 0 && ok) {
+        const float v1 = s.cmb_v[row_local];
+        const int i1 = s.cmb_i[row_local];
+        if (v1 > best || (v1 == best && i1 < best_b)) best_b = i1;
+        const int64_t row = row0 + row_local;
+        const int64_t M = isY ? C : N;
+        if (row < M) (isY ? by : bx)[int64_t(r) * M + row] = best_b;
+      }
+      named_barrier(1, 256);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the other may still reach its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void* Y,
@@ -459,6 +712,37 @@ cudaError_t launch_bucketize_tc(const rece_plan_s& p, const void* X, const void*
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tmB, B, uint64_t(c.n_r) * c.n_b, c.d, bn);
   if (e != cudaSuccess) return e;
+  if (c.d <= kRMaxK * kBK && int64_t(c.n_b) * c.d >= (int64_t(1) << 19) && sm_count() >= 2) {
+    // rows resident on pairs of SMs, B streamed once per 256 rows, M = 256 MMAs: where an
+    // item holds enough work (n_b d >= 2^19; at n_b = 4096, d = 256: 7.22 -> 6.29 ms) to
+    // carry the pair's per-item costs (at n_b = 1024, d = 128 the single-SM kernel is
+    // faster: 0.67 against 0.86 ms)
+    e = make_tmap_bf16(&tmB, B, uint64_t(c.n_r) * c.n_b, c.d, 128);
+    if (e != cudaSuccess) return e;
+    const int64_t items = (ceil_div(c.N, 2 * kBM) + ceil_div(c.C, 2 * kBM)) * c.n_r;
+    const int64_t pairs = items < sm_count() / 2 ? items : sm_count() / 2;
+    const size_t smem = sizeof(SmemPair) + 1024;
+    e = cudaFuncSetAttribute(k_bucketize_tc_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(2 * pairs));
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_bucketize_tc_pair, tmX, tmY, tmB, c.N, c.C, c.d, c.n_b,
+                           c.n_r, bx, by, status);
+    count_launches(1);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   if (c.d <= kRMaxK * kBK) {
     // rows resident, B streamed once per 256 rows
     const int bnr = c.n_b >= kRBN ? kRBN : ((c.n_b + 15) / 16) * 16;
