@@ -28,7 +28,8 @@ def bucket_ids_gpu(w, X, Y, B):
     return bx, by, px, py
 
 
-@pytest.mark.parametrize("d,n_b", [(64, 16), (64, 256), (128, 300), (192, 1024), (64, 1)])
+@pytest.mark.parametrize("d,n_b", [(64, 16), (64, 256), (128, 300), (192, 1024), (64, 1),
+                                   (256, 2048), (256, 2100)])
 def test_bucketize_tc_exact_on_integer_inputs(d, n_b):
     w = synth.Workload("int", N=1000, C=3001, d=d, dtype="bf16", n_b=n_b, n_c=4, n_ec=1,
                        n_r=2, k=8)
