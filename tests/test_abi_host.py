@@ -81,6 +81,9 @@ def test_null_arguments():
     assert L.rece_plan_create(None, None) == 1
     assert L.rece_plan_workspace_size(None, None) == 1
     assert L.rece_bucketize_sort(None, None, None, None, None, 0, None) == 1
+    assert L.rece_draw_projections(None, 0, 0, None, None) == 1
+    p = Plan(N=256, C=4096, d=64, n_b=16, n_c=8, n_ec=1, n_r=1, k=32)
+    assert L.rece_draw_projections(p._h, 0, 0, None, None) == 1  # NULL B
 
 
 def test_workspace_size_and_layout():
