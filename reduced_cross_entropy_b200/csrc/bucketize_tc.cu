@@ -450,13 +450,15 @@ __global__ void __launch_bounds__(kRThreads, 1) k_bucketize_tc_res(
 // (64 K elements a stage); the even CTA issues M = 256 x N = 256 MMAs, each CTA's TMEM
 // receiving its own 128 rows (two 256-column accumulators).  An MMA then reads from each
 // SM's shared memory half the bytes the single-SM kernel's M = 128 x N = 128 MMAs read
-// for the same work, which had shared-memory bandwidth, not the tensor pipe, bound the
-// bucketing; the rows of the next item load into a second buffer meanwhile.  Loads of
+// for the same work (about 120 bytes a clock there, near the SM's 128, which held that
+// kernel near 72% of the tensor peak); the rows of the next item load into a second
+// buffer meanwhile.  Loads of
 // both CTAs complete on the even CTA's barriers; the MMA commits (a stage or a row buffer
 // free, an accumulator full, all done) arrive on both CTAs' barriers at once (forwarding
 // them from the even CTA's threads instead made the kernel 1.6 times slower).  Eight
-// epilogue warps a CTA: warps q and q + 4 share TMEM lanes 32(q mod 4) and take column
-// halves, combined at the end of the item (ties to the lower vector).
+// epilogue warps a CTA (warps 3-10): epilogue warps e and e + 4 share the TMEM lanes of
+// their warp number mod 4 and take the two column halves of a slice, combined at the end
+// of the item (ties to the lower vector).
 constexpr int kPStages = 6;
 constexpr int kPBN = 256;                        // vectors per slice (N of the pair MMA)
 constexpr uint32_t kPSliceA = kBM * kBK * 2;     // 16 KB: 128 rows x 64 K
