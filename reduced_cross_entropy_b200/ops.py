@@ -328,7 +328,10 @@ class _ReceLossFn(torch.autograd.Function):
 def rece_loss(X, Y, targets, B, plan: Plan, ws=None):
     """Reduced cross-entropy loss with autograd (gradients for X and Y).
 
-    B [n_r, n_b, d]: the random vectors of this call (draw them afresh every step)."""
+    B: the random vectors of this call [n_r, n_b, d] (afresh every step), or a pair
+    (seed, step), for which the library draws them on the device (draw_projections)."""
     if ws is None:
         ws = plan.workspace(X.device)
+    if isinstance(B, tuple):
+        B = draw_projections(plan, int(B[0]), int(B[1]))
     return _ReceLossFn.apply(X, Y, targets, B, plan, ws)

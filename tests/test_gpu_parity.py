@@ -107,6 +107,32 @@ def test_draw_projections_match_oracle(dtype):
         compare(w, run_gpu(w, X, Y, t, B), run_oracle(w, X, Y, t, B))
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_autograd_wrapper_matches_the_calls_and_the_oracle(dtype):
+    """ops.rece_loss (torch autograd over rece_loss_fwd / rece_loss_bwd, B drawn on the
+    device from (seed, step)): the loss and the gradients torch hands back equal the direct
+    calls' on the same B, and the oracle's within the mode's tolerance."""
+    w = synth.Workload("autograd", N=700, C=5000, d=64, dtype=dtype, n_b=32, n_c=8, n_ec=1,
+                       n_r=2, k=40)
+    X, Y, t = synth.make_inputs(w, seed=3)
+    plan = ops.Plan(w.N, w.C, w.d, w.n_b, w.n_c, w.n_ec, w.n_r, w.k, mode=w.dtype)
+    Xd = to_dev(X, dtype).requires_grad_()
+    Yd = to_dev(Y, dtype).requires_grad_()
+    td = torch.from_numpy(t).cuda()
+    loss = ops.rece_loss(Xd, Yd, td, (3, 5), plan)
+    (0.5 * loss).backward()
+    B = ops.draw_projections(plan, 3, 5)
+    g = run_gpu(w, X, Y, t, B.float().cpu().numpy(), dloss=0.5)
+    assert loss.item() == g["loss"]
+    np.testing.assert_array_equal(Xd.grad.float().cpu().numpy(),
+                                  torch.from_numpy(g["dX"]).to(Xd.dtype).float().numpy())
+    np.testing.assert_array_equal(Yd.grad.float().cpu().numpy(),
+                                  torch.from_numpy(g["dY"]).to(Yd.dtype).float().numpy())
+    o = run_oracle(w, X, Y, t, B.float().cpu().numpy(), dloss=0.5)
+    tol = 1e-4 if dtype == "fp32" else 1e-2
+    assert abs(loss.item() - o["loss"]) <= tol * abs(o["loss"])
+
+
 def test_fp32_exact_whole_arrays_at_sasrec_scale():
     """The fp32 exact mode at the SASRec-scale benchmark shape (N = 25,600, C = 100,000,
     n_b = 256, n_c = 64, n_ec = 1, n_r = 2, k = 256), the whole arrays against the whole
