@@ -1,14 +1,16 @@
-// merge_tc.cu -- steps 4-5 for the tensor-core selection: one warp per row.
+// merge_tc.cu -- steps 4-5 for the tensor-core selection: a warp per row (k < 512) or a
+// CTA of four warps per row (k >= 512, further down).
 //
 // The row's candidates are the (score, sorted position) pairs its rounds emitted.  A pair
 // of round r is translated to its item j and dropped when j is the row's positive or when
 // j also lies in the row's window of an earlier round r' < r (that round saw the same
 // pair, so the union of the rounds stays de-duplicated -- the RECE paper's ln(count)
 // correction for repeated pairs amounts to counting each pair once).  The k best of the
-// rest by (score descending, item ascending) are found with a warp radix select (4-bit
-// digits of the score key from its highest varying bit, then the item ids if the k-th
-// place is tied), kept in the order of the candidate lists (a fixed order), and give the
-// row's loss (RECE, Algorithm 1's loss lines):
+// rest by (score descending, item ascending) are found with a radix select (digits of
+// the score key from its highest varying bit, then the item ids if the k-th place is
+// tied), kept in a fixed order (by round, then list order, or sorted position where the
+// backward's band products follow), and give the row's loss (RECE, Algorithm 1's loss
+// lines):
 //   lse_i = log(exp(l+) + sum_j exp(l_j)),  loss_i = lse_i - l+.
 // Exactness check: each round recorded the largest score it did not emit; if no list
 // overflowed and every such score is below the k-th kept score, nothing left out could
